@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the Lookahead Sparse Attention indexer hot path on B200.
+
+One step = one trigger window over one batch of synthetic sequences: project (stage 1),
+index score + threshold + OR + compaction (stages 2-4a), fetch from the mapped host cold
+pool (4b), and the Lightning-Indexer Top-k of all tau decode queries (5).  Prints ONE JSON
+line (rank 0).  `--impl reference` times the CPU oracle instead, on a bounded sample.
+
+Launch: python bench.py [--gpus 1 --steps K --warmup W]; for N > 1 under torchrun, each rank
+runs its own batch (independent sequences: weak scaling, no data-path collective).
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "ctx1m_fp8_b32"
+METRIC = "compressed entries scored+selected/sec at 1M ctx (whole tau-window path)"
+UNIT = "entries/s"
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["lsa", "reference"], default="lsa")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--threshold", type=float, default=0.5)
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--cpu-sample", type=int, default=0,
+                   help="entries of the oracle's bounded sample (default: sized for a few minutes of CPU work)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.file = None
+        try:
+            self.gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.gpu_id = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.count(",") >= 7]
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------ oracle sample
+
+def oracle_sample_workload(wl, n):
+    """A bounded sample of the workload: one sequence of n entries, same dims, dtypes and seed."""
+    return synth.workload(wl.name, B=1, S=(min(n, wl.S[0]),), fetch=(wl.fetch[0],), seed=wl.seed)
+
+
+def oracle_step(oracle, wl, inp):
+    """The whole path on the CPU oracle for the sample (project, score/OR/compact, gather, Top-k)."""
+    offs = inp.seq_offsets.numpy()
+    q, w = oracle.project(inp.h, inp.W_dq, inp.W_iuq, inp.W_w, wl.n_h, wl.d_I)
+    r = oracle.score(q, w, inp.K, inp.k_scale, offs, want_x=False)
+    idx, cnt = torch.from_numpy(r["idx"]), torch.from_numpy(r["count"])
+    sel = wl.sel_layer
+    ks = inp.k_scale[sel] if inp.k_scale is not None else None
+    oracle.gather(idx, cnt, offs, inp.pool, inp.K[sel], ks, wl.d_I)
+    oracle.lightning_topk(inp.q_dec, inp.w_dec, inp.K[sel], ks, idx, cnt, offs, wl.k)
+    return int(cnt.sum())
+
+
+def cpu_baseline(wl, n_entries, steps=1):
+    import oracle
+    sw = oracle_sample_workload(wl, n_entries)
+    inp = synth.make_inputs(sw)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle_step(oracle, sw, inp)
+        times.append(time.perf_counter() - t0)
+    units = sw.L * sw.total_S
+    return {"value": units / statistics.mean(times), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"one sequence of {sw.total_S} entries x {sw.L} layers of {wl.name} (same dims/dtypes), "
+                      f"whole path incl. S1 projection and Top-k of {sw.tau} queries; mean of {steps} run(s)"}
+
+
+# ------------------------------------------------------------------------------------ model of the bytes
+
+def algorithmic(wl, fetched_total):
+    """Algorithmic bytes / flops per launch of each stage (the units each launch processes)."""
+    T, L, B = wl.total_S, wl.L, wl.B
+    eb = {"f32": 4, "bf16": 2, "fp8": 1}
+    kb = wl.d_I * eb[wl.kdtype] + (4 if wl.kdtype == "fp8" else 0)       # key bytes per entry per layer
+    qb = eb[wl.dtype]
+    nq = wl.n_h * wl.d_I
+    proj_bytes = L * (wl.r * wl.d + nq * wl.r + wl.n_h * wl.d) * qb + L * B * (wl.d * qb + nq * qb + wl.n_h * 4)
+    score_bytes = L * T * kb + L * B * (nq * qb + wl.n_h * 4) + T // 8 + 4 * T * 0  # keys + queries + mask bits
+    gather_host = fetched_total * wl.row_bytes                            # crosses the host link
+    gather_dev = fetched_total * (wl.row_bytes + wl.d_I * eb[wl.kdtype] * 2 + 8)
+    topk_flops = 2.0 * wl.tau * wl.n_h * wl.d_I * fetched_total
+    return {"proj_bytes": proj_bytes, "score_bytes": score_bytes, "score_bytes_per_entry_layer": kb,
+            "gather_host_bytes": gather_host, "gather_dev_bytes": gather_dev, "topk_flops": topk_flops}
+
+
+def h2d_bandwidth(device, nbytes=1 << 30):
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream(device)
+    for _ in range(2):
+        dst.copy_(src, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(3):
+        dst.copy_(src, non_blocking=True)
+    e1.record(st)
+    torch.cuda.synchronize(device)
+    gbs = 3 * nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del src, dst
+    return gbs
+
+
+# ------------------------------------------------------------------------------------ lsa arm
+
+def run_lsa(args, rank, world, device):
+    import sparse_kv_cache_memoryindexer_b200 as lsa
+    torch.cuda.set_device(device)
+    base = synth.workload(args.workload)
+    wl = synth.workload(args.workload, seed=base.seed + 7919 * rank)
+    T = wl.total_S
+    dt, kdt = synth.DTYPES[wl.dtype], synth.DTYPES[wl.kdtype]
+    pool = lsa.MappedPool(T, wl.row_bytes)
+    inp = synth.make_inputs(wl, pool_out=pool.tensor)
+    st = torch.cuda.current_stream(device)
+
+    def d(t):
+        return None if t is None else t.to(device, non_blocking=False)
+
+    h, Wdq, Wiuq, Ww = d(inp.h), d(inp.W_dq), d(inp.W_iuq), d(inp.W_w)
+    K, ks, offs, qd, wd = d(inp.K), d(inp.k_scale), d(inp.seq_offsets), d(inp.q_dec), d(inp.w_dec)
+    path = lsa.IndexerPath(wl.L, wl.B, wl.d, wl.r, wl.n_h, wl.d_I, wl.tau, wl.k, T, wl.row_bytes, dt, kdt, device=device)
+    sel = wl.sel_layer
+
+    def stages():
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(st)
+        path.project(h, Wdq, Wiuq, Ww, st)
+        ev[1].record(st)
+        path.select(K, ks, offs, args.threshold, stream=st)
+        ev[2].record(st)
+        path.fetch(offs, pool.tensor, K[sel], None if ks is None else ks[sel], st)
+        ev[3].record(st)
+        path.topk(qd, wd, offs, st)
+        ev[4].record(st)
+        return ev
+
+    for _ in range(args.warmup):
+        stages()
+    torch.cuda.synchronize(device)
+    lsa.lsa_check_device(st)
+    fetched = int(path.count.sum().item())
+    h2d = h2d_bandwidth(device)
+
+    clocks = ClockSampler(device)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    n0 = lsa.launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    evs = [stages() for _ in range(args.steps)]
+    t1.record(st)
+    torch.cuda.synchronize(device)
+    launches = lsa.launch_count() - n0
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    lsa.lsa_check_device(st)
+    elapsed_ms = t0.elapsed_time(t1)
+    stage_ms = np.zeros(4)
+    for ev in evs:
+        for i in range(4):
+            stage_ms[i] += ev[i].elapsed_time(ev[i + 1])
+    stage_ms /= args.steps
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.pin_memory() for k, v in (("h", inp.h), ("K", inp.K), ("qd", inp.q_dec), ("wd", inp.w_dec))}
+        if inp.k_scale is not None:
+            host["ks"] = inp.k_scale.pin_memory()
+        out_i = torch.empty(path.topk_idx.shape, dtype=torch.int32).pin_memory()
+        out_c = torch.empty(path.count.shape, dtype=torch.int32).pin_memory()
+        h2d_b = sum(v.numel() * v.element_size() for v in host.values())
+        d2h_b = out_i.numel() * 4 + out_c.numel() * 4
+
+        def e2e_step():
+            h.copy_(host["h"], non_blocking=True)
+            K.copy_(host["K"], non_blocking=True)
+            if ks is not None:
+                ks.copy_(host["ks"], non_blocking=True)
+            qd.copy_(host["qd"], non_blocking=True)
+            wd.copy_(host["wd"], non_blocking=True)
+            path.run(h, Wdq, Wiuq, Ww, K, ks, offs, pool.tensor, qd, wd, sel_layer=sel, threshold=args.threshold,
+                     stream=st)
+            out_i.copy_(path.topk_idx, non_blocking=True)
+            out_c.copy_(path.count, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        if world > 1:
+            torch.distributed.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(st)
+        torch.cuda.synchronize(device)
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([e_ms], dtype=torch.float64, device=device)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": world * wl.L * T * args.e2e_steps / (e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
+        del host
+
+    result = None
+    if rank == 0:
+        peaks = load_peaks()
+        alg = algorithmic(wl, fetched)
+        ms = elapsed_ms / args.steps
+        value = world * wl.L * T * args.steps / (elapsed_ms * 1e-3)
+        sel_ms = stage_ms[1]
+        score_gbs = alg["score_bytes"] / (sel_ms * 1e-3) / 1e9
+        rooflines = {
+            "project": {"bound": "hbm", "achieved": alg["proj_bytes"] / (stage_ms[0] * 1e-3) / 1e9,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s", "ms": stage_ms[0]},
+            "score_select": {"bound": "hbm", "achieved": score_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "ms": sel_ms},
+            "fetch_gather": {"bound": "host_link", "achieved": alg["gather_host_bytes"] / (stage_ms[2] * 1e-3) / 1e9,
+                             "peak": h2d, "unit": "GB/s", "ms": stage_ms[2],
+                             "peak_note": "pinned host->device cudaMemcpy measured in this run"},
+            "lightning_topk": {"bound": "tensor", "achieved": alg["topk_flops"] / (stage_ms[3] * 1e-3) / 1e12,
+                               "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "ms": stage_ms[3]},
+        }
+        for r in rooflines.values():
+            r["frac"] = r["achieved"] / r["peak"]
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if wl.kdtype != "f32" else "f32",
+            "dtype_detail": f"keys {wl.kdtype}, queries/weights {wl.dtype}, fp32 accumulation",
+            "data": "synthetic (seeded; shapes of a 1M-token context, 4:1 compression)",
+            "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "S_per_seq": wl.S[0], "d": wl.d, "r": wl.r,
+                       "n_h": wl.n_h, "d_I": wl.d_I, "tau": wl.tau, "k": wl.k, "kv_row_bytes": wl.row_bytes,
+                       "keys": wl.kdtype, "threshold": args.threshold, "parallelism": f"dp{world} (sequences)",
+                       "l2": "inputs larger than L2 (key stream %.2f GB per step)" % (alg["score_bytes"] / 1e9),
+                       "fetch_rate": fetched / T},
+            "tau_window_ms": ms,
+            "stages_ms": {"project": stage_ms[0], "score_select": stage_ms[1], "fetch_gather": stage_ms[2],
+                          "lightning_topk": stage_ms[3]},
+            "score_select_entries_per_s": world * wl.L * T / (sel_ms * 1e-3),
+            "roofline": dict(kernel="score_select (index score + threshold + OR + compaction, one stream)",
+                             bound="hbm", achieved=score_gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                             frac=score_gbs / peaks["hbm_gbs"], traffic=None,
+                             bytes_per_launch=alg["score_bytes"], peak_source=peaks["source"]),
+            "rooflines": rooflines,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+        }
+    pool.free()
+    return result
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        import oracle
+        wl = synth.workload(args.workload)
+        # about two minutes of oracle work in total (~130 us per entry on 8 cores, whole path)
+        n = args.cpu_sample or int(min(65536, max(2048, 120.0 / (args.steps + args.warmup) / 130e-6)))
+        sw = oracle_sample_workload(wl, n)
+        inp = synth.make_inputs(sw)
+        for _ in range(args.warmup):
+            oracle_step(oracle, sw, inp)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_step(oracle, sw, inp)
+        el = time.perf_counter() - t0
+        value = sw.L * sw.total_S * args.steps / el
+        cb = {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+              "sample": f"one sequence of {sw.total_S} entries x {sw.L} layers of {wl.name} per step, whole path"}
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": {"workload": wl.name, "sample_entries": sw.total_S},
+                          "cpu_baseline": cb,
+                          "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    device = torch.device("cuda", local)
+    if world > 1:
+        torch.cuda.set_device(device)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    try:
+        res = run_lsa(args, rank, world, device)
+        if rank == 0:
+            if not args.no_cpu_baseline and world == 1:
+                res["cpu_baseline"] = cpu_baseline(synth.workload(args.workload), args.cpu_sample or 65536)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,181 @@
+/*
+ * lsa.h -- C ABI of the Lookahead Sparse Attention (LSA) indexer hot path on NVIDIA B200.
+ *
+ * The method (pages: "FlashMemory-DeepSeek-V4: Lightning Index Ultra-Long Context via
+ * Lookahead Sparse Attention", hyper.ai summary "Method", and the marsggbo blog review,
+ * sections 2.2, 3, 3.1, 3.2 and 4.2):  every tau = 64 decode steps a Memory Indexer projects
+ * the trigger token's hidden state into indexer queries, scores every preceding compressed
+ * index key with I = sigmoid(sum_h w_h ReLU(q_h . K_s)), fetches the entries with I >= 0.5 in
+ * any of its three layers from the CPU cold pool into GPU memory, and, at each decode step of
+ * the window, the native Lightning Indexer picks its Top-k entries among the fetched ones.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are device pointers owned by the caller, except the cold pool, which is
+ *     caller-owned page-locked host memory mapped into the device address space
+ *     (lsa_pool_alloc, cudaHostAlloc(..., cudaHostAllocMapped) or cudaHostRegister(...,
+ *     cudaHostRegisterMapped)).  The library keeps no pointer after a call returns and
+ *     allocates no device memory: scratch space is the caller's `workspace`.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream); arguments are validated on the host before anything is launched.
+ *   - Ragged batches: `seq_offsets` is a DEVICE array of B+1 int64 prefix offsets; sequence b
+ *     owns rows seq_offsets[b] .. seq_offsets[b+1]-1 of every [.][T] array, T = total_S =
+ *     seq_offsets[B], which the caller also passes by value.  Entry s of sequence b is row
+ *     seq_offsets[b] + s.  Every layer has the same entries (an entry is one compressed
+ *     position; the layers are OR-combined per entry).
+ *   - Errors: a non-LSA_OK status means nothing was launched (or, for LSA_ERR_CUDA, that a
+ *     launch failed); lsa_last_error() gives a message for the calling thread.  Kernels that
+ *     meet bad data (an index outside its sequence, a count above capacity, a negative or
+ *     NaN key scale, decreasing offsets) skip the access and set a device error word, which
+ *     lsa_check_device() reads and clears.  No kernel traps and no kernel waits on another.
+ *   - Dtypes: LSA_F32 (IEEE binary32), LSA_BF16 (bfloat16), LSA_FP8_E4M3 (OCP E4M3 with one
+ *     fp32 scale per key row: key value = scale * decode(code)).
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *lsa_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned buffer, unmapped pool */
+    LSA_ERR_UNSUPPORTED = 2,  /* dtype / shape combination without a kernel */
+    LSA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    LSA_ERR_DEVICE_CHECK = 4, /* lsa_check_device: a kernel flagged bad data */
+    LSA_ERR_WORKSPACE = 5     /* workspace smaller than the *_workspace_size answer */
+} lsa_status;
+
+typedef enum { LSA_F32 = 0, LSA_BF16 = 1, LSA_FP8_E4M3 = 2 } lsa_dtype;
+
+/* Largest Top-k the decode-step selection supports. */
+#define LSA_MAX_TOPK 4096
+
+/* Message of the last failing call on this thread ("" if none). Never NULL. */
+const char *lsa_last_error(void);
+
+/* Library version string. */
+const char *lsa_version(void);
+
+/* Number of kernels this library has launched in this process (all threads, all devices). */
+uint64_t lsa_launch_count(void);
+
+/* Synchronise `stream`, read and clear the device error word of the current device.
+ * Returns LSA_OK, LSA_ERR_DEVICE_CHECK (message lists the flags) or LSA_ERR_CUDA. */
+lsa_status lsa_check_device(lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Stage 1 -- Memory-Indexer projections (blog review section 3.1):
+ *     c^Q = h W^DQ,   q = c^Q W^IUQ,   w = h W^w,   for each layer l and sequence b.
+ *   h      [L][B][d]            dt       hidden state of the trigger token at each indexer layer
+ *   W_dq   [L][r][d]            dt       W^DQ stored transposed: row j holds column j (out x in)
+ *   W_iuq  [L][n_h*d_I][r]      dt       W^IUQ stored transposed; output o = head*d_I + e
+ *   W_w    [L][n_h][d]          dt       W^w stored transposed
+ *   q_out  [L][B][n_h][d_I]     dt       queries, rounded to dt (nearest-even)
+ *   w_out  [L][B][n_h]          fp32     head weights
+ * c^Q is rounded to dt before the second projection and lives in the workspace.
+ * dt: LSA_F32 or LSA_BF16.  Accumulation is fp32.  Workspace: lsa_project_workspace_size.
+ * ---------------------------------------------------------------------------------------- */
+size_t lsa_project_workspace_size(int L, int B, int d, int r, int n_h, int d_I, lsa_dtype dt);
+
+lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const void *W_w,
+                       lsa_dtype dt, int L, int B, int d, int r, int n_h, int d_I,
+                       void *q_out, float *w_out, void *workspace, size_t workspace_bytes,
+                       lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Stages 2-4a -- index score, threshold, OR over layers, compaction (blog review sections
+ * 3.1 and 4.2; hyper.ai summary "Method"):
+ *     x_{l,b,s} = sum_h w_{l,b,h} ReLU(scale_{l,s} q_{l,b,h} . K_{l,s}),   I = sigmoid(x),
+ *     entry s of sequence b is fetched iff I_{l,b,s} >= threshold for some layer l.
+ * The decision is taken on the logit, x >= log(threshold / (1 - threshold)) in fp32 (x >= 0 at
+ * 0.5, so an exact-zero logit is fetched).
+ *   q         [L][B][n_h][d_I]   fp32 when kdt = LSA_F32, else bf16
+ *   w         [L][B][n_h]        fp32
+ *   K         [L][T][d_I]        kdt
+ *   k_scale   [L][T]             fp32, required for LSA_FP8_E4M3 (finite, >= 0), else NULL
+ *   threshold                    in (0, 1); the pages use 0.5
+ *   scores_out  [L][T] fp32      sigmoid scores I (nullable; costs 4 bytes per entry-layer)
+ *   mask_out    [T] uint8        1 if fetched (nullable)
+ *   idx_out     [T] int32        segment b: the fetched s in ascending order in the first
+ *                                count_out[b] slots; the other slots are left unchanged
+ *   count_out   [B] int32        number of fetched entries of each sequence
+ * Kernels: tcgen05 tensor-core path for n_h = 64, d_I = 128 with bf16 or E4M3 keys; a SIMT
+ * path for other shapes (d_I in {32, 64, 128}, n_h <= 128) and for fp32.
+ * Workspace: lsa_score_select_workspace_size.
+ * ---------------------------------------------------------------------------------------- */
+size_t lsa_score_select_workspace_size(int L, int B, int64_t total_S);
+
+lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *K,
+                                     const float *k_scale, lsa_dtype kdt,
+                                     const int64_t *seq_offsets, int64_t total_S,
+                                     int L, int B, int n_h, int d_I, float threshold,
+                                     float *scores_out, uint8_t *mask_out,
+                                     int32_t *idx_out, int32_t *count_out,
+                                     void *workspace, size_t workspace_bytes, lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Stage 4b -- fetch C^MemComp from the CPU cold pool into the GPU hot buffer (hyper.ai
+ * summary "Method"; blog review section 3):
+ *     hot_kv[off_b + j] = pool[off_b + idx[off_b + j]]      for j < count[b]
+ * and, when K_sel is given, the same gather of the keys (and scales) of one layer, the keys
+ * the decode-step Lightning Indexer scores:
+ *     hot_K[off_b + j] = K_sel[off_b + idx[off_b + j]],  hot_scale likewise.
+ *   idx, count            as written by lsa_memindex_score_select (device)
+ *   pool                  mapped page-locked HOST memory, [T][row_bytes]
+ *   row_bytes             multiple of 16; pool, hot_kv 16-byte aligned
+ *   hot_kv                [T][row_bytes] device (capacity T; slots past count untouched)
+ *   K_sel, k_scale_sel    [T][d_I] kdt and [T] fp32 (nullable: K_sel NULL skips the keys;
+ *                         k_scale_sel required iff kdt = LSA_FP8_E4M3)
+ *   hot_K, hot_scale      [T][d_I] kdt and [T] fp32
+ * Out-of-range indices or counts are skipped and flagged in the device error word.
+ * ---------------------------------------------------------------------------------------- */
+lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count,
+                            const int64_t *seq_offsets, int64_t total_S, int B,
+                            const void *pool, size_t row_bytes, void *hot_kv,
+                            const void *K_sel, const float *k_scale_sel, lsa_dtype kdt, int d_I,
+                            void *hot_K, float *hot_scale, lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Stage 5 -- native Lightning Indexer Top-k over the fetched entries (blog review sections
+ * 2.2 and 3.2):  for decode query i of sequence b and fetched slot j < count[b],
+ *     y_{b,i,j} = sum_h w'_{b,i,h} ReLU(hot_scale_j q'_{b,i,h} . hot_K_j)
+ * and C^CoreComp_{b,i} = the k slots of largest y, reported as entry indices s = idx[off_b+j],
+ * ordered by y descending, ties to the smaller s; when count[b] < k the tail is -1 / -inf.
+ *   q_dec      [B][tau][n_h][d_I]   fp32 when kdt = LSA_F32, else bf16
+ *   w_dec      [B][tau][n_h]        fp32
+ *   hot_K, hot_scale                as written by lsa_fetch_gather (hot_scale iff FP8)
+ *   idx, count                      as written by lsa_memindex_score_select
+ *   k                               1 .. LSA_MAX_TOPK
+ *   topk_idx   [B][tau][k] int32
+ *   topk_score [B][tau][k] fp32     (nullable)
+ * Workspace: lsa_lightning_topk_workspace_size (holds the fp32 scores y).
+ * ---------------------------------------------------------------------------------------- */
+size_t lsa_lightning_topk_workspace_size(int B, int tau, int64_t total_S, int k);
+
+lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void *hot_K,
+                              const float *hot_scale, lsa_dtype kdt,
+                              const int32_t *idx, const int32_t *count,
+                              const int64_t *seq_offsets, int64_t total_S,
+                              int B, int tau, int n_h, int d_I, int k,
+                              int32_t *topk_idx, float *topk_score,
+                              void *workspace, size_t workspace_bytes, lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Cold-pool helpers: page-locked host memory mapped into every device's address space
+ * (cudaHostAlloc with the Mapped and Portable flags).  The pointer is valid on the host and,
+ * unchanged, in kernels.  lsa_pool_free releases memory from lsa_pool_alloc only.
+ * ---------------------------------------------------------------------------------------- */
+lsa_status lsa_pool_alloc(size_t bytes, void **ptr);
+lsa_status lsa_pool_free(void *ptr);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

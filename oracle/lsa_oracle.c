@@ -231,30 +231,42 @@ int lsa_oracle_score(const void *q, int qdt, const float *w, const void *K, cons
         return 1;
     const double t = log(threshold / (1.0 - threshold));
     const int64_t T = seq_offsets[B];
-#pragma omp parallel for schedule(dynamic)
+    uint8_t *fetched = (uint8_t *)malloc((size_t)(T > 0 ? T : 1));
+    if (!fetched)
+        return 2;
+    /* every entry of every sequence: the OR over layers of (x >= t) */
+#pragma omp parallel for schedule(dynamic, 256)
+    for (int64_t row = 0; row < T; row++) {
+        int b = 0;
+        while (seq_offsets[b + 1] <= row)  /* the sequence that owns this row */
+            b++;
+        int f = 0;
+        for (int l = 0; l < L; l++) {
+            size_t lrow = (size_t)l * T + row;
+            double scale = k_scale ? (double)k_scale[lrow] : 1.0;
+            double x = index_logit(q, qdt, ((size_t)l * B + b) * n_h * d_I, w, ((size_t)l * B + b) * n_h,
+                                   K, kdt, lrow * d_I, scale, n_h, d_I);
+            if (x_out) x_out[lrow] = x;
+            if (I_out) I_out[lrow] = lsa_oracle_sigmoid(x);
+            if (x >= t)
+                f = 1;
+        }
+        fetched[row] = (uint8_t)f;
+    }
+    /* the fetched set of each sequence, in ascending entry order */
     for (int b = 0; b < B; b++) {
         int64_t off = seq_offsets[b], S = seq_offsets[b + 1] - seq_offsets[b];
         int32_t n = 0;
         for (int64_t s = 0; s < S; s++) {
-            int fetched = 0;
-            for (int l = 0; l < L; l++) {
-                size_t row = (size_t)l * T + off + s;
-                double scale = k_scale ? (double)k_scale[row] : 1.0;
-                double x = index_logit(q, qdt, ((size_t)l * B + b) * n_h * d_I, w, ((size_t)l * B + b) * n_h,
-                                       K, kdt, row * d_I, scale, n_h, d_I);
-                if (x_out) x_out[row] = x;
-                if (I_out) I_out[row] = lsa_oracle_sigmoid(x);
-                if (x >= t)
-                    fetched = 1;
-            }
-            if (mask_out) mask_out[off + s] = (uint8_t)fetched;
-            if (fetched) {
+            if (mask_out) mask_out[off + s] = fetched[off + s];
+            if (fetched[off + s]) {
                 if (idx_out) idx_out[off + n] = (int32_t)s;
                 n++;
             }
         }
         if (count_out) count_out[b] = n;
     }
+    free(fetched);
     return 0;
 }
 

@@ -1,0 +1,411 @@
+// C ABI of the LSA indexer hot path (declared in include/lsa.h).  Host-side validation and
+// dispatch; every stage runs in the kernels included below (one translation unit).
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/lsa.h"
+#include "common.cuh"
+#include "gather.cuh"
+#include "project.cuh"
+#include "score_select.cuh"
+#include "score_tc.cuh"
+#include "topk.cuh"
+
+using namespace lsa;
+
+namespace {
+
+thread_local char g_msg[512] = "";
+std::atomic<uint64_t> g_launches{0};
+
+lsa_status fail(lsa_status st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+lsa_status ok()
+{
+    g_msg[0] = '\0';
+    return LSA_OK;
+}
+
+// After a launch: count it and turn a launch error into LSA_ERR_CUDA.
+lsa_status launched(const char *what)
+{
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+    return LSA_OK;
+}
+
+#define LSA_TRY(x)                            \
+    do {                                      \
+        lsa_status _st = (x);                 \
+        if (_st != LSA_OK) return _st;        \
+    } while (0)
+
+#define LSA_REQUIRE(cond, ...)                                        \
+    do {                                                              \
+        if (!(cond)) return fail(LSA_ERR_INVALID_ARG, __VA_ARGS__);   \
+    } while (0)
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t elem_bytes(int dt) { return dt == DT_F32 ? 4 : (dt == DT_BF16 ? 2 : 1); }
+
+int num_sms()
+{
+    static thread_local int cached_dev = -1, cached_sms = 148;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != cached_dev) {
+        cudaDeviceGetAttribute(&cached_sms, cudaDevAttrMultiProcessorCount, dev);
+        cached_dev = dev;
+    }
+    return cached_sms;
+}
+
+// Workspace layout of lsa_memindex_score_select.
+struct ScoreWs {
+    int *tile_start;     // [B+1]
+    uint32_t *tile_mask; // [max_tiles][4]
+};
+
+int64_t max_tiles(int B, int64_t T) { return T / TILE + B + 1; }
+
+size_t score_ws_bytes(int B, int64_t T)
+{
+    return align_up(sizeof(int) * (size_t)(B + 1), 256) + align_up((size_t)max_tiles(B, T) * 16, 256);
+}
+
+ScoreWs score_ws(void *ws, int B)
+{
+    char *p = (char *)ws;
+    ScoreWs w;
+    w.tile_start = (int *)p;
+    w.tile_mask = (uint32_t *)(p + align_up(sizeof(int) * (size_t)(B + 1), 256));
+    return w;
+}
+
+template <typename K>
+lsa_status set_smem(K kernel, size_t bytes)
+{
+    if (bytes > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    return LSA_OK;
+}
+
+// ---------------------------------------------------------------- SIMT score dispatch
+template <int D, int KDT, int QDT>
+lsa_status launch_score_simt(const void *q, const float *w, const void *K, const float *ks, const int64_t *offs,
+                             const int *tile_start, int B, int64_t T, int L, int n_h, float thr,
+                             float *scores, uint32_t *tile_mask, cudaStream_t st)
+{
+    const size_t smem = sizeof(float) * (size_t)(n_h * D + n_h);
+    LSA_TRY(set_smem(k_score_simt<D, KDT, QDT>, smem));
+    const int64_t grid = max_tiles(B, T);
+    k_score_simt<D, KDT, QDT><<<(unsigned)grid, TILE, smem, st>>>(q, w, K, ks, offs, tile_start, B, T, L, n_h, thr,
+                                                                  scores, tile_mask);
+    return launched("score (SIMT)");
+}
+
+template <int D>
+lsa_status score_simt_d(int kdt, const void *q, const float *w, const void *K, const float *ks, const int64_t *offs,
+                        const int *tile_start, int B, int64_t T, int L, int n_h, float thr, float *scores,
+                        uint32_t *tile_mask, cudaStream_t st)
+{
+    switch (kdt) {
+    case DT_F32:
+        return launch_score_simt<D, DT_F32, DT_F32>(q, w, K, ks, offs, tile_start, B, T, L, n_h, thr, scores,
+                                                    tile_mask, st);
+    case DT_BF16:
+        return launch_score_simt<D, DT_BF16, DT_BF16>(q, w, K, ks, offs, tile_start, B, T, L, n_h, thr, scores,
+                                                      tile_mask, st);
+    default:
+        return launch_score_simt<D, DT_FP8, DT_BF16>(q, w, K, ks, offs, tile_start, B, T, L, n_h, thr, scores,
+                                                     tile_mask, st);
+    }
+}
+
+template <int D, int KDT, int QDT>
+lsa_status launch_li_simt(const void *qd, const float *wd, const void *hotK, const float *hotsc,
+                          const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, int n_h, float *Y,
+                          cudaStream_t st)
+{
+    const size_t smem = sizeof(float) * (size_t)(n_h * D + n_h);
+    LSA_TRY(set_smem(k_li_score_simt<D, KDT, QDT>, smem));
+    int64_t gx = (T + TILE - 1) / TILE;
+    int64_t cap = (int64_t)num_sms() * 8 / (B > 0 ? B : 1) + 1;
+    if (gx > cap) gx = cap;
+    if (gx < 1) gx = 1;
+    dim3 grid((unsigned)gx, (unsigned)B);
+    k_li_score_simt<D, KDT, QDT><<<grid, TILE, smem, st>>>(qd, wd, hotK, hotsc, count, offs, tau, n_h, Y);
+    return launched("lightning score (SIMT)");
+}
+
+template <int D>
+lsa_status li_simt_d(int kdt, const void *qd, const float *wd, const void *hotK, const float *hotsc,
+                     const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, int n_h, float *Y,
+                     cudaStream_t st)
+{
+    switch (kdt) {
+    case DT_F32: return launch_li_simt<D, DT_F32, DT_F32>(qd, wd, hotK, hotsc, count, offs, B, T, tau, n_h, Y, st);
+    case DT_BF16:
+        return launch_li_simt<D, DT_BF16, DT_BF16>(qd, wd, hotK, hotsc, count, offs, B, T, tau, n_h, Y, st);
+    default: return launch_li_simt<D, DT_FP8, DT_BF16>(qd, wd, hotK, hotsc, count, offs, B, T, tau, n_h, Y, st);
+    }
+}
+
+bool valid_dtype(int dt) { return dt == DT_F32 || dt == DT_BF16 || dt == DT_FP8; }
+
+}  // namespace
+
+extern "C" {
+
+const char *lsa_last_error(void) { return g_msg; }
+
+const char *lsa_version(void) { return "lsa-b200 0.1 (sm_100a)"; }
+
+uint64_t lsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+lsa_status lsa_check_device(lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    unsigned int word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_err_word, sizeof(word));
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    if (word == 0) return ok();
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "clearing the device error word: %s", cudaGetErrorString(e));
+    return fail(LSA_ERR_DEVICE_CHECK, "device check flags 0x%x:%s%s%s%s%s", word,
+                (word & ERRF_OFFSETS) ? " bad-seq-offsets" : "", (word & ERRF_INDEX) ? " index-out-of-range" : "",
+                (word & ERRF_COUNT) ? " count-out-of-range" : "", (word & ERRF_SCALE) ? " bad-key-scale" : "",
+                (word & ERRF_TIMEOUT) ? " pipeline-wait-timeout" : "");
+}
+
+// ------------------------------------------------------------------------------ stage 1
+
+size_t lsa_project_workspace_size(int L, int B, int d, int r, int n_h, int d_I, lsa_dtype dt)
+{
+    (void)d; (void)n_h; (void)d_I;
+    if (L <= 0 || B <= 0 || r <= 0) return 0;
+    return align_up((size_t)L * B * r * elem_bytes(dt), 256);
+}
+
+lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const void *W_w, lsa_dtype dt,
+                       int L, int B, int d, int r, int n_h, int d_I, void *q_out, float *w_out, void *workspace,
+                       size_t workspace_bytes, lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(h && W_dq && W_iuq && W_w && q_out && w_out, "lsa_project: null pointer");
+    LSA_REQUIRE(L > 0 && B > 0 && d > 0 && r > 0 && n_h > 0 && d_I > 0, "lsa_project: sizes must be positive");
+    if (dt != LSA_F32 && dt != LSA_BF16) return fail(LSA_ERR_UNSUPPORTED, "lsa_project: dt must be F32 or BF16");
+    LSA_REQUIRE(d % 8 == 0 && r % 8 == 0, "lsa_project: d and r must be multiples of 8");
+    LSA_REQUIRE(aligned(h, 16) && aligned(W_dq, 16) && aligned(W_iuq, 16) && aligned(W_w, 16),
+                "lsa_project: h and weights must be 16-byte aligned");
+    const size_t need = lsa_project_workspace_size(L, B, d, r, n_h, d_I, dt);
+    if (!workspace || workspace_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "lsa_project: workspace needs %zu bytes", need);
+    LSA_REQUIRE(aligned(workspace, 256), "lsa_project: workspace must be 256-byte aligned");
+    const int nq = n_h * d_I;
+    void *c = workspace;
+    if (dt == LSA_BF16) {
+        k_rowdot<DT_BF16, DT_BF16><<<dim3((r + 7) / 8, L), 256, 0, st>>>(h, W_dq, c, B, d, r);
+        LSA_TRY(launched("project c"));
+        k_rowdot<DT_BF16, DT_F32><<<dim3((n_h + 7) / 8, L), 256, 0, st>>>(h, W_w, w_out, B, d, n_h);
+        LSA_TRY(launched("project w"));
+        k_rowdot<DT_BF16, DT_BF16><<<dim3((nq + 7) / 8, L), 256, 0, st>>>(c, W_iuq, q_out, B, r, nq);
+        LSA_TRY(launched("project q"));
+    } else {
+        k_rowdot<DT_F32, DT_F32><<<dim3((r + 7) / 8, L), 256, 0, st>>>(h, W_dq, c, B, d, r);
+        LSA_TRY(launched("project c"));
+        k_rowdot<DT_F32, DT_F32><<<dim3((n_h + 7) / 8, L), 256, 0, st>>>(h, W_w, w_out, B, d, n_h);
+        LSA_TRY(launched("project w"));
+        k_rowdot<DT_F32, DT_F32><<<dim3((nq + 7) / 8, L), 256, 0, st>>>(c, W_iuq, q_out, B, r, nq);
+        LSA_TRY(launched("project q"));
+    }
+    return ok();
+}
+
+// ------------------------------------------------------------------------------ stages 2-4a
+
+size_t lsa_score_select_workspace_size(int L, int B, int64_t total_S)
+{
+    (void)L;
+    if (B <= 0 || total_S < 0) return 0;
+    return score_ws_bytes(B, total_S);
+}
+
+lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *K, const float *k_scale,
+                                     lsa_dtype kdt, const int64_t *seq_offsets, int64_t total_S, int L, int B,
+                                     int n_h, int d_I, float threshold, float *scores_out, uint8_t *mask_out,
+                                     int32_t *idx_out, int32_t *count_out, void *workspace,
+                                     size_t workspace_bytes, lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(q && w && K && seq_offsets && idx_out && count_out, "lsa_memindex_score_select: null pointer");
+    LSA_REQUIRE(L > 0 && B > 0 && n_h > 0 && d_I > 0 && total_S >= 0,
+                "lsa_memindex_score_select: sizes must be positive");
+    LSA_REQUIRE(total_S < (int64_t)1 << 31, "lsa_memindex_score_select: total_S must be below 2^31");
+    if (!valid_dtype(kdt)) return fail(LSA_ERR_UNSUPPORTED, "lsa_memindex_score_select: unknown key dtype");
+    LSA_REQUIRE((kdt == LSA_FP8_E4M3) == (k_scale != nullptr),
+                "lsa_memindex_score_select: k_scale is required for FP8 keys and must be NULL otherwise");
+    LSA_REQUIRE(threshold > 0.f && threshold < 1.f, "lsa_memindex_score_select: threshold must be in (0, 1)");
+    const size_t need = score_ws_bytes(B, total_S);
+    if (!workspace || workspace_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "lsa_memindex_score_select: workspace needs %zu bytes", need);
+    LSA_REQUIRE(aligned(workspace, 256), "lsa_memindex_score_select: workspace must be 256-byte aligned");
+    const float thr_logit = (float)log((double)threshold / (1.0 - (double)threshold));
+    ScoreWs ws = score_ws(workspace, B);
+
+    k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, ws.tile_start);
+    LSA_TRY(launched("tile setup"));
+
+    const bool tc = (n_h == 64 && d_I == 128 && (kdt == LSA_BF16 || kdt == LSA_FP8_E4M3) && tc_score_available());
+    if (tc) {
+        LSA_REQUIRE(aligned(q, 16) && aligned(K, 16), "lsa_memindex_score_select: q and K must be 16-byte aligned");
+        LSA_TRY(launch_score_tc(q, w, K, k_scale, kdt, seq_offsets, ws.tile_start, B, total_S, L, thr_logit,
+                                scores_out, ws.tile_mask, num_sms(), st));
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    } else {
+        if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_memindex_score_select: n_h must be <= 128");
+        switch (d_I) {
+        case 32: LSA_TRY(score_simt_d<32>(kdt, q, w, K, k_scale, seq_offsets, ws.tile_start, B, total_S, L, n_h,
+                                          thr_logit, scores_out, ws.tile_mask, st)); break;
+        case 64: LSA_TRY(score_simt_d<64>(kdt, q, w, K, k_scale, seq_offsets, ws.tile_start, B, total_S, L, n_h,
+                                          thr_logit, scores_out, ws.tile_mask, st)); break;
+        case 128: LSA_TRY(score_simt_d<128>(kdt, q, w, K, k_scale, seq_offsets, ws.tile_start, B, total_S, L, n_h,
+                                            thr_logit, scores_out, ws.tile_mask, st)); break;
+        default: return fail(LSA_ERR_UNSUPPORTED, "lsa_memindex_score_select: d_I must be 32, 64 or 128");
+        }
+    }
+    k_compact<<<B, 1024, 0, st>>>(ws.tile_mask, ws.tile_start, seq_offsets, B, idx_out, count_out, mask_out);
+    LSA_TRY(launched("compact"));
+    return ok();
+}
+
+// ------------------------------------------------------------------------------ stage 4b
+
+lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int64_t *seq_offsets, int64_t total_S,
+                            int B, const void *pool, size_t row_bytes, void *hot_kv, const void *K_sel,
+                            const float *k_scale_sel, lsa_dtype kdt, int d_I, void *hot_K, float *hot_scale,
+                            lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(idx && count && seq_offsets && pool && hot_kv, "lsa_fetch_gather: null pointer");
+    LSA_REQUIRE(B > 0 && total_S >= 0, "lsa_fetch_gather: sizes must be positive");
+    LSA_REQUIRE(row_bytes > 0 && row_bytes % 16 == 0, "lsa_fetch_gather: row_bytes must be a positive multiple of 16");
+    if (row_bytes > 16 * 32 * GATHER_MAX_CHUNKS)
+        return fail(LSA_ERR_UNSUPPORTED, "lsa_fetch_gather: row_bytes above %d", 16 * 32 * GATHER_MAX_CHUNKS);
+    LSA_REQUIRE(aligned(pool, 16) && aligned(hot_kv, 16), "lsa_fetch_gather: pool and hot_kv must be 16-byte aligned");
+    void *dpool = nullptr;
+    cudaError_t e = cudaHostGetDevicePointer(&dpool, const_cast<void *>(pool), 0);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(LSA_ERR_INVALID_ARG, "lsa_fetch_gather: pool is not mapped page-locked host memory (%s)",
+                    cudaGetErrorString(e));
+    }
+    int krow16 = 0;
+    if (K_sel) {
+        if (!valid_dtype(kdt)) return fail(LSA_ERR_UNSUPPORTED, "lsa_fetch_gather: unknown key dtype");
+        LSA_REQUIRE(hot_K && d_I > 0, "lsa_fetch_gather: hot_K and d_I are required with K_sel");
+        LSA_REQUIRE((kdt == LSA_FP8_E4M3) == (k_scale_sel != nullptr) && (!k_scale_sel || hot_scale),
+                    "lsa_fetch_gather: scales are required for FP8 keys (and only for them)");
+        const size_t kb = (size_t)d_I * elem_bytes(kdt);
+        LSA_REQUIRE(kb % 16 == 0 && aligned(K_sel, 16) && aligned(hot_K, 16),
+                    "lsa_fetch_gather: key rows must be whole 16-byte chunks, 16-byte aligned");
+        krow16 = (int)(kb / 16);
+    }
+    const int warps_per_block = 8;
+    int64_t gx = ((total_S / (B > 0 ? B : 1)) + warps_per_block * GATHER_ROWS_PER_WARP - 1) /
+                 (warps_per_block * GATHER_ROWS_PER_WARP);
+    const int64_t cap = (int64_t)num_sms() * 4 / B + 1;
+    if (gx > cap) gx = cap;
+    if (gx < 1) gx = 1;
+    k_gather<<<dim3((unsigned)gx, (unsigned)B), 32 * warps_per_block, 0, st>>>(
+        idx, count, seq_offsets, (const uint8_t *)dpool, (int)(row_bytes / 16), (uint8_t *)hot_kv,
+        (const uint8_t *)K_sel, k_scale_sel, krow16, (uint8_t *)hot_K, hot_scale);
+    LSA_TRY(launched("gather"));
+    return ok();
+}
+
+// ------------------------------------------------------------------------------ stage 5
+
+size_t lsa_lightning_topk_workspace_size(int B, int tau, int64_t total_S, int k)
+{
+    (void)B; (void)k;
+    if (tau <= 0 || total_S < 0) return 0;
+    return align_up(sizeof(float) * (size_t)tau * (size_t)total_S, 256) + 256;
+}
+
+lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void *hot_K, const float *hot_scale,
+                              lsa_dtype kdt, const int32_t *idx, const int32_t *count, const int64_t *seq_offsets,
+                              int64_t total_S, int B, int tau, int n_h, int d_I, int k, int32_t *topk_idx,
+                              float *topk_score, void *workspace, size_t workspace_bytes, lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(q_dec && w_dec && hot_K && idx && count && seq_offsets && topk_idx, "lsa_lightning_topk: null pointer");
+    LSA_REQUIRE(B > 0 && tau > 0 && n_h > 0 && d_I > 0 && total_S >= 0, "lsa_lightning_topk: sizes must be positive");
+    LSA_REQUIRE(k >= 1 && k <= LSA_MAX_TOPK, "lsa_lightning_topk: k must be in [1, %d]", LSA_MAX_TOPK);
+    if (!valid_dtype(kdt)) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: unknown key dtype");
+    LSA_REQUIRE((kdt == LSA_FP8_E4M3) == (hot_scale != nullptr),
+                "lsa_lightning_topk: hot_scale is required for FP8 keys and must be NULL otherwise");
+    const size_t need = lsa_lightning_topk_workspace_size(B, tau, total_S, k);
+    if (!workspace || workspace_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "lsa_lightning_topk: workspace needs %zu bytes", need);
+    LSA_REQUIRE(aligned(workspace, 256), "lsa_lightning_topk: workspace must be 256-byte aligned");
+    LSA_REQUIRE((int64_t)tau * total_S < ((int64_t)1 << 40), "lsa_lightning_topk: tau * total_S too large");
+    if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: n_h must be <= 128");
+    float *Y = (float *)workspace;
+    switch (d_I) {
+    case 32: LSA_TRY(li_simt_d<32>(kdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
+    case 64: LSA_TRY(li_simt_d<64>(kdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
+    case 128: LSA_TRY(li_simt_d<128>(kdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
+    default: return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: d_I must be 32, 64 or 128");
+    }
+    int kpow2 = 1;
+    while (kpow2 < k) kpow2 <<= 1;
+    const size_t smem = sizeof(unsigned long long) * (size_t)kpow2;
+    LSA_TRY(set_smem(k_topk_select, smem));
+    k_topk_select<<<(unsigned)((int64_t)B * tau), SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, tau, k, kpow2,
+                                                                         topk_idx, topk_score);
+    LSA_TRY(launched("top-k select"));
+    return ok();
+}
+
+// ------------------------------------------------------------------------------ pool helpers
+
+lsa_status lsa_pool_alloc(size_t bytes, void **ptr)
+{
+    LSA_REQUIRE(ptr && bytes > 0, "lsa_pool_alloc: bad arguments");
+    *ptr = nullptr;
+    cudaError_t e = cudaHostAlloc(ptr, bytes, cudaHostAllocMapped | cudaHostAllocPortable);
+    if (e != cudaSuccess) {
+        *ptr = nullptr;
+        return fail(LSA_ERR_CUDA, "cudaHostAlloc(%zu): %s", bytes, cudaGetErrorString(e));
+    }
+    return ok();
+}
+
+lsa_status lsa_pool_free(void *ptr)
+{
+    if (!ptr) return ok();
+    cudaError_t e = cudaFreeHost(ptr);
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "cudaFreeHost: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,194 @@
+// Stage 5: native Lightning-Indexer score over the fetched entries and per-query Top-k
+// (blog review "FlashMemory-DeepSeek-V4", sections 2.2 and 3.2).
+//
+// Scores of sequence b, query i, fetched slot j live at Y[tau*off_b + i*S_b + j] (fp32).
+// Selection: per query, a radix select on order-preserving 32-bit keys (4 passes of 8 bits)
+// finds the k-th largest score; the survivors (all larger keys, plus the first equal keys in
+// slot order, i.e. smallest entry index) are sorted by (score desc, entry asc) with a bitonic
+// sort in shared memory.
+#pragma once
+#include "common.cuh"
+
+namespace lsa {
+
+// SIMT score: one thread per fetched slot, all tau queries of its sequence.
+template <int D, int KDT, int QDT>
+__global__ void __launch_bounds__(TILE) k_li_score_simt(const void *__restrict__ qd, const float *__restrict__ wd,
+                                                         const void *__restrict__ hotK,
+                                                         const float *__restrict__ hotsc,
+                                                         const int32_t *__restrict__ count,
+                                                         const int64_t *__restrict__ offs, int tau, int n_h,
+                                                         float *__restrict__ Y)
+{
+    extern __shared__ float smem[];
+    float *sq = smem;
+    float *sw = smem + n_h * D;
+    const int b = blockIdx.y;
+    const int64_t off = offs[b], S = offs[b + 1] - offs[b];
+    int F = count[b];
+    F = F < 0 ? 0 : (F > S ? (int)S : F);
+    for (int64_t j0 = (int64_t)blockIdx.x * TILE; j0 < F; j0 += (int64_t)gridDim.x * TILE) {
+        const int64_t j = j0 + threadIdx.x;
+        const bool valid = j < F;
+        float kr[D];
+        float scale = 1.f;
+        if (valid) {
+#pragma unroll
+            for (int e = 0; e < D; e++) kr[e] = load_elem<KDT>(hotK, (off + j) * D + e);
+            if (hotsc) {
+                scale = hotsc[off + j];
+                if (!(scale >= 0.f)) flag(ERRF_SCALE);
+            }
+        }
+        for (int i = 0; i < tau; i++) {
+            __syncthreads();
+            const int64_t q0 = (((int64_t)b * tau + i) * n_h) * D;
+            for (int t = threadIdx.x; t < n_h * D; t += blockDim.x) sq[t] = load_elem<QDT>(qd, q0 + t);
+            for (int t = threadIdx.x; t < n_h; t += blockDim.x) sw[t] = wd[((int64_t)b * tau + i) * n_h + t];
+            __syncthreads();
+            if (!valid) continue;
+            float y = 0.f;
+            for (int h = 0; h < n_h; h++) {
+                float dot = 0.f;
+#pragma unroll
+                for (int e = 0; e < D; e++) dot = fmaf(sq[h * D + e], kr[e], dot);
+                y = fmaf(sw[h], fmaxf(dot * scale, 0.f), y);
+            }
+            Y[(int64_t)tau * off + (int64_t)i * S + j] = y;
+        }
+    }
+}
+
+constexpr int SEL_THREADS = 512;
+
+// Block-wide exclusive scan of one int per thread (SEL_THREADS threads); returns the
+// exclusive prefix and writes the block total to *total.  Ends with a barrier.
+__device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int inc = warp_incl_scan(v);
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int t = lane < SEL_THREADS / 32 ? warp_tot[lane] : 0;
+        int ti = warp_incl_scan(t);
+        if (lane < SEL_THREADS / 32) warp_tot[lane] = ti - t;
+        if (lane == 31) *total = ti;
+    }
+    __syncthreads();
+    const int r = warp_tot[warp] + inc - v;
+    __syncthreads();
+    return r;
+}
+
+// One block per (sequence, query).  kpow2 = next power of two >= k (shared: kpow2 x 8 bytes).
+__global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__restrict__ Y,
+                                                             const int32_t *__restrict__ idx,
+                                                             const int32_t *__restrict__ count,
+                                                             const int64_t *__restrict__ offs, int tau, int k,
+                                                             int kpow2, int32_t *__restrict__ topk_idx,
+                                                             float *__restrict__ topk_score)
+{
+    extern __shared__ unsigned long long sel[];  // (key << 32) | ~slot
+    __shared__ unsigned int hist[256];
+    __shared__ int warp_tot[32];
+    __shared__ int tot_a, tot_b;
+    __shared__ unsigned int s_prefix, s_remaining;
+
+    const int b = blockIdx.x / tau, i = blockIdx.x % tau;
+    const int64_t off = offs[b], S = offs[b + 1] - offs[b];
+    int F = count[b];
+    F = F < 0 ? 0 : (F > S ? (int)S : F);
+    const float *row = Y + (int64_t)tau * off + (int64_t)i * S;
+
+    for (int t = threadIdx.x; t < kpow2; t += SEL_THREADS) sel[t] = 0ull;
+    __syncthreads();
+
+    if (F <= k) {
+        for (int j = threadIdx.x; j < F; j += SEL_THREADS)
+            sel[j] = ((unsigned long long)float_to_ordered(row[j]) << 32) | (uint32_t)(~(uint32_t)j);
+    } else {
+        uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
+        for (int pass = 0; pass < 4; pass++) {
+            const int shift = 24 - 8 * pass;
+            for (int t = threadIdx.x; t < 256; t += SEL_THREADS) hist[t] = 0;
+            __syncthreads();
+            for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
+                const uint32_t u = float_to_ordered(row[j]);
+                if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                uint32_t cum = 0, chosen = 0;
+                for (int d = 255; d >= 0; d--) {
+                    if (cum + hist[d] >= remaining) {
+                        chosen = (uint32_t)d;
+                        break;
+                    }
+                    cum += hist[d];
+                }
+                s_remaining = remaining - cum;
+                s_prefix = prefix | (chosen << shift);
+            }
+            __syncthreads();
+            prefix = s_prefix;
+            remaining = s_remaining;
+            pmask |= 255u << shift;
+            __syncthreads();
+        }
+        // prefix is now the k-th largest key; take every larger key and the first `remaining`
+        // equal keys in slot order.
+        int carry_gt = 0, carry_eq = 0;
+        const int n_gt_total = k - (int)remaining;
+        for (int base = 0; base < F; base += SEL_THREADS) {
+            const int j = base + threadIdx.x;
+            uint32_t u = 0;
+            int gt = 0, eq = 0;
+            if (j < F) {
+                u = float_to_ordered(row[j]);
+                gt = u > prefix;
+                eq = u == prefix;
+            }
+            const int pg = block_excl_scan(gt, warp_tot, &tot_a) + carry_gt;
+            const int pe = block_excl_scan(eq, warp_tot, &tot_b) + carry_eq;
+            if (gt) sel[pg] = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);
+            if (eq && pe < (int)remaining)
+                sel[n_gt_total + pe] = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);
+            carry_gt += tot_a;
+            carry_eq += tot_b;
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    // bitonic sort, descending
+    for (int size = 2; size <= kpow2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = threadIdx.x; t < kpow2 / 2; t += SEL_THREADS) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool desc = ((lo & size) == 0);
+                const unsigned long long a = sel[lo], c = sel[hi];
+                if ((a < c) == desc) {
+                    sel[lo] = c;
+                    sel[hi] = a;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    const int nsel = F < k ? F : k;
+    const int64_t o0 = ((int64_t)b * tau + i) * k;
+    for (int r = threadIdx.x; r < k; r += SEL_THREADS) {
+        if (r < nsel) {
+            const unsigned long long v = sel[r];
+            const uint32_t j = ~(uint32_t)(v & 0xffffffffull);
+            topk_idx[o0 + r] = __ldg(idx + off + j);
+            if (topk_score) topk_score[o0 + r] = ordered_to_float((uint32_t)(v >> 32));
+        } else {
+            topk_idx[o0 + r] = -1;
+            if (topk_score) topk_score[o0 + r] = -INFINITY;
+        }
+    }
+}
+
+}  // namespace lsa

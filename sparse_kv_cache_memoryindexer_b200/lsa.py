@@ -1,0 +1,203 @@
+"""Python binding of liblsa.so (include/lsa.h): argument marshalling only.
+
+Each function takes torch tensors, checks device/dtype/shape/contiguity, and passes raw
+pointers to the C entry point of the same name; every step runs in the library's CUDA
+kernels.  There is no CPU path: if liblsa.so is missing or fails to load, importing this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsa.so")
+
+LSA_F32, LSA_BF16, LSA_FP8_E4M3 = 0, 1, 2
+LSA_MAX_TOPK = 4096
+_STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "LSA_ERR_CUDA",
+           4: "LSA_ERR_DEVICE_CHECK", 5: "LSA_ERR_WORKSPACE"}
+DTYPE_CODE = {torch.float32: LSA_F32, torch.bfloat16: LSA_BF16, torch.float8_e4m3fn: LSA_FP8_E4M3}
+
+# every function declared in include/lsa.h
+EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_device",
+           "lsa_project_workspace_size", "lsa_project",
+           "lsa_score_select_workspace_size", "lsa_memindex_score_select",
+           "lsa_fetch_gather",
+           "lsa_lightning_topk_workspace_size", "lsa_lightning_topk",
+           "lsa_pool_alloc", "lsa_pool_free")
+
+
+class LSAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run sparse_kv_cache_memoryindexer_b200/build.py "
+                          "(or __graft_entry__.build())")
+    lib = C.CDLL(LIB_PATH)
+    P, I, I64, SZ, F = C.c_void_p, C.c_int, C.c_int64, C.c_size_t, C.c_float
+    sig = {
+        "lsa_last_error": (C.c_char_p, []),
+        "lsa_version": (C.c_char_p, []),
+        "lsa_launch_count": (C.c_uint64, []),
+        "lsa_check_device": (I, [P]),
+        "lsa_project_workspace_size": (SZ, [I, I, I, I, I, I, I]),
+        "lsa_project": (I, [P, P, P, P, I, I, I, I, I, I, I, P, P, P, SZ, P]),
+        "lsa_score_select_workspace_size": (SZ, [I, I, I64]),
+        "lsa_memindex_score_select": (I, [P, P, P, P, I, P, I64, I, I, I, I, F, P, P, P, P, P, SZ, P]),
+        "lsa_fetch_gather": (I, [P, P, P, I64, I, P, SZ, P, P, P, I, I, P, P, P]),
+        "lsa_lightning_topk_workspace_size": (SZ, [I, I, I64, I]),
+        "lsa_lightning_topk": (I, [P, P, P, P, I, P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P]),
+        "lsa_pool_alloc": (I, [SZ, C.POINTER(C.c_void_p)]),
+        "lsa_pool_free": (I, [P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, args
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise LSAError(status, _lib.lsa_last_error().decode())
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the LSA library must be contiguous")
+    return t.data_ptr()
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None and t.device.type != "cuda":
+            raise ValueError("device tensor expected (got a CPU tensor)")
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def version() -> str:
+    return _lib.lsa_version().decode()
+
+
+def launch_count() -> int:
+    return int(_lib.lsa_launch_count())
+
+
+def lsa_check_device(stream=None):
+    _check(_lib.lsa_check_device(_stream(stream)))
+
+
+# ------------------------------------------------------------------------ stage 1
+
+def lsa_project_workspace_size(L, B, d, r, n_h, d_I, dt) -> int:
+    return int(_lib.lsa_project_workspace_size(L, B, d, r, n_h, d_I, DTYPE_CODE[dt]))
+
+
+def lsa_project(h, W_dq, W_iuq, W_w, q_out, w_out, workspace, stream=None):
+    """c^Q = h W^DQ, q = c^Q W^IUQ, w = h W^w for every layer and sequence (see include/lsa.h)."""
+    _dev(h, W_dq, W_iuq, W_w, q_out, w_out, workspace)
+    L, B, d = h.shape
+    r = W_dq.shape[1]
+    _, _, n_h, d_I = q_out.shape
+    _check(_lib.lsa_project(_p(h), _p(W_dq), _p(W_iuq), _p(W_w), DTYPE_CODE[h.dtype], L, B, d, r, n_h, d_I,
+                            _p(q_out), _p(w_out), _p(workspace), workspace.numel() * workspace.element_size(),
+                            _stream(stream)))
+
+
+# ------------------------------------------------------------------------ stages 2-4a
+
+def lsa_score_select_workspace_size(L, B, total_S) -> int:
+    return int(_lib.lsa_score_select_workspace_size(L, B, total_S))
+
+
+def lsa_memindex_score_select(q, w, K, k_scale, seq_offsets, total_S, threshold, idx_out, count_out,
+                              workspace, scores_out=None, mask_out=None, stream=None):
+    """Index score, threshold, OR over layers and compaction (see include/lsa.h)."""
+    _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, workspace, scores_out, mask_out)
+    L, B, n_h, d_I = q.shape
+    _check(_lib.lsa_memindex_score_select(
+        _p(q), _p(w), _p(K), _p(k_scale), DTYPE_CODE[K.dtype], _p(seq_offsets), int(total_S), L, B, n_h, d_I,
+        float(threshold), _p(scores_out), _p(mask_out), _p(idx_out), _p(count_out), _p(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ------------------------------------------------------------------------ stage 4b
+
+def lsa_fetch_gather(idx, count, seq_offsets, total_S, pool, hot_kv, K_sel=None, k_scale_sel=None,
+                     hot_K=None, hot_scale=None, stream=None):
+    """Gather fetched rows from the mapped host cold pool (and the keys of one layer)."""
+    _dev(idx, count, seq_offsets, hot_kv, K_sel, k_scale_sel, hot_K, hot_scale)
+    if pool.device.type != "cpu":
+        raise ValueError("the cold pool must be (mapped page-locked) host memory")
+    B = count.numel()
+    row_bytes = pool.shape[1] * pool.element_size()
+    kdt = DTYPE_CODE[K_sel.dtype] if K_sel is not None else 0
+    d_I = K_sel.shape[-1] if K_sel is not None else 0
+    _check(_lib.lsa_fetch_gather(_p(idx), _p(count), _p(seq_offsets), int(total_S), B, _p(pool), row_bytes,
+                                 _p(hot_kv), _p(K_sel), _p(k_scale_sel), kdt, d_I, _p(hot_K), _p(hot_scale),
+                                 _stream(stream)))
+
+
+# ------------------------------------------------------------------------ stage 5
+
+def lsa_lightning_topk_workspace_size(B, tau, total_S, k) -> int:
+    return int(_lib.lsa_lightning_topk_workspace_size(B, tau, total_S, k))
+
+
+def lsa_lightning_topk(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, total_S, k, topk_idx,
+                       workspace, topk_score=None, stream=None):
+    """Native Lightning-Indexer Top-k over the fetched entries (see include/lsa.h)."""
+    _dev(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, topk_score)
+    B, tau, n_h, d_I = q_dec.shape
+    _check(_lib.lsa_lightning_topk(_p(q_dec), _p(w_dec), _p(hot_K), _p(hot_scale), DTYPE_CODE[hot_K.dtype],
+                                   _p(idx), _p(count), _p(seq_offsets), int(total_S), B, tau, n_h, d_I, int(k),
+                                   _p(topk_idx), _p(topk_score), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ------------------------------------------------------------------------ cold pool
+
+class MappedPool:
+    """Mapped page-locked host buffer from lsa_pool_alloc, viewed as a uint8 tensor [rows][row_bytes]."""
+
+    def __init__(self, rows: int, row_bytes: int):
+        ptr = C.c_void_p()
+        _check(_lib.lsa_pool_alloc(rows * row_bytes, C.byref(ptr)))
+        self.ptr = ptr.value
+        self.nbytes = rows * row_bytes
+        arr = (C.c_uint8 * self.nbytes).from_address(self.ptr)
+        self.tensor = torch.frombuffer(arr, dtype=torch.uint8).view(rows, row_bytes)
+
+    def free(self):
+        if self.ptr:
+            self.tensor = None
+            _check(_lib.lsa_pool_free(self.ptr))
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass

@@ -275,12 +275,14 @@ def _hidden_for(wl: Workload, l: int, bid: int, W_w64: np.ndarray, QR, w_t: np.n
     return h
 
 
-def make_inputs(wl: Workload, parts=("proj", "score", "pool", "dec"), threads: int = _THREADS) -> Inputs:
+def make_inputs(wl: Workload, parts=("proj", "score", "pool", "dec"), threads: int = _THREADS,
+                pool_out: torch.Tensor = None) -> Inputs:
     """Draw the inputs of ``wl``.
 
     parts: "proj" (h and projection weights), "score" (stage-level q, w and the keys),
     "pool" (cold-pool KV rows), "dec" (decode-step queries of the Lightning Indexer).
-    Keys are always drawn when "score" or "proj" is requested.
+    Keys are always drawn when "score" or "proj" is requested.  pool_out: an existing uint8
+    [sum S][row_bytes] host tensor (e.g. mapped page-locked memory) to fill in place.
     """
     parts = set(parts)
     ids = wl._ids()
@@ -341,7 +343,7 @@ def make_inputs(wl: Workload, parts=("proj", "score", "pool", "dec"), threads: i
 
     if "pool" in parts:
         T = wl.total_S
-        pool = torch.empty((T, wl.row_bytes), dtype=torch.uint8)
+        pool = pool_out if pool_out is not None else torch.empty((T, wl.row_bytes), dtype=torch.uint8)
 
         def pjob(b):
             s0, s1 = int(offs[b]), int(offs[b + 1])

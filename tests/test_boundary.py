@@ -1,0 +1,71 @@
+"""The C-ABI library: it loads without a GPU, exports every function include/lsa.h declares,
+and rejects bad arguments on the host before touching the device."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HDR = os.path.join(ROOT, "include", "lsa.h")
+
+
+def declared():
+    src = open(HDR).read()
+    return sorted(set(re.findall(r"^(?:lsa_status|size_t|const char \*|uint64_t)\s*\*?\s*(lsa_\w+)\(", src, re.M)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared()
+    for n in ("lsa_project", "lsa_memindex_score_select", "lsa_fetch_gather", "lsa_lightning_topk"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    out = subprocess.run(["nm", "-D", "--defined-only", lsa.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(lsa_\w+)$", out, re.M))
+    missing = [n for n in declared() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    assert set(lsa.EXPORTS) == set(declared())
+    for n in declared():
+        assert hasattr(lsa.library(), n)
+
+
+def test_library_is_built_for_sm100a_only():
+    from sparse_kv_cache_memoryindexer_b200 import build
+    log = open(os.path.join(os.path.dirname(build.LIB), "build.log")).read().splitlines()[0]
+    assert "arch=compute_100a,code=sm_100a" in log
+
+
+def test_host_side_validation_without_gpu():
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    lib = lsa.library()
+    # null pointers are rejected before any CUDA call
+    assert lib.lsa_project(None, None, None, None, 1, 1, 1, 8, 8, 1, 1, None, None, None, 0, None) == 1
+    assert b"null pointer" in lib.lsa_last_error()
+    assert lib.lsa_memindex_score_select(None, None, None, None, 1, None, 0, 1, 1, 1, 1, 0.5, None, None, None,
+                                         None, None, 0, None) == 1
+    assert lib.lsa_fetch_gather(None, None, None, 0, 1, None, 1024, None, None, None, 0, 0, None, None, None) == 1
+    assert lib.lsa_lightning_topk(None, None, None, None, 1, None, None, None, 0, 1, 1, 1, 1, 1, None, None, None, 0,
+                                  None) == 1
+    # threshold outside (0, 1), k above the maximum, unsupported dtype
+    p = C.c_void_p(256)
+    assert lib.lsa_memindex_score_select(p, p, p, None, 1, p, 10, 1, 1, 4, 32, 1.5, None, None, p, p, p, 1 << 20,
+                                         None) == 1
+    assert lib.lsa_lightning_topk(p, p, p, None, 1, p, p, p, 10, 1, 1, 1, 32, 5000, p, None, p, 1 << 20, None) == 1
+    assert lib.lsa_project(p, p, p, p, 2, 1, 1, 8, 8, 1, 1, p, p, p, 1 << 20, None) == 2
+    # a workspace that is too small
+    assert lib.lsa_memindex_score_select(p, p, p, None, 1, p, 1 << 20, 3, 4, 64, 128, 0.5, None, None, p, p, p, 16,
+                                         None) == 5
+    assert b"workspace needs" in lib.lsa_last_error()
+
+
+def test_workspace_sizes_cover_their_buffers():
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    import torch
+    T = 262144 * 32
+    assert lsa.lsa_score_select_workspace_size(3, 32, T) >= (T // 128) * 16
+    assert lsa.lsa_lightning_topk_workspace_size(32, 64, T, 2048) >= 64 * T * 4
+    assert lsa.lsa_project_workspace_size(3, 32, 4096, 2048, 64, 128, torch.bfloat16) >= 3 * 32 * 2048 * 2

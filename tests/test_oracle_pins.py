@@ -410,10 +410,10 @@ def test_pin(pin):
 
 MUTANTS = {
     "relu_dropped": ("x += (double)w[w0 + hh] * (dot > 0.0 ? dot : 0.0);", "x += (double)w[w0 + hh] * dot;"),
-    "strict_threshold": ("if (x >= t)\n                    fetched = 1;", "if (x > t)\n                    fetched = 1;"),
+    "strict_threshold": ("if (x >= t)\n                f = 1;", "if (x > t)\n                f = 1;"),
     "q_transposed": ("dot += elem(q, qdt, q0 + (size_t)hh * d_I + e)", "dot += elem(q, qdt, q0 + (size_t)e * n_h + hh)"),
     "scale_dropped": ("        dot *= scale;\n        x +=", "        x +="),
-    "and_instead_of_or": ("            int fetched = 0;\n", "            int fetched = 0, nf = 0;\n"),
+    "and_instead_of_or": ("        int f = 0;\n", "        int f = 0, nf = 0;\n"),
     "tie_breaks_high": ("return (a->s > b->s) - (a->s < b->s);", "return (a->s < b->s) - (a->s > b->s);"),
     "topk_relu_dropped": ("y += (double)w_dec[w0 + hh] * (dot > 0.0 ? dot : 0.0);", "y += (double)w_dec[w0 + hh] * dot;"),
     "c_not_rounded": ("c[j] = round_to(dt, acc);", "c[j] = acc;"),
@@ -425,9 +425,8 @@ MUTANTS = {
 def _extra_edit(name, src):
     if name == "and_instead_of_or":
         # fetched only when every layer passes
-        src = src.replace("if (x >= t)\n                    fetched = 1;", "if (x >= t)\n                    nf++;")
-        src = src.replace("            if (mask_out) mask_out[off + s] = (uint8_t)fetched;",
-                          "            fetched = (nf == L);\n            if (mask_out) mask_out[off + s] = (uint8_t)fetched;")
+        src = src.replace("if (x >= t)\n                f = 1;", "if (x >= t)\n                nf++;")
+        src = src.replace("        fetched[row] = (uint8_t)f;", "        fetched[row] = (uint8_t)(nf == L);")
     return src
 
 
