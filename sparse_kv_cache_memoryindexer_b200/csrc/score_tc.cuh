@@ -1,15 +1,583 @@
-// Tensor-core (tcgen05) index score for n_h = 64, d_I = 128: not built yet in this revision.
+// Tensor-core (tcgen05 + TMEM + TMA) Memory-Indexer index score for n_h = 64, d_I = 128
+// (blog review "FlashMemory-DeepSeek-V4", section 3.1; OR rule: section 4.2):
+//     x_{l,s} = sum_h w_{l,h} ReLU(scale_s * (q_{l,h} . K_{l,s})),   fetched if x >= logit(thr) in any l.
+//
+// MMA orientation: one tile = 128 entries of one sequence.  For each layer the tile's keys are
+// the A operand (M = 128 rows = TMEM lanes, K = d_I = 128) and the 64 head queries are the B
+// operand (N = 64), so the accumulator row of entry s holds its 64 head dot products and the
+// ReLU-weighted head sum runs inside one thread (one TMEM lane per entry).  The 0.5 threshold,
+// the OR over layers and the ballot into fetch words are fused in the epilogue.
+//
+// Warp roles (persistent CTA per SM, contiguous range of tiles):
+//   warp 0        TMA producer: key tiles (one per (tile, layer)) and the queries of each sequence
+//   warp 1        TMEM allocator + MMA issuer (one elected thread)
+//   warps 2..5    epilogue: tcgen05.ld of the accumulator, score, threshold, OR, ballot
+//   warps 6..9    (E4M3 keys only) converters: E4M3 tile -> bf16 A tile in shared memory (exact)
+// Every wait is bounded (about 2 s of global time): on time-out the CTA flags ERRF_TIMEOUT,
+// stops issuing work, waits (bounded) for its own copies in flight, frees TMEM and returns.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 
 namespace lsa {
 
-inline bool tc_score_available() { return false; }
+namespace tc {
 
-inline lsa_status launch_score_tc(const void *, const float *, const void *, const float *, int, const int64_t *,
-                                  const int *, int, int64_t, int, float, float *, uint32_t *, int, cudaStream_t)
+constexpr int NH = 64;           // heads (MMA N)
+constexpr int DI = 128;          // head dim (MMA K)
+constexpr int NACC = 8;          // TMEM accumulator slots of 64 columns (512 columns)
+constexpr int MAX_STAGES = 8;
+constexpr int MAX_L = 4;
+constexpr uint32_t IDESC = (1u << 4)          // D = fp32
+                         | (1u << 7)          // A = bf16
+                         | (1u << 10)         // B = bf16
+                         | ((NH >> 3) << 17)  // N = 64
+                         | ((128 >> 4) << 24);// M = 128
+constexpr uint64_t WAIT_NS = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t gtime()
 {
-    return LSA_ERR_UNSUPPORTED;
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(a), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `parity` to complete; false on abort or time-out (which sets abort).
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int *abort_flag)
+{
+    if (mbar_try(a, parity)) return true;
+    const uint64_t t0 = gtime();
+    while (true) {
+        if (mbar_try(a, parity)) return true;
+        if (*abort_flag) return false;
+        if (gtime() - t0 > WAIT_NS) {
+            *abort_flag = 1;
+            flag(ERRF_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Warp-uniform wait: lane 0 polls, the whole warp receives the same answer, then every lane
+// observes the completed phase itself (one try that cannot fail: the phase cannot advance again
+// before this warp arrives on the paired barrier), which orders its later reads after it.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t a, uint32_t parity, volatile int *abort_flag)
+{
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(a, parity, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) (void)mbar_try(a, parity);
+    return ok != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(a), "l"(b), "r"(IDESC), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+// 32 lanes x 32 columns of fp32 from TMEM into 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// E4M3 x 2 (low byte first) -> bf16 x 2, exact: e4m3 -> f16 (exact) -> f32 -> bf16 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two)
+{
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    float2 f = __half22float2(__half2(h));
+    __nv_bfloat162 b = __float22bfloat162_rn(f);
+    return *reinterpret_cast<uint32_t *>(&b);
+}
+
+struct Params {
+    const float *w;          // [L][B][64]
+    const float *kscale;     // [L][T] or null
+    const int64_t *offs;     // [B+1]
+    const int *tile_start;   // [B+1]
+    float *scores_out;       // [L][T] or null
+    uint32_t *tile_mask;     // [tiles][4]
+    int64_t T;
+    int B, L, stages, astages;
+    float thr;
+};
+
+struct SeqTracker {
+    // Sequence b owning tile t, found by walking forward from the previous answer.
+    int b;
+    __device__ __forceinline__ int of(const int *tile_start, int B, int t)
+    {
+        while (b + 1 <= B && __ldg(tile_start + b + 1) <= t) b++;
+        return b;
+    }
+};
+
+// Shared-memory plan (offsets from a 1024-byte aligned base).
+struct Smem {
+    uint32_t kraw, abuf, qbuf, sw, bars, misc, total;
+    __host__ __device__ static Smem plan(bool fp8, int L, int stages, int astages)
+    {
+        Smem s;
+        const uint32_t kstage = fp8 ? 128 * 128 : 128 * 256;
+        s.kraw = 0;
+        s.abuf = s.kraw + kstage * stages;
+        s.qbuf = s.abuf + (fp8 ? 128 * 256 * astages : 0);
+        s.sw = s.qbuf + 2 * L * NH * DI * 2;
+        s.bars = s.sw + 4 * L * NH * 4;
+        s.misc = s.bars + 8 * (4 * MAX_STAGES + 4 + 2 * NACC);
+        s.total = s.misc + 64 + 1024;  // + alignment slack
+        return s;
+    }
+};
+
+template <bool FP8>
+__global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
+    k_score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const Smem sp = Smem::plan(FP8, p.L, p.stages, p.astages);
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t kraw = sbase + sp.kraw, abuf = sbase + sp.abuf, qbuf = sbase + sp.qbuf;
+    float *sw = (float *)(base + sp.sw);
+    const uint32_t bars = sbase + sp.bars;
+    // barrier addresses
+    auto full = [&](int i) { return bars + 8u * i; };
+    auto empty = [&](int i) { return bars + 8u * (MAX_STAGES + i); };
+    auto afull = [&](int i) { return bars + 8u * (2 * MAX_STAGES + i); };
+    auto aempty = [&](int i) { return bars + 8u * (3 * MAX_STAGES + i); };
+    auto qfull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + i); };
+    auto qempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 2 + i); };
+    auto tfull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 4 + i); };
+    auto tempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 4 + NACC + i); };
+    uint32_t *tmem_holder = (uint32_t *)(base + sp.misc);
+    volatile int *abort_flag = (volatile int *)(base + sp.misc + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int L = p.L, B = p.B;
+    const int64_t T = p.T;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < p.stages; i++) {
+            mbar_init(full(i), 1);
+            mbar_init(empty(i), FP8 ? 4 : 1);
+        }
+        for (int i = 0; i < p.astages; i++) {
+            mbar_init(afull(i), 4);
+            mbar_init(aempty(i), 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(qfull(i), 1);
+            mbar_init(qempty(i), 1);
+        }
+        for (int i = 0; i < NACC; i++) {
+            mbar_init(tfull(i), 1);
+            mbar_init(tempty(i), 4);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int NT = __ldg(p.tile_start + B);
+    const int G = gridDim.x;
+    const int t_begin = (int)((int64_t)blockIdx.x * NT / G);
+    const int t_end = (int)((int64_t)(blockIdx.x + 1) * NT / G);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&kmap) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&qmap) : "memory");
+            SeqTracker tr{0};
+            int stage = 0;
+            uint32_t phase = 0;
+            int qslot = 1, prev_b = -1;
+            uint32_t quse[2] = {0, 0};
+            uint32_t last_phase[MAX_STAGES];
+            bool issued[MAX_STAGES];
+            for (int i = 0; i < MAX_STAGES; i++) issued[i] = false;
+            const uint32_t kbytes = FP8 ? 128 * 128 : 128 * 256;
+            const uint32_t kstage = kbytes;
+            bool ok = true;
+            for (int t = t_begin; t < t_end && ok; t++) {
+                const int b = tr.of(p.tile_start, B, t);
+                if (b != prev_b) {
+                    qslot ^= 1;
+                    if (!mbar_wait(qempty(qslot), (quse[qslot] & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    quse[qslot]++;
+                    mbar_expect_tx(qfull(qslot), (uint32_t)L * NH * DI * 2);
+                    for (int l = 0; l < L; l++) {
+                        const uint32_t qd = qbuf + (uint32_t)(qslot * L + l) * NH * DI * 2;
+                        const int row = (l * B + b) * NH;
+                        tma_load_2d(qd, &qmap, 0, row, qfull(qslot));
+                        tma_load_2d(qd + NH * 128, &qmap, 64, row, qfull(qslot));
+                    }
+                    prev_b = b;
+                }
+                const int64_t row0 = __ldg(p.offs + b) + (int64_t)(t - __ldg(p.tile_start + b)) * TILE;
+                for (int l = 0; l < L; l++) {
+                    if (!mbar_wait(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_expect_tx(full(stage), kbytes);
+                    const uint32_t dst = kraw + (uint32_t)stage * kstage;
+                    const int y = (int)(l * T + row0);
+                    if (FP8) {
+                        tma_load_2d(dst, &kmap, 0, y, full(stage));
+                    } else {
+                        tma_load_2d(dst, &kmap, 0, y, full(stage));
+                        tma_load_2d(dst + 128 * 128, &kmap, 64, y, full(stage));
+                    }
+                    issued[stage] = true;
+                    last_phase[stage] = phase;
+                    if (++stage == p.stages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (*abort_flag) {
+                // let the copies this thread started land before the CTA exits
+                volatile int never = 0;
+                for (int i = 0; i < p.stages; i++)
+                    if (issued[i]) mbar_wait(full(i), last_phase[i], &never);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            SeqTracker tr{0};
+            int stage = 0, as = 0, acc = 0;
+            uint32_t phase = 0, aphase = 0, accphase = 0;
+            int qslot = 1, prev_b = -1;
+            uint32_t quse[2] = {0, 0};
+            bool ok = true;
+            for (int t = t_begin; t < t_end && ok; t++) {
+                const int b = tr.of(p.tile_start, B, t);
+                if (b != prev_b) {
+                    qslot ^= 1;
+                    if (!mbar_wait(qfull(qslot), quse[qslot] & 1, abort_flag)) { ok = false; break; }
+                    quse[qslot]++;
+                    prev_b = b;
+                }
+                const bool last_of_seq = (t + 1 == t_end) || (__ldg(p.tile_start + b + 1) <= t + 1);
+                for (int l = 0; l < L; l++) {
+                    uint32_t a_base;
+                    if (FP8) {
+                        if (!mbar_wait(afull(as), aphase, abort_flag)) { ok = false; break; }
+                        a_base = abuf + (uint32_t)as * 128 * 256;
+                    } else {
+                        if (!mbar_wait(full(stage), phase, abort_flag)) { ok = false; break; }
+                        a_base = kraw + (uint32_t)stage * 128 * 256;
+                    }
+                    if (!mbar_wait(tempty(acc), accphase ^ 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t b_base = qbuf + (uint32_t)(qslot * L + l) * NH * DI * 2;
+                    const uint32_t d = tmem + (uint32_t)acc * NH;
+#pragma unroll
+                    for (int kk = 0; kk < DI / 16; kk++) {
+                        const uint32_t ka = a_base + (uint32_t)(kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32;
+                        const uint32_t kb = b_base + (uint32_t)(kk >> 2) * (NH * 128) + (uint32_t)(kk & 3) * 32;
+                        mma_bf16(d, sdesc(ka), sdesc(kb), kk > 0 ? 1u : 0u);
+                    }
+                    if (FP8) {
+                        mma_commit(aempty(as));
+                        if (++as == p.astages) { as = 0; aphase ^= 1; }
+                    } else {
+                        mma_commit(empty(stage));
+                        if (++stage == p.stages) { stage = 0; phase ^= 1; }
+                    }
+                    mma_commit(tfull(acc));
+                    if (l == L - 1 && last_of_seq) mma_commit(qempty(qslot));
+                    if (++acc == NACC) { acc = 0; accphase ^= 1; }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ------------------------------------------------------------- epilogue
+        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+        float *myw = sw + (size_t)quarter * L * NH;
+        SeqTracker tr{0};
+        int acc = 0;
+        uint32_t accphase = 0;
+        int prev_b = -1;
+        bool ok = true;
+        for (int t = t_begin; t < t_end && ok; t++) {
+            const int b = tr.of(p.tile_start, B, t);
+            if (b != prev_b) {
+                __syncwarp();
+                for (int i = lane; i < L * NH; i += 32) {
+                    const int l = i / NH, h = i % NH;
+                    myw[i] = __ldg(p.w + ((int64_t)l * B + b) * NH + h);
+                }
+                __syncwarp();
+                prev_b = b;
+            }
+            const int64_t S = __ldg(p.offs + b + 1) - __ldg(p.offs + b);
+            const int64_t s = (int64_t)(t - __ldg(p.tile_start + b)) * TILE + quarter * 32 + lane;
+            const bool valid = s < S;
+            const int64_t row = __ldg(p.offs + b) + s;
+            bool fetched = false;
+            for (int l = 0; l < L; l++) {
+                if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * NH;
+                float v0[32], v1[32];
+                tmem_ld32(taddr, v0);
+                tmem_ld32(taddr + 32, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty(acc));
+                if (++acc == NACC) { acc = 0; accphase ^= 1; }
+                const float *wl = myw + l * NH;
+                float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+#pragma unroll
+                for (int h = 0; h < 32; h += 4) {
+                    const float4 wa = *(const float4 *)(wl + h);
+                    const float4 wb = *(const float4 *)(wl + 32 + h);
+                    x0 = fmaf(wa.x, fmaxf(v0[h], 0.f), x0);
+                    x1 = fmaf(wa.y, fmaxf(v0[h + 1], 0.f), x1);
+                    x2 = fmaf(wa.z, fmaxf(v0[h + 2], 0.f), x2);
+                    x3 = fmaf(wa.w, fmaxf(v0[h + 3], 0.f), x3);
+                    x0 = fmaf(wb.x, fmaxf(v1[h], 0.f), x0);
+                    x1 = fmaf(wb.y, fmaxf(v1[h + 1], 0.f), x1);
+                    x2 = fmaf(wb.z, fmaxf(v1[h + 2], 0.f), x2);
+                    x3 = fmaf(wb.w, fmaxf(v1[h + 3], 0.f), x3);
+                }
+                float x = (x0 + x1) + (x2 + x3);
+                if (valid) {
+                    if (FP8) {
+                        const float sc = __ldg(p.kscale + (int64_t)l * T + row);
+                        if (!(sc >= 0.f)) flag(ERRF_SCALE);
+                        x *= sc;  // ReLU(sc * d) = sc * ReLU(d) for sc >= 0
+                    }
+                    if (p.scores_out) p.scores_out[(int64_t)l * T + row] = 1.f / (1.f + expf(-x));
+                    fetched |= (x >= p.thr);
+                }
+            }
+            if (!ok) break;
+            const unsigned m = __ballot_sync(0xffffffffu, fetched);
+            if (lane == 0) p.tile_mask[(int64_t)t * 4 + quarter] = m;
+        }
+    } else if (FP8) {
+        // ------------------------------------------------------------- E4M3 -> bf16 converters
+        const int r = threadIdx.x - 6 * 32;  // tile row 0..127 handled by this thread
+        SeqTracker tr{0};
+        int stage = 0, as = 0;
+        uint32_t phase = 0, aphase = 0;
+        bool ok = true;
+        for (int t = t_begin; t < t_end && ok; t++) {
+            for (int l = 0; l < L; l++) {
+                if (!mbar_wait_warp(full(stage), phase, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(aempty(as), aphase ^ 1, abort_flag)) { ok = false; break; }
+                const uint32_t src = kraw + (uint32_t)stage * 128 * 128 + (uint32_t)r * 128;
+                const uint32_t dst = abuf + (uint32_t)as * 128 * 256 + (uint32_t)r * 128;
+#pragma unroll
+                for (int u = 0; u < 8; u++) {
+                    uint4 v;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(src + (uint32_t)((u ^ (r & 7)) * 16)));
+                    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        o[2 * k] = e4m3x2_to_bf16x2((uint16_t)(in[k] & 0xffffu));
+                        o[2 * k + 1] = e4m3x2_to_bf16x2((uint16_t)(in[k] >> 16));
+                    }
+                    // bf16 16-byte units 2u and 2u+1 of this row (chunk of 64 elements each)
+#pragma unroll
+                    for (int hv = 0; hv < 2; hv++) {
+                        const int vv = 2 * u + hv;
+                        const uint32_t da = dst + (uint32_t)(vv >> 3) * (128 * 128) +
+                                            (uint32_t)(((vv & 7) ^ (r & 7)) * 16);
+                        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(da), "r"(o[4 * hv]),
+                                     "r"(o[4 * hv + 1]), "r"(o[4 * hv + 2]), "r"(o[4 * hv + 3])
+                                     : "memory");
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(empty(stage));
+                    mbar_arrive(afull(as));
+                }
+                if (++stage == p.stages) { stage = 0; phase ^= 1; }
+                if (++as == p.astages) { as = 0; aphase ^= 1; }
+            }
+        }
+        (void)tr;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------------------------ host side
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    }
+    return fn;
+}
+
+inline bool tc_score_available()
+{
+    if (getenv("LSA_DISABLE_TC")) return false;
+    return tensor_map_encoder() != nullptr;
+}
+
+// 2D row-major tensor [rows][cols] of `elem`-byte elements; box [box_rows][box_cols]; 128B swizzle.
+inline bool make_map_2d(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int elem, uint64_t rows,
+                        uint64_t cols, uint32_t box_cols, uint32_t box_rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)elem};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, const float *kscale, int kdt,
+                                  const int64_t *offs, const int *tile_start, int B, int64_t T, int L,
+                                  float thr, float *scores_out, uint32_t *tile_mask, int sms, cudaStream_t st)
+{
+    using namespace tc;
+    if (L < 1 || L > 3) return LSA_ERR_UNSUPPORTED;
+    const bool fp8 = (kdt == DT_FP8);
+    CUtensorMap kmap, qmap;
+    const uint64_t rows = (uint64_t)L * (uint64_t)T;
+    if (rows == 0) return LSA_OK;
+    bool ok = fp8 ? make_map_2d(&kmap, K, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, DI, 128, 128)
+                  : make_map_2d(&kmap, K, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, DI, 64, 128);
+    ok = ok && make_map_2d(&qmap, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * B * NH, DI, 64, NH);
+    if (!ok) return LSA_ERR_CUDA;
+    Params p;
+    p.w = w;
+    p.kscale = kscale;
+    p.offs = offs;
+    p.tile_start = tile_start;
+    p.scores_out = scores_out;
+    p.tile_mask = tile_mask;
+    p.T = T;
+    p.B = B;
+    p.L = L;
+    p.thr = thr;
+    const int max_smem = 227 * 1024;
+    if (fp8) {
+        p.astages = 2;
+        p.stages = 4;
+        while (p.stages > 2 && Smem::plan(true, L, p.stages, p.astages).total > (uint32_t)max_smem) p.stages--;
+    } else {
+        p.astages = 0;
+        p.stages = MAX_STAGES;
+        while (p.stages > 2 && Smem::plan(false, L, p.stages, 0).total > (uint32_t)max_smem) p.stages--;
+    }
+    const uint32_t smem = Smem::plan(fp8, L, p.stages, p.astages).total;
+    if (smem > (uint32_t)max_smem) return LSA_ERR_UNSUPPORTED;
+    cudaError_t e;
+    if (fp8) {
+        e = cudaFuncSetAttribute(k_score_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return LSA_ERR_CUDA;
+        k_score_tc<true><<<sms, 320, smem, st>>>(kmap, qmap, p);
+    } else {
+        e = cudaFuncSetAttribute(k_score_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return LSA_ERR_CUDA;
+        k_score_tc<false><<<sms, 192, smem, st>>>(kmap, qmap, p);
+    }
+    e = cudaGetLastError();
+    return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }
 
 }  // namespace lsa

@@ -117,8 +117,9 @@ def _build_workloads():
 WORKLOADS = _build_workloads()
 
 
-def workload(name: str, **overrides) -> Workload:
-    wl = WORKLOADS[name]
+def workload(base: str, **overrides) -> Workload:
+    """A named workload, optionally with fields replaced (B alone repeats the base lengths)."""
+    wl = WORKLOADS[base]
     if "B" in overrides and "S" not in overrides:
         B = overrides["B"]
         overrides["S"] = tuple(wl.S[i % wl.B] for i in range(B))

@@ -73,8 +73,16 @@ def run_select(m, inp, thr=0.5, q=None, w=None):
 
 # ------------------------------------------------------------------ stages 2-4a
 
+@pytest.fixture(params=["default", "simt"])
+def kernel_path(request, monkeypatch):
+    """'default' takes the tensor-core kernel where it applies; 'simt' forces the SIMT kernel."""
+    if request.param == "simt":
+        monkeypatch.setenv("LSA_DISABLE_TC", "1")
+    return request.param
+
+
 @pytest.mark.parametrize("name", list(CASES))
-def test_select_parity(m, name):
+def test_select_parity(m, name, kernel_path):
     wl, inp = inputs(name)
     offs = inp.seq_offsets.numpy()
     ref = oracle.score(inp.q, inp.w, inp.K, inp.k_scale, offs)
