@@ -39,6 +39,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["lsa", "reference"], default="lsa")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's batch)")
     p.add_argument("--threshold", type=float, default=0.5)
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--cpu-sample", type=int, default=0,
@@ -183,7 +184,8 @@ def run_lsa(args, rank, world, device):
     import sparse_kv_cache_memoryindexer_b200 as lsa
     torch.cuda.set_device(device)
     base = synth.workload(args.workload)
-    wl = synth.workload(args.workload, seed=base.seed + 7919 * rank)
+    over = {"B": args.batch} if args.batch else {}
+    wl = synth.workload(args.workload, seed=base.seed + 7919 * rank, **over)
     T = wl.total_S
     dt, kdt = synth.DTYPES[wl.dtype], synth.DTYPES[wl.kdtype]
     pool = lsa.MappedPool(T, wl.row_bytes)

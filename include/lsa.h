@@ -132,7 +132,9 @@ lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *
  *   hot_kv                [T][row_bytes] device (capacity T; slots past count untouched)
  *   K_sel, k_scale_sel    [T][d_I] kdt and [T] fp32 (nullable: K_sel NULL skips the keys;
  *                         k_scale_sel required iff kdt = LSA_FP8_E4M3)
- *   hot_K, hot_scale      [T][d_I] kdt and [T] fp32
+ *   hot_K, hot_scale      [T][d_I] and [T] fp32.  hot_K holds kdt for LSA_F32 / LSA_BF16 keys
+ *                         and bf16 for LSA_FP8_E4M3 keys: the E4M3 codes are decoded exactly
+ *                         (every E4M3 value is a bf16 value); the scale stays in hot_scale.
  * Out-of-range indices or counts are skipped and flagged in the device error word.
  * ---------------------------------------------------------------------------------------- */
 lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count,
@@ -149,12 +151,15 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count,
  * ordered by y descending, ties to the smaller s; when count[b] < k the tail is -1 / -inf.
  *   q_dec      [B][tau][n_h][d_I]   fp32 when kdt = LSA_F32, else bf16
  *   w_dec      [B][tau][n_h]        fp32
- *   hot_K, hot_scale                as written by lsa_fetch_gather (hot_scale iff FP8)
+ *   hot_K, hot_scale                as written by lsa_fetch_gather (hot_scale iff FP8); kdt is
+ *                                   the dtype of the original keys (LSA_FP8_E4M3: hot_K is bf16)
  *   idx, count                      as written by lsa_memindex_score_select
  *   k                               1 .. LSA_MAX_TOPK
  *   topk_idx   [B][tau][k] int32
  *   topk_score [B][tau][k] fp32     (nullable)
- * Workspace: lsa_lightning_topk_workspace_size (holds the fp32 scores y).
+ * Kernels: tcgen05 tensor-core scoring for n_h = 64, d_I = 128, tau a multiple of 4 (bf16 or
+ * E4M3 keys); a SIMT path otherwise.  Then a radix select per query.
+ * Workspace: lsa_lightning_topk_workspace_size (work plan and the fp32 scores y).
  * ---------------------------------------------------------------------------------------- */
 size_t lsa_lightning_topk_workspace_size(int B, int tau, int64_t total_S, int k);
 

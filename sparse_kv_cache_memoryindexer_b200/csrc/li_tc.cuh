@@ -1,0 +1,378 @@
+// Stage 5 on tensor cores: native Lightning-Indexer scores over the fetched entries
+// (blog review "FlashMemory-DeepSeek-V4", sections 2.2 and 3.2):
+//     y_{b,i,j} = sum_h w'_{b,i,h} ReLU(scale_j q'_{b,i,h} . hot_K_j),   j < count[b].
+//
+// MMA orientation: the hot keys of sequence b are the A operand (M = 128 keys per tile,
+// K = d_I = 128); the queries of a group of NQ = 4 decode steps are the B operand (N = 4 x 64
+// heads = 256), so each TMEM lane (one key) holds its 256 head dot products and the weighted
+// head sums of the 4 queries run inside one thread.  Scores go to Y[tau*off_b + i*S_b + j].
+//
+// Work item = (sequence b, chunk of CH key tiles, query group g); items of one chunk are
+// consecutive so that CTAs working at the same time share the chunk's keys in L2.
+// Hot keys are bf16 (E4M3 keys were decoded exactly to bf16 by the fetch, their per-entry scale
+// is applied here in the epilogue).
+// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..9 epilogue (two warps per TMEM
+// lane quarter, two queries each).  All waits are bounded as in the index-score kernel.
+#pragma once
+#include "tc_common.cuh"
+
+namespace lsa {
+
+namespace li {
+
+constexpr int NQ = 4;              // decode queries per MMA
+constexpr int NH = 64;             // heads
+constexpr int NCOL = NQ * NH;      // MMA N = 256
+constexpr int CH = 16;             // key tiles per work item
+constexpr int MAX_STAGES = 8;
+constexpr uint32_t IDESC = tc::idesc_bf16(128, NCOL);
+
+struct Params {
+    const float *wd;         // [B][tau][64]
+    const float *hsc;        // [T] or null
+    const int32_t *count;    // [B]
+    const int64_t *offs;     // [B+1]
+    const int *item_start;   // [B+1]
+    float *Y;                // [tau*T]
+    int64_t T;
+    int B, tau, groups, stages;
+};
+
+struct Smem {
+    uint32_t kraw, qbuf, sw, bars, misc, total;
+    __host__ __device__ static Smem plan(int stages)
+    {
+        Smem s;
+        s.kraw = 0;
+        s.qbuf = s.kraw + 128 * 256 * stages;
+        s.sw = s.qbuf + 2 * NCOL * tc::DI * 2;
+        s.bars = s.sw + 8 * 2 * NH * 4;
+        s.misc = s.bars + 8 * (4 * MAX_STAGES + 4 + 4);
+        s.total = s.misc + 64 + 1024;
+        return s;
+    }
+};
+
+struct Item {
+    int b, c, g;
+};
+
+__device__ __forceinline__ Item decode_item(const int *item_start, int B, int groups, int it)
+{
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(item_start + mid) <= it) lo = mid;
+        else hi = mid;
+    }
+    const int r = it - __ldg(item_start + lo);
+    return Item{lo, r / groups, r % groups};
+}
+
+__device__ __forceinline__ int fetched_count(const Params &p, int b, int64_t &S)
+{
+    S = __ldg(p.offs + b + 1) - __ldg(p.offs + b);
+    int F = __ldg(p.count + b);
+    return F < 0 ? 0 : (F > S ? (int)S : F);
+}
+
+// work items per sequence: ceil(ceil(F/128)/CH) chunks x groups.  One block.
+__global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
+                                                   int B, int groups, int *__restrict__ item_start)
+{
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
+    if (threadIdx.x == 0) {
+        carry = 0;
+        item_start[0] = 0;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base = 0; base < B; base += blockDim.x) {
+        const int b = base + threadIdx.x;
+        int n = 0;
+        if (b < B) {
+            const int64_t S = offs[b + 1] - offs[b];
+            int F = count[b];
+            if (F < 0 || F > S) flag(ERRF_COUNT);
+            F = F < 0 ? 0 : (F > S ? (int)S : F);
+            const int tiles = (F + TILE - 1) / TILE;
+            n = ((tiles + CH - 1) / CH) * groups;
+        }
+        const int inc = warp_incl_scan(n);
+        if (lane == 31) warp_tot[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            const int v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+            warp_tot[lane] = warp_incl_scan(v) - v;
+        }
+        __syncthreads();
+        const int pos = carry + warp_tot[warp] + inc;
+        if (b < B) item_start[b + 1] = pos;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = pos;
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(320, 1)
+    k_li_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, Params p)
+{
+    using namespace tc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const Smem sp = Smem::plan(p.stages);
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t kraw = sbase + sp.kraw, qbuf = sbase + sp.qbuf;
+    float *sw = (float *)(base + sp.sw);
+    const uint32_t bars = sbase + sp.bars;
+    auto full = [&](int i) { return bars + 8u * i; };
+    auto empty = [&](int i) { return bars + 8u * (MAX_STAGES + i); };
+    auto qfull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + i); };
+    auto qempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 2 + i); };
+    auto tfull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 4 + i); };
+    auto tempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 6 + i); };
+    uint32_t *tmem_holder = (uint32_t *)(base + sp.misc);
+    volatile int *abort_flag = (volatile int *)(base + sp.misc + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = p.B;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < p.stages; i++) {
+            mbar_init(full(i), 1);
+            mbar_init(empty(i), 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(qfull(i), 1);
+            mbar_init(qempty(i), 1);
+            mbar_init(tfull(i), 1);
+            mbar_init(tempty(i), 8);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const int NI = __ldg(p.item_start + B);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&kmap) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&qmap) : "memory");
+            int stage = 0, qslot = 1;
+            uint32_t phase = 0;
+            uint32_t quse[2] = {0, 0};
+            uint32_t last_phase[MAX_STAGES];
+            bool issued[MAX_STAGES];
+            for (int i = 0; i < MAX_STAGES; i++) issued[i] = false;
+            const uint32_t kbytes = 128 * 256;
+            bool ok = true;
+            for (int it = blockIdx.x; it < NI && ok; it += gridDim.x) {
+                const Item w = decode_item(p.item_start, B, p.groups, it);
+                int64_t S;
+                const int F = fetched_count(p, w.b, S);
+                const int ntiles = (F + TILE - 1) / TILE;
+                const int t0 = w.c * CH, t1 = min(ntiles, t0 + CH);
+                qslot ^= 1;
+                if (!mbar_wait(qempty(qslot), (quse[qslot] & 1) ^ 1, abort_flag)) { ok = false; break; }
+                quse[qslot]++;
+                mbar_expect_tx(qfull(qslot), NCOL * DI * 2);
+                const uint32_t qd = qbuf + (uint32_t)qslot * NCOL * DI * 2;
+                const int qrow = (w.b * p.tau + NQ * w.g) * NH;
+                tma_load_2d(qd, &qmap, 0, qrow, qfull(qslot));
+                tma_load_2d(qd + NCOL * 128, &qmap, 64, qrow, qfull(qslot));
+                const int64_t off = __ldg(p.offs + w.b);
+                for (int kt = t0; kt < t1; kt++) {
+                    if (!mbar_wait(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_expect_tx(full(stage), kbytes);
+                    const uint32_t dst = kraw + (uint32_t)stage * kbytes;
+                    const int y = (int)(off + (int64_t)kt * TILE);
+                    tma_load_2d(dst, &kmap, 0, y, full(stage));
+                    tma_load_2d(dst + 128 * 128, &kmap, 64, y, full(stage));
+                    issued[stage] = true;
+                    last_phase[stage] = phase;
+                    if (++stage == p.stages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (*abort_flag) {
+                volatile int never = 0;
+                for (int i = 0; i < p.stages; i++)
+                    if (issued[i]) mbar_wait(full(i), last_phase[i], &never);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int stage = 0, acc = 0, qslot = 1;
+            uint32_t phase = 0, accphase = 0;
+            uint32_t quse[2] = {0, 0};
+            bool ok = true;
+            for (int it = blockIdx.x; it < NI && ok; it += gridDim.x) {
+                const Item w = decode_item(p.item_start, B, p.groups, it);
+                int64_t S;
+                const int F = fetched_count(p, w.b, S);
+                const int ntiles = (F + TILE - 1) / TILE;
+                const int t0 = w.c * CH, t1 = min(ntiles, t0 + CH);
+                qslot ^= 1;
+                if (!mbar_wait(qfull(qslot), quse[qslot] & 1, abort_flag)) { ok = false; break; }
+                quse[qslot]++;
+                const uint32_t b_base = qbuf + (uint32_t)qslot * NCOL * DI * 2;
+                for (int kt = t0; kt < t1; kt++) {
+                    if (!mbar_wait(full(stage), phase, abort_flag)) { ok = false; break; }
+                    const uint32_t a_base = kraw + (uint32_t)stage * 128 * 256;
+                    if (!mbar_wait(tempty(acc), accphase ^ 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d = tmem + (uint32_t)acc * NCOL;
+#pragma unroll
+                    for (int kk = 0; kk < DI / 16; kk++) {
+                        const uint32_t ka = a_base + (uint32_t)(kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32;
+                        const uint32_t kb = b_base + (uint32_t)(kk >> 2) * (NCOL * 128) + (uint32_t)(kk & 3) * 32;
+                        mma_bf16(d, sdesc(ka), sdesc(kb), IDESC, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(empty(stage));
+                    if (++stage == p.stages) { stage = 0; phase ^= 1; }
+                    mma_commit(tfull(acc));
+                    if (kt == t1 - 1) mma_commit(qempty(qslot));
+                    if (++acc == 2) { acc = 0; accphase ^= 1; }
+                }
+                if (ok && t1 <= t0) mma_commit(qempty(qslot));  // an item without tiles still frees its slot
+            }
+        }
+        __syncwarp();
+    } else if (warp < 10) {
+        // ------------------------------------------------------------- epilogue
+        const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+        const int half = (warp - 2) >> 2;        // queries 2*half, 2*half+1 of the group
+        float *myw = sw + (size_t)(warp - 2) * 2 * NH;
+        int acc = 0;
+        uint32_t accphase = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < NI && ok; it += gridDim.x) {
+            const Item w = decode_item(p.item_start, B, p.groups, it);
+            int64_t S;
+            const int F = fetched_count(p, w.b, S);
+            const int ntiles = (F + TILE - 1) / TILE;
+            const int t0 = w.c * CH, t1 = min(ntiles, t0 + CH);
+            const int i0 = NQ * w.g + 2 * half;  // first of this warp's two queries
+            __syncwarp();
+            for (int t = lane; t < 2 * NH; t += 32)
+                myw[t] = __ldg(p.wd + ((int64_t)w.b * p.tau + i0 + t / NH) * NH + (t % NH));
+            __syncwarp();
+            const int64_t off = __ldg(p.offs + w.b);
+            float *Yb = p.Y + (int64_t)p.tau * off;
+            for (int kt = t0; kt < t1; kt++) {
+                if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const int64_t j = (int64_t)kt * TILE + quarter * 32 + lane;
+                const bool valid = j < F;
+                float sc = 1.f;
+                if (p.hsc && valid) {
+                    sc = __ldg(p.hsc + off + j);
+                    if (!(sc >= 0.f)) flag(ERRF_SCALE);
+                }
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * NCOL + 128 * half;
+                float y[2];
+#pragma unroll
+                for (int qq = 0; qq < 2; qq++) {
+                    float v0[32], v1[32];
+                    tmem_ld32(taddr + qq * NH, v0);
+                    tmem_ld32(taddr + qq * NH + 32, v1);
+                    tmem_wait_ld();
+                    if (qq == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty(acc));
+                    }
+                    const float *wq = myw + qq * NH;
+                    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+#pragma unroll
+                    for (int h = 0; h < 32; h += 4) {
+                        const float4 wa = *(const float4 *)(wq + h);
+                        const float4 wb = *(const float4 *)(wq + 32 + h);
+                        x0 = fmaf(wa.x, fmaxf(v0[h], 0.f), x0);
+                        x1 = fmaf(wa.y, fmaxf(v0[h + 1], 0.f), x1);
+                        x2 = fmaf(wa.z, fmaxf(v0[h + 2], 0.f), x2);
+                        x3 = fmaf(wa.w, fmaxf(v0[h + 3], 0.f), x3);
+                        x0 = fmaf(wb.x, fmaxf(v1[h], 0.f), x0);
+                        x1 = fmaf(wb.y, fmaxf(v1[h + 1], 0.f), x1);
+                        x2 = fmaf(wb.z, fmaxf(v1[h + 2], 0.f), x2);
+                        x3 = fmaf(wb.w, fmaxf(v1[h + 3], 0.f), x3);
+                    }
+                    y[qq] = ((x0 + x1) + (x2 + x3)) * sc;  // ReLU(sc d) = sc ReLU(d) for sc >= 0
+                }
+                if (++acc == 2) { acc = 0; accphase ^= 1; }
+                if (valid) {
+                    Yb[(int64_t)i0 * S + j] = y[0];
+                    Yb[(int64_t)(i0 + 1) * S + j] = y[1];
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+}  // namespace li
+
+// ------------------------------------------------------------------------------------ host side
+
+inline bool li_tc_supported(int n_h, int d_I, int tau, int kdt)
+{
+    return n_h == li::NH && d_I == tc::DI && tau % li::NQ == 0 && (kdt == DT_BF16 || kdt == DT_FP8) && tc_available();
+}
+
+// hotK: bf16 [T][128] (decoded E4M3 codes when hsc is given).  item_start: device [B+1].
+// Launches the item planner and the scoring kernel; *launches counts them.
+inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK, const float *hsc,
+                               const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, float *Y,
+                               int *item_start, int sms, cudaStream_t st, int *launches)
+{
+    using namespace li;
+    *launches = 0;
+    k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / NQ, item_start);
+    (*launches)++;
+    if (T == 0) return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+    CUtensorMap kmap, qmap;
+    bool ok = make_map_2d(&kmap, hotK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, tc::DI, 64, 128);
+    ok = ok && make_map_2d(&qmap, qd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)B * tau * NH, tc::DI, 64, NCOL);
+    if (!ok) return LSA_ERR_CUDA;
+    Params p;
+    p.wd = wd;
+    p.hsc = hsc;
+    p.count = count;
+    p.offs = offs;
+    p.item_start = item_start;
+    p.Y = Y;
+    p.T = T;
+    p.B = B;
+    p.tau = tau;
+    p.groups = tau / NQ;
+    const int max_smem = 227 * 1024;
+    p.stages = MAX_STAGES;
+    while (p.stages > 2 && Smem::plan(p.stages).total > (uint32_t)max_smem) p.stages--;
+    const uint32_t smem = Smem::plan(p.stages).total;
+    if (smem > (uint32_t)max_smem) return LSA_ERR_UNSUPPORTED;
+    cudaError_t e = cudaFuncSetAttribute(k_li_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return LSA_ERR_CUDA;
+    k_li_tc<<<sms, 320, smem, st>>>(kmap, qmap, p);
+    (*launches)++;
+    e = cudaGetLastError();
+    return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
+}  // namespace lsa

@@ -11,6 +11,7 @@
 #include "project.cuh"
 #include "score_select.cuh"
 #include "score_tc.cuh"
+#include "li_tc.cuh"
 #include "topk.cuh"
 
 using namespace lsa;
@@ -160,9 +161,8 @@ lsa_status li_simt_d(int kdt, const void *qd, const float *wd, const void *hotK,
 {
     switch (kdt) {
     case DT_F32: return launch_li_simt<D, DT_F32, DT_F32>(qd, wd, hotK, hotsc, count, offs, B, T, tau, n_h, Y, st);
-    case DT_BF16:
+    default:
         return launch_li_simt<D, DT_BF16, DT_BF16>(qd, wd, hotK, hotsc, count, offs, B, T, tau, n_h, Y, st);
-    default: return launch_li_simt<D, DT_FP8, DT_BF16>(qd, wd, hotK, hotsc, count, offs, B, T, tau, n_h, Y, st);
     }
 }
 
@@ -328,6 +328,8 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
         LSA_REQUIRE(kb % 16 == 0 && aligned(K_sel, 16) && aligned(hot_K, 16),
                     "lsa_fetch_gather: key rows must be whole 16-byte chunks, 16-byte aligned");
         krow16 = (int)(kb / 16);
+        if (kdt == LSA_FP8_E4M3 && krow16 > 32)
+            return fail(LSA_ERR_UNSUPPORTED, "lsa_fetch_gather: E4M3 key rows above 512 bytes");
     }
     const int warps_per_block = 8;
     int64_t gx = ((total_S / (B > 0 ? B : 1)) + warps_per_block * GATHER_ROWS_PER_WARP - 1) /
@@ -337,18 +339,19 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
     if (gx < 1) gx = 1;
     k_gather<<<dim3((unsigned)gx, (unsigned)B), 32 * warps_per_block, 0, st>>>(
         idx, count, seq_offsets, (const uint8_t *)dpool, (int)(row_bytes / 16), (uint8_t *)hot_kv,
-        (const uint8_t *)K_sel, k_scale_sel, krow16, (uint8_t *)hot_K, hot_scale);
+        (const uint8_t *)K_sel, k_scale_sel, krow16, kdt == LSA_FP8_E4M3, (uint8_t *)hot_K, hot_scale);
     LSA_TRY(launched("gather"));
     return ok();
 }
 
 // ------------------------------------------------------------------------------ stage 5
 
+// Workspace of lsa_lightning_topk: [item_start: B+1 ints][Y: tau * total_S floats].
 size_t lsa_lightning_topk_workspace_size(int B, int tau, int64_t total_S, int k)
 {
-    (void)B; (void)k;
-    if (tau <= 0 || total_S < 0) return 0;
-    return align_up(sizeof(float) * (size_t)tau * (size_t)total_S, 256) + 256;
+    (void)k;
+    if (B <= 0 || tau <= 0 || total_S < 0) return 0;
+    return align_up(sizeof(int) * (size_t)(B + 1), 256) + align_up(sizeof(float) * (size_t)tau * (size_t)total_S, 256);
 }
 
 lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void *hot_K, const float *hot_scale,
@@ -369,12 +372,24 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     LSA_REQUIRE(aligned(workspace, 256), "lsa_lightning_topk: workspace must be 256-byte aligned");
     LSA_REQUIRE((int64_t)tau * total_S < ((int64_t)1 << 40), "lsa_lightning_topk: tau * total_S too large");
     if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: n_h must be <= 128");
-    float *Y = (float *)workspace;
-    switch (d_I) {
-    case 32: LSA_TRY(li_simt_d<32>(kdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
-    case 64: LSA_TRY(li_simt_d<64>(kdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
-    case 128: LSA_TRY(li_simt_d<128>(kdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
-    default: return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: d_I must be 32, 64 or 128");
+    int *item_start = (int *)workspace;
+    float *Y = (float *)((char *)workspace + align_up(sizeof(int) * (size_t)(B + 1), 256));
+    // E4M3 keys arrive here decoded to bf16 by lsa_fetch_gather (scales in hot_scale)
+    const int hdt = (kdt == LSA_FP8_E4M3) ? DT_BF16 : kdt;
+    if (li_tc_supported(n_h, d_I, tau, kdt)) {
+        LSA_REQUIRE(aligned(q_dec, 16) && aligned(hot_K, 16), "lsa_lightning_topk: q_dec and hot_K must be 16-byte aligned");
+        int n = 0;
+        const lsa_status s = launch_li_tc(q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, Y,
+                                          item_start, num_sms(), st, &n);
+        g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
+        if (s != LSA_OK) return fail(s, "lsa_lightning_topk: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
+    } else {
+        switch (d_I) {
+        case 32: LSA_TRY(li_simt_d<32>(hdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
+        case 64: LSA_TRY(li_simt_d<64>(hdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
+        case 128: LSA_TRY(li_simt_d<128>(hdt, q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, n_h, Y, st)); break;
+        default: return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: d_I must be 32, 64 or 128");
+        }
     }
     int kpow2 = 1;
     while (kpow2 < k) kpow2 <<= 1;

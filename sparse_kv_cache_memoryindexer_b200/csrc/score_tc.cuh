@@ -16,145 +16,16 @@
 // Every wait is bounded (about 2 s of global time): on time-out the CTA flags ERRF_TIMEOUT,
 // stops issuing work, waits (bounded) for its own copies in flight, frees TMEM and returns.
 #pragma once
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "common.cuh"
+#include "tc_common.cuh"
 
 namespace lsa {
 
 namespace tc {
 
 constexpr int NH = 64;           // heads (MMA N)
-constexpr int DI = 128;          // head dim (MMA K)
 constexpr int NACC = 8;          // TMEM accumulator slots of 64 columns (512 columns)
 constexpr int MAX_STAGES = 8;
-constexpr int MAX_L = 4;
-constexpr uint32_t IDESC = (1u << 4)          // D = fp32
-                         | (1u << 7)          // A = bf16
-                         | (1u << 10)         // B = bf16
-                         | ((NH >> 3) << 17)  // N = 64
-                         | ((128 >> 4) << 24);// M = 128
-constexpr uint64_t WAIT_NS = 2000000000ull;
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ uint64_t gtime()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t a)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(a), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-// Wait for the phase of `parity` to complete; false on abort or time-out (which sets abort).
-__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int *abort_flag)
-{
-    if (mbar_try(a, parity)) return true;
-    const uint64_t t0 = gtime();
-    while (true) {
-        if (mbar_try(a, parity)) return true;
-        if (*abort_flag) return false;
-        if (gtime() - t0 > WAIT_NS) {
-            *abort_flag = 1;
-            flag(ERRF_TIMEOUT);
-            return false;
-        }
-    }
-}
-
-// Warp-uniform wait: lane 0 polls, the whole warp receives the same answer, then every lane
-// observes the completed phase itself (one try that cannot fail: the phase cannot advance again
-// before this warp arrives on the paired barrier), which orders its later reads after it.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t a, uint32_t parity, volatile int *abort_flag)
-{
-    int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(a, parity, abort_flag) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (ok) (void)mbar_try(a, parity);
-    return ok != 0;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"((uint64_t)map), "r"(x), "r"(y), "r"(bar) : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr)
-{
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(a), "l"(b), "r"(IDESC), "r"(accumulate));
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-
-// 32 lanes x 32 columns of fp32 from TMEM into 32 registers per thread.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// E4M3 x 2 (low byte first) -> bf16 x 2, exact: e4m3 -> f16 (exact) -> f32 -> bf16 (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two)
-{
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
-    float2 f = __half22float2(__half2(h));
-    __nv_bfloat162 b = __float22bfloat162_rn(f);
-    return *reinterpret_cast<uint32_t *>(&b);
-}
+constexpr uint32_t IDESC = idesc_bf16(128, NH);
 
 struct Params {
     const float *w;          // [L][B][64]
@@ -164,7 +35,7 @@ struct Params {
     float *scores_out;       // [L][T] or null
     uint32_t *tile_mask;     // [tiles][4]
     int64_t T;
-    int B, L, stages, astages;
+    int B, L, stages, astages, qslots;
     float thr;
 };
 
@@ -181,14 +52,14 @@ struct SeqTracker {
 // Shared-memory plan (offsets from a 1024-byte aligned base).
 struct Smem {
     uint32_t kraw, abuf, qbuf, sw, bars, misc, total;
-    __host__ __device__ static Smem plan(bool fp8, int L, int stages, int astages)
+    __host__ __device__ static Smem plan(bool fp8, int L, int stages, int astages, int qslots)
     {
         Smem s;
         const uint32_t kstage = fp8 ? 128 * 128 : 128 * 256;
         s.kraw = 0;
         s.abuf = s.kraw + kstage * stages;
         s.qbuf = s.abuf + (fp8 ? 128 * 256 * astages : 0);
-        s.sw = s.qbuf + 2 * L * NH * DI * 2;
+        s.sw = s.qbuf + qslots * L * NH * DI * 2;
         s.bars = s.sw + 4 * L * NH * 4;
         s.misc = s.bars + 8 * (4 * MAX_STAGES + 4 + 2 * NACC);
         s.total = s.misc + 64 + 1024;  // + alignment slack
@@ -202,7 +73,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const Smem sp = Smem::plan(FP8, p.L, p.stages, p.astages);
+    const Smem sp = Smem::plan(FP8, p.L, p.stages, p.astages, p.qslots);
     const uint32_t sbase = smem_u32(base);
     const uint32_t kraw = sbase + sp.kraw, abuf = sbase + sp.abuf, qbuf = sbase + sp.qbuf;
     float *sw = (float *)(base + sp.sw);
@@ -266,7 +137,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
             SeqTracker tr{0};
             int stage = 0;
             uint32_t phase = 0;
-            int qslot = 1, prev_b = -1;
+            int qslot = -1, prev_b = -1;
             uint32_t quse[2] = {0, 0};
             uint32_t last_phase[MAX_STAGES];
             bool issued[MAX_STAGES];
@@ -277,7 +148,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
             for (int t = t_begin; t < t_end && ok; t++) {
                 const int b = tr.of(p.tile_start, B, t);
                 if (b != prev_b) {
-                    qslot ^= 1;
+                    qslot = (qslot + 1) % p.qslots;
                     if (!mbar_wait(qempty(qslot), (quse[qslot] & 1) ^ 1, abort_flag)) { ok = false; break; }
                     quse[qslot]++;
                     mbar_expect_tx(qfull(qslot), (uint32_t)L * NH * DI * 2);
@@ -320,13 +191,13 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
             SeqTracker tr{0};
             int stage = 0, as = 0, acc = 0;
             uint32_t phase = 0, aphase = 0, accphase = 0;
-            int qslot = 1, prev_b = -1;
+            int qslot = -1, prev_b = -1;
             uint32_t quse[2] = {0, 0};
             bool ok = true;
             for (int t = t_begin; t < t_end && ok; t++) {
                 const int b = tr.of(p.tile_start, B, t);
                 if (b != prev_b) {
-                    qslot ^= 1;
+                    qslot = (qslot + 1) % p.qslots;
                     if (!mbar_wait(qfull(qslot), quse[qslot] & 1, abort_flag)) { ok = false; break; }
                     quse[qslot]++;
                     prev_b = b;
@@ -349,7 +220,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                     for (int kk = 0; kk < DI / 16; kk++) {
                         const uint32_t ka = a_base + (uint32_t)(kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32;
                         const uint32_t kb = b_base + (uint32_t)(kk >> 2) * (NH * 128) + (uint32_t)(kk & 3) * 32;
-                        mma_bf16(d, sdesc(ka), sdesc(kb), kk > 0 ? 1u : 0u);
+                        mma_bf16(d, sdesc(ka), sdesc(kb), IDESC, kk > 0 ? 1u : 0u);
                     }
                     if (FP8) {
                         mma_commit(aempty(as));
@@ -494,40 +365,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
 
 // ------------------------------------------------------------------------------------ host side
 
-inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-    }
-    return fn;
-}
-
-inline bool tc_score_available()
-{
-    if (getenv("LSA_DISABLE_TC")) return false;
-    return tensor_map_encoder() != nullptr;
-}
-
-// 2D row-major tensor [rows][cols] of `elem`-byte elements; box [box_rows][box_cols]; 128B swizzle.
-inline bool make_map_2d(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int elem, uint64_t rows,
-                        uint64_t cols, uint32_t box_cols, uint32_t box_rows)
-{
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * (uint64_t)elem};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
+inline bool tc_score_available() { return tc_available(); }
 
 inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, const float *kscale, int kdt,
                                   const int64_t *offs, const int *tile_start, int B, int64_t T, int L,
@@ -554,17 +392,15 @@ inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, 
     p.B = B;
     p.L = L;
     p.thr = thr;
+    // Shared memory goes first to key stages (bytes in flight hide the HBM latency); one query slot
+    // (reloaded at each sequence change, a rare event for a CTA's contiguous tile range) leaves room
+    // for more stages than two.
     const int max_smem = 227 * 1024;
-    if (fp8) {
-        p.astages = 2;
-        p.stages = 4;
-        while (p.stages > 2 && Smem::plan(true, L, p.stages, p.astages).total > (uint32_t)max_smem) p.stages--;
-    } else {
-        p.astages = 0;
-        p.stages = MAX_STAGES;
-        while (p.stages > 2 && Smem::plan(false, L, p.stages, 0).total > (uint32_t)max_smem) p.stages--;
-    }
-    const uint32_t smem = Smem::plan(fp8, L, p.stages, p.astages).total;
+    p.astages = fp8 ? 2 : 0;
+    p.qslots = 1;
+    p.stages = MAX_STAGES;
+    while (p.stages > 2 && Smem::plan(fp8, L, p.stages, p.astages, p.qslots).total > (uint32_t)max_smem) p.stages--;
+    const uint32_t smem = Smem::plan(fp8, L, p.stages, p.astages, p.qslots).total;
     if (smem > (uint32_t)max_smem) return LSA_ERR_UNSUPPORTED;
     cudaError_t e;
     if (fp8) {

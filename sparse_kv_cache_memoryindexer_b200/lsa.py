@@ -168,10 +168,12 @@ def lsa_lightning_topk_workspace_size(B, tau, total_S, k) -> int:
 
 def lsa_lightning_topk(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, total_S, k, topk_idx,
                        workspace, topk_score=None, stream=None):
-    """Native Lightning-Indexer Top-k over the fetched entries (see include/lsa.h)."""
+    """Native Lightning-Indexer Top-k over the fetched entries (see include/lsa.h).  With E4M3
+    keys, hot_K is the bf16 decode written by lsa_fetch_gather and hot_scale holds the scales."""
     _dev(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, topk_score)
     B, tau, n_h, d_I = q_dec.shape
-    _check(_lib.lsa_lightning_topk(_p(q_dec), _p(w_dec), _p(hot_K), _p(hot_scale), DTYPE_CODE[hot_K.dtype],
+    kdt = LSA_FP8_E4M3 if hot_scale is not None else DTYPE_CODE[hot_K.dtype]
+    _check(_lib.lsa_lightning_topk(_p(q_dec), _p(w_dec), _p(hot_K), _p(hot_scale), kdt,
                                    _p(idx), _p(count), _p(seq_offsets), int(total_S), B, tau, n_h, d_I, int(k),
                                    _p(topk_idx), _p(topk_score), _p(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))

@@ -35,7 +35,9 @@ class IndexerPath:
         self.scores = torch.empty((L, T), dtype=torch.float32, device=dev) if with_scores else None
         self.mask = torch.empty(T, dtype=u8, device=dev) if with_mask else None
         self.hot_kv = torch.empty((T, row_bytes), dtype=u8, device=dev)
-        self.hot_K = torch.empty((T, d_I), dtype=kdtype, device=dev)
+        # E4M3 keys are decoded to bf16 by the fetch (scales kept apart)
+        hot_dt = torch.bfloat16 if kdtype == torch.float8_e4m3fn else kdtype
+        self.hot_K = torch.empty((T, d_I), dtype=hot_dt, device=dev)
         self.hot_scale = torch.empty(T, dtype=torch.float32, device=dev) if kdtype == torch.float8_e4m3fn else None
         self.topk_idx = torch.empty((B, tau, k), dtype=torch.int32, device=dev)
         self.topk_score = torch.empty((B, tau, k), dtype=torch.float32, device=dev)

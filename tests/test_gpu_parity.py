@@ -125,7 +125,7 @@ def test_gather_parity(m, name):
         sel = wl.sel_layer
         Ks = dev(inp.K[sel].contiguous())
         ss = dev(inp.k_scale[sel].contiguous()) if inp.k_scale is not None else None
-        hot_K = torch.zeros_like(Ks)
+        hot_K = torch.zeros(Ks.shape, dtype=torch.bfloat16 if ss is not None else Ks.dtype, device="cuda")
         hot_s = torch.zeros_like(ss) if ss is not None else None
         m.lsa_fetch_gather(dev(idx), dev(cnt), dev(inp.seq_offsets), T, pool.tensor, hot_kv, Ks, ss, hot_K, hot_s)
         m.lsa_check_device()
@@ -136,6 +136,8 @@ def test_gather_parity(m, name):
             used[offs[b]:offs[b] + cnt[b]] = True
         used = torch.from_numpy(used)
         assert torch.equal(hot_kv.cpu()[used], r_kv[used])
+        if ss is not None:  # E4M3 codes arrive decoded to bf16 (exact)
+            r_K = r_K.float().to(torch.bfloat16)
         assert torch.equal(hot_K.cpu()[used].view(torch.uint8), r_K[used].view(torch.uint8))
         if ss is not None:
             assert torch.equal(hot_s.cpu()[used], r_s[used])
@@ -154,6 +156,8 @@ def run_topk(m, inp, idx, cnt, k, pool_needed=False):
     # the hot keys come from the oracle's gather (a byte copy), so this checks stage 5 alone
     _, hK, hs = oracle.gather(idx, cnt, inp.seq_offsets.numpy(), None, inp.K[sel], inp.k_scale[sel] if ss is not None else None,
                               wl.d_I)
+    if hs is not None:  # the decode-step kernel takes E4M3 hot keys decoded to bf16 (exact)
+        hK = hK.float().to(torch.bfloat16)
     ti = torch.empty((wl.B, wl.tau, k), dtype=torch.int32, device="cuda")
     ts = torch.empty((wl.B, wl.tau, k), dtype=torch.float32, device="cuda")
     ws = torch.empty(m.lsa_lightning_topk_workspace_size(wl.B, wl.tau, T, k), dtype=torch.uint8, device="cuda")
