@@ -74,25 +74,43 @@ int num_sms()
     return cached_sms;
 }
 
-// Workspace layout of lsa_memindex_score_select.
+// Workspace layout of lsa_memindex_score_select:
+//   tile_start [B+1] int | tile_mask [max_tiles][4] u32 | qh [L*B*64][128] f16 | wh [L*B*64] fp32
+// (qh / wh: the f16 queries and scaled head weights of the E4M3 tensor-core path).
 struct ScoreWs {
-    int *tile_start;     // [B+1]
-    uint32_t *tile_mask; // [max_tiles][4]
+    int *tile_start;
+    uint32_t *tile_mask;
+    void *qh;
+    float *wh;
 };
 
 int64_t max_tiles(int B, int64_t T) { return T / TILE + B + 1; }
 
-size_t score_ws_bytes(int B, int64_t T)
+size_t score_ws_parts(int L, int B, int64_t T, size_t part[4])
 {
-    return align_up(sizeof(int) * (size_t)(B + 1), 256) + align_up((size_t)max_tiles(B, T) * 16, 256);
+    part[0] = align_up(sizeof(int) * (size_t)(B + 1), 256);
+    part[1] = align_up((size_t)max_tiles(B, T) * 16, 256);
+    part[2] = align_up((size_t)L * B * 64 * 128 * 2, 256);
+    part[3] = align_up((size_t)L * B * 64 * 4, 256);
+    return part[0] + part[1] + part[2] + part[3];
 }
 
-ScoreWs score_ws(void *ws, int B)
+size_t score_ws_bytes(int L, int B, int64_t T)
 {
+    size_t part[4];
+    return score_ws_parts(L, B, T, part);
+}
+
+ScoreWs score_ws(void *ws, int L, int B, int64_t T)
+{
+    size_t part[4];
+    score_ws_parts(L, B, T, part);
     char *p = (char *)ws;
     ScoreWs w;
     w.tile_start = (int *)p;
-    w.tile_mask = (uint32_t *)(p + align_up(sizeof(int) * (size_t)(B + 1), 256));
+    w.tile_mask = (uint32_t *)(p + part[0]);
+    w.qh = (void *)(p + part[0] + part[1]);
+    w.wh = (float *)(p + part[0] + part[1] + part[2]);
     return w;
 }
 
@@ -244,9 +262,8 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
 
 size_t lsa_score_select_workspace_size(int L, int B, int64_t total_S)
 {
-    (void)L;
-    if (B <= 0 || total_S < 0) return 0;
-    return score_ws_bytes(B, total_S);
+    if (L <= 0 || B <= 0 || total_S < 0) return 0;
+    return score_ws_bytes(L, B, total_S);
 }
 
 lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *K, const float *k_scale,
@@ -264,22 +281,26 @@ lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *
     LSA_REQUIRE((kdt == LSA_FP8_E4M3) == (k_scale != nullptr),
                 "lsa_memindex_score_select: k_scale is required for FP8 keys and must be NULL otherwise");
     LSA_REQUIRE(threshold > 0.f && threshold < 1.f, "lsa_memindex_score_select: threshold must be in (0, 1)");
-    const size_t need = score_ws_bytes(B, total_S);
+    const size_t need = score_ws_bytes(L, B, total_S);
     if (!workspace || workspace_bytes < need)
         return fail(LSA_ERR_WORKSPACE, "lsa_memindex_score_select: workspace needs %zu bytes", need);
     LSA_REQUIRE(aligned(workspace, 256), "lsa_memindex_score_select: workspace must be 256-byte aligned");
     const float thr_logit = (float)log((double)threshold / (1.0 - (double)threshold));
-    ScoreWs ws = score_ws(workspace, B);
+    ScoreWs ws = score_ws(workspace, L, B, total_S);
 
     k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, ws.tile_start);
     LSA_TRY(launched("tile setup"));
 
-    const bool tc = (n_h == 64 && d_I == 128 && (kdt == LSA_BF16 || kdt == LSA_FP8_E4M3) && tc_score_available());
+    const bool tc = (n_h == 64 && d_I == 128 && L <= tc::MAX_L_TC && (kdt == LSA_BF16 || kdt == LSA_FP8_E4M3) &&
+                     tc_score_available());
     if (tc) {
         LSA_REQUIRE(aligned(q, 16) && aligned(K, 16), "lsa_memindex_score_select: q and K must be 16-byte aligned");
-        LSA_TRY(launch_score_tc(q, w, K, k_scale, kdt, seq_offsets, ws.tile_start, B, total_S, L, thr_logit,
-                                scores_out, ws.tile_mask, num_sms(), st));
-        g_launches.fetch_add(1, std::memory_order_relaxed);
+        int n = 0;
+        const lsa_status s = launch_score_tc(q, w, K, k_scale, kdt, seq_offsets, ws.tile_start, B, total_S, L,
+                                             thr_logit, scores_out, ws.tile_mask, ws.qh, ws.wh, num_sms(), st, &n);
+        g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
+        if (s != LSA_OK) return fail(s, "lsa_memindex_score_select: tensor-core launch failed (%s)",
+                                     cudaGetErrorString(cudaGetLastError()));
     } else {
         if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_memindex_score_select: n_h must be <= 128");
         switch (d_I) {

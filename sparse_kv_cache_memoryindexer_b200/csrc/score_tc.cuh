@@ -12,7 +12,16 @@
 //   warp 0        TMA producer: key tiles (one per (tile, layer)) and the queries of each sequence
 //   warp 1        TMEM allocator + MMA issuer (one elected thread)
 //   warps 2..5    epilogue: tcgen05.ld of the accumulator, score, threshold, OR, ballot
-//   warps 6..9    (E4M3 keys only) converters: E4M3 tile -> bf16 A tile in shared memory (exact)
+//   warps 6..13   (E4M3 keys only) converters: E4M3 tile (shared memory) -> f16 A tile written
+//                 straight into tensor memory (tcgen05.st), so the MMA reads A from TMEM and only
+//                 the queries from shared memory.  Two warps per TMEM lane quarter, each converting
+//                 half of every row, so that two independent chains share each sub-partition.
+// E4M3 keys run the MMA in f16: a bit-level decode gives each code's value times 2^-8 exactly
+// (e4m3x4_to_f16_scaled, K positions permuted (0,2,1,3) within groups of four); k_q_to_f16
+// converts the queries to f16 with the same permutation and a per-head power-of-two scale 2^e_h
+// (largest element in [2^14, 2^15)), and multiplies w_h by 2^(8 - e_h), so that
+// w_h ReLU(q_h . K) is unchanged.  Exact except for query elements more than 2^28 times smaller
+// than their head's largest, whose products lie below the fp32 rounding of the dot product.
 // Every wait is bounded (about 2 s of global time): on time-out the CTA flags ERRF_TIMEOUT,
 // stops issuing work, waits (bounded) for its own copies in flight, frees TMEM and returns.
 #pragma once
@@ -23,9 +32,45 @@ namespace lsa {
 namespace tc {
 
 constexpr int NH = 64;           // heads (MMA N)
-constexpr int NACC = 8;          // TMEM accumulator slots of 64 columns (512 columns)
+constexpr int NACC = 8;          // TMEM accumulator slots of 64 columns (bf16 keys: all 512 columns)
+constexpr int NACC_FP8 = 4;      // E4M3 keys: 4 accumulator slots (columns 0..255) ...
+constexpr int ASLOTS = 4;        // ... and 4 A-operand slots of 64 columns (columns 256..511)
 constexpr int MAX_STAGES = 8;
+constexpr int MAX_L_TC = 3;      // indexer layers handled by one launch
 constexpr uint32_t IDESC = idesc_bf16(128, NH);
+constexpr uint32_t IDESC_F16 = idesc_f16(128, NH);
+
+// Queries to f16 with a per-head power-of-two scale and the (0,2,1,3) permutation of each group of
+// four K positions (see the header comment); one warp per head, four consecutive elements per lane.
+// q [R][128] bf16, w [R] fp32 -> qh [R][128] f16, wh [R] fp32, R = L * B * 64.
+__global__ void __launch_bounds__(256) k_q_to_f16(const __nv_bfloat16 *__restrict__ q, const float *__restrict__ w,
+                                                  __half *__restrict__ qh, float *__restrict__ wh, int R)
+{
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= R) return;
+    float v[4];
+    float mx = 0.f;
+    const int perm[4] = {0, 2, 1, 3};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        v[k] = __bfloat162float(q[(int64_t)row * DI + 4 * lane + perm[k]]);
+        mx = fmaxf(mx, fabsf(v[k]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    int e = 0;
+    if (mx > 0.f) {
+        const int E = (int)((__float_as_uint(mx) >> 23) & 0xff) - 127;  // bf16 values are fp32-normal
+        e = 14 - E;
+        e = e < -100 ? -100 : (e > 100 ? 100 : e);
+    }
+    const float up = __uint_as_float((uint32_t)(127 + e) << 23);        // 2^e, exact
+    const float down = __uint_as_float((uint32_t)(127 + 8 - e) << 23);  // 2^(8-e): the keys carry 2^-8
+#pragma unroll
+    for (int k = 0; k < 4; k++) qh[(int64_t)row * DI + 4 * lane + k] = __float2half_rn(v[k] * up);
+    if (lane == 0) wh[row] = w[row] * down;
+}
 
 struct Params {
     const float *w;          // [L][B][64]
@@ -57,8 +102,8 @@ struct Smem {
         Smem s;
         const uint32_t kstage = fp8 ? 128 * 128 : 128 * 256;
         s.kraw = 0;
-        s.abuf = s.kraw + kstage * stages;
-        s.qbuf = s.abuf + (fp8 ? 128 * 256 * astages : 0);
+        s.abuf = s.kraw + kstage * stages;  // (unused: the E4M3 A operand lives in TMEM)
+        s.qbuf = s.abuf;
         s.sw = s.qbuf + qslots * L * NH * DI * 2;
         s.bars = s.sw + 4 * L * NH * 4;
         s.misc = s.bars + 8 * (4 * MAX_STAGES + 4 + 2 * NACC);
@@ -67,8 +112,10 @@ struct Smem {
     }
 };
 
+constexpr int CONV_WARPS = 8;
+
 template <bool FP8>
-__global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
+__global__ void __launch_bounds__(FP8 ? 192 + 32 * CONV_WARPS : 192, 1)
     k_score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, Params p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -93,21 +140,22 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int L = p.L, B = p.B;
     const int64_t T = p.T;
+    constexpr int nacc = FP8 ? NACC_FP8 : NACC;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; i++) {
             mbar_init(full(i), 1);
-            mbar_init(empty(i), FP8 ? 4 : 1);
+            mbar_init(empty(i), FP8 ? CONV_WARPS : 1);
         }
         for (int i = 0; i < p.astages; i++) {
-            mbar_init(afull(i), 4);
+            mbar_init(afull(i), CONV_WARPS);
             mbar_init(aempty(i), 1);
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(qfull(i), 1);
             mbar_init(qempty(i), 1);
         }
-        for (int i = 0; i < NACC; i++) {
+        for (int i = 0; i < nacc; i++) {
             mbar_init(tfull(i), 1);
             mbar_init(tempty(i), 4);
         }
@@ -207,7 +255,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                     uint32_t a_base;
                     if (FP8) {
                         if (!mbar_wait(afull(as), aphase, abort_flag)) { ok = false; break; }
-                        a_base = abuf + (uint32_t)as * 128 * 256;
+                        a_base = tmem + (uint32_t)(NACC_FP8 * NH + as * 64);  // TMEM columns of A slot `as`
                     } else {
                         if (!mbar_wait(full(stage), phase, abort_flag)) { ok = false; break; }
                         a_base = kraw + (uint32_t)stage * 128 * 256;
@@ -218,9 +266,13 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                     const uint32_t d = tmem + (uint32_t)acc * NH;
 #pragma unroll
                     for (int kk = 0; kk < DI / 16; kk++) {
-                        const uint32_t ka = a_base + (uint32_t)(kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32;
                         const uint32_t kb = b_base + (uint32_t)(kk >> 2) * (NH * 128) + (uint32_t)(kk & 3) * 32;
-                        mma_bf16(d, sdesc(ka), sdesc(kb), IDESC, kk > 0 ? 1u : 0u);
+                        if (FP8) {
+                            mma_f16_tmem_a(d, a_base + (uint32_t)kk * 8, sdesc(kb), IDESC_F16, kk > 0 ? 1u : 0u);
+                        } else {
+                            const uint32_t ka = a_base + (uint32_t)(kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32;
+                            mma_bf16(d, sdesc(ka), sdesc(kb), IDESC, kk > 0 ? 1u : 0u);
+                        }
                     }
                     if (FP8) {
                         mma_commit(aempty(as));
@@ -231,7 +283,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                     }
                     mma_commit(tfull(acc));
                     if (l == L - 1 && last_of_seq) mma_commit(qempty(qslot));
-                    if (++acc == NACC) { acc = 0; accphase ^= 1; }
+                    if (++acc == nacc) { acc = 0; accphase ^= 1; }
                 }
             }
         }
@@ -240,11 +292,23 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
         // ------------------------------------------------------------- epilogue
         const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
         float *myw = sw + (size_t)quarter * L * NH;
-        SeqTracker tr{0};
+        SeqTracker tr{0}, trn{0};
         int acc = 0;
         uint32_t accphase = 0;
         int prev_b = -1;
         bool ok = true;
+        // E4M3 scales are per entry and layer: load them one tile ahead so that the global-load
+        // latency overlaps the previous tile instead of stalling every layer-tile.
+        float sc_cur[MAX_L_TC] = {1.f, 1.f, 1.f}, sc_nxt[MAX_L_TC] = {1.f, 1.f, 1.f};
+        auto load_scales = [&](int tt, float (&out)[MAX_L_TC]) {
+            const int bb = trn.of(p.tile_start, B, tt);
+            const int64_t SS = __ldg(p.offs + bb + 1) - __ldg(p.offs + bb);
+            const int64_t ss = (int64_t)(tt - __ldg(p.tile_start + bb)) * TILE + quarter * 32 + lane;
+            const int64_t rr = __ldg(p.offs + bb) + ss;
+#pragma unroll
+            for (int l = 0; l < MAX_L_TC; l++) out[l] = (l < L && ss < SS) ? __ldg(p.kscale + (int64_t)l * T + rr) : 1.f;
+        };
+        if (FP8 && t_begin < t_end) load_scales(t_begin, sc_nxt);
         for (int t = t_begin; t < t_end && ok; t++) {
             const int b = tr.of(p.tile_start, B, t);
             if (b != prev_b) {
@@ -256,12 +320,19 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                 __syncwarp();
                 prev_b = b;
             }
+            if (FP8) {
+#pragma unroll
+                for (int l = 0; l < MAX_L_TC; l++) sc_cur[l] = sc_nxt[l];
+                if (t + 1 < t_end) load_scales(t + 1, sc_nxt);
+            }
             const int64_t S = __ldg(p.offs + b + 1) - __ldg(p.offs + b);
             const int64_t s = (int64_t)(t - __ldg(p.tile_start + b)) * TILE + quarter * 32 + lane;
             const bool valid = s < S;
             const int64_t row = __ldg(p.offs + b) + s;
             bool fetched = false;
-            for (int l = 0; l < L; l++) {
+#pragma unroll
+            for (int l = 0; l < MAX_L_TC; l++) {
+                if (l >= L) break;
                 if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * NH;
@@ -272,7 +343,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tempty(acc));
-                if (++acc == NACC) { acc = 0; accphase ^= 1; }
+                if (++acc == nacc) { acc = 0; accphase ^= 1; }
                 const float *wl = myw + l * NH;
                 float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
 #pragma unroll
@@ -291,7 +362,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                 float x = (x0 + x1) + (x2 + x3);
                 if (valid) {
                     if (FP8) {
-                        const float sc = __ldg(p.kscale + (int64_t)l * T + row);
+                        const float sc = sc_cur[l];
                         if (!(sc >= 0.f)) flag(ERRF_SCALE);
                         x *= sc;  // ReLU(sc * d) = sc * ReLU(d) for sc >= 0
                     }
@@ -304,9 +375,10 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
             if (lane == 0) p.tile_mask[(int64_t)t * 4 + quarter] = m;
         }
     } else if (FP8) {
-        // ------------------------------------------------------------- E4M3 -> bf16 converters
-        const int r = threadIdx.x - 6 * 32;  // tile row 0..127 handled by this thread
-        SeqTracker tr{0};
+        // ------------------------------------------------------------- E4M3 -> f16 converters
+        const int quarter = warp & 3;            // this warp may only touch TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;       // tile row (entry) converted by this thread
+        const int half = (warp - 6) >> 2;        // which 64 of the row's 128 codes (16-byte units 4h .. 4h+3)
         int stage = 0, as = 0;
         uint32_t phase = 0, aphase = 0;
         bool ok = true;
@@ -314,33 +386,29 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
             for (int l = 0; l < L; l++) {
                 if (!mbar_wait_warp(full(stage), phase, abort_flag)) { ok = false; break; }
                 if (!mbar_wait_warp(aempty(as), aphase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
                 const uint32_t src = kraw + (uint32_t)stage * 128 * 128 + (uint32_t)r * 128;
-                const uint32_t dst = abuf + (uint32_t)as * 128 * 256 + (uint32_t)r * 128;
+                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) +
+                                    (uint32_t)(NACC_FP8 * NH + as * 64 + 32 * half);
+                uint4 v[4];
 #pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    uint4 v;
+                for (int uu = 0; uu < 4; uu++) {
+                    const int u = 4 * half + uu;  // 16-byte unit of the row (codes 16u .. 16u+15)
                     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "=r"(v[uu].x), "=r"(v[uu].y), "=r"(v[uu].z), "=r"(v[uu].w)
                                  : "r"(src + (uint32_t)((u ^ (r & 7)) * 16)));
-                    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-                    uint32_t o[8];
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        o[2 * k] = e4m3x2_to_bf16x2((uint16_t)(in[k] & 0xffffu));
-                        o[2 * k + 1] = e4m3x2_to_bf16x2((uint16_t)(in[k] >> 16));
-                    }
-                    // bf16 16-byte units 2u and 2u+1 of this row (chunk of 64 elements each)
-#pragma unroll
-                    for (int hv = 0; hv < 2; hv++) {
-                        const int vv = 2 * u + hv;
-                        const uint32_t da = dst + (uint32_t)(vv >> 3) * (128 * 128) +
-                                            (uint32_t)(((vv & 7) ^ (r & 7)) * 16);
-                        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(da), "r"(o[4 * hv]),
-                                     "r"(o[4 * hv + 1]), "r"(o[4 * hv + 2]), "r"(o[4 * hv + 3])
-                                     : "memory");
-                    }
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                uint32_t o[32];
+#pragma unroll
+                for (int uu = 0; uu < 4; uu++) {
+                    e4m3x4_to_f16_scaled(v[uu].x, o[8 * uu + 0], o[8 * uu + 1]);
+                    e4m3x4_to_f16_scaled(v[uu].y, o[8 * uu + 2], o[8 * uu + 3]);
+                    e4m3x4_to_f16_scaled(v[uu].z, o[8 * uu + 4], o[8 * uu + 5]);
+                    e4m3x4_to_f16_scaled(v[uu].w, o[8 * uu + 6], o[8 * uu + 7]);
+                }
+                tmem_st32(ta, o);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(empty(stage));
@@ -350,7 +418,6 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                 if (++as == p.astages) { as = 0; aphase ^= 1; }
             }
         }
-        (void)tr;
     }
 
     tc_fence_before();
@@ -367,19 +434,31 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
 
 inline bool tc_score_available() { return tc_available(); }
 
+// qh_ws / wh_ws: workspace for the f16 queries and scaled head weights of the E4M3 path
+// ([L*B*64][128] f16 and [L*B*64] fp32).  *launches counts the kernels started.
 inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, const float *kscale, int kdt,
                                   const int64_t *offs, const int *tile_start, int B, int64_t T, int L,
-                                  float thr, float *scores_out, uint32_t *tile_mask, int sms, cudaStream_t st)
+                                  float thr, float *scores_out, uint32_t *tile_mask, void *qh_ws, float *wh_ws,
+                                  int sms, cudaStream_t st, int *launches)
 {
     using namespace tc;
-    if (L < 1 || L > 3) return LSA_ERR_UNSUPPORTED;
+    *launches = 0;
+    if (L < 1 || L > MAX_L_TC) return LSA_ERR_UNSUPPORTED;
     const bool fp8 = (kdt == DT_FP8);
+    if (fp8) {
+        const int R = L * B * NH;
+        k_q_to_f16<<<(R + 7) / 8, 256, 0, st>>>((const __nv_bfloat16 *)q, w, (__half *)qh_ws, wh_ws, R);
+        (*launches)++;
+        q = qh_ws;
+        w = wh_ws;
+    }
     CUtensorMap kmap, qmap;
     const uint64_t rows = (uint64_t)L * (uint64_t)T;
     if (rows == 0) return LSA_OK;
     bool ok = fp8 ? make_map_2d(&kmap, K, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, DI, 128, 128)
                   : make_map_2d(&kmap, K, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, DI, 64, 128);
-    ok = ok && make_map_2d(&qmap, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * B * NH, DI, 64, NH);
+    ok = ok && make_map_2d(&qmap, q, fp8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                           (uint64_t)L * B * NH, DI, 64, NH);
     if (!ok) return LSA_ERR_CUDA;
     Params p;
     p.w = w;
@@ -396,7 +475,7 @@ inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, 
     // (reloaded at each sequence change, a rare event for a CTA's contiguous tile range) leaves room
     // for more stages than two.
     const int max_smem = 227 * 1024;
-    p.astages = fp8 ? 2 : 0;
+    p.astages = fp8 ? ASLOTS : 0;
     p.qslots = 1;
     p.stages = MAX_STAGES;
     while (p.stages > 2 && Smem::plan(fp8, L, p.stages, p.astages, p.qslots).total > (uint32_t)max_smem) p.stages--;
@@ -406,11 +485,13 @@ inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, 
     if (fp8) {
         e = cudaFuncSetAttribute(k_score_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return LSA_ERR_CUDA;
-        k_score_tc<true><<<sms, 320, smem, st>>>(kmap, qmap, p);
+        k_score_tc<true><<<sms, 192 + 32 * CONV_WARPS, smem, st>>>(kmap, qmap, p);
+        (*launches)++;
     } else {
         e = cudaFuncSetAttribute(k_score_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return LSA_ERR_CUDA;
         k_score_tc<false><<<sms, 192, smem, st>>>(kmap, qmap, p);
+        (*launches)++;
     }
     e = cudaGetLastError();
     return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;

@@ -327,3 +327,43 @@ def test_unmapped_pool_is_rejected(m):
     hot = torch.zeros((T, wl.row_bytes), dtype=torch.uint8, device="cuda")
     with pytest.raises(m.LSAError, match="LSA_ERR_INVALID_ARG"):
         m.lsa_fetch_gather(dev(idx), dev(cnt), dev(inp.seq_offsets), T, inp.pool, hot)
+
+
+# ------------------------------------------------------------------ E4M3 code coverage
+
+def _fp8_case(codes_fn, seed):
+    wl = synth.workload("ctx1m_fp8_b32", B=2, S=(3000, 1291), fetch=(0.2, 0.2))
+    inp = synth.make_inputs(wl, parts=("score",))
+    rng = np.random.default_rng(seed)
+    codes = codes_fn(rng, inp.K.shape)
+    inp.K = torch.from_numpy(codes).view(torch.float8_e4m3fn)
+    return wl, inp
+
+
+def test_select_e4m3_subnormal_codes(m):
+    """Only subnormal E4M3 codes (exponent field 0) with scale 2^9, so every key value is a small
+    integer: a flush of subnormals anywhere on the device path would zero every logit."""
+    def codes(rng, shape):
+        mag = rng.integers(0, 8, size=shape).astype(np.uint8)          # 0x00..0x07
+        sign = (rng.random(shape) < 0.5).astype(np.uint8) << 7
+        return mag | sign
+    wl, inp = _fp8_case(codes, 21)
+    inp.k_scale = torch.full_like(inp.k_scale, 512.0)
+    offs = inp.seq_offsets.numpy()
+    ref = oracle.score(inp.q, inp.w, inp.K, inp.k_scale, offs)
+    assert np.abs(ref["x"]).max() > 1.0
+    mask, idx, cnt, I = run_select(m, inp)
+    check_select(mask, idx, cnt, I, ref, offs, what="subnormal codes")
+
+
+def test_select_e4m3_all_codes(m):
+    """Every finite E4M3 code (0x7F and 0xFF are NaN and excluded), uniformly, with random scales."""
+    def codes(rng, shape):
+        c = rng.integers(0, 254, size=shape).astype(np.uint8)          # 0..253
+        return np.where(c >= 0x7F, c + 1, c).astype(np.uint8)           # skip 0x7F; 0xFF never drawn
+    wl, inp = _fp8_case(codes, 22)
+    inp.k_scale = torch.from_numpy(np.random.default_rng(5).uniform(1e-3, 3e-3, inp.k_scale.shape).astype(np.float32))
+    offs = inp.seq_offsets.numpy()
+    ref = oracle.score(inp.q, inp.w, inp.K, inp.k_scale, offs)
+    mask, idx, cnt, I = run_select(m, inp)
+    check_select(mask, idx, cnt, I, ref, offs, what="all codes")
