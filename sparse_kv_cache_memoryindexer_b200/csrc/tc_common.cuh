@@ -72,6 +72,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile 
     }
 }
 
+// One lane of a converged warp (elect.sync): true on exactly one lane.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Warp-uniform wait: lane 0 polls, the whole warp receives the same answer, then every lane
 // observes the completed phase itself (one try that cannot fail: the phase cannot advance again
 // before this warp arrives on the paired barrier), which orders its later reads after it.
@@ -108,17 +120,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b
         ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
-// The same with the A operand in tensor memory (M lanes x K/2 columns of packed 16-bit pairs).
-__device__ __forceinline__ void mma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
-                                               uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate));
-}
-
 __device__ __forceinline__ void mma_commit(uint32_t bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -145,50 +146,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// 32 registers per thread into 32 consecutive columns of the thread's TMEM lane.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Four E4M3 codes (one 32-bit word, element 4j+t in byte t) -> two f16x2 words holding the codes'
-// values times 2^-8, exactly, for every code (subnormals included): the f16 pattern with the sign
-// at bit 15 and the code's 7 exponent/mantissa bits at bits 13..7 is that value (E4M3 exponent
-// field e becomes the f16 exponent field e, bias 15 instead of 7, and E4M3 subnormals become f16
-// subnormals).  Output order: even = (element 4j, 4j+2), odd = (4j+1, 4j+3), low half first,
-// i.e. the K positions 4j..4j+3 hold elements (0, 2, 1, 3) of the group; the queries are
-// permuted the same way.  NaN codes are not supported.
-__device__ __forceinline__ void e4m3x4_to_f16_scaled(uint32_t x, uint32_t &even, uint32_t &odd)
-{
-    even = ((x << 7) & 0x3F803F80u) | ((x << 8) & 0x80008000u);
-    odd = ((x >> 1) & 0x3F803F80u) | (x & 0x80008000u);
-}
-
-// E4M3 x 2 (low byte first) -> f16 x 2, exact (one conversion instruction).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two)
-{
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
-// E4M3 x 2 (low byte first) -> bf16 x 2, exact: e4m3 -> f16 (exact) -> f32 -> bf16 (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two)
-{
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
-    float2 f = __half22float2(__half2(h));
-    __nv_bfloat162 b = __float22bfloat162_rn(f);
-    return *reinterpret_cast<uint32_t *>(&b);
-}
 
 }  // namespace tc
 
