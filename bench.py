@@ -59,6 +59,33 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one k_score_tc launch, from one ncu
+# capture of a smaller batch of the same workload, per entry and layer: the kernel streams every key
+# row once, so the traffic grows in proportion to the entries.  Reported only while the kernel sources
+# hash to the value the capture was taken on (null otherwise).
+SCORE_TRAFFIC = {
+    "fp8": {"bytes_per_entry_layer": 133.49, "capture": "ctx1m_fp8_b32 with B=4 (1,048,576 entries x 3 layers)"},
+    "bf16": {"bytes_per_entry_layer": 260.99, "capture": "ctx500k_bf16_b8 with B=2 (262,144 entries x 3 layers)"},
+}
+SCORE_TRAFFIC_SRC = "604780a52da2a2e8"
+
+
+def score_kernel_src_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("score_tc.cuh", "tc_common.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "sparse_kv_cache_memoryindexer_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def score_traffic(wl):
+    tr = SCORE_TRAFFIC.get(wl.kdtype)
+    if tr is None or score_kernel_src_hash() != SCORE_TRAFFIC_SRC:
+        return None, None
+    return tr["bytes_per_entry_layer"] * wl.L * wl.total_S, tr["capture"]
+
+
 # ------------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -298,6 +325,7 @@ def run_lsa(args, rank, world, device):
         value = world * wl.L * T * args.steps / (elapsed_ms * 1e-3)
         sel_ms = stage_ms[1]
         score_gbs = alg["score_bytes"] / (sel_ms * 1e-3) / 1e9
+        traffic, traffic_src = score_traffic(wl)
         rooflines = {
             "project": {"bound": "hbm", "achieved": alg["proj_bytes"] / (stage_ms[0] * 1e-3) / 1e9,
                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "ms": stage_ms[0]},
@@ -307,7 +335,8 @@ def run_lsa(args, rank, world, device):
                              "peak": h2d, "unit": "GB/s", "ms": stage_ms[2],
                              "peak_note": "pinned host->device cudaMemcpy measured in this run"},
             "lightning_topk": {"bound": "tensor", "achieved": alg["topk_flops"] / (stage_ms[3] * 1e-3) / 1e12,
-                               "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "ms": stage_ms[3]},
+                               "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s", "ms": stage_ms[3],
+                               "peak_note": "sustained bf16 GEMM (timed inside the step)"},
         }
         for r in rooflines.values():
             r["frac"] = r["achieved"] / r["peak"]
@@ -328,7 +357,9 @@ def run_lsa(args, rank, world, device):
             "score_select_entries_per_s": world * wl.L * T / (sel_ms * 1e-3),
             "roofline": dict(kernel="score_select (index score + threshold + OR + compaction, one stream)",
                              bound="hbm", achieved=score_gbs, peak=peaks["hbm_gbs"], unit="GB/s",
-                             frac=score_gbs / peaks["hbm_gbs"], traffic=None,
+                             frac=score_gbs / peaks["hbm_gbs"], traffic=traffic,
+                             traffic_note=None if traffic is None else
+                             "ncu DRAM bytes of k_score_tc on %s, scaled by entries" % traffic_src,
                              bytes_per_launch=alg["score_bytes"], peak_source=peaks["source"]),
             "rooflines": rooflines,
             "gpu_launches": launches,
