@@ -120,6 +120,36 @@ lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *
                                      void *workspace, size_t workspace_bytes, lsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Stages 2-4a without a workspace.  The method has no counterpart of this entry point: it is
+ * a convenience for callers that cannot allocate device memory at the point where they select,
+ * for instance a host that runs with a fixed device-memory budget reserved at start-up, or one
+ * whose allocator must not be entered on the decode path, and so cannot supply a workspace.
+ *
+ * Same arguments, outputs and errors as lsa_memindex_score_select, without workspace and
+ * workspace_bytes: the scratch is an array of LSA_STATIC_SCORE_SCRATCH_BYTES bytes of device
+ * memory owned by the library (one per device, reserved when the library's device code is
+ * loaded).  The call allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - Limit: sizes whose lsa_score_select_workspace_size(L, B, total_S) exceeds
+ *     LSA_STATIC_SCORE_SCRATCH_BYTES are rejected with LSA_ERR_WORKSPACE and a message naming
+ *     both sizes (8 MiB holds, e.g., L = 3, B = 64 and 16 M entries); nothing is launched.
+ *   - Nothing needs to start at zero: every scratch byte a call reads, it writes first.
+ *   - The first call on each device does a one-time setup with that device current (it looks
+ *     up the scratch's device address); make that first call before any stream capture starts.
+ *   - One scratch per device: calls that may overlap on one device (different streams, or
+ *     different host threads, without an ordering between them) race on it and give wrong
+ *     results.  Order them, e.g. issue them on one stream.
+ * ---------------------------------------------------------------------------------------- */
+#define LSA_STATIC_SCORE_SCRATCH_BYTES (8u << 20)
+
+lsa_status lsa_memindex_score_select_static(const void *q, const float *w, const void *K,
+                                            const float *k_scale, lsa_dtype kdt,
+                                            const int64_t *seq_offsets, int64_t total_S,
+                                            int L, int B, int n_h, int d_I, float threshold,
+                                            float *scores_out, uint8_t *mask_out,
+                                            int32_t *idx_out, int32_t *count_out,
+                                            lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Stage 4b -- fetch C^MemComp from the CPU cold pool into the GPU hot buffer (hyper.ai
  * summary "Method"; blog review section 3):
  *     hot_kv[off_b + j] = pool[off_b + idx[off_b + j]]      for j < count[b]

@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/lsa.h"
 #include "common.cuh"
@@ -442,6 +443,71 @@ lsa_status lsa_pool_free(void *ptr)
     cudaError_t e = cudaFreeHost(ptr);
     if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "cudaFreeHost: %s", cudaGetErrorString(e));
     return ok();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ score/select without a workspace
+// lsa_memindex_score_select_static: the same computation as lsa_memindex_score_select, with its
+// scratch in a fixed array of device memory that the library owns (declared below, reserved when
+// the library's device code is loaded), so that a call performs no allocation of any kind.
+
+namespace {
+
+// The scratch of the allocation-free entry point: one copy per device.  Nothing in it needs to
+// hold any value before a call: every byte the call reads is written earlier in the same call.
+static __device__ __align__(256) unsigned char g_score_scratch[LSA_STATIC_SCORE_SCRATCH_BYTES];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxScratchDevices];  // device address of g_score_scratch, per device
+
+// The device address of the scratch on the current device, looked up once per device.
+lsa_status static_scratch(void **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail(LSA_ERR_CUDA, "lsa_memindex_score_select_static: cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxScratchDevices)
+        return fail(LSA_ERR_UNSUPPORTED, "lsa_memindex_score_select_static: device %d beyond the %d supported", dev,
+                    kMaxScratchDevices);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_score_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(LSA_ERR_CUDA, "lsa_memindex_score_select_static: cudaGetSymbolAddress on device %d: %s", dev,
+                        cudaGetErrorString(e));
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return LSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lsa_status lsa_memindex_score_select_static(const void *q, const float *w, const void *K, const float *k_scale,
+                                            lsa_dtype kdt, const int64_t *seq_offsets, int64_t total_S, int L,
+                                            int B, int n_h, int d_I, float threshold, float *scores_out,
+                                            uint8_t *mask_out, int32_t *idx_out, int32_t *count_out,
+                                            lsa_stream_t stream)
+{
+    LSA_REQUIRE(L > 0 && B > 0 && total_S >= 0 && total_S < (int64_t)1 << 31,
+                "lsa_memindex_score_select_static: L and B must be positive, total_S in [0, 2^31)");
+    const size_t need = score_ws_bytes(L, B, total_S);
+    if (need > (size_t)LSA_STATIC_SCORE_SCRATCH_BYTES)
+        return fail(LSA_ERR_WORKSPACE,
+                    "lsa_memindex_score_select_static: L=%d, B=%d, total_S=%lld need %zu bytes of scratch, more than "
+                    "the %zu-byte static scratch; use lsa_memindex_score_select with a workspace",
+                    L, B, (long long)total_S, need, (size_t)LSA_STATIC_SCORE_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    LSA_TRY(static_scratch(&scratch));
+    return lsa_memindex_score_select(q, w, K, k_scale, kdt, seq_offsets, total_S, L, B, n_h, d_I, threshold,
+                                     scores_out, mask_out, idx_out, count_out, scratch,
+                                     (size_t)LSA_STATIC_SCORE_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

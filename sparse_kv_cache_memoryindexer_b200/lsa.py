@@ -25,6 +25,7 @@ DTYPE_CODE = {torch.float32: LSA_F32, torch.bfloat16: LSA_BF16, torch.float8_e4m
 EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_device",
            "lsa_project_workspace_size", "lsa_project",
            "lsa_score_select_workspace_size", "lsa_memindex_score_select",
+           "lsa_memindex_score_select_static",
            "lsa_fetch_gather",
            "lsa_lightning_topk_workspace_size", "lsa_lightning_topk",
            "lsa_pool_alloc", "lsa_pool_free")
@@ -51,6 +52,7 @@ def _load():
         "lsa_project": (I, [P, P, P, P, I, I, I, I, I, I, I, P, P, P, SZ, P]),
         "lsa_score_select_workspace_size": (SZ, [I, I, I64]),
         "lsa_memindex_score_select": (I, [P, P, P, P, I, P, I64, I, I, I, I, F, P, P, P, P, P, SZ, P]),
+        "lsa_memindex_score_select_static": (I, [P, P, P, P, I, P, I64, I, I, I, I, F, P, P, P, P, P]),
         "lsa_fetch_gather": (I, [P, P, P, I64, I, P, SZ, P, P, P, I, I, P, P, P]),
         "lsa_lightning_topk_workspace_size": (SZ, [I, I, I64, I]),
         "lsa_lightning_topk": (I, [P, P, P, P, I, P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P]),
@@ -141,6 +143,20 @@ def lsa_memindex_score_select(q, w, K, k_scale, seq_offsets, total_S, threshold,
         _p(q), _p(w), _p(K), _p(k_scale), DTYPE_CODE[K.dtype], _p(seq_offsets), int(total_S), L, B, n_h, d_I,
         float(threshold), _p(scores_out), _p(mask_out), _p(idx_out), _p(count_out), _p(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+STATIC_SCORE_SCRATCH_BYTES = 8 << 20  # LSA_STATIC_SCORE_SCRATCH_BYTES in include/lsa.h
+
+
+def lsa_memindex_score_select_static(q, w, K, k_scale, seq_offsets, total_S, threshold, idx_out, count_out,
+                                     scores_out=None, mask_out=None, stream=None):
+    """lsa_memindex_score_select with the library's own per-device scratch instead of a workspace:
+    the call allocates nothing (see include/lsa.h for the size limit and the ordering rule)."""
+    _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
+    L, B, n_h, d_I = q.shape
+    _check(_lib.lsa_memindex_score_select_static(
+        _p(q), _p(w), _p(K), _p(k_scale), DTYPE_CODE[K.dtype], _p(seq_offsets), int(total_S), L, B, n_h, d_I,
+        float(threshold), _p(scores_out), _p(mask_out), _p(idx_out), _p(count_out), _stream(stream)))
 
 
 # ------------------------------------------------------------------------ stage 4b
