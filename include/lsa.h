@@ -78,7 +78,8 @@ lsa_status lsa_check_device(lsa_stream_t stream);
  *   W_w    [L][n_h][d]          dt       W^w stored transposed
  *   q_out  [L][B][n_h][d_I]     dt       queries, rounded to dt (nearest-even)
  *   w_out  [L][B][n_h]          fp32     head weights
- * c^Q is rounded to dt before the second projection and lives in the workspace.
+ * c^Q is rounded to dt before the second projection; on return the workspace starts with
+ * c^Q [L][B][r] in dt.
  * dt: LSA_F32 or LSA_BF16.  Accumulation is fp32.  Workspace: lsa_project_workspace_size.
  * ---------------------------------------------------------------------------------------- */
 size_t lsa_project_workspace_size(int L, int B, int d, int r, int n_h, int d_I, lsa_dtype dt);
@@ -157,11 +158,16 @@ lsa_status lsa_memindex_score_select_static(const void *q, const float *w, const
  * the decode-step Lightning Indexer scores:
  *     hot_K[off_b + j] = K_sel[off_b + idx[off_b + j]],  hot_scale likewise.
  *   idx, count            as written by lsa_memindex_score_select (device)
- *   pool                  mapped page-locked HOST memory, [T][row_bytes]
+ *   pool                  mapped page-locked HOST memory, [T][row_bytes] (nullable together
+ *                         with hot_kv: the rows are skipped)
  *   row_bytes             multiple of 16; pool, hot_kv 16-byte aligned
  *   hot_kv                [T][row_bytes] device (capacity T; slots past count untouched)
  *   K_sel, k_scale_sel    [T][d_I] kdt and [T] fp32 (nullable: K_sel NULL skips the keys;
  *                         k_scale_sel required iff kdt = LSA_FP8_E4M3)
+ * At least one of pool and K_sel is given.  A rows-only call (K_sel NULL) is a small launch
+ * (32 CTAs of 128 threads, up to 8192 sequences) that the host link keeps busy on its own: it is
+ * meant to run on a second stream beside the keys-only call (pool NULL) and the Lightning Top-k,
+ * which needs only the keys.
  *   hot_K, hot_scale      [T][d_I] and [T] fp32.  hot_K holds kdt for LSA_F32 / LSA_BF16 keys
  *                         and bf16 for LSA_FP8_E4M3 keys: the E4M3 codes are decoded exactly
  *                         (every E4M3 value is a bf16 value); the scale stays in hot_scale.

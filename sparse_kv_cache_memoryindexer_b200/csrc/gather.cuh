@@ -14,6 +14,11 @@ namespace lsa {
 
 constexpr int GATHER_ROWS_PER_WARP = 4;
 constexpr int GATHER_MAX_CHUNKS = 4;  // row_bytes <= 4 * 32 * 16 = 2048 per in-flight row
+#ifndef LSA_GATHER_LINK_CTAS
+#define LSA_GATHER_LINK_CTAS 32
+#endif
+constexpr int GATHER_LINK_CTAS = LSA_GATHER_LINK_CTAS;  // CTAs of the rows-only launch (128 threads each)
+constexpr int GATHER_ROWS_MAX_B = 8192; // sequences of the rows-only launch (shared prefix of B + 1 ints)
 
 // 16 E4M3 codes -> 16 bf16 values (exact: every E4M3 value is a bf16 value).
 __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 v, uint4 &lo, uint4 &hi)
@@ -103,6 +108,157 @@ __global__ void __launch_bounds__(256) k_gather(const int32_t *__restrict__ idx,
                 if (ksc && lane == 0) hotsc[off + j0 + r] = __ldg(ksc + src[r]);
             }
         }
+    }
+}
+
+// Shared-memory exclusive prefix pre[0..B] of the counts (clamped to [0, S_b], a bad count flagged),
+// built by one CTA of 128 threads; returns the total.  Every thread calls it.
+__device__ __forceinline__ int block_count_prefix(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
+                                                  int B, int *pre, int *warp_sum)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    auto clamped = [&](int b) {
+        const int64_t S = offs[b + 1] - offs[b];
+        int F = count[b];
+        if (F < 0 || F > S) {
+            if (blockIdx.x == 0) flag(ERRF_COUNT);
+            F = F < 0 ? 0 : (int)S;
+        }
+        return F;
+    };
+    const int per = (B + 127) / 128;
+    const int lo = min(B, (int)threadIdx.x * per), hi = min(B, lo + per);
+    int sum = 0;
+    for (int b = lo; b < hi; b++) sum += clamped(b);
+    const int inc = warp_incl_scan(sum);
+    if (lane == 31) warp_sum[warp] = inc;
+    __syncthreads();
+    int base = 0, total = 0;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        base += k < warp ? warp_sum[k] : 0;
+        total += warp_sum[k];
+    }
+    int run = base + inc - sum;
+    for (int b = lo; b < hi; b++) {
+        pre[b] = run;
+        run += clamped(b);
+    }
+    if (threadIdx.x == 0) pre[B] = total;
+    __syncthreads();
+    return total;
+}
+
+// The sequence of fetched-row number g (g < pre[B]): the largest b with pre[b] <= g, which is never
+// an empty sequence.
+__device__ __forceinline__ int sequence_of_row(const int *pre, int B, int64_t g)
+{
+    int a = 0, z = B - 1;
+    while (a < z) {
+        const int mid = (a + z + 1) >> 1;
+        if (pre[mid] <= g) a = mid;
+        else z = mid - 1;
+    }
+    return a;
+}
+
+// Keys only (device to device): every 16-byte chunk of every fetched key row is one work unit, all
+// rows of all sequences numbered in one range (prefix of the counts in shared memory, as in
+// k_gather_rows), so the launch is balanced and every load is a full coalesced chunk.  E4M3 chunks
+// are decoded to 32 bytes of bf16; chunk 0 of a row also copies the row's scale.
+__global__ void __launch_bounds__(128) k_gather_keys(const int32_t *__restrict__ idx,
+                                                     const int32_t *__restrict__ count,
+                                                     const int64_t *__restrict__ offs, int B,
+                                                     const uint8_t *__restrict__ Ksel, const float *__restrict__ ksc,
+                                                     int krow16, bool kconv, uint8_t *__restrict__ hotK,
+                                                     float *__restrict__ hotsc)
+{
+    extern __shared__ int pre[];
+    __shared__ int warp_sum[4];
+    const int total = block_count_prefix(count, offs, B, pre, warp_sum);
+    const int64_t kb = (int64_t)krow16 * 16, kbo = kconv ? 2 * kb : kb;
+    const int64_t units = (int64_t)total * krow16;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t g = u / krow16;
+        const int ch = (int)(u - g * krow16);
+        const int b = sequence_of_row(pre, B, g);
+        const int64_t off = offs[b], S = offs[b + 1] - off;
+        const int64_t j = g - pre[b];
+        const int s = __ldg(idx + off + j);
+        if (s < 0 || s >= S) {
+            if (ch == 0) flag(ERRF_INDEX);
+            continue;
+        }
+        const int64_t src = off + s, dst = off + j;
+        const uint4 v = __ldg((const uint4 *)(Ksel + src * kb + (int64_t)ch * 16));
+        if (kconv) {
+            uint4 lo, hi;
+            e4m3x16_to_bf16(v, lo, hi);
+            uint4 *d = (uint4 *)(hotK + dst * kbo + (int64_t)ch * 32);
+            d[0] = lo;
+            d[1] = hi;
+        } else {
+            *(uint4 *)(hotK + dst * kbo + (int64_t)ch * 16) = v;
+        }
+        if (ksc && ch == 0) hotsc[dst] = __ldg(ksc + src);
+    }
+}
+
+// Rows only, for a launch that runs beside other kernels: few small CTAs (the host link needs only
+// a few hundred KB of reads in flight), every fetched row of every sequence numbered in one range
+// so that ragged counts cannot leave most warps idle.  Each CTA first builds the exclusive prefix
+// pre[0..B] of the counts in shared memory ((B + 1) ints), then warp w takes rows
+// g = 4 (w + i W) .. + 3 and finds the sequence of g by binary search in pre.
+template <int CH>  // 16-byte chunks per lane and row (row_bytes <= CH * 512)
+__global__ void __launch_bounds__(128) k_gather_rows(const int32_t *__restrict__ idx,
+                                                     const int32_t *__restrict__ count,
+                                                     const int64_t *__restrict__ offs, int B,
+                                                     const uint8_t *__restrict__ pool, int row16,
+                                                     uint8_t *__restrict__ hot_kv)
+{
+    extern __shared__ int pre[];
+    __shared__ int warp_sum[4];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int total = block_count_prefix(count, offs, B, pre, warp_sum);
+
+    const int64_t rb = (int64_t)row16 * 16;
+    const int64_t wstride = (int64_t)gridDim.x * 4;
+    for (int64_t g0 = ((int64_t)blockIdx.x * 4 + warp) * GATHER_ROWS_PER_WARP; g0 < total;
+         g0 += wstride * GATHER_ROWS_PER_WARP) {
+        int64_t src[GATHER_ROWS_PER_WARP], dst[GATHER_ROWS_PER_WARP];
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++) {
+            src[r] = -1;
+            dst[r] = 0;
+            const int64_t g = g0 + r;
+            if (g < total) {
+                const int a = sequence_of_row(pre, B, g);
+                const int64_t off = offs[a], S = offs[a + 1] - off;
+                const int64_t j = g - pre[a];
+                const int s = __ldg(idx + off + j);
+                if (s >= 0 && s < S) {
+                    src[r] = off + s;
+                    dst[r] = off + j;
+                } else if (lane == 0) {
+                    flag(ERRF_INDEX);
+                }
+            }
+        }
+        uint4 v[GATHER_ROWS_PER_WARP][CH];
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++)
+#pragma unroll
+            for (int c = 0; c < CH; c++) {
+                const int ch = lane + 32 * c;
+                if (src[r] >= 0 && ch < row16) v[r][c] = ld_stream16(pool + src[r] * rb + (int64_t)ch * 16);
+            }
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++)
+#pragma unroll
+            for (int c = 0; c < CH; c++) {
+                const int ch = lane + 32 * c;
+                if (src[r] >= 0 && ch < row16) *(uint4 *)(hot_kv + dst[r] * rb + (int64_t)ch * 16) = v[r][c];
+            }
     }
 }
 

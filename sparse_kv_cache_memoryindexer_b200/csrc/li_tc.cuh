@@ -8,7 +8,11 @@
 // head sums of the 4 queries run inside one thread.  Scores go to Y[tau*off_b + i*S_b + j].
 //
 // Work item = (sequence b, chunk of CH key tiles, query group g); items of one chunk are
-// consecutive so that CTAs working at the same time share the chunk's keys in L2.
+// consecutive so that CTAs working at the same time share the chunk's keys in L2.  CTAs claim
+// items from a global counter (not a fixed share each), so that CTAs slowed by other kernels on
+// their SM (the host-link row gather runs beside this kernel) take fewer items instead of setting
+// the finish time.  The producer claims; the claimed item numbers reach the MMA and epilogue warps
+// through a ring of NRING entries in shared memory that every consumer reads in order.
 // Hot keys are bf16 (E4M3 keys were decoded exactly to bf16 by the fetch, their per-entry scale
 // is applied here in the epilogue).
 // Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..9 epilogue (two warps per TMEM
@@ -25,6 +29,7 @@ constexpr int NH = 64;             // heads
 constexpr int NCOL = NQ * NH;      // MMA N = 256
 constexpr int CH = 16;             // key tiles per work item
 constexpr int MAX_STAGES = 8;
+constexpr int NRING = 4;           // claimed items in flight inside a CTA
 constexpr uint32_t IDESC = tc::idesc_bf16(128, NCOL);
 
 struct Params {
@@ -33,6 +38,7 @@ struct Params {
     const int32_t *count;    // [B]
     const int64_t *offs;     // [B+1]
     const int *item_start;   // [B+1]
+    int *item_counter;       // next unclaimed item, zeroed by k_li_items
     float *Y;                // [tau*T]
     int64_t T;
     int B, tau, groups, stages;
@@ -47,7 +53,7 @@ struct Smem {
         s.qbuf = s.kraw + 128 * 256 * stages;
         s.sw = s.qbuf + 2 * NCOL * tc::DI * 2;
         s.bars = s.sw + 8 * 2 * NH * 4;
-        s.misc = s.bars + 8 * (4 * MAX_STAGES + 4 + 4);
+        s.misc = s.bars + 8 * (4 * MAX_STAGES + 8 + 2 * NRING);
         s.total = s.misc + 64 + 1024;
         return s;
     }
@@ -78,13 +84,15 @@ __device__ __forceinline__ int fetched_count(const Params &p, int b, int64_t &S)
 
 // work items per sequence: ceil(ceil(F/128)/CH) chunks x groups.  One block.
 __global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
-                                                   int B, int groups, int *__restrict__ item_start)
+                                                   int B, int groups, int *__restrict__ item_start,
+                                                   int *__restrict__ item_counter)
 {
     __shared__ int warp_tot[32];
     __shared__ int carry;
     if (threadIdx.x == 0) {
         carry = 0;
         item_start[0] = 0;
+        *item_counter = 0;
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -132,8 +140,11 @@ __global__ void __launch_bounds__(320, 1)
     auto qempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 2 + i); };
     auto tfull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 4 + i); };
     auto tempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 6 + i); };
+    auto ifull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 8 + i); };
+    auto iempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 8 + NRING + i); };
     uint32_t *tmem_holder = (uint32_t *)(base + sp.misc);
     volatile int *abort_flag = (volatile int *)(base + sp.misc + 8);
+    volatile int *ring = (volatile int *)(base + sp.misc + 16);  // NRING claimed item numbers
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = p.B;
@@ -148,6 +159,10 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(qempty(i), 1);
             mbar_init(tfull(i), 1);
             mbar_init(tempty(i), 8);
+        }
+        for (int i = 0; i < NRING; i++) {
+            mbar_init(ifull(i), 1);
+            mbar_init(iempty(i), 9);  // the MMA warp and the 8 epilogue warps
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -176,7 +191,16 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = 0; i < MAX_STAGES; i++) issued[i] = false;
             const uint32_t kbytes = 128 * 256;
             bool ok = true;
-            for (int it = blockIdx.x; it < NI && ok; it += gridDim.x) {
+            int islot = 0;
+            uint32_t iphase = 0;
+            while (ok) {
+                const int claim = atomicAdd(p.item_counter, 1);
+                const int it = claim < NI ? claim : -1;  // -1: no work left, the consumers stop
+                if (!mbar_wait(iempty(islot), iphase ^ 1, abort_flag)) { ok = false; break; }
+                ring[islot] = it;
+                mbar_arrive(ifull(islot));  // release: the ring entry is visible to the waiters
+                if (++islot == NRING) { islot = 0; iphase ^= 1; }
+                if (it < 0) break;
                 const Item w = decode_item(p.item_start, B, p.groups, it);
                 int64_t S;
                 const int F = fetched_count(p, w.b, S);
@@ -217,7 +241,14 @@ __global__ void __launch_bounds__(320, 1)
             uint32_t phase = 0, accphase = 0;
             uint32_t quse[2] = {0, 0};
             bool ok = true;
-            for (int it = blockIdx.x; it < NI && ok; it += gridDim.x) {
+            int islot = 0;
+            uint32_t iphase = 0;
+            while (ok) {
+                if (!mbar_wait(ifull(islot), iphase, abort_flag)) { ok = false; break; }
+                const int it = ring[islot];
+                mbar_arrive(iempty(islot));
+                if (++islot == NRING) { islot = 0; iphase ^= 1; }
+                if (it < 0) break;
                 const Item w = decode_item(p.item_start, B, p.groups, it);
                 int64_t S;
                 const int F = fetched_count(p, w.b, S);
@@ -257,7 +288,15 @@ __global__ void __launch_bounds__(320, 1)
         int acc = 0;
         uint32_t accphase = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < NI && ok; it += gridDim.x) {
+        int islot = 0;
+        uint32_t iphase = 0;
+        while (ok) {
+            if (!mbar_wait_warp(ifull(islot), iphase, abort_flag)) { ok = false; break; }
+            const int it = ring[islot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(iempty(islot));
+            if (++islot == NRING) { islot = 0; iphase ^= 1; }
+            if (it < 0) break;
             const Item w = decode_item(p.item_start, B, p.groups, it);
             int64_t S;
             const int F = fetched_count(p, w.b, S);
@@ -336,15 +375,16 @@ inline bool li_tc_supported(int n_h, int d_I, int tau, int kdt)
     return n_h == li::NH && d_I == tc::DI && tau % li::NQ == 0 && (kdt == DT_BF16 || kdt == DT_FP8) && tc_available();
 }
 
-// hotK: bf16 [T][128] (decoded E4M3 codes when hsc is given).  item_start: device [B+1].
+// hotK: bf16 [T][128] (decoded E4M3 codes when hsc is given).  item_start: device [B+1];
+// item_counter: one device int (zeroed by the planner).
 // Launches the item planner and the scoring kernel; *launches counts them.
 inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK, const float *hsc,
                                const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, float *Y,
-                               int *item_start, int sms, cudaStream_t st, int *launches)
+                               int *item_start, int *item_counter, int sms, cudaStream_t st, int *launches)
 {
     using namespace li;
     *launches = 0;
-    k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / NQ, item_start);
+    k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / NQ, item_start, item_counter);
     (*launches)++;
     if (T == 0) return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
     CUtensorMap kmap, qmap;
@@ -357,6 +397,7 @@ inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK
     p.count = count;
     p.offs = offs;
     p.item_start = item_start;
+    p.item_counter = item_counter;
     p.Y = Y;
     p.T = T;
     p.B = B;

@@ -327,18 +327,24 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
                             lsa_stream_t stream)
 {
     cudaStream_t st = (cudaStream_t)stream;
-    LSA_REQUIRE(idx && count && seq_offsets && pool && hot_kv, "lsa_fetch_gather: null pointer");
+    LSA_REQUIRE(idx && count && seq_offsets, "lsa_fetch_gather: null pointer");
+    LSA_REQUIRE((pool == nullptr) == (hot_kv == nullptr), "lsa_fetch_gather: pool and hot_kv are given together");
+    LSA_REQUIRE(pool || K_sel, "lsa_fetch_gather: nothing to gather (pool and K_sel are both NULL)");
     LSA_REQUIRE(B > 0 && total_S >= 0, "lsa_fetch_gather: sizes must be positive");
-    LSA_REQUIRE(row_bytes > 0 && row_bytes % 16 == 0, "lsa_fetch_gather: row_bytes must be a positive multiple of 16");
-    if (row_bytes > 16 * 32 * GATHER_MAX_CHUNKS)
-        return fail(LSA_ERR_UNSUPPORTED, "lsa_fetch_gather: row_bytes above %d", 16 * 32 * GATHER_MAX_CHUNKS);
-    LSA_REQUIRE(aligned(pool, 16) && aligned(hot_kv, 16), "lsa_fetch_gather: pool and hot_kv must be 16-byte aligned");
     void *dpool = nullptr;
-    cudaError_t e = cudaHostGetDevicePointer(&dpool, const_cast<void *>(pool), 0);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return fail(LSA_ERR_INVALID_ARG, "lsa_fetch_gather: pool is not mapped page-locked host memory (%s)",
-                    cudaGetErrorString(e));
+    if (pool) {
+        LSA_REQUIRE(row_bytes > 0 && row_bytes % 16 == 0,
+                    "lsa_fetch_gather: row_bytes must be a positive multiple of 16");
+        if (row_bytes > 16 * 32 * GATHER_MAX_CHUNKS)
+            return fail(LSA_ERR_UNSUPPORTED, "lsa_fetch_gather: row_bytes above %d", 16 * 32 * GATHER_MAX_CHUNKS);
+        LSA_REQUIRE(aligned(pool, 16) && aligned(hot_kv, 16),
+                    "lsa_fetch_gather: pool and hot_kv must be 16-byte aligned");
+        cudaError_t e = cudaHostGetDevicePointer(&dpool, const_cast<void *>(pool), 0);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return fail(LSA_ERR_INVALID_ARG, "lsa_fetch_gather: pool is not mapped page-locked host memory (%s)",
+                        cudaGetErrorString(e));
+        }
     }
     int krow16 = 0;
     if (K_sel) {
@@ -353,6 +359,26 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
         if (kdt == LSA_FP8_E4M3 && krow16 > 32)
             return fail(LSA_ERR_UNSUPPORTED, "lsa_fetch_gather: E4M3 key rows above 512 bytes");
     }
+    const int row16 = pool ? (int)(row_bytes / 16) : 0;
+    if (pool && !K_sel && B <= GATHER_ROWS_MAX_B) {
+        // rows only: a small launch meant to run beside other work (see k_gather_rows)
+        const size_t smem = sizeof(int) * (size_t)(B + 1);
+        const dim3 grid(GATHER_LINK_CTAS), block(128);
+        const uint8_t *src = (const uint8_t *)dpool;
+        if (row16 <= 32) k_gather_rows<1><<<grid, block, smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
+        else if (row16 <= 64) k_gather_rows<2><<<grid, block, smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
+        else k_gather_rows<4><<<grid, block, smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
+        LSA_TRY(launched("gather rows"));
+        return ok();
+    }
+    if (!pool && B <= GATHER_ROWS_MAX_B) {
+        // keys only: one thread per 16-byte chunk of every fetched key row
+        const size_t smem = sizeof(int) * (size_t)(B + 1);
+        k_gather_keys<<<num_sms() * 8, 128, smem, st>>>(idx, count, seq_offsets, B, (const uint8_t *)K_sel, k_scale_sel,
+                                                        krow16, kdt == LSA_FP8_E4M3, (uint8_t *)hot_K, hot_scale);
+        LSA_TRY(launched("gather keys"));
+        return ok();
+    }
     const int warps_per_block = 8;
     int64_t gx = ((total_S / (B > 0 ? B : 1)) + warps_per_block * GATHER_ROWS_PER_WARP - 1) /
                  (warps_per_block * GATHER_ROWS_PER_WARP);
@@ -360,7 +386,7 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
     if (gx > cap) gx = cap;
     if (gx < 1) gx = 1;
     k_gather<<<dim3((unsigned)gx, (unsigned)B), 32 * warps_per_block, 0, st>>>(
-        idx, count, seq_offsets, (const uint8_t *)dpool, (int)(row_bytes / 16), (uint8_t *)hot_kv,
+        idx, count, seq_offsets, (const uint8_t *)dpool, row16, (uint8_t *)hot_kv,
         (const uint8_t *)K_sel, k_scale_sel, krow16, kdt == LSA_FP8_E4M3, (uint8_t *)hot_K, hot_scale);
     LSA_TRY(launched("gather"));
     return ok();
@@ -368,12 +394,12 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
 
 // ------------------------------------------------------------------------------ stage 5
 
-// Workspace of lsa_lightning_topk: [item_start: B+1 ints][Y: tau * total_S floats].
+// Workspace of lsa_lightning_topk: [item_start: B+1 ints, item counter: 1 int][Y: tau * total_S floats].
 size_t lsa_lightning_topk_workspace_size(int B, int tau, int64_t total_S, int k)
 {
     (void)k;
     if (B <= 0 || tau <= 0 || total_S < 0) return 0;
-    return align_up(sizeof(int) * (size_t)(B + 1), 256) + align_up(sizeof(float) * (size_t)tau * (size_t)total_S, 256);
+    return align_up(sizeof(int) * (size_t)(B + 2), 256) + align_up(sizeof(float) * (size_t)tau * (size_t)total_S, 256);
 }
 
 lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void *hot_K, const float *hot_scale,
@@ -395,14 +421,15 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     LSA_REQUIRE((int64_t)tau * total_S < ((int64_t)1 << 40), "lsa_lightning_topk: tau * total_S too large");
     if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: n_h must be <= 128");
     int *item_start = (int *)workspace;
-    float *Y = (float *)((char *)workspace + align_up(sizeof(int) * (size_t)(B + 1), 256));
+    int *item_counter = item_start + B + 1;
+    float *Y = (float *)((char *)workspace + align_up(sizeof(int) * (size_t)(B + 2), 256));
     // E4M3 keys arrive here decoded to bf16 by lsa_fetch_gather (scales in hot_scale)
     const int hdt = (kdt == LSA_FP8_E4M3) ? DT_BF16 : kdt;
     if (li_tc_supported(n_h, d_I, tau, kdt)) {
         LSA_REQUIRE(aligned(q_dec, 16) && aligned(hot_K, 16), "lsa_lightning_topk: q_dec and hot_K must be 16-byte aligned");
         int n = 0;
         const lsa_status s = launch_li_tc(q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, Y,
-                                          item_start, num_sms(), st, &n);
+                                          item_start, item_counter, num_sms(), st, &n);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK) return fail(s, "lsa_lightning_topk: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
     } else {

@@ -163,12 +163,13 @@ def lsa_memindex_score_select_static(q, w, K, k_scale, seq_offsets, total_S, thr
 
 def lsa_fetch_gather(idx, count, seq_offsets, total_S, pool, hot_kv, K_sel=None, k_scale_sel=None,
                      hot_K=None, hot_scale=None, stream=None):
-    """Gather fetched rows from the mapped host cold pool (and the keys of one layer)."""
+    """Gather fetched rows from the mapped host cold pool and/or the keys of one layer (pool and
+    hot_kv None: keys only; K_sel None: rows only, a small launch meant for a second stream)."""
     _dev(idx, count, seq_offsets, hot_kv, K_sel, k_scale_sel, hot_K, hot_scale)
-    if pool.device.type != "cpu":
+    if pool is not None and pool.device.type != "cpu":
         raise ValueError("the cold pool must be (mapped page-locked) host memory")
     B = count.numel()
-    row_bytes = pool.shape[1] * pool.element_size()
+    row_bytes = pool.shape[1] * pool.element_size() if pool is not None else 0
     kdt = DTYPE_CODE[K_sel.dtype] if K_sel is not None else 0
     d_I = K_sel.shape[-1] if K_sel is not None else 0
     _check(_lib.lsa_fetch_gather(_p(idx), _p(count), _p(seq_offsets), int(total_S), B, _p(pool), row_bytes,

@@ -42,6 +42,7 @@ class IndexerPath:
         self.topk_idx = torch.empty((B, tau, k), dtype=torch.int32, device=dev)
         self.topk_score = torch.empty((B, tau, k), dtype=torch.float32, device=dev)
         self.ws_topk = ws(lsa.lsa_lightning_topk_workspace_size(B, tau, T, k))
+        self._link = torch.cuda.Stream(device=dev)  # the host-link row gather of run()
 
     def project(self, h, W_dq, W_iuq, W_w, stream=None):
         lsa.lsa_project(h, W_dq, W_iuq, W_w, self.q, self.w, self.ws_proj, stream=stream)
@@ -52,8 +53,18 @@ class IndexerPath:
                                       scores_out=self.scores, mask_out=self.mask, stream=stream)
 
     def fetch(self, seq_offsets, pool, K_sel, k_scale_sel, stream=None):
+        """Rows and keys in one launch."""
         lsa.lsa_fetch_gather(self.idx, self.count, seq_offsets, self.total_S, pool, self.hot_kv, K_sel, k_scale_sel,
                              self.hot_K, self.hot_scale, stream=stream)
+
+    def fetch_keys(self, seq_offsets, K_sel, k_scale_sel, stream=None):
+        """The keys of the fetched entries only (device to device; the Top-k needs nothing else)."""
+        lsa.lsa_fetch_gather(self.idx, self.count, seq_offsets, self.total_S, None, None, K_sel, k_scale_sel,
+                             self.hot_K, self.hot_scale, stream=stream)
+
+    def fetch_rows(self, seq_offsets, pool, stream=None):
+        """The KV rows of the fetched entries only, over the host link."""
+        lsa.lsa_fetch_gather(self.idx, self.count, seq_offsets, self.total_S, pool, self.hot_kv, stream=stream)
 
     def topk(self, q_dec, w_dec, seq_offsets, stream=None):
         lsa.lsa_lightning_topk(q_dec, w_dec, self.hot_K, self.hot_scale, self.idx, self.count, seq_offsets,
@@ -61,9 +72,33 @@ class IndexerPath:
                                stream=stream)
 
     def run(self, h, W_dq, W_iuq, W_w, K, k_scale, seq_offsets, pool, q_dec, w_dec, sel_layer=0,
-            threshold=0.5, stream=None):
-        """The whole hot path for one trigger window."""
-        self.project(h, W_dq, W_iuq, W_w, stream)
-        self.select(K, k_scale, seq_offsets, threshold, stream=stream)
-        self.fetch(seq_offsets, pool, K[sel_layer], None if k_scale is None else k_scale[sel_layer], stream)
-        self.topk(q_dec, w_dec, seq_offsets, stream)
+            threshold=0.5, stream=None, events=None):
+        """The whole hot path for one trigger window.
+
+        The KV rows cross the host link on a second stream while the keys are gathered and the
+        Top-k runs on `stream` (the Top-k reads only the keys); `stream` waits for both before
+        it returns, so work queued on it afterwards sees the whole window.  events: optional
+        list of 7 timing events, recorded at the stage boundaries (start, after project, after
+        select, after the keys, after the Top-k, after the rows (second stream), end).
+        """
+        st = torch.cuda.current_stream() if stream is None else stream
+        ev = events if events is not None else [None] * 7
+        rec = lambda e, s: e.record(s) if e is not None else None
+        rec(ev[0], st)
+        self.project(h, W_dq, W_iuq, W_w, st)
+        rec(ev[1], st)
+        self.select(K, k_scale, seq_offsets, threshold, stream=st)
+        rec(ev[2], st)
+        selected = torch.cuda.Event()
+        selected.record(st)
+        self._link.wait_event(selected)
+        self.fetch_rows(seq_offsets, pool, self._link)
+        rec(ev[5], self._link)
+        rows_done = torch.cuda.Event()
+        rows_done.record(self._link)
+        self.fetch_keys(seq_offsets, K[sel_layer], None if k_scale is None else k_scale[sel_layer], st)
+        rec(ev[3], st)
+        self.topk(q_dec, w_dec, seq_offsets, st)
+        rec(ev[4], st)
+        st.wait_event(rows_done)
+        rec(ev[6], st)

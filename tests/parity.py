@@ -10,6 +10,8 @@ whose oracle score is within that bound of the k-th score may swap in or out of 
 import numpy as np
 import torch
 
+import oracle
+
 SIGMOID_TOL = 2e-3
 
 
@@ -87,3 +89,34 @@ def check_topk_query(gi, gs, y_or, s_list, tol, k, what=""):
         assert not chosen[must_out].any(), f"{what}: {chosen[must_out].sum()} clear non-Top-k entries selected"
         return int((~must_in & ~must_out).sum())
     return 0
+
+
+def check_project(h, W_dq, W_iuq, W_w, n_h, d_I, q_gpu, w_gpu, c_gpu, what=""):
+    """Stage 1 against the oracle, in two exact halves (all tensors on the CPU, [L][B]... layout).
+
+    c = h W^DQ rounded to the storage type: the GPU's fp32 sum and the oracle's exact sum may round
+    to neighbouring values, |dc| <= ulp + 2^-22 d sum|h W|.  A neighbour of c moves q by far more
+    than one ulp of q where q cancels, so q is checked against the oracle's second projection of
+    the GPU's own c (identity as W^DQ makes the oracle's first projection an exact copy of c):
+    |dq| <= ulp + 2^-22 r sum|c W^IUQ|.  w = h W^w in fp32: |dw| <= 2^-22 d sum|h W^w|.
+    """
+    L, B, d = h.shape
+    r = W_dq.shape[1]
+    bf = h.dtype == torch.bfloat16
+    ulp = (lambda a, b: torch.maximum(a.abs(), b.abs()) * 2.0 ** -7) if bf else (lambda a, b: torch.zeros_like(a))
+    q_ref, w_ref, c_ref = oracle.project(h, W_dq, W_iuq, W_w, n_h, d_I, want_c=True)
+    h64 = h.double()
+    wb = (2.0 ** -22) * d * torch.einsum("lbi,lhi->lbh", h64.abs(), W_w.double().abs())
+    assert ((w_gpu.double() - w_ref.double()).abs() <= wb).all(), f"{what}: w"
+    cb = (2.0 ** -22) * d * torch.einsum("lbi,lji->lbj", h64.abs(), W_dq.double().abs())
+    dc = (c_gpu.double() - c_ref.double()).abs()
+    assert (dc <= ulp(c_gpu.double(), c_ref.double()) * 1.0001 + cb).all(), f"{what}: c"
+    if bf:  # neighbours only where the exact c lies near a rounding boundary
+        assert (dc > 0).double().mean() < 0.15, f"{what}: too many c differ"
+    eye = torch.eye(r, dtype=h.dtype).expand(L, r, r).contiguous()
+    q2, _ = oracle.project(c_gpu.contiguous(), eye, W_iuq, torch.zeros((L, n_h, r), dtype=h.dtype), n_h, d_I)
+    qb = (2.0 ** -22) * r * torch.einsum("lbj,loj->lbo", c_gpu.double().abs(), W_iuq.double().abs())
+    dq = (q_gpu.double() - q2.double()).reshape(qb.shape).abs()
+    assert (dq <= ulp(q_gpu.double(), q2.double()).reshape(qb.shape) * 1.0001 + qb).all(), f"{what}: q"
+    if bf:
+        assert (dq > 0).double().mean() < 0.05, f"{what}: too many q differ"
