@@ -13,6 +13,7 @@
 #include "score_select.cuh"
 #include "score_tc.cuh"
 #include "li_tc.cuh"
+#include "proj_tc.cuh"
 #include "topk.cuh"
 
 using namespace lsa;
@@ -241,7 +242,16 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
     LSA_REQUIRE(aligned(workspace, 256), "lsa_project: workspace must be 256-byte aligned");
     const int nq = n_h * d_I;
     void *c = workspace;
-    if (dt == LSA_BF16) {
+    if (proj_tc_supported(dt, B, d) && proj_tc_supported(dt, B, r)) {
+        const int sms = num_sms();
+        lsa_status s = launch_proj_tc(h, W_dq, c, false, L, B, r, d, sms, st);
+        if (s == LSA_OK) s = launched("project c (tensor cores)");
+        if (s == LSA_OK) s = launch_proj_tc(h, W_w, w_out, true, L, B, n_h, d, sms, st);
+        if (s == LSA_OK) s = launched("project w (tensor cores)");
+        if (s == LSA_OK) s = launch_proj_tc(c, W_iuq, q_out, false, L, B, nq, r, sms, st);
+        if (s == LSA_OK) s = launched("project q (tensor cores)");
+        if (s != LSA_OK) return fail(s, "lsa_project: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
+    } else if (dt == LSA_BF16) {
         k_rowdot<DT_BF16, DT_BF16><<<dim3((r + 7) / 8, L), 256, 0, st>>>(h, W_dq, c, B, d, r);
         LSA_TRY(launched("project c"));
         k_rowdot<DT_BF16, DT_F32><<<dim3((n_h + 7) / 8, L), 256, 0, st>>>(h, W_w, w_out, B, d, n_h);

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import synth
-from parity import check_project, check_select, check_topk_query, keys_as_float, li_tolerance
+from parity import check_project, check_select, check_topk_query, keys_as_float, li_tolerance, or_exempt
 
 pytestmark = pytest.mark.gpu
 
@@ -243,9 +243,19 @@ def test_topk_ties_prefer_smaller_entry(m):
 
 # ------------------------------------------------------------------ stage 1 and the whole path
 
-@pytest.mark.parametrize("name", ["tiny_fp32", "ctx128k_bf16"])
-def test_project_parity(m, name):
-    wl = CASES[name]()
+PROJ_CASES = {
+    "tiny_fp32": lambda: synth.workload("tiny_fp32"),
+    "ctx128k_bf16": lambda: synth.workload("ctx128k_bf16"),
+    # batch sizes that are not a multiple of the MMA N step (16) and span several 32-column loads
+    "b37": lambda: synth.workload("ctx128k_bf16", B=37, S=(64,) * 37, fetch=(0.1,) * 37, name="proj_b37"),
+    "b100_small": lambda: synth.workload("ctx128k_bf16", B=100, S=(64,) * 100, fetch=(0.1,) * 100, d=512, r=256,
+                                         name="proj_b100"),
+}
+
+
+@pytest.mark.parametrize("name", list(PROJ_CASES))
+def test_project_parity(m, name, kernel_path):
+    wl = PROJ_CASES[name]()
     inp = synth.make_inputs(wl, parts=("proj",))
     q_ref, w_ref = oracle.project(inp.h, inp.W_dq, inp.W_iuq, inp.W_w, wl.n_h, wl.d_I)
     q = torch.empty_like(q_ref, device="cuda")
@@ -261,16 +271,18 @@ def test_project_parity(m, name):
 
 @pytest.mark.parametrize("name", ["tiny_fp32", "ctx128k_bf16"])
 def test_whole_path_parity(m, name):
+    """One window through IndexerPath.run against the oracle.  Each stage is checked on its own
+    inputs (the GPU's outputs of the stage before); the chain as a whole is checked on the fetch
+    decisions: equal to the oracle's own chain except entries near the threshold under either
+    set of queries (projection roundings may land one bf16 step apart, which moves a score)."""
     wl = CASES[name]()
     inp = synth.make_inputs(wl)
     offs = inp.seq_offsets.numpy()
     T = wl.total_S
-    # oracle chain
-    q_r, w_r = oracle.project(inp.h, inp.W_dq, inp.W_iuq, inp.W_w, wl.n_h, wl.d_I)
     sel = wl.sel_layer
     ks = inp.k_scale
-    ref = oracle.score(q_r, w_r, inp.K, ks, offs)
-    # CUDA path through one IndexerPath window
+    q_r, w_r = oracle.project(inp.h, inp.W_dq, inp.W_iuq, inp.W_w, wl.n_h, wl.d_I)
+    chain = oracle.score(q_r, w_r, inp.K, ks, offs)
     path = m.IndexerPath(wl.L, wl.B, wl.d, wl.r, wl.n_h, wl.d_I, wl.tau, wl.k, T, wl.row_bytes,
                          synth.DTYPES[wl.dtype], synth.DTYPES[wl.kdtype], with_scores=True, with_mask=True)
     pool = m.MappedPool(T, wl.row_bytes)
@@ -280,18 +292,28 @@ def test_whole_path_parity(m, name):
                  pool.tensor, dev(inp.q_dec), dev(inp.w_dec), sel_layer=sel)
         m.lsa_check_device()
         mask, idx, cnt = path.mask.cpu().numpy(), path.idx.cpu().numpy(), path.count.cpu().numpy()
-        check_select(mask, idx, cnt, path.scores.cpu().numpy(), ref, offs, what=name)
-        r_kv, r_K, r_s = oracle.gather(torch.from_numpy(ref["idx"]), torch.from_numpy(ref["count"]), offs, inp.pool,
-                                       inp.K[sel], ks[sel] if ks is not None else None, wl.d_I)
+        # stage 1 on its inputs
+        c = path.ws_proj[:wl.L * wl.B * wl.r * path.q.element_size()].view(path.q.dtype).view(wl.L, wl.B, wl.r)
+        check_project(inp.h, inp.W_dq, inp.W_iuq, inp.W_w, wl.n_h, wl.d_I, path.q.cpu(), path.w.cpu(), c.cpu(),
+                      what=name)
+        # stages 2-4a on their inputs
+        stage = oracle.score(path.q.cpu(), path.w.cpu(), inp.K, ks, offs)
+        check_select(mask, idx, cnt, path.scores.cpu().numpy(), stage, offs, what=name)
+        # the chain's decisions
+        ex = or_exempt(chain["I"]) | or_exempt(stage["I"]) | (chain["mask"] != stage["mask"])
+        bad = (mask != chain["mask"]) & ~ex
+        assert not bad.any(), f"{name}: {bad.sum()} decisions differ from the oracle chain outside the band"
+        assert ex.mean() < 0.05  # the band holds a few entries, not the bulk (tiny: 16 of 512)
+        # stage 4b and 5 on their inputs (the GPU's index lists)
+        ti_, ci_ = torch.from_numpy(idx), torch.from_numpy(cnt)
+        r_kv, _, _ = oracle.gather(ti_, ci_, offs, inp.pool, None, None, wl.d_I)
+        used = np.zeros(T, dtype=bool)
         for b in range(wl.B):
-            if cnt[b] != ref["count"][b] or not np.array_equal(idx[offs[b]:offs[b] + cnt[b]],
-                                                              ref["idx"][offs[b]:offs[b] + cnt[b]]):
-                continue  # an exempt near-threshold entry flipped: later stages see another set
-            sl = slice(offs[b], offs[b] + cnt[b])
-            assert torch.equal(path.hot_kv.cpu()[sl], r_kv[sl])
-            ti, ts = path.topk_idx.cpu().numpy(), path.topk_score.cpu().numpy()
-            check_topk(inp, torch.from_numpy(ref["idx"]), torch.from_numpy(ref["count"]), wl.k, ti, ts,
-                       [(b, i) for i in range(wl.tau)])
+            used[offs[b]:offs[b] + cnt[b]] = True
+        used = torch.from_numpy(used)
+        assert torch.equal(path.hot_kv.cpu()[used], r_kv[used])
+        ti, ts = path.topk_idx.cpu().numpy(), path.topk_score.cpu().numpy()
+        check_topk(inp, ti_, ci_, wl.k, ti, ts, [(b, i) for b in range(wl.B) for i in range(wl.tau)])
     finally:
         pool.free()
 
