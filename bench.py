@@ -49,6 +49,35 @@ def parse_args():
     return p.parse_args()
 
 
+# ------------------------------------------------------------------------------------ ranks
+
+def dist_env():
+    """(rank, world size, local rank) from the launcher's environment (1 process without one)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_workload(name, rank, batch=0):
+    """The workload of one rank: same shapes on every rank, its own seed (sequences are independent)."""
+    base = synth.workload(name)
+    over = {"B": batch} if batch else {}
+    return synth.workload(name, seed=base.seed + 7919 * rank, **over)
+
+
+def max_over_ranks(ms, world, device):
+    """The job's time is the slowest rank's (every rank takes part in the same collective)."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank, steps, elapsed_ms):
+    """Units all ranks processed per second of the (max-over-ranks) elapsed time."""
+    return world * units_per_rank * steps / (elapsed_ms * 1e-3)
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -214,9 +243,7 @@ def h2d_bandwidth(device, nbytes=1 << 30):
 def run_lsa(args, rank, world, device):
     import sparse_kv_cache_memoryindexer_b200 as lsa
     torch.cuda.set_device(device)
-    base = synth.workload(args.workload)
-    over = {"B": args.batch} if args.batch else {}
-    wl = synth.workload(args.workload, seed=base.seed + 7919 * rank, **over)
+    wl = rank_workload(args.workload, rank, args.batch)
     T = wl.total_S
     dt, kdt = synth.DTYPES[wl.dtype], synth.DTYPES[wl.kdtype]
     pool = lsa.MappedPool(T, wl.row_bytes)
@@ -270,10 +297,7 @@ def run_lsa(args, rank, world, device):
         for i, (a, b) in enumerate(spans):
             stage_ms[i] += ev[a].elapsed_time(ev[b])
     stage_ms /= args.steps
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
 
     # end to end through the public API with host buffers
     e2e = None
@@ -309,11 +333,8 @@ def run_lsa(args, rank, world, device):
         b.record(st)
         torch.cuda.synchronize(device)
         e_ms = a.elapsed_time(b)
-        if world > 1:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = {"value": world * wl.L * T * args.e2e_steps / (e_ms * 1e-3), "unit": UNIT,
+        e_ms = max_over_ranks(e_ms, world, device)
+        e2e = {"value": job_throughput(world, wl.L * T, args.e2e_steps, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
         del host
@@ -323,7 +344,7 @@ def run_lsa(args, rank, world, device):
         peaks = load_peaks()
         alg = algorithmic(wl, fetched)
         ms = elapsed_ms / args.steps
-        value = world * wl.L * T * args.steps / (elapsed_ms * 1e-3)
+        value = job_throughput(world, wl.L * T, args.steps, elapsed_ms)
         sel_ms = stage_ms[1]
         score_gbs = alg["score_bytes"] / (sel_ms * 1e-3) / 1e9
         traffic, traffic_src = score_traffic(wl)
@@ -377,9 +398,7 @@ def run_lsa(args, rank, world, device):
 
 def main():
     args = parse_args()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = dist_env()
 
     if args.impl == "reference":
         if rank != 0:
