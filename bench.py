@@ -46,6 +46,7 @@ def parse_args():
                    help="entries of the oracle's bounded sample (default: sized for a few minutes of CPU work)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-incremental", action="store_true", help="skip the incremental-fetch measurement")
     return p.parse_args()
 
 
@@ -240,6 +241,59 @@ def h2d_bandwidth(device, nbytes=1 << 30):
 
 # ------------------------------------------------------------------------------------ lsa arm
 
+def drifted_lists(idx, cnt, offs, drift, seed):
+    """The next window's fetch lists: each sequence keeps 1 - drift of its entries and replaces the
+    rest by entries it did not fetch (so the count stays about the same); ascending."""
+    rng = np.random.default_rng(seed)
+    new_idx = np.full_like(idx, -1)
+    new_cnt = np.zeros_like(cnt)
+    for b in range(cnt.size):
+        S = int(offs[b + 1] - offs[b])
+        P = idx[offs[b]:offs[b] + cnt[b]].astype(np.int64)
+        kept = P[rng.random(P.size) >= drift]
+        free = np.ones(S, dtype=bool)
+        free[P] = False
+        cand = np.nonzero(free)[0]
+        add = rng.choice(cand, min(cand.size, P.size - kept.size), replace=False) if cand.size else cand
+        N = np.unique(np.concatenate([kept, add]))
+        new_idx[offs[b]:offs[b] + N.size] = N
+        new_cnt[b] = N.size
+    return new_idx, new_cnt
+
+
+def measure_incremental(lsa, path, wl, offs, pool, st, drift=0.1, reps=5):
+    """S4b incremental: the next window's rows with this window's rows resident (device copies for
+    the common entries, the host link for the rest), timed alone on the stream."""
+    T = wl.total_S
+    offs_h = offs.cpu().numpy()
+    idx_n, cnt_n = drifted_lists(path.idx.cpu().numpy(), path.count.cpu().numpy(), offs_h, drift, seed=wl.seed + 17)
+    idx_d = torch.from_numpy(idx_n).to(offs.device)
+    cnt_d = torch.from_numpy(cnt_n).to(offs.device)
+    hot_new = torch.empty_like(path.hot_kv)
+    ws = torch.empty(lsa.lsa_fetch_incremental_workspace_size(wl.B, T), dtype=torch.uint8, device=offs.device)
+    host_rows = torch.zeros(1, dtype=torch.int32, device=offs.device)
+
+    def call():
+        lsa.lsa_fetch_gather_incremental(idx_d, cnt_d, offs, T, path.idx, path.count, offs, T, path.hot_kv,
+                                         pool.tensor, hot_new, ws, host_rows_out=host_rows, stream=st)
+    for _ in range(2):
+        call()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(reps):
+        call()
+    b.record(st)
+    torch.cuda.synchronize()
+    lsa.lsa_check_device(st)
+    ms = a.elapsed_time(b) / reps
+    n_host, rows = int(host_rows.item()), int(cnt_n.sum())
+    del hot_new, ws
+    return {"drift": drift, "rows": rows, "host_rows": n_host, "ms": ms,
+            "host_link_GBps": n_host * wl.row_bytes / (ms * 1e-3) / 1e9,
+            "note": "next window = this window with %d %% of each sequence's entries replaced; timed alone"
+                    % round(100 * drift)}
+
+
 def run_lsa(args, rank, world, device):
     import sparse_kv_cache_memoryindexer_b200 as lsa
     torch.cuda.set_device(device)
@@ -339,6 +393,10 @@ def run_lsa(args, rank, world, device):
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
         del host
 
+    incr = None
+    if not args.no_incremental and world == 1:
+        incr = measure_incremental(lsa, path, wl, offs, pool, st)
+
     result = None
     if rank == 0:
         peaks = load_peaks()
@@ -391,6 +449,7 @@ def run_lsa(args, rank, world, device):
             "gpu_launches": launches,
             "clocks": clk,
             "e2e": e2e,
+            "incremental_fetch": None if incr is None else dict(incr, full_fetch_ms=stage_ms[4]),
         }
     pool.free()
     return result

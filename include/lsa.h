@@ -165,7 +165,7 @@ lsa_status lsa_memindex_score_select_static(const void *q, const float *w, const
  *   K_sel, k_scale_sel    [T][d_I] kdt and [T] fp32 (nullable: K_sel NULL skips the keys;
  *                         k_scale_sel required iff kdt = LSA_FP8_E4M3)
  * At least one of pool and K_sel is given.  A rows-only call (K_sel NULL) is a small launch
- * (32 CTAs of 128 threads, up to 8192 sequences) that the host link keeps busy on its own: it is
+ * (128 CTAs of 128 threads, up to 8192 sequences) that the host link keeps busy on its own: it is
  * meant to run on a second stream beside the keys-only call (pool NULL) and the Lightning Top-k,
  * which needs only the keys.
  *   hot_K, hot_scale      [T][d_I] and [T] fp32.  hot_K holds kdt for LSA_F32 / LSA_BF16 keys
@@ -178,6 +178,39 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count,
                             const void *pool, size_t row_bytes, void *hot_kv,
                             const void *K_sel, const float *k_scale_sel, lsa_dtype kdt, int d_I,
                             void *hot_K, float *hot_scale, lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Stage 4b, incremental -- the fetch of one window when the previous window's hot rows are still
+ * resident.  The pages fetch from the cold pool once per trigger window (hyper.ai summary, one-line
+ * summary and "Method"); an entry that the previous window fetched and this one selects again need
+ * not cross the host link a second time.
+ *     hot_kv[off_b + j] = pool[off_b + idx[off_b + j]]      for j < count[b]       (as above)
+ * where a row whose entry s = idx[off_b + j] is also in the previous window's list of sequence b
+ * (prev_idx[poff_b + j'] = s, j' < prev_count[b]) is copied on the device from
+ * prev_hot_kv[poff_b + j'], and only the other rows cross the host link.
+ *   idx, count, seq_offsets, total_S    this window (as written by lsa_memindex_score_select)
+ *   prev_idx, prev_count,               the previous window of the same B sequences, whose
+ *   prev_seq_offsets, prev_total_S      entries keep their numbers (sequences may have grown);
+ *                                       each prev_idx segment ascending (as the select writes it;
+ *                                       otherwise rows are fetched that could have been copied)
+ *   prev_hot_kv    [prev_total_S][row_bytes] device: the previous window's rows (read only)
+ *   pool, row_bytes                     as lsa_fetch_gather; pool laid out at this window's offsets
+ *   hot_kv         [total_S][row_bytes] device, must not overlap prev_hot_kv (double buffer)
+ *   host_rows_out  nullable device int32: the number of rows read over the host link
+ * Workspace: lsa_fetch_incremental_workspace_size (a slot map, the list of rows to fetch and their
+ * count).  At most 8192 sequences.  Three launches: lookup, device copy, host rows (128 CTAs, as the
+ * rows-only call of lsa_fetch_gather).  The method has no incremental fetch of its own: it is the
+ * first widening of the path beyond one window.
+ * ---------------------------------------------------------------------------------------- */
+size_t lsa_fetch_incremental_workspace_size(int B, int64_t total_S);
+
+lsa_status lsa_fetch_gather_incremental(const int32_t *idx, const int32_t *count,
+                                        const int64_t *seq_offsets, int64_t total_S, int B,
+                                        const int32_t *prev_idx, const int32_t *prev_count,
+                                        const int64_t *prev_seq_offsets, int64_t prev_total_S,
+                                        const void *prev_hot_kv, const void *pool, size_t row_bytes,
+                                        void *hot_kv, int32_t *host_rows_out,
+                                        void *workspace, size_t workspace_bytes, lsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
  * Stage 5 -- native Lightning Indexer Top-k over the fetched entries (blog review sections

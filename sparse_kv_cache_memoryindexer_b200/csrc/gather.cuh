@@ -15,7 +15,7 @@ namespace lsa {
 constexpr int GATHER_ROWS_PER_WARP = 4;
 constexpr int GATHER_MAX_CHUNKS = 4;  // row_bytes <= 4 * 32 * 16 = 2048 per in-flight row
 #ifndef LSA_GATHER_LINK_CTAS
-#define LSA_GATHER_LINK_CTAS 32
+#define LSA_GATHER_LINK_CTAS 128
 #endif
 constexpr int GATHER_LINK_CTAS = LSA_GATHER_LINK_CTAS;  // CTAs of the rows-only launch (128 threads each)
 constexpr int GATHER_ROWS_MAX_B = 8192; // sequences of the rows-only launch (shared prefix of B + 1 ints)
@@ -258,6 +258,148 @@ __global__ void __launch_bounds__(128) k_gather_rows(const int32_t *__restrict__
             for (int c = 0; c < CH; c++) {
                 const int ch = lane + 32 * c;
                 if (src[r] >= 0 && ch < row16) *(uint4 *)(hot_kv + dst[r] * rb + (int64_t)ch * 16) = v[r][c];
+            }
+    }
+}
+
+// ------------------------------------------------------------------ incremental fetch
+// The hot buffer of the previous window (rows of C_{t-tau}, at that window's offsets) stays
+// resident; the new window's buffer gets the rows of C_t: rows in both sets by a device copy, only
+// C_t \ C_{t-tau} over the host link.  Sequences keep their entry numbering between windows (they
+// may grow).  Three launches, all over the new fetched rows numbered in one range:
+//   k_incr_map    one thread per row: look the entry up in the previous (ascending) list of its
+//                 sequence; map[slot] = previous slot, or -1 and the row number appended to miss[]
+//   k_incr_copy   one thread per 16-byte chunk of every row with a previous slot (device copy)
+//   k_incr_fetch  the link launch over miss[0 .. *nmiss): as k_gather_rows
+// A previous list that is not ascending only costs host reads (a missed lookup fetches the row).
+
+__device__ __forceinline__ int prev_count_clamped(const int32_t *pcount, const int64_t *poffs, int b)
+{
+    const int64_t pS = poffs[b + 1] - poffs[b];
+    int F = pcount[b];
+    if (F < 0 || F > pS) {
+        flag(ERRF_COUNT);
+        F = F < 0 ? 0 : (int)pS;
+    }
+    return F;
+}
+
+__global__ void __launch_bounds__(128) k_incr_map(const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+                                                  const int64_t *__restrict__ offs, int B,
+                                                  const int32_t *__restrict__ pidx, const int32_t *__restrict__ pcount,
+                                                  const int64_t *__restrict__ poffs, int32_t *__restrict__ map,
+                                                  int32_t *__restrict__ miss, int *__restrict__ nmiss)
+{
+    extern __shared__ int pre[];
+    __shared__ int warp_sum[4];
+    const int total = block_count_prefix(count, offs, B, pre, warp_sum);
+    const int lane = threadIdx.x & 31;
+    // every thread of a warp runs the same number of iterations (the ballot below needs them all)
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); g0 < total; g0 += stride) {
+        const int64_t g = g0 + lane;
+        bool missed = false;
+        if (g < total) {
+            const int b = sequence_of_row(pre, B, g);
+            const int64_t off = offs[b], S = offs[b + 1] - off, j = g - pre[b];
+            const int s = __ldg(idx + off + j);
+            int slot = -1;
+            if (s < 0 || s >= S) {
+                flag(ERRF_INDEX);
+            } else {
+                const int64_t poff = poffs[b];
+                int lo = 0, hi = prev_count_clamped(pcount, poffs, b);  // lower bound of s in the previous list
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (__ldg(pidx + poff + mid) < s) lo = mid + 1;
+                    else hi = mid;
+                }
+                const int pc = prev_count_clamped(pcount, poffs, b);
+                if (lo < pc && __ldg(pidx + poff + lo) == s) slot = lo;
+                else missed = true;
+            }
+            map[off + j] = slot;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, missed);
+        int base = 0;
+        if (lane == 0 && bal) base = atomicAdd(nmiss, __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (missed) miss[base + __popc(bal & ((1u << lane) - 1))] = (int32_t)g;
+    }
+}
+
+__global__ void __launch_bounds__(128) k_incr_copy(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
+                                                   int B, const int64_t *__restrict__ poffs,
+                                                   const int32_t *__restrict__ map, const uint8_t *__restrict__ prev_hot,
+                                                   int row16, uint8_t *__restrict__ hot)
+{
+    extern __shared__ int pre[];
+    __shared__ int warp_sum[4];
+    const int total = block_count_prefix(count, offs, B, pre, warp_sum);
+    const int64_t rb = (int64_t)row16 * 16;
+    const int64_t units = (int64_t)total * row16;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t g = u / row16;
+        const int ch = (int)(u - g * row16);
+        const int b = sequence_of_row(pre, B, g);
+        const int64_t slot = offs[b] + (g - pre[b]);
+        const int m = map[slot];
+        if (m < 0) continue;
+        const uint4 v = __ldg((const uint4 *)(prev_hot + (poffs[b] + m) * rb + (int64_t)ch * 16));
+        *(uint4 *)(hot + slot * rb + (int64_t)ch * 16) = v;
+    }
+}
+
+template <int CH>
+__global__ void __launch_bounds__(128) k_incr_fetch(const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+                                                    const int64_t *__restrict__ offs, int B,
+                                                    const int32_t *__restrict__ miss, const int *__restrict__ nmiss,
+                                                    const uint8_t *__restrict__ pool, int row16, uint8_t *__restrict__ hot,
+                                                    int32_t *__restrict__ host_rows)
+{
+    extern __shared__ int pre[];
+    __shared__ int warp_sum[4];
+    const int total = block_count_prefix(count, offs, B, pre, warp_sum);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int n = *nmiss;
+    n = n < 0 ? 0 : (n > total ? total : n);
+    if (host_rows && blockIdx.x == 0 && threadIdx.x == 0) *host_rows = n;
+    const int64_t rb = (int64_t)row16 * 16;
+    const int64_t wstride = (int64_t)gridDim.x * 4;
+    for (int64_t i0 = ((int64_t)blockIdx.x * 4 + warp) * GATHER_ROWS_PER_WARP; i0 < n;
+         i0 += wstride * GATHER_ROWS_PER_WARP) {
+        int64_t src[GATHER_ROWS_PER_WARP], dst[GATHER_ROWS_PER_WARP];
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++) {
+            src[r] = -1;
+            dst[r] = 0;
+            if (i0 + r < n) {
+                const int64_t g = miss[i0 + r];
+                if (g >= 0 && g < total) {
+                    const int b = sequence_of_row(pre, B, g);
+                    const int64_t off = offs[b], S = offs[b + 1] - off, j = g - pre[b];
+                    const int s = __ldg(idx + off + j);
+                    if (s >= 0 && s < S) {
+                        src[r] = off + s;
+                        dst[r] = off + j;
+                    }
+                }
+            }
+        }
+        uint4 v[GATHER_ROWS_PER_WARP][CH];
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++)
+#pragma unroll
+            for (int c = 0; c < CH; c++) {
+                const int ch = lane + 32 * c;
+                if (src[r] >= 0 && ch < row16) v[r][c] = ld_stream16(pool + src[r] * rb + (int64_t)ch * 16);
+            }
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++)
+#pragma unroll
+            for (int c = 0; c < CH; c++) {
+                const int ch = lane + 32 * c;
+                if (src[r] >= 0 && ch < row16) *(uint4 *)(hot + dst[r] * rb + (int64_t)ch * 16) = v[r][c];
             }
     }
 }

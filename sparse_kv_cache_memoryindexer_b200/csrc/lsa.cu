@@ -402,6 +402,80 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
     return ok();
 }
 
+// ------------------------------------------------------------------------------ stage 4b, incremental
+
+// Workspace of lsa_fetch_gather_incremental: [map: total_S int32][miss: total_S int32][miss count].
+size_t lsa_fetch_incremental_workspace_size(int B, int64_t total_S)
+{
+    if (B <= 0 || total_S < 0) return 0;
+    return 2 * align_up(sizeof(int32_t) * (size_t)(total_S > 0 ? total_S : 1), 256) + 256;
+}
+
+lsa_status lsa_fetch_gather_incremental(const int32_t *idx, const int32_t *count, const int64_t *seq_offsets,
+                                        int64_t total_S, int B, const int32_t *prev_idx, const int32_t *prev_count,
+                                        const int64_t *prev_seq_offsets, int64_t prev_total_S,
+                                        const void *prev_hot_kv, const void *pool, size_t row_bytes, void *hot_kv,
+                                        int32_t *host_rows_out, void *workspace, size_t workspace_bytes,
+                                        lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(idx && count && seq_offsets && prev_idx && prev_count && prev_seq_offsets && prev_hot_kv && pool &&
+                    hot_kv,
+                "lsa_fetch_gather_incremental: null pointer");
+    LSA_REQUIRE(B > 0 && total_S >= 0 && prev_total_S >= 0, "lsa_fetch_gather_incremental: sizes must be positive");
+    LSA_REQUIRE(total_S < (int64_t)1 << 31, "lsa_fetch_gather_incremental: total_S must be below 2^31");
+    if (B > GATHER_ROWS_MAX_B)
+        return fail(LSA_ERR_UNSUPPORTED, "lsa_fetch_gather_incremental: at most %d sequences", GATHER_ROWS_MAX_B);
+    LSA_REQUIRE(row_bytes > 0 && row_bytes % 16 == 0 && row_bytes <= 16 * 32 * GATHER_MAX_CHUNKS,
+                "lsa_fetch_gather_incremental: row_bytes must be a multiple of 16, at most %d",
+                16 * 32 * GATHER_MAX_CHUNKS);
+    LSA_REQUIRE(aligned(pool, 16) && aligned(hot_kv, 16) && aligned(prev_hot_kv, 16),
+                "lsa_fetch_gather_incremental: row buffers must be 16-byte aligned");
+    {
+        const uintptr_t a0 = (uintptr_t)hot_kv, a1 = a0 + (uintptr_t)total_S * row_bytes;
+        const uintptr_t b0 = (uintptr_t)prev_hot_kv, b1 = b0 + (uintptr_t)prev_total_S * row_bytes;
+        LSA_REQUIRE(a1 <= b0 || b1 <= a0, "lsa_fetch_gather_incremental: hot_kv and prev_hot_kv overlap");
+    }
+    const size_t need = lsa_fetch_incremental_workspace_size(B, total_S);
+    if (!workspace || workspace_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "lsa_fetch_gather_incremental: workspace needs %zu bytes", need);
+    LSA_REQUIRE(aligned(workspace, 256), "lsa_fetch_gather_incremental: workspace must be 256-byte aligned");
+    void *dpool = nullptr;
+    cudaError_t e = cudaHostGetDevicePointer(&dpool, const_cast<void *>(pool), 0);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(LSA_ERR_INVALID_ARG, "lsa_fetch_gather_incremental: pool is not mapped page-locked host memory (%s)",
+                    cudaGetErrorString(e));
+    }
+    const size_t part = align_up(sizeof(int32_t) * (size_t)(total_S > 0 ? total_S : 1), 256);
+    int32_t *map = (int32_t *)workspace;
+    int32_t *miss = (int32_t *)((char *)workspace + part);
+    int *nmiss = (int *)((char *)workspace + 2 * part);
+    e = cudaMemsetAsync(nmiss, 0, sizeof(int), st);
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_fetch_gather_incremental: %s", cudaGetErrorString(e));
+    const size_t smem = sizeof(int) * (size_t)(B + 1);
+    const int row16 = (int)(row_bytes / 16);
+    const int sms = num_sms();
+    k_incr_map<<<sms * 4, 128, smem, st>>>(idx, count, seq_offsets, B, prev_idx, prev_count, prev_seq_offsets, map, miss,
+                                           nmiss);
+    LSA_TRY(launched("incremental fetch: lookup"));
+    k_incr_copy<<<sms * 8, 128, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
+                                            row16, (uint8_t *)hot_kv);
+    LSA_TRY(launched("incremental fetch: device copy"));
+    const uint8_t *src = (const uint8_t *)dpool;
+    if (row16 <= 32)
+        k_incr_fetch<1><<<GATHER_LINK_CTAS, 128, smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
+                                                             (uint8_t *)hot_kv, host_rows_out);
+    else if (row16 <= 64)
+        k_incr_fetch<2><<<GATHER_LINK_CTAS, 128, smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
+                                                             (uint8_t *)hot_kv, host_rows_out);
+    else
+        k_incr_fetch<4><<<GATHER_LINK_CTAS, 128, smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
+                                                             (uint8_t *)hot_kv, host_rows_out);
+    LSA_TRY(launched("incremental fetch: host rows"));
+    return ok();
+}
+
 // ------------------------------------------------------------------------------ stage 5
 
 // Workspace of lsa_lightning_topk: [item_start: B+1 ints, item counter: 1 int][Y: tau * total_S floats].

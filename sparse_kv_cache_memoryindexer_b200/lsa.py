@@ -26,7 +26,7 @@ EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_devic
            "lsa_project_workspace_size", "lsa_project",
            "lsa_score_select_workspace_size", "lsa_memindex_score_select",
            "lsa_memindex_score_select_static",
-           "lsa_fetch_gather",
+           "lsa_fetch_gather", "lsa_fetch_incremental_workspace_size", "lsa_fetch_gather_incremental",
            "lsa_lightning_topk_workspace_size", "lsa_lightning_topk",
            "lsa_pool_alloc", "lsa_pool_free")
 
@@ -54,6 +54,8 @@ def _load():
         "lsa_memindex_score_select": (I, [P, P, P, P, I, P, I64, I, I, I, I, F, P, P, P, P, P, SZ, P]),
         "lsa_memindex_score_select_static": (I, [P, P, P, P, I, P, I64, I, I, I, I, F, P, P, P, P, P]),
         "lsa_fetch_gather": (I, [P, P, P, I64, I, P, SZ, P, P, P, I, I, P, P, P]),
+        "lsa_fetch_incremental_workspace_size": (SZ, [I, I64]),
+        "lsa_fetch_gather_incremental": (I, [P, P, P, I64, I, P, P, P, I64, P, P, SZ, P, P, P, SZ, P]),
         "lsa_lightning_topk_workspace_size": (SZ, [I, I, I64, I]),
         "lsa_lightning_topk": (I, [P, P, P, P, I, P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P]),
         "lsa_pool_alloc": (I, [SZ, C.POINTER(C.c_void_p)]),
@@ -175,6 +177,27 @@ def lsa_fetch_gather(idx, count, seq_offsets, total_S, pool, hot_kv, K_sel=None,
     _check(_lib.lsa_fetch_gather(_p(idx), _p(count), _p(seq_offsets), int(total_S), B, _p(pool), row_bytes,
                                  _p(hot_kv), _p(K_sel), _p(k_scale_sel), kdt, d_I, _p(hot_K), _p(hot_scale),
                                  _stream(stream)))
+
+
+def lsa_fetch_incremental_workspace_size(B, total_S) -> int:
+    return int(_lib.lsa_fetch_incremental_workspace_size(B, total_S))
+
+
+def lsa_fetch_gather_incremental(idx, count, seq_offsets, total_S, prev_idx, prev_count, prev_seq_offsets,
+                                 prev_total_S, prev_hot_kv, pool, hot_kv, workspace, host_rows_out=None,
+                                 stream=None):
+    """The window's rows with the previous window's rows resident: common entries are copied on the
+    device, only the others cross the host link (see include/lsa.h)."""
+    _dev(idx, count, seq_offsets, prev_idx, prev_count, prev_seq_offsets, prev_hot_kv, hot_kv, workspace,
+         host_rows_out)
+    if pool.device.type != "cpu":
+        raise ValueError("the cold pool must be (mapped page-locked) host memory")
+    B = count.numel()
+    row_bytes = pool.shape[1] * pool.element_size()
+    _check(_lib.lsa_fetch_gather_incremental(
+        _p(idx), _p(count), _p(seq_offsets), int(total_S), B, _p(prev_idx), _p(prev_count), _p(prev_seq_offsets),
+        int(prev_total_S), _p(prev_hot_kv), _p(pool), row_bytes, _p(hot_kv), _p(host_rows_out), _p(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 # ------------------------------------------------------------------------ stage 5

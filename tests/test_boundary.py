@@ -62,6 +62,28 @@ def test_host_side_validation_without_gpu():
     assert b"workspace needs" in lib.lsa_last_error()
 
 
+def test_incremental_fetch_host_validation_without_gpu():
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    lib = lsa.library()
+    p = C.c_void_p(4096)
+    args = dict(idx=p, count=p, offs=p, T=100, B=2, pidx=p, pcount=p, poffs=p, pT=100, phot=p, pool=p, rb=1024,
+                hot=p, host_rows=None, ws=p, wsb=1 << 20, st=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.lsa_fetch_gather_incremental(a["idx"], a["count"], a["offs"], a["T"], a["B"], a["pidx"],
+                                                a["pcount"], a["poffs"], a["pT"], a["phot"], a["pool"], a["rb"],
+                                                a["hot"], a["host_rows"], a["ws"], a["wsb"], a["st"])
+    assert call(prev_dummy=None, pidx=None) == 1 and b"null pointer" in lib.lsa_last_error()
+    assert call(rb=1000) == 1                                   # not a multiple of 16
+    # the two hot buffers overlap (rows 0..99 of each start 1 KB apart)
+    assert call(hot=C.c_void_p(1 << 20), phot=C.c_void_p((1 << 20) + 1024)) == 1
+    assert b"overlap" in lib.lsa_last_error()
+    # a workspace that is too small
+    assert call(hot=C.c_void_p(1 << 30), phot=C.c_void_p(1 << 20), wsb=16) == 5
+    assert lsa.lsa_fetch_incremental_workspace_size(2, 100) >= 2 * 100 * 4 + 4
+
+
 def test_workspace_sizes_cover_their_buffers():
     from sparse_kv_cache_memoryindexer_b200 import lsa
     import torch
