@@ -13,6 +13,7 @@ enum : int { DT_F32 = 0, DT_BF16 = 1, DT_FP8 = 2 };
 
 // Entries per score tile: one TMEM lane / one thread per entry.
 constexpr int TILE = 128;
+constexpr int COMPACT_TILES = 256;  // tiles per CTA of the compaction (one per thread)
 
 // Bits of the device error word (read and cleared by lsa_check_device).
 enum : unsigned {

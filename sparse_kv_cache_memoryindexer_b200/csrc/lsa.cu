@@ -77,10 +77,12 @@ int num_sms()
 }
 
 // Workspace layout of lsa_memindex_score_select:
-//   tile_start [B+1] int | tile_mask [max_tiles][4] u32 | qh [L*B*64][128] f16 | wh [L*B*64] fp32
-// (qh / wh: the f16 queries and scaled head weights of the E4M3 tensor-core path).
+//   tile_start [B+1] int, chunk_start [B+1] int | tile_mask [max_tiles][4] u32 |
+//   qh [L*B][128][128] E4M3 | wh [L*B*64] fp32
+// (qh / wh: the split queries and scaled head weights of the E4M3 tensor-core path).
 struct ScoreWs {
     int *tile_start;
+    int *chunk_start;
     uint32_t *tile_mask;
     void *qh;
     float *wh;
@@ -90,7 +92,7 @@ int64_t max_tiles(int B, int64_t T) { return T / TILE + B + 1; }
 
 size_t score_ws_parts(int L, int B, int64_t T, size_t part[4])
 {
-    part[0] = align_up(sizeof(int) * (size_t)(B + 1), 256);
+    part[0] = align_up(sizeof(int) * (size_t)(2 * B + 2), 256);  // tile starts, compaction chunk starts
     part[1] = align_up((size_t)max_tiles(B, T) * 16, 256);
     part[2] = align_up((size_t)L * B * 64 * 128 * 2, 256);
     part[3] = align_up((size_t)L * B * 64 * 4, 256);
@@ -110,6 +112,7 @@ ScoreWs score_ws(void *ws, int L, int B, int64_t T)
     char *p = (char *)ws;
     ScoreWs w;
     w.tile_start = (int *)p;
+    w.chunk_start = (int *)p + (B + 1);
     w.tile_mask = (uint32_t *)(p + part[0]);
     w.qh = (void *)(p + part[0] + part[1]);
     w.wh = (float *)(p + part[0] + part[1] + part[2]);
@@ -299,16 +302,18 @@ lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *
     const float thr_logit = (float)log((double)threshold / (1.0 - (double)threshold));
     ScoreWs ws = score_ws(workspace, L, B, total_S);
 
-    k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, ws.tile_start);
-    LSA_TRY(launched("tile setup"));
-
     const bool tc = (n_h == 64 && d_I == 128 && L <= tc::MAX_L_TC && (kdt == LSA_BF16 || kdt == LSA_FP8_E4M3) &&
                      tc_score_available());
+    if (tc) LSA_REQUIRE(aligned(q, 16) && aligned(K, 16), "lsa_memindex_score_select: q and K must be 16-byte aligned");
+    if (!(tc && kdt == LSA_FP8_E4M3)) {  // (the E4M3 tensor-core path does the setup in its query split)
+        k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, ws.tile_start, ws.chunk_start, count_out);
+        LSA_TRY(launched("tile setup"));
+    }
     if (tc) {
-        LSA_REQUIRE(aligned(q, 16) && aligned(K, 16), "lsa_memindex_score_select: q and K must be 16-byte aligned");
         int n = 0;
-        const lsa_status s = launch_score_tc(q, w, K, k_scale, kdt, seq_offsets, ws.tile_start, B, total_S, L,
-                                             thr_logit, scores_out, ws.tile_mask, ws.qh, ws.wh, num_sms(), st, &n);
+        const lsa_status s = launch_score_tc(q, w, K, k_scale, kdt, seq_offsets, ws.tile_start, ws.chunk_start,
+                                             count_out, B, total_S, L, thr_logit, scores_out, ws.tile_mask, ws.qh,
+                                             ws.wh, num_sms(), st, &n);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK) return fail(s, "lsa_memindex_score_select: tensor-core launch failed (%s)",
                                      cudaGetErrorString(cudaGetLastError()));
@@ -324,7 +329,9 @@ lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *
         default: return fail(LSA_ERR_UNSUPPORTED, "lsa_memindex_score_select: d_I must be 32, 64 or 128");
         }
     }
-    k_compact<<<B, 1024, 0, st>>>(ws.tile_mask, ws.tile_start, seq_offsets, B, idx_out, count_out, mask_out);
+    const int64_t chunks = (max_tiles(B, total_S) + COMPACT_TILES - 1) / COMPACT_TILES + B;
+    k_compact<<<(unsigned)chunks, COMPACT_TILES, 0, st>>>(ws.tile_mask, ws.tile_start, ws.chunk_start, seq_offsets, B,
+                                                        idx_out, count_out, mask_out);
     LSA_TRY(launched("compact"));
     return ok();
 }

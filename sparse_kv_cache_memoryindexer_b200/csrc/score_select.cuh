@@ -11,8 +11,10 @@
 namespace lsa {
 
 // tile_start[b] = sum_{b' < b} ceil(S_b' / TILE), b = 0..B.  One block; also validates offsets.
-__global__ void __launch_bounds__(1024) k_tile_setup(const int64_t *__restrict__ offs, int B, int64_t T,
-                                                     int *__restrict__ tile_start)
+// Run by every thread of one block (any size that is a multiple of 32).
+__device__ __forceinline__ void tile_setup_body(const int64_t *__restrict__ offs, int B, int64_t T,
+                                                int *__restrict__ tile_start, int *__restrict__ chunk_start,
+                                                int32_t *__restrict__ count_out)
 {
     __shared__ int warp_tot[32];
     __shared__ int carry;
@@ -22,6 +24,42 @@ __global__ void __launch_bounds__(1024) k_tile_setup(const int64_t *__restrict__
         if (offs[0] != 0 || offs[B] != T) flag(ERRF_OFFSETS);
     }
     __syncthreads();
+    // chunk_start: exclusive prefix of ceil(tiles_b / COMPACT_TILES), the compaction's CTAs per
+    // sequence; an empty sequence has none, so its count is written here.
+    {
+        __shared__ int wt[32];
+        __shared__ int ccarry;
+        if (threadIdx.x == 0) {
+            ccarry = 0;
+            chunk_start[0] = 0;
+        }
+        __syncthreads();
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        for (int base = 0; base < B; base += blockDim.x) {
+            const int b = base + threadIdx.x;
+            int n = 0;
+            if (b < B) {
+                int64_t S = offs[b + 1] - offs[b];
+                if (S < 0) S = 0;
+                if (S == 0) count_out[b] = 0;
+                const int64_t tiles = (S + TILE - 1) / TILE;
+                n = (int)((tiles + COMPACT_TILES - 1) / COMPACT_TILES);
+            }
+            int inc = warp_incl_scan(n);
+            if (lane == 31) wt[warp] = inc;
+            __syncthreads();
+            if (warp == 0) {
+                int v = lane < (int)(blockDim.x >> 5) ? wt[lane] : 0;
+                wt[lane] = warp_incl_scan(v) - v;
+            }
+            __syncthreads();
+            const int pos = ccarry + wt[warp] + inc;
+            if (b < B) chunk_start[b + 1] = pos;
+            __syncthreads();
+            if (threadIdx.x == blockDim.x - 1) ccarry = pos;
+            __syncthreads();
+        }
+    }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int base = 0; base < B; base += blockDim.x) {
         const int b = base + threadIdx.x;
@@ -48,6 +86,13 @@ __global__ void __launch_bounds__(1024) k_tile_setup(const int64_t *__restrict__
         if (threadIdx.x == blockDim.x - 1) carry = pos;
         __syncthreads();
     }
+}
+
+__global__ void __launch_bounds__(1024) k_tile_setup(const int64_t *__restrict__ offs, int B, int64_t T,
+                                                     int *__restrict__ tile_start, int *__restrict__ chunk_start,
+                                                     int32_t *__restrict__ count_out)
+{
+    tile_setup_body(offs, B, T, tile_start, chunk_start, count_out);
 }
 
 // SIMT index score (any dtype, d_I = D in {32, 64, 128}, n_h <= 128).  One thread per entry.
@@ -103,56 +148,77 @@ __global__ void __launch_bounds__(TILE) k_score_simt(const void *__restrict__ q,
 
 // Compaction (stage 4a): one block per sequence scans its tiles' fetch words in order and writes
 // the ascending list of fetched entries, the count, and optionally a byte mask.
-__global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ tile_mask,
-                                                  const int *__restrict__ tile_start,
-                                                  const int64_t *__restrict__ offs, int B,
-                                                  int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out,
-                                                  uint8_t *__restrict__ mask_out)
+// Stage 4a: the ascending list of fetched entries of each sequence from the fetch words.  One CTA
+// per chunk of COMPACT_TILES tiles of one sequence: its sequence-local start is the number of
+// fetched entries in the sequence's earlier tiles (summed from their fetch words, a few KB read
+// from L2), its tiles' starts come from a block scan, and each warp writes the entries of its 32
+// tiles with consecutive lanes on consecutive list positions.
+__device__ __forceinline__ int popc4(uint4 m) { return __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w); }
+
+__global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__restrict__ tile_mask,
+                                                          const int *__restrict__ tile_start,
+                                                          const int *__restrict__ chunk_start,
+                                                          const int64_t *__restrict__ offs, int B,
+                                                          int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out,
+                                                          uint8_t *__restrict__ mask_out)
 {
-    __shared__ int warp_tot[32];
-    __shared__ int carry;
-    const int b = blockIdx.x;
-    const int t0 = tile_start[b], t1 = tile_start[b + 1];
-    const int64_t off = offs[b], S = offs[b + 1] - offs[b];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) carry = 0;
-    __syncthreads();
-    for (int base = t0; base < t1; base += blockDim.x) {
-        const int t = base + threadIdx.x;
-        uint4 m = make_uint4(0, 0, 0, 0);
-        if (t < t1) m = *(const uint4 *)(tile_mask + (int64_t)t * 4);
-        const int c = __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
-        const int inc = warp_incl_scan(c);
-        if (lane == 31) warp_tot[warp] = inc;
-        __syncthreads();
-        if (warp == 0) {
-            int v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
-            warp_tot[lane] = warp_incl_scan(v) - v;
-        }
-        __syncthreads();
-        int pos = carry + warp_tot[warp] + inc - c;
-        if (t < t1) {
-            const int64_t s0 = (int64_t)(t - t0) * TILE;
-            const uint32_t words[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                uint32_t bits = words[k];
-                while (bits) {
-                    const int bit = __ffs(bits) - 1;
-                    bits &= bits - 1;
-                    idx_out[off + pos++] = (int32_t)(s0 + 32 * k + bit);
-                }
-            }
-            if (mask_out) {
-                for (int e = 0; e < TILE && s0 + e < S; e++)
-                    mask_out[off + s0 + e] = (uint8_t)((words[e >> 5] >> (e & 31)) & 1u);
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) carry = pos;  // last thread's running end = block total
-        __syncthreads();
+    __shared__ int red[COMPACT_TILES / 32];
+    __shared__ int scan[COMPACT_TILES / 32];
+    const int c = blockIdx.x;
+    if (c >= chunk_start[B]) return;
+    int lo = 0, hi = B - 1;  // the sequence of chunk c: largest b with chunk_start[b] <= c
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_start[mid] <= c) lo = mid;
+        else hi = mid - 1;
     }
-    if (threadIdx.x == 0) count_out[b] = carry;
+    const int b = lo;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t0 = tile_start[b], t1 = tile_start[b + 1];
+    const int ci = c - chunk_start[b];
+    const int ct0 = t0 + ci * COMPACT_TILES, ct1 = min(t1, ct0 + COMPACT_TILES);
+    const int64_t off = offs[b], S = offs[b + 1] - off;
+    // fetched entries before this chunk
+    int part = 0;
+    for (int t = t0 + threadIdx.x; t < ct0; t += COMPACT_TILES) part += popc4(*(const uint4 *)(tile_mask + (int64_t)t * 4));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) red[warp] = part;
+    // this chunk: one tile per thread
+    const int t = ct0 + threadIdx.x;
+    uint4 m = make_uint4(0, 0, 0, 0);
+    if (t < ct1) m = *(const uint4 *)(tile_mask + (int64_t)t * 4);
+    const int cnt = popc4(m);
+    const int inc = warp_incl_scan(cnt);
+    if (lane == 31) scan[warp] = inc;
+    __syncthreads();
+    int base = 0, before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < COMPACT_TILES / 32; w++) {
+        base += red[w];
+        before += w < warp ? scan[w] : 0;
+        total += scan[w];
+    }
+    const int pos = base + before + inc - cnt;  // list position of this tile's first entry
+    if (ct1 == t1 && threadIdx.x == 0) count_out[b] = base + total;
+    // coalesced writes: the warp walks its 32 tiles
+    for (int j = 0; j < 32; j++) {
+        const int tj = ct0 + warp * 32 + j;
+        if (tj >= ct1) break;
+        const uint32_t w0 = __shfl_sync(0xffffffffu, m.x, j), w1 = __shfl_sync(0xffffffffu, m.y, j);
+        const uint32_t w2 = __shfl_sync(0xffffffffu, m.z, j), w3 = __shfl_sync(0xffffffffu, m.w, j);
+        int p = __shfl_sync(0xffffffffu, pos, j);
+        const int64_t s0 = (int64_t)(tj - t0) * TILE;
+        const uint32_t below = (1u << lane) - 1u;
+        const uint32_t words[4] = {w0, w1, w2, w3};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const uint32_t wk = words[k];
+            if ((wk >> lane) & 1u) idx_out[off + p + __popc(wk & below)] = (int32_t)(s0 + 32 * k + lane);
+            p += __popc(wk);
+            if (mask_out && s0 + 32 * k + lane < S) mask_out[off + s0 + 32 * k + lane] = (uint8_t)((wk >> lane) & 1u);
+        }
+    }
 }
 
 }  // namespace lsa

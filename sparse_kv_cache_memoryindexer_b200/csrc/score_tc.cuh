@@ -62,12 +62,19 @@ __device__ __forceinline__ void mma_e4m3(uint32_t tmem_d, uint64_t a, uint64_t b
 }
 
 // Queries for the E4M3 MMA (see the header comment); one warp per head row (l, b, h), four
-// consecutive elements per lane.  q [R][128] bf16, w [R] fp32, R = L * B * 64 ->
+// consecutive elements per lane.  The last block of the launch does the tile setup of the select
+// instead (one launch less on the stage).  q [R][128] bf16, w [R] fp32, R = L * B * 64 ->
 // qs [(R/64)][128][128] E4M3 (rows 0..63 hi of heads 0..63, rows 64..127 lo), ws [R] fp32.
 __global__ void __launch_bounds__(256) k_q_split_e4m3(const __nv_bfloat16 *__restrict__ q,
                                                       const float *__restrict__ w, uint8_t *__restrict__ qs,
-                                                      float *__restrict__ ws, int R)
+                                                      float *__restrict__ ws, int R, const int64_t *__restrict__ offs,
+                                                      int B, int64_t T, int *__restrict__ tile_start,
+                                                      int *__restrict__ chunk_start, int32_t *__restrict__ count_out)
 {
+    if (blockIdx.x == gridDim.x - 1) {
+        tile_setup_body(offs, B, T, tile_start, chunk_start, count_out);
+        return;
+    }
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= R) return;
@@ -118,12 +125,34 @@ struct Params {
 };
 
 struct SeqTracker {
-    // Sequence b owning tile t, found by walking forward from the previous answer.
-    int b;
-    __device__ __forceinline__ int of(const int *tile_start, int B, int t)
+    // Sequence b owning tile t (t < tile_start[B]), found by walking forward from the previous
+    // answer.  The per-sequence values are loaded once per sequence and kept in registers:
+    // next = tile_start[b + 1], first = tile_start[b], off = offs[b], S = offs[b + 1] - offs[b].
+    // (Entry offsets fit in 32 bits: the total is below 2^31.)
+    int b = 0, next = -1, first = 0, off = 0, S = 0;
+    __device__ __forceinline__ int of(const int *tile_start, const int64_t *offs, int t)
     {
-        while (b + 1 <= B && __ldg(tile_start + b + 1) <= t) b++;
+        if (next < 0 || next <= t) {
+            if (next < 0) next = __ldg(tile_start + 1);  // b = 0
+            while (next <= t) next = __ldg(tile_start + (++b) + 1);
+            first = __ldg(tile_start + b);
+            off = (int)__ldg(offs + b);
+            S = (int)(__ldg(offs + b + 1) - __ldg(offs + b));
+        }
         return b;
+    }
+};
+
+// Stage (or accumulator slot) and phase of the successive jobs of one parity group.
+struct Ring {
+    int i = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int n)
+    {
+        if (++i == n) {
+            i = 0;
+            phase ^= 1;
+        }
     }
 };
 
@@ -218,7 +247,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&kmap) : "memory");
             if (m == 0) asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&qmap) : "memory");
         }
-        SeqTracker tr{0};
+        SeqTracker tr;
+        Ring ring;
         uint32_t quse = 0;
         int prev_b = -1;
         uint32_t last_phase[MAX_STAGES / 2];
@@ -226,7 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < MAX_STAGES / 2; i++) issued[i] = false;
         bool ok = true;
         for (int t = t_begin + (m == 0 ? 0 : 1); t < t_end && ok; t += (m == 0 ? 1 : 2)) {
-            const int b = tr.of(p.tile_start, B, t);
+            const int b = tr.of(p.tile_start, p.offs, t);
             if (m == 0 && b != prev_b) {
                 if (!mbar_wait_warp(qempty, (quse & 1) ^ 1, abort_flag)) { ok = false; break; }
                 quse++;
@@ -246,12 +276,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 prev_b = b;
             }
             if (((t - t_begin) & 1) != m) continue;
-            const int64_t row0 = __ldg(p.offs + b) + (int64_t)(t - __ldg(p.tile_start + b)) * TILE;
+            const int64_t row0 = tr.off + (int64_t)(t - tr.first) * TILE;
             for (int l = 0; l < L; l++) {
-                const int64_t k = (int64_t)((t - t_begin) >> 1) * L + l;  // job index within the group
-                const int ls = (int)(k % SP);
+                const int ls = ring.i;
                 const int stage = m * SP + ls;
-                const uint32_t phase = (uint32_t)((k / SP) & 1);
+                const uint32_t phase = ring.phase;
+                ring.next(SP);
                 if (!mbar_wait_warp(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
                 if (leader) {
                     mbar_expect_tx(full(stage), kbytes);
@@ -279,13 +309,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         // Both walk every tile to track sequences: at the last tile of a sequence each releases the
         // query slot, by a commit after its own MMAs of that sequence, or a plain arrive if none.
         const int m = warp == 1 ? 0 : 1;
-        SeqTracker tr{0};
+        SeqTracker tr;
+        Ring kring, aring;
         uint32_t quse = 0;
         int prev_b = -1;
         bool used_q = false;
         bool ok = true;
         for (int t = t_begin; t < t_end && ok; t++) {
-            const int b = tr.of(p.tile_start, B, t);
+            const int b = tr.of(p.tile_start, p.offs, t);
             if (b != prev_b) {
                 // every issuer waits for every sequence's query load in order (also for sequences it
                 // has no tile of), so that it is never two phases ahead of the query barrier
@@ -298,11 +329,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (mine) {
                 used_q = true;
                 for (int l = 0; l < L; l++) {
-                    const int64_t k = (int64_t)((t - t_begin) >> 1) * L + l;  // job index within the group
-                    const int stage = m * SP + (int)(k % SP);
-                    const int acc = m * AP + (int)(k % AP);
-                    if (!mbar_wait_warp(full(stage), (uint32_t)((k / SP) & 1), abort_flag)) { ok = false; break; }
-                    if (!mbar_wait_warp(tempty(acc), (uint32_t)(((k / AP) & 1) ^ 1), abort_flag)) { ok = false; break; }
+                    const int stage = m * SP + kring.i, acc = m * AP + aring.i;
+                    const uint32_t kphase = kring.phase, aphase = aring.phase;
+                    kring.next(SP);
+                    aring.next(AP);
+                    if (!mbar_wait_warp(full(stage), kphase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait_warp(tempty(acc), aphase ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_base = kraw + (uint32_t)stage * kbytes;
                     const uint32_t b_base = qbuf + (uint32_t)l * 16384;
@@ -327,7 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 if (!ok) break;
             }
-            const bool last_of_seq = (t + 1 == t_end) || (__ldg(p.tile_start + b + 1) <= t + 1);
+            const bool last_of_seq = (t + 1 == t_end) || (tr.next <= t + 1);
             if (last_of_seq) {
                 if (elect_one()) {
                     if (used_q) mma_commit(qempty);
@@ -341,17 +373,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
         const int parity = (warp - 2) >> 2;      // this warp takes the tiles t_begin + parity + 2i
         float *myw = sw + (size_t)(warp - 2) * L * NH;
-        SeqTracker tr{0}, trn{0};
+        SeqTracker tr, trn;
+        Ring aring;
         int prev_b = -1;
         bool ok = true;
         // E4M3 scales are per entry and layer: load them one tile ahead so that the global-load
         // latency overlaps the previous tile instead of stalling every job.
         float sc_nxt0 = 1.f, sc_nxt1 = 1.f, sc_nxt2 = 1.f;
         auto load_scales = [&](int tt) {
-            const int bb = trn.of(p.tile_start, B, tt);
-            const int64_t SS = __ldg(p.offs + bb + 1) - __ldg(p.offs + bb);
-            const int64_t ss = (int64_t)(tt - __ldg(p.tile_start + bb)) * TILE + quarter * 32 + lane;
-            const int64_t rr = __ldg(p.offs + bb) + ss;
+            trn.of(p.tile_start, p.offs, tt);
+            const int64_t SS = trn.S;
+            const int64_t ss = (int64_t)(tt - trn.first) * TILE + quarter * 32 + lane;
+            const int64_t rr = trn.off + ss;
             const bool in = ss < SS;
             sc_nxt0 = in ? __ldg(p.kscale + rr) : 1.f;
             sc_nxt1 = (in && L > 1) ? __ldg(p.kscale + T + rr) : 1.f;
@@ -359,7 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         };
         if (FP8 && t_begin + parity < t_end) load_scales(t_begin + parity);
         for (int t = t_begin + parity; t < t_end && ok; t += 2) {
-            const int b = tr.of(p.tile_start, B, t);
+            const int b = tr.of(p.tile_start, p.offs, t);
             if (b != prev_b) {
                 __syncwarp();
                 for (int i = lane; i < L * NH; i += 32) {
@@ -371,16 +404,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             const float sc0 = sc_nxt0, sc1 = sc_nxt1, sc2 = sc_nxt2;
             if (FP8 && t + 2 < t_end) load_scales(t + 2);
-            const int64_t S = __ldg(p.offs + b + 1) - __ldg(p.offs + b);
-            const int64_t s = (int64_t)(t - __ldg(p.tile_start + b)) * TILE + quarter * 32 + lane;
+            const int64_t S = tr.S;
+            const int64_t s = (int64_t)(t - tr.first) * TILE + quarter * 32 + lane;
             const bool valid = s < S;
-            const int64_t row = __ldg(p.offs + b) + s;
+            const int64_t row = tr.off + s;
             bool fetched = false;
 #pragma unroll 1
             for (int l = 0; l < L; l++) {
-                const int64_t k = (int64_t)((t - t_begin) >> 1) * L + l;  // job index within the group
-                const int acc = parity * AP + (int)(k % AP);
-                const uint32_t accphase = (uint32_t)((k / AP) & 1);
+                const int acc = parity * AP + aring.i;
+                const uint32_t accphase = aring.phase;
+                aring.next(AP);
                 if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ncol);
@@ -446,10 +479,12 @@ inline bool tc_score_available() { return tc_available(); }
 
 // qs_ws / ws_ws: workspace for the split E4M3 queries and the scaled head weights of the E4M3
 // path ([L*B][128][128] bytes and [L*B*64] fp32).  *launches counts the kernels started.
+// For E4M3 keys the query split also runs the tile setup (chunk_start, count_out: see k_tile_setup);
+// for bf16 keys the caller has run k_tile_setup before.
 inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, const float *kscale, int kdt,
-                                  const int64_t *offs, const int *tile_start, int B, int64_t T, int L,
-                                  float thr, float *scores_out, uint32_t *tile_mask, void *qs_ws, float *ws_ws,
-                                  int sms, cudaStream_t st, int *launches)
+                                  const int64_t *offs, int *tile_start, int *chunk_start, int32_t *count_out, int B,
+                                  int64_t T, int L, float thr, float *scores_out, uint32_t *tile_mask, void *qs_ws,
+                                  float *ws_ws, int sms, cudaStream_t st, int *launches)
 {
     using namespace tc;
     *launches = 0;
@@ -457,7 +492,8 @@ inline lsa_status launch_score_tc(const void *q, const float *w, const void *K, 
     const bool fp8 = (kdt == DT_FP8);
     if (fp8) {
         const int R = L * B * NH;
-        k_q_split_e4m3<<<(R + 7) / 8, 256, 0, st>>>((const __nv_bfloat16 *)q, w, (uint8_t *)qs_ws, ws_ws, R);
+        k_q_split_e4m3<<<(R + 7) / 8 + 1, 256, 0, st>>>((const __nv_bfloat16 *)q, w, (uint8_t *)qs_ws, ws_ws, R, offs, B, T,
+                                                        tile_start, chunk_start, count_out);
         (*launches)++;
         q = qs_ws;
         w = ws_ws;
