@@ -47,6 +47,7 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-incremental", action="store_true", help="skip the incremental-fetch measurement")
+    p.add_argument("--no-decode-steps", action="store_true", help="skip the per-step decode measurement")
     return p.parse_args()
 
 
@@ -241,6 +242,54 @@ def h2d_bandwidth(device, nbytes=1 << 30):
 
 # ------------------------------------------------------------------------------------ lsa arm
 
+def measure_decode_steps(lsa, path, wl, offs, qd, wd, st, reps=3):
+    """S5 per decode step: tau calls of lsa_lightning_topk_step (one query per sequence each, over
+    the fetched entries plus the entries compressed so far in the window: one per 4 steps), eager
+    and replayed from a CUDA graph, beside the batched call for all tau queries, each timed alone."""
+    tau, B, k, T = wl.tau, wl.B, wl.k, wl.total_S
+    W = max(1, tau // 4)
+    dev = offs.device
+    g = torch.Generator(device="cpu").manual_seed(wl.seed + 23)
+    winK = (torch.randn((B, W, wl.d_I), generator=g) * 0.05).to(torch.bfloat16 if wl.kdtype != "f32" else
+                                                                   torch.float32).to(dev)
+    wcs = torch.tensor([[min(W, i // 4)] * B for i in range(tau)], dtype=torch.int32, device=dev)
+    ti = torch.empty((tau, B, k), dtype=torch.int32, device=dev)
+    ts = torch.empty((tau, B, k), dtype=torch.float32, device=dev)
+    ws = torch.empty(lsa.lsa_lightning_topk_step_workspace_size(B, T, wl.n_h, wl.d_I, W), dtype=torch.uint8, device=dev)
+
+    def steps():
+        for i in range(tau):
+            lsa.lsa_lightning_topk_step(qd[:, i], wd[:, i], path.hot_K, path.hot_scale, path.idx, path.count, offs, T, k,
+                                        ti[i], ws, win_K=winK, win_count=wcs[i], topk_score=ts[i])
+
+    cs = torch.cuda.Stream(device=dev)  # graphs are not captured on the default stream
+    cs.wait_stream(st)
+
+    def timed(fn):
+        fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(cs)
+        for _ in range(reps):
+            fn()
+        b.record(cs)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    with torch.cuda.stream(cs):
+        eager = timed(steps)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cs):
+            steps()
+        replay = timed(graph.replay)
+        batched = timed(lambda: path.topk(qd, wd, offs, cs))
+    torch.cuda.synchronize()
+    lsa.lsa_check_device(st)
+    del graph
+    return {"steps": tau, "window_entries_per_sequence": W, "eager_ms_per_step": eager / tau,
+            "graph_ms_per_step": replay / tau, "graph_ms_per_window": replay, "batched_ms_per_window": batched,
+            "note": "S5 per decode step over the fetched entries plus one new entry per 4 steps; timed alone"}
+
+
 def drifted_lists(idx, cnt, offs, drift, seed):
     """The next window's fetch lists: each sequence keeps 1 - drift of its entries and replaces the
     rest by entries it did not fetch (so the count stays about the same); ascending."""
@@ -396,6 +445,9 @@ def run_lsa(args, rank, world, device):
     incr = None
     if not args.no_incremental and world == 1:
         incr = measure_incremental(lsa, path, wl, offs, pool, st)
+    steps = None
+    if not args.no_decode_steps and world == 1:
+        steps = measure_decode_steps(lsa, path, wl, offs, qd, wd, st)
 
     result = None
     if rank == 0:
@@ -450,6 +502,7 @@ def run_lsa(args, rank, world, device):
             "clocks": clk,
             "e2e": e2e,
             "incremental_fetch": None if incr is None else dict(incr, full_fetch_ms=stage_ms[4]),
+            "decode_steps": steps,
         }
     pool.free()
     return result

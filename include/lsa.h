@@ -241,6 +241,41 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
                               void *workspace, size_t workspace_bytes, lsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Stage 5 for one decode step -- the decode-time form of the native Lightning Indexer Top-k
+ * (blog review sections 2.2 and 3.2): at step i of the window every sequence has one query, and
+ * its candidates are the entries fetched at the trigger plus the entries compressed since then
+ * (they are in device memory, not in the cold pool; the pages leave their handling open).
+ *     y_{b,j} as in lsa_lightning_topk for the fetched slots j < count[b], and
+ *     y_{b,count[b]+j} = sum_h w_{b,h} ReLU(win_scale_{b,j} q_{b,h} . win_K_{b,j})   for j < win_count[b]
+ * Top-k as in lsa_lightning_topk; a window entry j is reported as entry number S_b + j (entries
+ * keep counting after the sequence's S_b), so ties still go to the smaller entry number.
+ *   q_step, q_batch_stride    query of each sequence: element (b, h, e) at b*q_batch_stride +
+ *                             h*d_I + e (bf16, or fp32 for LSA_F32 keys); a column of
+ *                             lsa_lightning_topk's q_dec [B][tau][n_h][d_I] works directly
+ *   w_step, w_batch_stride    fp32 head weights, (b, h) at b*w_batch_stride + h
+ *   hot_K, hot_scale, kdt, idx, count, seq_offsets, total_S   as lsa_lightning_topk
+ *   win_K      [B][W][d_I] device, in the hot-key type (bf16 for LSA_BF16 and LSA_FP8_E4M3
+ *              keys, fp32 for LSA_F32); win_scale [B][W] fp32 (nullable: scale 1)
+ *   win_count  [B] device int32: window entries visible at this step (0 .. W)
+ *   topk_idx [B][k] int32, topk_score [B][k] fp32 (nullable)
+ * Workspace: lsa_lightning_topk_step_workspace_size.  The call allocates nothing and launches
+ * only kernels, so the tau steps of a window can be recorded once in a CUDA graph and replayed.
+ * The method has no separate per-step call: this is the second widening beyond one window.
+ * ---------------------------------------------------------------------------------------- */
+size_t lsa_lightning_topk_step_workspace_size(int B, int64_t total_S, int n_h, int d_I, int W);
+
+lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride,
+                                   const float *w_step, int64_t w_batch_stride,
+                                   const void *hot_K, const float *hot_scale, lsa_dtype kdt,
+                                   const int32_t *idx, const int32_t *count,
+                                   const int64_t *seq_offsets, int64_t total_S,
+                                   const void *win_K, const float *win_scale,
+                                   const int32_t *win_count, int W,
+                                   int B, int n_h, int d_I, int k,
+                                   int32_t *topk_idx, float *topk_score,
+                                   void *workspace, size_t workspace_bytes, lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Cold-pool helpers: page-locked host memory mapped into every device's address space
  * (cudaHostAlloc with the Mapped and Portable flags).  The pointer is valid on the host and,
  * unchanged, in kernels.  lsa_pool_free releases memory from lsa_pool_alloc only.

@@ -534,10 +534,104 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     int kpow2 = 1;
     while (kpow2 < k) kpow2 <<= 1;
     const size_t smem = sizeof(unsigned long long) * (size_t)kpow2;
-    LSA_TRY(set_smem(k_topk_select, smem));
-    k_topk_select<<<(unsigned)((int64_t)B * tau), SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, tau, k, kpow2,
+    LSA_TRY(set_smem(k_topk_select<false>, smem));
+    k_topk_select<false><<<(unsigned)((int64_t)B * tau), SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, tau, k, kpow2,
                                                                          topk_idx, topk_score);
     LSA_TRY(launched("top-k select"));
+    return ok();
+}
+
+// ------------------------------------------------------------------------------ stage 5, one decode step
+
+// Workspace of lsa_lightning_topk_step: [item_start B+1, counter][Y: 4 * total_S][tail: B * W]
+// [queries: B * 4 * n_h * d_I (4-byte elements)][weights: B * 4 * n_h].
+static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[5])
+{
+    part[0] = align_up(sizeof(int) * (size_t)(B + 2), 256);
+    part[1] = align_up(sizeof(float) * 4 * (size_t)(total_S > 0 ? total_S : 1), 256);
+    part[2] = align_up(sizeof(float) * (size_t)B * (W > 0 ? W : 1), 256);
+    part[3] = align_up((size_t)4 * B * 4 * n_h * d_I, 256);
+    part[4] = align_up(sizeof(float) * (size_t)B * 4 * n_h, 256);
+    return part[0] + part[1] + part[2] + part[3] + part[4];
+}
+
+size_t lsa_lightning_topk_step_workspace_size(int B, int64_t total_S, int n_h, int d_I, int W)
+{
+    if (B <= 0 || total_S < 0 || n_h <= 0 || d_I <= 0 || W < 0) return 0;
+    size_t part[5];
+    return step_ws_parts(B, total_S, n_h, d_I, W, part);
+}
+
+lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, const float *w_step,
+                                   int64_t w_batch_stride, const void *hot_K, const float *hot_scale, lsa_dtype kdt,
+                                   const int32_t *idx, const int32_t *count, const int64_t *seq_offsets,
+                                   int64_t total_S, const void *win_K, const float *win_scale,
+                                   const int32_t *win_count, int W, int B, int n_h, int d_I, int k,
+                                   int32_t *topk_idx, float *topk_score, void *workspace, size_t workspace_bytes,
+                                   lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(q_step && w_step && hot_K && idx && count && seq_offsets && topk_idx,
+                "lsa_lightning_topk_step: null pointer");
+    LSA_REQUIRE(B > 0 && n_h > 0 && d_I > 0 && total_S >= 0 && W >= 0, "lsa_lightning_topk_step: sizes must be positive");
+    LSA_REQUIRE(W == 0 || (win_K && win_count), "lsa_lightning_topk_step: W > 0 needs win_K and win_count");
+    LSA_REQUIRE(q_batch_stride >= (int64_t)n_h * d_I && w_batch_stride >= n_h,
+                "lsa_lightning_topk_step: batch strides below one query");
+    LSA_REQUIRE(k >= 1 && k <= LSA_MAX_TOPK, "lsa_lightning_topk_step: k must be in [1, %d]", LSA_MAX_TOPK);
+    LSA_REQUIRE(total_S < (int64_t)1 << 31, "lsa_lightning_topk_step: total_S must be below 2^31");
+    if (!valid_dtype(kdt)) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk_step: unknown key dtype");
+    LSA_REQUIRE((kdt == LSA_FP8_E4M3) == (hot_scale != nullptr),
+                "lsa_lightning_topk_step: hot_scale is required for FP8 keys and must be NULL otherwise");
+    if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk_step: n_h must be <= 128");
+    if (d_I != 32 && d_I != 64 && d_I != 128)
+        return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk_step: d_I must be 32, 64 or 128");
+    size_t part[5];
+    const size_t need = step_ws_parts(B, total_S, n_h, d_I, W, part);
+    if (!workspace || workspace_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "lsa_lightning_topk_step: workspace needs %zu bytes", need);
+    LSA_REQUIRE(aligned(workspace, 256), "lsa_lightning_topk_step: workspace must be 256-byte aligned");
+    char *p = (char *)workspace;
+    int *item_start = (int *)p;
+    int *item_counter = item_start + B + 1;
+    float *Y = (float *)(p + part[0]);
+    float *tail = (float *)(p + part[0] + part[1]);
+    void *qw = (void *)(p + part[0] + part[1] + part[2]);
+    float *ww = (float *)(p + part[0] + part[1] + part[2] + part[3]);
+    const int hdt = (kdt == LSA_FP8_E4M3) ? DT_BF16 : kdt;  // hot keys: E4M3 arrives decoded to bf16
+    const bool tc = li_tc_supported(n_h, d_I, 4, kdt);
+    const int TQ = tc ? 4 : 1;
+    const int64_t rows = (int64_t)B * TQ * n_h;
+    k_step_prep<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(q_step, q_batch_stride, w_step, w_batch_stride, hdt, B, TQ,
+                                                            n_h, d_I, qw, ww);
+    LSA_TRY(launched("decode step: queries"));
+    if (tc) {
+        LSA_REQUIRE(aligned(hot_K, 16), "lsa_lightning_topk_step: hot_K must be 16-byte aligned");
+        int n = 0;
+        const lsa_status s = launch_li_tc(qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, TQ, Y, item_start,
+                                          item_counter, num_sms(), st, &n);
+        g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
+        if (s != LSA_OK)
+            return fail(s, "lsa_lightning_topk_step: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
+    } else {
+        switch (d_I) {
+        case 32: LSA_TRY(li_simt_d<32>(hdt, qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, 1, n_h, Y, st)); break;
+        case 64: LSA_TRY(li_simt_d<64>(hdt, qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, 1, n_h, Y, st)); break;
+        default: LSA_TRY(li_simt_d<128>(hdt, qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, 1, n_h, Y, st)); break;
+        }
+    }
+    if (W > 0) {
+        const int64_t warps = (int64_t)B * W;
+        k_li_window<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(qw, ww, TQ, hdt, win_K, win_scale, win_count, B, W,
+                                                                 n_h, d_I, tail);
+        LSA_TRY(launched("decode step: window entries"));
+    }
+    int kpow2 = 1;
+    while (kpow2 < k) kpow2 <<= 1;
+    const size_t smem = sizeof(unsigned long long) * (size_t)kpow2;
+    LSA_TRY(set_smem(k_topk_select<true>, smem));
+    k_topk_select<true><<<(unsigned)B, SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, 1, k, kpow2, topk_idx,
+                                                               topk_score, tail, W > 0 ? win_count : nullptr, W, TQ);
+    LSA_TRY(launched("decode step: select"));
     return ok();
 }
 

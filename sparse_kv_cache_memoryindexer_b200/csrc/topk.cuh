@@ -82,12 +82,19 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total)
 }
 
 // One block per (sequence, query).  kpow2 = next power of two >= k (shared: kpow2 x 8 bytes).
+// TAIL: after the F fetched slots of sequence b come tail_count[b] (at most W) more candidates,
+// the entries compressed during the window (scores tail[b*W + j], entry numbers S_b + j); the Y rows
+// then have tau_y queries per sequence of which block (b, i) reads query i.
+template <bool TAIL>
 __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__restrict__ Y,
                                                              const int32_t *__restrict__ idx,
                                                              const int32_t *__restrict__ count,
                                                              const int64_t *__restrict__ offs, int tau, int k,
                                                              int kpow2, int32_t *__restrict__ topk_idx,
-                                                             float *__restrict__ topk_score)
+                                                             float *__restrict__ topk_score,
+                                                             const float *__restrict__ tail = nullptr,
+                                                             const int32_t *__restrict__ tail_count = nullptr,
+                                                             int W = 0, int tau_y = 0)
 {
     extern __shared__ unsigned long long sel[];  // (key << 32) | ~slot
     __shared__ unsigned int hist[256];
@@ -97,16 +104,24 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
 
     const int b = blockIdx.x / tau, i = blockIdx.x % tau;
     const int64_t off = offs[b], S = offs[b + 1] - offs[b];
-    int F = count[b];
-    F = F < 0 ? 0 : (F > S ? (int)S : F);
-    const float *row = Y + (int64_t)tau * off + (int64_t)i * S;
+    int F0 = count[b];
+    F0 = F0 < 0 ? 0 : (F0 > S ? (int)S : F0);
+    const float *row = Y + (int64_t)(TAIL ? tau_y : tau) * off + (int64_t)i * S;
+    int nt = 0;
+    if (TAIL && tail_count) {
+        nt = tail_count[b];
+        nt = nt < 0 ? 0 : (nt > W ? W : nt);
+    }
+    const float *trow = TAIL ? tail + (int64_t)b * W : nullptr;
+    const int F = F0 + nt;  // candidates
+    auto cand = [&](int j) { return (!TAIL || j < F0) ? row[j] : trow[j - F0]; };
 
     for (int t = threadIdx.x; t < kpow2; t += SEL_THREADS) sel[t] = 0ull;
     __syncthreads();
 
     if (F <= k) {
         for (int j = threadIdx.x; j < F; j += SEL_THREADS)
-            sel[j] = ((unsigned long long)float_to_ordered(row[j]) << 32) | (uint32_t)(~(uint32_t)j);
+            sel[j] = ((unsigned long long)float_to_ordered(cand(j)) << 32) | (uint32_t)(~(uint32_t)j);
     } else {
         uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
         for (int pass = 0; pass < 4; pass++) {
@@ -114,7 +129,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
             for (int t = threadIdx.x; t < 256; t += SEL_THREADS) hist[t] = 0;
             __syncthreads();
             for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
-                const uint32_t u = float_to_ordered(row[j]);
+                const uint32_t u = float_to_ordered(cand(j));
                 if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
             }
             __syncthreads();
@@ -145,7 +160,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
             uint32_t u = 0;
             int gt = 0, eq = 0;
             if (j < F) {
-                u = float_to_ordered(row[j]);
+                u = float_to_ordered(cand(j));
                 gt = u > prefix;
                 eq = u == prefix;
             }
@@ -182,13 +197,78 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
         if (r < nsel) {
             const unsigned long long v = sel[r];
             const uint32_t j = ~(uint32_t)(v & 0xffffffffull);
-            topk_idx[o0 + r] = __ldg(idx + off + j);
+            topk_idx[o0 + r] = ((int)j < F0) ? __ldg(idx + off + j) : (int32_t)(S + (j - F0));
             if (topk_score) topk_score[o0 + r] = ordered_to_float((uint32_t)(v >> 32));
         } else {
             topk_idx[o0 + r] = -1;
             if (topk_score) topk_score[o0 + r] = -INFINITY;
         }
     }
+}
+
+// ------------------------------------------------------------------ one decode step
+// Stage 5 for one decode step: each sequence's query of the step is copied into TQ query slots
+// (slot 0; the others are zero, as are their weights) so that the scorers built for groups of
+// queries serve the step unchanged.  qs / ws are the step's queries and weights with a batch
+// stride (elements) between sequences.
+__global__ void __launch_bounds__(256) k_step_prep(const void *__restrict__ qs, int64_t q_bstride,
+                                                   const float *__restrict__ ws, int64_t w_bstride, int dt, int B,
+                                                   int TQ, int n_h, int d_I, void *__restrict__ q_out,
+                                                   float *__restrict__ w_out)
+{
+    const int64_t rows = (int64_t)B * TQ * n_h;
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    const int h = (int)(r % n_h);
+    const int qi = (int)((r / n_h) % TQ);
+    const int b = (int)(r / ((int64_t)n_h * TQ));
+    const size_t es = dt == DT_F32 ? 4 : 2;
+    uint8_t *dst = (uint8_t *)q_out + (size_t)r * d_I * es;
+    const uint8_t *src = (const uint8_t *)qs + ((size_t)b * q_bstride + (size_t)h * d_I) * es;
+    for (int e = lane; e < d_I; e += 32) {
+        if (es == 4) ((float *)dst)[e] = qi == 0 ? ((const float *)src)[e] : 0.f;
+        else ((uint16_t *)dst)[e] = qi == 0 ? ((const uint16_t *)src)[e] : (uint16_t)0;
+    }
+    if (lane == 0) w_out[r] = qi == 0 ? ws[(size_t)b * w_bstride + h] : 0.f;
+}
+
+// Scores of the entries compressed during the window: one warp per (sequence, entry j < W);
+// y = sum_h w_h ReLU(scale_j q_h . k_j).  Keys [B][W][d_I] in the hot-key type, scales nullable.
+__global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, const float *__restrict__ w,
+                                                   int TQ, int dt, const void *__restrict__ winK,
+                                                   const float *__restrict__ winsc,
+                                                   const int32_t *__restrict__ win_count, int B, int W, int n_h,
+                                                   int d_I, float *__restrict__ tail)
+{
+    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (gw >= (int64_t)B * W) return;
+    const int b = (int)(gw / W), j = (int)(gw % W);
+    int n = win_count[b];
+    if (n < 0 || n > W) {
+        if (lane == 0 && j == 0) flag(ERRF_COUNT);
+        n = n < 0 ? 0 : W;
+    }
+    if (j >= n) return;
+    const float sc = winsc ? winsc[(int64_t)b * W + j] : 1.f;
+    if (winsc && lane == 0 && !(sc >= 0.f)) flag(ERRF_SCALE);
+    const size_t es = dt == DT_F32 ? 4 : 2;
+    const uint8_t *kr = (const uint8_t *)winK + ((size_t)b * W + j) * d_I * es;
+    float y = 0.f;
+    for (int h = lane; h < n_h; h += 32) {
+        const uint8_t *qr = (const uint8_t *)q + ((size_t)b * TQ * n_h + h) * d_I * es;  // query slot 0
+        float d = 0.f;
+        for (int e = 0; e < d_I; e++) {
+            const float qv = es == 4 ? ((const float *)qr)[e] : __bfloat162float(((const __nv_bfloat16 *)qr)[e]);
+            const float kv = es == 4 ? ((const float *)kr)[e] : __bfloat162float(((const __nv_bfloat16 *)kr)[e]);
+            d = fmaf(qv, kv, d);
+        }
+        y = fmaf(w[(size_t)b * TQ * n_h + h], fmaxf(sc * d, 0.f), y);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
+    if (lane == 0) tail[(int64_t)b * W + j] = y;
 }
 
 }  // namespace lsa

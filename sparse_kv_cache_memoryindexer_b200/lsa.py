@@ -28,6 +28,7 @@ EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_devic
            "lsa_memindex_score_select_static",
            "lsa_fetch_gather", "lsa_fetch_incremental_workspace_size", "lsa_fetch_gather_incremental",
            "lsa_lightning_topk_workspace_size", "lsa_lightning_topk",
+           "lsa_lightning_topk_step_workspace_size", "lsa_lightning_topk_step",
            "lsa_pool_alloc", "lsa_pool_free")
 
 
@@ -58,6 +59,8 @@ def _load():
         "lsa_fetch_gather_incremental": (I, [P, P, P, I64, I, P, P, P, I64, P, P, SZ, P, P, P, SZ, P]),
         "lsa_lightning_topk_workspace_size": (SZ, [I, I, I64, I]),
         "lsa_lightning_topk": (I, [P, P, P, P, I, P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P]),
+        "lsa_lightning_topk_step_workspace_size": (SZ, [I, I64, I, I, I]),
+        "lsa_lightning_topk_step": (I, [P, I64, P, I64, P, P, I, P, P, P, I64, P, P, P, I, I, I, I, I, P, P, P, SZ, P]),
         "lsa_pool_alloc": (I, [SZ, C.POINTER(C.c_void_p)]),
         "lsa_pool_free": (I, [P]),
     }
@@ -86,6 +89,13 @@ def _p(t):
         raise TypeError("expected a torch.Tensor")
     if not t.is_contiguous():
         raise ValueError("tensors passed to the LSA library must be contiguous")
+    return t.data_ptr()
+
+
+def _p_rows(t):
+    """Pointer of a view whose rows are contiguous but whose outer (batch) stride may be larger."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
     return t.data_ptr()
 
 
@@ -220,6 +230,29 @@ def lsa_lightning_topk(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, 
 
 
 # ------------------------------------------------------------------------ cold pool
+
+def lsa_lightning_topk_step_workspace_size(B, total_S, n_h, d_I, W) -> int:
+    return int(_lib.lsa_lightning_topk_step_workspace_size(B, total_S, n_h, d_I, W))
+
+
+def lsa_lightning_topk_step(q_step, w_step, hot_K, hot_scale, idx, count, seq_offsets, total_S, k, topk_idx,
+                            workspace, win_K=None, win_scale=None, win_count=None, topk_score=None, kdt=None,
+                            stream=None):
+    """One decode step: q_step [B][n_h][d_I] and w_step [B][n_h] may be strided views (e.g. a
+    column q_dec[:, i] of the window's queries); window entries win_K [B][W][d_I] with win_count [B]."""
+    _dev(q_step, w_step, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, win_K, win_scale, win_count,
+         topk_score)
+    B, n_h, d_I = q_step.shape
+    if q_step.stride(2) != 1 or q_step.stride(1) != d_I or w_step.stride(1) != 1:
+        raise ValueError("q_step rows and w_step rows must be contiguous (a batch stride is allowed)")
+    if kdt is None:
+        kdt = DTYPE_CODE[torch.float8_e4m3fn] if hot_scale is not None else DTYPE_CODE[hot_K.dtype]
+    W = win_K.shape[1] if win_K is not None else 0
+    _check(_lib.lsa_lightning_topk_step(
+        _p_rows(q_step), q_step.stride(0), _p_rows(w_step), w_step.stride(0), _p(hot_K), _p(hot_scale), kdt, _p(idx), _p(count),
+        _p(seq_offsets), int(total_S), _p(win_K), _p(win_scale), _p(win_count), W, B, n_h, d_I, int(k), _p(topk_idx),
+        _p(topk_score), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
 
 class MappedPool:
     """Mapped page-locked host buffer from lsa_pool_alloc, viewed as a uint8 tensor [rows][row_bytes]."""
