@@ -36,8 +36,10 @@ def _load(path):
     h.lsa_oracle_score_entries.argtypes = [P, I, P, P, P, I, P, I, I, I, I, I64, P, P, P]
     h.lsa_oracle_gather.argtypes = [P, P, P, I, P, I64, P, P, P, I, I, P, P]
     h.lsa_oracle_lightning_topk.argtypes = [P, I, P, P, P, I, P, P, P, I, I, I, I, I, I64, P, P, P, P, P]
+    h.lsa_oracle_golden_labels.argtypes = [P, P, I, I, I, D, I, P, P, P]
     for f in ("project", "score", "score_entries", "gather", "lightning_topk"):
         getattr(h, "lsa_oracle_" + f).restype = I
+    h.lsa_oracle_golden_labels.restype = I
     return h
 
 
@@ -229,3 +231,23 @@ def lightning_topk(q_dec, w_dec, K_sel, k_scale_sel, idx, count, seq_offsets, k:
                                          y.ctypes.data if y is not None else None)
     _check(rc, "lightning_topk")
     return {"idx": out_i, "score": out_s, "y": y}
+
+
+def golden_labels(z, seq_offsets, p: float = 0.6, theta: int = 3, want_golden: bool = False):
+    """Golden labels of one future window from raw indexer logits z [tau][Lc][T] (float32).
+
+    Returns dict: label [T] uint8 (golden for some token of the window), nsize [B][tau][Lc] int32
+    (nucleus sizes), golden [tau][T] uint8 when want_golden.
+    """
+    tau, Lc, T = z.shape
+    offs = np.ascontiguousarray(seq_offsets, dtype=np.int64)
+    B = offs.size - 1
+    zz = np.ascontiguousarray(z.numpy() if hasattr(z, "numpy") else z, dtype=np.float32)
+    label = np.zeros(T, dtype=np.uint8)
+    nsize = np.zeros((B, tau, Lc), dtype=np.int32)
+    golden = np.zeros((tau, T), dtype=np.uint8) if want_golden else None
+    rc = lib().lsa_oracle_golden_labels(zz.ctypes.data, offs.ctypes.data, B, tau, Lc, float(p), int(theta),
+                                        label.ctypes.data, golden.ctypes.data if golden is not None else None,
+                                        nsize.ctypes.data)
+    _check(rc, "golden_labels")
+    return {"label": label, "nsize": nsize, "golden": golden}

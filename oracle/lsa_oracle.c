@@ -17,6 +17,11 @@
  *         sum followed by Top-k, run over C_t^MemComp only, giving C_i^CoreComp.
  *   [FP8] OCP 8-bit floating point specification, E4M3 encoding (bias 7, no infinities,
  *         S.1111.111 is NaN).  bf16 is the upper half of an IEEE-754 binary32.
+ *   [GL]  blog review, section 4.1 "golden labels"; hyper.ai summary, "Dataset"; gist.science
+ *         summary, section 2.2: per token of the future window and per CSA layer, softmax over
+ *         the raw indexer logits, keep the top-p (p = 0.6) nucleus; an entry is golden for the
+ *         token if at least theta = 3 layers keep it; the window's label set is the union of
+ *         its tokens' golden sets.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - the threshold is inclusive, decided on the logit: I >= thr  <=>  x >= log(thr/(1-thr))
@@ -380,5 +385,82 @@ int lsa_oracle_lightning_topk(const void *q_dec, int qdt, const float *w_dec, co
         }
         free(v);
     }
+    return status;
+}
+
+/* ----------------------------------------------------------------------------------------
+ * [GL] Golden labels of one future window.
+ *   z          [tau][Lc][T] fp32 raw indexer logits: token i, CSA layer l, entry offs[b] + s
+ *   p          nucleus mass (the pages use 0.6), theta votes needed (the pages use 3)
+ *   label_out  [T] uint8: 1 if entry s of sequence b is golden for some token of the window
+ *   golden_out [tau][T] uint8 (nullable): the golden set of each token
+ *   nsize_out  [B][tau][Lc] int32 (nullable): nucleus size of each (sequence, token, layer)
+ * Per (b, i, l): softmax over the S_b entries, in double; entries taken by probability
+ * descending (ties: smaller entry first) until the taken mass reaches p of the total (the
+ * entry that reaches it is taken).  The comparison uses the unnormalised masses
+ * e_s = exp(z_s - max z): taken while  sum e < p * sum_all e.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct { double z; int32_t s; } logit_t;
+
+static int by_logit_then_index(const void *pa, const void *pb)
+{
+    const logit_t *a = (const logit_t *)pa, *b = (const logit_t *)pb;
+    if (a->z > b->z) return -1;
+    if (a->z < b->z) return 1;
+    return (a->s > b->s) - (a->s < b->s);
+}
+
+int lsa_oracle_golden_labels(const float *z, const int64_t *seq_offsets, int B, int tau, int Lc, double p,
+                             int theta, uint8_t *label_out, uint8_t *golden_out, int32_t *nsize_out)
+{
+    const int64_t T = seq_offsets[B];
+    int status = 0;
+    uint8_t *kept = (uint8_t *)calloc((size_t)tau * Lc * (size_t)(T > 0 ? T : 1), 1);  /* nucleus membership */
+    if (!kept) return 2;
+#pragma omp parallel for collapse(3) schedule(dynamic)
+    for (int b = 0; b < B; b++)
+        for (int i = 0; i < tau; i++)
+            for (int l = 0; l < Lc; l++) {
+                const int64_t off = seq_offsets[b], S = seq_offsets[b + 1] - off;
+                const float *row = z + ((size_t)i * Lc + l) * (size_t)T + off;
+                uint8_t *krow = kept + ((size_t)i * Lc + l) * (size_t)T + off;
+                int32_t taken = 0;
+                if (S > 0) {
+                    logit_t *v = (logit_t *)malloc(sizeof(logit_t) * (size_t)S);
+                    if (!v) { status = 2; continue; }
+                    double zmax = -INFINITY, total = 0.0;
+                    for (int64_t s = 0; s < S; s++)
+                        if ((double)row[s] > zmax) zmax = (double)row[s];
+                    for (int64_t s = 0; s < S; s++) {
+                        v[s].z = (double)row[s];
+                        v[s].s = (int32_t)s;
+                        total += exp((double)row[s] - zmax);
+                    }
+                    qsort(v, (size_t)S, sizeof(logit_t), by_logit_then_index);
+                    const double target = p * total;
+                    double mass = 0.0;
+                    for (int64_t r = 0; r < S; r++) {
+                        if (mass >= target) break;
+                        mass += exp(v[r].z - zmax);
+                        krow[v[r].s] = 1;
+                        taken++;
+                    }
+                    free(v);
+                }
+                if (nsize_out) nsize_out[((size_t)b * tau + i) * Lc + l] = taken;
+            }
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < T; e++) {
+        uint8_t any = 0;
+        for (int i = 0; i < tau; i++) {
+            int votes = 0;
+            for (int l = 0; l < Lc; l++) votes += kept[((size_t)i * Lc + l) * (size_t)T + e];
+            const uint8_t g = votes >= theta;
+            if (golden_out) golden_out[(size_t)i * T + e] = g;
+            any |= g;
+        }
+        label_out[e] = any;
+    }
+    free(kept);
     return status;
 }

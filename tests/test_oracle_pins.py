@@ -398,6 +398,88 @@ def pin_topk_single_head_closed_form():
     np.testing.assert_allclose(out["y"][0], want, rtol=1e-14, atol=1e-14)
 
 
+# ------------------------------------------------------------------ golden labels (blog review 4.1)
+
+def _golden_rows(rows, p=0.6, theta=1):
+    """One sequence, tokens = rows (list of [Lc][S] logit arrays)."""
+    z = np.asarray(rows, dtype=np.float32)            # [tau][Lc][S]
+    return oracle.golden_labels(z, [0, z.shape[2]], p=p, theta=theta, want_golden=True)
+
+
+def pin_golden_dominant_entry_is_the_whole_nucleus():
+    row = np.zeros(100, dtype=np.float32)
+    row[37] = 10.0          # mass 1 against 99 * e^-10 = 0.0045: far above 0.6 of the total
+    out = _golden_rows([[row]])
+    assert out["nsize"][0, 0, 0] == 1
+    assert np.nonzero(out["label"])[0].tolist() == [37]
+
+
+def pin_golden_uniform_logits_take_ceil_p_s_smallest_entries():
+    # equal probabilities 1/S: the nucleus is the first ceil(0.6 S) entries in index order
+    for S, want in ((7, 5), (1000, 600), (12, 8), (3, 2)):
+        out = _golden_rows([[np.full(S, 0.25, dtype=np.float32)]])
+        assert out["nsize"][0, 0, 0] == want, (S, out["nsize"])
+        assert np.nonzero(out["label"])[0].tolist() == list(range(want))
+
+
+def pin_golden_masses_closed_form():
+    # probabilities 0.15, 0.55, 0.30 (in that entry order): p = 0.6 needs 0.55 + 0.30
+    row = np.log(np.array([0.15, 0.55, 0.30])).astype(np.float32)
+    assert np.nonzero(_golden_rows([[row]], p=0.6)["label"])[0].tolist() == [1, 2]
+    assert np.nonzero(_golden_rows([[row]], p=0.5)["label"])[0].tolist() == [1]
+    assert np.nonzero(_golden_rows([[row]], p=0.9)["label"])[0].tolist() == [0, 1, 2]
+
+
+def pin_golden_votes_need_theta_layers():
+    S, Lc = 20, 5
+    layers = np.zeros((Lc, S), dtype=np.float32)
+    layers[0:3, 7] = 12.0   # three layers keep entry 7 alone
+    layers[3:5, 9] = 12.0   # two layers keep entry 9 alone
+    assert np.nonzero(_golden_rows([layers], theta=3)["label"])[0].tolist() == [7]
+    assert np.nonzero(_golden_rows([layers], theta=2)["label"])[0].tolist() == [7, 9]
+    assert not _golden_rows([layers], theta=6)["label"].any()
+
+
+def pin_golden_window_is_the_union_of_tokens():
+    S, Lc = 16, 3
+    t0 = np.zeros((Lc, S), dtype=np.float32)
+    t0[:, 4] = 12.0
+    t1 = np.zeros((Lc, S), dtype=np.float32)
+    t1[:, 11] = 12.0
+    out = _golden_rows([t0, t1], theta=3)
+    assert np.nonzero(out["golden"][0])[0].tolist() == [4]
+    assert np.nonzero(out["golden"][1])[0].tolist() == [11]
+    assert np.nonzero(out["label"])[0].tolist() == [4, 11]
+
+
+def pin_golden_sequences_are_separate_softmaxes():
+    S = (7, 0, 4, 4)
+    z = np.zeros((1, 1, sum(S)), dtype=np.float32)
+    z[0, 0, 0:7] = 0.5                  # sequence 0: uniform, ceil(4.2) = 5 entries
+    z[0, 0, 7 + 2] = 12.0               # sequence 2: entry 2 dominates
+    z[0, 0, 11:15] = -3.0               # sequence 3: uniform again, ceil(2.4) = 3 entries
+    out = oracle.golden_labels(z, [0, 7, 7, 11, 15], theta=1)
+    assert out["nsize"][:, 0, 0].tolist() == [5, 0, 1, 3]
+    assert np.nonzero(out["label"])[0].tolist() == [0, 1, 2, 3, 4, 9, 11, 12, 13]
+
+
+def pin_golden_nucleus_is_minimal_and_monotone():
+    rng = np.random.default_rng(3)
+    S = 500
+    row = (rng.standard_normal(S) * 2.0).astype(np.float32)
+    row[rng.choice(S, 12, replace=False)] += 6.0
+    e = np.exp(row.astype(np.float64) - row.max())
+    sets = {}
+    for p in (0.3, 0.6, 0.8):
+        kept = np.nonzero(_golden_rows([[row]], p=p)["label"])[0]
+        sets[p] = set(kept.tolist())
+        mass = e[kept].sum()
+        assert mass >= p * e.sum() * (1 - 1e-12)                               # reaches p
+        assert mass - e[kept].min() < p * e.sum()                              # nothing to spare
+        assert e[kept].min() >= np.delete(e, kept).max(initial=0.0)            # the largest ones
+    assert sets[0.3] <= sets[0.6] <= sets[0.8]
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -419,6 +501,14 @@ MUTANTS = {
     "c_not_rounded": ("c[j] = round_to(dt, acc);", "c[j] = acc;"),
     "e4m3_bias_off": ("v = ldexp(8.0 + (double)m, e - 10);", "v = ldexp(8.0 + (double)m, e - 9);"),
     "w_uses_wdq": ("acc += elem(h, dt, hb + i) * elem(W_w, dt,", "acc += elem(h, dt, hb + i) * elem(W_dq, dt,"),
+    "golden_strict_mass": ("if (mass >= target) break;", "if (mass > target) break;"),
+    "golden_vote_off_by_one": ("const uint8_t g = votes >= theta;", "const uint8_t g = votes > theta;"),
+    "golden_last_token_only": ("any |= g;", "any = g;"),
+    "golden_tie_high": ("if (a->z < b->z) return 1;\n    return (a->s > b->s) - (a->s < b->s);",
+                        "if (a->z < b->z) return 1;\n    return (a->s < b->s) - (a->s > b->s);"),
+    "golden_mass_not_exp": ("mass += exp(v[r].z - zmax);", "mass += v[r].z - zmax;"),
+    "golden_softmax_over_all_sequences": ("const float *row = z + ((size_t)i * Lc + l) * (size_t)T + off;",
+                                          "const float *row = z + ((size_t)i * Lc + l) * (size_t)T;"),
 }
 
 
