@@ -48,6 +48,7 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-incremental", action="store_true", help="skip the incremental-fetch measurement")
     p.add_argument("--no-decode-steps", action="store_true", help="skip the per-step decode measurement")
+    p.add_argument("--no-golden", action="store_true", help="skip the golden-label measurement")
     return p.parse_args()
 
 
@@ -241,6 +242,36 @@ def h2d_bandwidth(device, nbytes=1 << 30):
 
 
 # ------------------------------------------------------------------------------------ lsa arm
+
+def measure_golden(lsa, device, B=8, S=32768, tau=64, Lc=21, reps=5):
+    """Golden labels of one window for B sequences of S entries (128K-token documents at 4:1),
+    tau tokens x Lc CSA layers of raw logits; timed alone.  Roofline: the logits, read once."""
+    z, offs = synth.golden_logits([S] * B, tau=tau, Lc=Lc, seed=2024)
+    zd, od = z.to(device), offs.to(device)
+    T = B * S
+    label = torch.empty(T, dtype=torch.uint8, device=device)
+    ws = torch.empty(lsa.lsa_golden_labels_workspace_size(tau, Lc, T), dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream(device)
+    lsa.lsa_golden_labels(zd, od, label, ws, stream=st)
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(reps):
+        lsa.lsa_golden_labels(zd, od, label, ws, stream=st)
+    b.record(st)
+    torch.cuda.synchronize(device)
+    lsa.lsa_check_device(st)
+    ms = a.elapsed_time(b) / reps
+    nbytes = z.numel() * 4 + T
+    peaks = load_peaks()
+    out = {"B": B, "S": S, "tau": tau, "layers": Lc, "ms": ms, "golden_per_sequence": int(label.sum().item()) / B,
+           "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "bytes_per_launch": nbytes},
+           "note": "softmax + top-p 0.6 + 3-of-21 vote + window union over synthetic logits; timed alone"}
+    out["roofline"]["frac"] = out["roofline"]["achieved"] / out["roofline"]["peak"]
+    del zd, ws, label
+    return out
+
 
 def measure_decode_steps(lsa, path, wl, offs, qd, wd, st, reps=3):
     """S5 per decode step: tau calls of lsa_lightning_topk_step (one query per sequence each, over
@@ -448,6 +479,9 @@ def run_lsa(args, rank, world, device):
     steps = None
     if not args.no_decode_steps and world == 1:
         steps = measure_decode_steps(lsa, path, wl, offs, qd, wd, st)
+    gold = None
+    if not args.no_golden and world == 1:
+        gold = measure_golden(lsa, device)
 
     result = None
     if rank == 0:
@@ -503,6 +537,7 @@ def run_lsa(args, rank, world, device):
             "e2e": e2e,
             "incremental_fetch": None if incr is None else dict(incr, full_fetch_ms=stage_ms[4]),
             "decode_steps": steps,
+            "golden_labels": gold,
         }
     pool.free()
     return result

@@ -276,6 +276,27 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride,
                                    void *workspace, size_t workspace_bytes, lsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Golden labels of one future window, the indexer's training targets (blog review section 4.1;
+ * hyper.ai summary, "Dataset"; gist.science summary, section 2.2):
+ *   for every token i < tau of the window and CSA layer l < Lc: P = softmax over the sequence's
+ *   entries of the raw indexer logits z[i][l][.]; nucleus = the entries taken by probability
+ *   descending (ties: smaller entry first) until their mass reaches p; golden_i = entries kept by
+ *   at least theta layers; label = union of golden_i over the window.  The pages use p = 0.6,
+ *   theta = 3 and the 21 CSA layers.
+ *   z            [tau][Lc][T] fp32 device, entry s of sequence b at column seq_offsets[b] + s
+ *   label_out    [T] uint8 device: 1 for a golden entry of the window, else 0
+ *   nsize_out    [B][tau][Lc] int32 device (nullable): nucleus sizes
+ * Softmax masses and their sums are taken in double.  Workspace:
+ * lsa_golden_labels_workspace_size (a bit plane per token and layer, cleared by the call).
+ * ---------------------------------------------------------------------------------------- */
+size_t lsa_golden_labels_workspace_size(int tau, int Lc, int64_t total_S);
+
+lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t total_S,
+                             int B, int tau, int Lc, double p, int theta,
+                             uint8_t *label_out, int32_t *nsize_out,
+                             void *workspace, size_t workspace_bytes, lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Cold-pool helpers: page-locked host memory mapped into every device's address space
  * (cudaHostAlloc with the Mapped and Portable flags).  The pointer is valid on the host and,
  * unchanged, in kernels.  lsa_pool_free releases memory from lsa_pool_alloc only.

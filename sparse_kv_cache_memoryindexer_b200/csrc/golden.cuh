@@ -1,0 +1,327 @@
+// Golden labels of one future window (blog review "FlashMemory-DeepSeek-V4", section 4.1;
+// hyper.ai summary, "Dataset"; gist.science summary, section 2.2): for every token i of the window
+// and every CSA layer l, softmax over the raw indexer logits of the sequence's entries and keep the
+// top-p nucleus (entries by probability descending, ties to the smaller entry, until the kept mass
+// reaches p of the total); an entry is golden for token i if at least theta layers keep it; the
+// window's label set is the union over its tokens.
+//
+// k_golden_nucleus   one CTA per (sequence, token, layer) row.  The kept set is {key > K*} plus the
+//                    first n of {key == K*} in entry order, where key is the order-preserving
+//                    integer image of the logit.  One pass gives the total mass Z = sum e
+//                    (e = exp(z - max z), double) and, for a few depths D, the mass and count of
+//                    the entries within D of the maximum.  The nucleus lies inside the smallest such
+//                    set whose mass reaches p Z; when that set has at most CAND entries they are
+//                    sorted in shared memory (logit descending, entry ascending) and scanned in
+//                    double for the crossing.  Otherwise (flat rows) K* and n come from a
+//                    most-significant-digit-first radix search on the key driven by the masses.
+//                    The row's kept bits go to a [tau][Lc][ceil(T/32)] bit plane, one atomicOr per
+//                    32-entry word (words can straddle two sequences).
+// k_golden_vote      one warp per 32-entry word: votes over the Lc layers per token, theta test,
+//                    OR over the tokens, one label byte per entry.
+#pragma once
+#include "common.cuh"
+
+namespace lsa {
+
+namespace golden {
+
+constexpr int THREADS = 256;
+constexpr int CAND = 4096;       // candidates sorted in shared memory
+constexpr int ND = 6;            // depths below the maximum tried for the candidate set
+__device__ __forceinline__ float depth(int k) { return k == 0 ? 4.f : (k == 1 ? 8.f : (k == 2 ? 12.f : (k == 3 ? 16.f : (k == 4 ? 24.f : 40.f)))); }
+
+__device__ __forceinline__ float block_max(float v, float *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = -INFINITY;
+    for (int w = 0; w < THREADS / 32; w++) r = fmaxf(r, red[w]);
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ double block_sum(double v, double *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    double r = 0.0;
+    for (int w = 0; w < THREADS / 32; w++) r += red[w];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restrict__ z, const int64_t *__restrict__ offs,
+                                                            int64_t T, int B, int tau, int Lc, double p,
+                                                            uint32_t *__restrict__ bits, int64_t W32,
+                                                            int32_t *__restrict__ nsize)
+{
+    __shared__ double hmass[256];
+    __shared__ int hcnt[256];
+    __shared__ unsigned long long cand[CAND];  // (key << 32) | ~entry
+    __shared__ double dmass[ND][THREADS / 32];
+    __shared__ int dcnt[ND][THREADS / 32];
+    __shared__ int s_nc, s_depth, s_cross;
+    __shared__ float fred[THREADS / 32];
+    __shared__ double dred[THREADS / 32];
+    __shared__ uint32_t s_prefix;
+    __shared__ double s_need;
+    __shared__ int s_taken_above, s_last_eq;
+    __shared__ int warp_tot[32];
+    const int r = blockIdx.x;
+    const int b = r / (tau * Lc), i = (r / Lc) % tau, l = r % Lc;
+    const int64_t off = offs[b], S = offs[b + 1] - off;
+    if (S <= 0) {
+        if (threadIdx.x == 0 && nsize) nsize[r] = 0;
+        return;
+    }
+    const float *row = z + ((int64_t)i * Lc + l) * T + off;
+    float m = -INFINITY;
+    for (int64_t s = threadIdx.x; s < S; s += THREADS) m = fmaxf(m, row[s]);
+    m = block_max(m, fred);
+    double tot = 0.0, dm[ND];
+    int dc[ND];
+#pragma unroll
+    for (int k = 0; k < ND; k++) {
+        dm[k] = 0.0;
+        dc[k] = 0;
+    }
+    for (int64_t s = threadIdx.x; s < S; s += THREADS) {
+        const float zs = row[s];
+        const double e = exp((double)zs - (double)m);
+        tot += e;
+#pragma unroll
+        for (int k = 0; k < ND; k++)
+            if (m - zs < depth(k)) {
+                dm[k] += e;
+                dc[k]++;
+            }
+    }
+    {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+        for (int k = 0; k < ND; k++) {
+            double v = dm[k];
+            int c = dc[k];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                v += __shfl_xor_sync(0xffffffffu, v, o);
+                c += __shfl_xor_sync(0xffffffffu, c, o);
+            }
+            if (lane == 0) {
+                dmass[k][warp] = v;
+                dcnt[k][warp] = c;
+            }
+        }
+    }
+    tot = block_sum(tot, dred);  // (its barriers also publish dmass / dcnt)
+    const double target = p * tot;
+    if (threadIdx.x == 0) {
+        s_depth = -1;
+        for (int k = 0; k < ND; k++) {
+            double v = 0.0;
+            int c = 0;
+            for (int w = 0; w < THREADS / 32; w++) {
+                v += dmass[k][w];
+                c += dcnt[k][w];
+            }
+            if (v >= target && c <= CAND) {
+                s_depth = k;
+                break;
+            }
+        }
+        s_nc = 0;
+        s_cross = INT_MAX;
+    }
+    __syncthreads();
+    if (s_depth >= 0) {
+        // ---- candidate path: the entries within depth(k) of the maximum, sorted
+        const float D = depth(s_depth);
+        for (int64_t s = threadIdx.x; s < S; s += THREADS) {
+            const float zs = row[s];
+            if (m - zs < D) {
+                const int at = atomicAdd(&s_nc, 1);
+                if (at < CAND)
+                    cand[at] = ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s);
+            }
+        }
+        __syncthreads();
+        const int nc = s_nc < CAND ? s_nc : CAND;
+        int np2 = 1;
+        while (np2 < nc) np2 <<= 1;
+        for (int t = nc + threadIdx.x; t < np2; t += THREADS) cand[t] = 0ull;
+        __syncthreads();
+        for (int size = 2; size <= np2; size <<= 1) {  // bitonic sort, descending
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int t = threadIdx.x; t < np2 / 2; t += THREADS) {
+                    const int lo = 2 * t - (t & (stride - 1)), hi = lo + stride;
+                    const bool desc = (lo & size) == 0;
+                    const unsigned long long a = cand[lo], c = cand[hi];
+                    if ((a < c) == desc) {
+                        cand[lo] = c;
+                        cand[hi] = a;
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        // cumulative mass in sorted order; the first position where it reaches the target
+        double carry = 0.0;
+        for (int base = 0; base < nc; base += THREADS) {
+            const int r0 = base + threadIdx.x;
+            const double e = r0 < nc ? exp((double)ordered_to_float((uint32_t)(cand[r0] >> 32)) - (double)m) : 0.0;
+            // block inclusive scan of e (warp scan + warp totals)
+            const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+            double v = e;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (lane == 31) dred[warp] = v;
+            __syncthreads();
+            double before = 0.0, total = 0.0;
+            for (int w = 0; w < THREADS / 32; w++) {
+                before += w < warp ? dred[w] : 0.0;
+                total += dred[w];
+            }
+            const double inc = carry + before + v;
+            if (r0 < nc && inc >= target) atomicMin(&s_cross, r0);  // the first position reaching it
+            carry += total;
+            __syncthreads();
+            if (s_cross < INT_MAX) break;
+        }
+        __syncthreads();
+        const int cross = s_cross < INT_MAX ? s_cross : nc - 1;
+        if (threadIdx.x == 0) {
+            s_prefix = (uint32_t)(cand[cross] >> 32);
+            s_last_eq = (int)(~(uint32_t)(cand[cross] & 0xffffffffull));
+            if (nsize) nsize[r] = cross + 1;
+        }
+        __syncthreads();
+    } else {
+
+    // radix search: all keys above the prefix are kept; `need` is the mass still to be taken
+    uint32_t prefix = 0, pmask = 0;
+    double need = target;
+    int above = 0;
+    for (int pass = 0; pass < 4; pass++) {
+        const int shift = 24 - 8 * pass;
+        for (int t = threadIdx.x; t < 256; t += THREADS) {
+            hmass[t] = 0.0;
+            hcnt[t] = 0;
+        }
+        __syncthreads();
+        for (int64_t s = threadIdx.x; s < S; s += THREADS) {
+            const uint32_t u = float_to_ordered(row[s]);
+            if ((u & pmask) == prefix) {
+                const int d = (int)((u >> shift) & 255u);
+                atomicAdd(&hmass[d], exp((double)row[s] - (double)m));
+                atomicAdd(&hcnt[d], 1);
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double cum = 0.0;
+            int chosen = -1, last = -1, cabove = 0;
+            for (int d = 255; d >= 0; d--) {
+                if (hcnt[d] == 0) continue;
+                last = d;
+                if (cum + hmass[d] >= need) {
+                    chosen = d;
+                    break;
+                }
+                cum += hmass[d];
+                cabove += hcnt[d];
+            }
+            if (chosen < 0) {  // rounding left `need` above the remaining mass: keep everything down to the last key
+                chosen = last;
+                cum -= hmass[last];
+                cabove -= hcnt[last];
+            }
+            s_need = need - cum;
+            s_prefix = prefix | ((uint32_t)chosen << shift);
+            s_taken_above = cabove;
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        need = s_need;
+        above += s_taken_above;
+        pmask |= 255u << shift;
+        __syncthreads();
+    }
+    // keys equal to the prefix: the first n_eq in entry order
+    const uint32_t K = prefix;
+    const int cnt_eq = hcnt[(K & 255u)];
+    const double eK = exp((double)ordered_to_float(K) - (double)m);
+    int n_eq = (int)ceil(need / eK);
+    n_eq = n_eq < 1 ? 1 : (n_eq > cnt_eq ? cnt_eq : n_eq);
+    // the entry index of the n_eq-th equal key (a scan in entry order; only when keys tie)
+    if (threadIdx.x == 0) s_last_eq = (int)S;
+    __syncthreads();
+    if (n_eq < cnt_eq) {
+        int carry = 0;
+        for (int64_t base = 0; base < S; base += THREADS) {
+            const int64_t s = base + threadIdx.x;
+            const int eq = (s < S) && float_to_ordered(row[s]) == K;
+            const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+            const int inc = warp_incl_scan(eq);
+            if (lane == 31) warp_tot[warp] = inc;
+            __syncthreads();
+            int before = 0, tot_eq = 0;
+            for (int w = 0; w < THREADS / 32; w++) {
+                before += w < warp ? warp_tot[w] : 0;
+                tot_eq += warp_tot[w];
+            }
+            if (eq && carry + before + inc == n_eq) s_last_eq = (int)s;
+            carry += tot_eq;
+            __syncthreads();
+            if (carry >= n_eq) break;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s_prefix = K;
+        if (nsize) nsize[r] = above + n_eq;
+    }
+    __syncthreads();
+    }  // radix path
+    const uint32_t K = s_prefix;
+    const int64_t last_eq = s_last_eq;
+    // kept bits, one atomicOr per 32-entry word of the global entry numbering
+    uint32_t *plane = bits + ((int64_t)i * Lc + l) * W32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int64_t g0 = ((off >> 5) + warp) << 5; g0 < off + S; g0 += (int64_t)THREADS) {
+        const int64_t g = g0 + lane, s = g - off;
+        bool keep = false;
+        if (g >= off && s < S) {
+            const uint32_t u = float_to_ordered(row[s]);
+            keep = u > K || (u == K && s <= last_eq);
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0 && bal) atomicOr(plane + (g0 >> 5), bal);
+    }
+}
+
+__global__ void __launch_bounds__(THREADS) k_golden_vote(const uint32_t *__restrict__ bits, int64_t W32, int64_t T,
+                                                         int tau, int Lc, int theta, uint8_t *__restrict__ label)
+{
+    const int64_t w = (int64_t)blockIdx.x * (THREADS / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= W32) return;
+    bool any = false;
+    for (int i = 0; i < tau; i++) {
+        int votes = 0;
+        for (int l = 0; l < Lc; l++) votes += (__ldg(bits + ((int64_t)i * Lc + l) * W32 + w) >> lane) & 1u;
+        any |= votes >= theta;
+    }
+    const int64_t g = w * 32 + lane;
+    if (g < T) label[g] = any ? 1 : 0;
+}
+
+}  // namespace golden
+
+}  // namespace lsa

@@ -14,6 +14,7 @@
 #include "score_tc.cuh"
 #include "li_tc.cuh"
 #include "proj_tc.cuh"
+#include "golden.cuh"
 #include "topk.cuh"
 
 using namespace lsa;
@@ -632,6 +633,42 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     k_topk_select<true><<<(unsigned)B, SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, 1, k, kpow2, topk_idx,
                                                                topk_score, tail, W > 0 ? win_count : nullptr, W, TQ);
     LSA_TRY(launched("decode step: select"));
+    return ok();
+}
+
+// ------------------------------------------------------------------------------ golden labels
+
+size_t lsa_golden_labels_workspace_size(int tau, int Lc, int64_t total_S)
+{
+    if (tau <= 0 || Lc <= 0 || total_S < 0) return 0;
+    return align_up(sizeof(uint32_t) * (size_t)tau * Lc * (size_t)((total_S + 31) / 32 + 1), 256);
+}
+
+lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t total_S, int B, int tau, int Lc,
+                             double p, int theta, uint8_t *label_out, int32_t *nsize_out, void *workspace,
+                             size_t workspace_bytes, lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(z && seq_offsets && label_out, "lsa_golden_labels: null pointer");
+    LSA_REQUIRE(B > 0 && tau > 0 && Lc > 0 && total_S >= 0, "lsa_golden_labels: sizes must be positive");
+    LSA_REQUIRE(p > 0.0 && p <= 1.0, "lsa_golden_labels: p must be in (0, 1]");
+    LSA_REQUIRE(theta >= 1, "lsa_golden_labels: theta must be at least 1");
+    LSA_REQUIRE((int64_t)B * tau * Lc < ((int64_t)1 << 31), "lsa_golden_labels: too many rows");
+    const size_t need = lsa_golden_labels_workspace_size(tau, Lc, total_S);
+    if (!workspace || workspace_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "lsa_golden_labels: workspace needs %zu bytes", need);
+    LSA_REQUIRE(aligned(workspace, 256), "lsa_golden_labels: workspace must be 256-byte aligned");
+    if (total_S == 0) return ok();
+    const int64_t W32 = (total_S + 31) / 32;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t) * (size_t)tau * Lc * W32, st);
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_golden_labels: %s", cudaGetErrorString(e));
+    uint32_t *bits = (uint32_t *)workspace;
+    golden::k_golden_nucleus<<<(unsigned)((int64_t)B * tau * Lc), golden::THREADS, 0, st>>>(
+        z, seq_offsets, total_S, B, tau, Lc, p, bits, W32, nsize_out);
+    LSA_TRY(launched("golden labels: nucleus"));
+    golden::k_golden_vote<<<(unsigned)((W32 + golden::THREADS / 32 - 1) / (golden::THREADS / 32)), golden::THREADS, 0,
+                            st>>>(bits, W32, total_S, tau, Lc, theta, label_out);
+    LSA_TRY(launched("golden labels: vote"));
     return ok();
 }
 

@@ -29,6 +29,7 @@ EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_devic
            "lsa_fetch_gather", "lsa_fetch_incremental_workspace_size", "lsa_fetch_gather_incremental",
            "lsa_lightning_topk_workspace_size", "lsa_lightning_topk",
            "lsa_lightning_topk_step_workspace_size", "lsa_lightning_topk_step",
+           "lsa_golden_labels_workspace_size", "lsa_golden_labels",
            "lsa_pool_alloc", "lsa_pool_free")
 
 
@@ -60,6 +61,8 @@ def _load():
         "lsa_lightning_topk_workspace_size": (SZ, [I, I, I64, I]),
         "lsa_lightning_topk": (I, [P, P, P, P, I, P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P]),
         "lsa_lightning_topk_step_workspace_size": (SZ, [I, I64, I, I, I]),
+        "lsa_golden_labels_workspace_size": (SZ, [I, I, I64]),
+        "lsa_golden_labels": (I, [P, P, I64, I, I, I, C.c_double, I, P, P, P, SZ, P]),
         "lsa_lightning_topk_step": (I, [P, I64, P, I64, P, P, I, P, P, P, I64, P, P, P, I, I, I, I, I, P, P, P, SZ, P]),
         "lsa_pool_alloc": (I, [SZ, C.POINTER(C.c_void_p)]),
         "lsa_pool_free": (I, [P]),
@@ -230,6 +233,20 @@ def lsa_lightning_topk(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, 
 
 
 # ------------------------------------------------------------------------ cold pool
+
+def lsa_golden_labels_workspace_size(tau, Lc, total_S) -> int:
+    return int(_lib.lsa_golden_labels_workspace_size(tau, Lc, total_S))
+
+
+def lsa_golden_labels(z, seq_offsets, label_out, workspace, p=0.6, theta=3, nsize_out=None, stream=None):
+    """Golden labels of one window from raw indexer logits z [tau][Lc][T] fp32 (see include/lsa.h)."""
+    _dev(z, seq_offsets, label_out, workspace, nsize_out)
+    tau, Lc, T = z.shape
+    B = seq_offsets.numel() - 1
+    _check(_lib.lsa_golden_labels(_p(z), _p(seq_offsets), T, B, tau, Lc, float(p), int(theta), _p(label_out),
+                                  _p(nsize_out), _p(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)))
+
 
 def lsa_lightning_topk_step_workspace_size(B, total_S, n_h, d_I, W) -> int:
     return int(_lib.lsa_lightning_topk_step_workspace_size(B, total_S, n_h, d_I, W))

@@ -382,3 +382,42 @@ def random_fetch_list(wl: Workload, rate: float, seed: int = 0):
         idx[offs[b]:offs[b] + sel.size] = sel
         cnt[b] = sel.size
     return torch.from_numpy(idx), torch.from_numpy(cnt)
+
+
+def golden_logits(S, tau: int = 64, Lc: int = 21, seed: int = 2024, planted_frac: float = 0.012,
+                  delta: float = 6.0, agree: float = 0.8, spurious: int = 10):
+    """Raw indexer logits of one future window for the golden-label step, z [tau][Lc][T] float32,
+    and seq_offsets [B+1] int64 (entry s of sequence b at column seq_offsets[b] + s).
+
+    Background logits are N(0, 1).  Each sequence has a fraction `planted_frac` of relevant entries
+    in contiguous runs of 8-64; a relevant entry gets +delta + N(0, 0.5) in each (token, layer)
+    row with probability `agree`, so most layers agree on it.  Every row also lifts `spurious`
+    random entries by delta: peaks that one layer sees and the others do not.  With the defaults
+    the softmax mass of a row is about 70 % relevant entries, and the cross-layer vote keeps a few
+    hundred entries per sequence (the pages report 100-1,000 golden entries per window).
+    """
+    S = [int(x) for x in S]
+    offs = np.zeros(len(S) + 1, dtype=np.int64)
+    offs[1:] = np.cumsum(S)
+    T = int(offs[-1])
+    g = torch.Generator().manual_seed(seed)
+    z = torch.randn((tau, Lc, T), generator=g, dtype=torch.float32)
+    rng = np.random.default_rng(seed)
+    planted = []
+    for b, n in enumerate(S):
+        want = int(planted_frac * n)
+        got = []
+        while sum(len(r) for r in got) < want and n > 64:
+            start = int(rng.integers(0, n - 64))
+            got.append(np.arange(start, start + int(rng.integers(8, 65))))
+        if got:
+            planted.append(offs[b] + np.unique(np.concatenate(got)))
+    planted = torch.from_numpy(np.concatenate(planted)) if planted else torch.zeros(0, dtype=torch.int64)
+    if planted.numel():
+        on = torch.rand((tau, Lc, planted.numel()), generator=g) < agree
+        lift = delta + 0.5 * torch.randn((tau, Lc, planted.numel()), generator=g)
+        z[:, :, planted] += torch.where(on, lift, torch.zeros_like(lift))
+    if T and spurious:
+        cols = torch.randint(0, T, (tau, Lc, spurious), generator=g)
+        z.scatter_add_(2, cols, torch.full((tau, Lc, spurious), delta))
+    return z, torch.from_numpy(offs)
