@@ -14,8 +14,8 @@ import torch
 
 from . import build as _build
 
-DT = {"f32": 0, "bf16": 1, "fp8": 2}
-_TORCH_DT = {torch.float32: "f32", torch.bfloat16: "bf16", torch.float8_e4m3fn: "fp8"}
+DT = {"f32": 0, "bf16": 1, "fp8": 2, "f64": 3}   # f64: exact inputs, for the training-step pins only
+_TORCH_DT = {torch.float32: "f32", torch.bfloat16: "bf16", torch.float8_e4m3fn: "fp8", torch.float64: "f64"}
 
 _lib = None
 
@@ -37,9 +37,11 @@ def _load(path):
     h.lsa_oracle_gather.argtypes = [P, P, P, I, P, I64, P, P, P, I, I, P, P]
     h.lsa_oracle_lightning_topk.argtypes = [P, I, P, P, P, I, P, P, P, I, I, I, I, I, I64, P, P, P, P, P]
     h.lsa_oracle_golden_labels.argtypes = [P, P, I, I, I, D, I, P, P, P]
+    h.lsa_oracle_train_step.argtypes = [P, P, P, P, I, P, P, I, P, P, I, I, I, I, I, I, D, D, P, P, P, P]
     for f in ("project", "score", "score_entries", "gather", "lightning_topk"):
         getattr(h, "lsa_oracle_" + f).restype = I
     h.lsa_oracle_golden_labels.restype = I
+    h.lsa_oracle_train_step.restype = I
     return h
 
 
@@ -251,3 +253,28 @@ def golden_labels(z, seq_offsets, p: float = 0.6, theta: int = 3, want_golden: b
                                         nsize.ctypes.data)
     _check(rc, "golden_labels")
     return {"label": label, "nsize": nsize, "golden": golden}
+
+
+def train_step(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets, n_h: int, d_I: int, gamma: float = 0.0,
+               alpha: float = -1.0):
+    """Loss and gradients of one indexer training step (focal loss; gamma = 0, alpha < 0 is BCE).
+
+    h [L][B][d], W_dq [L][r][d], W_iuq [L][n_h*d_I][r], W_w [L][n_h][d] (one dtype: f32, bf16 or
+    f64 = exact); K [L][T][d_I], k_scale [L][T] or None; labels [T] (0/1).
+    Returns dict: loss (float), g_Wdq, g_Wiuq, g_Ww (float64 arrays in the weights' shapes).
+    """
+    L, B, d = h.shape
+    r = W_dq.shape[1]
+    offs = np.ascontiguousarray(seq_offsets, dtype=np.int64)
+    lab = np.ascontiguousarray(np.asarray(labels), dtype=np.uint8)
+    g_dq = np.zeros(tuple(W_dq.shape), dtype=np.float64)
+    g_iuq = np.zeros(tuple(W_iuq.shape), dtype=np.float64)
+    g_w = np.zeros(tuple(W_w.shape), dtype=np.float64)
+    loss = np.zeros(1, dtype=np.float64)
+    ks = [_c(x) for x in (h, W_dq, W_iuq, W_w, K, k_scale)]
+    rc = lib().lsa_oracle_train_step(ks[0][1], ks[1][1], ks[2][1], ks[3][1], _dt(h), ks[4][1], ks[5][1], _dt(K),
+                                     lab.ctypes.data, offs.ctypes.data, L, B, d, r, n_h, d_I, float(gamma),
+                                     float(alpha), loss.ctypes.data, g_dq.ctypes.data, g_iuq.ctypes.data,
+                                     g_w.ctypes.data)
+    _check(rc, "train_step")
+    return {"loss": float(loss[0]), "g_Wdq": g_dq, "g_Wiuq": g_iuq, "g_Ww": g_w}

@@ -17,6 +17,9 @@
  *         sum followed by Top-k, run over C_t^MemComp only, giving C_i^CoreComp.
  *   [FP8] OCP 8-bit floating point specification, E4M3 encoding (bias 7, no infinities,
  *         S.1111.111 is NaN).  bf16 is the upper half of an IEEE-754 binary32.
+ *   [TR]  hyper.ai summary, "Method"; blog review, section 3: the indexer is trained alone
+ *         against frozen keys K^IComp, only W^DQ, W^IUQ and W^w being trained, with binary
+ *         cross-entropy on the lookahead scores, and a focal loss in the final recipe.
  *   [GL]  blog review, section 4.1 "golden labels"; hyper.ai summary, "Dataset"; gist.science
  *         summary, section 2.2: per token of the future window and per CSA layer, softmax over
  *         the raw indexer logits, keep the top-p (p = 0.6) nucleus; an entry is golden for the
@@ -42,7 +45,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2, ORC_F64 = 3 };  /* F64: inputs kept exact (pins only) */
 
 /* ------------------------------------------------------------ stored-value decoding */
 
@@ -74,6 +77,7 @@ static double elem(const void *base, int dt, size_t i)
     case ORC_F32: return (double)((const float *)base)[i];
     case ORC_BF16: return bf16_value(((const uint16_t *)base)[i]);
     case ORC_FP8_E4M3: return e4m3_value(((const uint8_t *)base)[i]);
+    case ORC_F64: return ((const double *)base)[i];
     }
     return NAN;
 }
@@ -119,6 +123,8 @@ void lsa_oracle_e4m3_decode_array(const uint8_t *codes, double *out, int64_t n)
 /* the value a real number takes once stored in dtype dt (fp32 or bf16, nearest-even) */
 static double round_to(int dt, double x)
 {
+    if (dt == ORC_F64)
+        return x;
     if (dt == ORC_F32)
         return (double)(float)x;
     return bf16_value(lsa_oracle_bf16_bits(x));
@@ -462,5 +468,138 @@ int lsa_oracle_golden_labels(const float *z, const int64_t *seq_offsets, int B, 
         label_out[e] = any;
     }
     free(kept);
+    return status;
+}
+
+/* ----------------------------------------------------------------------------------------
+ * [TR] One training step of the indexer: loss and gradients of W^DQ, W^IUQ, W^w.
+ *   h, W_dq, W_iuq, W_w as lsa_oracle_project (dt: F32, BF16, or F64 = exact inputs);
+ *   K [L][T][d_I] kdt + k_scale [L][T] (nullable) frozen; labels [T] uint8 (the window's golden
+ *   set, the same target for the L indexers).
+ * Forward as the memory indexer ([MI]): c = round(h W^DQ), q = round(c W^IUQ), w = h W^w,
+ *   a_h = scale_s q_h . K_s,  x = sum_h w_h ReLU(a_h),  p = sigmoid(x).
+ * Loss: mean over the L*T (layer, entry) pairs of the focal loss
+ *   l = -at (1 - pt)^gamma log(pt),  pt = y ? p : 1 - p,  at = alpha < 0 ? 1 : (y ? alpha : 1 - alpha),
+ *   which is binary cross-entropy at gamma = 0, alpha < 0.
+ * Backward: the rounding of c and q is passed straight through (d round(v) / dv = 1); the ReLU
+ *   derivative is 1[a > 0].  Outputs loss_out [1] and the gradients g_* in the weights' layouts.
+ * ---------------------------------------------------------------------------------------- */
+static double focal_dx(double x, int y, double gamma, double alpha, double *loss)
+{
+    const double p = 1.0 / (1.0 + exp(-x));
+    const double pt = y ? p : 1.0 - p;
+    const double at = alpha < 0.0 ? 1.0 : (y ? alpha : 1.0 - alpha);
+    /* log(pt) from the logit, stable: log sigmoid(+-x) */
+    const double lpt = y ? -log1p(exp(-x)) : -log1p(exp(x));
+    const double q1 = 1.0 - pt;
+    *loss = -at * pow(q1, gamma) * lpt;
+    /* dl/dpt = at (gamma (1-pt)^(gamma-1) log pt - (1-pt)^gamma / pt);  dpt/dx = +-p (1-p) */
+    double dl_dx;
+    if (gamma == 0.0)
+        dl_dx = at * (y ? p - 1.0 : p);
+    else
+        dl_dx = at * (gamma * pow(q1, gamma - 1.0) * lpt * pt * q1 - pow(q1, gamma) * q1) * (y ? 1.0 : -1.0);
+    return dl_dx;
+}
+
+int lsa_oracle_train_step(const void *h, const void *W_dq, const void *W_iuq, const void *W_w, int dt,
+                          const void *K, const float *k_scale, int kdt, const uint8_t *labels,
+                          const int64_t *seq_offsets, int L, int B, int d, int r, int n_h, int d_I,
+                          double gamma, double alpha, double *loss_out, double *g_Wdq, double *g_Wiuq,
+                          double *g_Ww)
+{
+    if (dt != ORC_F32 && dt != ORC_BF16 && dt != ORC_F64)
+        return 1;
+    const int nq = n_h * d_I;
+    const int64_t T = seq_offsets[B];
+    const double N = (double)L * (double)T;
+    const size_t LB = (size_t)L * B;
+    double *cs = (double *)calloc(LB * r, sizeof(double));
+    double *dq = (double *)calloc(LB * nq, sizeof(double));
+    double *dw = (double *)calloc(LB * n_h, sizeof(double));
+    double *lossp = (double *)calloc(LB, sizeof(double));
+    if (!cs || !dq || !dw || !lossp) { free(cs); free(dq); free(dw); free(lossp); return 2; }
+    int status = 0;
+    /* forward and the per-(layer, sequence) gradients of q and w */
+#pragma omp parallel for schedule(dynamic) collapse(2)
+    for (int l = 0; l < L; l++) {
+        for (int b = 0; b < B; b++) {
+            const size_t lb = (size_t)l * B + b, hb = lb * d;
+            double *c = cs + lb * r;
+            double *q = (double *)malloc(sizeof(double) * nq);
+            double *w = (double *)malloc(sizeof(double) * n_h);
+            double *a = (double *)malloc(sizeof(double) * n_h);
+            if (!q || !w || !a) { status = 2; free(q); free(w); free(a); continue; }
+            for (int j = 0; j < r; j++) {
+                double acc = 0.0;
+                for (int i = 0; i < d; i++) acc += elem(h, dt, hb + i) * elem(W_dq, dt, ((size_t)l * r + j) * d + i);
+                c[j] = round_to(dt, acc);
+            }
+            for (int o = 0; o < nq; o++) {
+                double acc = 0.0;
+                for (int j = 0; j < r; j++) acc += c[j] * elem(W_iuq, dt, ((size_t)l * nq + o) * r + j);
+                q[o] = round_to(dt, acc);
+            }
+            for (int hh = 0; hh < n_h; hh++) {
+                double acc = 0.0;
+                for (int i = 0; i < d; i++) acc += elem(h, dt, hb + i) * elem(W_w, dt, ((size_t)l * n_h + hh) * d + i);
+                w[hh] = dt == ORC_F64 ? acc : (double)(float)acc;
+            }
+            const int64_t off = seq_offsets[b], S = seq_offsets[b + 1] - off;
+            double lsum = 0.0;
+            for (int64_t s = 0; s < S; s++) {
+                const size_t row = (size_t)l * T + off + s;
+                const double scale = k_scale ? (double)k_scale[row] : 1.0;
+                double x = 0.0;
+                for (int hh = 0; hh < n_h; hh++) {
+                    double dot = 0.0;
+                    for (int e = 0; e < d_I; e++) dot += q[(size_t)hh * d_I + e] * elem(K, kdt, row * d_I + e);
+                    a[hh] = scale * dot;
+                    x += w[hh] * (a[hh] > 0.0 ? a[hh] : 0.0);
+                }
+                double ls;
+                const double g = focal_dx(x, labels[off + s] != 0, gamma, alpha, &ls) / N;
+                lsum += ls;
+                for (int hh = 0; hh < n_h; hh++) {
+                    if (a[hh] > 0.0) {
+                        dw[lb * n_h + hh] += g * a[hh];
+                        const double gq = g * w[hh] * scale;
+                        for (int e = 0; e < d_I; e++) dq[lb * nq + (size_t)hh * d_I + e] += gq * elem(K, kdt, row * d_I + e);
+                    }
+                }
+            }
+            lossp[lb] = lsum;
+            free(q); free(w); free(a);
+        }
+    }
+    double loss = 0.0;
+    for (size_t lb = 0; lb < LB; lb++) loss += lossp[lb];
+    *loss_out = loss / N;
+    /* weight gradients: dc = dq W^IUQ (straight through the rounding), then outer products over b */
+#pragma omp parallel for schedule(dynamic)
+    for (int l = 0; l < L; l++) {
+        double *dc = (double *)malloc(sizeof(double) * r);
+        if (!dc) { status = 2; continue; }
+        for (size_t o = 0; o < (size_t)nq * r; o++) g_Wiuq[(size_t)l * nq * r + o] = 0.0;
+        for (size_t o = 0; o < (size_t)r * d; o++) g_Wdq[(size_t)l * r * d + o] = 0.0;
+        for (size_t o = 0; o < (size_t)n_h * d; o++) g_Ww[(size_t)l * n_h * d + o] = 0.0;
+        for (int b = 0; b < B; b++) {
+            const size_t lb = (size_t)l * B + b, hb = lb * d;
+            const double *c = cs + lb * r;
+            for (int j = 0; j < r; j++) {
+                double acc = 0.0;
+                for (int o = 0; o < nq; o++) acc += dq[lb * nq + o] * elem(W_iuq, dt, ((size_t)l * nq + o) * r + j);
+                dc[j] = acc;
+            }
+            for (int o = 0; o < nq; o++)
+                for (int j = 0; j < r; j++) g_Wiuq[((size_t)l * nq + o) * r + j] += dq[lb * nq + o] * c[j];
+            for (int j = 0; j < r; j++)
+                for (int i = 0; i < d; i++) g_Wdq[((size_t)l * r + j) * d + i] += dc[j] * elem(h, dt, hb + i);
+            for (int hh = 0; hh < n_h; hh++)
+                for (int i = 0; i < d; i++) g_Ww[((size_t)l * n_h + hh) * d + i] += dw[lb * n_h + hh] * elem(h, dt, hb + i);
+        }
+        free(dc);
+    }
+    free(cs); free(dq); free(dw); free(lossp);
     return status;
 }

@@ -480,6 +480,79 @@ def pin_golden_nucleus_is_minimal_and_monotone():
     assert sets[0.3] <= sets[0.6] <= sets[0.8]
 
 
+# ------------------------------------------------------------------ training step (hyper.ai "Method")
+
+def _ones(*shape):
+    return torch.ones(shape, dtype=torch.float64)
+
+
+def pin_train_loss_at_zero_logit():
+    # all keys zero: x = 0, p = 1/2 for every entry; BCE is ln 2, focal (gamma 2, alpha 0.25)
+    # is at (1/2)^2 ln 2 with at = 0.25 for positives and 0.75 for negatives
+    K = torch.zeros((2, 6, 3), dtype=torch.float64)
+    lab = [1, 0, 0, 1, 1, 0]
+    h = torch.randn((2, 2, 5), dtype=torch.float64)
+    W = (torch.randn((2, 4, 5), dtype=torch.float64), torch.randn((2, 6, 4), dtype=torch.float64),
+         torch.randn((2, 2, 5), dtype=torch.float64))
+    out = oracle.train_step(h, *W, K, None, lab, [0, 2, 6], 2, 3)
+    assert abs(out["loss"] - math.log(2.0)) < 1e-15
+    assert not out["g_Wdq"].any() and not out["g_Wiuq"].any() and not out["g_Ww"].any()  # ReLU'(0) = 0
+    foc = oracle.train_step(h, *W, K, None, lab, [0, 2, 6], 2, 3, gamma=2.0, alpha=0.25)
+    want = np.mean([(0.25 if y else 0.75) * 0.25 * math.log(2.0) for y in lab])
+    assert abs(foc["loss"] - want) < 1e-15
+
+
+def pin_train_identity_chain_closed_form():
+    # d = r = n_h = d_I = 1 and every weight 1: c = q = w = h = 1, x_s = ReLU(scale_s K_s), and each
+    # of the three gradients is (1/T) sum_s (p_s - y_s) ReLU(scale_s K_s) by the chain rule
+    K = torch.tensor([[[0.0], [1.5], [-2.0], [0.7], [3.0]]], dtype=torch.float64)
+    ks = torch.tensor([[1.0, 0.5, 2.0, 1.0, 0.25]], dtype=torch.float32)
+    lab = [1, 0, 1, 0, 1]
+    out = oracle.train_step(_ones(1, 1, 1), _ones(1, 1, 1), _ones(1, 1, 1), _ones(1, 1, 1), K, ks, lab, [0, 5], 1, 1)
+    x = np.maximum(0.0, K.numpy().ravel() * ks.numpy().ravel().astype(np.float64))
+    p = 1.0 / (1.0 + np.exp(-x))
+    y = np.array(lab, dtype=np.float64)
+    g = ((p - y) * x).sum() / 5
+    for k in ("g_Wdq", "g_Wiuq", "g_Ww"):
+        assert abs(out[k].item() - g) < 1e-15, k
+    assert abs(out["loss"] - np.mean(-(y * np.log(p) + (1 - y) * np.log1p(-p)))) < 1e-14
+
+
+def _fd_case(seed):
+    g = torch.Generator().manual_seed(seed)
+    L, B, d, r, n_h, d_I = 2, 2, 6, 4, 3, 5
+    S = (5, 7)
+    T = sum(S)
+    h = torch.randn((L, B, d), generator=g, dtype=torch.float64)
+    W = [torch.randn(sh, generator=g, dtype=torch.float64) * 0.7 for sh in ((L, r, d), (L, n_h * d_I, r), (L, n_h, d))]
+    K = torch.randn((L, T, d_I), generator=g, dtype=torch.float64)
+    ks = (torch.rand((L, T), generator=g) + 0.5).to(torch.float32)
+    lab = (torch.rand(T, generator=g) < 0.4).to(torch.uint8).numpy()
+    return h, W, K, ks, lab, [0, S[0], T], n_h, d_I
+
+
+def pin_train_gradients_match_finite_differences():
+    # exact inputs (f64): the loss is smooth away from ReLU kinks; central differences of the
+    # oracle's own loss check every gradient formula (a dropped term, a wrong sign or a transposed
+    # weight would show), for binary cross-entropy and for the focal loss
+    for seed, gamma, alpha in ((1, 0.0, -1.0), (2, 2.0, 0.25)):
+        h, W, K, ks, lab, offs, n_h, d_I = _fd_case(seed)
+        out = oracle.train_step(h, *W, K, ks, lab, offs, n_h, d_I, gamma=gamma, alpha=alpha)
+        rng = np.random.default_rng(seed)
+        for wi, key in enumerate(("g_Wdq", "g_Wiuq", "g_Ww")):
+            for _ in range(6):
+                at = tuple(int(rng.integers(0, n)) for n in W[wi].shape)
+                eps = 1e-6
+                Wp = [w.clone() for w in W]
+                Wm = [w.clone() for w in W]
+                Wp[wi][at] += eps
+                Wm[wi][at] -= eps
+                lp = oracle.train_step(h, *Wp, K, ks, lab, offs, n_h, d_I, gamma=gamma, alpha=alpha)["loss"]
+                lm = oracle.train_step(h, *Wm, K, ks, lab, offs, n_h, d_I, gamma=gamma, alpha=alpha)["loss"]
+                fd = (lp - lm) / (2 * eps)
+                assert abs(fd - out[key][at]) <= 1e-7 + 1e-5 * abs(fd), (key, at, fd, out[key][at])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -507,6 +580,12 @@ MUTANTS = {
     "golden_tie_high": ("if (a->z < b->z) return 1;\n    return (a->s > b->s) - (a->s < b->s);",
                         "if (a->z < b->z) return 1;\n    return (a->s < b->s) - (a->s > b->s);"),
     "golden_mass_not_exp": ("mass += exp(v[r].z - zmax);", "mass += v[r].z - zmax;"),
+    "train_relu_grad_dropped": ("                    if (a[hh] > 0.0) {\n                        dw[", "                    if (1) {\n                        dw["),
+    "train_dc_transposed": ("acc += dq[lb * nq + o] * elem(W_iuq, dt, ((size_t)l * nq + o) * r + j);",
+                            "acc += dq[lb * nq + o] * elem(W_iuq, dt, ((size_t)l * r + j) * nq + o);"),
+    "train_focal_sign": ("* lpt * pt * q1 - pow(q1, gamma) * q1) * (y ? 1.0 : -1.0);", "* lpt * pt * q1 - pow(q1, gamma) * q1) * (y ? -1.0 : 1.0);"),
+    "train_loss_not_mean": ("*loss_out = loss / N;", "*loss_out = loss;"),
+    "train_scale_dropped_in_dq": ("const double gq = g * w[hh] * scale;", "const double gq = g * w[hh];"),
     "golden_softmax_over_all_sequences": ("const float *row = z + ((size_t)i * Lc + l) * (size_t)T + off;",
                                           "const float *row = z + ((size_t)i * Lc + l) * (size_t)T;"),
 }
