@@ -49,6 +49,7 @@ def parse_args():
     p.add_argument("--no-incremental", action="store_true", help="skip the incremental-fetch measurement")
     p.add_argument("--no-decode-steps", action="store_true", help="skip the per-step decode measurement")
     p.add_argument("--no-golden", action="store_true", help="skip the golden-label measurement")
+    p.add_argument("--no-train", action="store_true", help="skip the training-step measurement")
     return p.parse_args()
 
 
@@ -242,6 +243,46 @@ def h2d_bandwidth(device, nbytes=1 << 30):
 
 
 # ------------------------------------------------------------------------------------ lsa arm
+
+def measure_train(lsa, device, B=8, S=32768, reps=5):
+    """One indexer training step (BCE) on 128K-token shapes: 3 layers, B sequences of S entries,
+    d 4096, r 2048, 64 heads x 128, bf16 weights and keys; timed alone.  Roofline: the CUDA-core
+    fp32 rate (148 SMs x 128 FMA lanes x 2 flop x 1965 MHz) for the two per-entry products."""
+    wl = synth.workload("ctx128k_bf16", B=B, S=(S,) * B, fetch=(0.135,) * B, name="train_128k")
+    inp = synth.make_inputs(wl, parts=("proj", "score"))
+    d = lambda t: t.to(device)
+    h, Wdq, Wiuq, Ww, K, offs = d(inp.h), d(inp.W_dq), d(inp.W_iuq), d(inp.W_w), d(inp.K), d(inp.seq_offsets)
+    g = torch.Generator().manual_seed(wl.seed + 5)
+    labels = d((torch.rand(wl.total_S, generator=g) < 0.135).to(torch.uint8))
+    loss = torch.zeros(1, dtype=torch.float64, device=device)
+    gW = [torch.empty(w.shape, dtype=torch.float32, device=device) for w in (Wdq, Wiuq, Ww)]
+    ws = torch.empty(lsa.lsa_indexer_train_workspace_size(wl.L, B, wl.total_S, wl.d, wl.r, wl.n_h, wl.d_I,
+                                                          torch.bfloat16), dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream(device)
+
+    def step():
+        lsa.lsa_indexer_train_step(h, Wdq, Wiuq, Ww, K, None, labels, offs, loss, gW[0], gW[1], gW[2], ws, wl.n_h,
+                                   wl.d_I, stream=st)
+    step()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(reps):
+        step()
+    b.record(st)
+    torch.cuda.synchronize(device)
+    lsa.lsa_check_device(st)
+    ms = a.elapsed_time(b) / reps
+    flops = 2.0 * 2.0 * wl.L * wl.total_S * wl.n_h * wl.d_I
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    out = {"L": wl.L, "B": B, "S": S, "ms": ms, "loss": float(loss.item()),
+           "entries_per_s": wl.L * wl.total_S / (ms * 1e-3),
+           "roofline": {"bound": "alu", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                        "peak_note": "fp32 CUDA-core FMA rate at 1965 MHz"},
+           "note": "forward + BCE + backward of W^DQ, W^IUQ, W^w; timed alone"}
+    out["roofline"]["frac"] = out["roofline"]["achieved"] / peak
+    return out
+
 
 def measure_golden(lsa, device, B=8, S=32768, tau=64, Lc=21, reps=5):
     """Golden labels of one window for B sequences of S entries (128K-token documents at 4:1),
@@ -482,6 +523,9 @@ def run_lsa(args, rank, world, device):
     gold = None
     if not args.no_golden and world == 1:
         gold = measure_golden(lsa, device)
+    trn = None
+    if not args.no_train and world == 1:
+        trn = measure_train(lsa, device)
 
     result = None
     if rank == 0:
@@ -538,6 +582,7 @@ def run_lsa(args, rank, world, device):
             "incremental_fetch": None if incr is None else dict(incr, full_fetch_ms=stage_ms[4]),
             "decode_steps": steps,
             "golden_labels": gold,
+            "train_step": trn,
         }
     pool.free()
     return result

@@ -297,6 +297,35 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
                              void *workspace, size_t workspace_bytes, lsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * One training step of the memory indexer (hyper.ai summary, "Method"; blog review section 3):
+ * the indexer is trained alone against frozen keys, only W^DQ, W^IUQ and W^w change, with binary
+ * cross-entropy on the lookahead scores or, in the pages' final recipe, a focal loss.
+ *   forward   as lsa_project and the index score: x_{l,b,s} = sum_h w_h ReLU(scale_s q_h . K_s),
+ *             p = sigmoid(x)
+ *   loss      mean over the L * total_S (layer, entry) pairs of
+ *             -at (1 - pt)^gamma log(pt),  pt = y ? p : 1 - p,  at = alpha < 0 ? 1 : (y ? alpha : 1 - alpha)
+ *             (gamma = 0, alpha < 0 is binary cross-entropy); y = labels[offs_b + s] (the window's
+ *             golden set, e.g. from lsa_golden_labels; the same target for the L indexers)
+ *   backward  the rounding of c and q to dt is passed straight through; ReLU'(a) = 1[a > 0]
+ *   h, W_dq, W_iuq, W_w   as lsa_project (dt: LSA_F32 with LSA_F32 keys, LSA_BF16 with LSA_BF16
+ *                         or LSA_FP8_E4M3 keys); K [L][T][d_I] kdt, k_scale [L][T] (FP8 only)
+ *   labels    [T] uint8 device (0 / 1)
+ *   loss_out  [1] double device; g_Wdq [L][r][d], g_Wiuq [L][n_h*d_I][r], g_Ww [L][n_h][d] fp32
+ *             device (overwritten)
+ * n_h <= 64, d_I <= 128.  Workspace: lsa_indexer_train_workspace_size.  The method has no
+ * training kernel of its own on these pages: this is the fourth widening beyond one window.
+ * ---------------------------------------------------------------------------------------- */
+size_t lsa_indexer_train_workspace_size(int L, int B, int64_t total_S, int d, int r, int n_h, int d_I,
+                                        lsa_dtype dt);
+
+lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W_iuq, const void *W_w,
+                                  lsa_dtype dt, const void *K, const float *k_scale, lsa_dtype kdt,
+                                  const uint8_t *labels, const int64_t *seq_offsets, int64_t total_S,
+                                  int L, int B, int d, int r, int n_h, int d_I, float gamma, float alpha,
+                                  double *loss_out, float *g_Wdq, float *g_Wiuq, float *g_Ww,
+                                  void *workspace, size_t workspace_bytes, lsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Cold-pool helpers: page-locked host memory mapped into every device's address space
  * (cudaHostAlloc with the Mapped and Portable flags).  The pointer is valid on the host and,
  * unchanged, in kernels.  lsa_pool_free releases memory from lsa_pool_alloc only.

@@ -15,6 +15,7 @@
 #include "li_tc.cuh"
 #include "proj_tc.cuh"
 #include "golden.cuh"
+#include "train.cuh"
 #include "topk.cuh"
 
 using namespace lsa;
@@ -669,6 +670,109 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
     golden::k_golden_vote<<<(unsigned)((W32 + golden::THREADS / 32 - 1) / (golden::THREADS / 32)), golden::THREADS, 0,
                             st>>>(bits, W32, total_S, tau, Lc, theta, label_out);
     LSA_TRY(launched("golden labels: vote"));
+    return ok();
+}
+
+// ------------------------------------------------------------------------------ training step
+
+// Workspace of lsa_indexer_train_step: c, q (dt), w, dq, dw, dc (fp32), tile and chunk starts, counts.
+static size_t train_ws_parts(int L, int B, int64_t T, int d, int r, int n_h, int d_I, lsa_dtype dt, size_t part[8])
+{
+    const size_t eb = elem_bytes(dt), LB = (size_t)L * B, nq = (size_t)n_h * d_I;
+    (void)T; (void)d;
+    part[0] = align_up(LB * r * eb, 256);               // c (the projection's workspace)
+    part[1] = align_up(LB * nq * eb, 256);              // q
+    part[2] = align_up(LB * n_h * 4, 256);              // w
+    part[3] = align_up(LB * nq * 4, 256);               // dq
+    part[4] = align_up(LB * n_h * 4, 256);              // dw
+    part[5] = align_up(LB * r * 4, 256);                // dc
+    part[6] = align_up(sizeof(int) * (size_t)(3 * B + 3), 256);  // tile starts, chunk starts, counts
+    part[7] = 256;                                      // loss (double)
+    size_t t = 0;
+    for (int i = 0; i < 8; i++) t += part[i];
+    return t;
+}
+
+size_t lsa_indexer_train_workspace_size(int L, int B, int64_t total_S, int d, int r, int n_h, int d_I, lsa_dtype dt)
+{
+    if (L <= 0 || B <= 0 || total_S < 0 || d <= 0 || r <= 0 || n_h <= 0 || d_I <= 0) return 0;
+    size_t part[8];
+    return train_ws_parts(L, B, total_S, d, r, n_h, d_I, dt, part);
+}
+
+lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W_iuq, const void *W_w, lsa_dtype dt,
+                                  const void *K, const float *k_scale, lsa_dtype kdt, const uint8_t *labels,
+                                  const int64_t *seq_offsets, int64_t total_S, int L, int B, int d, int r, int n_h,
+                                  int d_I, float gamma, float alpha, double *loss_out, float *g_Wdq, float *g_Wiuq,
+                                  float *g_Ww, void *workspace, size_t workspace_bytes, lsa_stream_t stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    LSA_REQUIRE(h && W_dq && W_iuq && W_w && K && labels && seq_offsets && loss_out && g_Wdq && g_Wiuq && g_Ww,
+                "lsa_indexer_train_step: null pointer");
+    LSA_REQUIRE(L > 0 && B > 0 && total_S > 0 && d > 0 && r > 0 && n_h > 0 && d_I > 0,
+                "lsa_indexer_train_step: sizes must be positive");
+    LSA_REQUIRE(total_S < (int64_t)1 << 31, "lsa_indexer_train_step: total_S must be below 2^31");
+    LSA_REQUIRE(gamma >= 0.f && alpha <= 1.f, "lsa_indexer_train_step: gamma >= 0 and alpha <= 1 (alpha < 0: no weighting)");
+    LSA_REQUIRE((kdt == LSA_FP8_E4M3) == (k_scale != nullptr),
+                "lsa_indexer_train_step: k_scale is required for FP8 keys and must be NULL otherwise");
+    const bool combo = (dt == LSA_F32 && kdt == LSA_F32) || (dt == LSA_BF16 && (kdt == LSA_BF16 || kdt == LSA_FP8_E4M3));
+    if (!combo) return fail(LSA_ERR_UNSUPPORTED, "lsa_indexer_train_step: dtypes F32/F32, BF16/BF16 or BF16/FP8 only");
+    if (n_h > train::NHMAX || d_I > train::DMAX)
+        return fail(LSA_ERR_UNSUPPORTED, "lsa_indexer_train_step: n_h <= 64 and d_I <= 128");
+    size_t part[8];
+    const size_t need = train_ws_parts(L, B, total_S, d, r, n_h, d_I, dt, part);
+    if (!workspace || workspace_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "lsa_indexer_train_step: workspace needs %zu bytes", need);
+    LSA_REQUIRE(aligned(workspace, 256), "lsa_indexer_train_step: workspace must be 256-byte aligned");
+    char *p = (char *)workspace;
+    void *c = p;
+    void *q = p + part[0];
+    float *w = (float *)(p + part[0] + part[1]);
+    float *dq = (float *)(p + part[0] + part[1] + part[2]);
+    float *dw = (float *)(p + part[0] + part[1] + part[2] + part[3]);
+    float *dc = (float *)(p + part[0] + part[1] + part[2] + part[3] + part[4]);
+    int *tile_start = (int *)(p + part[0] + part[1] + part[2] + part[3] + part[4] + part[5]);
+    int *chunk_start = tile_start + (B + 1);
+    int32_t *cnt = chunk_start + (B + 1);
+    double *loss = (double *)(p + part[0] + part[1] + part[2] + part[3] + part[4] + part[5] + part[6]);
+    (void)loss;
+    const int nq = n_h * d_I;
+    cudaError_t e = cudaMemsetAsync(dq, 0, part[3] + part[4], st);  // dq and dw are adjacent
+    if (e == cudaSuccess) e = cudaMemsetAsync(loss_out, 0, sizeof(double), st);
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_indexer_train_step: %s", cudaGetErrorString(e));
+    LSA_TRY(lsa_project(h, W_dq, W_iuq, W_w, dt, L, B, d, r, n_h, d_I, q, w, c, part[0], stream));
+    k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, tile_start, chunk_start, cnt);
+    LSA_TRY(launched("training step: tiles"));
+    const size_t smem = train::entries_smem();
+    const dim3 grid((unsigned)(total_S / train::TT + B + 1), (unsigned)L);
+    const double invN = 1.0 / ((double)L * (double)total_S);
+#define LSA_TRAIN_ENTRIES(QD, KD)                                                                                  \
+    do {                                                                                                           \
+        LSA_TRY(set_smem(train::k_train_entries<QD, KD>, smem));                                                   \
+        train::k_train_entries<QD, KD><<<grid, train::THREADS, smem, st>>>(q, w, K, k_scale, labels, seq_offsets,  \
+                                                                           tile_start, B, total_S, n_h, d_I, gamma,  \
+                                                                           alpha, invN, dq, dw, loss_out);         \
+    } while (0)
+    if (dt == LSA_F32) LSA_TRAIN_ENTRIES(DT_F32, DT_F32);
+    else if (kdt == LSA_BF16) LSA_TRAIN_ENTRIES(DT_BF16, DT_BF16);
+    else LSA_TRAIN_ENTRIES(DT_BF16, DT_FP8);
+#undef LSA_TRAIN_ENTRIES
+    LSA_TRY(launched("training step: entries"));
+    const int64_t ndc = (int64_t)L * B * r;
+    const int64_t n_iuq = (int64_t)L * nq * r, n_dq = (int64_t)L * r * d, n_w = (int64_t)L * n_h * d;
+    if (dt == LSA_F32) {
+        train::k_train_dc<DT_F32><<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        train::k_outer<DT_F32><<<(unsigned)((n_iuq + 255) / 256), 256, 0, st>>>(dq, c, L, B, nq, r, g_Wiuq);
+        train::k_outer<DT_F32><<<(unsigned)((n_dq + 255) / 256), 256, 0, st>>>(dc, h, L, B, r, d, g_Wdq);
+        train::k_outer<DT_F32><<<(unsigned)((n_w + 255) / 256), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);
+    } else {
+        train::k_train_dc<DT_BF16><<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        train::k_outer<DT_BF16><<<(unsigned)((n_iuq + 255) / 256), 256, 0, st>>>(dq, c, L, B, nq, r, g_Wiuq);
+        train::k_outer<DT_BF16><<<(unsigned)((n_dq + 255) / 256), 256, 0, st>>>(dc, h, L, B, r, d, g_Wdq);
+        train::k_outer<DT_BF16><<<(unsigned)((n_w + 255) / 256), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);
+    }
+    LSA_TRY(launched("training step: weight gradients"));
+    g_launches.fetch_add(3, std::memory_order_relaxed);
     return ok();
 }
 

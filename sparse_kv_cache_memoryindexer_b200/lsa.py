@@ -30,6 +30,7 @@ EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_devic
            "lsa_lightning_topk_workspace_size", "lsa_lightning_topk",
            "lsa_lightning_topk_step_workspace_size", "lsa_lightning_topk_step",
            "lsa_golden_labels_workspace_size", "lsa_golden_labels",
+           "lsa_indexer_train_workspace_size", "lsa_indexer_train_step",
            "lsa_pool_alloc", "lsa_pool_free")
 
 
@@ -63,6 +64,9 @@ def _load():
         "lsa_lightning_topk_step_workspace_size": (SZ, [I, I64, I, I, I]),
         "lsa_golden_labels_workspace_size": (SZ, [I, I, I64]),
         "lsa_golden_labels": (I, [P, P, I64, I, I, I, C.c_double, I, P, P, P, SZ, P]),
+        "lsa_indexer_train_workspace_size": (SZ, [I, I, I64, I, I, I, I, I]),
+        "lsa_indexer_train_step": (I, [P, P, P, P, I, P, P, I, P, P, I64, I, I, I, I, I, I, F, F, P, P, P, P, P, SZ,
+                                       P]),
         "lsa_lightning_topk_step": (I, [P, I64, P, I64, P, P, I, P, P, P, I64, P, P, P, I, I, I, I, I, P, P, P, SZ, P]),
         "lsa_pool_alloc": (I, [SZ, C.POINTER(C.c_void_p)]),
         "lsa_pool_free": (I, [P]),
@@ -246,6 +250,23 @@ def lsa_golden_labels(z, seq_offsets, label_out, workspace, p=0.6, theta=3, nsiz
     _check(_lib.lsa_golden_labels(_p(z), _p(seq_offsets), T, B, tau, Lc, float(p), int(theta), _p(label_out),
                                   _p(nsize_out), _p(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)))
+
+
+def lsa_indexer_train_workspace_size(L, B, total_S, d, r, n_h, d_I, dtype) -> int:
+    return int(_lib.lsa_indexer_train_workspace_size(L, B, total_S, d, r, n_h, d_I, DTYPE_CODE[dtype]))
+
+
+def lsa_indexer_train_step(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets, loss_out, g_Wdq, g_Wiuq, g_Ww,
+                           workspace, n_h, d_I, gamma=0.0, alpha=-1.0, stream=None):
+    """Loss and gradients of W^DQ, W^IUQ, W^w for one training step (see include/lsa.h)."""
+    _dev(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets, loss_out, g_Wdq, g_Wiuq, g_Ww, workspace)
+    L, B, d = h.shape
+    r = W_dq.shape[1]
+    T = K.shape[1]
+    _check(_lib.lsa_indexer_train_step(
+        _p(h), _p(W_dq), _p(W_iuq), _p(W_w), DTYPE_CODE[h.dtype], _p(K), _p(k_scale), DTYPE_CODE[K.dtype], _p(labels),
+        _p(seq_offsets), T, L, B, d, r, n_h, d_I, float(gamma), float(alpha), _p(loss_out), _p(g_Wdq), _p(g_Wiuq),
+        _p(g_Ww), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def lsa_lightning_topk_step_workspace_size(B, total_S, n_h, d_I, W) -> int:
