@@ -312,7 +312,8 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
  *   labels    [T] uint8 device (0 / 1)
  *   loss_out  [1] double device; g_Wdq [L][r][d], g_Wiuq [L][n_h*d_I][r], g_Ww [L][n_h][d] fp32
  *             device (overwritten)
- * n_h <= 64, d_I <= 128.  Workspace: lsa_indexer_train_workspace_size.  The method has no
+ * n_h <= 64, d_I <= 128, B <= 16, d and r multiples of 8.  Workspace:
+ * lsa_indexer_train_workspace_size.  The method has no
  * training kernel of its own on these pages: this is the fourth widening beyond one window.
  * ---------------------------------------------------------------------------------------- */
 size_t lsa_indexer_train_workspace_size(int L, int B, int64_t total_S, int d, int r, int n_h, int d_I,

@@ -719,6 +719,8 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
     if (!combo) return fail(LSA_ERR_UNSUPPORTED, "lsa_indexer_train_step: dtypes F32/F32, BF16/BF16 or BF16/FP8 only");
     if (n_h > train::NHMAX || d_I > train::DMAX)
         return fail(LSA_ERR_UNSUPPORTED, "lsa_indexer_train_step: n_h <= 64 and d_I <= 128");
+    if (B > train::DC_BMAX) return fail(LSA_ERR_UNSUPPORTED, "lsa_indexer_train_step: at most %d sequences", train::DC_BMAX);
+    LSA_REQUIRE(d % 8 == 0 && r % 8 == 0, "lsa_indexer_train_step: d and r must be multiples of 8");
     size_t part[8];
     const size_t need = train_ws_parts(L, B, total_S, d, r, n_h, d_I, dt, part);
     if (!workspace || workspace_bytes < need)
@@ -744,7 +746,7 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
     k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, tile_start, chunk_start, cnt);
     LSA_TRY(launched("training step: tiles"));
     const size_t smem = train::entries_smem();
-    const dim3 grid((unsigned)(total_S / train::TT + B + 1), (unsigned)L);
+    const dim3 grid((unsigned)((total_S / train::TT + B + 1 + train::TPC - 1) / train::TPC), (unsigned)L);
     const double invN = 1.0 / ((double)L * (double)total_S);
 #define LSA_TRAIN_ENTRIES(QD, KD)                                                                                  \
     do {                                                                                                           \
@@ -758,15 +760,15 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
     else LSA_TRAIN_ENTRIES(DT_BF16, DT_FP8);
 #undef LSA_TRAIN_ENTRIES
     LSA_TRY(launched("training step: entries"));
-    const int64_t ndc = (int64_t)L * B * r;
-    const int64_t n_iuq = (int64_t)L * nq * r, n_dq = (int64_t)L * r * d, n_w = (int64_t)L * n_h * d;
+    const dim3 gdc((unsigned)((r + 31) / 32), (unsigned)L);
+    const int64_t n_iuq = (int64_t)L * nq * r / 4, n_dq = (int64_t)L * r * d / 4, n_w = (int64_t)L * n_h * d / 4;
     if (dt == LSA_F32) {
-        train::k_train_dc<DT_F32><<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        train::k_train_dc<DT_F32><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
         train::k_outer<DT_F32><<<(unsigned)((n_iuq + 255) / 256), 256, 0, st>>>(dq, c, L, B, nq, r, g_Wiuq);
         train::k_outer<DT_F32><<<(unsigned)((n_dq + 255) / 256), 256, 0, st>>>(dc, h, L, B, r, d, g_Wdq);
         train::k_outer<DT_F32><<<(unsigned)((n_w + 255) / 256), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);
     } else {
-        train::k_train_dc<DT_BF16><<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        train::k_train_dc<DT_BF16><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
         train::k_outer<DT_BF16><<<(unsigned)((n_iuq + 255) / 256), 256, 0, st>>>(dq, c, L, B, nq, r, g_Wiuq);
         train::k_outer<DT_BF16><<<(unsigned)((n_dq + 255) / 256), 256, 0, st>>>(dc, h, L, B, r, d, g_Wdq);
         train::k_outer<DT_BF16><<<(unsigned)((n_w + 255) / 256), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);

@@ -3,12 +3,11 @@
 // window's golden labels, gradients of W^DQ, W^IUQ and W^w (the rounding of c and q to their
 // storage type is passed straight through).
 //
-//   k_train_entries   one CTA per (128-entry tile of one sequence, layer): the tile's keys and the
-//                     sequence's queries in shared memory (fp32); two threads per entry compute the
-//                     64 head dot products a_h (32 each), x = sum_h w_h ReLU(a_h), the loss and
-//                     g = dl/dx / N; then dw_h += g ReLU(a_h) and dq_h += (g w_h 1[a_h > 0] scale) K_s
-//                     (a 64 x 128 x 128 product per tile, two threads per key dimension), added to the
-//                     sequence's gradients with atomics.
+//   k_train_entries   TPC consecutive 128-entry tiles (global tile order) of one layer per CTA: the
+//                     tile's keys and the sequence's queries in shared memory (fp32); per entry the
+//                     64 head dot products a_h, x = sum_h w_h ReLU(a_h), the loss and g = dl/dx / N;
+//                     then dw_h += g ReLU(a_h) and dq_h += (g w_h 1[a_h > 0] scale) K_s (a 64 x 128 x
+//                     128 product per tile), added to the sequence's gradients with atomics.
 //   k_train_dc        dc = dq W^IUQ (one thread per (layer, sequence, j)).
 //   k_outer           g_W[l][m][n] = sum_b U[l][b][m] V[l][b][n]: the three weight gradients.
 #pragma once
@@ -23,164 +22,304 @@ constexpr int THREADS = 256;  // two per entry
 constexpr int NHMAX = 64;
 constexpr int DMAX = 128;
 
+// Register-tiled SIMT: in the forward, warp hg takes heads 8 hg .. 8 hg + 7 and lane takes entries
+// lane + 32 i (i < 4), so each thread holds 4 x 8 products; in the dq product warp hq takes heads
+// 8 hq .. + 7 and lane takes key dimensions lane + 32 j (j < 4).  Keys sit in shared memory as rows
+// of d_I + 1 floats (odd stride: the column reads of both phases are free of bank conflicts), the
+// queries transposed [d_I][64] and G [TT][68] (16-byte rows), so the per-head operands are float4
+// broadcasts.  A CTA walks TPC consecutive tiles and adds its dq / dw to the sequence's gradients
+// only when the sequence changes or at its end.
+constexpr int TPC = 8;
+constexpr int GP = NHMAX + 4;
+
 template <int QDT, int KDT>
-__global__ void __launch_bounds__(THREADS) k_train_entries(const void *__restrict__ q, const float *__restrict__ w,
-                                                           const void *__restrict__ K, const float *__restrict__ ksc,
-                                                           const uint8_t *__restrict__ labels,
-                                                           const int64_t *__restrict__ offs,
-                                                           const int *__restrict__ tile_start, int B, int64_t T,
-                                                           int n_h, int d_I, float gamma, float alpha, double invN,
-                                                           float *__restrict__ dq, float *__restrict__ dw,
-                                                           double *__restrict__ loss)
+__global__ void __launch_bounds__(THREADS, 1) k_train_entries(const void *__restrict__ q, const float *__restrict__ w,
+                                                              const void *__restrict__ K, const float *__restrict__ ksc,
+                                                              const uint8_t *__restrict__ labels,
+                                                              const int64_t *__restrict__ offs,
+                                                              const int *__restrict__ tile_start, int B, int64_t T,
+                                                              int n_h, int d_I, float gamma, float alpha, double invN,
+                                                              float *__restrict__ dq, float *__restrict__ dw,
+                                                              double *__restrict__ loss)
 {
-    extern __shared__ float sm[];
-    float *qs = sm;                                  // [n_h][d_I]
-    float *ks = qs + NHMAX * DMAX;                   // [TT][d_I + 1]
-    float *gs = ks + TT * (DMAX + 1);                // [TT][n_h + 1]
-    __shared__ float wsm[NHMAX], dwsm[NHMAX];
+    extern __shared__ __align__(16) float sm[];
+    float *qT = sm;                                  // [DMAX][NHMAX]
+    float *gs = qT + DMAX * NHMAX;                   // [TT][GP]
+    float *ks = gs + TT * GP;                        // [TT][d_I + 1]
+    __shared__ float wsm[NHMAX], xpart[THREADS / 32][TT], gsm[TT], scsm[TT];
     __shared__ double lred[THREADS / 32];
     const int l = blockIdx.y;
-    const int t = blockIdx.x;
     const int NT = tile_start[B];
-    if (t >= NT) return;
-    int lo = 0, hi = B - 1;  // the sequence of tile t
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (tile_start[mid] <= t) lo = mid;
-        else hi = mid - 1;
-    }
-    const int b = lo;
-    const int64_t off = offs[b], S = offs[b + 1] - off;
-    const int64_t s0 = (int64_t)(t - tile_start[b]) * TT;
-    const int nrow = (int)min((int64_t)TT, S - s0);
-    const int KP = d_I + 1, GP = n_h + 1;
-    // stage the queries, head weights and keys (fp32)
-    const int64_t qb = ((int64_t)l * B + b) * n_h * d_I;
-    for (int i = threadIdx.x; i < n_h * d_I; i += THREADS) qs[i] = load_elem<QDT>(q, qb + i);
-    for (int i = threadIdx.x; i < n_h; i += THREADS) {
-        wsm[i] = w[((int64_t)l * B + b) * n_h + i];
-        dwsm[i] = 0.f;
-    }
-    for (int i = threadIdx.x; i < TT * d_I; i += THREADS) {
-        const int rr = i / d_I, e = i % d_I;
-        ks[rr * KP + e] = rr < nrow ? load_elem<KDT>(K, ((int64_t)l * T + off + s0 + rr) * d_I + e) : 0.f;
-    }
-    __syncthreads();
-    // forward: thread (entry rr, half hf) takes heads hf*32 .. hf*32+31
-    const int rr = threadIdx.x >> 1, hf = threadIdx.x & 1;
-    const bool valid = rr < nrow;
-    const float scale = (KDT == DT_FP8 && valid) ? ksc[(int64_t)l * T + off + s0 + rr] : 1.f;
-    float a[32];
-#pragma unroll
-    for (int k = 0; k < 32; k++) a[k] = 0.f;
-    const int h0 = hf * 32;
-    for (int e = 0; e < d_I; e++) {
-        const float kv = ks[rr * KP + e];
-#pragma unroll
-        for (int k = 0; k < 32; k++)
-            if (h0 + k < n_h) a[k] = fmaf(qs[(h0 + k) * d_I + e], kv, a[k]);
-    }
-    float xp = 0.f;
-#pragma unroll
-    for (int k = 0; k < 32; k++) {
-        a[k] *= scale;
-        if (h0 + k < n_h) xp = fmaf(wsm[h0 + k], fmaxf(a[k], 0.f), xp);
-    }
-    const float x = xp + __shfl_xor_sync(0xffffffffu, xp, 1);  // the two halves of the entry
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int KP = d_I + 1;
+    const int hg0 = warp * 8;                        // this warp's 8 heads (both phases)
+    float dqa[8][4], dwa[8];
     double lsum = 0.0;
-    float g = 0.f;
-    if (valid) {
-        const int y = labels[off + s0 + rr] != 0;
-        const float p = 1.f / (1.f + expf(-x));
-        const float pt = y ? p : 1.f - p;
-        const float at = alpha < 0.f ? 1.f : (y ? alpha : 1.f - alpha);
-        const float lpt = y ? -log1pf(expf(-x)) : -log1pf(expf(x));
-        const float q1 = 1.f - pt;
-        float dl;
-        if (gamma == 0.f) {
-            dl = at * (y ? p - 1.f : p);
-            if (hf == 0) lsum = -(double)at * lpt;
-        } else {
-            dl = at * (gamma * powf(q1, gamma - 1.f) * lpt * pt * q1 - powf(q1, gamma) * q1) * (y ? 1.f : -1.f);
-            if (hf == 0) lsum = -(double)at * powf(q1, gamma) * lpt;
+    int cur_b = -1;
+    auto flush = [&](int bb) {
+        float *dqb = dq + ((int64_t)l * B + bb) * n_h * d_I;
+#pragma unroll
+        for (int k = 0; k < 8; k++)
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int e = lane + 32 * j;
+                if (hg0 + k < n_h && e < d_I && dqa[k][j] != 0.f) atomicAdd(dqb + (hg0 + k) * d_I + e, dqa[k][j]);
+            }
+        if (lane == 0)
+#pragma unroll
+            for (int k = 0; k < 8; k++)
+                if (hg0 + k < n_h && dwa[k] != 0.f) atomicAdd(dw + ((int64_t)l * B + bb) * n_h + hg0 + k, dwa[k]);
+    };
+    for (int tt = 0; tt < TPC; tt++) {
+        const int t = blockIdx.x * TPC + tt;
+        if (t >= NT) break;
+        int lo = 0, hi = B - 1;  // the sequence of tile t
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tile_start[mid] <= t) lo = mid;
+            else hi = mid - 1;
         }
-        g = (float)(dl * invN);
-    }
-    // G[rr][h] = g w_h 1[a_h > 0] scale;  dw_h += g ReLU(a_h)
+        const int b = lo;
+        if (b != cur_b) {
+            if (cur_b >= 0) flush(cur_b);
 #pragma unroll
-    for (int k = 0; k < 32; k++) {
-        const bool head = h0 + k < n_h;
-        if (head) gs[rr * GP + h0 + k] = (valid && a[k] > 0.f) ? g * wsm[h0 + k] * scale : 0.f;
-        float c = (valid && head) ? g * fmaxf(a[k], 0.f) : 0.f;
+            for (int k = 0; k < 8; k++) {
+                dwa[k] = 0.f;
 #pragma unroll
-        for (int o = 16; o >= 2; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);  // lanes of the same half
-        if ((threadIdx.x & 31) < 2 && head) atomicAdd(&dwsm[h0 + k], c);
+                for (int j = 0; j < 4; j++) dqa[k][j] = 0.f;
+            }
+            __syncthreads();  // the previous tile's readers of qT are done
+            const int64_t qb = ((int64_t)l * B + b) * n_h * d_I;
+            for (int i = threadIdx.x; i < DMAX * NHMAX; i += THREADS) qT[i] = 0.f;
+            __syncthreads();
+            {
+                // the queries [n_h][d_I], 16-byte vector loads issued together, stored transposed
+                constexpr int QB = QDT == DT_F32 ? 4 : 2;
+                constexpr int QPV = 16 / QB;
+                constexpr int NQV = (NHMAX * DMAX / QPV + THREADS - 1) / THREADS;
+                const int vpr = d_I / QPV;
+                const uint8_t *qp = (const uint8_t *)q + qb * QB;
+                uint4 buf[NQV];
+#pragma unroll
+                for (int v = 0; v < NQV; v++) {
+                    const int idx = threadIdx.x + v * THREADS;
+                    buf[v] = idx < n_h * vpr ? __ldg((const uint4 *)(qp + (int64_t)idx * 16)) : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int v = 0; v < NQV; v++) {
+                    const int idx = threadIdx.x + v * THREADS;
+                    if (idx < n_h * vpr) {
+                        const int hh = idx / vpr, e0 = (idx % vpr) * QPV;
+                        const uint32_t wv[4] = {buf[v].x, buf[v].y, buf[v].z, buf[v].w};
+#pragma unroll
+                        for (int j = 0; j < QPV; j++)
+                            qT[(e0 + j) * NHMAX + hh] = QDT == DT_F32 ? __uint_as_float(wv[j])
+                                                                     : bf16_bits_to_float((unsigned short)(wv[j >> 1] >> (16 * (j & 1))));
+                    }
+                }
+            }
+            for (int i = threadIdx.x; i < NHMAX; i += THREADS) wsm[i] = i < n_h ? w[((int64_t)l * B + b) * n_h + i] : 0.f;
+            cur_b = b;
+        }
+        const int64_t off = offs[b], S = offs[b + 1] - off;
+        const int64_t s0 = (int64_t)(t - tile_start[b]) * TT;
+        const int nrow = (int)min((int64_t)TT, S - s0);
+        __syncthreads();  // qT / wsm ready; the previous tile's readers of ks / gs are done
+        {
+            // 16-byte vector loads, all issued before any conversion (d_I is a multiple of EPV)
+            constexpr int EB = KDT == DT_F32 ? 4 : (KDT == DT_BF16 ? 2 : 1);
+            constexpr int EPV = 16 / EB;
+            constexpr int NV = (TT * DMAX / EPV + THREADS - 1) / THREADS;
+            const int vpr = d_I / EPV;
+            const uint8_t *kb = (const uint8_t *)K + ((int64_t)l * T + off + s0) * d_I * EB;
+            uint4 buf[NV];
+#pragma unroll
+            for (int v = 0; v < NV; v++) {
+                const int idx = threadIdx.x + v * THREADS;
+                const int rr = idx / vpr;
+                buf[v] = make_uint4(0u, 0u, 0u, 0u);
+                if (idx < TT * vpr && rr < nrow) buf[v] = __ldg((const uint4 *)(kb + (int64_t)idx * 16));
+            }
+#pragma unroll
+            for (int v = 0; v < NV; v++) {
+                const int idx = threadIdx.x + v * THREADS;
+                if (idx < TT * vpr) {
+                    const int rr = idx / vpr, e0 = (idx % vpr) * EPV;
+                    const uint32_t wv[4] = {buf[v].x, buf[v].y, buf[v].z, buf[v].w};
+                    float *dst = ks + rr * KP + e0;
+#pragma unroll
+                    for (int j = 0; j < EPV; j++) {
+                        float f;
+                        if (KDT == DT_F32) f = __uint_as_float(wv[j]);
+                        else if (KDT == DT_BF16) f = bf16_bits_to_float((unsigned short)(wv[j >> 1] >> (16 * (j & 1))));
+                        else f = e4m3_to_float((unsigned char)(wv[j >> 2] >> (8 * (j & 3))));
+                        dst[j] = f;
+                    }
+                }
+            }
+        }
+        if (threadIdx.x < TT)
+            scsm[threadIdx.x] = (KDT == DT_FP8 && (int)threadIdx.x < nrow) ? ksc[(int64_t)l * T + off + s0 + threadIdx.x] : 1.f;
+        __syncthreads();
+        // forward: a[i][k] = scale (q_{hg0+k} . K_{lane+32i})
+        float a[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+#pragma unroll
+            for (int k = 0; k < 8; k++) a[i][k] = 0.f;
+        for (int e = 0; e < d_I; e++) {
+            const float4 q0 = *(const float4 *)(qT + e * NHMAX + hg0), q1 = *(const float4 *)(qT + e * NHMAX + hg0 + 4);
+            const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float kv = ks[(lane + 32 * i) * KP + e];
+#pragma unroll
+                for (int k = 0; k < 8; k++) a[i][k] = fmaf(qv[k], kv, a[i][k]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float sc = scsm[lane + 32 * i];
+            float xp = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; k++) {
+                a[i][k] *= sc;
+                xp = fmaf(wsm[hg0 + k], fmaxf(a[i][k], 0.f), xp);
+            }
+            xpart[warp][lane + 32 * i] = xp;
+        }
+        __syncthreads();
+        // per entry: x, loss, g = dl/dx / N
+        if (threadIdx.x < TT) {
+            const int rr = threadIdx.x;
+            float g = 0.f;
+            if (rr < nrow) {
+                float x = 0.f;
+#pragma unroll
+                for (int wv = 0; wv < THREADS / 32; wv++) x += xpart[wv][rr];
+                const int y = labels[off + s0 + rr] != 0;
+                const float p = 1.f / (1.f + expf(-x));
+                const float pt = y ? p : 1.f - p;
+                const float at = alpha < 0.f ? 1.f : (y ? alpha : 1.f - alpha);
+                const float lpt = y ? -log1pf(expf(-x)) : -log1pf(expf(x));
+                const float q1 = 1.f - pt;
+                float dl;
+                if (gamma == 0.f) {
+                    dl = at * (y ? p - 1.f : p);
+                    lsum -= (double)at * lpt;
+                } else {
+                    dl = at * (gamma * powf(q1, gamma - 1.f) * lpt * pt * q1 - powf(q1, gamma) * q1) * (y ? 1.f : -1.f);
+                    lsum -= (double)at * powf(q1, gamma) * lpt;
+                }
+                g = (float)(dl * invN);
+            }
+            gsm[rr] = g;
+        }
+        __syncthreads();
+        // G[r][h] = g w_h 1[a > 0] scale_r;  dw_h += g ReLU(a)
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int rr = lane + 32 * i;
+            const float g = gsm[rr], sc = scsm[rr];
+#pragma unroll
+            for (int k = 0; k < 8; k++) {
+                gs[rr * GP + hg0 + k] = a[i][k] > 0.f ? g * wsm[hg0 + k] * sc : 0.f;
+                float c = g * fmaxf(a[i][k], 0.f);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+                dwa[k] += c;  // every lane holds the warp's sum; lane 0 adds it at the flush
+            }
+        }
+        __syncthreads();
+        // dq[h][e] += sum_r G[r][h] K[r][e]
+        for (int rr = 0; rr < nrow; rr++) {
+            const float4 g0 = *(const float4 *)(gs + rr * GP + hg0), g1 = *(const float4 *)(gs + rr * GP + hg0 + 4);
+            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int e = lane + 32 * j;
+                const float kv = e < d_I ? ks[rr * KP + e] : 0.f;
+#pragma unroll
+                for (int k = 0; k < 8; k++) dqa[k][j] = fmaf(gv[k], kv, dqa[k][j]);
+            }
+        }
     }
+    if (cur_b >= 0) flush(cur_b);
     // loss
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    if ((threadIdx.x & 31) == 0) lred[threadIdx.x >> 5] = lsum;
+    if (lane == 0) lred[warp] = lsum;
     __syncthreads();
-    // dq[h][e] += sum_rr G[rr][h] K[rr][e]: thread (e, half) takes heads half*32 .. +31
-    {
-        const int e = threadIdx.x >> 1, hh0 = (threadIdx.x & 1) * 32;
-        if (e < d_I) {
-            float acc[32];
-#pragma unroll
-            for (int k = 0; k < 32; k++) acc[k] = 0.f;
-            for (int r2 = 0; r2 < nrow; r2++) {
-                const float kv = ks[r2 * KP + e];
-#pragma unroll
-                for (int k = 0; k < 32; k++)
-                    if (hh0 + k < n_h) acc[k] = fmaf(gs[r2 * GP + hh0 + k], kv, acc[k]);
-            }
-            float *dqb = dq + ((int64_t)l * B + b) * n_h * d_I;
-#pragma unroll
-            for (int k = 0; k < 32; k++)
-                if (hh0 + k < n_h && acc[k] != 0.f) atomicAdd(dqb + (hh0 + k) * d_I + e, acc[k]);
-        }
-    }
-    if (threadIdx.x < n_h) atomicAdd(dw + ((int64_t)l * B + b) * n_h + threadIdx.x, dwsm[threadIdx.x]);
     if (threadIdx.x == 0) {
-        double s = 0.0;
-        for (int i = 0; i < THREADS / 32; i++) s += lred[i];
-        atomicAdd(loss, s * invN);
+        double s2 = 0.0;
+        for (int i = 0; i < THREADS / 32; i++) s2 += lred[i];
+        if (s2 != 0.0) atomicAdd(loss, s2 * invN);
     }
 }
 
-// dc[l][b][j] = sum_o dq[l][b][o] W_iuq[l][o][j]
+// dc[l][b][j] = sum_o dq[l][b][o] W_iuq[l][o][j]: one CTA per (layer, 32 columns j); warp w sums the
+// rows o = w + 8 k for all B sequences at once (lane = column, so each W^IUQ row segment is one
+// coalesced read and W^IUQ is read once), then the 8 partial sums meet in shared memory.
+constexpr int DC_BMAX = 16;
+
 template <int DT>
 __global__ void __launch_bounds__(256) k_train_dc(const float *__restrict__ dq, const void *__restrict__ W_iuq, int L,
                                                   int B, int nq, int r, float *__restrict__ dc)
 {
-    const int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    if (idx >= (int64_t)L * B * r) return;
-    const int j = (int)(idx % r);
-    const int64_t lb = idx / r;
-    const int l = (int)(lb / B);
-    const float *dqb = dq + lb * nq;
-    float acc = 0.f;
-    for (int o = 0; o < nq; o++) acc = fmaf(dqb[o], load_elem<DT>(W_iuq, ((int64_t)l * nq + o) * r + j), acc);
-    dc[idx] = acc;
+    __shared__ float part[8][DC_BMAX][32];
+    const int l = blockIdx.y, j = blockIdx.x * 32 + (threadIdx.x & 31), warp = threadIdx.x >> 5;
+    float acc[DC_BMAX];
+#pragma unroll
+    for (int bb = 0; bb < DC_BMAX; bb++) acc[bb] = 0.f;
+    const float *dql = dq + (int64_t)l * B * nq;
+    if (j < r) {
+#pragma unroll 4
+        for (int o = warp; o < nq; o += 8) {
+            const float wv = load_elem<DT>(W_iuq, ((int64_t)l * nq + o) * r + j);
+#pragma unroll
+            for (int bb = 0; bb < DC_BMAX; bb++)
+                if (bb < B) acc[bb] = fmaf(__ldg(dql + (int64_t)bb * nq + o), wv, acc[bb]);
+        }
+    }
+#pragma unroll
+    for (int bb = 0; bb < DC_BMAX; bb++) part[warp][bb][threadIdx.x & 31] = acc[bb];
+    __syncthreads();
+    for (int i = threadIdx.x; i < B * 32; i += 256) {
+        const int bb = i / 32, jj = i % 32;
+        if (blockIdx.x * 32 + jj < r) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w8 = 0; w8 < 8; w8++) sum += part[w8][bb][jj];
+            dc[((int64_t)l * B + bb) * r + blockIdx.x * 32 + jj] = sum;
+        }
+    }
 }
 
-// out[l][m][n] = sum_b U[l][b][m] V[l][b][n]; U fp32, V of type VDT
+// out[l][m][n] = sum_b U[l][b][m] V[l][b][n] (U fp32, V of type VDT); 4 consecutive n per thread
+// (N is a multiple of 4), one 16-byte store each.
 template <int VDT>
 __global__ void __launch_bounds__(256) k_outer(const float *__restrict__ U, const void *__restrict__ V, int L, int B,
                                                int M, int N, float *__restrict__ out)
 {
     const int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    if (idx >= (int64_t)L * M * N) return;
-    const int n = (int)(idx % N);
-    const int64_t lm = idx / N;
+    const int N4 = N / 4;
+    if (idx >= (int64_t)L * M * N4) return;
+    const int n = (int)(idx % N4) * 4;
+    const int64_t lm = idx / N4;
     const int m = (int)(lm % M), l = (int)(lm / M);
-    float acc = 0.f;
-    for (int b = 0; b < B; b++)
-        acc = fmaf(U[((int64_t)l * B + b) * M + m], load_elem<VDT>(V, ((int64_t)l * B + b) * N + n), acc);
-    out[idx] = acc;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int b = 0; b < B; b++) {
+        const float u = __ldg(U + ((int64_t)l * B + b) * M + m);
+        const int64_t vb = ((int64_t)l * B + b) * N + n;
+        acc.x = fmaf(u, load_elem<VDT>(V, vb), acc.x);
+        acc.y = fmaf(u, load_elem<VDT>(V, vb + 1), acc.y);
+        acc.z = fmaf(u, load_elem<VDT>(V, vb + 2), acc.z);
+        acc.w = fmaf(u, load_elem<VDT>(V, vb + 3), acc.w);
+    }
+    *(float4 *)(out + ((int64_t)l * M + m) * N + n) = acc;
 }
 
-inline size_t entries_smem(void) { return sizeof(float) * ((size_t)NHMAX * DMAX + (size_t)TT * (DMAX + 1) + (size_t)TT * (NHMAX + 1)); }
+inline size_t entries_smem(void) { return sizeof(float) * ((size_t)DMAX * NHMAX + (size_t)TT * GP + (size_t)TT * (DMAX + 1)); }
 
 }  // namespace train
 
