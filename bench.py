@@ -50,6 +50,8 @@ def parse_args():
     p.add_argument("--no-decode-steps", action="store_true", help="skip the per-step decode measurement")
     p.add_argument("--no-golden", action="store_true", help="skip the golden-label measurement")
     p.add_argument("--no-train", action="store_true", help="skip the training-step measurement")
+    p.add_argument("--only", choices=["golden", "train"], default=None,
+                   help="run only this self-contained measurement (one GPU) and print its JSON line")
     return p.parse_args()
 
 
@@ -623,6 +625,12 @@ def main():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
     device = torch.device("cuda", local)
+    if args.only:
+        import sparse_kv_cache_memoryindexer_b200 as lsa
+        torch.cuda.set_device(device)
+        res = measure_golden(lsa, device) if args.only == "golden" else measure_train(lsa, device)
+        print(json.dumps(dict(res, only=args.only)), flush=True)
+        return 0
     if world > 1:
         torch.cuda.set_device(device)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
