@@ -200,9 +200,33 @@ def cpu_baseline(wl, n_entries, steps=1):
         oracle_step(oracle, sw, inp)
         times.append(time.perf_counter() - t0)
     units = sw.L * sw.total_S
-    return {"value": units / statistics.mean(times), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+    cores = oracle.threads()
+    # the same oracle on one core, over a smaller sample of the same workload
+    sw1 = oracle_sample_workload(wl, max(1024, n_entries // 16))
+    inp1 = synth.make_inputs(sw1)
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle_step(oracle, sw1, inp1)
+        one = sw1.L * sw1.total_S / (time.perf_counter() - t0)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": units / statistics.mean(times), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "value_1core": one, "cpu_model": cpu_model(),
             "sample": f"one sequence of {sw.total_S} entries x {sw.L} layers of {wl.name} (same dims/dtypes), "
-                      f"whole path incl. S1 projection and Top-k of {sw.tau} queries; mean of {steps} run(s)"}
+                      f"whole path incl. S1 projection and Top-k of {sw.tau} queries; mean of {steps} run(s); "
+                      f"value_1core: {sw1.total_S} entries on one core"}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 # ------------------------------------------------------------------------------------ model of the bytes
@@ -573,7 +597,8 @@ def run_lsa(args, rank, world, device):
             "score_select_entries_per_s": world * wl.L * T / (sel_ms * 1e-3),
             "roofline": dict(kernel="score_select (index score + threshold + OR + compaction, one stream)",
                              bound="hbm", achieved=score_gbs, peak=peaks["hbm_gbs"], unit="GB/s",
-                             frac=score_gbs / peaks["hbm_gbs"], traffic=traffic,
+                             frac=score_gbs / peaks["hbm_gbs"], frac_of_nominal_8tbs=score_gbs / 8000.0,
+                             traffic=traffic,
                              traffic_note=None if traffic is None else
                              "ncu DRAM bytes of k_score_tc on %s, scaled by entries" % traffic_src,
                              bytes_per_launch=alg["score_bytes"], peak_source=peaks["source"]),
