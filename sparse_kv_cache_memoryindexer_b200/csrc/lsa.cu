@@ -16,6 +16,7 @@
 #include "proj_tc.cuh"
 #include "golden.cuh"
 #include "train.cuh"
+#include "step_select.cuh"
 #include "topk.cuh"
 
 using namespace lsa;
@@ -546,21 +547,40 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
 // ------------------------------------------------------------------------------ stage 5, one decode step
 
 // Workspace of lsa_lightning_topk_step: [item_start B+1, counter][Y: 4 * total_S][tail: B * W]
-// [queries: B * 4 * n_h * d_I (4-byte elements)][weights: B * 4 * n_h].
-static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[5])
+// [queries: B * 4 * n_h * d_I (4-byte elements)][weights: B * 4 * n_h][select: chunk starts, state,
+// histograms, chunk counts, the selection (LSA_MAX_TOPK per sequence)].
+static int64_t step_max_chunks(int B, int64_t total_S, int W)
+{
+    return (total_S + (int64_t)B * W) / stepsel::CH + B + 1;
+}
+
+static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[5])
+{
+    const int64_t mc = step_max_chunks(B, total_S, W);
+    sp[0] = align_up(sizeof(int) * (size_t)(B + 1), 256);
+    sp[1] = align_up(sizeof(uint32_t) * 4 * (size_t)B, 256);
+    sp[2] = align_up(sizeof(int) * 256 * (size_t)B, 256);
+    sp[3] = align_up(sizeof(int) * 2 * (size_t)mc, 256);
+    sp[4] = align_up(sizeof(unsigned long long) * (size_t)B * LSA_MAX_TOPK, 256);
+    return sp[0] + sp[1] + sp[2] + sp[3] + sp[4];
+}
+
+static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[6])
 {
     part[0] = align_up(sizeof(int) * (size_t)(B + 2), 256);
     part[1] = align_up(sizeof(float) * 4 * (size_t)(total_S > 0 ? total_S : 1), 256);
     part[2] = align_up(sizeof(float) * (size_t)B * (W > 0 ? W : 1), 256);
     part[3] = align_up((size_t)4 * B * 4 * n_h * d_I, 256);
     part[4] = align_up(sizeof(float) * (size_t)B * 4 * n_h, 256);
-    return part[0] + part[1] + part[2] + part[3] + part[4];
+    size_t sp[5];
+    part[5] = step_sel_parts(B, total_S, W, sp);
+    return part[0] + part[1] + part[2] + part[3] + part[4] + part[5];
 }
 
 size_t lsa_lightning_topk_step_workspace_size(int B, int64_t total_S, int n_h, int d_I, int W)
 {
     if (B <= 0 || total_S < 0 || n_h <= 0 || d_I <= 0 || W < 0) return 0;
-    size_t part[5];
+    size_t part[6];
     return step_ws_parts(B, total_S, n_h, d_I, W, part);
 }
 
@@ -587,7 +607,7 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk_step: n_h must be <= 128");
     if (d_I != 32 && d_I != 64 && d_I != 128)
         return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk_step: d_I must be 32, 64 or 128");
-    size_t part[5];
+    size_t part[6];
     const size_t need = step_ws_parts(B, total_S, n_h, d_I, W, part);
     if (!workspace || workspace_bytes < need)
         return fail(LSA_ERR_WORKSPACE, "lsa_lightning_topk_step: workspace needs %zu bytes", need);
@@ -627,13 +647,37 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
                                                                  n_h, d_I, tail);
         LSA_TRY(launched("decode step: window entries"));
     }
+    // the select, spread over chunks of candidates (see step_select.cuh)
+    size_t sp[5];
+    step_sel_parts(B, total_S, W, sp);
+    char *sb = p + part[0] + part[1] + part[2] + part[3] + part[4];
+    int *chunk_start = (int *)sb;
+    uint32_t *state = (uint32_t *)(sb + sp[0]);
+    int *ghist = (int *)(sb + sp[0] + sp[1]);
+    int *gtc = (int *)(sb + sp[0] + sp[1] + sp[2]);
+    const int64_t mc = step_max_chunks(B, total_S, W);
+    int *eqc = gtc + mc;
+    unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
+    const int32_t *tcnt = W > 0 ? win_count : nullptr;
+    stepsel::k_ss_setup<<<1, 1024, 0, st>>>(count, seq_offsets, tcnt, W, B, k, chunk_start, state, ghist);
+    for (int pass = 0; pass < 4; pass++) {
+        stepsel::k_ss_hist<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B,
+                                                                 chunk_start, state, pass, ghist);
+        stepsel::k_ss_digit<<<(unsigned)B, 256, 0, st>>>(state, ghist, pass);
+    }
+    stepsel::k_ss_count<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
+                                                              state, gtc, eqc);
+    stepsel::k_ss_scan<<<(unsigned)B, 32, 0, st>>>(chunk_start, gtc, eqc);
+    stepsel::k_ss_write<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
+                                                              state, gtc, eqc, LSA_MAX_TOPK, sel);
     int kpow2 = 1;
     while (kpow2 < k) kpow2 <<= 1;
     const size_t smem = sizeof(unsigned long long) * (size_t)kpow2;
-    LSA_TRY(set_smem(k_topk_select<true>, smem));
-    k_topk_select<true><<<(unsigned)B, SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, 1, k, kpow2, topk_idx,
-                                                               topk_score, tail, W > 0 ? win_count : nullptr, W, TQ);
+    LSA_TRY(set_smem(stepsel::k_ss_sort, smem));
+    stepsel::k_ss_sort<<<(unsigned)B, stepsel::SORT_TH, smem, st>>>(sel, LSA_MAX_TOPK, state, idx, count, seq_offsets,
+                                                                   k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
+    g_launches.fetch_add(11, std::memory_order_relaxed);
     return ok();
 }
 
