@@ -3,11 +3,14 @@
 //     y_{b,i,j} = sum_h w'_{b,i,h} ReLU(scale_j q'_{b,i,h} . hot_K_j),   j < count[b].
 //
 // MMA orientation: the hot keys of sequence b are the A operand (M = 128 keys per tile,
-// K = d_I = 128); the queries of a group of NQ = 4 decode steps are the B operand (N = 4 x 64
-// heads = 256), so each TMEM lane (one key) holds its 256 head dot products and the weighted
-// head sums of the 4 queries run inside one thread.  Scores go to Y[tau*off_b + i*S_b + j].
+// K = d_I = 128); the queries of a group of nq decode steps are the B operand (N = nq x 64 heads:
+// 256 for the batched call, nq = 4; 64 for one decode step, nq = 1), so each TMEM lane (one key)
+// holds its head dot products and the weighted head sums of the group's queries run inside one
+// thread.  Scores go to Y[tau*off_b + i*S_b + j].  With nq = 1 the query buffers shrink to a
+// quarter and the freed shared memory holds more key stages (the one-query call has no key reuse
+// and is bound by keys in flight, not by the tensor core).
 //
-// Work item = (sequence b, chunk of CH key tiles, query group g); items of one chunk are
+// Work item = (sequence b, chunk of ch key tiles, query group g); items of one chunk are
 // consecutive so that CTAs working at the same time share the chunk's keys in L2.  CTAs claim
 // items from a global counter (not a fixed share each), so that CTAs slowed by other kernels on
 // their SM (the host-link row gather runs beside this kernel) take fewer items instead of setting
@@ -24,13 +27,13 @@ namespace lsa {
 
 namespace li {
 
-constexpr int NQ = 4;              // decode queries per MMA
+constexpr int NQ = 4;              // decode queries per MMA (batched call; one decode step: 1)
 constexpr int NH = 64;             // heads
-constexpr int NCOL = NQ * NH;      // MMA N = 256
-constexpr int CH = 16;             // key tiles per work item
+constexpr int NCOL = NQ * NH;      // MMA N = 256 (TMEM columns per accumulator slot)
+constexpr int CH = 16;             // key tiles per work item (batched call; one decode step: CH_STEP)
+constexpr int CH_STEP = 4;
 constexpr int MAX_STAGES = 8;
 constexpr int NRING = 4;           // claimed items in flight inside a CTA
-constexpr uint32_t IDESC = tc::idesc_bf16(128, NCOL);
 
 struct Params {
     const float *wd;         // [B][tau][64]
@@ -42,16 +45,17 @@ struct Params {
     float *Y;                // [tau*T]
     int64_t T;
     int B, tau, groups, stages;
+    int ch;                  // key tiles per work item
 };
 
 struct Smem {
     uint32_t kraw, qbuf, sw, bars, misc, total;
-    __host__ __device__ static Smem plan(int stages)
+    __host__ __device__ static Smem plan(int stages, int nq)
     {
         Smem s;
         s.kraw = 0;
         s.qbuf = s.kraw + 128 * 256 * stages;
-        s.sw = s.qbuf + 2 * NCOL * tc::DI * 2;
+        s.sw = s.qbuf + 2 * nq * NH * tc::DI * 2;
         s.bars = s.sw + 8 * 2 * NH * 4;
         s.misc = s.bars + 8 * (4 * MAX_STAGES + 8 + 2 * NRING);
         s.total = s.misc + 64 + 1024;
@@ -82,9 +86,9 @@ __device__ __forceinline__ int fetched_count(const Params &p, int b, int64_t &S)
     return F < 0 ? 0 : (F > S ? (int)S : F);
 }
 
-// work items per sequence: ceil(ceil(F/128)/CH) chunks x groups.  One block.
+// work items per sequence: ceil(ceil(F/128)/ch) chunks x groups.  One block.
 __global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
-                                                   int B, int groups, int *__restrict__ item_start,
+                                                   int B, int groups, int ch, int *__restrict__ item_start,
                                                    int *__restrict__ item_counter)
 {
     __shared__ int warp_tot[32];
@@ -105,7 +109,7 @@ __global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ c
             if (F < 0 || F > S) flag(ERRF_COUNT);
             F = F < 0 ? 0 : (F > S ? (int)S : F);
             const int tiles = (F + TILE - 1) / TILE;
-            n = ((tiles + CH - 1) / CH) * groups;
+            n = ((tiles + ch - 1) / ch) * groups;
         }
         const int inc = warp_incl_scan(n);
         if (lane == 31) warp_tot[warp] = inc;
@@ -123,13 +127,17 @@ __global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ c
     }
 }
 
+template <int NQV>  // queries per group: NQ (batched call) or 1 (one decode step)
 __global__ void __launch_bounds__(320, 1)
     k_li_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, Params p)
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const Smem sp = Smem::plan(p.stages);
+    const Smem sp = Smem::plan(p.stages, NQV);
+    constexpr int ncol = NQV * NH;                          // MMA N
+    constexpr uint32_t qbytes = (uint32_t)ncol * DI * 2;    // one query slot
+    constexpr uint32_t idesc = tc::idesc_bf16(128, ncol);
     const uint32_t sbase = smem_u32(base);
     const uint32_t kraw = sbase + sp.kraw, qbuf = sbase + sp.qbuf;
     float *sw = (float *)(base + sp.sw);
@@ -205,15 +213,15 @@ __global__ void __launch_bounds__(320, 1)
                 int64_t S;
                 const int F = fetched_count(p, w.b, S);
                 const int ntiles = (F + TILE - 1) / TILE;
-                const int t0 = w.c * CH, t1 = min(ntiles, t0 + CH);
+                const int t0 = w.c * p.ch, t1 = min(ntiles, t0 + p.ch);
                 qslot ^= 1;
                 if (!mbar_wait(qempty(qslot), (quse[qslot] & 1) ^ 1, abort_flag)) { ok = false; break; }
                 quse[qslot]++;
-                mbar_expect_tx(qfull(qslot), NCOL * DI * 2);
-                const uint32_t qd = qbuf + (uint32_t)qslot * NCOL * DI * 2;
-                const int qrow = (w.b * p.tau + NQ * w.g) * NH;
+                mbar_expect_tx(qfull(qslot), qbytes);
+                const uint32_t qd = qbuf + (uint32_t)qslot * qbytes;
+                const int qrow = (w.b * p.tau + NQV * w.g) * NH;
                 tma_load_2d(qd, &qmap, 0, qrow, qfull(qslot));
-                tma_load_2d(qd + NCOL * 128, &qmap, 64, qrow, qfull(qslot));
+                tma_load_2d(qd + (uint32_t)ncol * 128, &qmap, 64, qrow, qfull(qslot));
                 const int64_t off = __ldg(p.offs + w.b);
                 for (int kt = t0; kt < t1; kt++) {
                     if (!mbar_wait(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
@@ -253,11 +261,11 @@ __global__ void __launch_bounds__(320, 1)
                 int64_t S;
                 const int F = fetched_count(p, w.b, S);
                 const int ntiles = (F + TILE - 1) / TILE;
-                const int t0 = w.c * CH, t1 = min(ntiles, t0 + CH);
+                const int t0 = w.c * p.ch, t1 = min(ntiles, t0 + p.ch);
                 qslot ^= 1;
                 if (!mbar_wait(qfull(qslot), quse[qslot] & 1, abort_flag)) { ok = false; break; }
                 quse[qslot]++;
-                const uint32_t b_base = qbuf + (uint32_t)qslot * NCOL * DI * 2;
+                const uint32_t b_base = qbuf + (uint32_t)qslot * qbytes;
                 for (int kt = t0; kt < t1; kt++) {
                     if (!mbar_wait(full(stage), phase, abort_flag)) { ok = false; break; }
                     const uint32_t a_base = kraw + (uint32_t)stage * 128 * 256;
@@ -267,8 +275,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int kk = 0; kk < DI / 16; kk++) {
                         const uint32_t ka = a_base + (uint32_t)(kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32;
-                        const uint32_t kb = b_base + (uint32_t)(kk >> 2) * (NCOL * 128) + (uint32_t)(kk & 3) * 32;
-                        mma_bf16(d, sdesc(ka), sdesc(kb), IDESC, kk > 0 ? 1u : 0u);
+                        const uint32_t kb = b_base + (uint32_t)(kk >> 2) * ((uint32_t)ncol * 128) + (uint32_t)(kk & 3) * 32;
+                        mma_bf16(d, sdesc(ka), sdesc(kb), idesc, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(empty(stage));
                     if (++stage == p.stages) { stage = 0; phase ^= 1; }
@@ -284,6 +292,7 @@ __global__ void __launch_bounds__(320, 1)
         // ------------------------------------------------------------- epilogue
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
         const int half = (warp - 2) >> 2;        // queries 2*half, 2*half+1 of the group
+        const int nqw = NQV >= 4 ? 2 : (half == 0 ? NQV : 0);  // of them in the group
         float *myw = sw + (size_t)(warp - 2) * 2 * NH;
         int acc = 0;
         uint32_t accphase = 0;
@@ -301,10 +310,10 @@ __global__ void __launch_bounds__(320, 1)
             int64_t S;
             const int F = fetched_count(p, w.b, S);
             const int ntiles = (F + TILE - 1) / TILE;
-            const int t0 = w.c * CH, t1 = min(ntiles, t0 + CH);
-            const int i0 = NQ * w.g + 2 * half;  // first of this warp's two queries
+            const int t0 = w.c * p.ch, t1 = min(ntiles, t0 + p.ch);
+            const int i0 = NQV * w.g + 2 * half;  // first of this warp's queries
             __syncwarp();
-            for (int t = lane; t < 2 * NH; t += 32)
+            for (int t = lane; t < nqw * NH; t += 32)
                 myw[t] = __ldg(p.wd + ((int64_t)w.b * p.tau + i0 + t / NH) * NH + (t % NH));
             __syncwarp();
             const int64_t off = __ldg(p.offs + w.b);
@@ -320,14 +329,20 @@ __global__ void __launch_bounds__(320, 1)
                     if (!(sc >= 0.f)) flag(ERRF_SCALE);
                 }
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * NCOL + 128 * half;
-                float y[2];
+                float y[2] = {0.f, 0.f};
+                if (nqw == 0) {  // nothing of this warp in the slot: release it at once
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty(acc));
+                }
 #pragma unroll
                 for (int qq = 0; qq < 2; qq++) {
+                    if (qq >= nqw) break;
                     float v0[32], v1[32];
                     tmem_ld32(taddr + qq * NH, v0);
                     tmem_ld32(taddr + qq * NH + 32, v1);
                     tmem_wait_ld();
-                    if (qq == 1) {
+                    if (qq == nqw - 1) {  // the slot's last read by this warp
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(tempty(acc));
@@ -351,8 +366,8 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 if (++acc == 2) { acc = 0; accphase ^= 1; }
                 if (valid) {
-                    Yb[(int64_t)i0 * S + j] = y[0];
-                    Yb[(int64_t)(i0 + 1) * S + j] = y[1];
+                    if (nqw > 0) Yb[(int64_t)i0 * S + j] = y[0];
+                    if (nqw > 1) Yb[(int64_t)(i0 + 1) * S + j] = y[1];
                 }
             }
         }
@@ -370,26 +385,31 @@ __global__ void __launch_bounds__(320, 1)
 
 // ------------------------------------------------------------------------------------ host side
 
-inline bool li_tc_supported(int n_h, int d_I, int tau, int kdt)
+// nq: decode queries per MMA group, li::NQ for the batched call, 1 for one decode step.
+inline bool li_tc_supported(int n_h, int d_I, int tau, int kdt, int nq = li::NQ)
 {
-    return n_h == li::NH && d_I == tc::DI && tau % li::NQ == 0 && (kdt == DT_BF16 || kdt == DT_FP8) && tc_available();
+    return n_h == li::NH && d_I == tc::DI && (nq == li::NQ || nq == 1) && tau % nq == 0 &&
+           (kdt == DT_BF16 || kdt == DT_FP8) && tc_available();
 }
 
 // hotK: bf16 [T][128] (decoded E4M3 codes when hsc is given).  item_start: device [B+1];
 // item_counter: one device int (zeroed by the planner).
-// Launches the item planner and the scoring kernel; *launches counts them.
+// nq: queries per MMA group (li_tc_supported).  Launches the item planner and the scoring kernel;
+// *launches counts them.
 inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK, const float *hsc,
-                               const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, float *Y,
+                               const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, int nq, float *Y,
                                int *item_start, int *item_counter, int sms, cudaStream_t st, int *launches)
 {
     using namespace li;
     *launches = 0;
-    k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / NQ, item_start, item_counter);
+    if (nq != NQ && nq != 1) return LSA_ERR_UNSUPPORTED;
+    const int ch = nq == NQ ? CH : CH_STEP;
+    k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / nq, ch, item_start, item_counter);
     (*launches)++;
     if (T == 0) return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
     CUtensorMap kmap, qmap;
     bool ok = make_map_2d(&kmap, hotK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, tc::DI, 64, 128);
-    ok = ok && make_map_2d(&qmap, qd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)B * tau * NH, tc::DI, 64, NCOL);
+    ok = ok && make_map_2d(&qmap, qd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)B * tau * NH, tc::DI, 64, nq * NH);
     if (!ok) return LSA_ERR_CUDA;
     Params p;
     p.wd = wd;
@@ -402,15 +422,17 @@ inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK
     p.T = T;
     p.B = B;
     p.tau = tau;
-    p.groups = tau / NQ;
+    p.groups = tau / nq;
+    p.ch = ch;
     const int max_smem = 227 * 1024;
     p.stages = MAX_STAGES;
-    while (p.stages > 2 && Smem::plan(p.stages).total > (uint32_t)max_smem) p.stages--;
-    const uint32_t smem = Smem::plan(p.stages).total;
+    while (p.stages > 2 && Smem::plan(p.stages, nq).total > (uint32_t)max_smem) p.stages--;
+    const uint32_t smem = Smem::plan(p.stages, nq).total;
     if (smem > (uint32_t)max_smem) return LSA_ERR_UNSUPPORTED;
-    cudaError_t e = cudaFuncSetAttribute(k_li_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = nq == NQ ? k_li_tc<NQ> : k_li_tc<1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return LSA_ERR_CUDA;
-    k_li_tc<<<sms, 320, smem, st>>>(kmap, qmap, p);
+    kern<<<sms, 320, smem, st>>>(kmap, qmap, p);
     (*launches)++;
     e = cudaGetLastError();
     return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;

@@ -522,8 +522,8 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     if (li_tc_supported(n_h, d_I, tau, kdt)) {
         LSA_REQUIRE(aligned(q_dec, 16) && aligned(hot_K, 16), "lsa_lightning_topk: q_dec and hot_K must be 16-byte aligned");
         int n = 0;
-        const lsa_status s = launch_li_tc(q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, Y,
-                                          item_start, item_counter, num_sms(), st, &n);
+        const lsa_status s = launch_li_tc(q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, li::NQ,
+                                          Y, item_start, item_counter, num_sms(), st, &n);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK) return fail(s, "lsa_lightning_topk: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
     } else {
@@ -546,9 +546,9 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
 
 // ------------------------------------------------------------------------------ stage 5, one decode step
 
-// Workspace of lsa_lightning_topk_step: [item_start B+1, counter][Y: 4 * total_S][tail: B * W]
-// [queries: B * 4 * n_h * d_I (4-byte elements)][weights: B * 4 * n_h][select: chunk starts, state,
-// histograms, chunk counts, the selection (LSA_MAX_TOPK per sequence)].
+// Workspace of lsa_lightning_topk_step: [item_start B+1, counter][Y: total_S][tail: B * W]
+// [queries: B * n_h * d_I (4-byte elements)][weights: B * n_h][select: chunk starts, state,
+// histograms and pass counters, chunk counts, the selection (LSA_MAX_TOPK per sequence)].
 static int64_t step_max_chunks(int B, int64_t total_S, int W)
 {
     return (total_S + (int64_t)B * W) / stepsel::CH + B + 1;
@@ -559,7 +559,7 @@ static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[5])
     const int64_t mc = step_max_chunks(B, total_S, W);
     sp[0] = align_up(sizeof(int) * (size_t)(B + 1), 256);
     sp[1] = align_up(sizeof(uint32_t) * 4 * (size_t)B, 256);
-    sp[2] = align_up(sizeof(int) * 256 * (size_t)B, 256);
+    sp[2] = align_up(sizeof(int) * 258 * (size_t)B, 256);  // digit histograms, two finish counters
     sp[3] = align_up(sizeof(int) * 2 * (size_t)mc, 256);
     sp[4] = align_up(sizeof(unsigned long long) * (size_t)B * LSA_MAX_TOPK, 256);
     return sp[0] + sp[1] + sp[2] + sp[3] + sp[4];
@@ -568,10 +568,10 @@ static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[5])
 static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[6])
 {
     part[0] = align_up(sizeof(int) * (size_t)(B + 2), 256);
-    part[1] = align_up(sizeof(float) * 4 * (size_t)(total_S > 0 ? total_S : 1), 256);
+    part[1] = align_up(sizeof(float) * (size_t)(total_S > 0 ? total_S : 1), 256);
     part[2] = align_up(sizeof(float) * (size_t)B * (W > 0 ? W : 1), 256);
-    part[3] = align_up((size_t)4 * B * 4 * n_h * d_I, 256);
-    part[4] = align_up(sizeof(float) * (size_t)B * 4 * n_h, 256);
+    part[3] = align_up((size_t)4 * B * n_h * d_I, 256);
+    part[4] = align_up(sizeof(float) * (size_t)B * n_h, 256);
     size_t sp[5];
     part[5] = step_sel_parts(B, total_S, W, sp);
     return part[0] + part[1] + part[2] + part[3] + part[4] + part[5];
@@ -620,8 +620,9 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     void *qw = (void *)(p + part[0] + part[1] + part[2]);
     float *ww = (float *)(p + part[0] + part[1] + part[2] + part[3]);
     const int hdt = (kdt == LSA_FP8_E4M3) ? DT_BF16 : kdt;  // hot keys: E4M3 arrives decoded to bf16
-    const bool tc = li_tc_supported(n_h, d_I, 4, kdt);
-    const int TQ = tc ? 4 : 1;
+    // one query per sequence: the tensor-core scorer runs with one-query groups (MMA N = n_h)
+    const bool tc = li_tc_supported(n_h, d_I, 1, kdt, 1);
+    const int TQ = 1;
     const int64_t rows = (int64_t)B * TQ * n_h;
     k_step_prep<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(q_step, q_batch_stride, w_step, w_batch_stride, hdt, B, TQ,
                                                             n_h, d_I, qw, ww);
@@ -629,7 +630,7 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     if (tc) {
         LSA_REQUIRE(aligned(hot_K, 16), "lsa_lightning_topk_step: hot_K must be 16-byte aligned");
         int n = 0;
-        const lsa_status s = launch_li_tc(qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, TQ, Y, item_start,
+        const lsa_status s = launch_li_tc(qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, TQ, 1, Y, item_start,
                                           item_counter, num_sms(), st, &n);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK)
@@ -659,15 +660,13 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     int *eqc = gtc + mc;
     unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
     const int32_t *tcnt = W > 0 ? win_count : nullptr;
+    int *done_hist = ghist + 256 * (size_t)B, *done_count = done_hist + B;
     stepsel::k_ss_setup<<<1, 1024, 0, st>>>(count, seq_offsets, tcnt, W, B, k, chunk_start, state, ghist);
-    for (int pass = 0; pass < 4; pass++) {
+    for (int pass = 0; pass < 4; pass++)
         stepsel::k_ss_hist<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B,
-                                                                 chunk_start, state, pass, ghist);
-        stepsel::k_ss_digit<<<(unsigned)B, 256, 0, st>>>(state, ghist, pass);
-    }
+                                                                 chunk_start, state, pass, ghist, done_hist);
     stepsel::k_ss_count<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
-                                                              state, gtc, eqc);
-    stepsel::k_ss_scan<<<(unsigned)B, 32, 0, st>>>(chunk_start, gtc, eqc);
+                                                              state, gtc, eqc, done_count);
     stepsel::k_ss_write<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
                                                               state, gtc, eqc, LSA_MAX_TOPK, sel);
     int kpow2 = 1;
@@ -677,7 +676,7 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     stepsel::k_ss_sort<<<(unsigned)B, stepsel::SORT_TH, smem, st>>>(sel, LSA_MAX_TOPK, state, idx, count, seq_offsets,
                                                                    k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
-    g_launches.fetch_add(11, std::memory_order_relaxed);
+    g_launches.fetch_add(7, std::memory_order_relaxed);  // setup, 4 histogram passes, count, write (+ sort)
     return ok();
 }
 

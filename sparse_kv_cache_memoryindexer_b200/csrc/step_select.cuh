@@ -1,20 +1,22 @@
 // Top-k select of one decode step, spread over many CTAs.  A step has one query per sequence, so
 // the one-CTA-per-query select of the batched call would leave all but B SMs idle; here the
-// candidates of a query (its fetched slots, then its window entries: see k_topk_select<true>) are
-// cut into chunks of CH, and the most-significant-digit-first radix search on the order-preserving
-// keys runs with one CTA per chunk:
+// candidates of a query (its F fetched slots, then its window entries as candidates F .. F + n - 1,
+// reported as entries S_b + j) are cut into chunks of CH, and the most-significant-digit-first
+// radix search on the order-preserving keys runs with one CTA per chunk:
 //   k_ss_setup   per query: candidates, chunk ranges (a prefix over the sequences), search state
 //   k_ss_hist    per chunk: histogram of the next 8-bit digit of the keys that match the prefix so
-//                far, added to the query's histogram in global memory
-//   k_ss_digit   per query: the digit where the count from the top reaches the keys still wanted
-//   (4 passes of hist + digit: the k-th largest key K*)
-//   k_ss_count   per chunk: keys above K* and keys equal to it
-//   k_ss_scan    per query: chunk offsets of both counts (slot order)
+//                far, added to the query's histogram in global memory; the query's last chunk to
+//                finish then picks the digit where the count from the top reaches the keys still
+//                wanted (4 passes: the k-th largest key K*)
+//   k_ss_count   per chunk: keys above K* and keys equal to it; the query's last chunk turns the
+//                chunk counts into chunk offsets (slot order)
 //   k_ss_write   per chunk: every key above K*, and the first equal keys in slot order, to the
 //                query's selection
 //   k_ss_sort    per query: bitonic sort of the selection (key descending, slot ascending) and the
 //                output, as the one-CTA select writes it.
-// Kernel boundaries are the only synchronisation between CTAs.
+// CTAs of one launch do not wait for one another: the per-query step after a launch's chunks runs
+// in whichever chunk CTA of the query finishes last (a counter per query, reset by that CTA), and
+// kernel boundaries order the rest.
 #pragma once
 #include "common.cuh"
 
@@ -54,7 +56,8 @@ __device__ __forceinline__ uint32_t key_of(const Query &q, int j)
 }
 
 // state per query: [0] prefix (the key bits fixed so far), [1] keys still wanted at the prefix,
-// [2] keys above the final K*, [3] candidates
+// [2] keys above the final K*, [3] candidates.  ghist: [B][256] digit histograms, then the
+// per-query finish counters of k_ss_hist [B] and of k_ss_count [B].
 __global__ void __launch_bounds__(1024) k_ss_setup(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
                                                    const int32_t *__restrict__ tail_count, int W, int B, int k,
                                                    int *__restrict__ chunk_start, uint32_t *__restrict__ state,
@@ -66,7 +69,7 @@ __global__ void __launch_bounds__(1024) k_ss_setup(const int32_t *__restrict__ c
         carry = 0;
         chunk_start[0] = 0;
     }
-    for (int i = threadIdx.x; i < B * 256; i += blockDim.x) ghist[i] = 0;
+    for (int i = threadIdx.x; i < B * 258; i += blockDim.x) ghist[i] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int base = 0; base < B; base += blockDim.x) {
@@ -113,17 +116,62 @@ __device__ __forceinline__ int query_of_chunk(const int *chunk_start, int B, int
     return lo;
 }
 
+// Called by every thread of the chunk CTA after its part of a per-query sum is in global memory:
+// true in the CTA that finishes the query's chunks last (which then also resets the counter).
+__device__ __forceinline__ bool last_chunk_of_query(int *done, int b, int nch)
+{
+    __shared__ int is_last;
+    __threadfence();  // this CTA's global writes before its count
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        is_last = atomicAdd(done + b, 1) == nch - 1;
+        if (is_last) done[b] = 0;  // nobody else counts on this query in this launch
+    }
+    __syncthreads();
+    if (!is_last) return false;
+    __threadfence();  // the other chunks' writes, counted before ours, are read after this
+    return true;
+}
+
+// Block-wide exclusive scans of two counts (TH threads): positions and totals.
+__device__ __forceinline__ void block_excl_scan2(int a, int b, int &pa, int &pb, int &ta, int &tb)
+{
+    __shared__ int wa[TH / 32], wb[TH / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ia = warp_incl_scan(a), ib = warp_incl_scan(b);
+    if (lane == 31) {
+        wa[warp] = ia;
+        wb[warp] = ib;
+    }
+    __syncthreads();
+    int ba = 0, bb = 0, sa = 0, sb = 0;
+#pragma unroll
+    for (int w = 0; w < TH / 32; w++) {
+        ba += w < warp ? wa[w] : 0;
+        bb += w < warp ? wb[w] : 0;
+        sa += wa[w];
+        sb += wb[w];
+    }
+    pa = ba + ia - a;
+    pb = bb + ib - b;
+    ta = sa;
+    tb = sb;
+    __syncthreads();  // wa, wb free for the next call
+}
+
 __global__ void __launch_bounds__(TH) k_ss_hist(const float *__restrict__ Y, int tau_y, const int32_t *__restrict__ count,
                                                 const int64_t *__restrict__ offs, const float *__restrict__ tail,
                                                 const int32_t *__restrict__ tail_count, int W, int B,
-                                                const int *__restrict__ chunk_start,
-                                                const uint32_t *__restrict__ state, int pass, int *__restrict__ ghist)
+                                                const int *__restrict__ chunk_start, uint32_t *state, int pass,
+                                                int *ghist, int *done)
 {
+    static_assert(TH == 256, "one digit bin per thread in the digit step");
     __shared__ int hist[256];
     const int c = blockIdx.x;
     if (c >= chunk_start[B]) return;
     const int b = query_of_chunk(chunk_start, B, c);
-    if (state[4 * b + 1] == 0u) return;  // takes all its candidates
+    const uint32_t remaining = state[4 * b + 1];
+    if (remaining == 0u) return;  // takes all its candidates (the same for every chunk of b)
     const Query q = query(b, Y, tau_y, count, offs, tail, tail_count, W);
     const int nc = q.F0 + q.nt;
     const int j0 = (c - chunk_start[b]) * CH, j1 = min(nc, j0 + CH);
@@ -139,27 +187,20 @@ __global__ void __launch_bounds__(TH) k_ss_hist(const float *__restrict__ Y, int
     __syncthreads();
     for (int t = threadIdx.x; t < 256; t += TH)
         if (hist[t]) atomicAdd(ghist + b * 256 + t, hist[t]);
-}
-
-__global__ void __launch_bounds__(256) k_ss_digit(uint32_t *__restrict__ state, int *__restrict__ ghist, int pass)
-{
-    const int b = blockIdx.x;
-    __shared__ int h[256];
-    h[threadIdx.x] = ghist[b * 256 + threadIdx.x];
-    ghist[b * 256 + threadIdx.x] = 0;  // ready for the next pass
-    __syncthreads();
-    if (threadIdx.x == 0 && state[4 * b + 1] != 0u) {
-        const int shift = 24 - 8 * pass;
-        uint32_t remaining = state[4 * b + 1], cum = 0;
-        int chosen = 0;
-        for (int d = 255; d >= 0; d--) {
-            if (cum + (uint32_t)h[d] >= remaining) {
-                chosen = d;
-                break;
-            }
-            cum += (uint32_t)h[d];
-        }
-        state[4 * b + 0] |= (uint32_t)chosen << shift;
+    if (!last_chunk_of_query(done, b, chunk_start[b + 1] - chunk_start[b])) return;
+    // the digit: thread t holds bin 255 - t, so an inclusive scan over the threads counts the keys
+    // at or above each digit; exactly one bin has above < remaining <= at or above
+    const int dg = 255 - (int)threadIdx.x;
+    const int h = atomicExch(ghist + b * 256 + dg, 0);  // read, and clear for the next pass
+    int pos, unused_p, total, unused_t;
+    block_excl_scan2(h, 0, pos, unused_p, total, unused_t);
+    const uint32_t above = (uint32_t)pos, upto = (uint32_t)(pos + h);
+    const bool chosen = h > 0 && above < remaining && upto >= remaining;
+    // fewer matching keys than wanted cannot happen (every pass counts the same keys); digit 0 then
+    const bool none = threadIdx.x == TH - 1 && (uint32_t)total < remaining;
+    if (chosen || none) {
+        const uint32_t cum = none ? (uint32_t)total : above;
+        state[4 * b + 0] = prefix | ((uint32_t)(none ? 0 : dg) << shift);
         state[4 * b + 1] = remaining - cum;
         state[4 * b + 2] += cum;
     }
@@ -169,8 +210,7 @@ __global__ void __launch_bounds__(TH) k_ss_count(const float *__restrict__ Y, in
                                                  const int64_t *__restrict__ offs, const float *__restrict__ tail,
                                                  const int32_t *__restrict__ tail_count, int W, int B,
                                                  const int *__restrict__ chunk_start,
-                                                 const uint32_t *__restrict__ state, int *__restrict__ gtc,
-                                                 int *__restrict__ eqc)
+                                                 const uint32_t *__restrict__ state, int *gtc, int *eqc, int *done)
 {
     __shared__ int sgt, seq;
     const int c = blockIdx.x;
@@ -202,21 +242,21 @@ __global__ void __launch_bounds__(TH) k_ss_count(const float *__restrict__ Y, in
         gtc[c] = sgt;
         eqc[c] = seq;
     }
-}
-
-// per query: exclusive offsets of the chunk counts, in chunk (slot) order
-__global__ void __launch_bounds__(32) k_ss_scan(const int *__restrict__ chunk_start, int *__restrict__ gtc,
-                                                int *__restrict__ eqc)
-{
-    const int b = blockIdx.x;
-    if (threadIdx.x != 0) return;
-    int g = 0, e = 0;
-    for (int c = chunk_start[b]; c < chunk_start[b + 1]; c++) {
-        const int tg = gtc[c], te = eqc[c];
-        gtc[c] = g;
-        eqc[c] = e;
-        g += tg;
-        e += te;
+    const int c0 = chunk_start[b], c1 = chunk_start[b + 1];
+    if (!last_chunk_of_query(done, b, c1 - c0)) return;
+    // exclusive offsets of the query's chunk counts, in chunk (slot) order
+    int carry_g = 0, carry_e = 0;
+    for (int base = c0; base < c1; base += TH) {
+        const int cc = base + threadIdx.x;
+        const int g = cc < c1 ? __ldcg(gtc + cc) : 0, e = cc < c1 ? __ldcg(eqc + cc) : 0;
+        int pg, pe, tg, te;
+        block_excl_scan2(g, e, pg, pe, tg, te);
+        if (cc < c1) {
+            gtc[cc] = carry_g + pg;
+            eqc[cc] = carry_e + pe;
+        }
+        carry_g += tg;
+        carry_e += te;
     }
 }
 

@@ -38,6 +38,10 @@ CASES = {
     "bf16": lambda: synth.workload("ctx128k_bf16", B=3, S=(3000, 700, 4100), fetch=(0.2, 0.3, 0.1), name="step_bf16"),
     "fp8": lambda: synth.workload("ctx1m_fp8_b32", B=2, S=(5000, 2600), name="step_fp8"),
     "fp32": lambda: synth.workload("tiny_fp32"),
+    # several 2,048-candidate chunks per query (6,000 + window and 2,400 + window candidates), so the
+    # select's per-query steps run after chunk CTAs that finish in any order
+    "bf16_long": lambda: synth.workload("ctx128k_bf16", B=2, S=(30000, 12000), fetch=(0.2, 0.3),
+                                        name="step_bf16_long"),
 }
 _cache = {}
 
@@ -127,8 +131,9 @@ def test_step_with_window_entries(m, name, kernel_path):
         check_against_oracle(name, i, wc, k, ti, ts)
 
 
-def test_step_without_window_equals_batched_column(m):
-    wl, inp, Ks, ks, idx, cnt, hK, hs, winK = case("bf16")
+@pytest.mark.parametrize("name", ["bf16", "bf16_long"])
+def test_step_without_window_equals_batched_column(m, name):
+    wl, inp, Ks, ks, idx, cnt, hK, hs, winK = case(name)
     T, k = wl.total_S, 128
     tk = torch.empty((wl.B, wl.tau, k), dtype=torch.int32, device="cuda")
     tsc = torch.empty((wl.B, wl.tau, k), dtype=torch.float32, device="cuda")
@@ -137,7 +142,7 @@ def test_step_without_window_equals_batched_column(m):
                          inp.seq_offsets.cuda(), T, k, tk, ws, topk_score=tsc)
     m.lsa_check_device()
     for i in (0, 1, 2, 3, 17, wl.tau - 1):
-        ti, ts = run_step(m, "bf16", i, None, k, with_window=False)
+        ti, ts = run_step(m, name, i, None, k, with_window=False)
         assert np.array_equal(ti, tk[:, i].cpu().numpy())
         assert np.array_equal(ts, tsc[:, i].cpu().numpy())
 
