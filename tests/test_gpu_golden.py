@@ -82,3 +82,34 @@ def test_golden_random_heavy_ties(m):
     offs = torch.from_numpy(np.concatenate([[0], np.cumsum(S)]).astype(np.int64))
     z = torch.randint(0, 6, (4, 21, sum(S)), generator=g).float() * 0.75
     check(m, z, offs)
+
+
+def candidate_set_fits(row, p, cand=4096, depths=(4.0, 8.0, 12.0, 16.0, 24.0, 40.0)):
+    """Whether some set of entries within a depth of the row's maximum logit reaches mass p with at
+    most `cand` entries (the kernel then sorts that set; otherwise it takes its radix search)."""
+    z = row.astype(np.float64)
+    e = np.exp(z - z.max())
+    for D in depths:
+        inside = (np.float32(row.max()) - row) < D
+        if e[inside].sum() >= p * e.sum() and inside.sum() <= cand:
+            return True
+    return False
+
+
+@pytest.mark.parametrize("p", [0.6, 0.95])
+def test_golden_long_flat_rows_take_the_radix_search(m, p):
+    # nuclei of thousands of entries within a narrow band of logits: no candidate set of at most
+    # 4096 entries reaches p, so every row of the two long sequences runs the radix search (flat
+    # logits, and logits from five values with exact ties); the short sequence stays on the sort
+    g = torch.Generator().manual_seed(17)
+    S = (20000, 9000, 1500)
+    offs = torch.from_numpy(np.concatenate([[0], np.cumsum(S)]).astype(np.int64))
+    tau, Lc = 2, 3
+    z = torch.rand((tau, Lc, sum(S)), generator=g)
+    z[1] = torch.randint(0, 5, (Lc, sum(S)), generator=g).float() * 0.01
+    zn = z.numpy()
+    for i in range(tau):
+        for l in range(Lc):
+            for b in range(2):
+                assert not candidate_set_fits(zn[i, l, offs[b]:offs[b + 1]], p)
+    check(m, z, offs, p=p, theta=2)
