@@ -28,15 +28,15 @@ def offsets(S):
     return o
 
 
-def content(S_max, seed):
+def content(S_max, seed, row=ROW):
     """Row bytes of entry (b, s): the same in every window (a KV row does not change)."""
-    return [np.random.default_rng((seed, b)).integers(0, 256, size=(n, ROW), dtype=np.uint8) for b, n in
+    return [np.random.default_rng((seed, b)).integers(0, 256, size=(n, row), dtype=np.uint8) for b, n in
             enumerate(S_max)]
 
 
-def pool_for(rows, S, m):
+def pool_for(rows, S, m, row=ROW):
     o = offsets(S)
-    pool = m.MappedPool(int(o[-1]), ROW)
+    pool = m.MappedPool(int(o[-1]), row)
     for b, n in enumerate(S):
         if n:
             pool.tensor[o[b]:o[b] + n] = torch.from_numpy(rows[b][:n])
@@ -53,16 +53,16 @@ def lists_to_arrays(lists, S, fill=-7):
     return torch.from_numpy(idx), torch.from_numpy(cnt), torch.from_numpy(o)
 
 
-def run_case(m, S_prev, S_new, prev_lists, new_lists, seed=0, host_check=None):
-    rows = content([max(a, b) for a, b in zip(S_prev, S_new)], seed)
-    pool_prev, pool_new = pool_for(rows, S_prev, m), pool_for(rows, S_new, m)
+def run_case(m, S_prev, S_new, prev_lists, new_lists, seed=0, host_check=None, row=ROW):
+    rows = content([max(a, b) for a, b in zip(S_prev, S_new)], seed, row)
+    pool_prev, pool_new = pool_for(rows, S_prev, m, row), pool_for(rows, S_new, m, row)
     try:
         pi, pc, po = lists_to_arrays(prev_lists, S_prev)
         ni, nc, no = lists_to_arrays(new_lists, S_new)
         Tp, Tn = int(po[-1]), int(no[-1])
         prev_hot, _, _ = oracle.gather(pi, pc, po.numpy(), pool_prev.tensor[:max(Tp, 1)].clone())
         ref_hot, _, _ = oracle.gather(ni, nc, no.numpy(), pool_new.tensor[:max(Tn, 1)].clone())
-        hot = torch.zeros((max(Tn, 1), ROW), dtype=torch.uint8, device="cuda")
+        hot = torch.zeros((max(Tn, 1), row), dtype=torch.uint8, device="cuda")
         host_rows = torch.full((1,), -1, dtype=torch.int32, device="cuda")
         ws = torch.empty(m.lsa_fetch_incremental_workspace_size(len(S_new), Tn), dtype=torch.uint8, device="cuda")
         m.lsa_fetch_gather_incremental(ni.cuda(), nc.cuda(), no.cuda(), Tn, pi.cuda(), pc.cuda(), po.cuda(), Tp,
@@ -133,3 +133,12 @@ def test_incremental_full_sequences(m):
     prev = [np.arange(0, 64, 2, dtype=np.int32), np.arange(300, dtype=np.int32), np.zeros(0, dtype=np.int32)]
     new = [np.arange(64, dtype=np.int32), np.arange(1, 300, 3, dtype=np.int32), np.arange(2, dtype=np.int32)]
     assert run_case(m, S, S, prev, new, seed=9) == 32 + 0 + 2
+
+
+@pytest.mark.parametrize("row", [48, 2048])
+def test_incremental_row_sizes(m, row):
+    # 3 chunks of 16 bytes per row (most lanes idle) and the largest row (four chunks per lane),
+    # through the device copy and the host-link launch
+    prev, new = drifted(S_PREV, S_NEW, rate=0.2, keep=0.85, add=0.05, seed=11)
+    n_host = run_case(m, S_PREV, S_NEW, prev, new, seed=12, row=row)
+    assert 0 < n_host < sum(len(N) for N in new)
