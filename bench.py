@@ -251,6 +251,15 @@ def algorithmic(wl, fetched_total):
             "topk_flops": topk_flops}
 
 
+def workload_config(wl, threshold, world):
+    """The `config` object of the JSON line: the workload's names and sizes, the same in both arms."""
+    alg = algorithmic(wl, 0)
+    return {"workload": wl.name, "B": wl.B, "L": wl.L, "S_per_seq": wl.S[0], "d": wl.d, "r": wl.r,
+            "n_h": wl.n_h, "d_I": wl.d_I, "tau": wl.tau, "k": wl.k, "kv_row_bytes": wl.row_bytes,
+            "keys": wl.kdtype, "threshold": threshold, "parallelism": f"dp{world} (sequences)",
+            "l2": "inputs larger than L2 (key stream %.2f GB per step)" % (alg["score_bytes"] / 1e9)}
+
+
 def h2d_bandwidth(device, nbytes=1 << 30):
     src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
     dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -585,11 +594,8 @@ def run_lsa(args, rank, world, device):
             "vs_baseline": None, "dtype": "bf16" if wl.kdtype != "f32" else "f32",
             "dtype_detail": f"keys {wl.kdtype}, queries/weights {wl.dtype}, fp32 accumulation",
             "data": "synthetic (seeded; shapes of a 1M-token context, 4:1 compression)",
-            "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "S_per_seq": wl.S[0], "d": wl.d, "r": wl.r,
-                       "n_h": wl.n_h, "d_I": wl.d_I, "tau": wl.tau, "k": wl.k, "kv_row_bytes": wl.row_bytes,
-                       "keys": wl.kdtype, "threshold": args.threshold, "parallelism": f"dp{world} (sequences)",
-                       "l2": "inputs larger than L2 (key stream %.2f GB per step)" % (alg["score_bytes"] / 1e9),
-                       "fetch_rate": fetched / T},
+            "config": workload_config(wl, args.threshold, world),
+            "fetch_rate": fetched / T,
             "tau_window_ms": ms,
             "stages_ms": {"project": stage_ms[0], "score_select": stage_ms[1], "fetch_keys": stage_ms[2],
                           "lightning_topk": stage_ms[3], "fetch_rows (overlapped)": stage_ms[4],
@@ -623,7 +629,7 @@ def main():
         if rank != 0:
             return 0
         import oracle
-        wl = synth.workload(args.workload)
+        wl = rank_workload(args.workload, 0, args.batch)
         # about two minutes of oracle work in total (~130 us per entry on 8 cores, whole path)
         n = args.cpu_sample or int(min(65536, max(2048, 120.0 / (args.steps + args.warmup) / 130e-6)))
         sw = oracle_sample_workload(wl, n)
@@ -640,7 +646,7 @@ def main():
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                          "data": "synthetic", "config": {"workload": wl.name, "sample_entries": sw.total_S},
+                          "data": "synthetic", "config": workload_config(wl, args.threshold, world),
                           "cpu_baseline": cb,
                           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
               flush=True)

@@ -64,3 +64,27 @@ def test_reference_arm_runs_on_rank_zero_only():
                         "--warmup", "0"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_line_matches_the_gpu_arm():
+    """Rank 0 prints one JSON line with the GPU arm's metric, unit and config (the oracle timed on
+    a bounded sample of the same workload) and an e2e with no host-device bytes."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--cpu-sample", "512"], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["metric"] == bench.METRIC and out["unit"] == bench.UNIT
+    assert out["higher_is_better"] is True and out["n_gpus"] == 1 and out["value"] > 0
+    assert out["config"] == bench.workload_config(synth.workload(bench.DEFAULT_WORKLOAD), 0.5, 1)
+    assert out["e2e"] == {"value": out["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+    cb = out["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == out["value"] and cb["cores"] >= 1 and "512" in cb["sample"]
