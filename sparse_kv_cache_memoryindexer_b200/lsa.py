@@ -106,6 +106,20 @@ def _p_rows(t):
     return t.data_ptr()
 
 
+def _need(dtype, **named):
+    """Element types the C ABI reads or writes (include/lsa.h): checked here, since a pointer does
+    not carry one and a wrong width would send a kernel past the end of a buffer."""
+    for name, t in named.items():
+        if t is not None and t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _offsets(seq_offsets, B):
+    _need(torch.int64, seq_offsets=seq_offsets)
+    if seq_offsets.numel() != B + 1:
+        raise ValueError(f"seq_offsets must hold B + 1 = {B + 1} prefix offsets, got {seq_offsets.numel()}")
+
+
 def _dev(*ts):
     for t in ts:
         if t is not None and t.device.type != "cuda":
@@ -138,6 +152,8 @@ def lsa_project_workspace_size(L, B, d, r, n_h, d_I, dt) -> int:
 
 def lsa_project(h, W_dq, W_iuq, W_w, q_out, w_out, workspace, stream=None):
     """c^Q = h W^DQ, q = c^Q W^IUQ, w = h W^w for every layer and sequence (see include/lsa.h)."""
+    _need(h.dtype, W_dq=W_dq, W_iuq=W_iuq, W_w=W_w, q_out=q_out)
+    _need(torch.float32, w_out=w_out)
     _dev(h, W_dq, W_iuq, W_w, q_out, w_out, workspace)
     L, B, d = h.shape
     r = W_dq.shape[1]
@@ -153,9 +169,18 @@ def lsa_score_select_workspace_size(L, B, total_S) -> int:
     return int(_lib.lsa_score_select_workspace_size(L, B, total_S))
 
 
+def _score_select_types(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out):
+    _need(torch.float32 if K.dtype == torch.float32 else torch.bfloat16, q=q)
+    _need(torch.float32, w=w, k_scale=k_scale, scores_out=scores_out)
+    _need(torch.int32, idx_out=idx_out, count_out=count_out)
+    _need(torch.uint8, mask_out=mask_out)
+    _offsets(seq_offsets, q.shape[1])
+
+
 def lsa_memindex_score_select(q, w, K, k_scale, seq_offsets, total_S, threshold, idx_out, count_out,
                               workspace, scores_out=None, mask_out=None, stream=None):
     """Index score, threshold, OR over layers and compaction (see include/lsa.h)."""
+    _score_select_types(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
     _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, workspace, scores_out, mask_out)
     L, B, n_h, d_I = q.shape
     _check(_lib.lsa_memindex_score_select(
@@ -171,6 +196,7 @@ def lsa_memindex_score_select_static(q, w, K, k_scale, seq_offsets, total_S, thr
                                      scores_out=None, mask_out=None, stream=None):
     """lsa_memindex_score_select with the library's own per-device scratch instead of a workspace:
     the call allocates nothing (see include/lsa.h for the size limit and the ordering rule)."""
+    _score_select_types(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
     _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
     L, B, n_h, d_I = q.shape
     _check(_lib.lsa_memindex_score_select_static(
@@ -184,6 +210,11 @@ def lsa_fetch_gather(idx, count, seq_offsets, total_S, pool, hot_kv, K_sel=None,
                      hot_K=None, hot_scale=None, stream=None):
     """Gather fetched rows from the mapped host cold pool and/or the keys of one layer (pool and
     hot_kv None: keys only; K_sel None: rows only, a small launch meant for a second stream)."""
+    _need(torch.int32, idx=idx, count=count)
+    _offsets(seq_offsets, count.numel())
+    _need(torch.float32, k_scale_sel=k_scale_sel, hot_scale=hot_scale)
+    if K_sel is not None:
+        _need(torch.bfloat16 if K_sel.dtype == torch.float8_e4m3fn else K_sel.dtype, hot_K=hot_K)
     _dev(idx, count, seq_offsets, hot_kv, K_sel, k_scale_sel, hot_K, hot_scale)
     if pool is not None and pool.device.type != "cpu":
         raise ValueError("the cold pool must be (mapped page-locked) host memory")
@@ -205,6 +236,9 @@ def lsa_fetch_gather_incremental(idx, count, seq_offsets, total_S, prev_idx, pre
                                  stream=None):
     """The window's rows with the previous window's rows resident: common entries are copied on the
     device, only the others cross the host link (see include/lsa.h)."""
+    _need(torch.int32, idx=idx, count=count, prev_idx=prev_idx, prev_count=prev_count, host_rows_out=host_rows_out)
+    _offsets(seq_offsets, count.numel())
+    _offsets(prev_seq_offsets, prev_count.numel())
     _dev(idx, count, seq_offsets, prev_idx, prev_count, prev_seq_offsets, prev_hot_kv, hot_kv, workspace,
          host_rows_out)
     if pool.device.type != "cpu":
@@ -227,6 +261,10 @@ def lsa_lightning_topk(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, 
                        workspace, topk_score=None, stream=None):
     """Native Lightning-Indexer Top-k over the fetched entries (see include/lsa.h).  With E4M3
     keys, hot_K is the bf16 decode written by lsa_fetch_gather and hot_scale holds the scales."""
+    _need(torch.float32 if hot_K.dtype == torch.float32 else torch.bfloat16, q_dec=q_dec)
+    _need(torch.float32, w_dec=w_dec, hot_scale=hot_scale, topk_score=topk_score)
+    _need(torch.int32, idx=idx, count=count, topk_idx=topk_idx)
+    _offsets(seq_offsets, q_dec.shape[0])
     _dev(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, topk_score)
     B, tau, n_h, d_I = q_dec.shape
     kdt = LSA_FP8_E4M3 if hot_scale is not None else DTYPE_CODE[hot_K.dtype]
@@ -244,6 +282,10 @@ def lsa_golden_labels_workspace_size(tau, Lc, total_S) -> int:
 
 def lsa_golden_labels(z, seq_offsets, label_out, workspace, p=0.6, theta=3, nsize_out=None, stream=None):
     """Golden labels of one window from raw indexer logits z [tau][Lc][T] fp32 (see include/lsa.h)."""
+    _need(torch.float32, z=z)
+    _need(torch.uint8, label_out=label_out)
+    _need(torch.int32, nsize_out=nsize_out)
+    _need(torch.int64, seq_offsets=seq_offsets)
     _dev(z, seq_offsets, label_out, workspace, nsize_out)
     tau, Lc, T = z.shape
     B = seq_offsets.numel() - 1
@@ -259,6 +301,11 @@ def lsa_indexer_train_workspace_size(L, B, total_S, d, r, n_h, d_I, dtype) -> in
 def lsa_indexer_train_step(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets, loss_out, g_Wdq, g_Wiuq, g_Ww,
                            workspace, n_h, d_I, gamma=0.0, alpha=-1.0, stream=None):
     """Loss and gradients of W^DQ, W^IUQ, W^w for one training step (see include/lsa.h)."""
+    _need(h.dtype, W_dq=W_dq, W_iuq=W_iuq, W_w=W_w)
+    _need(torch.float32, k_scale=k_scale, g_Wdq=g_Wdq, g_Wiuq=g_Wiuq, g_Ww=g_Ww)
+    _need(torch.uint8, labels=labels)
+    _need(torch.float64, loss_out=loss_out)
+    _offsets(seq_offsets, h.shape[1])
     _dev(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets, loss_out, g_Wdq, g_Wiuq, g_Ww, workspace)
     L, B, d = h.shape
     r = W_dq.shape[1]
@@ -278,6 +325,11 @@ def lsa_lightning_topk_step(q_step, w_step, hot_K, hot_scale, idx, count, seq_of
                             stream=None):
     """One decode step: q_step [B][n_h][d_I] and w_step [B][n_h] may be strided views (e.g. a
     column q_dec[:, i] of the window's queries); window entries win_K [B][W][d_I] with win_count [B]."""
+    _need(torch.float32 if hot_K.dtype == torch.float32 else torch.bfloat16, q_step=q_step)
+    _need(hot_K.dtype, win_K=win_K)
+    _need(torch.float32, w_step=w_step, hot_scale=hot_scale, win_scale=win_scale, topk_score=topk_score)
+    _need(torch.int32, idx=idx, count=count, win_count=win_count, topk_idx=topk_idx)
+    _offsets(seq_offsets, q_step.shape[0])
     _dev(q_step, w_step, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, win_K, win_scale, win_count,
          topk_score)
     B, n_h, d_I = q_step.shape

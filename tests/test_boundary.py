@@ -91,3 +91,53 @@ def test_workspace_sizes_cover_their_buffers():
     assert lsa.lsa_score_select_workspace_size(3, 32, T) >= (T // 128) * 16
     assert lsa.lsa_lightning_topk_workspace_size(32, 64, T, 2048) >= 64 * T * 4
     assert lsa.lsa_project_workspace_size(3, 32, 4096, 2048, 64, 128, torch.bfloat16) >= 3 * 32 * 2048 * 2
+
+
+def test_binding_rejects_wrong_element_types_before_the_device():
+    """A pointer carries no element type: the binding checks the widths the C ABI reads (int32
+    indices and counts, int64 offsets, fp32 weights and scales, uint8 labels) on the host, so a
+    wrong one is an exception, not a kernel reading past a buffer.  CPU tensors: the checks come
+    before the device check."""
+    import torch
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    i32 = lambda *s: torch.zeros(s, dtype=torch.int32)
+    i64 = lambda *s: torch.zeros(s, dtype=torch.int64)
+    f32 = lambda *s: torch.zeros(s, dtype=torch.float32)
+    bf = lambda *s: torch.zeros(s, dtype=torch.bfloat16)
+    u8 = lambda *s: torch.zeros(s, dtype=torch.uint8)
+    ws = u8(256)
+    with pytest.raises(TypeError, match="idx must be torch.int32"):
+        lsa.lsa_fetch_gather(i64(10), i32(2), i64(3), 10, None, None, bf(10, 128), None, bf(10, 128))
+    with pytest.raises(TypeError, match="seq_offsets must be torch.int64"):
+        lsa.lsa_fetch_gather(i32(10), i32(2), i32(3), 10, None, None, bf(10, 128), None, bf(10, 128))
+    with pytest.raises(ValueError, match="B \\+ 1 = 3"):
+        lsa.lsa_fetch_gather(i32(10), i32(2), i64(4), 10, None, None, bf(10, 128), None, bf(10, 128))
+    with pytest.raises(TypeError, match="hot_K must be torch.bfloat16"):   # E4M3 keys arrive as bf16
+        lsa.lsa_fetch_gather(i32(10), i32(2), i64(3), 10, None, None,
+                             torch.zeros((10, 128), dtype=torch.float8_e4m3fn), f32(10), f32(10, 128), f32(10))
+    with pytest.raises(TypeError, match="w must be torch.float32"):
+        lsa.lsa_memindex_score_select(bf(3, 2, 64, 128), bf(3, 2, 64), bf(3, 10, 128), None, i64(3), 10, 0.5,
+                                      i32(10), i32(2), ws)
+    with pytest.raises(TypeError, match="q must be torch.bfloat16"):
+        lsa.lsa_memindex_score_select(f32(3, 2, 64, 128), f32(3, 2, 64), bf(3, 10, 128), None, i64(3), 10, 0.5,
+                                      i32(10), i32(2), ws)
+    with pytest.raises(TypeError, match="count_out must be torch.int32"):
+        lsa.lsa_memindex_score_select_static(bf(3, 2, 64, 128), f32(3, 2, 64), bf(3, 10, 128), None, i64(3), 10, 0.5,
+                                             i32(10), i64(2))
+    with pytest.raises(TypeError, match="q_dec must be torch.bfloat16"):
+        lsa.lsa_lightning_topk(f32(2, 4, 64, 128), f32(2, 4, 64), bf(10, 128), None, i32(10), i32(2), i64(3), 10, 8,
+                               i32(2, 4, 8), ws)
+    with pytest.raises(TypeError, match="win_K must be torch.bfloat16"):
+        lsa.lsa_lightning_topk_step(bf(2, 64, 128), f32(2, 64), bf(10, 128), None, i32(10), i32(2), i64(3), 10, 8,
+                                    i32(2, 8), ws, win_K=f32(2, 4, 128), win_count=i32(2))
+    with pytest.raises(TypeError, match="z must be torch.float32"):
+        lsa.lsa_golden_labels(torch.zeros((2, 3, 10), dtype=torch.float64), i64(3), u8(10), ws)
+    with pytest.raises(TypeError, match="labels must be torch.uint8"):
+        lsa.lsa_indexer_train_step(bf(3, 2, 64), bf(3, 32, 64), bf(3, 64 * 32, 32), bf(3, 64, 64), bf(3, 10, 32),
+                                   None, i32(10), i64(3), torch.zeros(1, dtype=torch.float64), f32(3, 32, 64),
+                                   f32(3, 64 * 32, 32), f32(3, 64, 64), ws, 64, 32)
+    with pytest.raises(TypeError, match="host_rows_out must be torch.int32"):
+        lsa.lsa_fetch_gather_incremental(i32(10), i32(2), i64(3), 10, i32(10), i32(2), i64(3), 10, u8(10, 16),
+                                         u8(10, 16), u8(10, 16), ws, host_rows_out=i64(1))
+    with pytest.raises(ValueError, match="device tensor expected"):     # right types: the device check follows
+        lsa.lsa_fetch_gather(i32(10), i32(2), i64(3), 10, None, None, bf(10, 128), None, bf(10, 128))
