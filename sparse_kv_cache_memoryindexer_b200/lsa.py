@@ -114,6 +114,20 @@ def _need(dtype, **named):
             raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _cap(n, **named):
+    """Buffers the kernels index up to n elements (sizes from include/lsa.h): too small a buffer
+    would be read or written past its end."""
+    for name, t in named.items():
+        if t is not None and t.numel() < n:
+            raise ValueError(f"{name} holds {t.numel()} elements, the call needs {n}")
+
+
+def _cap_bytes(nbytes, **named):
+    for name, t in named.items():
+        if t is not None and t.numel() * t.element_size() < nbytes:
+            raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, the call needs {nbytes}")
+
+
 def _offsets(seq_offsets, B):
     _need(torch.int64, seq_offsets=seq_offsets)
     if seq_offsets.numel() != B + 1:
@@ -154,10 +168,10 @@ def lsa_project(h, W_dq, W_iuq, W_w, q_out, w_out, workspace, stream=None):
     """c^Q = h W^DQ, q = c^Q W^IUQ, w = h W^w for every layer and sequence (see include/lsa.h)."""
     _need(h.dtype, W_dq=W_dq, W_iuq=W_iuq, W_w=W_w, q_out=q_out)
     _need(torch.float32, w_out=w_out)
-    _dev(h, W_dq, W_iuq, W_w, q_out, w_out, workspace)
     L, B, d = h.shape
     r = W_dq.shape[1]
     _, _, n_h, d_I = q_out.shape
+    _dev(h, W_dq, W_iuq, W_w, q_out, w_out, workspace)
     _check(_lib.lsa_project(_p(h), _p(W_dq), _p(W_iuq), _p(W_w), DTYPE_CODE[h.dtype], L, B, d, r, n_h, d_I,
                             _p(q_out), _p(w_out), _p(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream)))
@@ -169,20 +183,28 @@ def lsa_score_select_workspace_size(L, B, total_S) -> int:
     return int(_lib.lsa_score_select_workspace_size(L, B, total_S))
 
 
-def _score_select_types(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out):
+def _score_select_types(q, w, K, k_scale, seq_offsets, total_S, idx_out, count_out, scores_out, mask_out):
     _need(torch.float32 if K.dtype == torch.float32 else torch.bfloat16, q=q)
     _need(torch.float32, w=w, k_scale=k_scale, scores_out=scores_out)
     _need(torch.int32, idx_out=idx_out, count_out=count_out)
     _need(torch.uint8, mask_out=mask_out)
     _offsets(seq_offsets, q.shape[1])
+    L, B, n_h, d_I = q.shape
+    T = int(total_S)
+    if K.shape[1] < T:
+        raise ValueError(f"K holds {K.shape[1]} entries per layer, total_S is {T}")
+    _cap(L * B * n_h, w=w)
+    _cap(L * T, k_scale=k_scale, scores_out=scores_out)
+    _cap(T, idx_out=idx_out, mask_out=mask_out)
+    _cap(B, count_out=count_out)
 
 
 def lsa_memindex_score_select(q, w, K, k_scale, seq_offsets, total_S, threshold, idx_out, count_out,
                               workspace, scores_out=None, mask_out=None, stream=None):
     """Index score, threshold, OR over layers and compaction (see include/lsa.h)."""
-    _score_select_types(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
-    _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, workspace, scores_out, mask_out)
+    _score_select_types(q, w, K, k_scale, seq_offsets, total_S, idx_out, count_out, scores_out, mask_out)
     L, B, n_h, d_I = q.shape
+    _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, workspace, scores_out, mask_out)
     _check(_lib.lsa_memindex_score_select(
         _p(q), _p(w), _p(K), _p(k_scale), DTYPE_CODE[K.dtype], _p(seq_offsets), int(total_S), L, B, n_h, d_I,
         float(threshold), _p(scores_out), _p(mask_out), _p(idx_out), _p(count_out), _p(workspace),
@@ -196,9 +218,9 @@ def lsa_memindex_score_select_static(q, w, K, k_scale, seq_offsets, total_S, thr
                                      scores_out=None, mask_out=None, stream=None):
     """lsa_memindex_score_select with the library's own per-device scratch instead of a workspace:
     the call allocates nothing (see include/lsa.h for the size limit and the ordering rule)."""
-    _score_select_types(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
-    _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
+    _score_select_types(q, w, K, k_scale, seq_offsets, total_S, idx_out, count_out, scores_out, mask_out)
     L, B, n_h, d_I = q.shape
+    _dev(q, w, K, k_scale, seq_offsets, idx_out, count_out, scores_out, mask_out)
     _check(_lib.lsa_memindex_score_select_static(
         _p(q), _p(w), _p(K), _p(k_scale), DTYPE_CODE[K.dtype], _p(seq_offsets), int(total_S), L, B, n_h, d_I,
         float(threshold), _p(scores_out), _p(mask_out), _p(idx_out), _p(count_out), _stream(stream)))
@@ -215,13 +237,18 @@ def lsa_fetch_gather(idx, count, seq_offsets, total_S, pool, hot_kv, K_sel=None,
     _need(torch.float32, k_scale_sel=k_scale_sel, hot_scale=hot_scale)
     if K_sel is not None:
         _need(torch.bfloat16 if K_sel.dtype == torch.float8_e4m3fn else K_sel.dtype, hot_K=hot_K)
-    _dev(idx, count, seq_offsets, hot_kv, K_sel, k_scale_sel, hot_K, hot_scale)
     if pool is not None and pool.device.type != "cpu":
         raise ValueError("the cold pool must be (mapped page-locked) host memory")
     B = count.numel()
     row_bytes = pool.shape[1] * pool.element_size() if pool is not None else 0
     kdt = DTYPE_CODE[K_sel.dtype] if K_sel is not None else 0
     d_I = K_sel.shape[-1] if K_sel is not None else 0
+    T = int(total_S)
+    _cap(T, idx=idx, k_scale_sel=k_scale_sel, hot_scale=hot_scale)
+    _cap(T * d_I, K_sel=K_sel, hot_K=hot_K)
+    if pool is not None:
+        _cap_bytes(T * row_bytes, pool=pool, hot_kv=hot_kv)
+    _dev(idx, count, seq_offsets, hot_kv, K_sel, k_scale_sel, hot_K, hot_scale)
     _check(_lib.lsa_fetch_gather(_p(idx), _p(count), _p(seq_offsets), int(total_S), B, _p(pool), row_bytes,
                                  _p(hot_kv), _p(K_sel), _p(k_scale_sel), kdt, d_I, _p(hot_K), _p(hot_scale),
                                  _stream(stream)))
@@ -239,12 +266,17 @@ def lsa_fetch_gather_incremental(idx, count, seq_offsets, total_S, prev_idx, pre
     _need(torch.int32, idx=idx, count=count, prev_idx=prev_idx, prev_count=prev_count, host_rows_out=host_rows_out)
     _offsets(seq_offsets, count.numel())
     _offsets(prev_seq_offsets, prev_count.numel())
-    _dev(idx, count, seq_offsets, prev_idx, prev_count, prev_seq_offsets, prev_hot_kv, hot_kv, workspace,
-         host_rows_out)
     if pool.device.type != "cpu":
         raise ValueError("the cold pool must be (mapped page-locked) host memory")
     B = count.numel()
     row_bytes = pool.shape[1] * pool.element_size()
+    _cap(int(total_S), idx=idx)
+    _cap(int(prev_total_S), prev_idx=prev_idx)
+    _cap(1, host_rows_out=host_rows_out)
+    _cap_bytes(int(total_S) * row_bytes, pool=pool, hot_kv=hot_kv)
+    _cap_bytes(int(prev_total_S) * row_bytes, prev_hot_kv=prev_hot_kv)
+    _dev(idx, count, seq_offsets, prev_idx, prev_count, prev_seq_offsets, prev_hot_kv, hot_kv, workspace,
+         host_rows_out)
     _check(_lib.lsa_fetch_gather_incremental(
         _p(idx), _p(count), _p(seq_offsets), int(total_S), B, _p(prev_idx), _p(prev_count), _p(prev_seq_offsets),
         int(prev_total_S), _p(prev_hot_kv), _p(pool), row_bytes, _p(hot_kv), _p(host_rows_out), _p(workspace),
@@ -265,16 +297,22 @@ def lsa_lightning_topk(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, 
     _need(torch.float32, w_dec=w_dec, hot_scale=hot_scale, topk_score=topk_score)
     _need(torch.int32, idx=idx, count=count, topk_idx=topk_idx)
     _offsets(seq_offsets, q_dec.shape[0])
-    _dev(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, topk_score)
     B, tau, n_h, d_I = q_dec.shape
     kdt = LSA_FP8_E4M3 if hot_scale is not None else DTYPE_CODE[hot_K.dtype]
+    T = int(total_S)
+    _cap(B * tau * n_h, w_dec=w_dec)
+    _cap(T, idx=idx, hot_scale=hot_scale)
+    _cap(T * d_I, hot_K=hot_K)
+    _cap(B, count=count)
+    _cap(B * tau * int(k), topk_idx=topk_idx, topk_score=topk_score)
+    _dev(q_dec, w_dec, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, topk_score)
     _check(_lib.lsa_lightning_topk(_p(q_dec), _p(w_dec), _p(hot_K), _p(hot_scale), kdt,
                                    _p(idx), _p(count), _p(seq_offsets), int(total_S), B, tau, n_h, d_I, int(k),
                                    _p(topk_idx), _p(topk_score), _p(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
-# ------------------------------------------------------------------------ cold pool
+# ------------------------------------------------------------------------ golden labels, training step
 
 def lsa_golden_labels_workspace_size(tau, Lc, total_S) -> int:
     return int(_lib.lsa_golden_labels_workspace_size(tau, Lc, total_S))
@@ -286,9 +324,11 @@ def lsa_golden_labels(z, seq_offsets, label_out, workspace, p=0.6, theta=3, nsiz
     _need(torch.uint8, label_out=label_out)
     _need(torch.int32, nsize_out=nsize_out)
     _need(torch.int64, seq_offsets=seq_offsets)
-    _dev(z, seq_offsets, label_out, workspace, nsize_out)
     tau, Lc, T = z.shape
     B = seq_offsets.numel() - 1
+    _cap(T, label_out=label_out)
+    _cap(B * tau * Lc, nsize_out=nsize_out)
+    _dev(z, seq_offsets, label_out, workspace, nsize_out)
     _check(_lib.lsa_golden_labels(_p(z), _p(seq_offsets), T, B, tau, Lc, float(p), int(theta), _p(label_out),
                                   _p(nsize_out), _p(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)))
@@ -306,10 +346,16 @@ def lsa_indexer_train_step(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets,
     _need(torch.uint8, labels=labels)
     _need(torch.float64, loss_out=loss_out)
     _offsets(seq_offsets, h.shape[1])
-    _dev(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets, loss_out, g_Wdq, g_Wiuq, g_Ww, workspace)
     L, B, d = h.shape
     r = W_dq.shape[1]
     T = K.shape[1]
+    _cap(T, labels=labels)
+    _cap(L * T, k_scale=k_scale)
+    _cap(1, loss_out=loss_out)
+    _cap(W_dq.numel(), g_Wdq=g_Wdq)
+    _cap(W_iuq.numel(), g_Wiuq=g_Wiuq)
+    _cap(W_w.numel(), g_Ww=g_Ww)
+    _dev(h, W_dq, W_iuq, W_w, K, k_scale, labels, seq_offsets, loss_out, g_Wdq, g_Wiuq, g_Ww, workspace)
     _check(_lib.lsa_indexer_train_step(
         _p(h), _p(W_dq), _p(W_iuq), _p(W_w), DTYPE_CODE[h.dtype], _p(K), _p(k_scale), DTYPE_CODE[K.dtype], _p(labels),
         _p(seq_offsets), T, L, B, d, r, n_h, d_I, float(gamma), float(alpha), _p(loss_out), _p(g_Wdq), _p(g_Wiuq),
@@ -330,19 +376,27 @@ def lsa_lightning_topk_step(q_step, w_step, hot_K, hot_scale, idx, count, seq_of
     _need(torch.float32, w_step=w_step, hot_scale=hot_scale, win_scale=win_scale, topk_score=topk_score)
     _need(torch.int32, idx=idx, count=count, win_count=win_count, topk_idx=topk_idx)
     _offsets(seq_offsets, q_step.shape[0])
-    _dev(q_step, w_step, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, win_K, win_scale, win_count,
-         topk_score)
     B, n_h, d_I = q_step.shape
     if q_step.stride(2) != 1 or q_step.stride(1) != d_I or w_step.stride(1) != 1:
         raise ValueError("q_step rows and w_step rows must be contiguous (a batch stride is allowed)")
     if kdt is None:
         kdt = DTYPE_CODE[torch.float8_e4m3fn] if hot_scale is not None else DTYPE_CODE[hot_K.dtype]
     W = win_K.shape[1] if win_K is not None else 0
+    T = int(total_S)
+    _cap(T, idx=idx, hot_scale=hot_scale)
+    _cap(T * d_I, hot_K=hot_K)
+    _cap(B, count=count, win_count=win_count)
+    _cap(B * W, win_scale=win_scale)
+    _cap(B * int(k), topk_idx=topk_idx, topk_score=topk_score)
+    _dev(q_step, w_step, hot_K, hot_scale, idx, count, seq_offsets, topk_idx, workspace, win_K, win_scale, win_count,
+         topk_score)
     _check(_lib.lsa_lightning_topk_step(
         _p_rows(q_step), q_step.stride(0), _p_rows(w_step), w_step.stride(0), _p(hot_K), _p(hot_scale), kdt, _p(idx), _p(count),
         _p(seq_offsets), int(total_S), _p(win_K), _p(win_scale), _p(win_count), W, B, n_h, d_I, int(k), _p(topk_idx),
         _p(topk_score), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
+
+# ------------------------------------------------------------------------ cold pool
 
 class MappedPool:
     """Mapped page-locked host buffer from lsa_pool_alloc, viewed as a uint8 tensor [rows][row_bytes]."""

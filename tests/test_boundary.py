@@ -141,3 +141,41 @@ def test_binding_rejects_wrong_element_types_before_the_device():
                                          u8(10, 16), u8(10, 16), ws, host_rows_out=i64(1))
     with pytest.raises(ValueError, match="device tensor expected"):     # right types: the device check follows
         lsa.lsa_fetch_gather(i32(10), i32(2), i64(3), 10, None, None, bf(10, 128), None, bf(10, 128))
+
+
+def test_binding_rejects_buffers_smaller_than_the_call():
+    """Capacities follow from the sizes passed (total_S, B, k): a buffer too small for them is an
+    exception on the host, never a kernel writing past its end."""
+    import torch
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    i32 = lambda *s: torch.zeros(s, dtype=torch.int32)
+    i64 = lambda *s: torch.zeros(s, dtype=torch.int64)
+    f32 = lambda *s: torch.zeros(s, dtype=torch.float32)
+    bf = lambda *s: torch.zeros(s, dtype=torch.bfloat16)
+    u8 = lambda *s: torch.zeros(s, dtype=torch.uint8)
+    ws = u8(256)
+    with pytest.raises(ValueError, match="idx_out holds 9 elements, the call needs 10"):
+        lsa.lsa_memindex_score_select(bf(3, 2, 64, 128), f32(3, 2, 64), bf(3, 10, 128), None, i64(3), 10, 0.5,
+                                      i32(9), i32(2), ws)
+    with pytest.raises(ValueError, match="K holds 10 entries per layer, total_S is 11"):
+        lsa.lsa_memindex_score_select(bf(3, 2, 64, 128), f32(3, 2, 64), bf(3, 10, 128), None, i64(3), 11, 0.5,
+                                      i32(11), i32(2), ws)
+    with pytest.raises(ValueError, match="hot_kv holds 1008 bytes, the call needs 1024"):
+        lsa.lsa_fetch_gather(i32(64), i32(2), i64(3), 64, u8(64, 16), u8(63, 16))
+    with pytest.raises(ValueError, match="hot_K holds"):
+        lsa.lsa_fetch_gather(i32(10), i32(2), i64(3), 10, None, None, bf(10, 128), None, bf(9, 128))
+    with pytest.raises(ValueError, match="topk_idx holds"):
+        lsa.lsa_lightning_topk(bf(2, 4, 64, 128), f32(2, 4, 64), bf(10, 128), None, i32(10), i32(2), i64(3), 10, 8,
+                               i32(2, 4, 7), ws)
+    with pytest.raises(ValueError, match="topk_idx holds"):
+        lsa.lsa_lightning_topk_step(bf(2, 64, 128), f32(2, 64), bf(10, 128), None, i32(10), i32(2), i64(3), 10, 8,
+                                    i32(2, 4), ws)
+    with pytest.raises(ValueError, match="label_out holds"):
+        lsa.lsa_golden_labels(f32(2, 3, 10), i64(3), u8(9), ws)
+    with pytest.raises(ValueError, match="prev_hot_kv holds"):
+        lsa.lsa_fetch_gather_incremental(i32(10), i32(2), i64(3), 10, i32(10), i32(2), i64(3), 10, u8(9, 16),
+                                         u8(10, 16), u8(10, 16), ws)
+    with pytest.raises(ValueError, match="g_Wiuq holds"):
+        lsa.lsa_indexer_train_step(bf(3, 2, 64), bf(3, 32, 64), bf(3, 64 * 32, 32), bf(3, 64, 64), bf(3, 10, 32),
+                                   None, u8(10), i64(3), torch.zeros(1, dtype=torch.float64), f32(3, 32, 64),
+                                   f32(3, 64 * 32, 31), f32(3, 64, 64), ws, 64, 32)
