@@ -179,3 +179,44 @@ def test_binding_rejects_buffers_smaller_than_the_call():
         lsa.lsa_indexer_train_step(bf(3, 2, 64), bf(3, 32, 64), bf(3, 64 * 32, 32), bf(3, 64, 64), bf(3, 10, 32),
                                    None, u8(10), i64(3), torch.zeros(1, dtype=torch.float64), f32(3, 32, 64),
                                    f32(3, 64 * 32, 31), f32(3, 64, 64), ws, 64, 32)
+
+
+def test_binding_host_checks_pass_well_formed_calls():
+    """Well-typed, large enough CPU tensors get through every host-side check of every call and
+    stop only at the device check (the C library is not called)."""
+    import torch
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    i32 = lambda *s: torch.zeros(s, dtype=torch.int32)
+    i64 = lambda *s: torch.zeros(s, dtype=torch.int64)
+    f32 = lambda *s: torch.zeros(s, dtype=torch.float32)
+    bf = lambda *s: torch.zeros(s, dtype=torch.bfloat16)
+    u8 = lambda *s: torch.zeros(s, dtype=torch.uint8)
+    e4 = lambda *s: torch.zeros(s, dtype=torch.float8_e4m3fn)
+    ws = u8(256)
+    L, B, T, d, r, nh, dI, tau, k, W = 3, 2, 10, 64, 32, 64, 128, 4, 8, 4
+    calls = [
+        lambda: lsa.lsa_project(bf(L, B, d), bf(L, r, d), bf(L, nh * dI, r), bf(L, nh, d), bf(L, B, nh, dI),
+                                f32(L, B, nh), ws),
+        lambda: lsa.lsa_memindex_score_select(bf(L, B, nh, dI), f32(L, B, nh), e4(L, T, dI), f32(L, T), i64(B + 1), T,
+                                              0.5, i32(T), i32(B), ws, scores_out=f32(L, T), mask_out=u8(T)),
+        lambda: lsa.lsa_memindex_score_select_static(f32(L, B, nh, dI), f32(L, B, nh), f32(L, T, dI), None,
+                                                     i64(B + 1), T, 0.5, i32(T), i32(B)),
+        lambda: lsa.lsa_fetch_gather(i32(T), i32(B), i64(B + 1), T, u8(T, 64), u8(T, 64), e4(T, dI), f32(T),
+                                     bf(T, dI), f32(T)),
+        lambda: lsa.lsa_fetch_gather_incremental(i32(T), i32(B), i64(B + 1), T, i32(T), i32(B), i64(B + 1), T,
+                                                 u8(T, 64), u8(T, 64), u8(T, 64), ws, host_rows_out=i32(1)),
+        lambda: lsa.lsa_lightning_topk(bf(B, tau, nh, dI), f32(B, tau, nh), bf(T, dI), f32(T), i32(T), i32(B),
+                                       i64(B + 1), T, k, i32(B, tau, k), ws, topk_score=f32(B, tau, k)),
+        lambda: lsa.lsa_lightning_topk_step(bf(B, tau, nh, dI)[:, 1], f32(B, tau, nh)[:, 1], bf(T, dI), f32(T),
+                                            i32(T), i32(B), i64(B + 1), T, k, i32(B, k), ws, win_K=bf(B, W, dI),
+                                            win_scale=f32(B, W), win_count=i32(B), topk_score=f32(B, k)),
+        lambda: lsa.lsa_golden_labels(f32(tau, 5, T), i64(B + 1), u8(T), ws, nsize_out=i32(B, tau, 5)),
+        lambda: lsa.lsa_indexer_train_step(bf(L, B, d), bf(L, r, d), bf(L, nh * dI, r), bf(L, nh, d), e4(L, T, dI),
+                                           f32(L, T), u8(T), i64(B + 1), torch.zeros(1, dtype=torch.float64),
+                                           f32(L, r, d), f32(L, nh * dI, r), f32(L, nh, d), ws, nh, dI),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="device tensor expected"):
+            call()
+    with pytest.raises(TypeError, match="q_out must be torch.bfloat16"):
+        lsa.lsa_project(bf(L, B, d), bf(L, r, d), bf(L, nh * dI, r), bf(L, nh, d), f32(L, B, nh, dI), f32(L, B, nh), ws)
