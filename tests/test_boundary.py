@@ -220,3 +220,23 @@ def test_binding_host_checks_pass_well_formed_calls():
             call()
     with pytest.raises(TypeError, match="q_out must be torch.bfloat16"):
         lsa.lsa_project(bf(L, B, d), bf(L, r, d), bf(L, nh * dI, r), bf(L, nh, d), f32(L, B, nh, dI), f32(L, B, nh), ws)
+
+
+def test_build_from_a_clean_tree(tmp_path):
+    """__graft_entry__.build() on the committed sources alone (no liblsa.so or oracle library yet)
+    compiles both and imports the package."""
+    import shutil
+    if shutil.which("nvcc") is None or shutil.which("gcc") is None:
+        pytest.skip("nvcc and gcc are needed")
+    files = subprocess.run(["git", "ls-files"], cwd=ROOT, capture_output=True, text=True, check=True).stdout.split()
+    for f in files:
+        dst = tmp_path / f
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy2(os.path.join(ROOT, f), dst)
+    assert not (tmp_path / "sparse_kv_cache_memoryindexer_b200" / "liblsa.so").exists()
+    r = subprocess.run(["python", "-c", "import __graft_entry__ as g; g.build(); "
+                        "import sparse_kv_cache_memoryindexer_b200 as m, oracle; print(m.version(), oracle.threads())"],
+                       cwd=tmp_path, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    assert (tmp_path / "sparse_kv_cache_memoryindexer_b200" / "liblsa.so").exists()
+    assert (tmp_path / "oracle" / "liblsa_oracle.so").exists()
