@@ -518,7 +518,7 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     int *item_counter = item_start + B + 1;
     float *Y = (float *)((char *)workspace + align_up(sizeof(int) * (size_t)(B + 2), 256));
     // E4M3 keys arrive here decoded to bf16 by lsa_fetch_gather (scales in hot_scale)
-    const int hdt = (kdt == LSA_FP8_E4M3) ? DT_BF16 : kdt;
+    const int hdt = (kdt == LSA_FP8_E4M3) ? (int)DT_BF16 : (int)kdt;
     if (li_tc_supported(n_h, d_I, tau, kdt)) {
         LSA_REQUIRE(aligned(q_dec, 16) && aligned(hot_K, 16), "lsa_lightning_topk: q_dec and hot_K must be 16-byte aligned");
         int n = 0;
@@ -619,7 +619,7 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     float *tail = (float *)(p + part[0] + part[1]);
     void *qw = (void *)(p + part[0] + part[1] + part[2]);
     float *ww = (float *)(p + part[0] + part[1] + part[2] + part[3]);
-    const int hdt = (kdt == LSA_FP8_E4M3) ? DT_BF16 : kdt;  // hot keys: E4M3 arrives decoded to bf16
+    const int hdt = (kdt == LSA_FP8_E4M3) ? (int)DT_BF16 : (int)kdt;  // hot keys: E4M3 arrives decoded to bf16
     // one query per sequence: the tensor-core scorer runs with one-query groups (MMA N = n_h)
     const bool tc = li_tc_supported(n_h, d_I, 1, kdt, 1);
     const int TQ = 1;
@@ -779,8 +779,6 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
     int *tile_start = (int *)(p + part[0] + part[1] + part[2] + part[3] + part[4] + part[5]);
     int *chunk_start = tile_start + (B + 1);
     int32_t *cnt = chunk_start + (B + 1);
-    double *loss = (double *)(p + part[0] + part[1] + part[2] + part[3] + part[4] + part[5] + part[6]);
-    (void)loss;
     const int nq = n_h * d_I;
     cudaError_t e = cudaMemsetAsync(dq, 0, part[3] + part[4], st);  // dq and dw are adjacent
     if (e == cudaSuccess) e = cudaMemsetAsync(loss_out, 0, sizeof(double), st);

@@ -269,7 +269,6 @@ __global__ void __launch_bounds__(TH) k_ss_write(const float *__restrict__ Y, in
                                                  unsigned long long *__restrict__ sel)
 {
     __shared__ int warp_tot[32];
-    __shared__ int tot_a, tot_b;
     const int c = blockIdx.x;
     if (c >= chunk_start[B]) return;
     const int b = query_of_chunk(chunk_start, B, c);
@@ -314,8 +313,6 @@ __global__ void __launch_bounds__(TH) k_ss_write(const float *__restrict__ Y, in
         carry_gt += tot[0];
         carry_eq += tot[1];
     }
-    (void)tot_a;
-    (void)tot_b;
 }
 
 __global__ void __launch_bounds__(SORT_TH) k_ss_sort(const unsigned long long *__restrict__ sel, int kcap,
