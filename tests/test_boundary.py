@@ -12,7 +12,8 @@ HDR = os.path.join(ROOT, "include", "lsa.h")
 
 
 def declared():
-    src = open(HDR).read()
+    with open(HDR) as f:
+        src = f.read()
     return sorted(set(re.findall(r"^(?:lsa_status|size_t|const char \*|uint64_t)\s*\*?\s*(lsa_\w+)\(", src, re.M)))
 
 
@@ -35,7 +36,8 @@ def test_library_exports_every_declared_symbol():
 
 def test_library_is_built_for_sm100a_only():
     from sparse_kv_cache_memoryindexer_b200 import build
-    log = open(os.path.join(os.path.dirname(build.LIB), "build.log")).read().splitlines()[0]
+    with open(os.path.join(os.path.dirname(build.LIB), "build.log")) as f:
+        log = f.read().splitlines()[0]
     assert "arch=compute_100a,code=sm_100a" in log
 
 
