@@ -69,6 +69,13 @@ uint64_t lsa_launch_count(void);
  * Returns LSA_OK, LSA_ERR_DEVICE_CHECK (message lists the flags) or LSA_ERR_CUDA. */
 lsa_status lsa_check_device(lsa_stream_t stream);
 
+/* Self-test of the failure detection: one CTA waits, bounded, on a barrier that nothing completes.
+ * The wait gives up after its limit (2 s, the limit of every wait inside the pipelined kernels),
+ * sets the device error word (pipeline-wait-timeout, read by lsa_check_device) and the kernel
+ * returns; the context stays usable.  status_out: device int32 [2], written with {0, 1} (the wait
+ * did not complete; the CTA's abort flag is set).  Asynchronous on `stream`. */
+lsa_status lsa_selftest_wait_timeout(int32_t *status_out, lsa_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Stage 1 -- Memory-Indexer projections (blog review section 3.1):
  *     c^Q = h W^DQ,   q = c^Q W^IUQ,   w = h W^w,   for each layer l and sequence b.

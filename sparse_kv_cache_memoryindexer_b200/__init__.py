@@ -7,7 +7,8 @@ from .lsa import (LSAError, MappedPool, lsa_check_device, lsa_fetch_gather, lsa_
                   lsa_indexer_train_workspace_size,
                   lsa_lightning_topk_workspace_size, lsa_memindex_score_select,
                   lsa_memindex_score_select_static, lsa_project,
-                  lsa_project_workspace_size, lsa_score_select_workspace_size, launch_count, version)
+                  lsa_project_workspace_size, lsa_score_select_workspace_size, lsa_selftest_wait_timeout,
+                  launch_count, version)
 from .pipeline import IndexerPath
 
 __all__ = ["LSAError", "MappedPool", "IndexerPath", "lsa_check_device", "lsa_fetch_gather",
@@ -17,4 +18,4 @@ __all__ = ["LSAError", "MappedPool", "IndexerPath", "lsa_check_device", "lsa_fet
            "lsa_indexer_train_step", "lsa_indexer_train_workspace_size", "lsa_memindex_score_select",
            "lsa_memindex_score_select_static",
            "lsa_project", "lsa_project_workspace_size", "lsa_score_select_workspace_size",
-           "launch_count", "version"]
+           "lsa_selftest_wait_timeout", "launch_count", "version"]

@@ -18,6 +18,7 @@
 #include "train.cuh"
 #include "step_select.cuh"
 #include "topk.cuh"
+#include "selftest.cuh"
 
 using namespace lsa;
 
@@ -220,6 +221,14 @@ lsa_status lsa_check_device(lsa_stream_t stream)
                 (word & ERRF_OFFSETS) ? " bad-seq-offsets" : "", (word & ERRF_INDEX) ? " index-out-of-range" : "",
                 (word & ERRF_COUNT) ? " count-out-of-range" : "", (word & ERRF_SCALE) ? " bad-key-scale" : "",
                 (word & ERRF_TIMEOUT) ? " pipeline-wait-timeout" : "");
+}
+
+lsa_status lsa_selftest_wait_timeout(int32_t *status_out, lsa_stream_t stream)
+{
+    LSA_REQUIRE(status_out, "lsa_selftest_wait_timeout: null pointer");
+    k_selftest_wait<<<1, 32, 0, (cudaStream_t)stream>>>(status_out);
+    LSA_TRY(launched("self-test: bounded wait"));
+    return ok();
 }
 
 // ------------------------------------------------------------------------------ stage 1

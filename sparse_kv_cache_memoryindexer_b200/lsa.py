@@ -22,7 +22,7 @@ _STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "
 DTYPE_CODE = {torch.float32: LSA_F32, torch.bfloat16: LSA_BF16, torch.float8_e4m3fn: LSA_FP8_E4M3}
 
 # every function declared in include/lsa.h
-EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_device",
+EXPORTS = ("lsa_last_error", "lsa_version", "lsa_launch_count", "lsa_check_device", "lsa_selftest_wait_timeout",
            "lsa_project_workspace_size", "lsa_project",
            "lsa_score_select_workspace_size", "lsa_memindex_score_select",
            "lsa_memindex_score_select_static",
@@ -51,6 +51,7 @@ def _load():
         "lsa_version": (C.c_char_p, []),
         "lsa_launch_count": (C.c_uint64, []),
         "lsa_check_device": (I, [P]),
+        "lsa_selftest_wait_timeout": (I, [P, P]),
         "lsa_project_workspace_size": (SZ, [I, I, I, I, I, I, I]),
         "lsa_project": (I, [P, P, P, P, I, I, I, I, I, I, I, P, P, P, SZ, P]),
         "lsa_score_select_workspace_size": (SZ, [I, I, I64]),
@@ -156,6 +157,15 @@ def launch_count() -> int:
 
 def lsa_check_device(stream=None):
     _check(_lib.lsa_check_device(_stream(stream)))
+
+
+def lsa_selftest_wait_timeout(status_out, stream=None):
+    """A bounded wait that nothing completes gives up after 2 s and flags the device error word
+    (see include/lsa.h); status_out: device int32 [2]."""
+    _need(torch.int32, status_out=status_out)
+    _cap(2, status_out=status_out)
+    _dev(status_out)
+    _check(_lib.lsa_selftest_wait_timeout(_p(status_out), _stream(stream)))
 
 
 # ------------------------------------------------------------------------ stage 1
