@@ -171,19 +171,6 @@ def test_gather_rows_many_ragged_sequences(m):
         gather_and_check(m, wl, inp, idx, cnt, "split")
 
 
-@pytest.mark.parametrize("mode", ["both", "split"])
-@pytest.mark.parametrize("row_bytes", [48, 1040, 2048])
-def test_gather_row_sizes(m, row_bytes, mode):
-    """Rows of 3 chunks of 16 bytes (most lanes idle), of 65 chunks (one lane in the third round) and
-    of 128 chunks, the largest row the fetch takes (four chunks per lane): every variant of the
-    rows-only launch and the chunk masks of the combined one, with E4M3 keys decoded alongside."""
-    wl = synth.workload("ctx1m_fp8_b32", B=3, S=(3000, 0, 1291), fetch=(0.2, 0.2, 0.2), row_bytes=row_bytes,
-                        name=f"rows{row_bytes}")
-    inp = synth.make_inputs(wl, parts=("score", "pool"))
-    idx, cnt = synth.random_fetch_list(wl, 0.3, seed=8)
-    gather_and_check(m, wl, inp, idx, cnt, mode)
-
-
 # ------------------------------------------------------------------ stage 5
 
 def run_topk(m, inp, idx, cnt, k, pool_needed=False):
@@ -415,3 +402,18 @@ def test_select_e4m3_all_codes(m):
     ref = oracle.score(inp.q, inp.w, inp.K, inp.k_scale, offs)
     mask, idx, cnt, I = run_select(m, inp)
     check_select(mask, idx, cnt, I, ref, offs, what="all codes")
+
+
+# ------------------------------------------------------------------ stage 4b: row sizes
+
+@pytest.mark.parametrize("mode", ["both", "split"])
+@pytest.mark.parametrize("row_bytes", [48, 1040, 2048])
+def test_gather_row_sizes(m, row_bytes, mode):
+    """Rows of 3 chunks of 16 bytes (most lanes idle), of 65 chunks (one lane in the third round) and
+    of 128 chunks, the largest row the fetch takes (four chunks per lane): every variant of the
+    rows-only launch and the chunk masks of the combined one, with E4M3 keys decoded alongside."""
+    wl = synth.workload("ctx1m_fp8_b32", B=3, S=(3000, 0, 1291), fetch=(0.2, 0.2, 0.2), row_bytes=row_bytes,
+                        name=f"rows{row_bytes}")
+    inp = synth.make_inputs(wl, parts=("score", "pool"))
+    idx, cnt = synth.random_fetch_list(wl, 0.3, seed=8)
+    gather_and_check(m, wl, inp, idx, cnt, mode)
