@@ -165,3 +165,22 @@ def test_topk_sampled_queries(window):
         tol = li_tolerance(inp.q_dec[b, i], inp.w_dec[b, i], Kf)
         y = ref["y"][n, offs[b]:offs[b] + F]
         check_topk_query(ti[b, i], ts[b, i], y, s_list, tol, wl.k, what=f"{wl.name} query ({b}, {i})")
+
+
+def test_decode_step_equals_batched_column(window, m):
+    """The per-step call at full size, without window entries: step i's Top-k (indices and scores)
+    equals column i of the window's batched call bit for bit (the same products and head sums, the
+    same ordering of equal scores).  The small-size tests pin both against the oracle."""
+    wl, inp, _, path = window
+    T = wl.total_S
+    qd, wd, offs = inp.q_dec.cuda(), inp.w_dec.cuda(), inp.seq_offsets.cuda()
+    ti = torch.empty((wl.B, wl.k), dtype=torch.int32, device="cuda")
+    ts = torch.empty((wl.B, wl.k), dtype=torch.float32, device="cuda")
+    ws = torch.empty(m.lsa_lightning_topk_step_workspace_size(wl.B, T, wl.n_h, wl.d_I, 0), dtype=torch.uint8,
+                     device="cuda")
+    for i in (0, wl.tau - 1):
+        m.lsa_lightning_topk_step(qd[:, i], wd[:, i], path.hot_K, path.hot_scale, path.idx, path.count, offs, T,
+                                  wl.k, ti, ws, topk_score=ts)
+        m.lsa_check_device()
+        assert torch.equal(ti, path.topk_idx[:, i]), f"{wl.name} step {i}: indices differ"
+        assert torch.equal(ts, path.topk_score[:, i]), f"{wl.name} step {i}: scores differ"
