@@ -6,9 +6,21 @@ review's sections 3-3.2: project -> score/threshold/OR/compact -> fetch -> Light
 """
 from __future__ import annotations
 
+from contextlib import contextmanager
+
 import torch
 
 from . import lsa
+
+
+@contextmanager
+def _stage(name):
+    """NVTX range around a stage's launches (ncu --nvtx / nsys show the stage boundaries)."""
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
 
 
 class IndexerPath:
@@ -85,20 +97,25 @@ class IndexerPath:
         ev = events if events is not None else [None] * 7
         rec = lambda e, s: e.record(s) if e is not None else None
         rec(ev[0], st)
-        self.project(h, W_dq, W_iuq, W_w, st)
+        with _stage("lsa.project"):
+            self.project(h, W_dq, W_iuq, W_w, st)
         rec(ev[1], st)
-        self.select(K, k_scale, seq_offsets, threshold, stream=st)
+        with _stage("lsa.score_select"):
+            self.select(K, k_scale, seq_offsets, threshold, stream=st)
         rec(ev[2], st)
         selected = torch.cuda.Event()
         selected.record(st)
         self._link.wait_event(selected)
-        self.fetch_rows(seq_offsets, pool, self._link)
+        with _stage("lsa.fetch_rows"):
+            self.fetch_rows(seq_offsets, pool, self._link)
         rec(ev[5], self._link)
         rows_done = torch.cuda.Event()
         rows_done.record(self._link)
-        self.fetch_keys(seq_offsets, K[sel_layer], None if k_scale is None else k_scale[sel_layer], st)
+        with _stage("lsa.fetch_keys"):
+            self.fetch_keys(seq_offsets, K[sel_layer], None if k_scale is None else k_scale[sel_layer], st)
         rec(ev[3], st)
-        self.topk(q_dec, w_dec, seq_offsets, st)
+        with _stage("lsa.lightning_topk"):
+            self.topk(q_dec, w_dec, seq_offsets, st)
         rec(ev[4], st)
         st.wait_event(rows_done)
         rec(ev[6], st)
