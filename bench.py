@@ -239,7 +239,7 @@ def algorithmic(wl, fetched_total):
     qb = eb[wl.dtype]
     nq = wl.n_h * wl.d_I
     proj_bytes = L * (wl.r * wl.d + nq * wl.r + wl.n_h * wl.d) * qb + L * B * (wl.d * qb + nq * qb + wl.n_h * 4)
-    score_bytes = L * T * kb + L * B * (nq * qb + wl.n_h * 4) + T // 8 + 4 * T * 0  # keys + queries + mask bits
+    score_bytes = L * T * kb + L * B * (nq * qb + wl.n_h * 4) + T // 8  # keys + queries and weights + fetch bits
     gather_host = fetched_total * wl.row_bytes                            # crosses the host link
     gather_dev = fetched_total * (wl.row_bytes + wl.d_I * eb[wl.kdtype] * 2 + 8)
     # keys gather: read the key row (+ scale) and the index, write the hot key (bf16 for E4M3) (+ scale)
