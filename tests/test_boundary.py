@@ -242,3 +242,23 @@ def test_build_from_a_clean_tree(tmp_path):
     assert r.returncode == 0, r.stderr[-3000:]
     assert (tmp_path / "sparse_kv_cache_memoryindexer_b200" / "liblsa.so").exists()
     assert (tmp_path / "oracle" / "liblsa_oracle.so").exists()
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/lsa.h is a C header (C99, no C++ or CUDA types) and a C program links against the
+    library with it."""
+    import shutil
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    from sparse_kv_cache_memoryindexer_b200 import lsa
+    src = tmp_path / "use.c"
+    src.write_text('#include "lsa.h"\n#include <stdio.h>\n'
+                   'static lsa_status (*const check)(lsa_stream_t) = lsa_check_device;\n'
+                   'int main(void) {\n'
+                   '  size_t ws = lsa_score_select_workspace_size(3, 2, 100);\n'
+                   '  printf("%s %llu %zu\\n", lsa_version(), (unsigned long long)lsa_launch_count(), ws);\n'
+                   '  return check == NULL; }\n')
+    libdir = os.path.dirname(lsa.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-L", libdir, "-llsa", "-o", str(tmp_path / "use")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
