@@ -220,13 +220,14 @@ __global__ void __launch_bounds__(TH) k_ss_count(const float *__restrict__ Y, in
     const int nc = q.F0 + q.nt;
     const int j0 = (c - chunk_start[b]) * CH, j1 = min(nc, j0 + CH);
     const uint32_t K = state[4 * b + 0];
+    const bool all = state[4 * b + 1] == 0u;  // at most k candidates: every one, whatever its key
     if (threadIdx.x == 0) sgt = seq = 0;
     __syncthreads();
     int ng = 0, ne = 0;
     for (int j = j0 + threadIdx.x; j < j1; j += TH) {
         const uint32_t u = key_of(q, j);
-        ng += u > K;
-        ne += u == K;
+        ng += (all || u > K) ? 1 : 0;
+        ne += (!all && u == K) ? 1 : 0;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -277,6 +278,7 @@ __global__ void __launch_bounds__(TH) k_ss_write(const float *__restrict__ Y, in
     const int j0 = (c - chunk_start[b]) * CH, j1 = min(nc, j0 + CH);
     const uint32_t K = state[4 * b + 0];
     const int want_eq = (int)state[4 * b + 1], n_gt = (int)state[4 * b + 2];
+    const bool all = want_eq == 0;  // at most k candidates: every one, whatever its key
     unsigned long long *out = sel + (int64_t)b * kcap;
     int carry_gt = gtb[c], carry_eq = eqb[c];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -286,8 +288,8 @@ __global__ void __launch_bounds__(TH) k_ss_write(const float *__restrict__ Y, in
         int gt = 0, eq = 0;
         if (j < j1) {
             u = key_of(q, j);
-            gt = u > K;
-            eq = u == K;
+            gt = (all || u > K) ? 1 : 0;
+            eq = (!all && u == K) ? 1 : 0;
         }
         // block exclusive scans of gt and eq
         int pos[2];
@@ -348,8 +350,9 @@ __global__ void __launch_bounds__(SORT_TH) k_ss_sort(const unsigned long long *_
         const int64_t o = (int64_t)b * k + r;
         if (r < nsel) {
             const unsigned long long v = sk[r];
-            const uint32_t j = ~(uint32_t)(v & 0xffffffffull);
-            topk_idx[o] = ((int)j < F0) ? __ldg(idx + off + j) : (int32_t)(S + (j - F0));
+            const int j = (int)~(uint32_t)(v & 0xffffffffull);  // candidate slot
+            topk_idx[o] = (j >= 0 && j < F0) ? __ldg(idx + off + j)
+                                             : ((j >= F0 && j < nc) ? (int32_t)(S + (j - F0)) : -1);
             if (topk_score) topk_score[o] = ordered_to_float((uint32_t)(v >> 32));
         } else {
             topk_idx[o] = -1;

@@ -196,8 +196,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
     for (int r = threadIdx.x; r < k; r += SEL_THREADS) {
         if (r < nsel) {
             const unsigned long long v = sel[r];
-            const uint32_t j = ~(uint32_t)(v & 0xffffffffull);
-            topk_idx[o0 + r] = ((int)j < F0) ? __ldg(idx + off + j) : (int32_t)(S + (j - F0));
+            const int j = (int)~(uint32_t)(v & 0xffffffffull);  // candidate slot (always below F)
+            topk_idx[o0 + r] = (j >= 0 && j < F0) ? __ldg(idx + off + j)
+                                                  : ((j >= F0 && j < F) ? (int32_t)(S + (j - F0)) : -1);
             if (topk_score) topk_score[o0 + r] = ordered_to_float((uint32_t)(v >> 32));
         } else {
             topk_idx[o0 + r] = -1;
