@@ -120,3 +120,163 @@ def check_project(h, W_dq, W_iuq, W_w, n_h, d_I, q_gpu, w_gpu, c_gpu, what=""):
     assert (dq <= ulp(q_gpu.double(), q2.double()).reshape(qb.shape) * 1.0001 + qb).all(), f"{what}: q"
     if bf:
         assert (dq > 0).double().mean() < 0.05, f"{what}: too many q differ"
+
+
+# ------------------------------------------------------------------------------ training step
+
+def exact_train_case(dt, kdt, L=2, S=(300, 0, 129, 517), d=512, r=256, n_h=64, d_I=128, seed=7, h_nz=24,
+                     wiuq_nz=8, label_rate=0.25):
+    """Inputs of one indexer training step on which every forward quantity is exact in fp32 on the
+    GPU, in bf16/E4M3 storage and in the oracle's double: h has h_nz entries of +-1 per (layer,
+    sequence), W^DQ entries are -1, 0 or 1 (so |c| <= h_nz), each W^IUQ row has wiuq_nz entries +-1
+    (so q is an integer of magnitude <= h_nz * wiuq_nz <= 256, exact in bf16), W^w entries are
+    {-1, 0, 1} / 32 and keys {-1, 0, 1} times a power of two (bf16 values 2^-6; E4M3 codes with
+    per-entry scales 2^-6 or 2^-7).  The head dot products, the ReLU gates and the logits are then
+    the same on both sides (`train_bounds` asserts the premise), so the two sides differ only by the
+    fp32 evaluation of the loss derivative and the fp32 sums of the gradients.
+
+    dt: torch.float32 or torch.bfloat16 (h and weights); kdt: the key type (float32, bfloat16 or
+    float8_e4m3fn).  Returns (h, [W_dq, W_iuq, W_w], K, k_scale, labels, seq_offsets, n_h, d_I).
+    """
+    rng = np.random.default_rng(seed)
+    B = len(S)
+    nq = n_h * d_I
+    offs = np.concatenate([[0], np.cumsum(S)]).astype(np.int64)
+    T = int(offs[-1])
+    h = np.zeros((L, B, d))
+    for l in range(L):
+        for b in range(B):
+            pos = rng.choice(d, h_nz, replace=False)
+            h[l, b, pos] = rng.choice([-1.0, 1.0], h_nz)
+    W_dq = rng.integers(-1, 2, size=(L, r, d)).astype(np.float64)
+    W_iuq = np.zeros((L, nq, r))
+    for l in range(L):
+        cols = np.argsort(rng.random((nq, r)), axis=1)[:, :wiuq_nz]
+        W_iuq[l, np.arange(nq)[:, None], cols] = rng.choice([-1.0, 1.0], (nq, wiuq_nz))
+    W_w = rng.integers(-1, 2, size=(L, n_h, d)) / 32.0
+    codes = rng.integers(-1, 2, size=(L, T, d_I)).astype(np.float64)
+    labels = (rng.random(T) < label_rate).astype(np.uint8)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dt)
+    if kdt == torch.float8_e4m3fn:
+        K = torch.from_numpy(codes.astype(np.float32)).to(kdt)
+        k_scale = torch.from_numpy(rng.choice([2.0 ** -6, 2.0 ** -7], (L, T)).astype(np.float32))
+    else:
+        K = torch.from_numpy((codes * 2.0 ** -6).astype(np.float32)).to(kdt)
+        k_scale = None
+    return (t(h), [t(W_dq), t(W_iuq), t(W_w)], K, k_scale, torch.from_numpy(labels), torch.from_numpy(offs),
+            n_h, d_I)
+
+
+def _focal_terms(x, y, gamma, alpha):
+    """Per-entry focal loss and its derivative in the logit (binary cross-entropy at gamma = 0,
+    alpha < 0), in double."""
+    p = 1.0 / (1.0 + np.exp(-x))
+    pt = np.where(y, p, 1.0 - p)
+    at = np.ones_like(x) if alpha < 0 else np.where(y, alpha, 1.0 - alpha)
+    lpt = np.where(y, -np.log1p(np.exp(-x)), -np.log1p(np.exp(x)))
+    q1 = 1.0 - pt
+    loss = -at * q1 ** gamma * lpt
+    if gamma == 0.0:
+        dl = at * np.where(y, p - 1.0, p)
+    else:
+        dl = at * (gamma * q1 ** (gamma - 1.0) * lpt * pt * q1 - q1 ** gamma * q1) * np.where(y, 1.0, -1.0)
+    return loss, dl, at
+
+
+def train_bounds(case, gamma=0.0, alpha=-1.0):
+    """Per-element bounds on |GPU - oracle| for the loss and the three weight gradients of one
+    training step on exact inputs (`exact_train_case`).
+
+    The forward is exact on both sides (asserted here), so the differences are:
+      * the loss derivative g_s = dl/dx / N, evaluated in fp32 from an exact logit: its absolute
+        error is below 2^-18 a_t / N for binary cross-entropy and the focal loss with gamma <= 2
+        (a few ulps of each fp32 factor; |dl/dx| <= a_t), and G_sh = g_s w_h scale_s is two more
+        fp32 roundings (2^-23 relative);
+      * every fp32 sum, in whatever order (register tiles, warp shuffles, atomics, tensor-core
+        accumulation): at most 2^-22 m sum |term|, m the number of its nonzero terms (four times the
+        classical m 2^-24 bound; adding an exact zero rounds nothing, and these inputs are sparse);
+      * the errors of dq and dw carried through dc = dq W^IUQ and the outer products over sequences.
+    Returns dict with the exact forward's magnitudes and the bounds E_loss, E_g_Wdq, E_g_Wiuq, E_g_Ww.
+    """
+    h, (W_dq, W_iuq, W_w), K, k_scale, labels, offs, n_h, d_I = case
+    L, B, d = h.shape
+    r = W_dq.shape[1]
+    nq = n_h * d_I
+    offs = np.asarray(offs)
+    T = int(offs[-1])
+    N = float(L * T)
+    H = h.double().numpy()
+    Wdq, Wiuq, Ww = W_dq.double().numpy(), W_iuq.double().numpy(), W_w.double().numpy()
+    Kraw = K.float().double().numpy()                                  # stored values (E4M3: the codes)
+    sc = k_scale.double().numpy() if k_scale is not None else np.ones((L, T))
+    c = np.einsum("lbi,lji->lbj", H, Wdq)
+    q = np.einsum("lbj,loj->lbo", c, Wiuq)
+    w = np.einsum("lbi,lhi->lbh", H, Ww)
+    assert np.all(np.abs(c) <= 256) and np.all(c == np.round(c)), "premise: c exact in bf16"
+    assert np.all(np.abs(q) <= 256) and np.all(q == np.round(q)), "premise: q exact in bf16"
+    y = np.asarray(labels).astype(bool)
+    u22, u23 = 2.0 ** -22, 2.0 ** -23
+    E_dq = np.zeros((L, B, nq))
+    A_dq = np.zeros((L, B, nq))   # |dq| + E_dq
+    E_dw = np.zeros((L, B, n_h))
+    A_dw = np.zeros((L, B, n_h))
+    loss_abs = 0.0
+    loss = 0.0
+    for l in range(L):
+        for b in range(B):
+            s0, s1 = int(offs[b]), int(offs[b + 1])
+            S = s1 - s0
+            if S == 0:
+                continue
+            Kr = Kraw[l, s0:s1]
+            scs = sc[l, s0:s1]
+            qh = q[l, b].reshape(n_h, d_I)
+            a = (Kr @ qh.T) * scs[:, None]                            # [S][n_h], exact
+            relu = np.maximum(a, 0.0)
+            wx = np.abs(w[l, b])[None, :] * relu
+            assert wx.sum(1).max() < 2.0 ** 12, "premise: logits exact in fp32"
+            x = (w[l, b][None, :] * relu).sum(1)
+            ls, dl, at = _focal_terms(x, y[s0:s1], gamma, alpha)
+            loss += ls.sum()
+            loss_abs += np.abs(ls).sum()
+            g = dl / N
+            dg = 2.0 ** -18 * at / N
+            pos = a > 0
+            G = g[:, None] * w[l, b][None, :] * scs[:, None] * pos
+            dG = (dg[:, None] * np.abs(w[l, b])[None, :] * scs[:, None] + u23 * np.abs(G)) * pos
+            aK = np.abs(Kr)
+            m = (G != 0).T.astype(np.float64) @ (aK > 0)              # nonzero terms of each dq sum
+            e = dG.T @ aK + u22 * m * (np.abs(G).T @ aK)              # [n_h][d_I]
+            E_dq[l, b] = e.reshape(nq)
+            A_dq[l, b] = np.abs(G.T @ Kr).reshape(nq) + E_dq[l, b]
+            mw = (g != 0).astype(np.float64) @ (relu > 0)
+            E_dw[l, b] = dg @ relu + u22 * mw * (np.abs(g) @ relu)
+            A_dw[l, b] = np.abs(g @ relu) + E_dw[l, b]
+    nz = lambda x: (x != 0).astype(np.float64)
+    aW = np.abs(Wiuq)
+    m_dc = np.einsum("lbo,loj->lbj", nz(A_dq), nz(Wiuq))
+    E_dc = np.einsum("lbo,loj->lbj", E_dq, aW) + u22 * m_dc * np.einsum("lbo,loj->lbj", A_dq, aW)
+    A_dc = np.einsum("lbo,loj->lbj", A_dq, aW) + E_dc                  # a bound on |dc| + its error
+    ac, aH = np.abs(c), np.abs(H)
+    m_iuq = np.einsum("lbo,lbj->loj", nz(A_dq), nz(c))
+    m_wdq = np.einsum("lbj,lbi->lji", nz(A_dc), nz(H))
+    m_ww = np.einsum("lbh,lbi->lhi", nz(A_dw), nz(H))
+    E_iuq = np.einsum("lbo,lbj->loj", E_dq, ac) + u22 * m_iuq * np.einsum("lbo,lbj->loj", A_dq, ac)
+    E_wdq = np.einsum("lbj,lbi->lji", E_dc, aH) + u22 * m_wdq * np.einsum("lbj,lbi->lji", A_dc, aH)
+    E_ww = np.einsum("lbh,lbi->lhi", E_dw, aH) + u22 * m_ww * np.einsum("lbh,lbi->lhi", A_dw, aH)
+    return {"loss": loss / N, "E_loss": 2.0 ** -20 * loss_abs / N + 1e-15,
+            "E_g_Wdq": E_wdq, "E_g_Wiuq": E_iuq, "E_g_Ww": E_ww}
+
+
+def check_train(loss, grads, ref, bounds, what=""):
+    """loss (float) and grads (g_Wdq, g_Wiuq, g_Ww as float64 arrays) of the CUDA path against the
+    oracle's `ref`, element by element within `bounds` (train_bounds)."""
+    assert abs(loss - ref["loss"]) <= bounds["E_loss"], f"{what}: loss {loss} vs {ref['loss']}"
+    for got, key in zip(grads, ("g_Wdq", "g_Wiuq", "g_Ww")):
+        assert np.isfinite(got).all(), f"{what}: {key} not finite"
+        err = np.abs(got - ref[key])
+        bad = err > bounds["E_" + key]
+        if bad.any():
+            i = np.unravel_index(np.argmax(err - bounds["E_" + key]), err.shape)
+            raise AssertionError(f"{what}: {key}: {int(bad.sum())} of {bad.size} elements outside their bound; "
+                                 f"worst at {i}: got {got[i]!r}, oracle {ref[key][i]!r}, bound {bounds['E_' + key][i]!r}")

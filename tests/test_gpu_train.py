@@ -1,12 +1,17 @@
 """Indexer training step (lsa_indexer_train_step) against the oracle: loss and the gradients of
-W^DQ, W^IUQ, W^w.
+W^DQ, W^IUQ, W^w (hyper.ai summary, "Method": only these three matrices are trained, against frozen
+keys, with binary cross-entropy and then a focal loss).
 
-Tolerances from the arithmetic: the GPU accumulates in fp32 (about 2^-24 relative per term, sums
-of a few thousand terms); with fp32 weights both sides round c and q to fp32 at the same points,
-so gradients agree to a relative L2 error far below 1e-4.  With bf16 weights c and q are rounded to
-bf16, and a value whose exact sum lies near a rounding boundary may land one bf16 step (2^-8
-relative) apart on the two sides; those few flips move the scores and so the gradients, which
-are compared to a relative L2 error of 2e-2 (a wrong term, sign or index gives O(1)).
+Parity rule: element by element.  On exact inputs (tests/parity.py, exact_train_case: every head
+dot product, ReLU gate and logit is exact on both sides) each element of the loss and of the three
+gradients must lie within its own bound (train_bounds): the fp32 error of the loss derivative and
+of every fp32 sum, counted per element from the magnitudes of that element's terms.  Cases: fp32,
+bf16 weights with bf16 keys and with E4M3 keys; binary cross-entropy and the focal loss; ragged
+sequences (an empty one, tails inside a 128-entry tile) and sequences spanning several CTAs.
+
+The same step on seeded Gaussian inputs (where c and q round to bf16 and a value whose exact sum
+lies near a rounding boundary may land one bf16 step apart on the two sides) is also compared as
+a whole: relative L2 error 1e-4 with fp32 weights, 2e-2 with bf16 weights.
 """
 import numpy as np
 import pytest
@@ -14,6 +19,7 @@ import torch
 
 import oracle
 import synth
+from parity import check_train, exact_train_case, train_bounds
 
 pytestmark = pytest.mark.gpu
 
@@ -90,3 +96,16 @@ def test_train_step_rejects_unsupported(m):
     h, W, K, ks, labels, offs, n_h, d_I = fp32_case()
     with pytest.raises(m.LSAError, match="dtypes"):
         run(m, (h.to(torch.bfloat16), [w.to(torch.bfloat16) for w in W], K, ks, labels, offs, n_h, d_I))
+
+
+EXACT_DTYPES = [(torch.float32, torch.float32), (torch.bfloat16, torch.bfloat16), (torch.bfloat16, torch.float8_e4m3fn)]
+
+
+@pytest.mark.parametrize("dt,kdt", EXACT_DTYPES, ids=["f32", "bf16", "bf16-e4m3"])
+@pytest.mark.parametrize("gamma,alpha", [(0.0, -1.0), (2.0, 0.25)], ids=["bce", "focal"])
+@pytest.mark.parametrize("S", [(300, 0, 129, 517), (2500, 1, 3100)], ids=["ragged", "multi-cta"])
+def test_train_step_elementwise(m, dt, kdt, gamma, alpha, S):
+    case = exact_train_case(dt, kdt, S=S)
+    bounds = train_bounds(case, gamma, alpha)
+    loss, gW, ref = run(m, case, gamma, alpha)
+    check_train(loss, gW, ref, bounds, what=f"{dt}/{kdt} gamma={gamma} S={S}")
