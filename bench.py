@@ -41,7 +41,7 @@ def parse_args():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     p.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's batch)")
     p.add_argument("--threshold", type=float, default=0.5)
-    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end measurement (default: --steps)")
     p.add_argument("--cpu-sample", type=int, default=0,
                    help="entries of the oracle's bounded sample (default: sized for a few minutes of CPU work)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -50,6 +50,8 @@ def parse_args():
     p.add_argument("--no-decode-steps", action="store_true", help="skip the per-step decode measurement")
     p.add_argument("--no-golden", action="store_true", help="skip the golden-label measurement")
     p.add_argument("--no-train", action="store_true", help="skip the training-step measurement")
+    p.add_argument("--no-steady", action="store_true", help="skip the steady-state window measurement")
+    p.add_argument("--no-fetch-rates", action="store_true", help="skip the fetch rates of the other workloads")
     p.add_argument("--only", choices=["golden", "train"], default=None,
                    help="run only this self-contained measurement (one GPU) and print its JSON line")
     return p.parse_args()
@@ -450,6 +452,104 @@ def measure_incremental(lsa, path, wl, offs, pool, st, drift=0.1, reps=5):
                     % round(100 * drift)}
 
 
+def fetched_mask(idx, count, offs):
+    """Per-entry fetch decisions [T] (bool, host) from the compacted lists."""
+    idx, count, offs = (np.asarray(x) for x in (idx, count, offs))
+    m = np.zeros(int(offs[-1]), dtype=bool)
+    for b in range(count.size):
+        m[offs[b] + idx[offs[b]:offs[b] + count[b]]] = True
+    return m
+
+
+def rate_summary(wl, count, fetched, planted):
+    """Achieved fetch rates of one workload against its targets (and of its planted entries)."""
+    S = np.asarray(wl.S, dtype=np.float64)
+    per = np.asarray(count, dtype=np.float64) / np.maximum(S, 1)
+    tgt = np.asarray(wl.fetch, dtype=np.float64)
+    out = {"B": wl.B, "target_mean": float((tgt * S).sum() / S.sum()), "achieved": float(per @ S / S.sum())}
+    if wl.B > 1:
+        dev = per - tgt
+        out["per_sequence"] = {"max_abs_dev": float(np.abs(dev).max()), "mean_abs_dev": float(np.abs(dev).mean()),
+                               "corr": float(np.corrcoef(per, tgt)[0, 1]) if np.ptp(tgt) > 0 else None}
+    if planted is not None and planted.any():
+        out["planted_fraction"] = float(planted.mean())
+        out["planted_fetched"] = float(fetched[planted].mean())
+        out["background_fetched"] = float(fetched[~planted].mean())
+    return out
+
+
+def measure_fetch_rates(lsa, device, skip=()):
+    """Whole-path fetch rates (project, score, threshold, OR) of every workload, untimed."""
+    out = {}
+    for name in synth.WORKLOADS:
+        if name in skip:
+            continue
+        wl = synth.workload(name)
+        inp = synth.make_inputs(wl, parts=("proj", "score"))
+        d = lambda t: None if t is None else t.to(device)
+        dt = synth.DTYPES[wl.dtype]
+        q = torch.empty((wl.L, wl.B, wl.n_h, wl.d_I), dtype=dt, device=device)
+        w = torch.empty((wl.L, wl.B, wl.n_h), dtype=torch.float32, device=device)
+        wsp = torch.empty(max(256, lsa.lsa_project_workspace_size(wl.L, wl.B, wl.d, wl.r, wl.n_h, wl.d_I, dt)),
+                          dtype=torch.uint8, device=device)
+        lsa.lsa_project(d(inp.h), d(inp.W_dq), d(inp.W_iuq), d(inp.W_w), q, w, wsp)
+        T = wl.total_S
+        idx = torch.empty(T, dtype=torch.int32, device=device)
+        cnt = torch.empty(wl.B, dtype=torch.int32, device=device)
+        wss = torch.empty(lsa.lsa_score_select_workspace_size(wl.L, wl.B, T), dtype=torch.uint8, device=device)
+        offs = d(inp.seq_offsets)
+        lsa.lsa_memindex_score_select(q, w, d(inp.K), d(inp.k_scale), offs, T, 0.5, idx, cnt, wss)
+        torch.cuda.synchronize(device)
+        lsa.lsa_check_device()
+        c = cnt.cpu().numpy()
+        m = fetched_mask(idx.cpu().numpy(), c, inp.seq_offsets.numpy())
+        out[name] = rate_summary(wl, c, m, inp.planted.any(0).numpy() if wl.planted > 0 else None)
+        del q, w, wsp, idx, cnt, wss, offs, inp
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_steady(lsa, path, wl, tensors, pool, st, steps, warmup, drift=0.1):
+    """The steady-state window: the same window as the headline step, with the previous window's
+    rows resident (its list = this window's with `drift` of each sequence's entries replaced), so
+    the rows come from the incremental fetch; timed with the same stage events."""
+    h, Wdq, Wiuq, Ww, K, ks, offs, qd, wd, sel = tensors
+    T = wl.total_S
+    offs_h = offs.cpu().numpy()
+    p_idx, p_cnt = drifted_lists(path.idx.cpu().numpy(), path.count.cpu().numpy(), offs_h, drift, seed=wl.seed + 29)
+    p_idx, p_cnt = torch.from_numpy(p_idx).to(offs.device), torch.from_numpy(p_cnt).to(offs.device)
+    p_hot = torch.empty_like(path.hot_kv)
+    lsa.lsa_fetch_gather(p_idx, p_cnt, offs, T, pool.tensor, p_hot, stream=st)   # the previous window's rows
+    prev = (p_idx, p_cnt, offs, T, p_hot)
+
+    def window(ev=None):
+        path.run(h, Wdq, Wiuq, Ww, K, ks, offs, pool.tensor, qd, wd, sel_layer=sel, stream=st, events=ev, prev=prev)
+    for _ in range(warmup):
+        window()
+    torch.cuda.synchronize()
+    evs = []
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+        window(ev)
+        evs.append(ev)
+    b.record(st)
+    torch.cuda.synchronize()
+    lsa.lsa_check_device(st)
+    ms = a.elapsed_time(b) / steps
+    spans = {"project": (0, 1), "score_select": (1, 2), "fetch_keys": (2, 3), "lightning_topk": (3, 4),
+             "fetch_rows_incremental (overlapped)": (2, 5), "window": (0, 6)}
+    stages = {k: sum(e[i].elapsed_time(e[j]) for e in evs) / steps for k, (i, j) in spans.items()}
+    host_rows = int(path.host_rows.item())
+    rows = int(path.count.sum().item())
+    del p_hot
+    return {"window_ms": ms, "entries_per_s": wl.L * T / (ms * 1e-3), "drift": drift, "rows": rows,
+            "host_rows": host_rows, "stages_ms": stages, "steps": steps,
+            "note": "project + score/select + [rows: incremental fetch from the previous window's hot buffer, "
+                    "%d %% of each sequence's entries new | keys + Top-k]; same public call as the headline" % round(100 * drift)}
+
+
 def run_lsa(args, rank, world, device):
     import sparse_kv_cache_memoryindexer_b200 as lsa
     torch.cuda.set_device(device)
@@ -465,7 +565,8 @@ def run_lsa(args, rank, world, device):
 
     h, Wdq, Wiuq, Ww = d(inp.h), d(inp.W_dq), d(inp.W_iuq), d(inp.W_w)
     K, ks, offs, qd, wd = d(inp.K), d(inp.k_scale), d(inp.seq_offsets), d(inp.q_dec), d(inp.w_dec)
-    path = lsa.IndexerPath(wl.L, wl.B, wl.d, wl.r, wl.n_h, wl.d_I, wl.tau, wl.k, T, wl.row_bytes, dt, kdt, device=device)
+    path = lsa.IndexerPath(wl.L, wl.B, wl.d, wl.r, wl.n_h, wl.d_I, wl.tau, wl.k, T, wl.row_bytes, dt, kdt, device=device,
+                           incremental=True)
     sel = wl.sel_layer
 
     def stages():
@@ -480,6 +581,9 @@ def run_lsa(args, rank, world, device):
     torch.cuda.synchronize(device)
     lsa.lsa_check_device(st)
     fetched = int(path.count.sum().item())
+    head_rates = rate_summary(wl, path.count.cpu().numpy(),
+                              fetched_mask(path.idx.cpu().numpy(), path.count.cpu().numpy(), inp.seq_offsets.numpy()),
+                              inp.planted.any(0).numpy() if wl.planted > 0 else None)
     h2d = h2d_bandwidth(device)
 
     clocks = ClockSampler(device)
@@ -532,23 +636,28 @@ def run_lsa(args, rank, world, device):
             out_i.copy_(path.topk_idx, non_blocking=True)
             out_c.copy_(path.count, non_blocking=True)
 
+        e2e_steps = args.e2e_steps or args.steps
         e2e_step()
         torch.cuda.synchronize(device)
         if world > 1:
             torch.distributed.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(st)
-        for _ in range(args.e2e_steps):
+        for _ in range(e2e_steps):
             e2e_step()
         b.record(st)
         torch.cuda.synchronize(device)
         e_ms = a.elapsed_time(b)
         e_ms = max_over_ranks(e_ms, world, device)
-        e2e = {"value": job_throughput(world, wl.L * T, args.e2e_steps, e_ms), "unit": UNIT,
+        e2e = {"value": job_throughput(world, wl.L * T, e2e_steps, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
-               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
+               "ms_per_step": e_ms / e2e_steps, "steps": e2e_steps}
         del host
 
+    steady = None
+    if not args.no_steady and world == 1:
+        steady = measure_steady(lsa, path, wl, (h, Wdq, Wiuq, Ww, K, ks, offs, qd, wd, sel), pool, st,
+                                args.steps, args.warmup)
     incr = None
     if not args.no_incremental and world == 1:
         incr = measure_incremental(lsa, path, wl, offs, pool, st)
@@ -561,6 +670,12 @@ def run_lsa(args, rank, world, device):
     trn = None
     if not args.no_train and world == 1:
         trn = measure_train(lsa, device)
+    rates = None
+    if not args.no_fetch_rates and world == 1:
+        del path
+        torch.cuda.empty_cache()
+        rates = measure_fetch_rates(lsa, device, skip=(wl.name,))
+        rates[wl.name] = head_rates
 
     result = None
     if rank == 0:
@@ -591,11 +706,13 @@ def run_lsa(args, rank, world, device):
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if wl.kdtype != "f32" else "f32",
+            "vs_baseline": None,
+            "dtype": {"fp8": "fp8_e4m3 keys / bf16 queries", "bf16": "bf16", "f32": "f32"}[wl.kdtype],
             "dtype_detail": f"keys {wl.kdtype}, queries/weights {wl.dtype}, fp32 accumulation",
             "data": "synthetic (seeded; shapes of a 1M-token context, 4:1 compression)",
             "config": workload_config(wl, args.threshold, world),
             "fetch_rate": fetched / T,
+            "fetch_rates": rates if rates is not None else {wl.name: head_rates},
             "tau_window_ms": ms,
             "stages_ms": {"project": stage_ms[0], "score_select": stage_ms[1], "fetch_keys": stage_ms[2],
                           "lightning_topk": stage_ms[3], "fetch_rows (overlapped)": stage_ms[4],
@@ -612,6 +729,7 @@ def run_lsa(args, rank, world, device):
             "gpu_launches": launches,
             "clocks": clk,
             "e2e": e2e,
+            "steady_window": steady,
             "incremental_fetch": None if incr is None else dict(incr, full_fetch_ms=stage_ms[4]),
             "decode_steps": steps,
             "golden_labels": gold,

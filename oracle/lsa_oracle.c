@@ -26,7 +26,7 @@
  *         token if at least theta = 3 layers keep it; the window's label set is the union of
  *         its tokens' golden sets.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *   - the threshold is inclusive, decided on the logit: I >= thr  <=>  x >= log(thr/(1-thr))
  *     (x >= 0 at thr = 0.5, so an exact-zero logit is fetched);
  *   - no softmax scale, norm or rotary embedding appears in the formulas, so none is applied;

@@ -545,10 +545,10 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     }
     int kpow2 = 1;
     while (kpow2 < k) kpow2 <<= 1;
-    const size_t smem = sizeof(unsigned long long) * (size_t)kpow2;
-    LSA_TRY(set_smem(k_topk_select<false>, smem));
-    k_topk_select<false><<<(unsigned)((int64_t)B * tau), SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, tau, k, kpow2,
-                                                                         topk_idx, topk_score);
+    const size_t smem = sizeof(unsigned long long) * ((size_t)kpow2 + SEL_CAP);
+    LSA_TRY(set_smem(k_topk_select, smem));
+    k_topk_select<<<(unsigned)((int64_t)B * tau), SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, tau, k, kpow2,
+                                                                  topk_idx, topk_score);
     LSA_TRY(launched("top-k select"));
     return ok();
 }

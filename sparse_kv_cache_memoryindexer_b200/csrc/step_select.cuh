@@ -300,13 +300,13 @@ __global__ void __launch_bounds__(TH) k_ss_write(const float *__restrict__ Y, in
             const int inc = warp_incl_scan(v);
             if (lane == 31) warp_tot[warp] = inc;
             __syncthreads();
-            int before = 0, all = 0;
+            int before = 0, total = 0;
             for (int w = 0; w < TH / 32; w++) {
                 before += w < warp ? warp_tot[w] : 0;
-                all += warp_tot[w];
+                total += warp_tot[w];
             }
             pos[k2] = before + inc - v;
-            tot[k2] = all;
+            tot[k2] = total;
             __syncthreads();
         }
         const unsigned long long key64 = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);

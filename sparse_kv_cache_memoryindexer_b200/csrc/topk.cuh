@@ -2,10 +2,10 @@
 // (blog review "FlashMemory-DeepSeek-V4", sections 2.2 and 3.2).
 //
 // Scores of sequence b, query i, fetched slot j live at Y[tau*off_b + i*S_b + j] (fp32).
-// Selection: per query, a radix select on order-preserving 32-bit keys (4 passes of 8 bits)
-// finds the k-th largest score; the survivors (all larger keys, plus the first equal keys in
-// slot order, i.e. smallest entry index) are sorted by (score desc, entry asc) with a bitonic
-// sort in shared memory.
+// Selection: per query, a radix select on order-preserving 32-bit keys finds the k-th largest
+// score (12 + 10 + 10 bits, two reads of the scores); the survivors (all larger keys, plus the
+// first equal keys in slot order, i.e. smallest entry index) are sorted by (score desc, entry asc)
+// with a bitonic sort in shared memory.
 #pragma once
 #include "common.cuh"
 
@@ -81,97 +81,191 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total)
     return r;
 }
 
-// One block per (sequence, query).  kpow2 = next power of two >= k (shared: kpow2 x 8 bytes).
-// TAIL: after the F fetched slots of sequence b come tail_count[b] (at most W) more candidates,
-// the entries compressed during the window (scores tail[b*W + j], entry numbers S_b + j); the Y rows
-// then have tau_y queries per sequence of which block (b, i) reads query i.
-template <bool TAIL>
+// Order-preserving keys of a query's candidates are split as 12 + 10 + 10 bits.  SEL_CAP keys of the
+// k-th key's 12-bit bucket are staged in shared memory, so that the two finer passes read shared
+// memory instead of the scores again.
+constexpr int SEL_BINS = 4096;
+constexpr int SEL_CAP = 4096;
+
+// The bin holding the `want`-th largest key of a histogram of NB bins (thread t owns NB / SEL_THREADS
+// consecutive bins, highest first): *bin_out, and *above_out = keys in higher bins.  want >= 1 and
+// at most the histogram's total.  Ends with a barrier.
+template <int NB>
+__device__ __forceinline__ void sel_find_bin(const unsigned int *hist, int want, int *warp_tot, int *tot, int *bin_out,
+                                             int *above_out)
+{
+    constexpr int PER = NB / SEL_THREADS;
+    const int hi = NB - PER * (int)threadIdx.x;  // bins [hi - PER, hi)
+    int cnt = 0;
+#pragma unroll
+    for (int q = 1; q <= PER; q++) cnt += (int)hist[hi - q];
+    int above = block_excl_scan(cnt, warp_tot, tot);
+    if (above < want && above + cnt >= want) {
+#pragma unroll
+        for (int q = 1; q <= PER; q++) {
+            const int c = (int)hist[hi - q];
+            if (above + c >= want) {
+                *bin_out = hi - q;
+                *above_out = above;
+                break;
+            }
+            above += c;
+        }
+    }
+    __syncthreads();
+}
+
+// One block per (sequence, query).  kpow2 = next power of two >= k; dynamic shared memory:
+// kpow2 + SEL_CAP 8-byte keys.  When the candidates exceed k: a 12-bit histogram of the keys
+// (one read of the scores) gives the bucket of the k-th largest key; a second read writes every key
+// of a higher bucket to the selection in slot order and stages the bucket's own keys (slot order)
+// in shared memory; two 10-bit passes over those find the k-th key K, and the staged keys above K,
+// then the first keys equal to K in slot order (smallest entry index), complete the selection.  A
+// bucket of more than SEL_CAP keys takes three 8-bit passes over the scores instead.  The k keys
+// are sorted by (score desc, slot asc) with a bitonic sort in shared memory.
 __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__restrict__ Y,
                                                              const int32_t *__restrict__ idx,
                                                              const int32_t *__restrict__ count,
                                                              const int64_t *__restrict__ offs, int tau, int k,
                                                              int kpow2, int32_t *__restrict__ topk_idx,
-                                                             float *__restrict__ topk_score,
-                                                             const float *__restrict__ tail = nullptr,
-                                                             const int32_t *__restrict__ tail_count = nullptr,
-                                                             int W = 0, int tau_y = 0)
+                                                             float *__restrict__ topk_score)
 {
-    extern __shared__ unsigned long long sel[];  // (key << 32) | ~slot
-    __shared__ unsigned int hist[256];
+    extern __shared__ unsigned long long sel[];  // [kpow2] (key << 32) | ~slot, then [SEL_CAP] staged keys
+    unsigned long long *stage = sel + kpow2;
+    __shared__ unsigned int hist[SEL_BINS];
     __shared__ int warp_tot[32];
-    __shared__ int tot_a, tot_b;
-    __shared__ unsigned int s_prefix, s_remaining;
+    __shared__ int tot_a, tot_b, s_bin, s_above;
 
     const int b = blockIdx.x / tau, i = blockIdx.x % tau;
     const int64_t off = offs[b], S = offs[b + 1] - offs[b];
-    int F0 = count[b];
-    F0 = F0 < 0 ? 0 : (F0 > S ? (int)S : F0);
-    const float *row = Y + (int64_t)(TAIL ? tau_y : tau) * off + (int64_t)i * S;
-    int nt = 0;
-    if (TAIL && tail_count) {
-        nt = tail_count[b];
-        nt = nt < 0 ? 0 : (nt > W ? W : nt);
-    }
-    const float *trow = TAIL ? tail + (int64_t)b * W : nullptr;
-    const int F = F0 + nt;  // candidates
-    auto cand = [&](int j) { return (!TAIL || j < F0) ? row[j] : trow[j - F0]; };
+    int F = count[b];
+    F = F < 0 ? 0 : (F > S ? (int)S : F);
+    const float *row = Y + (int64_t)tau * off + (int64_t)i * S;
+    const int lane = threadIdx.x & 31;
+    auto key64 = [](uint32_t u, int j) { return ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j); };
 
     for (int t = threadIdx.x; t < kpow2; t += SEL_THREADS) sel[t] = 0ull;
     __syncthreads();
 
     if (F <= k) {
-        for (int j = threadIdx.x; j < F; j += SEL_THREADS)
-            sel[j] = ((unsigned long long)float_to_ordered(cand(j)) << 32) | (uint32_t)(~(uint32_t)j);
+        for (int j = threadIdx.x; j < F; j += SEL_THREADS) sel[j] = key64(float_to_ordered(__ldg(row + j)), j);
     } else {
-        uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
-        for (int pass = 0; pass < 4; pass++) {
-            const int shift = 24 - 8 * pass;
-            for (int t = threadIdx.x; t < 256; t += SEL_THREADS) hist[t] = 0;
-            __syncthreads();
-            for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
-                const uint32_t u = float_to_ordered(cand(j));
-                if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                uint32_t cum = 0, chosen = 0;
-                for (int d = 255; d >= 0; d--) {
-                    if (cum + hist[d] >= remaining) {
-                        chosen = (uint32_t)d;
-                        break;
-                    }
-                    cum += hist[d];
-                }
-                s_remaining = remaining - cum;
-                s_prefix = prefix | (chosen << shift);
-            }
-            __syncthreads();
-            prefix = s_prefix;
-            remaining = s_remaining;
-            pmask |= 255u << shift;
-            __syncthreads();
+        // read 1: 12-bit histogram (lanes with the same bucket add once)
+        for (int t = threadIdx.x; t < SEL_BINS; t += SEL_THREADS) hist[t] = 0;
+        __syncthreads();
+        for (int base = 0; base < F; base += SEL_THREADS) {
+            const int j = base + threadIdx.x;
+            const uint32_t bk = j < F ? float_to_ordered(__ldg(row + j)) >> 20 : 0xFFFFFFFFu;
+            const unsigned peers = __match_any_sync(0xffffffffu, bk);
+            if (bk != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bk], (unsigned)__popc(peers));
         }
-        // prefix is now the k-th largest key; take every larger key and the first `remaining`
-        // equal keys in slot order.
+        __syncthreads();
+        sel_find_bin<SEL_BINS>(hist, k, warp_tot, &tot_a, &s_bin, &s_above);
+        const uint32_t beta = (uint32_t)s_bin;
+        const int above = s_above;              // keys of higher buckets: all selected
+        const int nbeta = (int)hist[beta];
+        const bool staged = nbeta <= SEL_CAP;
+        __syncthreads();
+        // read 2: higher buckets to the selection, the k-th key's bucket to the stage (slot order)
         int carry_gt = 0, carry_eq = 0;
-        const int n_gt_total = k - (int)remaining;
         for (int base = 0; base < F; base += SEL_THREADS) {
             const int j = base + threadIdx.x;
             uint32_t u = 0;
             int gt = 0, eq = 0;
             if (j < F) {
-                u = float_to_ordered(cand(j));
-                gt = u > prefix;
-                eq = u == prefix;
+                u = float_to_ordered(__ldg(row + j));
+                gt = (u >> 20) > beta;
+                eq = (u >> 20) == beta;
             }
             const int pg = block_excl_scan(gt, warp_tot, &tot_a) + carry_gt;
             const int pe = block_excl_scan(eq, warp_tot, &tot_b) + carry_eq;
-            if (gt) sel[pg] = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);
-            if (eq && pe < (int)remaining)
-                sel[n_gt_total + pe] = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);
+            if (gt) sel[pg] = key64(u, j);
+            if (eq && staged) stage[pe] = key64(u, j);
             carry_gt += tot_a;
             carry_eq += tot_b;
             __syncthreads();
+        }
+        const int want = k - above;             // keys still to take from bucket beta (>= 1)
+        if (staged) {
+            // two 10-bit passes over the staged keys
+            uint32_t prefix = beta << 20, pmask = 0xFFF00000u;
+            int remaining = want;
+#pragma unroll 1
+            for (int pass = 0; pass < 2; pass++) {
+                const int shift = 10 - 10 * pass;
+                for (int t = threadIdx.x; t < 1024; t += SEL_THREADS) hist[t] = 0;
+                __syncthreads();
+                for (int q = threadIdx.x; q < nbeta; q += SEL_THREADS) {
+                    const uint32_t u = (uint32_t)(stage[q] >> 32);
+                    if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 1023u], 1u);
+                }
+                __syncthreads();
+                sel_find_bin<1024>(hist, remaining, warp_tot, &tot_a, &s_bin, &s_above);
+                prefix |= (uint32_t)s_bin << shift;
+                remaining -= s_above;
+                pmask |= 1023u << shift;
+                __syncthreads();
+            }
+            // prefix is the k-th largest key; take the staged keys above it, then the first
+            // `remaining` equal to it in slot order
+            int cg = 0, ce = 0;
+            for (int base = 0; base < nbeta; base += SEL_THREADS) {
+                const int q = base + threadIdx.x;
+                unsigned long long v = 0ull;
+                int gt = 0, eq = 0;
+                if (q < nbeta) {
+                    v = stage[q];
+                    const uint32_t u = (uint32_t)(v >> 32);
+                    gt = u > prefix;
+                    eq = u == prefix;
+                }
+                const int pg = block_excl_scan(gt, warp_tot, &tot_a) + cg;
+                const int pe = block_excl_scan(eq, warp_tot, &tot_b) + ce;
+                if (gt) sel[above + pg] = v;
+                if (eq && pe < remaining) sel[k - remaining + pe] = v;
+                cg += tot_a;
+                ce += tot_b;
+                __syncthreads();
+            }
+        } else {
+            // a crowded bucket: three 8-bit passes over the scores for the low 20 bits
+            uint32_t prefix = beta << 20, pmask = 0xFFF00000u;
+            int remaining = want;
+#pragma unroll 1
+            for (int pass = 0; pass < 3; pass++) {
+                const int shift = pass < 2 ? 12 - 8 * pass : 0;
+                const uint32_t bins = pass < 2 ? 255u : 15u;
+                for (int t = threadIdx.x; t < 1024; t += SEL_THREADS) hist[t] = 0;
+                __syncthreads();
+                for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
+                    const uint32_t u = float_to_ordered(__ldg(row + j));
+                    if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & bins], 1u);
+                }
+                __syncthreads();
+                sel_find_bin<1024>(hist, remaining, warp_tot, &tot_a, &s_bin, &s_above);
+                prefix |= (uint32_t)s_bin << shift;
+                remaining -= s_above;
+                pmask |= bins << shift;
+                __syncthreads();
+            }
+            int cg = 0, ce = 0;
+            for (int base = 0; base < F; base += SEL_THREADS) {
+                const int j = base + threadIdx.x;
+                uint32_t u = 0;
+                int gt = 0, eq = 0;
+                if (j < F) {
+                    u = float_to_ordered(__ldg(row + j));
+                    gt = (u >> 20) == beta && u > prefix;
+                    eq = u == prefix;
+                }
+                const int pg = block_excl_scan(gt, warp_tot, &tot_a) + cg;
+                const int pe = block_excl_scan(eq, warp_tot, &tot_b) + ce;
+                if (gt) sel[above + pg] = key64(u, j);
+                if (eq && pe < remaining) sel[k - remaining + pe] = key64(u, j);
+                cg += tot_a;
+                ce += tot_b;
+                __syncthreads();
+            }
         }
     }
     __syncthreads();
@@ -197,8 +291,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
         if (r < nsel) {
             const unsigned long long v = sel[r];
             const int j = (int)~(uint32_t)(v & 0xffffffffull);  // candidate slot (always below F)
-            topk_idx[o0 + r] = (j >= 0 && j < F0) ? __ldg(idx + off + j)
-                                                  : ((j >= F0 && j < F) ? (int32_t)(S + (j - F0)) : -1);
+            topk_idx[o0 + r] = (j >= 0 && j < F) ? __ldg(idx + off + j) : -1;
             if (topk_score) topk_score[o0 + r] = ordered_to_float((uint32_t)(v >> 32));
         } else {
             topk_idx[o0 + r] = -1;

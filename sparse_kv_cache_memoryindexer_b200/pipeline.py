@@ -27,7 +27,7 @@ class IndexerPath:
     """Device buffers for one window of B sequences (ragged, total_S entries per layer)."""
 
     def __init__(self, L, B, d, r, n_h, d_I, tau, k, total_S, row_bytes, dtype, kdtype,
-                 device="cuda", with_scores=False, with_mask=False):
+                 device="cuda", with_scores=False, with_mask=False, incremental=False):
         self.L, self.B, self.d, self.r, self.n_h, self.d_I = L, B, d, r, n_h, d_I
         self.tau, self.k, self.total_S, self.row_bytes = tau, k, int(total_S), row_bytes
         self.dtype, self.kdtype = dtype, kdtype
@@ -54,6 +54,9 @@ class IndexerPath:
         self.topk_idx = torch.empty((B, tau, k), dtype=torch.int32, device=dev)
         self.topk_score = torch.empty((B, tau, k), dtype=torch.float32, device=dev)
         self.ws_topk = ws(lsa.lsa_lightning_topk_workspace_size(B, tau, T, k))
+        # the incremental row fetch of run(prev=...): workspace and the count of rows that crossed the link
+        self.ws_incr = ws(lsa.lsa_fetch_incremental_workspace_size(B, T)) if incremental else None
+        self.host_rows = torch.zeros(1, dtype=torch.int32, device=dev) if incremental else None
         self._link = torch.cuda.Stream(device=dev)  # the host-link row gather of run()
 
     def project(self, h, W_dq, W_iuq, W_w, stream=None):
@@ -78,13 +81,22 @@ class IndexerPath:
         """The KV rows of the fetched entries only, over the host link."""
         lsa.lsa_fetch_gather(self.idx, self.count, seq_offsets, self.total_S, pool, self.hot_kv, stream=stream)
 
+    def fetch_rows_incremental(self, seq_offsets, pool, prev, stream=None):
+        """The KV rows of the fetched entries with the previous window's rows resident: rows that
+        both windows fetched are copied on the device, only the others cross the host link.
+        prev = (idx, count, seq_offsets, total_S, hot_kv) of the previous window."""
+        p_idx, p_count, p_offs, p_T, p_hot = prev
+        lsa.lsa_fetch_gather_incremental(self.idx, self.count, seq_offsets, self.total_S, p_idx, p_count, p_offs, p_T,
+                                         p_hot, pool, self.hot_kv, self.ws_incr, host_rows_out=self.host_rows,
+                                         stream=stream)
+
     def topk(self, q_dec, w_dec, seq_offsets, stream=None):
         lsa.lsa_lightning_topk(q_dec, w_dec, self.hot_K, self.hot_scale, self.idx, self.count, seq_offsets,
                                self.total_S, self.k, self.topk_idx, self.ws_topk, topk_score=self.topk_score,
                                stream=stream)
 
     def run(self, h, W_dq, W_iuq, W_w, K, k_scale, seq_offsets, pool, q_dec, w_dec, sel_layer=0,
-            threshold=0.5, stream=None, events=None):
+            threshold=0.5, stream=None, events=None, prev=None):
         """The whole hot path for one trigger window.
 
         The KV rows cross the host link on a second stream while the keys are gathered and the
@@ -92,6 +104,9 @@ class IndexerPath:
         it returns, so work queued on it afterwards sees the whole window.  events: optional
         list of 7 timing events, recorded at the stage boundaries (start, after project, after
         select, after the keys, after the Top-k, after the rows (second stream), end).
+        prev: the previous window's (idx, count, seq_offsets, total_S, hot_kv); the rows then come
+        from the incremental fetch (the path must be built with incremental=True), and the
+        previous hot buffer must stay untouched until `stream` has passed this window.
         """
         st = torch.cuda.current_stream() if stream is None else stream
         ev = events if events is not None else [None] * 7
@@ -107,7 +122,10 @@ class IndexerPath:
         selected.record(st)
         self._link.wait_event(selected)
         with _stage("lsa.fetch_rows"):
-            self.fetch_rows(seq_offsets, pool, self._link)
+            if prev is None:
+                self.fetch_rows(seq_offsets, pool, self._link)
+            else:
+                self.fetch_rows_incremental(seq_offsets, pool, prev, self._link)
         rec(ev[5], self._link)
         rows_done = torch.cuda.Event()
         rows_done.record(self._link)

@@ -13,13 +13,32 @@ low-rank query projection) and the hyper.ai summary's dataset paragraph (context
 16K-512K tokens).  Fetch rates are steered toward the 13.5 % average footprint of that
 review's section 5 table, or a per-sequence rate from 1 % to 40 % for the ragged mix.
 
+Planted entries (workloads with ``planted > 0``): each layer has one unit direction u_h per
+head, drawn by the generator.  The projection weights carry it: column 0 of W^IUQ holds
+(sqrt(d_I) / PLANT_ALPHA) u_h in head h's rows, and every hidden state is built so that
+c^Q[0] = h W^DQ[0] equals PLANT_ALPHA (the same linear construction that pins h W^w to the drawn
+head weights), so the queries that stage 1 produces contain sqrt(d_I) u_h; the stage-level query
+draws contain the same component.  A planted key of sequence b is cos * v + sqrt(1 - cos^2) * n,
+v = normalise(sum_h w_h u_h) with the sequence's own head weights w and n a unit vector
+orthogonal to v: it lifts the heads of positive weight and sinks those of negative weight.
+None of this evaluates a projection or a score.
+
+Fetch-rate calibration: the head-weight shift comes from a normal model of the score of random
+keys; the fetch rate it gives through the whole path (stage 1 included) differs from the target
+by a few percent of the entries.  ``fetch_calibration.json`` holds, per workload, seed and
+sequence, the model target that gives the wanted rate through the whole path on that
+sequence's own inputs (written by ``tests/calibrate_fetch.py`` with the CPU oracle); it is used
+when the workload's name, seed and target match, and the target is used as is otherwise.
+
 Determinism: every tensor slice is drawn from its own ``numpy.random.default_rng`` stream
 keyed by (seed, part, layer, sequence), so a subset of sequences can be regenerated alone
 and is bit-identical to the same sequences of the full batch.
 """
 from __future__ import annotations
 
+import json
 import math
+import os
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 
@@ -34,7 +53,12 @@ DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3
 DTYPE_CODE = {"f32": 0, "bf16": 1, "fp8": 2}
 
 _PART = {"h": 1, "wdq": 2, "wiuq": 3, "ww": 4, "key": 5, "plant": 6, "pool": 7,
-         "q": 8, "w": 9, "qdec": 10, "wdec": 11, "lens": 12, "rate": 13}
+         "q": 8, "w": 9, "qdec": 10, "wdec": 11, "lens": 12, "rate": 13, "pdir": 14}
+
+# Planted direction in the queries: c^Q[0] = PLANT_ALPHA and W^IUQ[:, 0] = (sqrt(d_I) / PLANT_ALPHA) u_h,
+# so the planted component of every head's query is sqrt(d_I) u_h, as long as the random part of a
+# query with unit-variance elements.
+PLANT_ALPHA = 4.0
 
 _THREADS = 8
 
@@ -56,7 +80,7 @@ class Workload:
     dtype: str                  # h, weights and queries: "f32" or "bf16"
     kdtype: str                 # K^IComp: "f32", "bf16" or "fp8"
     fetch: tuple                # per-sequence target fetch fraction (after the OR)
-    planted: float = 0.0        # fraction of entries planted near the trigger query
+    planted: float = 0.0        # fraction of entries planted along the queries' planted directions
     planted_run: tuple = (1, 1) # planted entries come in runs of this length range
     planted_cos: float = 0.6
     seed: int = 1000
@@ -197,6 +221,31 @@ def _per_layer_rate(p_or: float, L: int) -> float:
     return 1.0 - (1.0 - p_or) ** (1.0 / L)
 
 
+CALIBRATION_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "fetch_calibration.json")
+
+
+def _load_calibration():
+    try:
+        with open(CALIBRATION_FILE) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
+
+
+_CALIBRATION = _load_calibration()
+
+
+def model_target(wl: "Workload", b: int) -> float:
+    """The target handed to the normal model for sequence b of wl: the calibrated value when the
+    workload's name, seed, sequence id and wanted rate match an entry of the calibration file,
+    the wanted rate itself otherwise."""
+    cal = _CALIBRATION.get(wl.name)
+    bid = wl._ids()[b]
+    if cal and cal.get("seed") == wl.seed and bid < len(cal["target"]) and cal["target"][bid] == wl.fetch[b]:
+        return float(cal["model_target"][bid])
+    return float(wl.fetch[b])
+
+
 @dataclass
 class Inputs:
     """All inputs of one workload as CPU torch tensors in their storage dtypes."""
@@ -223,19 +272,30 @@ def _draw_head_weights(wl: Workload, l: int, bid: int, p_or: float) -> np.ndarra
     return (g + delta).astype(np.float32)
 
 
+def plant_directions(wl: Workload, l: int) -> np.ndarray:
+    """Unit planted direction of every head of layer l, [n_h][d_I] float64."""
+    U = _rng(wl, "pdir", l).standard_normal((wl.n_h, wl.d_I))
+    return U / np.linalg.norm(U, axis=1, keepdims=True)
+
+
 def _draw_queries(wl: Workload, l: int, bid: int) -> np.ndarray:
-    return _rng(wl, "q", l, bid).standard_normal((wl.n_h, wl.d_I), dtype=np.float32)
+    q = _rng(wl, "q", l, bid).standard_normal((wl.n_h, wl.d_I), dtype=np.float32)
+    if wl.planted > 0:
+        q += (math.sqrt(wl.d_I) * plant_directions(wl, l)).astype(np.float32)
+    return q
 
 
-def _keys_for(wl: Workload, l: int, b: int, bid: int, q_b: np.ndarray, w_b: np.ndarray):
-    """Keys of one (layer, sequence): Gaussian N(0, 1/d_I) rows plus planted entries."""
+def _keys_for(wl: Workload, l: int, b: int, bid: int, U: np.ndarray, w_b: np.ndarray):
+    """Keys of one (layer, sequence): Gaussian N(0, 1/d_I) rows plus planted entries along
+    v = normalise(sum_h w_h u_h) (U: the layer's planted directions, w_b the head weights)."""
     S = wl.S[b]
     K = _normal_rows(wl, "key", (l, bid), S, wl.d_I, 1.0 / math.sqrt(wl.d_I))
     planted = np.zeros(S, dtype=bool)
     if wl.planted > 0:
-        prng = _rng(wl, "plant", l, bid)
-        # direction of the trigger query: sum over heads of w_h q_h (generator's own draws)
-        u = (w_b.astype(np.float64)[:, None] * q_b.astype(np.float64)).sum(0)
+        # the planted positions are the sequence's (the same entries in every layer: an entry is
+        # one compressed position of the context); the directions are the layer's
+        prng = _rng(wl, "plant", bid)
+        u = (w_b.astype(np.float64)[:, None] * U).sum(0)
         u /= np.linalg.norm(u) + 1e-300
         target = int(round(wl.planted * S))
         lo, hi = wl.planted_run
@@ -244,7 +304,7 @@ def _keys_for(wl: Workload, l: int, b: int, bid: int, q_b: np.ndarray, w_b: np.n
             start = int(prng.integers(0, max(1, S - run + 1)))
             planted[start:start + run] = True
         idx = np.nonzero(planted)[0]
-        n = prng.standard_normal((idx.size, wl.d_I))
+        n = _rng(wl, "plant", l, bid).standard_normal((idx.size, wl.d_I))
         n -= (n @ u)[:, None] * u[None, :]
         n /= np.linalg.norm(n, axis=1, keepdims=True) + 1e-300
         c = wl.planted_cos
@@ -264,15 +324,17 @@ def _encode_keys(K: np.ndarray, kdt: str):
     return codes, scale
 
 
-def _hidden_for(wl: Workload, l: int, bid: int, W_w64: np.ndarray, QR, w_t: np.ndarray):
-    """Hidden state whose head weights h W^w equal w_t (exactly, before rounding h).
+def _hidden_for(wl: Workload, l: int, bid: int, QR, t: np.ndarray):
+    """Hidden state h with h M = t exactly (before rounding h), for the constraint matrix M whose
+    columns are W^w's (h W^w = the drawn head weights) and, with planted entries, W^DQ's row 0
+    (c^Q[0] = PLANT_ALPHA).
 
-    Construction from W^w alone: with W^w's column space spanned by an orthonormal Q
-    (W^w = Q R), h = h0 - Q Q^T h0 + Q R^{-T} w_t, where h0 ~ N(0, I).
+    Construction from the weights alone: with M = Q R (Q orthonormal), h = h0 - Q Q^T h0 +
+    Q R^{-T} t, where h0 ~ N(0, I).
     """
     Q, R = QR
     h0 = _rng(wl, "h", l, bid).standard_normal(wl.d)
-    h = h0 - Q @ (Q.T @ h0) + Q @ np.linalg.solve(R.T, w_t.astype(np.float64))
+    h = h0 - Q @ (Q.T @ h0) + Q @ np.linalg.solve(R.T, t.astype(np.float64))
     return h
 
 
@@ -297,12 +359,12 @@ def make_inputs(wl: Workload, parts=("proj", "score", "pool", "dec"), threads: i
     for l in range(L):
         for b in range(B):
             qs[l, b] = _draw_queries(wl, l, ids[b])
-            ws[l, b] = _draw_head_weights(wl, l, ids[b], wl.fetch[b])
+            ws[l, b] = _draw_head_weights(wl, l, ids[b], model_target(wl, b))
     q_t = _cast(qs, wl.dtype)
     if "score" in parts or "proj" in parts:
         inp.q = q_t
         inp.w = torch.from_numpy(ws)
-        q_used = q_t.float().numpy()
+        Us = [plant_directions(wl, l) for l in range(L)] if wl.planted > 0 else [None] * L
         T = wl.total_S
         K_all = torch.empty((L, T, wl.d_I), dtype=DTYPES[wl.kdtype])
         sc_all = torch.empty((L, T), dtype=torch.float32) if wl.kdtype == "fp8" else None
@@ -310,7 +372,7 @@ def make_inputs(wl: Workload, parts=("proj", "score", "pool", "dec"), threads: i
 
         def job(lb):
             l, b = lb
-            K, pl = _keys_for(wl, l, b, ids[b], q_used[l, b], ws[l, b])
+            K, pl = _keys_for(wl, l, b, ids[b], Us[l], ws[l, b])
             Kt, sc = _encode_keys(K, wl.kdtype)
             s0, s1 = int(offs[b]), int(offs[b + 1])
             K_all[l, s0:s1] = Kt
@@ -327,18 +389,25 @@ def make_inputs(wl: Workload, parts=("proj", "score", "pool", "dec"), threads: i
         W_dq = np.empty((L, r, d), dtype=np.float32)
         W_iuq = np.empty((L, nq, r), dtype=np.float32)
         W_w = np.empty((L, wl.n_h, d), dtype=np.float32)
+        planted = wl.planted > 0
+        beta = math.sqrt(wl.d_I) / PLANT_ALPHA
         for l in range(L):
             _normal_rows(wl, "wdq", (l,), r, d, 1.0 / math.sqrt(d), out=W_dq[l])
             _normal_rows(wl, "wiuq", (l,), nq, r, 1.0 / math.sqrt(r), out=W_iuq[l])
             _normal_rows(wl, "ww", (l,), wl.n_h, d, 1.0 / math.sqrt(d), out=W_w[l])
+            if planted:
+                W_iuq[l, :, 0] = (beta * plant_directions(wl, l)).reshape(nq)
         inp.W_dq, inp.W_iuq, inp.W_w = _cast(W_dq, wl.dtype), _cast(W_iuq, wl.dtype), _cast(W_w, wl.dtype)
-        # h is built against the *stored* (rounded) W^w so that h W^w lands on the target
+        # h is built against the *stored* (rounded) weights so that h W^w (and c^Q[0]) land on the targets
         hs = np.zeros((L, B, d), dtype=np.float64)
         for l in range(L):
-            Ww64 = inp.W_w[l].double().numpy()          # [n_h][d] = (W^w)^T
-            QR = np.linalg.qr(Ww64.T)                   # columns of W^w: d x n_h
+            M = inp.W_w[l].double().numpy()             # [n_h][d] = (W^w)^T
+            if planted:
+                M = np.concatenate([M, inp.W_dq[l, :1].double().numpy()], axis=0)
+            QR = np.linalg.qr(M.T)                      # d x (n_h [+ 1])
             for b in range(B):
-                hs[l, b] = _hidden_for(wl, l, ids[b], Ww64, QR, ws[l, b])
+                t = np.concatenate([ws[l, b], [PLANT_ALPHA]]) if planted else ws[l, b]
+                hs[l, b] = _hidden_for(wl, l, ids[b], QR, t)
         inp.h = _cast(hs, wl.dtype)
         inp.w_target = torch.from_numpy(ws.copy())
 

@@ -184,3 +184,25 @@ def test_decode_step_equals_batched_column(window, m):
         m.lsa_check_device()
         assert torch.equal(ti, path.topk_idx[:, i]), f"{wl.name} step {i}: indices differ"
         assert torch.equal(ts, path.topk_score[:, i]), f"{wl.name} step {i}: scores differ"
+
+
+def test_fetch_rates_follow_the_workload(window):
+    """The whole path fetches the workload's stated share of the entries: about 13.5 % of each
+    batch (blog review, section 5 table), each ragged sequence near its own target (1-40 %), and
+    the planted entries (relevant to the queries that stage 1 produces) far more often than the rest."""
+    wl, inp, _, path = window
+    offs = inp.seq_offsets.numpy()
+    mask, cnt = gpu_mask(path, wl, offs)
+    S = np.asarray(wl.S, dtype=np.float64)
+    per = cnt / S
+    achieved = float(cnt.sum() / S.sum())
+    tgt = np.asarray(wl.fetch)
+    if np.ptp(tgt) == 0:
+        assert abs(achieved - tgt[0]) <= 0.005, (wl.name, achieved)
+    else:
+        assert np.abs(per - tgt).max() <= 0.02, (wl.name, np.abs(per - tgt).max())
+        assert np.corrcoef(per, tgt)[0, 1] > 0.99
+    if wl.planted > 0:
+        pl = inp.planted.any(0).numpy()
+        got = mask.cpu().numpy().astype(bool)
+        assert got[pl].mean() > 0.95 and got[~pl].mean() < 0.15, (got[pl].mean(), got[~pl].mean())

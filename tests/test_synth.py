@@ -53,3 +53,23 @@ def test_parts_do_not_change_values():
     assert torch.equal(score_only.w, full.w)
     proj_only = synth.make_inputs(wl, parts=("proj",))
     assert torch.equal(proj_only.h, full.h) and torch.equal(proj_only.W_iuq, full.W_iuq)
+
+
+def test_calibrated_fetch_rate_through_the_whole_path():
+    """The calibration of the head-weight model (synth/fetch_calibration.json, written by
+    tests/calibrate_fetch.py) makes the oracle's whole path fetch the wanted share of the 128K
+    workload (13.5 %, blog review section 5 table) and of the tiny one (15 %); the planted entries
+    of the 128K workload are fetched far more often than the others."""
+    import oracle
+    for name, tol in (("ctx128k_bf16", 0.002), ("tiny_fp32", 0.02)):
+        wl = synth.workload(name)
+        assert synth.model_target(wl, 0) != wl.fetch[0], f"{name}: no calibration entry applies"
+        inp = synth.make_inputs(wl, parts=("proj", "score"))
+        q, w = oracle.project(inp.h, inp.W_dq, inp.W_iuq, inp.W_w, wl.n_h, wl.d_I)
+        r = oracle.score(q, w, inp.K, inp.k_scale, inp.seq_offsets.numpy(), want_x=False)
+        rate = r["count"].sum() / wl.total_S
+        assert abs(rate - wl.fetch[0]) <= tol, (name, rate)
+        if wl.planted > 0:
+            m = r["mask"].astype(bool)
+            pl = inp.planted.any(0).numpy()
+            assert m[pl].mean() > 0.95 and m[~pl].mean() < 0.13

@@ -91,3 +91,30 @@ def test_static_rejects_sizes_beyond_the_scratch(m):
     assert st == 5  # LSA_ERR_WORKSPACE
     msg = lib.lsa_last_error().decode()
     assert "static scratch" in msg and str(lsa.STATIC_SCORE_SCRATCH_BYTES) in msg
+
+
+def test_static_calls_allocate_no_device_memory(m):
+    # the first call on a device looks up the scratch address and loads the kernels; after it,
+    # further calls on both key types leave the device's free memory and torch's allocator as
+    # they were (outputs are allocated before the measurement)
+    cases = {k: _case(k) for k in ("bf16", "fp8")}
+    outs = {k: _outputs(c[0]) for k, c in cases.items()}
+
+    def call(k):
+        wl, q, w, K, ks, offs = cases[k]
+        idx, cnt, mask, sc = outs[k]
+        m.lsa_memindex_score_select_static(q, w, K, ks, offs, wl.total_S, 0.5, idx, cnt, scores_out=sc, mask_out=mask)
+
+    for k in cases:
+        call(k)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0, reserved0 = torch.cuda.memory_allocated(), torch.cuda.memory_reserved()
+    for _ in range(3):
+        for k in cases:
+            call(k)
+    torch.cuda.synchronize()
+    m.lsa_check_device()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
+    assert torch.cuda.memory_allocated() == alloc0 and torch.cuda.memory_reserved() == reserved0
