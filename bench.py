@@ -52,7 +52,7 @@ def parse_args():
     p.add_argument("--no-train", action="store_true", help="skip the training-step measurement")
     p.add_argument("--no-steady", action="store_true", help="skip the steady-state window measurement")
     p.add_argument("--no-fetch-rates", action="store_true", help="skip the fetch rates of the other workloads")
-    p.add_argument("--only", choices=["golden", "train"], default=None,
+    p.add_argument("--only", choices=["golden", "train", "decode"], default=None,
                    help="run only this self-contained measurement (one GPU) and print its JSON line")
     return p.parse_args()
 
@@ -283,8 +283,8 @@ def h2d_bandwidth(device, nbytes=1 << 30):
 
 def measure_train(lsa, device, B=8, S=32768, reps=5):
     """One indexer training step (BCE) on 128K-token shapes: 3 layers, B sequences of S entries,
-    d 4096, r 2048, 64 heads x 128, bf16 weights and keys; timed alone.  Roofline: the CUDA-core
-    fp32 rate (148 SMs x 128 FMA lanes x 2 flop x 1965 MHz) for the two per-entry products."""
+    d 4096, r 2048, 64 heads x 128, bf16 weights and keys; timed alone.  Roofline: the two per-entry
+    products (a = K q^T and dq = G^T K, 4 L T n_h d_I flop) against the sustained bf16 tensor rate."""
     wl = synth.workload("ctx128k_bf16", B=B, S=(S,) * B, fetch=(0.135,) * B, name="train_128k")
     inp = synth.make_inputs(wl, parts=("proj", "score"))
     d = lambda t: t.to(device)
@@ -311,12 +311,15 @@ def measure_train(lsa, device, B=8, S=32768, reps=5):
     lsa.lsa_check_device(st)
     ms = a.elapsed_time(b) / reps
     flops = 2.0 * 2.0 * wl.L * wl.total_S * wl.n_h * wl.d_I
-    peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    peak = load_peaks()["bf16_tflops_sustained"]
+    key_bytes = wl.L * wl.total_S * wl.d_I * 2
     out = {"L": wl.L, "B": B, "S": S, "ms": ms, "loss": float(loss.item()),
            "entries_per_s": wl.L * wl.total_S / (ms * 1e-3),
-           "roofline": {"bound": "alu", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
-                        "peak_note": "fp32 CUDA-core FMA rate at 1965 MHz"},
-           "note": "forward + BCE + backward of W^DQ, W^IUQ, W^w; timed alone"}
+           "roofline": {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                        "peak_note": "sustained bf16 GEMM (measured)",
+                        "key_stream_GBps": key_bytes / (ms * 1e-3) / 1e9},
+           "note": "forward + BCE + backward of W^DQ, W^IUQ, W^w (projection, per-entry products on tcgen05, "
+                   "dc and the three outer products); timed alone"}
     out["roofline"]["frac"] = out["roofline"]["achieved"] / peak
     return out
 
@@ -397,6 +400,27 @@ def measure_decode_steps(lsa, path, wl, offs, qd, wd, st, reps=3):
     return {"steps": tau, "window_entries_per_sequence": W, "eager_ms_per_step": eager / tau,
             "graph_ms_per_step": replay / tau, "graph_ms_per_window": replay, "batched_ms_per_window": batched,
             "note": "S5 per decode step over the fetched entries plus one new entry per 4 steps; timed alone"}
+
+
+def measure_decode_only(lsa, device, args):
+    """One window of the workload (to fetch the keys), then the per-step decode measurement alone."""
+    wl = rank_workload(args.workload, 0, args.batch)
+    T = wl.total_S
+    pool = lsa.MappedPool(T, wl.row_bytes)
+    inp = synth.make_inputs(wl, pool_out=pool.tensor)
+    d = lambda t: None if t is None else t.to(device)
+    h, Wdq, Wiuq, Ww, K, ks = d(inp.h), d(inp.W_dq), d(inp.W_iuq), d(inp.W_w), d(inp.K), d(inp.k_scale)
+    offs, qd, wd = d(inp.seq_offsets), d(inp.q_dec), d(inp.w_dec)
+    path = lsa.IndexerPath(wl.L, wl.B, wl.d, wl.r, wl.n_h, wl.d_I, wl.tau, wl.k, T, wl.row_bytes,
+                           synth.DTYPES[wl.dtype], synth.DTYPES[wl.kdtype], device=device)
+    st = torch.cuda.current_stream(device)
+    path.run(h, Wdq, Wiuq, Ww, K, ks, offs, pool.tensor, qd, wd, sel_layer=wl.sel_layer, stream=st)
+    torch.cuda.synchronize(device)
+    lsa.lsa_check_device(st)
+    out = measure_decode_steps(lsa, path, wl, offs, qd, wd, st)
+    out["workload"] = wl.name
+    pool.free()
+    return out
 
 
 def drifted_lists(idx, cnt, offs, drift, seed):
@@ -613,12 +637,26 @@ def run_lsa(args, rank, world, device):
     stage_ms /= args.steps
     elapsed_ms = max_over_ranks(elapsed_ms, world, device)
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers.  Per window the host supplies the trigger
+    # hidden states, the decode queries and weights, and the index keys of the entries compressed
+    # during the window (tau/4 per sequence and layer at 4:1, written into the last tau/4 slots of
+    # each sequence); the index-key cache itself stays on the device like the weights (the method
+    # offloads the compressed KV rows, which the fetch reads from the host pool inside the window).
     e2e = None
     if not args.no_e2e:
-        host = {k: v.pin_memory() for k, v in (("h", inp.h), ("K", inp.K), ("qd", inp.q_dec), ("wd", inp.w_dec))}
+        Wn = max(1, wl.tau // 4)
+        offs_h = inp.seq_offsets.numpy()
+        rows = np.array([l * T + offs_h[b + 1] - Wn + j for l in range(wl.L) for b in range(wl.B)
+                         for j in range(Wn) if offs_h[b + 1] - offs_h[b] >= Wn], dtype=np.int64)
+        rows_d = torch.from_numpy(rows).to(device)
+        kraw = (lambda t: t.view(torch.uint8)) if inp.K.dtype == torch.float8_e4m3fn else (lambda t: t)
+        host = {"h": inp.h.pin_memory(), "qd": inp.q_dec.pin_memory(), "wd": inp.w_dec.pin_memory(),
+                "K_new": kraw(inp.K).reshape(-1, wl.d_I)[torch.from_numpy(rows)].pin_memory()}
+        stage = {"K_new": torch.empty_like(host["K_new"], device=device)}
         if inp.k_scale is not None:
-            host["ks"] = inp.k_scale.pin_memory()
+            host["ks_new"] = inp.k_scale.reshape(-1)[torch.from_numpy(rows)].pin_memory()
+            stage["ks_new"] = torch.empty_like(host["ks_new"], device=device)
+        K_rows = kraw(K).view(-1, wl.d_I)
         out_i = torch.empty(path.topk_idx.shape, dtype=torch.int32).pin_memory()
         out_c = torch.empty(path.count.shape, dtype=torch.int32).pin_memory()
         h2d_b = sum(v.numel() * v.element_size() for v in host.values())
@@ -626,11 +664,13 @@ def run_lsa(args, rank, world, device):
 
         def e2e_step():
             h.copy_(host["h"], non_blocking=True)
-            K.copy_(host["K"], non_blocking=True)
-            if ks is not None:
-                ks.copy_(host["ks"], non_blocking=True)
             qd.copy_(host["qd"], non_blocking=True)
             wd.copy_(host["wd"], non_blocking=True)
+            stage["K_new"].copy_(host["K_new"], non_blocking=True)
+            K_rows.index_copy_(0, rows_d, stage["K_new"])
+            if ks is not None:
+                stage["ks_new"].copy_(host["ks_new"], non_blocking=True)
+                ks.view(-1).index_copy_(0, rows_d, stage["ks_new"])
             path.run(h, Wdq, Wiuq, Ww, K, ks, offs, pool.tensor, qd, wd, sel_layer=sel, threshold=args.threshold,
                      stream=st)
             out_i.copy_(path.topk_idx, non_blocking=True)
@@ -651,7 +691,10 @@ def run_lsa(args, rank, world, device):
         e_ms = max_over_ranks(e_ms, world, device)
         e2e = {"value": job_throughput(world, wl.L * T, e2e_steps, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
-               "ms_per_step": e_ms / e2e_steps, "steps": e2e_steps}
+               "ms_per_step": e_ms / e2e_steps, "steps": e2e_steps,
+               "inputs": "per window: trigger hidden states, decode queries and weights, the index keys (and scales) "
+                         "of the %d entries per sequence and layer compressed during the window; out: Top-k indices "
+                         "and fetched counts" % Wn}
         del host
 
     steady = None
@@ -777,7 +820,12 @@ def main():
     if args.only:
         import sparse_kv_cache_memoryindexer_b200 as lsa
         torch.cuda.set_device(device)
-        res = measure_golden(lsa, device) if args.only == "golden" else measure_train(lsa, device)
+        if args.only == "golden":
+            res = measure_golden(lsa, device)
+        elif args.only == "train":
+            res = measure_train(lsa, device)
+        else:
+            res = measure_decode_only(lsa, device, args)
         print(json.dumps(dict(res, only=args.only)), flush=True)
         return 0
     if world > 1:

@@ -14,10 +14,14 @@ namespace lsa {
 
 constexpr int GATHER_ROWS_PER_WARP = 4;
 constexpr int GATHER_MAX_CHUNKS = 4;  // row_bytes <= 4 * 32 * 16 = 2048 per in-flight row
-#ifndef LSA_GATHER_LINK_CTAS
-#define LSA_GATHER_LINK_CTAS 128
-#endif
-constexpr int GATHER_LINK_CTAS = LSA_GATHER_LINK_CTAS;  // CTAs of the rows-only launch (128 threads each)
+// The launches that read the host pool (k_gather_rows, k_incr_fetch) run beside the Lightning Top-k:
+// a few SMs with many reads in flight each.  A warp keeps GATHER_ROWS_PER_WARP rows in flight, so
+// 16 CTAs of 1024 threads hold 2 MB of 1 KB rows in flight, enough for the host link, on 16 SMs;
+// a CTA-per-SM spread of the same reads slowed the Top-k beside it several times over (the host
+// reads in flight hold every SM's load path).
+constexpr int GATHER_LINK_CTAS = 16;
+template <int CH>
+constexpr int link_threads() { return CH <= 2 ? 1024 : 512; }  // 64 or 128 registers a thread
 constexpr int GATHER_ROWS_MAX_B = 8192; // sequences of the rows-only launch (shared prefix of B + 1 ints)
 
 // 16 E4M3 codes -> 16 bf16 values (exact: every E4M3 value is a bf16 value).
@@ -112,11 +116,13 @@ __global__ void __launch_bounds__(256) k_gather(const int32_t *__restrict__ idx,
 }
 
 // Shared-memory exclusive prefix pre[0..B] of the counts (clamped to [0, S_b], a bad count flagged),
-// built by one CTA of 128 threads; returns the total.  Every thread calls it.
+// built by one CTA of any size up to 1024 threads (warp_sum: 32 ints of shared memory); returns the
+// total.  Every thread calls it.
 __device__ __forceinline__ int block_count_prefix(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
                                                   int B, int *pre, int *warp_sum)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nt = blockDim.x, nw = nt >> 5;
     auto clamped = [&](int b) {
         const int64_t S = offs[b + 1] - offs[b];
         int F = count[b];
@@ -126,7 +132,7 @@ __device__ __forceinline__ int block_count_prefix(const int32_t *__restrict__ co
         }
         return F;
     };
-    const int per = (B + 127) / 128;
+    const int per = (B + nt - 1) / nt;
     const int lo = min(B, (int)threadIdx.x * per), hi = min(B, lo + per);
     int sum = 0;
     for (int b = lo; b < hi; b++) sum += clamped(b);
@@ -134,8 +140,7 @@ __device__ __forceinline__ int block_count_prefix(const int32_t *__restrict__ co
     if (lane == 31) warp_sum[warp] = inc;
     __syncthreads();
     int base = 0, total = 0;
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
+    for (int k = 0; k < nw; k++) {
         base += k < warp ? warp_sum[k] : 0;
         total += warp_sum[k];
     }
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(128) k_gather_keys(const int32_t *__restrict__
                                                      float *__restrict__ hotsc)
 {
     extern __shared__ int pre[];
-    __shared__ int warp_sum[4];
+    __shared__ int warp_sum[32];
     const int total = block_count_prefix(count, offs, B, pre, warp_sum);
     const int64_t kb = (int64_t)krow16 * 16, kbo = kconv ? 2 * kb : kb;
     const int64_t units = (int64_t)total * krow16;
@@ -204,26 +209,26 @@ __global__ void __launch_bounds__(128) k_gather_keys(const int32_t *__restrict__
     }
 }
 
-// Rows only, for a launch that runs beside other kernels: few small CTAs (the host link needs only
-// a few hundred KB of reads in flight), every fetched row of every sequence numbered in one range
-// so that ragged counts cannot leave most warps idle.  Each CTA first builds the exclusive prefix
-// pre[0..B] of the counts in shared memory ((B + 1) ints), then warp w takes rows
-// g = 4 (w + i W) .. + 3 and finds the sequence of g by binary search in pre.
+// Rows only, for a launch that runs beside other kernels: GATHER_LINK_CTAS fat CTAs, every fetched
+// row of every sequence numbered in one range so that ragged counts cannot leave most warps idle.
+// Each CTA first builds the exclusive prefix pre[0..B] of the counts in shared memory ((B + 1)
+// ints), then warp w of the W warps of the launch takes rows g = 4 (w + i W) .. + 3 and finds the
+// sequence of g by binary search in pre.
 template <int CH>  // 16-byte chunks per lane and row (row_bytes <= CH * 512)
-__global__ void __launch_bounds__(128) k_gather_rows(const int32_t *__restrict__ idx,
+__global__ void __launch_bounds__(link_threads<CH>()) k_gather_rows(const int32_t *__restrict__ idx,
                                                      const int32_t *__restrict__ count,
                                                      const int64_t *__restrict__ offs, int B,
                                                      const uint8_t *__restrict__ pool, int row16,
                                                      uint8_t *__restrict__ hot_kv)
 {
     extern __shared__ int pre[];
-    __shared__ int warp_sum[4];
+    __shared__ int warp_sum[32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int total = block_count_prefix(count, offs, B, pre, warp_sum);
 
     const int64_t rb = (int64_t)row16 * 16;
-    const int64_t wstride = (int64_t)gridDim.x * 4;
-    for (int64_t g0 = ((int64_t)blockIdx.x * 4 + warp) * GATHER_ROWS_PER_WARP; g0 < total;
+    const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t g0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + warp) * GATHER_ROWS_PER_WARP; g0 < total;
          g0 += wstride * GATHER_ROWS_PER_WARP) {
         int64_t src[GATHER_ROWS_PER_WARP], dst[GATHER_ROWS_PER_WARP];
 #pragma unroll
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(128) k_incr_map(const int32_t *__restrict__ id
                                                   int32_t *__restrict__ miss, int *__restrict__ nmiss)
 {
     extern __shared__ int pre[];
-    __shared__ int warp_sum[4];
+    __shared__ int warp_sum[32];
     const int total = block_count_prefix(count, offs, B, pre, warp_sum);
     const int lane = threadIdx.x & 31;
     // every thread of a warp runs the same number of iterations (the ballot below needs them all)
@@ -334,7 +339,7 @@ __global__ void __launch_bounds__(128) k_incr_copy(const int32_t *__restrict__ c
                                                    int row16, uint8_t *__restrict__ hot)
 {
     extern __shared__ int pre[];
-    __shared__ int warp_sum[4];
+    __shared__ int warp_sum[32];
     const int total = block_count_prefix(count, offs, B, pre, warp_sum);
     const int64_t rb = (int64_t)row16 * 16;
     const int64_t units = (int64_t)total * row16;
@@ -351,22 +356,22 @@ __global__ void __launch_bounds__(128) k_incr_copy(const int32_t *__restrict__ c
 }
 
 template <int CH>
-__global__ void __launch_bounds__(128) k_incr_fetch(const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+__global__ void __launch_bounds__(link_threads<CH>()) k_incr_fetch(const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
                                                     const int64_t *__restrict__ offs, int B,
                                                     const int32_t *__restrict__ miss, const int *__restrict__ nmiss,
                                                     const uint8_t *__restrict__ pool, int row16, uint8_t *__restrict__ hot,
                                                     int32_t *__restrict__ host_rows)
 {
     extern __shared__ int pre[];
-    __shared__ int warp_sum[4];
+    __shared__ int warp_sum[32];
     const int total = block_count_prefix(count, offs, B, pre, warp_sum);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int n = *nmiss;
     n = n < 0 ? 0 : (n > total ? total : n);
     if (host_rows && blockIdx.x == 0 && threadIdx.x == 0) *host_rows = n;
     const int64_t rb = (int64_t)row16 * 16;
-    const int64_t wstride = (int64_t)gridDim.x * 4;
-    for (int64_t i0 = ((int64_t)blockIdx.x * 4 + warp) * GATHER_ROWS_PER_WARP; i0 < n;
+    const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t i0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + warp) * GATHER_ROWS_PER_WARP; i0 < n;
          i0 += wstride * GATHER_ROWS_PER_WARP) {
         int64_t src[GATHER_ROWS_PER_WARP], dst[GATHER_ROWS_PER_WARP];
 #pragma unroll

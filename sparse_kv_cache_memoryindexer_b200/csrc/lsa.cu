@@ -16,6 +16,7 @@
 #include "proj_tc.cuh"
 #include "golden.cuh"
 #include "train.cuh"
+#include "train_tc.cuh"
 #include "step_select.cuh"
 #include "topk.cuh"
 #include "selftest.cuh"
@@ -123,10 +124,12 @@ ScoreWs score_ws(void *ws, int L, int B, int64_t T)
     return w;
 }
 
+// Dynamic shared memory of a launch: the limit is set explicitly (static plus dynamic above 48 KB
+// needs it even when the dynamic part alone is below 48 KB).
 template <typename K>
 lsa_status set_smem(K kernel, size_t bytes)
 {
-    if (bytes > 48 * 1024) {
+    if (bytes > 0) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
@@ -392,11 +395,11 @@ lsa_status lsa_fetch_gather(const int32_t *idx, const int32_t *count, const int6
     if (pool && !K_sel && B <= GATHER_ROWS_MAX_B) {
         // rows only: a small launch meant to run beside other work (see k_gather_rows)
         const size_t smem = sizeof(int) * (size_t)(B + 1);
-        const dim3 grid(GATHER_LINK_CTAS), block(128);
+        const dim3 grid(GATHER_LINK_CTAS);
         const uint8_t *src = (const uint8_t *)dpool;
-        if (row16 <= 32) k_gather_rows<1><<<grid, block, smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
-        else if (row16 <= 64) k_gather_rows<2><<<grid, block, smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
-        else k_gather_rows<4><<<grid, block, smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
+        if (row16 <= 32) k_gather_rows<1><<<grid, link_threads<1>(), smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
+        else if (row16 <= 64) k_gather_rows<2><<<grid, link_threads<2>(), smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
+        else k_gather_rows<4><<<grid, link_threads<4>(), smem, st>>>(idx, count, seq_offsets, B, src, row16, (uint8_t *)hot_kv);
         LSA_TRY(launched("gather rows"));
         return ok();
     }
@@ -483,13 +486,13 @@ lsa_status lsa_fetch_gather_incremental(const int32_t *idx, const int32_t *count
     LSA_TRY(launched("incremental fetch: device copy"));
     const uint8_t *src = (const uint8_t *)dpool;
     if (row16 <= 32)
-        k_incr_fetch<1><<<GATHER_LINK_CTAS, 128, smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
+        k_incr_fetch<1><<<GATHER_LINK_CTAS, link_threads<1>(), smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
                                                              (uint8_t *)hot_kv, host_rows_out);
     else if (row16 <= 64)
-        k_incr_fetch<2><<<GATHER_LINK_CTAS, 128, smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
+        k_incr_fetch<2><<<GATHER_LINK_CTAS, link_threads<2>(), smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
                                                              (uint8_t *)hot_kv, host_rows_out);
     else
-        k_incr_fetch<4><<<GATHER_LINK_CTAS, 128, smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
+        k_incr_fetch<4><<<GATHER_LINK_CTAS, link_threads<4>(), smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
                                                              (uint8_t *)hot_kv, host_rows_out);
     LSA_TRY(launched("incremental fetch: host rows"));
     return ok();
@@ -795,9 +798,23 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
     LSA_TRY(lsa_project(h, W_dq, W_iuq, W_w, dt, L, B, d, r, n_h, d_I, q, w, c, part[0], stream));
     k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, tile_start, chunk_start, cnt);
     LSA_TRY(launched("training step: tiles"));
+    const double invN = 1.0 / ((double)L * (double)total_S);
+    if (train_tc::supported(dt, kdt, n_h, d_I)) {
+        const dim3 grid((unsigned)((total_S / train_tc::TT + B + 1 + train_tc::TPC - 1) / train_tc::TPC), (unsigned)L);
+#define LSA_TRAIN_ENTRIES_TC(KD)                                                                                   \
+        do {                                                                                                       \
+            LSA_TRY(set_smem(train_tc::k_train_entries_tc<KD>, train_tc::SMEM_BYTES));                            \
+            train_tc::k_train_entries_tc<KD><<<grid, train_tc::THREADS, train_tc::SMEM_BYTES, st>>>(              \
+                (const __nv_bfloat16 *)q, w, (const uint8_t *)K, k_scale, labels, seq_offsets, tile_start, B,       \
+                total_S, gamma, alpha, invN, dq, dw, loss_out);                                                    \
+        } while (0)
+        if (kdt == LSA_BF16) LSA_TRAIN_ENTRIES_TC(DT_BF16);
+        else LSA_TRAIN_ENTRIES_TC(DT_FP8);
+#undef LSA_TRAIN_ENTRIES_TC
+        LSA_TRY(launched("training step: entries (tensor cores)"));
+    } else {
     const size_t smem = train::entries_smem();
     const dim3 grid((unsigned)((total_S / train::TT + B + 1 + train::TPC - 1) / train::TPC), (unsigned)L);
-    const double invN = 1.0 / ((double)L * (double)total_S);
 #define LSA_TRAIN_ENTRIES(QD, KD)                                                                                  \
     do {                                                                                                           \
         LSA_TRY(set_smem(train::k_train_entries<QD, KD>, smem));                                                   \
@@ -810,6 +827,7 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
     else LSA_TRAIN_ENTRIES(DT_BF16, DT_FP8);
 #undef LSA_TRAIN_ENTRIES
     LSA_TRY(launched("training step: entries"));
+    }
     const dim3 gdc((unsigned)((r + 31) / 32), (unsigned)L);
     const int64_t n_iuq = (int64_t)L * nq * r / 4, n_dq = (int64_t)L * r * d / 4, n_w = (int64_t)L * n_h * d / 4;
     if (dt == LSA_F32) {
