@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(link_threads<CH>()) k_gather_rows(const int32_
 // may grow).  Three launches, all over the new fetched rows numbered in one range:
 //   k_incr_map    one thread per row: look the entry up in the previous (ascending) list of its
 //                 sequence; map[slot] = previous slot, or -1 and the row number appended to miss[]
-//   k_incr_copy   one thread per 16-byte chunk of every row with a previous slot (device copy)
+//   k_incr_copy   one warp per row with a previous slot (device copy), several rows in flight
 //   k_incr_fetch  the link launch over miss[0 .. *nmiss): as k_gather_rows
 // A previous list that is not ascending only costs host reads (a missed lookup fetches the row).
 
@@ -333,7 +333,8 @@ __global__ void __launch_bounds__(128) k_incr_map(const int32_t *__restrict__ id
     }
 }
 
-__global__ void __launch_bounds__(128) k_incr_copy(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
+template <int CH>  // 16-byte chunks per lane and row (row_bytes <= CH * 512)
+__global__ void __launch_bounds__(256) k_incr_copy(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
                                                    int B, const int64_t *__restrict__ poffs,
                                                    const int32_t *__restrict__ map, const uint8_t *__restrict__ prev_hot,
                                                    int row16, uint8_t *__restrict__ hot)
@@ -341,17 +342,43 @@ __global__ void __launch_bounds__(128) k_incr_copy(const int32_t *__restrict__ c
     extern __shared__ int pre[];
     __shared__ int warp_sum[32];
     const int total = block_count_prefix(count, offs, B, pre, warp_sum);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t rb = (int64_t)row16 * 16;
-    const int64_t units = (int64_t)total * row16;
-    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t g = u / row16;
-        const int ch = (int)(u - g * row16);
-        const int b = sequence_of_row(pre, B, g);
-        const int64_t slot = offs[b] + (g - pre[b]);
-        const int m = map[slot];
-        if (m < 0) continue;
-        const uint4 v = __ldg((const uint4 *)(prev_hot + (poffs[b] + m) * rb + (int64_t)ch * 16));
-        *(uint4 *)(hot + slot * rb + (int64_t)ch * 16) = v;
+    const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    // one warp per row, GATHER_ROWS_PER_WARP rows in flight per warp
+    for (int64_t g0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + warp) * GATHER_ROWS_PER_WARP; g0 < total;
+         g0 += wstride * GATHER_ROWS_PER_WARP) {
+        int64_t src[GATHER_ROWS_PER_WARP], dst[GATHER_ROWS_PER_WARP];
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++) {
+            src[r] = -1;
+            dst[r] = 0;
+            const int64_t g = g0 + r;
+            if (g < total) {
+                const int b = sequence_of_row(pre, B, g);
+                const int64_t slot = offs[b] + (g - pre[b]);
+                const int m = map[slot];
+                if (m >= 0) {
+                    src[r] = poffs[b] + m;
+                    dst[r] = slot;
+                }
+            }
+        }
+        uint4 v[GATHER_ROWS_PER_WARP][CH];
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++)
+#pragma unroll
+            for (int c = 0; c < CH; c++) {
+                const int ch = lane + 32 * c;
+                if (src[r] >= 0 && ch < row16) v[r][c] = __ldg((const uint4 *)(prev_hot + src[r] * rb + (int64_t)ch * 16));
+            }
+#pragma unroll
+        for (int r = 0; r < GATHER_ROWS_PER_WARP; r++)
+#pragma unroll
+            for (int c = 0; c < CH; c++) {
+                const int ch = lane + 32 * c;
+                if (src[r] >= 0 && ch < row16) *(uint4 *)(hot + dst[r] * rb + (int64_t)ch * 16) = v[r][c];
+            }
     }
 }
 

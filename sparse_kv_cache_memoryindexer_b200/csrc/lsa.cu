@@ -1,5 +1,6 @@
 // C ABI of the LSA indexer hot path (declared in include/lsa.h).  Host-side validation and
 // dispatch; every stage runs in the kernels included below (one translation unit).
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -236,11 +237,13 @@ lsa_status lsa_selftest_wait_timeout(int32_t *status_out, lsa_stream_t stream)
 
 // ------------------------------------------------------------------------------ stage 1
 
+// Workspace of lsa_project: c in the storage type [L][B][r], then its fp32 sums [L][B][r] (the
+// tensor-core path adds the partial sums of its K ranges there before rounding c once).
 size_t lsa_project_workspace_size(int L, int B, int d, int r, int n_h, int d_I, lsa_dtype dt)
 {
     (void)d; (void)n_h; (void)d_I;
     if (L <= 0 || B <= 0 || r <= 0) return 0;
-    return align_up((size_t)L * B * r * elem_bytes(dt), 256);
+    return align_up((size_t)L * B * r * elem_bytes(dt), 256) + align_up((size_t)L * B * r * 4, 256);
 }
 
 lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const void *W_w, lsa_dtype dt,
@@ -261,12 +264,26 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
     const int nq = n_h * d_I;
     void *c = workspace;
     if (proj_tc_supported(dt, B, d) && proj_tc_supported(dt, B, r)) {
+        // c and w in one launch, split along d so that every SM streams weights (fp32 partial sums
+        // added into zeroed buffers); c rounded to bf16 once; then q, all of r per tile
         const int sms = num_sms();
-        lsa_status s = launch_proj_tc(h, W_dq, c, false, L, B, r, d, sms, st);
-        if (s == LSA_OK) s = launched("project c (tensor cores)");
-        if (s == LSA_OK) s = launch_proj_tc(h, W_w, w_out, true, L, B, n_h, d, sms, st);
-        if (s == LSA_OK) s = launched("project w (tensor cores)");
-        if (s == LSA_OK) s = launch_proj_tc(c, W_iuq, q_out, false, L, B, nq, r, sms, st);
+        const int64_t nc = (int64_t)L * B * r;
+        float *c32 = (float *)((char *)workspace + align_up((size_t)nc * elem_bytes(dt), 256));
+        cudaError_t e = cudaMemsetAsync(c32, 0, sizeof(float) * (size_t)nc, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(w_out, 0, sizeof(float) * (size_t)L * B * n_h, st);
+        if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_project: %s", cudaGetErrorString(e));
+        const ProjProblem cw[2] = {{W_dq, c32, r, true}, {W_w, w_out, n_h, true}};
+        const bool split[2] = {true, true};
+        lsa_status s = launch_proj_tc(h, cw, split, 2, L, B, d, sms, 2, st);
+        if (s == LSA_OK) s = launched("project c and w (tensor cores)");
+        if (s == LSA_OK) {
+            k_proj_round<<<(unsigned)std::min<int64_t>((nc + 255) / 256, (int64_t)sms * 8), 256, 0, st>>>(
+                c32, (__nv_bfloat16 *)c, nc);
+            s = launched("project: round c");
+        }
+        const ProjProblem qp = {W_iuq, q_out, nq, false};
+        const bool nosplit = false;
+        if (s == LSA_OK) s = launch_proj_tc(c, &qp, &nosplit, 1, L, B, r, sms, 2, st);
         if (s == LSA_OK) s = launched("project q (tensor cores)");
         if (s != LSA_OK) return fail(s, "lsa_project: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
     } else if (dt == LSA_BF16) {
@@ -481,8 +498,15 @@ lsa_status lsa_fetch_gather_incremental(const int32_t *idx, const int32_t *count
     k_incr_map<<<sms * 4, 128, smem, st>>>(idx, count, seq_offsets, B, prev_idx, prev_count, prev_seq_offsets, map, miss,
                                            nmiss);
     LSA_TRY(launched("incremental fetch: lookup"));
-    k_incr_copy<<<sms * 8, 128, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
-                                            row16, (uint8_t *)hot_kv);
+    if (row16 <= 32)
+        k_incr_copy<1><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
+                                                   row16, (uint8_t *)hot_kv);
+    else if (row16 <= 64)
+        k_incr_copy<2><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
+                                                   row16, (uint8_t *)hot_kv);
+    else
+        k_incr_copy<4><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
+                                                   row16, (uint8_t *)hot_kv);
     LSA_TRY(launched("incremental fetch: device copy"));
     const uint8_t *src = (const uint8_t *)dpool;
     if (row16 <= 32)
@@ -566,13 +590,14 @@ static int64_t step_max_chunks(int B, int64_t total_S, int W)
     return (total_S + (int64_t)B * W) / stepsel::CH + B + 1;
 }
 
+// Select workspace of one decode step: chunk starts, state, bucket histograms with finish counters,
+// the stage (capacity S_b + W keys per query) and the selection (LSA_MAX_TOPK keys per query).
 static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[5])
 {
-    const int64_t mc = step_max_chunks(B, total_S, W);
     sp[0] = align_up(sizeof(int) * (size_t)(B + 1), 256);
-    sp[1] = align_up(sizeof(uint32_t) * 4 * (size_t)B, 256);
-    sp[2] = align_up(sizeof(int) * 258 * (size_t)B, 256);  // digit histograms, two finish counters
-    sp[3] = align_up(sizeof(int) * 2 * (size_t)mc, 256);
+    sp[1] = align_up(sizeof(uint32_t) * stepsel::NS * (size_t)B, 256);
+    sp[2] = align_up(sizeof(int) * (stepsel::NB + 1) * (size_t)B, 256);
+    sp[3] = align_up(sizeof(unsigned long long) * (size_t)(total_S + (int64_t)B * W + 1), 256);
     sp[4] = align_up(sizeof(unsigned long long) * (size_t)B * LSA_MAX_TOPK, 256);
     return sp[0] + sp[1] + sp[2] + sp[3] + sp[4];
 }
@@ -667,28 +692,23 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     int *chunk_start = (int *)sb;
     uint32_t *state = (uint32_t *)(sb + sp[0]);
     int *ghist = (int *)(sb + sp[0] + sp[1]);
-    int *gtc = (int *)(sb + sp[0] + sp[1] + sp[2]);
-    const int64_t mc = step_max_chunks(B, total_S, W);
-    int *eqc = gtc + mc;
+    unsigned long long *stage = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2]);
     unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
+    const int64_t mc = step_max_chunks(B, total_S, W);
     const int32_t *tcnt = W > 0 ? win_count : nullptr;
-    int *done_hist = ghist + 256 * (size_t)B, *done_count = done_hist + B;
     stepsel::k_ss_setup<<<1, 1024, 0, st>>>(count, seq_offsets, tcnt, W, B, k, chunk_start, state, ghist);
-    for (int pass = 0; pass < 4; pass++)
-        stepsel::k_ss_hist<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B,
-                                                                 chunk_start, state, pass, ghist, done_hist);
-    stepsel::k_ss_count<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
-                                                              state, gtc, eqc, done_count);
+    stepsel::k_ss_hist12<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
+                                                               state, ghist);
     stepsel::k_ss_write<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
-                                                              state, gtc, eqc, LSA_MAX_TOPK, sel);
+                                                              state, LSA_MAX_TOPK, sel, stage);
     int kpow2 = 1;
     while (kpow2 < k) kpow2 <<= 1;
-    const size_t smem = sizeof(unsigned long long) * (size_t)kpow2;
-    LSA_TRY(set_smem(stepsel::k_ss_sort, smem));
-    stepsel::k_ss_sort<<<(unsigned)B, stepsel::SORT_TH, smem, st>>>(sel, LSA_MAX_TOPK, state, idx, count, seq_offsets,
-                                                                   k, kpow2, topk_idx, topk_score);
+    const size_t smem = sizeof(unsigned long long) * ((size_t)kpow2 + stepsel::SCAP);
+    LSA_TRY(set_smem(stepsel::k_ss_final, smem));
+    stepsel::k_ss_final<<<(unsigned)B, stepsel::SORT_TH, smem, st>>>(sel, LSA_MAX_TOPK, stage, state, W, idx, count,
+                                                                    seq_offsets, k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
-    g_launches.fetch_add(7, std::memory_order_relaxed);  // setup, 4 histogram passes, count, write (+ sort)
+    g_launches.fetch_add(3, std::memory_order_relaxed);  // setup, histogram, write (+ final)
     return ok();
 }
 
@@ -734,8 +754,8 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
 static size_t train_ws_parts(int L, int B, int64_t T, int d, int r, int n_h, int d_I, lsa_dtype dt, size_t part[8])
 {
     const size_t eb = elem_bytes(dt), LB = (size_t)L * B, nq = (size_t)n_h * d_I;
-    (void)T; (void)d;
-    part[0] = align_up(LB * r * eb, 256);               // c (the projection's workspace)
+    (void)T;
+    part[0] = lsa_project_workspace_size(L, B, d, r, n_h, d_I, dt);  // c (the projection's workspace)
     part[1] = align_up(LB * nq * eb, 256);              // q
     part[2] = align_up(LB * n_h * 4, 256);              // w
     part[3] = align_up(LB * nq * 4, 256);               // dq
@@ -792,7 +812,7 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
     int *chunk_start = tile_start + (B + 1);
     int32_t *cnt = chunk_start + (B + 1);
     const int nq = n_h * d_I;
-    cudaError_t e = cudaMemsetAsync(dq, 0, part[3] + part[4], st);  // dq and dw are adjacent
+    cudaError_t e = cudaMemsetAsync(dq, 0, part[3] + part[4] + part[5], st);  // dq, dw and dc are adjacent
     if (e == cudaSuccess) e = cudaMemsetAsync(loss_out, 0, sizeof(double), st);
     if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_indexer_train_step: %s", cudaGetErrorString(e));
     LSA_TRY(lsa_project(h, W_dq, W_iuq, W_w, dt, L, B, d, r, n_h, d_I, q, w, c, part[0], stream));
@@ -828,19 +848,27 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
 #undef LSA_TRAIN_ENTRIES
     LSA_TRY(launched("training step: entries"));
     }
-    const dim3 gdc((unsigned)((r + 31) / 32), (unsigned)L);
-    const int64_t n_iuq = (int64_t)L * nq * r / 4, n_dq = (int64_t)L * r * d / 4, n_w = (int64_t)L * n_h * d / 4;
+    const dim3 gdc((unsigned)((r + train::DC_COLS - 1) / train::DC_COLS), (unsigned)((nq + train::DC_OCH - 1) / train::DC_OCH),
+                   (unsigned)L);
+    auto gout = [&](int M, int N) {
+        return dim3((unsigned)((N / 4 + 255) / 256), (unsigned)((M + train::OUT_MR - 1) / train::OUT_MR), (unsigned)L);
+    };
+#define LSA_OUTER3(VD, BM)                                                                                   \
+    do {                                                                                                     \
+        train::k_outer<VD, BM><<<gout(nq, r), 256, 0, st>>>(dq, c, L, B, nq, r, g_Wiuq);                     \
+        train::k_outer<VD, BM><<<gout(r, d), 256, 0, st>>>(dc, h, L, B, r, d, g_Wdq);                        \
+        train::k_outer<VD, BM><<<gout(n_h, d), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);                     \
+    } while (0)
     if (dt == LSA_F32) {
         train::k_train_dc<DT_F32><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
-        train::k_outer<DT_F32><<<(unsigned)((n_iuq + 255) / 256), 256, 0, st>>>(dq, c, L, B, nq, r, g_Wiuq);
-        train::k_outer<DT_F32><<<(unsigned)((n_dq + 255) / 256), 256, 0, st>>>(dc, h, L, B, r, d, g_Wdq);
-        train::k_outer<DT_F32><<<(unsigned)((n_w + 255) / 256), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);
+        if (B <= 8) LSA_OUTER3(DT_F32, 8);
+        else LSA_OUTER3(DT_F32, train::DC_BMAX);
     } else {
         train::k_train_dc<DT_BF16><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
-        train::k_outer<DT_BF16><<<(unsigned)((n_iuq + 255) / 256), 256, 0, st>>>(dq, c, L, B, nq, r, g_Wiuq);
-        train::k_outer<DT_BF16><<<(unsigned)((n_dq + 255) / 256), 256, 0, st>>>(dc, h, L, B, r, d, g_Wdq);
-        train::k_outer<DT_BF16><<<(unsigned)((n_w + 255) / 256), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);
+        if (B <= 8) LSA_OUTER3(DT_BF16, 8);
+        else LSA_OUTER3(DT_BF16, train::DC_BMAX);
     }
+#undef LSA_OUTER3
     LSA_TRY(launched("training step: weight gradients"));
     g_launches.fetch_add(3, std::memory_order_relaxed);
     return ok();

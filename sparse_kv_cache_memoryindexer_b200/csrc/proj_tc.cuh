@@ -5,12 +5,17 @@
 // (K contiguous).  The weights dominate the bytes (B is a batch of sequences, at most 256), so
 // the weight rows are the MMA A operand (M = 128 output rows per tile, streamed once by TMA) and
 // the batch is the B operand (N = B rounded up to 16; the small X tiles are re-read from L2 by
-// every CTA).  A tile covers all of K: its accumulator (N fp32 columns of TMEM) is complete when
-// the epilogue reads it, which rounds to the output type (bf16 nearest-even, or fp32) and writes
-// Y[l][b][o] with consecutive lanes on consecutive o.
+// every CTA).
+//
+// A launch serves one or two problems with the same X (c and w both read h).  Its work units are
+// (problem, 128-row tile, range of K): a problem whose tiles alone would leave SMs idle is split
+// along K, its units adding fp32 partial sums into a zeroed fp32 output with atomics (c is rounded
+// to bf16 by k_proj_round afterwards; w is fp32 anyway); a problem with enough tiles takes all of K
+// per unit and its epilogue rounds to the output type (bf16 nearest-even, or fp32) and stores.
+// Either way every output is one fp32 sum of its K products, rounded once.
 //
 // Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue (one TMEM lane
-// quarter each).  Two accumulators, so a tile's epilogue overlaps the next tile's MMAs.  Every
+// quarter each).  Two accumulators, so a unit's epilogue overlaps the next unit's MMAs.  Every
 // ring is consumed in order by one consumer (group); waits are bounded as in the other
 // tensor-core kernels.
 #pragma once
@@ -25,13 +30,51 @@ constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 6 * 32;
 constexpr uint32_t A_BYTES = 128 * KB * 2;
 
+struct Prob {
+    void *out;          // [L][B][R]: bf16 or fp32 (stored), or fp32 (ksplit > 1: added atomically)
+    int R;              // output rows
+    int out_f32;
+    int mtiles;         // 128-row tiles per layer
+    int ksplit;         // K ranges per tile
+    int nkb_per;        // K blocks per range
+    int units;          // L * mtiles * ksplit
+};
+
 struct Params {
-    void *out;          // [L][B][R] bf16 or fp32
-    int L, B, R, K;     // layers, batch, output rows, reduction length
+    Prob pr[2];
+    int nprob;
+    int L, B, K;        // layers, batch, reduction length
     int NB;             // MMA N = B rounded up to 16
     int stages;
-    int out_f32;
 };
+
+struct Unit {
+    int prob, l, m0, kb0, kb1;
+    void *out;
+    int R, out_f32, ksplit;
+};
+
+// The problem fields are picked with selects (no dynamic index into the kernel parameters).
+__device__ __forceinline__ Unit unit_of(const Params &p, int u, int nkb)
+{
+    Unit x;
+    x.prob = u < p.pr[0].units ? 0 : 1;
+    const bool one = x.prob == 1;
+    const int ksplit = one ? p.pr[1].ksplit : p.pr[0].ksplit;
+    const int mtiles = one ? p.pr[1].mtiles : p.pr[0].mtiles;
+    const int nkb_per = one ? p.pr[1].nkb_per : p.pr[0].nkb_per;
+    const int v = u - (one ? p.pr[0].units : 0);
+    const int t = v / ksplit, ks = v % ksplit;
+    x.l = t / mtiles;
+    x.m0 = (t % mtiles) * 128;
+    x.kb0 = ks * nkb_per;
+    x.kb1 = min(nkb, x.kb0 + nkb_per);
+    x.out = one ? p.pr[1].out : p.pr[0].out;
+    x.R = one ? p.pr[1].R : p.pr[0].R;
+    x.out_f32 = one ? p.pr[1].out_f32 : p.pr[0].out_f32;
+    x.ksplit = ksplit;
+    return x;
+}
 
 __host__ __device__ inline uint32_t b_bytes(int NB) { return (uint32_t)NB * KB * 2; }
 __host__ __device__ inline uint32_t stage_bytes(int NB) { return A_BYTES + b_bytes(NB); }
@@ -45,8 +88,9 @@ __host__ __device__ inline uint32_t tmem_cols(int NB)  // two accumulators, a po
     return c;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    k_proj_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, Params p)
+__global__ void __launch_bounds__(THREADS)
+    k_proj_tc(const __grid_constant__ CUtensorMap wmap0, const __grid_constant__ CUtensorMap wmap1,
+              const __grid_constant__ CUtensorMap xmap, Params p)
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -63,8 +107,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int *abort_flag = (volatile int *)(misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mtiles = (p.R + 127) / 128;
-    const int ntiles = p.L * mtiles;
+    const int nunits = p.pr[0].units + (p.nprob > 1 ? p.pr[1].units : 0);
     const int nkb = (p.K + KB - 1) / KB;
     const uint32_t ncols = tmem_cols(p.NB), acol = acc_cols(p.NB);
 
@@ -94,7 +137,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------- TMA producer
         const bool leader = elect_one();
         if (leader) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&wmap) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&wmap0) : "memory");
+            if (p.nprob > 1) asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&wmap1) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&xmap) : "memory");
         }
         int stage = 0;
@@ -103,15 +147,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool issued[MAX_STAGES];
         for (int i = 0; i < MAX_STAGES; i++) issued[i] = false;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const int l = t / mtiles, m0 = (t % mtiles) * 128;
-            for (int kb = 0; kb < nkb; kb++) {
+        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+            const Unit x = unit_of(p, u, nkb);
+            const CUtensorMap *wm = x.prob == 0 ? &wmap0 : &wmap1;
+            for (int kb = x.kb0; kb < x.kb1; kb++) {
                 if (!mbar_wait_warp(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
                 if (leader) {
                     mbar_expect_tx(full(stage), sbytes);
                     const uint32_t dst = sbase + (uint32_t)stage * sbytes;
-                    tma_load_2d(dst, &wmap, kb * KB, l * p.R + m0, full(stage));
-                    tma_load_2d(dst + A_BYTES, &xmap, kb * KB, l * p.B, full(stage));
+                    tma_load_2d(dst, wm, kb * KB, x.l * x.R + x.m0, full(stage));
+                    tma_load_2d(dst + A_BYTES, &xmap, kb * KB, x.l * p.B, full(stage));
                 }
                 __syncwarp();
                 issued[stage] = true;
@@ -131,11 +176,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         int stage = 0, acc = 0;
         uint32_t phase = 0, accphase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+            const Unit x = unit_of(p, u, nkb);
             if (!mbar_wait_warp(tempty(acc), accphase ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d = tmem + (uint32_t)acc * acol;
-            for (int kb = 0; kb < nkb; kb++) {
+            for (int kb = x.kb0; kb < x.kb1; kb++) {
                 if (!mbar_wait_warp(full(stage), phase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a_base = sbase + (uint32_t)stage * sbytes;
@@ -143,9 +189,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < KB / 16; kk++)
-                        mma_bf16(d, sdesc(a_base + 32 * kk), sdesc(b_base + 32 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16(d, sdesc(a_base + 32 * kk), sdesc(b_base + 32 * kk), idesc, (kb > x.kb0 || kk > 0) ? 1u : 0u);
                     mma_commit(empty(stage));
-                    if (kb == nkb - 1) mma_commit(tfull(acc));
+                    if (kb == x.kb1 - 1) mma_commit(tfull(acc));
                 }
                 __syncwarp();
                 if (++stage == p.stages) { stage = 0; phase ^= 1; }
@@ -158,12 +204,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         int acc = 0;
         uint32_t accphase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const int l = t / mtiles, m0 = (t % mtiles) * 128;
+        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+            const Unit x = unit_of(p, u, nkb);
             if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const int o = m0 + quarter * 32 + lane;
-            const bool valid = o < p.R;
+            const int o = x.m0 + quarter * 32 + lane;
+            const bool valid = o < x.R;
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * acol;
             for (int b0 = 0; b0 < p.NB; b0 += 32) {
                 float v[32];
@@ -173,9 +219,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int i = 0; i < 32; i++) {
                     const int b = b0 + i;
                     if (valid && b < p.B) {
-                        const int64_t at = ((int64_t)l * p.B + b) * p.R + o;
-                        if (p.out_f32) ((float *)p.out)[at] = v[i];
-                        else ((__nv_bfloat16 *)p.out)[at] = __float2bfloat16_rn(v[i]);
+                        const int64_t at = ((int64_t)x.l * p.B + b) * x.R + o;
+                        if (x.ksplit > 1) atomicAdd((float *)x.out + at, v[i]);
+                        else if (x.out_f32) ((float *)x.out)[at] = v[i];
+                        else ((__nv_bfloat16 *)x.out)[at] = __float2bfloat16_rn(v[i]);
                     }
                 }
             }
@@ -200,34 +247,79 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 inline bool proj_tc_supported(int dt, int B, int K) { return dt == DT_BF16 && B >= 1 && B <= 256 && K % 8 == 0 && tc_available(); }
 
-// out[l][b][o] = sum_k X[l][b][k] W[l][o][k]; X bf16 [L][B][K], W bf16 [L][R][K], out bf16 or fp32.
-inline lsa_status launch_proj_tc(const void *X, const void *W, void *out, bool out_f32, int L, int B, int R, int K,
-                                 int sms, cudaStream_t st)
+// One problem of a launch: out[l][b][o] = sum_k X[l][b][k] W[l][o][k], W bf16 [L][R][K].
+struct ProjProblem {
+    const void *W;
+    void *out;          // fp32 (added atomically) when split along K, else stored as bf16 or fp32
+    int R;
+    bool out_f32;
+};
+
+// K ranges of a problem so that all problems of a launch reach about `want_units` units (at least
+// two K blocks each); split == false keeps all of K per unit.
+inline void proj_split(int L, int R, int K, int want_units, bool split, int &ksplit, int &nkb_per)
 {
     using namespace proj;
-    CUtensorMap wmap, xmap;
+    const int nkb = (K + KB - 1) / KB;
+    const int tiles = L * ((R + 127) / 128);
+    int ks = 1;
+    if (split) {
+        ks = (want_units + tiles - 1) / tiles;
+        const int cap = nkb / 2 > 1 ? nkb / 2 : 1;
+        ks = ks < 1 ? 1 : (ks > cap ? cap : ks);
+    }
+    nkb_per = (nkb + ks - 1) / ks;
+    ksplit = (nkb + nkb_per - 1) / nkb_per;
+}
+
+// One launch over one or two problems sharing X bf16 [L][B][K]; split problems need a zeroed fp32
+// output.  stages_max bounds the pipeline (fewer stages leave room for two CTAs per SM).
+inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const bool *split, int nprob, int L, int B,
+                                 int K, int sms, int ctas_per_sm, cudaStream_t st)
+{
+    using namespace proj;
+    CUtensorMap wmap[2], xmap;
     proj::Params p;
-    p.out = out;
+    p.nprob = nprob;
     p.L = L;
     p.B = B;
-    p.R = R;
     p.K = K;
     p.NB = (B + 15) / 16 * 16;
-    p.out_f32 = out_f32 ? 1 : 0;
-    bool ok = make_map_2d(&wmap, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * R, (uint64_t)K, KB, 128);
-    ok = ok && make_map_2d(&xmap, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * B, (uint64_t)K, KB, (uint32_t)p.NB);
+    const int want = sms * ctas_per_sm;
+    bool ok = make_map_2d(&xmap, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * B, (uint64_t)K, KB, (uint32_t)p.NB);
+    int total = 0;
+    for (int i = 0; i < 2; i++) {
+        const ProjProblem &q = pb[i < nprob ? i : 0];
+        Prob &r = p.pr[i];
+        r.out = q.out;
+        r.R = q.R;
+        r.out_f32 = q.out_f32 ? 1 : 0;
+        r.mtiles = (q.R + 127) / 128;
+        proj_split(L, q.R, K, want, i < nprob && split[i], r.ksplit, r.nkb_per);
+        r.units = i < nprob ? L * r.mtiles * r.ksplit : 0;
+        total += r.units;
+        ok = ok && make_map_2d(&wmap[i], q.W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * q.R, (uint64_t)K, KB, 128);
+    }
     if (!ok) return LSA_ERR_CUDA;
-    const uint32_t max_smem = 227 * 1024;
+    const uint32_t max_smem = (uint32_t)((227 * 1024) / ctas_per_sm) - 1024;
     p.stages = MAX_STAGES;
     while (p.stages > 2 && smem_total(p.NB, p.stages) > max_smem) p.stages--;
     const uint32_t smem = smem_total(p.NB, p.stages);
     if (smem > max_smem) return LSA_ERR_UNSUPPORTED;
     cudaError_t e = cudaFuncSetAttribute(k_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return LSA_ERR_CUDA;
-    const int ntiles = L * ((R + 127) / 128);
-    k_proj_tc<<<ntiles < sms ? ntiles : sms, THREADS, smem, st>>>(wmap, xmap, p);
+    const int grid = total < want ? total : want;
+    k_proj_tc<<<grid, THREADS, smem, st>>>(wmap[0], wmap[1], xmap, p);
     e = cudaGetLastError();
     return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
+// c (fp32 sums) -> bf16, n elements.
+__global__ void __launch_bounds__(256) k_proj_round(const float *__restrict__ in, __nv_bfloat16 *__restrict__ out,
+                                                    int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256)
+        out[i] = __float2bfloat16_rn(in[i]);
 }
 
 }  // namespace lsa

@@ -11,15 +11,18 @@
 //   bf16 keys  kind::f16, N = 64 heads, 8 MMAs of K = 16 per job.
 //   E4M3 keys  kind::f8f6f4 straight from the TMA tile (no conversion), K = 32.  The bf16 queries
 //              are split by k_q_split_e4m3 into two E4M3 parts, q_h 2^s_h = hi_h + lo_h (s_h puts
-//              the head's largest element in [2^7, 2^8)), stacked as N = 128 columns (hi heads,
-//              then lo heads): 4 MMAs per job; the epilogue adds the two partial dot products and
-//              w_h is pre-multiplied by 2^-s_h.  hi + lo is the query exactly (8 significant
-//              bits = 4 + 4) for every element at least 2^-9 times its head's largest; smaller
-//              elements fall into the E4M3 subnormal range and keep an absolute error below
-//              2^-17 of the head's largest.  Each E4M3 x E4M3 product is exact and accumulates
-//              in fp32.
-// Fewer, larger MMA instructions matter: issue, not math, bounds a job (each 128 x 64 x 16 MMA
-// costs far more than its 32 cycles of math).
+//              the head's largest element in [2^7, 2^8)), stored as 128 rows (hi heads, then lo
+//              heads); a job runs 8 MMAs of N = 64 into one 64-column accumulator, the 4 over the
+//              hi rows and then the 4 over the lo rows of the same key tile, so the sum of the
+//              two partial dot products comes out of the tensor core; w_h is pre-multiplied by
+//              2^-s_h.  hi + lo is the query exactly (8 significant bits = 4 + 4) for every
+//              element at least 2^-9 times its head's largest; smaller elements fall into the
+//              E4M3 subnormal range and keep an absolute error below 2^-17 of the head's largest.
+//              Each E4M3 x E4M3 product is exact and accumulates in fp32.
+// The epilogue's weighted ReLU sum runs as packed fp32 pairs (fma.rn.f32x2), two heads per
+// instruction.  Timings that led here: hi | lo as N = 128 columns with the sum in the epilogue
+// 696 us, the same with a packed epilogue 676 us, accumulated in the MMA with a packed epilogue
+// 656 us (1M x 32 entries x 3 layers).
 //
 // Warp roles (persistent CTA per SM, contiguous range of tiles; every role's warp runs converged):
 //   warps 0, 11 TMA producers, one per parity group (an elected lane issues): key tiles; warp 0
@@ -48,9 +51,9 @@ constexpr int NH = 64;           // heads
 constexpr int MAX_STAGES = 12;
 constexpr int MAX_L_TC = 3;      // indexer layers handled by one launch
 constexpr int NACC_BF16 = 8;     // TMEM accumulator slots: 8 x 64 columns (bf16 keys)
-constexpr int NACC_E4M3 = 4;     //                         4 x 128 columns (E4M3 keys: hi | lo)
+constexpr int NACC_E4M3 = 8;     //                         8 x 64 columns (E4M3 keys: hi + lo accumulated)
 constexpr uint32_t IDESC_BF16 = idesc_bf16(128, NH);
-constexpr uint32_t IDESC_E4M3 = idesc_f16(128, 2 * NH);  // format code 0 is E4M3 under kind::f8f6f4
+constexpr uint32_t IDESC_E4M3 = idesc_f16(128, NH);  // format code 0 is E4M3 under kind::f8f6f4
 
 __device__ __forceinline__ void mma_e4m3(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate)
 {
@@ -110,6 +113,17 @@ __global__ void __launch_bounds__(256) k_q_split_e4m3(const __nv_bfloat16 *__res
     *(uint32_t *)(base + (int64_t)h * DI + 4 * lane) = hi4;
     *(uint32_t *)(base + (int64_t)(NH + h) * DI + 4 * lane) = lo4;
     if (lane == 0) ws[row] = w[row] * down;
+}
+
+// d = a * b + c on two fp32 lanes at once (one fma.rn.f32x2; each lane rounds as fmaf).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
 }
 
 struct Params {
@@ -184,7 +198,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     k_score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, Params p)
 {
     constexpr int nacc = FP8 ? NACC_E4M3 : NACC_BF16;
-    constexpr int ncol = FP8 ? 2 * NH : NH;           // accumulator columns per job
+    constexpr int ncol = NH;                          // accumulator columns per job
     constexpr int AP = nacc / 2;                       // accumulator slots per parity group
     const int SP = p.stages / 2;                       // key stages per parity group
     constexpr uint32_t kbytes = FP8 ? 128 * 128 : 128 * 256;
@@ -342,8 +356,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (elect_one()) {
                         if (FP8) {
 #pragma unroll
-                            for (int kk = 0; kk < DI / 32; kk++)
+                            for (int kk = 0; kk < DI / 32; kk++)  // hi rows (bytes 0 .. 8191 of the query tile)
                                 mma_e4m3(d, sdesc(a_base + 32 * kk), sdesc(b_base + 32 * kk), IDESC_E4M3, kk > 0 ? 1u : 0u);
+#pragma unroll
+                            for (int kk = 0; kk < DI / 32; kk++)  // lo rows, accumulated into the same columns
+                                mma_e4m3(d, sdesc(a_base + 32 * kk), sdesc(b_base + 8192 + 32 * kk), IDESC_E4M3, 1u);
                         } else {
 #pragma unroll
                             for (int kk = 0; kk < DI / 16; kk++) {
@@ -418,20 +435,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc_fence_after();
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ncol);
                 const float *wl = myw + l * NH;
-                float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+                float2 xa = make_float2(0.f, 0.f), xb = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int hh = 0; hh < 2; hh++) {  // heads 32*hh .. 32*hh + 31
                     float v[32];
                     tmem_ld32(taddr + 32 * hh, v);
-                    if (FP8) {
-                        float vl[32];
-                        tmem_ld32(taddr + NH + 32 * hh, vl);  // the lo parts of the same heads
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; i++) v[i] += vl[i];
-                    } else {
-                        tmem_wait_ld();
-                    }
+                    tmem_wait_ld();
                     if (hh == 1) {
                         tc_fence_before();
                         __syncwarp();
@@ -440,13 +449,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int h = 0; h < 32; h += 4) {
                         const float4 wa = *(const float4 *)(wl + 32 * hh + h);
-                        x0 = fmaf(wa.x, fmaxf(v[h], 0.f), x0);
-                        x1 = fmaf(wa.y, fmaxf(v[h + 1], 0.f), x1);
-                        x2 = fmaf(wa.z, fmaxf(v[h + 2], 0.f), x2);
-                        x3 = fmaf(wa.w, fmaxf(v[h + 3], 0.f), x3);
+                        xa = fma2(make_float2(wa.x, wa.y), make_float2(fmaxf(v[h], 0.f), fmaxf(v[h + 1], 0.f)), xa);
+                        xb = fma2(make_float2(wa.z, wa.w), make_float2(fmaxf(v[h + 2], 0.f), fmaxf(v[h + 3], 0.f)), xb);
                     }
                 }
-                float x = (x0 + x1) + (x2 + x3);
+                float x = (xa.x + xa.y) + (xb.x + xb.y);
                 if (valid) {
                     if (FP8) {
                         const float sc = l == 0 ? sc0 : (l == 1 ? sc1 : sc2);

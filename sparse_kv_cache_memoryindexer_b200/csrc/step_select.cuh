@@ -1,22 +1,22 @@
 // Top-k select of one decode step, spread over many CTAs.  A step has one query per sequence, so
 // the one-CTA-per-query select of the batched call would leave all but B SMs idle; here the
 // candidates of a query (its F fetched slots, then its window entries as candidates F .. F + n - 1,
-// reported as entries S_b + j) are cut into chunks of CH, and the most-significant-digit-first
-// radix search on the order-preserving keys runs with one CTA per chunk:
-//   k_ss_setup   per query: candidates, chunk ranges (a prefix over the sequences), search state
-//   k_ss_hist    per chunk: histogram of the next 8-bit digit of the keys that match the prefix so
-//                far, added to the query's histogram in global memory; the query's last chunk to
-//                finish then picks the digit where the count from the top reaches the keys still
-//                wanted (4 passes: the k-th largest key K*)
-//   k_ss_count   per chunk: keys above K* and keys equal to it; the query's last chunk turns the
-//                chunk counts into chunk offsets (slot order)
-//   k_ss_write   per chunk: every key above K*, and the first equal keys in slot order, to the
-//                query's selection
-//   k_ss_sort    per query: bitonic sort of the selection (key descending, slot ascending) and the
-//                output, as the one-CTA select writes it.
-// CTAs of one launch do not wait for one another: the per-query step after a launch's chunks runs
-// in whichever chunk CTA of the query finishes last (a counter per query, reset by that CTA), and
-// kernel boundaries order the rest.
+// reported as entries S_b + j) are cut into chunks of CH with one CTA per chunk.  A candidate's
+// 64-bit key is (order-preserving score key << 32) | ~slot: larger score first, then smaller slot,
+// and no two keys are equal.
+//   k_ss_setup   per query: candidates, chunk ranges (a prefix over the sequences), state
+//   k_ss_hist12  per chunk: histogram of the top 12 bits of the score keys, added to the query's
+//                histogram in global memory; the query's last chunk to finish picks the bucket
+//                beta holding the k-th largest key (the keys above beta are all selected)
+//   k_ss_write   per chunk: keys of higher buckets appended to the query's selection, keys of
+//                bucket beta appended to the query's stage (order does not matter: the keys carry
+//                their slots)
+//   k_ss_final   per query: the `want` largest staged keys (a sort in shared memory, or a radix
+//                select over the stage for a crowded bucket) complete the selection; bitonic sort
+//                of the k keys and the output, as the one-CTA select writes it.
+// A query with at most k candidates takes them all.  CTAs of one launch do not wait for one
+// another: the per-query step after the histogram runs in whichever chunk CTA of the query finishes
+// last (a counter per query, reset by that CTA), and kernel boundaries order the rest.
 #pragma once
 #include "common.cuh"
 
@@ -26,7 +26,10 @@ namespace stepsel {
 
 constexpr int CH = 2048;   // candidates per chunk
 constexpr int TH = 256;    // threads per chunk CTA
-constexpr int SORT_TH = 512;
+constexpr int SORT_TH = 1024;
+constexpr int NB = 4096;   // buckets of the first pass (top 12 bits of the score key)
+constexpr int SCAP = 8192; // staged keys a final CTA sorts in shared memory
+constexpr int NS = 8;      // state words per query
 
 struct Query {
     const float *row;   // fetched scores (query slot 0 of the Y layout)
@@ -55,9 +58,9 @@ __device__ __forceinline__ uint32_t key_of(const Query &q, int j)
     return float_to_ordered(j < q.F0 ? q.row[j] : q.trow[j - q.F0]);
 }
 
-// state per query: [0] prefix (the key bits fixed so far), [1] keys still wanted at the prefix,
-// [2] keys above the final K*, [3] candidates.  ghist: [B][256] digit histograms, then the
-// per-query finish counters of k_ss_hist [B] and of k_ss_count [B].
+// state per query (NS words): [0] bucket beta, [1] keys wanted from bucket beta (0: the query takes
+// every candidate), [2] keys of higher buckets, [3] candidates, [4] keys appended to the selection,
+// [5] keys appended to the stage.  ghist: [B][NB] bucket histograms, then the finish counters [B].
 __global__ void __launch_bounds__(1024) k_ss_setup(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
                                                    const int32_t *__restrict__ tail_count, int W, int B, int k,
                                                    int *__restrict__ chunk_start, uint32_t *__restrict__ state,
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(1024) k_ss_setup(const int32_t *__restrict__ c
         carry = 0;
         chunk_start[0] = 0;
     }
-    for (int i = threadIdx.x; i < B * 258; i += blockDim.x) ghist[i] = 0;
+    for (int i = threadIdx.x; i < B * (NB + 1); i += blockDim.x) ghist[i] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int base = 0; base < B; base += blockDim.x) {
@@ -83,11 +86,15 @@ __global__ void __launch_bounds__(1024) k_ss_setup(const int32_t *__restrict__ c
             nt = nt < 0 ? 0 : (nt > W ? W : nt);
             const int nc = F + nt;
             n = (nc + CH - 1) / CH;
-            // a query with at most k candidates takes them all: prefix 0 is below every key
-            state[4 * b + 0] = 0u;
-            state[4 * b + 1] = nc > k ? (uint32_t)k : 0u;
-            state[4 * b + 2] = nc > k ? 0u : (uint32_t)nc;
-            state[4 * b + 3] = (uint32_t)nc;
+            uint32_t *st = state + NS * b;
+            st[0] = 0u;
+            st[1] = nc > k ? (uint32_t)k : 0u;
+            st[2] = 0u;
+            st[3] = (uint32_t)nc;
+            st[4] = 0u;
+            st[5] = 0u;
+            st[6] = 0u;
+            st[7] = 0u;
         }
         const int inc = warp_incl_scan(n);
         if (lane == 31) wt[warp] = inc;
@@ -159,178 +166,196 @@ __device__ __forceinline__ void block_excl_scan2(int a, int b, int &pa, int &pb,
     __syncthreads();  // wa, wb free for the next call
 }
 
-__global__ void __launch_bounds__(TH) k_ss_hist(const float *__restrict__ Y, int tau_y, const int32_t *__restrict__ count,
-                                                const int64_t *__restrict__ offs, const float *__restrict__ tail,
-                                                const int32_t *__restrict__ tail_count, int W, int B,
-                                                const int *__restrict__ chunk_start, uint32_t *state, int pass,
-                                                int *ghist, int *done)
+__global__ void __launch_bounds__(TH) k_ss_hist12(const float *__restrict__ Y, int tau_y,
+                                                  const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
+                                                  const float *__restrict__ tail, const int32_t *__restrict__ tail_count,
+                                                  int W, int B, const int *__restrict__ chunk_start, uint32_t *state,
+                                                  int *ghist)
 {
-    static_assert(TH == 256, "one digit bin per thread in the digit step");
-    __shared__ int hist[256];
+    __shared__ int hist[NB];
+    __shared__ int s_beta, s_above;
     const int c = blockIdx.x;
     if (c >= chunk_start[B]) return;
     const int b = query_of_chunk(chunk_start, B, c);
-    const uint32_t remaining = state[4 * b + 1];
-    if (remaining == 0u) return;  // takes all its candidates (the same for every chunk of b)
+    uint32_t *st = state + NS * b;
+    const int want = (int)st[1];
+    if (want == 0) return;  // takes all its candidates (the same for every chunk of b)
     const Query q = query(b, Y, tau_y, count, offs, tail, tail_count, W);
     const int nc = q.F0 + q.nt;
     const int j0 = (c - chunk_start[b]) * CH, j1 = min(nc, j0 + CH);
-    const int shift = 24 - 8 * pass;
-    const uint32_t pmask = pass == 0 ? 0u : ~((1u << (32 - 8 * pass)) - 1u);
-    const uint32_t prefix = state[4 * b + 0];
-    for (int t = threadIdx.x; t < 256; t += TH) hist[t] = 0;
+    for (int t = threadIdx.x; t < NB; t += TH) hist[t] = 0;
     __syncthreads();
-    for (int j = j0 + threadIdx.x; j < j1; j += TH) {
-        const uint32_t u = key_of(q, j);
-        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
-    }
+    for (int j = j0 + threadIdx.x; j < j1; j += TH) atomicAdd(&hist[key_of(q, j) >> 20], 1);
     __syncthreads();
-    for (int t = threadIdx.x; t < 256; t += TH)
-        if (hist[t]) atomicAdd(ghist + b * 256 + t, hist[t]);
+    int *gh = ghist + (int64_t)b * NB;
+    for (int t = threadIdx.x; t < NB; t += TH)
+        if (hist[t]) atomicAdd(gh + t, hist[t]);
+    int *done = ghist + (int64_t)B * NB;
     if (!last_chunk_of_query(done, b, chunk_start[b + 1] - chunk_start[b])) return;
-    // the digit: thread t holds bin 255 - t, so an inclusive scan over the threads counts the keys
-    // at or above each digit; exactly one bin has above < remaining <= at or above
-    const int dg = 255 - (int)threadIdx.x;
-    const int h = atomicExch(ghist + b * 256 + dg, 0);  // read, and clear for the next pass
-    int pos, unused_p, total, unused_t;
-    block_excl_scan2(h, 0, pos, unused_p, total, unused_t);
-    const uint32_t above = (uint32_t)pos, upto = (uint32_t)(pos + h);
-    const bool chosen = h > 0 && above < remaining && upto >= remaining;
-    // fewer matching keys than wanted cannot happen (every pass counts the same keys); digit 0 then
-    const bool none = threadIdx.x == TH - 1 && (uint32_t)total < remaining;
-    if (chosen || none) {
-        const uint32_t cum = none ? (uint32_t)total : above;
-        state[4 * b + 0] = prefix | ((uint32_t)(none ? 0 : dg) << shift);
-        state[4 * b + 1] = remaining - cum;
-        state[4 * b + 2] += cum;
-    }
-}
-
-__global__ void __launch_bounds__(TH) k_ss_count(const float *__restrict__ Y, int tau_y, const int32_t *__restrict__ count,
-                                                 const int64_t *__restrict__ offs, const float *__restrict__ tail,
-                                                 const int32_t *__restrict__ tail_count, int W, int B,
-                                                 const int *__restrict__ chunk_start,
-                                                 const uint32_t *__restrict__ state, int *gtc, int *eqc, int *done)
-{
-    __shared__ int sgt, seq;
-    const int c = blockIdx.x;
-    if (c >= chunk_start[B]) return;
-    const int b = query_of_chunk(chunk_start, B, c);
-    const Query q = query(b, Y, tau_y, count, offs, tail, tail_count, W);
-    const int nc = q.F0 + q.nt;
-    const int j0 = (c - chunk_start[b]) * CH, j1 = min(nc, j0 + CH);
-    const uint32_t K = state[4 * b + 0];
-    const bool all = state[4 * b + 1] == 0u;  // at most k candidates: every one, whatever its key
-    if (threadIdx.x == 0) sgt = seq = 0;
-    __syncthreads();
-    int ng = 0, ne = 0;
-    for (int j = j0 + threadIdx.x; j < j1; j += TH) {
-        const uint32_t u = key_of(q, j);
-        ng += (all || u > K) ? 1 : 0;
-        ne += (!all && u == K) ? 1 : 0;
-    }
+    // the bucket of the want-th largest key: thread t owns buckets NB - 16 (t + 1) .. NB - 16 t - 1
+    constexpr int PER = NB / TH;
+    const int hi = NB - PER * (int)threadIdx.x;
+    int cnt = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        ng += __shfl_xor_sync(0xffffffffu, ng, o);
-        ne += __shfl_xor_sync(0xffffffffu, ne, o);
-    }
-    if ((threadIdx.x & 31) == 0) {
-        atomicAdd(&sgt, ng);
-        atomicAdd(&seq, ne);
+    for (int i = 1; i <= PER; i++) cnt += __ldcg(gh + hi - i);
+    int above, unused_p, total, unused_t;
+    block_excl_scan2(cnt, 0, above, unused_p, total, unused_t);
+    if (above < want && above + cnt >= want) {
+        for (int i = 1; i <= PER; i++) {
+            const int h = __ldcg(gh + hi - i);
+            if (above + h >= want) {
+                s_beta = hi - i;
+                s_above = above;
+                break;
+            }
+            above += h;
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        gtc[c] = sgt;
-        eqc[c] = seq;
-    }
-    const int c0 = chunk_start[b], c1 = chunk_start[b + 1];
-    if (!last_chunk_of_query(done, b, c1 - c0)) return;
-    // exclusive offsets of the query's chunk counts, in chunk (slot) order
-    int carry_g = 0, carry_e = 0;
-    for (int base = c0; base < c1; base += TH) {
-        const int cc = base + threadIdx.x;
-        const int g = cc < c1 ? __ldcg(gtc + cc) : 0, e = cc < c1 ? __ldcg(eqc + cc) : 0;
-        int pg, pe, tg, te;
-        block_excl_scan2(g, e, pg, pe, tg, te);
-        if (cc < c1) {
-            gtc[cc] = carry_g + pg;
-            eqc[cc] = carry_e + pe;
-        }
-        carry_g += tg;
-        carry_e += te;
+        st[0] = (uint32_t)s_beta;
+        st[2] = (uint32_t)s_above;
+        st[1] = (uint32_t)(want - s_above);
     }
 }
 
 __global__ void __launch_bounds__(TH) k_ss_write(const float *__restrict__ Y, int tau_y, const int32_t *__restrict__ count,
                                                  const int64_t *__restrict__ offs, const float *__restrict__ tail,
                                                  const int32_t *__restrict__ tail_count, int W, int B,
-                                                 const int *__restrict__ chunk_start,
-                                                 const uint32_t *__restrict__ state, const int *__restrict__ gtb,
-                                                 const int *__restrict__ eqb, int kcap,
-                                                 unsigned long long *__restrict__ sel)
+                                                 const int *__restrict__ chunk_start, uint32_t *state, int kcap,
+                                                 unsigned long long *__restrict__ sel,
+                                                 unsigned long long *__restrict__ stage)
 {
-    __shared__ int warp_tot[32];
     const int c = blockIdx.x;
     if (c >= chunk_start[B]) return;
     const int b = query_of_chunk(chunk_start, B, c);
+    uint32_t *st = state + NS * b;
     const Query q = query(b, Y, tau_y, count, offs, tail, tail_count, W);
     const int nc = q.F0 + q.nt;
     const int j0 = (c - chunk_start[b]) * CH, j1 = min(nc, j0 + CH);
-    const uint32_t K = state[4 * b + 0];
-    const int want_eq = (int)state[4 * b + 1], n_gt = (int)state[4 * b + 2];
-    const bool all = want_eq == 0;  // at most k candidates: every one, whatever its key
+    const bool all = st[1] == 0u;  // at most k candidates: every one, whatever its key
+    const uint32_t beta = st[0];
     unsigned long long *out = sel + (int64_t)b * kcap;
-    int carry_gt = gtb[c], carry_eq = eqb[c];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned long long *stg = stage + q.off + (int64_t)b * W;  // capacity S_b + W
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
     for (int base = j0; base < j1; base += TH) {
         const int j = base + threadIdx.x;
         uint32_t u = 0;
-        int gt = 0, eq = 0;
+        bool gt = false, eq = false;
         if (j < j1) {
             u = key_of(q, j);
-            gt = (all || u > K) ? 1 : 0;
-            eq = (!all && u == K) ? 1 : 0;
+            gt = all || (u >> 20) > beta;
+            eq = !all && (u >> 20) == beta;
         }
-        // block exclusive scans of gt and eq
-        int pos[2];
-        int tot[2];
-#pragma unroll
-        for (int k2 = 0; k2 < 2; k2++) {
-            const int v = k2 == 0 ? gt : eq;
-            const int inc = warp_incl_scan(v);
-            if (lane == 31) warp_tot[warp] = inc;
-            __syncthreads();
-            int before = 0, total = 0;
-            for (int w = 0; w < TH / 32; w++) {
-                before += w < warp ? warp_tot[w] : 0;
-                total += warp_tot[w];
-            }
-            pos[k2] = before + inc - v;
-            tot[k2] = total;
-            __syncthreads();
+        const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+        int pg = 0, pe = 0;
+        if (lane == 0) {
+            if (bg) pg = (int)atomicAdd(st + 4, (uint32_t)__popc(bg));
+            if (be) pe = (int)atomicAdd(st + 5, (uint32_t)__popc(be));
         }
+        pg = __shfl_sync(0xffffffffu, pg, 0);
+        pe = __shfl_sync(0xffffffffu, pe, 0);
         const unsigned long long key64 = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);
-        if (gt) out[carry_gt + pos[0]] = key64;
-        if (eq && carry_eq + pos[1] < want_eq) out[n_gt + carry_eq + pos[1]] = key64;
-        carry_gt += tot[0];
-        carry_eq += tot[1];
+        if (gt) out[pg + __popc(bg & lt)] = key64;
+        if (eq) stg[pe + __popc(be & lt)] = key64;
     }
 }
 
-__global__ void __launch_bounds__(SORT_TH) k_ss_sort(const unsigned long long *__restrict__ sel, int kcap,
-                                                      const uint32_t *__restrict__ state,
+// Per query (SORT_TH threads): the selection's keys of higher buckets plus the want largest keys of
+// bucket beta, sorted by key descending (score descending, slot ascending), then the output.
+// Dynamic shared memory: kpow2 + SCAP keys.
+__global__ void __launch_bounds__(SORT_TH) k_ss_final(const unsigned long long *__restrict__ sel, int kcap,
+                                                      const unsigned long long *__restrict__ stage,
+                                                      const uint32_t *__restrict__ state, int W,
                                                       const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
                                                       const int64_t *__restrict__ offs, int k, int kpow2,
                                                       int32_t *__restrict__ topk_idx, float *__restrict__ topk_score)
 {
     extern __shared__ unsigned long long sk[];
+    unsigned long long *ss = sk + kpow2;
+    __shared__ int hist[256];
+    __shared__ int s_dig, s_above, s_n;
     const int b = blockIdx.x;
-    const int nc = (int)state[4 * b + 3];
+    const uint32_t *st = state + NS * b;
+    const int nc = (int)st[3];
+    const int want = (int)st[1];
+    const int above = (int)st[2];
     const int nsel = nc < k ? nc : k;
     const int64_t off = offs[b], S = offs[b + 1] - off;
     int F0 = count[b];
     F0 = F0 < 0 ? 0 : (F0 > S ? (int)S : F0);
-    for (int t = threadIdx.x; t < kpow2; t += SORT_TH) sk[t] = t < nsel ? sel[(int64_t)b * kcap + t] : 0ull;
+    const unsigned long long *mine = sel + (int64_t)b * kcap;
+    const int nfirst = want == 0 ? nsel : above;  // keys already in the selection
+    for (int t = threadIdx.x; t < kpow2; t += SORT_TH) sk[t] = t < nfirst ? mine[t] : 0ull;
+    if (want > 0) {
+        const unsigned long long *stg = stage + off + (int64_t)b * W;
+        const int ns = (int)st[5];  // the keys of bucket beta (at least want)
+        if (ns <= SCAP) {
+            int np = 1;
+            while (np < ns) np <<= 1;
+            for (int t = threadIdx.x; t < np; t += SORT_TH) ss[t] = t < ns ? stg[t] : 0ull;
+            __syncthreads();
+            for (int size = 2; size <= np; size <<= 1) {
+                for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                    for (int t = threadIdx.x; t < np / 2; t += SORT_TH) {
+                        const int lo = 2 * t - (t & (stride - 1)), hi = lo + stride;
+                        const bool desc = (lo & size) == 0;
+                        const unsigned long long a = ss[lo], c = ss[hi];
+                        if ((a < c) == desc) {
+                            ss[lo] = c;
+                            ss[hi] = a;
+                        }
+                    }
+                    __syncthreads();
+                }
+            }
+            for (int t = threadIdx.x; t < want; t += SORT_TH) sk[above + t] = ss[t];
+        } else {
+            // a crowded bucket: radix select of the want-th largest key over the stage (the top 12
+            // bits are beta in every staged key; 52 bits remain: 8-bit digits, the last one 4 bits)
+            unsigned long long prefix = (unsigned long long)st[0] << 52, pmask = 0xFFFull << 52;
+            int remaining = want;
+            for (int pass = 0; pass < 7; pass++) {
+                const int shift = pass < 6 ? 44 - 8 * pass : 0;
+                const unsigned long long dmask = pass < 6 ? 255ull : 15ull;
+                for (int t = threadIdx.x; t < 256; t += SORT_TH) hist[t] = 0;
+                __syncthreads();
+                for (int i = threadIdx.x; i < ns; i += SORT_TH) {
+                    const unsigned long long v = stg[i];
+                    if ((v & pmask) == prefix) atomicAdd(&hist[(int)((v >> shift) & dmask)], 1);
+                }
+                __syncthreads();
+                if (threadIdx.x == 0) {
+                    int cum = 0, dg = 0;
+                    for (int d = 255; d >= 0; d--) {
+                        if (cum + hist[d] >= remaining) {
+                            dg = d;
+                            break;
+                        }
+                        cum += hist[d];
+                    }
+                    s_dig = dg;
+                    s_above = cum;
+                }
+                __syncthreads();
+                prefix |= (unsigned long long)s_dig << shift;
+                pmask |= dmask << shift;
+                remaining -= s_above;
+                __syncthreads();
+            }
+            // prefix is the want-th largest staged key: take every staged key at or above it
+            if (threadIdx.x == 0) s_n = 0;
+            __syncthreads();
+            for (int i = threadIdx.x; i < ns; i += SORT_TH) {
+                const unsigned long long v = stg[i];
+                if (v >= prefix) {
+                    const int pos = atomicAdd(&s_n, 1);
+                    if (pos < want) sk[above + pos] = v;
+                }
+            }
+        }
+    }
     __syncthreads();
     for (int size = 2; size <= kpow2; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {

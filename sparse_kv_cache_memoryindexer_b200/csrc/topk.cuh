@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(256) k_step_prep(const void *__restrict__ qs, 
 
 // Scores of the entries compressed during the window: one warp per (sequence, entry j < W);
 // y = sum_h w_h ReLU(scale_j q_h . k_j).  Keys [B][W][d_I] in the hot-key type, scales nullable.
+// Lane l holds key elements l * E .. l * E + E - 1 (E = d_I / 32); per head the lanes read their
+// part of the query row (one coalesced row per head) and a warp sum gives the dot product.
 __global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, const float *__restrict__ w,
                                                    int TQ, int dt, const void *__restrict__ winK,
                                                    const float *__restrict__ winsc,
@@ -347,21 +349,30 @@ __global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, c
     if (j >= n) return;
     const float sc = winsc ? winsc[(int64_t)b * W + j] : 1.f;
     if (winsc && lane == 0 && !(sc >= 0.f)) flag(ERRF_SCALE);
-    const size_t es = dt == DT_F32 ? 4 : 2;
-    const uint8_t *kr = (const uint8_t *)winK + ((size_t)b * W + j) * d_I * es;
-    float y = 0.f;
-    for (int h = lane; h < n_h; h += 32) {
-        const uint8_t *qr = (const uint8_t *)q + ((size_t)b * TQ * n_h + h) * d_I * es;  // query slot 0
-        float d = 0.f;
-        for (int e = 0; e < d_I; e++) {
-            const float qv = es == 4 ? ((const float *)qr)[e] : __bfloat162float(((const __nv_bfloat16 *)qr)[e]);
-            const float kv = es == 4 ? ((const float *)kr)[e] : __bfloat162float(((const __nv_bfloat16 *)kr)[e]);
-            d = fmaf(qv, kv, d);
-        }
-        y = fmaf(w[(size_t)b * TQ * n_h + h], fmaxf(sc * d, 0.f), y);
-    }
+    const int E = d_I >> 5;  // 1, 2 or 4
+    const bool f32 = dt == DT_F32;
+    const int64_t kb = ((int64_t)b * W + j) * d_I + (int64_t)lane * E;
+    float kv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
+    for (int e = 0; e < 4; e++)
+        if (e < E) kv[e] = f32 ? __ldg((const float *)winK + kb + e) : bf16_bits_to_float(__ldg((const unsigned short *)winK + kb + e));
+    const int64_t qb = (int64_t)b * TQ * n_h * d_I + (int64_t)lane * E;  // query slot 0
+    const float *wr = w + (int64_t)b * TQ * n_h;
+    float y = 0.f;
+    for (int h = 0; h < n_h; h++) {
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            if (e < E) {
+                const int64_t at = qb + (int64_t)h * d_I + e;
+                const float qv = f32 ? __ldg((const float *)q + at) : bf16_bits_to_float(__ldg((const unsigned short *)q + at));
+                d = fmaf(qv, kv[e], d);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        y = fmaf(__ldg(wr + h), fmaxf(sc * d, 0.f), y);
+    }
     if (lane == 0) tail[(int64_t)b * W + j] = y;
 }
 

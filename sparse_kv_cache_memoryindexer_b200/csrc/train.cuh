@@ -8,7 +8,7 @@
 //                     64 head dot products a_h, x = sum_h w_h ReLU(a_h), the loss and g = dl/dx / N;
 //                     then dw_h += g ReLU(a_h) and dq_h += (g w_h 1[a_h > 0] scale) K_s (a 64 x 128 x
 //                     128 product per tile), added to the sequence's gradients with atomics.
-//   k_train_dc        dc = dq W^IUQ (one thread per (layer, sequence, j)).
+//   k_train_dc        dc = dq W^IUQ (split over rows of W^IUQ, partial sums added with atomics).
 //   k_outer           g_W[l][m][n] = sum_b U[l][b][m] V[l][b][n]: the three weight gradients.
 #pragma once
 #include "common.cuh"
@@ -257,66 +257,104 @@ __global__ void __launch_bounds__(THREADS, 1) k_train_entries(const void *__rest
     }
 }
 
-// dc[l][b][j] = sum_o dq[l][b][o] W_iuq[l][o][j]: one CTA per (layer, 32 columns j); warp w sums the
-// rows o = w + 8 k for all B sequences at once (lane = column, so each W^IUQ row segment is one
-// coalesced read and W^IUQ is read once), then the 8 partial sums meet in shared memory.
+// dc[l][b][j] = sum_o dq[l][b][o] W_iuq[l][o][j] (W^IUQ read once, memory-bound): one CTA per
+// (layer, 512 columns, DC_OCH rows o); thread t takes columns 2t, 2t + 1 of the block (one 4- or
+// 8-byte load of W per row, coalesced), the CTA's dq rows of all sequences sit in shared memory, and
+// the partial sums over the CTA's rows are added to dc (zeroed before) with atomics.
 constexpr int DC_BMAX = 16;
+constexpr int DC_OCH = 512;
+constexpr int DC_COLS = 512;
 
 template <int DT>
 __global__ void __launch_bounds__(256) k_train_dc(const float *__restrict__ dq, const void *__restrict__ W_iuq, int L,
                                                   int B, int nq, int r, float *__restrict__ dc)
 {
-    __shared__ float part[8][DC_BMAX][32];
-    const int l = blockIdx.y, j = blockIdx.x * 32 + (threadIdx.x & 31), warp = threadIdx.x >> 5;
-    float acc[DC_BMAX];
+    __shared__ float sdq[DC_BMAX][DC_OCH];
+    const int l = blockIdx.z;
+    const int o0 = blockIdx.y * DC_OCH;
+    const int j = blockIdx.x * DC_COLS + 2 * threadIdx.x;
+    const int on = min(DC_OCH, nq - o0);
+    for (int i = threadIdx.x; i < B * DC_OCH; i += 256) {
+        const int bb = i / DC_OCH, o = i % DC_OCH;
+        sdq[bb][o] = o < on ? __ldg(dq + ((int64_t)l * B + bb) * nq + o0 + o) : 0.f;
+    }
+    __syncthreads();
+    if (j >= r) return;
+    float acc[DC_BMAX][2];
 #pragma unroll
-    for (int bb = 0; bb < DC_BMAX; bb++) acc[bb] = 0.f;
-    const float *dql = dq + (int64_t)l * B * nq;
-    if (j < r) {
-#pragma unroll 4
-        for (int o = warp; o < nq; o += 8) {
-            const float wv = load_elem<DT>(W_iuq, ((int64_t)l * nq + o) * r + j);
+    for (int bb = 0; bb < DC_BMAX; bb++) acc[bb][0] = acc[bb][1] = 0.f;
+    const int64_t wrow = (int64_t)l * nq + o0;
+#pragma unroll 8
+    for (int o = 0; o < on; o++) {
+        float w0, w1;
+        if (DT == DT_F32) {
+            const float2 v = __ldg((const float2 *)((const float *)W_iuq + (wrow + o) * r + j));
+            w0 = v.x;
+            w1 = v.y;
+        } else {
+            const uint32_t v = __ldg((const unsigned int *)((const unsigned short *)W_iuq + (wrow + o) * r + j));
+            w0 = bf16_bits_to_float((unsigned short)(v & 0xffffu));
+            w1 = bf16_bits_to_float((unsigned short)(v >> 16));
+        }
 #pragma unroll
-            for (int bb = 0; bb < DC_BMAX; bb++)
-                if (bb < B) acc[bb] = fmaf(__ldg(dql + (int64_t)bb * nq + o), wv, acc[bb]);
+        for (int bb = 0; bb < DC_BMAX; bb++) {
+            if (bb < B) {
+                const float d = sdq[bb][o];
+                acc[bb][0] = fmaf(d, w0, acc[bb][0]);
+                acc[bb][1] = fmaf(d, w1, acc[bb][1]);
+            }
         }
     }
 #pragma unroll
-    for (int bb = 0; bb < DC_BMAX; bb++) part[warp][bb][threadIdx.x & 31] = acc[bb];
-    __syncthreads();
-    for (int i = threadIdx.x; i < B * 32; i += 256) {
-        const int bb = i / 32, jj = i % 32;
-        if (blockIdx.x * 32 + jj < r) {
-            float sum = 0.f;
-#pragma unroll
-            for (int w8 = 0; w8 < 8; w8++) sum += part[w8][bb][jj];
-            dc[((int64_t)l * B + bb) * r + blockIdx.x * 32 + jj] = sum;
+    for (int bb = 0; bb < DC_BMAX; bb++) {
+        if (bb < B) {
+            float *dst = dc + ((int64_t)l * B + bb) * r + j;
+            if (acc[bb][0] != 0.f) atomicAdd(dst, acc[bb][0]);
+            if (acc[bb][1] != 0.f) atomicAdd(dst + 1, acc[bb][1]);
         }
     }
 }
 
-// out[l][m][n] = sum_b U[l][b][m] V[l][b][n] (U fp32, V of type VDT); 4 consecutive n per thread
-// (N is a multiple of 4), one 16-byte store each.
-template <int VDT>
+// out[l][m][n] = sum_b U[l][b][m] V[l][b][n] (U fp32, V of type VDT), written once (store-bound):
+// thread t of block (x, y, l) takes 4 consecutive n (one 16-byte store per row) and OUT_MR rows m,
+// with V[l][0..B)[n..n+3] kept in registers.  N is a multiple of 4, B at most DC_BMAX.
+constexpr int OUT_MR = 8;
+
+template <int VDT, int BM>  // BM: B rounded up to 8 or DC_BMAX (registers for V)
 __global__ void __launch_bounds__(256) k_outer(const float *__restrict__ U, const void *__restrict__ V, int L, int B,
                                                int M, int N, float *__restrict__ out)
 {
-    const int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    const int N4 = N / 4;
-    if (idx >= (int64_t)L * M * N4) return;
-    const int n = (int)(idx % N4) * 4;
-    const int64_t lm = idx / N4;
-    const int m = (int)(lm % M), l = (int)(lm / M);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int b = 0; b < B; b++) {
-        const float u = __ldg(U + ((int64_t)l * B + b) * M + m);
-        const int64_t vb = ((int64_t)l * B + b) * N + n;
-        acc.x = fmaf(u, load_elem<VDT>(V, vb), acc.x);
-        acc.y = fmaf(u, load_elem<VDT>(V, vb + 1), acc.y);
-        acc.z = fmaf(u, load_elem<VDT>(V, vb + 2), acc.z);
-        acc.w = fmaf(u, load_elem<VDT>(V, vb + 3), acc.w);
+    const int l = blockIdx.z;
+    const int n = (blockIdx.x * 256 + threadIdx.x) * 4;
+    const int m0 = blockIdx.y * OUT_MR;
+    if (n >= N) return;
+    float4 vb[BM];
+#pragma unroll
+    for (int bb = 0; bb < BM; bb++) {
+        vb[bb] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (bb < B) {
+            const int64_t at = ((int64_t)l * B + bb) * N + n;
+            vb[bb] = make_float4(load_elem<VDT>(V, at), load_elem<VDT>(V, at + 1), load_elem<VDT>(V, at + 2),
+                                 load_elem<VDT>(V, at + 3));
+        }
     }
-    *(float4 *)(out + ((int64_t)l * M + m) * N + n) = acc;
+#pragma unroll 2
+    for (int mi = 0; mi < OUT_MR; mi++) {
+        const int m = m0 + mi;
+        if (m >= M) break;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int bb = 0; bb < BM; bb++) {
+            if (bb < B) {
+                const float u = __ldg(U + ((int64_t)l * B + bb) * M + m);
+                acc.x = fmaf(u, vb[bb].x, acc.x);
+                acc.y = fmaf(u, vb[bb].y, acc.y);
+                acc.z = fmaf(u, vb[bb].z, acc.z);
+                acc.w = fmaf(u, vb[bb].w, acc.w);
+            }
+        }
+        *(float4 *)(out + ((int64_t)l * M + m) * N + n) = acc;
+    }
 }
 
 inline size_t entries_smem(void) { return sizeof(float) * ((size_t)DMAX * NHMAX + (size_t)TT * GP + (size_t)TT * (DMAX + 1)); }

@@ -1,12 +1,13 @@
 """Numpy models of the two Top-k selects' steps against a plain sort (key descending, ties to the
 smaller slot), on the CPU.
 
-Decode-step select (csrc/step_select.cuh): over chunks of 2,048 candidates, four radix passes of 8
-bits pick the k-th key K (per-chunk histograms added into the query's, the digit chosen by an
-exclusive scan from the top), then every chunk writes its candidates above K in slot order and the
-first want_eq candidates equal to K after them, and a final sort orders the k survivors.  With at
-most k candidates the select takes every candidate whatever its key, including a key that orders
-as 0.
+Decode-step select (csrc/step_select.cuh): over chunks of 2,048 candidates, a 12-bit histogram of
+the score keys gives the bucket of the k-th largest key; keys of higher buckets go to the selection
+and the bucket's keys to a stage, both in an arbitrary order (the model shuffles them), because every
+key carries its slot: key64 = (score key << 32) | ~slot orders by score, then smaller slot, and no
+two keys are equal.  The bucket's largest keys come from a sort (at most SCAP staged keys) or, for
+a crowded bucket, a 64-bit radix select over the stage; one sort orders the k keys.  With at most k
+candidates the select takes every candidate whatever its key, including a key that orders as 0.
 
 Batched select (csrc/topk.cuh, k_topk_select): a 12-bit histogram of all keys gives the bucket of
 the k-th key; keys of higher buckets are selected in slot order and the bucket's keys are staged
@@ -24,50 +25,57 @@ import pytest
 CH = 2048
 
 
-def select_model(u, k):
-    """u: uint32 order-preserving keys of one query's candidates (slot order); returns the selected
-    slots in output order."""
+def _find_bin(hist, want):
+    """Bin holding the want-th largest key (bins scanned from the top) and the keys above it."""
+    above = 0
+    for b in range(hist.size - 1, -1, -1):
+        if above + hist[b] >= want:
+            return b, above
+        above += int(hist[b])
+    raise AssertionError("want exceeds the histogram's total")
+
+
+def key64(u):
+    """(score key << 32) | ~slot: larger score first, then smaller slot; no two keys equal."""
+    slots = np.arange(u.size, dtype=np.uint64)
+    return (u.astype(np.uint64) << np.uint64(32)) | (~slots & np.uint64(0xFFFFFFFF))
+
+
+def select_model(u, k, scap=8192, seed=0):
+    """The decode-step select (k_ss_hist12, k_ss_write, k_ss_final): 12-bit bucket histogram, keys
+    of higher buckets and of the k-th key's bucket appended in an arbitrary order (shuffled here),
+    the bucket's want largest keys by a sort (at most scap keys) or a 64-bit radix select over the
+    stage, then one sort of the k keys; returns the selected slots in output order."""
+    rng = np.random.default_rng(seed)
     nc = u.size
-    remaining = k if nc > k else 0
-    n_gt = 0 if nc > k else nc
-    prefix = 0
-    chunks = [(j0, min(nc, j0 + CH)) for j0 in range(0, nc, CH)]
-    for ps in range(4):
-        if remaining == 0:
-            break
-        shift = 24 - 8 * ps
-        pmask = 0 if ps == 0 else (~((1 << (32 - 8 * ps)) - 1)) & 0xFFFFFFFF
-        g = np.zeros(256, dtype=np.int64)
-        for j0, j1 in chunks:
-            uu = u[j0:j1]
-            m = (uu & pmask) == prefix
-            g += np.bincount((uu[m] >> shift) & 255, minlength=256)
-        h = g[::-1]                       # thread t holds bin 255 - t
-        incl = np.cumsum(h)
-        above = incl - h
-        chosen = np.nonzero((h > 0) & (above < remaining) & (incl >= remaining))[0]
-        assert chosen.size == 1
-        t = int(chosen[0])
-        prefix |= (255 - t) << shift
-        remaining -= int(above[t])
-        n_gt += int(above[t])
-    K, want_eq = prefix, remaining
-    take_all = want_eq == 0               # nc <= k: every candidate, whatever its key
-    out = {}
-    cg = ce = 0
-    for j0, j1 in chunks:
-        for j in range(j0, j1):
-            if take_all or u[j] > K:
-                out[cg] = j
-                cg += 1
-            elif u[j] == K:
-                if ce < want_eq:
-                    out[n_gt + ce] = j
-                ce += 1
-    nsel = min(nc, k)
-    assert cg == n_gt and len(out) == nsel
-    slots = np.array([out[i] for i in range(nsel)], dtype=np.int64)
-    order = np.lexsort((slots, -u[slots].astype(np.int64)))
+    kk = key64(u)
+    if nc <= k:
+        slots = rng.permutation(nc)
+    else:
+        hist = np.bincount(u >> 20, minlength=4096)
+        beta, above = _find_bin(hist, k)
+        gt = rng.permutation(np.nonzero((u >> 20) > beta)[0])
+        staged = rng.permutation(np.nonzero((u >> 20) == beta)[0])
+        assert gt.size == above
+        want = k - above
+        if staged.size <= scap:
+            top = staged[np.lexsort((staged, -u[staged].astype(np.int64)))][:want]
+        else:
+            prefix, pmask, rem = np.uint64(beta) << np.uint64(52), np.uint64(0xFFF) << np.uint64(52), want
+            v = kk[staged]
+            for ps in range(7):
+                shift = np.uint64(44 - 8 * ps if ps < 6 else 0)
+                dmask = np.uint64(255 if ps < 6 else 15)
+                m = (v & pmask) == prefix
+                h = np.bincount(((v[m] >> shift) & dmask).astype(np.int64), minlength=256)
+                d, ab = _find_bin(h, rem)
+                prefix |= np.uint64(d) << shift
+                pmask |= dmask << shift
+                rem -= ab
+            top = staged[v >= prefix]
+            assert top.size == want
+        slots = np.concatenate([gt, top]).astype(np.int64)
+    order = np.argsort(kk[slots])[::-1]          # key descending: score descending, slot ascending
     return slots[order]
 
 
@@ -92,12 +100,13 @@ def keys(rng, kind, nc):
 
 @pytest.mark.parametrize("kind", ["random", "ties_every_digit", "ties_low_digits", "all_equal", "zeros_and_ones",
                                   "float"])
-def test_select_model_equals_plain_sort(kind):
+@pytest.mark.parametrize("scap", [8192, 16])
+def test_select_model_equals_plain_sort(kind, scap):
     rng = np.random.default_rng(zlib.crc32(kind.encode()))
     for nc in (0, 1, 5, 100, 2047, 2048, 2049, 5000, 9000):
         for k in (1, 7, 64, 2048, 4096):
             u = keys(rng, kind, nc)
-            assert np.array_equal(select_model(u, k), plain_sort(u, k)), (kind, nc, k)
+            assert np.array_equal(select_model(u, k, scap, seed=nc + k), plain_sort(u, k)), (kind, nc, k, scap)
 
 
 def test_few_candidates_keep_a_zero_key():
@@ -109,16 +118,6 @@ def test_few_candidates_keep_a_zero_key():
 
 
 # ------------------------------------------------------------------ batched select (csrc/topk.cuh)
-
-def _find_bin(hist, want):
-    """Bin holding the want-th largest key (bins scanned from the top) and the keys above it."""
-    above = 0
-    for b in range(hist.size - 1, -1, -1):
-        if above + hist[b] >= want:
-            return b, above
-        above += int(hist[b])
-    raise AssertionError("want exceeds the histogram's total")
-
 
 def batched_select_model(u, k, cap=4096):
     """The batched call's select (k_topk_select): a 12-bit histogram, the k-th key's bucket staged
