@@ -101,10 +101,10 @@ def load_peaks():
 # row once, so the traffic grows in proportion to the entries.  Reported only while the kernel sources
 # hash to the value the capture was taken on (null otherwise).
 SCORE_TRAFFIC = {
-    "fp8": {"bytes_per_entry_layer": 133.52, "capture": "ctx1m_fp8_b32 with B=4 (1,048,576 entries x 3 layers)"},
-    "bf16": {"bytes_per_entry_layer": 261.30, "capture": "ctx500k_bf16_b8 with B=2 (262,144 entries x 3 layers)"},
+    "fp8": {"bytes_per_entry_layer": 133.10, "capture": "ctx1m_fp8_b32 with B=4 (1,048,576 entries x 3 layers)"},
+    "bf16": {"bytes_per_entry_layer": 260.23, "capture": "ctx500k_bf16_b8 with B=2 (262,144 entries x 3 layers)"},
 }
-SCORE_TRAFFIC_SRC = "5df49d53b262df0f"
+SCORE_TRAFFIC_SRC = "75fc9bee86641ea6"
 
 
 def score_kernel_src_hash():

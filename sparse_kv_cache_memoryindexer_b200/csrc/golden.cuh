@@ -5,7 +5,8 @@
 // reaches p of the total); an entry is golden for token i if at least theta layers keep it; the
 // window's label set is the union over its tokens.
 //
-// k_golden_nucleus   one CTA per (sequence, token, layer) row.  The kept set is {key > K*} plus the
+// k_golden_nucleus   one CTA per (sequence, token, layer) row, the row staged in shared memory when
+//                    it fits (one read from DRAM).  The kept set is {key > K*} plus the
 //                    first n of {key == K*} in entry order, where key is the order-preserving
 //                    integer image of the logit.  One pass gives the total mass Z = sum e
 //                    (e = exp(z - max z), double) and, for a few depths D, the mass and count of
@@ -25,7 +26,7 @@ namespace lsa {
 
 namespace golden {
 
-constexpr int THREADS = 256;
+constexpr int THREADS = 1024;
 constexpr int CAND = 4096;       // candidates sorted in shared memory
 constexpr int ND = 6;            // depths below the maximum tried for the candidate set
 __device__ __forceinline__ float depth(int k) { return k == 0 ? 4.f : (k == 1 ? 8.f : (k == 2 ? 12.f : (k == 3 ? 16.f : (k == 4 ? 24.f : 40.f)))); }
@@ -54,11 +55,15 @@ __device__ __forceinline__ double block_sum(double v, double *red)
     return r;
 }
 
+// Dynamic shared memory: room for `stage_cap` logits; a row of at most stage_cap entries is copied
+// there first (read from DRAM once, eight independent loads in flight per thread) and every pass
+// reads it from shared memory; a longer row is read from global memory at every pass.
 __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restrict__ z, const int64_t *__restrict__ offs,
                                                             int64_t T, int B, int tau, int Lc, double p,
                                                             uint32_t *__restrict__ bits, int64_t W32,
-                                                            int32_t *__restrict__ nsize)
+                                                            int32_t *__restrict__ nsize, int stage_cap)
 {
+    extern __shared__ float srow[];
     __shared__ double hmass[256];
     __shared__ int hcnt[256];
     __shared__ unsigned long long cand[CAND];  // (key << 32) | ~entry
@@ -79,6 +84,23 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
         return;
     }
     const float *row = z + ((int64_t)i * Lc + l) * T + off;
+    if (S <= stage_cap) {
+        for (int64_t base = 0; base < S; base += 8 * THREADS) {
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const int64_t s = base + q * THREADS + threadIdx.x;
+                v[q] = s < S ? __ldg(row + s) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const int64_t s = base + q * THREADS + threadIdx.x;
+                if (s < S) srow[s] = v[q];
+            }
+        }
+        __syncthreads();
+        row = srow;
+    }
     float m = -INFINITY;
     for (int64_t s = threadIdx.x; s < S; s += THREADS) m = fmaxf(m, row[s]);
     m = block_max(m, fred);
@@ -150,24 +172,10 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
         }
         __syncthreads();
         const int nc = s_nc < CAND ? s_nc : CAND;
-        int np2 = 1;
+        int np2 = 64;
         while (np2 < nc) np2 <<= 1;
         for (int t = nc + threadIdx.x; t < np2; t += THREADS) cand[t] = 0ull;
-        __syncthreads();
-        for (int size = 2; size <= np2; size <<= 1) {  // bitonic sort, descending
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                for (int t = threadIdx.x; t < np2 / 2; t += THREADS) {
-                    const int lo = 2 * t - (t & (stride - 1)), hi = lo + stride;
-                    const bool desc = (lo & size) == 0;
-                    const unsigned long long a = cand[lo], c = cand[hi];
-                    if ((a < c) == desc) {
-                        cand[lo] = c;
-                        cand[hi] = a;
-                    }
-                }
-                __syncthreads();
-            }
-        }
+        block_sort_desc_u64(cand, np2);  // descending
         // cumulative mass in sorted order; the first position where it reaches the target
         double carry = 0.0;
         for (int base = 0; base < nc; base += THREADS) {

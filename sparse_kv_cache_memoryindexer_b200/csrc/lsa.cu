@@ -498,16 +498,7 @@ lsa_status lsa_fetch_gather_incremental(const int32_t *idx, const int32_t *count
     k_incr_map<<<sms * 4, 128, smem, st>>>(idx, count, seq_offsets, B, prev_idx, prev_count, prev_seq_offsets, map, miss,
                                            nmiss);
     LSA_TRY(launched("incremental fetch: lookup"));
-    if (row16 <= 32)
-        k_incr_copy<1><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
-                                                   row16, (uint8_t *)hot_kv);
-    else if (row16 <= 64)
-        k_incr_copy<2><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
-                                                   row16, (uint8_t *)hot_kv);
-    else
-        k_incr_copy<4><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
-                                                   row16, (uint8_t *)hot_kv);
-    LSA_TRY(launched("incremental fetch: device copy"));
+    // the host rows first: their launch takes its few SMs before the other stream's kernels fill the rest
     const uint8_t *src = (const uint8_t *)dpool;
     if (row16 <= 32)
         k_incr_fetch<1><<<GATHER_LINK_CTAS, link_threads<1>(), smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
@@ -519,7 +510,17 @@ lsa_status lsa_fetch_gather_incremental(const int32_t *idx, const int32_t *count
         k_incr_fetch<4><<<GATHER_LINK_CTAS, link_threads<4>(), smem, st>>>(idx, count, seq_offsets, B, miss, nmiss, src, row16,
                                                              (uint8_t *)hot_kv, host_rows_out);
     LSA_TRY(launched("incremental fetch: host rows"));
-    return ok();
+        if (row16 <= 32)
+        k_incr_copy<1><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
+                                                   row16, (uint8_t *)hot_kv);
+    else if (row16 <= 64)
+        k_incr_copy<2><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
+                                                   row16, (uint8_t *)hot_kv);
+    else
+        k_incr_copy<4><<<sms * 4, 256, smem, st>>>(count, seq_offsets, B, prev_seq_offsets, map, (const uint8_t *)prev_hot_kv,
+                                                   row16, (uint8_t *)hot_kv);
+    LSA_TRY(launched("incremental fetch: device copy"));
+return ok();
 }
 
 // ------------------------------------------------------------------------------ stage 5
@@ -570,12 +571,21 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
         default: return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: d_I must be 32, 64 or 128");
         }
     }
-    int kpow2 = 1;
+    int kpow2 = 64;  // the block sort works on at least 64 keys
     while (kpow2 < k) kpow2 <<= 1;
-    const size_t smem = sizeof(unsigned long long) * ((size_t)kpow2 + SEL_CAP);
+    // the queries' score keys stay in shared memory up to the capacity left beside the static part
+    int fcap = 0;
+    {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, k_topk_select) != cudaSuccess)
+            return fail(LSA_ERR_CUDA, "lsa_lightning_topk: %s", cudaGetErrorString(cudaGetLastError()));
+        const int64_t room = (int64_t)227 * 1024 - (int64_t)fa.sharedSizeBytes - (int64_t)topk_select_smem(kpow2, 0) - 1024;
+        fcap = room > 0 ? (int)(room / 4) : 0;
+    }
+    const size_t smem = topk_select_smem(kpow2, fcap);
     LSA_TRY(set_smem(k_topk_select, smem));
     k_topk_select<<<(unsigned)((int64_t)B * tau), SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, tau, k, kpow2,
-                                                                  topk_idx, topk_score);
+                                                                  fcap, topk_idx, topk_score);
     LSA_TRY(launched("top-k select"));
     return ok();
 }
@@ -681,8 +691,14 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     }
     if (W > 0) {
         const int64_t warps = (int64_t)B * W;
-        k_li_window<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(qw, ww, TQ, hdt, win_K, win_scale, win_count, B, W,
-                                                                 n_h, d_I, tail);
+        const unsigned gw = (unsigned)((warps + 7) / 8);
+#define LSA_LI_WINDOW(E, F)                                                                                       \
+    k_li_window<E, F><<<gw, 256, 0, st>>>(qw, ww, TQ, win_K, win_scale, win_count, B, W, n_h, tail)
+        const bool f32 = hdt == (int)DT_F32;
+        if (d_I == 32) { if (f32) LSA_LI_WINDOW(1, true); else LSA_LI_WINDOW(1, false); }
+        else if (d_I == 64) { if (f32) LSA_LI_WINDOW(2, true); else LSA_LI_WINDOW(2, false); }
+        else { if (f32) LSA_LI_WINDOW(4, true); else LSA_LI_WINDOW(4, false); }
+#undef LSA_LI_WINDOW
         LSA_TRY(launched("decode step: window entries"));
     }
     // the select, spread over chunks of candidates (see step_select.cuh)
@@ -696,12 +712,13 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
     const int64_t mc = step_max_chunks(B, total_S, W);
     const int32_t *tcnt = W > 0 ? win_count : nullptr;
-    stepsel::k_ss_setup<<<1, 1024, 0, st>>>(count, seq_offsets, tcnt, W, B, k, chunk_start, state, ghist);
+    const unsigned nclear = (unsigned)(((int64_t)B * (stepsel::NB + 1) + 4095) / 4096);
+    stepsel::k_ss_setup<<<1 + nclear, 1024, 0, st>>>(count, seq_offsets, tcnt, W, B, k, chunk_start, state, ghist);
     stepsel::k_ss_hist12<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
                                                                state, ghist);
     stepsel::k_ss_write<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
                                                               state, LSA_MAX_TOPK, sel, stage);
-    int kpow2 = 1;
+    int kpow2 = 64;  // the block sort works on at least 64 keys
     while (kpow2 < k) kpow2 <<= 1;
     const size_t smem = sizeof(unsigned long long) * ((size_t)kpow2 + stepsel::SCAP);
     LSA_TRY(set_smem(stepsel::k_ss_final, smem));
@@ -739,8 +756,18 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t) * (size_t)tau * Lc * W32, st);
     if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_golden_labels: %s", cudaGetErrorString(e));
     uint32_t *bits = (uint32_t *)workspace;
-    golden::k_golden_nucleus<<<(unsigned)((int64_t)B * tau * Lc), golden::THREADS, 0, st>>>(
-        z, seq_offsets, total_S, B, tau, Lc, p, bits, W32, nsize_out);
+    int stage_cap = 0;
+    {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, golden::k_golden_nucleus) != cudaSuccess)
+            return fail(LSA_ERR_CUDA, "lsa_golden_labels: %s", cudaGetErrorString(cudaGetLastError()));
+        const int64_t room = ((int64_t)227 * 1024 - (int64_t)fa.sharedSizeBytes - 1024) / 4;
+        stage_cap = (int)std::min<int64_t>(room > 0 ? room : 0, total_S);
+    }
+    const size_t gsmem = sizeof(float) * (size_t)stage_cap;
+    LSA_TRY(set_smem(golden::k_golden_nucleus, gsmem));
+    golden::k_golden_nucleus<<<(unsigned)((int64_t)B * tau * Lc), golden::THREADS, gsmem, st>>>(
+        z, seq_offsets, total_S, B, tau, Lc, p, bits, W32, nsize_out, stage_cap);
     LSA_TRY(launched("golden labels: nucleus"));
     golden::k_golden_vote<<<(unsigned)((W32 + golden::THREADS / 32 - 1) / (golden::THREADS / 32)), golden::THREADS, 0,
                             st>>>(bits, W32, total_S, tau, Lc, theta, label_out);

@@ -4,7 +4,8 @@
 // reported as entries S_b + j) are cut into chunks of CH with one CTA per chunk.  A candidate's
 // 64-bit key is (order-preserving score key << 32) | ~slot: larger score first, then smaller slot,
 // and no two keys are equal.
-//   k_ss_setup   per query: candidates, chunk ranges (a prefix over the sequences), state
+//   k_ss_setup   per query: candidates, chunk ranges (a prefix over the sequences), state; its other
+//                CTAs clear the histograms
 //   k_ss_hist12  per chunk: histogram of the top 12 bits of the score keys, added to the query's
 //                histogram in global memory; the query's last chunk to finish picks the bucket
 //                beta holding the k-th largest key (the keys above beta are all selected)
@@ -66,13 +67,17 @@ __global__ void __launch_bounds__(1024) k_ss_setup(const int32_t *__restrict__ c
                                                    int *__restrict__ chunk_start, uint32_t *__restrict__ state,
                                                    int *__restrict__ ghist)
 {
+    if (blockIdx.x > 0) {  // CTAs 1.. clear the histograms and finish counters, 4096 words each
+        const int64_t i0 = (int64_t)(blockIdx.x - 1) * 4096, n = (int64_t)B * (NB + 1);
+        for (int64_t i = i0 + threadIdx.x; i < n && i < i0 + 4096; i += blockDim.x) ghist[i] = 0;
+        return;
+    }
     __shared__ int wt[32];
     __shared__ int carry;
     if (threadIdx.x == 0) {
         carry = 0;
         chunk_start[0] = 0;
     }
-    for (int i = threadIdx.x; i < B * (NB + 1); i += blockDim.x) ghist[i] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int base = 0; base < B; base += blockDim.x) {
@@ -292,24 +297,10 @@ __global__ void __launch_bounds__(SORT_TH) k_ss_final(const unsigned long long *
         const unsigned long long *stg = stage + off + (int64_t)b * W;
         const int ns = (int)st[5];  // the keys of bucket beta (at least want)
         if (ns <= SCAP) {
-            int np = 1;
+            int np = 64;
             while (np < ns) np <<= 1;
             for (int t = threadIdx.x; t < np; t += SORT_TH) ss[t] = t < ns ? stg[t] : 0ull;
-            __syncthreads();
-            for (int size = 2; size <= np; size <<= 1) {
-                for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                    for (int t = threadIdx.x; t < np / 2; t += SORT_TH) {
-                        const int lo = 2 * t - (t & (stride - 1)), hi = lo + stride;
-                        const bool desc = (lo & size) == 0;
-                        const unsigned long long a = ss[lo], c = ss[hi];
-                        if ((a < c) == desc) {
-                            ss[lo] = c;
-                            ss[hi] = a;
-                        }
-                    }
-                    __syncthreads();
-                }
-            }
+            block_sort_desc_u64(ss, np);
             for (int t = threadIdx.x; t < want; t += SORT_TH) sk[above + t] = ss[t];
         } else {
             // a crowded bucket: radix select of the want-th largest key over the stage (the top 12
@@ -356,21 +347,7 @@ __global__ void __launch_bounds__(SORT_TH) k_ss_final(const unsigned long long *
             }
         }
     }
-    __syncthreads();
-    for (int size = 2; size <= kpow2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = threadIdx.x; t < kpow2 / 2; t += SORT_TH) {
-                const int lo = 2 * t - (t & (stride - 1)), hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const unsigned long long a = sk[lo], c = sk[hi];
-                if ((a < c) == desc) {
-                    sk[lo] = c;
-                    sk[hi] = a;
-                }
-            }
-            __syncthreads();
-        }
-    }
+    block_sort_desc_u64(sk, kpow2);
     for (int r = threadIdx.x; r < k; r += SORT_TH) {
         const int64_t o = (int64_t)b * k + r;
         if (r < nsel) {

@@ -2,10 +2,9 @@
 // (blog review "FlashMemory-DeepSeek-V4", sections 2.2 and 3.2).
 //
 // Scores of sequence b, query i, fetched slot j live at Y[tau*off_b + i*S_b + j] (fp32).
-// Selection: per query, a radix select on order-preserving 32-bit keys finds the k-th largest
-// score (12 + 10 + 10 bits, two reads of the scores); the survivors (all larger keys, plus the
-// first equal keys in slot order, i.e. smallest entry index) are sorted by (score desc, entry asc)
-// with a bitonic sort in shared memory.
+// Selection: per query, the k-th largest score is found on order-preserving keys held in shared
+// memory (a 12-bit bucket histogram, then the bucket's keys); the survivors are sorted by (score
+// desc, entry asc) with a bitonic sort in shared memory (k_topk_select).
 #pragma once
 #include "common.cuh"
 
@@ -59,7 +58,7 @@ __global__ void __launch_bounds__(TILE) k_li_score_simt(const void *__restrict__
     }
 }
 
-constexpr int SEL_THREADS = 512;
+constexpr int SEL_THREADS = 1024;
 
 // Block-wide exclusive scan of one int per thread (SEL_THREADS threads); returns the
 // exclusive prefix and writes the block total to *total.  Ends with a barrier.
@@ -81,11 +80,11 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total)
     return r;
 }
 
-// Order-preserving keys of a query's candidates are split as 12 + 10 + 10 bits.  SEL_CAP keys of the
-// k-th key's 12-bit bucket are staged in shared memory, so that the two finer passes read shared
-// memory instead of the scores again.
+// The k-th largest key of a query is found from a 12-bit histogram of the order-preserving score
+// keys (its bucket beta) and then inside the bucket; a candidate's 64-bit key (score key << 32) |
+// ~slot orders by score and then by smaller slot, and no two are equal.
 constexpr int SEL_BINS = 4096;
-constexpr int SEL_CAP = 4096;
+constexpr int SEL_CAP = 4096;      // bucket keys sorted in shared memory
 
 // The bin holding the `want`-th largest key of a histogram of NB bins (thread t owns NB / SEL_THREADS
 // consecutive bins, highest first): *bin_out, and *above_out = keys in higher bins.  want >= 1 and
@@ -115,26 +114,34 @@ __device__ __forceinline__ void sel_find_bin(const unsigned int *hist, int want,
     __syncthreads();
 }
 
-// One block per (sequence, query).  kpow2 = next power of two >= k; dynamic shared memory:
-// kpow2 + SEL_CAP 8-byte keys.  When the candidates exceed k: a 12-bit histogram of the keys
-// (one read of the scores) gives the bucket of the k-th largest key; a second read writes every key
-// of a higher bucket to the selection in slot order and stages the bucket's own keys (slot order)
-// in shared memory; two 10-bit passes over those find the k-th key K, and the staged keys above K,
-// then the first keys equal to K in slot order (smallest entry index), complete the selection.  A
-// bucket of more than SEL_CAP keys takes three 8-bit passes over the scores instead.  The k keys
-// are sorted by (score desc, slot asc) with a bitonic sort in shared memory.
+// Shared memory of k_topk_select for kpow2 and a key capacity fcap (dynamic part).
+__host__ __device__ inline size_t topk_select_smem(int kpow2, int fcap)
+{
+    return sizeof(unsigned long long) * ((size_t)kpow2 + SEL_CAP) + sizeof(uint32_t) * (size_t)fcap;
+}
+
+// One block per (sequence, query).  kpow2 = next power of two >= max(k, 64).  Dynamic shared memory:
+// kpow2 selection keys, SEL_CAP staged keys, then the query's score keys when it has at most fcap
+// candidates (read from the scores once, eight independent loads in flight per thread; a larger
+// query reads its scores from global memory at every pass).  With more than k candidates: a 12-bit
+// histogram gives the bucket beta of the k-th largest key; the keys of higher buckets are appended
+// to the selection and the bucket's keys to the stage (any order: the keys carry their slots); the
+// stage sorted by key gives the bucket's largest keys.  A bucket of more than SEL_CAP keys is
+// resolved by three more radix passes (8/8/4 bits) and an ordered pass (the first keys equal to
+// the k-th in slot order).  The k keys are sorted by (score desc, slot asc).
 __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__restrict__ Y,
                                                              const int32_t *__restrict__ idx,
                                                              const int32_t *__restrict__ count,
                                                              const int64_t *__restrict__ offs, int tau, int k,
-                                                             int kpow2, int32_t *__restrict__ topk_idx,
+                                                             int kpow2, int fcap, int32_t *__restrict__ topk_idx,
                                                              float *__restrict__ topk_score)
 {
-    extern __shared__ unsigned long long sel[];  // [kpow2] (key << 32) | ~slot, then [SEL_CAP] staged keys
+    extern __shared__ unsigned long long sel[];  // [kpow2] selection, [SEL_CAP] stage, then keys
     unsigned long long *stage = sel + kpow2;
+    uint32_t *keys = (uint32_t *)(stage + SEL_CAP);
     __shared__ unsigned int hist[SEL_BINS];
     __shared__ int warp_tot[32];
-    __shared__ int tot_a, tot_b, s_bin, s_above;
+    __shared__ int tot_a, tot_b, s_bin, s_above, s_ngt, s_nst;
 
     const int b = blockIdx.x / tau, i = blockIdx.x % tau;
     const int64_t off = offs[b], S = offs[b + 1] - offs[b];
@@ -142,93 +149,74 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
     F = F < 0 ? 0 : (F > S ? (int)S : F);
     const float *row = Y + (int64_t)tau * off + (int64_t)i * S;
     const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    const bool resident = F <= fcap;
     auto key64 = [](uint32_t u, int j) { return ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j); };
+    auto key_at = [&](int j) -> uint32_t { return resident ? keys[j] : float_to_ordered(__ldg(row + j)); };
 
+    if (resident) {
+        for (int base = 0; base < F; base += 8 * SEL_THREADS) {
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const int j = base + q * SEL_THREADS + threadIdx.x;
+                v[q] = j < F ? __ldg(row + j) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const int j = base + q * SEL_THREADS + threadIdx.x;
+                if (j < F) keys[j] = float_to_ordered(v[q]);
+            }
+        }
+    }
     for (int t = threadIdx.x; t < kpow2; t += SEL_THREADS) sel[t] = 0ull;
     __syncthreads();
 
     if (F <= k) {
-        for (int j = threadIdx.x; j < F; j += SEL_THREADS) sel[j] = key64(float_to_ordered(__ldg(row + j)), j);
+        for (int j = threadIdx.x; j < F; j += SEL_THREADS) sel[j] = key64(key_at(j), j);
     } else {
-        // read 1: 12-bit histogram (lanes with the same bucket add once)
         for (int t = threadIdx.x; t < SEL_BINS; t += SEL_THREADS) hist[t] = 0;
+        if (threadIdx.x == 0) s_ngt = s_nst = 0;
         __syncthreads();
-        for (int base = 0; base < F; base += SEL_THREADS) {
-            const int j = base + threadIdx.x;
-            const uint32_t bk = j < F ? float_to_ordered(__ldg(row + j)) >> 20 : 0xFFFFFFFFu;
-            const unsigned peers = __match_any_sync(0xffffffffu, bk);
-            if (bk != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bk], (unsigned)__popc(peers));
-        }
+        for (int j = threadIdx.x; j < F; j += SEL_THREADS) atomicAdd(&hist[key_at(j) >> 20], 1u);
         __syncthreads();
         sel_find_bin<SEL_BINS>(hist, k, warp_tot, &tot_a, &s_bin, &s_above);
         const uint32_t beta = (uint32_t)s_bin;
         const int above = s_above;              // keys of higher buckets: all selected
         const int nbeta = (int)hist[beta];
         const bool staged = nbeta <= SEL_CAP;
-        __syncthreads();
-        // read 2: higher buckets to the selection, the k-th key's bucket to the stage (slot order)
-        int carry_gt = 0, carry_eq = 0;
+        const int want = k - above;             // keys still to take from bucket beta (>= 1)
+        // higher buckets to the selection, bucket beta to the stage (appends in any order)
         for (int base = 0; base < F; base += SEL_THREADS) {
             const int j = base + threadIdx.x;
             uint32_t u = 0;
-            int gt = 0, eq = 0;
+            bool gt = false, eq = false;
             if (j < F) {
-                u = float_to_ordered(__ldg(row + j));
+                u = key_at(j);
                 gt = (u >> 20) > beta;
-                eq = (u >> 20) == beta;
+                eq = staged && (u >> 20) == beta;
             }
-            const int pg = block_excl_scan(gt, warp_tot, &tot_a) + carry_gt;
-            const int pe = block_excl_scan(eq, warp_tot, &tot_b) + carry_eq;
-            if (gt) sel[pg] = key64(u, j);
-            if (eq && staged) stage[pe] = key64(u, j);
-            carry_gt += tot_a;
-            carry_eq += tot_b;
-            __syncthreads();
+            const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+            int pg = 0, pe = 0;
+            if (lane == 0) {
+                if (bg) pg = atomicAdd(&s_ngt, __popc(bg));
+                if (be) pe = atomicAdd(&s_nst, __popc(be));
+            }
+            pg = __shfl_sync(0xffffffffu, pg, 0);
+            pe = __shfl_sync(0xffffffffu, pe, 0);
+            if (gt) sel[pg + __popc(bg & lt)] = key64(u, j);
+            if (eq) stage[pe + __popc(be & lt)] = key64(u, j);
         }
-        const int want = k - above;             // keys still to take from bucket beta (>= 1)
+        __syncthreads();
         if (staged) {
-            // two 10-bit passes over the staged keys
-            uint32_t prefix = beta << 20, pmask = 0xFFF00000u;
-            int remaining = want;
-#pragma unroll 1
-            for (int pass = 0; pass < 2; pass++) {
-                const int shift = 10 - 10 * pass;
-                for (int t = threadIdx.x; t < 1024; t += SEL_THREADS) hist[t] = 0;
-                __syncthreads();
-                for (int q = threadIdx.x; q < nbeta; q += SEL_THREADS) {
-                    const uint32_t u = (uint32_t)(stage[q] >> 32);
-                    if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 1023u], 1u);
-                }
-                __syncthreads();
-                sel_find_bin<1024>(hist, remaining, warp_tot, &tot_a, &s_bin, &s_above);
-                prefix |= (uint32_t)s_bin << shift;
-                remaining -= s_above;
-                pmask |= 1023u << shift;
-                __syncthreads();
-            }
-            // prefix is the k-th largest key; take the staged keys above it, then the first
-            // `remaining` equal to it in slot order
-            int cg = 0, ce = 0;
-            for (int base = 0; base < nbeta; base += SEL_THREADS) {
-                const int q = base + threadIdx.x;
-                unsigned long long v = 0ull;
-                int gt = 0, eq = 0;
-                if (q < nbeta) {
-                    v = stage[q];
-                    const uint32_t u = (uint32_t)(v >> 32);
-                    gt = u > prefix;
-                    eq = u == prefix;
-                }
-                const int pg = block_excl_scan(gt, warp_tot, &tot_a) + cg;
-                const int pe = block_excl_scan(eq, warp_tot, &tot_b) + ce;
-                if (gt) sel[above + pg] = v;
-                if (eq && pe < remaining) sel[k - remaining + pe] = v;
-                cg += tot_a;
-                ce += tot_b;
-                __syncthreads();
-            }
+            int np = 64;
+            while (np < nbeta) np <<= 1;
+            for (int t = nbeta + threadIdx.x; t < np; t += SEL_THREADS) stage[t] = 0ull;
+            block_sort_desc_u64(stage, np);
+            for (int t = threadIdx.x; t < want; t += SEL_THREADS) sel[above + t] = stage[t];
         } else {
-            // a crowded bucket: three 8-bit passes over the scores for the low 20 bits
+            // a crowded bucket: three radix passes (8/8/4 bits) for the k-th key K, then the
+            // bucket's keys above K and the first keys equal to K in slot order
             uint32_t prefix = beta << 20, pmask = 0xFFF00000u;
             int remaining = want;
 #pragma unroll 1
@@ -238,7 +226,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
                 for (int t = threadIdx.x; t < 1024; t += SEL_THREADS) hist[t] = 0;
                 __syncthreads();
                 for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
-                    const uint32_t u = float_to_ordered(__ldg(row + j));
+                    const uint32_t u = key_at(j);
                     if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & bins], 1u);
                 }
                 __syncthreads();
@@ -254,7 +242,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
                 uint32_t u = 0;
                 int gt = 0, eq = 0;
                 if (j < F) {
-                    u = float_to_ordered(__ldg(row + j));
+                    u = key_at(j);
                     gt = (u >> 20) == beta && u > prefix;
                     eq = u == prefix;
                 }
@@ -268,23 +256,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
             }
         }
     }
-    __syncthreads();
-    // bitonic sort, descending
-    for (int size = 2; size <= kpow2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = threadIdx.x; t < kpow2 / 2; t += SEL_THREADS) {
-                const int lo = 2 * t - (t & (stride - 1));
-                const int hi = lo + stride;
-                const bool desc = ((lo & size) == 0);
-                const unsigned long long a = sel[lo], c = sel[hi];
-                if ((a < c) == desc) {
-                    sel[lo] = c;
-                    sel[hi] = a;
-                }
-            }
-            __syncthreads();
-        }
-    }
+    block_sort_desc_u64(sel, kpow2);
     const int nsel = F < k ? F : k;
     const int64_t o0 = ((int64_t)b * tau + i) * k;
     for (int r = threadIdx.x; r < k; r += SEL_THREADS) {
@@ -329,14 +301,17 @@ __global__ void __launch_bounds__(256) k_step_prep(const void *__restrict__ qs, 
 
 // Scores of the entries compressed during the window: one warp per (sequence, entry j < W);
 // y = sum_h w_h ReLU(scale_j q_h . k_j).  Keys [B][W][d_I] in the hot-key type, scales nullable.
-// Lane l holds key elements l * E .. l * E + E - 1 (E = d_I / 32); per head the lanes read their
-// part of the query row (one coalesced row per head) and a warp sum gives the dot product.
-__global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, const float *__restrict__ w,
-                                                   int TQ, int dt, const void *__restrict__ winK,
-                                                   const float *__restrict__ winsc,
+// Lane l holds key elements l E .. l E + E - 1 (E = d_I / 32).  Heads go in groups of 16: the
+// lanes' query parts of the 16 heads are loaded first (one coalesced row per head), then the 16
+// partial dot products are summed over the warp by a reduce-scatter (16 shuffles: after it, lanes
+// l and l ^ 1 hold the whole dot product of one head of the group).
+template <int E, bool F32>
+__global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, const float *__restrict__ w, int TQ,
+                                                   const void *__restrict__ winK, const float *__restrict__ winsc,
                                                    const int32_t *__restrict__ win_count, int B, int W, int n_h,
-                                                   int d_I, float *__restrict__ tail)
+                                                   float *__restrict__ tail)
 {
+    constexpr int D = 32 * E;
     const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (gw >= (int64_t)B * W) return;
@@ -349,29 +324,48 @@ __global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, c
     if (j >= n) return;
     const float sc = winsc ? winsc[(int64_t)b * W + j] : 1.f;
     if (winsc && lane == 0 && !(sc >= 0.f)) flag(ERRF_SCALE);
-    const int E = d_I >> 5;  // 1, 2 or 4
-    const bool f32 = dt == DT_F32;
-    const int64_t kb = ((int64_t)b * W + j) * d_I + (int64_t)lane * E;
-    float kv[4] = {0.f, 0.f, 0.f, 0.f};
+    auto ld = [&](const void *base, int64_t at) {
+        return F32 ? __ldg((const float *)base + at) : bf16_bits_to_float(__ldg((const unsigned short *)base + at));
+    };
+    float kv[E];
 #pragma unroll
-    for (int e = 0; e < 4; e++)
-        if (e < E) kv[e] = f32 ? __ldg((const float *)winK + kb + e) : bf16_bits_to_float(__ldg((const unsigned short *)winK + kb + e));
-    const int64_t qb = (int64_t)b * TQ * n_h * d_I + (int64_t)lane * E;  // query slot 0
+    for (int e = 0; e < E; e++) kv[e] = ld(winK, ((int64_t)b * W + j) * D + lane * E + e);
+    const int64_t qb = (int64_t)b * TQ * n_h * D + (int64_t)lane * E;  // query slot 0
     const float *wr = w + (int64_t)b * TQ * n_h;
+    // the head of the group whose dot product this lane holds after the reduce-scatter
+    const int hl = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
     float y = 0.f;
-    for (int h = 0; h < n_h; h++) {
-        float d = 0.f;
+    for (int h0 = 0; h0 < n_h; h0 += 16) {
+        float qv[16][E];
 #pragma unroll
-        for (int e = 0; e < 4; e++) {
-            if (e < E) {
-                const int64_t at = qb + (int64_t)h * d_I + e;
-                const float qv = f32 ? __ldg((const float *)q + at) : bf16_bits_to_float(__ldg((const unsigned short *)q + at));
-                d = fmaf(qv, kv[e], d);
+        for (int g = 0; g < 16; g++)
+#pragma unroll
+            for (int e = 0; e < E; e++) qv[g][e] = h0 + g < n_h ? ld(q, qb + (int64_t)(h0 + g) * D + e) : 0.f;
+        float v[16];
+#pragma unroll
+        for (int g = 0; g < 16; g++) {
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; e++) d = fmaf(qv[g][e], kv[e], d);
+            v[g] = d;
+        }
+        // reduce-scatter: 16 -> 8 -> 4 -> 2 -> 1 values per lane, then the lane pair
+#pragma unroll
+        for (int half = 8, m = 16; half >= 1; half >>= 1, m >>= 1) {
+            const bool upper = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < half; i++) {
+                const float send = upper ? v[i] : v[half + i];
+                const float keep = upper ? v[half + i] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
             }
         }
+        const float dot = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+        const int h = h0 + hl;
+        float c = ((lane & 1) == 0 && h < n_h) ? __ldg(wr + h) * fmaxf(sc * dot, 0.f) : 0.f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        y = fmaf(__ldg(wr + h), fmaxf(sc * d, 0.f), y);
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        y += c;
     }
     if (lane == 0) tail[(int64_t)b * W + j] = y;
 }

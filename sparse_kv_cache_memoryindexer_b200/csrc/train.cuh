@@ -259,10 +259,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_train_entries(const void *__rest
 
 // dc[l][b][j] = sum_o dq[l][b][o] W_iuq[l][o][j] (W^IUQ read once, memory-bound): one CTA per
 // (layer, 512 columns, DC_OCH rows o); thread t takes columns 2t, 2t + 1 of the block (one 4- or
-// 8-byte load of W per row, coalesced), the CTA's dq rows of all sequences sit in shared memory, and
-// the partial sums over the CTA's rows are added to dc (zeroed before) with atomics.
+// 8-byte load of W per row, coalesced, 16 rows in flight), the CTA's dq rows of all sequences sit in
+// shared memory, and the partial sums over the CTA's rows are added to dc (zeroed before) with
+// atomics.
 constexpr int DC_BMAX = 16;
-constexpr int DC_OCH = 512;
+constexpr int DC_OCH = 128;
 constexpr int DC_COLS = 512;
 
 template <int DT>
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(256) k_train_dc(const float *__restrict__ dq, 
 #pragma unroll
     for (int bb = 0; bb < DC_BMAX; bb++) acc[bb][0] = acc[bb][1] = 0.f;
     const int64_t wrow = (int64_t)l * nq + o0;
-#pragma unroll 8
+#pragma unroll 16
     for (int o = 0; o < on; o++) {
         float w0, w1;
         if (DT == DT_F32) {
@@ -324,9 +325,15 @@ template <int VDT, int BM>  // BM: B rounded up to 8 or DC_BMAX (registers for V
 __global__ void __launch_bounds__(256) k_outer(const float *__restrict__ U, const void *__restrict__ V, int L, int B,
                                                int M, int N, float *__restrict__ out)
 {
+    __shared__ float su[BM][OUT_MR];
     const int l = blockIdx.z;
     const int n = (blockIdx.x * 256 + threadIdx.x) * 4;
     const int m0 = blockIdx.y * OUT_MR;
+    if (threadIdx.x < BM * OUT_MR) {  // the CTA's rows of U for every sequence
+        const int bb = threadIdx.x / OUT_MR, mi = threadIdx.x % OUT_MR;
+        su[bb][mi] = (bb < B && m0 + mi < M) ? __ldg(U + ((int64_t)l * B + bb) * M + m0 + mi) : 0.f;
+    }
+    __syncthreads();
     if (n >= N) return;
     float4 vb[BM];
 #pragma unroll
@@ -346,7 +353,7 @@ __global__ void __launch_bounds__(256) k_outer(const float *__restrict__ U, cons
 #pragma unroll
         for (int bb = 0; bb < BM; bb++) {
             if (bb < B) {
-                const float u = __ldg(U + ((int64_t)l * B + bb) * M + m);
+                const float u = su[bb][mi];
                 acc.x = fmaf(u, vb[bb].x, acc.x);
                 acc.y = fmaf(u, vb[bb].y, acc.y);
                 acc.z = fmaf(u, vb[bb].z, acc.z);

@@ -57,7 +57,9 @@ class IndexerPath:
         # the incremental row fetch of run(prev=...): workspace and the count of rows that crossed the link
         self.ws_incr = ws(lsa.lsa_fetch_incremental_workspace_size(B, T)) if incremental else None
         self.host_rows = torch.zeros(1, dtype=torch.int32, device=dev) if incremental else None
-        self._link = torch.cuda.Stream(device=dev)  # the host-link row gather of run()
+        # the host-link row gather of run(), at a higher priority than the caller's stream so that its
+        # few fat CTAs are placed before the Top-k's persistent CTAs fill the SMs
+        self._link = torch.cuda.Stream(device=dev, priority=-1)
 
     def project(self, h, W_dq, W_iuq, W_w, stream=None):
         lsa.lsa_project(h, W_dq, W_iuq, W_w, self.q, self.w, self.ws_proj, stream=stream)

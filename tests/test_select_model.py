@@ -10,9 +10,9 @@ a crowded bucket, a 64-bit radix select over the stage; one sort orders the k ke
 candidates the select takes every candidate whatever its key, including a key that orders as 0.
 
 Batched select (csrc/topk.cuh, k_topk_select): a 12-bit histogram of all keys gives the bucket of
-the k-th key; keys of higher buckets are selected in slot order and the bucket's keys are staged
-(at most SEL_CAP of them) for two 10-bit passes; a crowded bucket takes three 8/8/4-bit passes over
-all keys instead.
+the k-th key; keys of higher buckets and the bucket's keys (at most SEL_CAP of them) are appended in
+any order, and the stage sorted by 64-bit key gives the bucket's largest keys; a crowded bucket takes
+three 8/8/4-bit passes over all keys and an ordered pass instead.
 
 The cases cover heavy ties in every digit, all-equal keys, keys of 0, k at and above the candidate
 count, and empty queries.
@@ -119,40 +119,42 @@ def test_few_candidates_keep_a_zero_key():
 
 # ------------------------------------------------------------------ batched select (csrc/topk.cuh)
 
-def batched_select_model(u, k, cap=4096):
-    """The batched call's select (k_topk_select): a 12-bit histogram, the k-th key's bucket staged
-    (at most `cap` keys) for two 10-bit passes, or three 8/8/4-bit passes over all keys when the
-    bucket is crowded; returns the selected slots in output order."""
+def batched_select_model(u, k, cap=4096, seed=0):
+    """The batched call's select (k_topk_select): a 12-bit histogram gives the bucket beta of the
+    k-th key; keys of higher buckets and (at most `cap`) keys of bucket beta are appended in any
+    order (shuffled here), the stage sorted by 64-bit key gives the bucket's largest keys; a
+    crowded bucket takes three 8/8/4-bit passes over all keys and an ordered pass; returns the
+    selected slots in output order."""
+    rng = np.random.default_rng(seed)
     F = u.size
+    kk = key64(u)
     if F <= k:
-        slots = np.arange(F)
+        slots = rng.permutation(F)
     else:
         hist = np.bincount(u >> 20, minlength=4096)
         beta, above = _find_bin(hist, k)
-        sel = list(np.nonzero((u >> 20) > beta)[0])               # slot order
-        assert len(sel) == above
+        sel = rng.permutation(np.nonzero((u >> 20) > beta)[0])
+        assert sel.size == above
         want = k - above
         if hist[beta] <= cap:
-            staged = np.nonzero((u >> 20) == beta)[0]             # slot order
-            passes = [(10, 1023), (0, 1023)]
-            pool = staged
+            staged = rng.permutation(np.nonzero((u >> 20) == beta)[0])
+            top = staged[np.argsort(kk[staged])[::-1]][:want]
         else:
-            passes = [(12, 255), (4, 255), (0, 15)]
-            pool = np.arange(F)
-        prefix, pmask, remaining = beta << 20, 0xFFF00000, want
-        for shift, bins in passes:
-            m = (u[pool] & pmask) == prefix
-            h = np.bincount((u[pool][m] >> shift) & bins, minlength=1024)
-            d, ab = _find_bin(h, remaining)
-            prefix |= d << shift
-            remaining -= ab
-            pmask |= bins << shift
-        inb = pool[(u[pool] >> 20) == beta]
-        gt = [j for j in inb if u[j] > prefix]
-        eq = [j for j in inb if u[j] == prefix][:remaining]
-        assert len(gt) == want - remaining
-        slots = np.array(sel + gt + eq, dtype=np.int64)
-    order = np.lexsort((slots, -u[slots].astype(np.int64)))
+            prefix, pmask, remaining = beta << 20, 0xFFF00000, want
+            for shift, bins in ((12, 255), (4, 255), (0, 15)):
+                m = (u & pmask) == prefix
+                h = np.bincount((u[m] >> shift) & bins, minlength=1024)
+                d, ab = _find_bin(h, remaining)
+                prefix |= d << shift
+                remaining -= ab
+                pmask |= bins << shift
+            inb = np.arange(F)[(u >> 20) == beta]
+            gt = [j for j in inb if u[j] > prefix]
+            eq = [j for j in inb if u[j] == prefix][:remaining]
+            assert len(gt) == want - remaining
+            top = np.array(gt + eq, dtype=np.int64)
+        slots = np.concatenate([sel, top]).astype(np.int64)
+    order = np.argsort(kk[slots])[::-1]
     return slots[order]
 
 
@@ -164,4 +166,60 @@ def test_batched_select_model_equals_plain_sort(kind, cap):
     for nc in (0, 1, 100, 2047, 2049, 5000, 20000):
         for k in (1, 7, 512, 2048, 4096):
             u = keys(rng, kind, nc)
-            assert np.array_equal(batched_select_model(u, k, cap), plain_sort(u, k)), (kind, nc, k, cap)
+            assert np.array_equal(batched_select_model(u, k, cap, seed=nc + k), plain_sort(u, k)), (kind, nc, k, cap)
+
+
+# ------------------------------------------------------------------ block sort (csrc/common.cuh)
+
+def block_sort_desc_model(v, nw=32):
+    """block_sort_desc_u64: bitonic sort, strides >= 64 through shared memory, strides below 64 in
+    each warp's 64 keys (two per lane, partners by shuffle); v: uint64 array, len a power of two
+    >= 64.  Returns the sorted copy."""
+    v = v.copy()
+    n = v.size
+    size = 2
+    while size <= n:
+        stride = size >> 1
+        while stride >= 64:
+            t = np.arange(n // 2)
+            lo = 2 * t - (t & (stride - 1))
+            hi = lo + stride
+            desc = (lo & size) == 0
+            a, c = v[lo].copy(), v[hi].copy()
+            swap = (a < c) == desc
+            v[lo] = np.where(swap, c, a)
+            v[hi] = np.where(swap, a, c)
+            stride >>= 1
+        for blk in range(n // 64):
+            lane = np.arange(32)
+            e0 = blk * 64 + 2 * lane
+            a, b = v[e0].copy(), v[e0 + 1].copy()
+            desc = (e0 & size) == 0
+            st = min(size >> 1, 32)
+            while st >= 2:
+                m = st >> 1
+                low = (e0 & st) == 0
+                pa, pb = a[lane ^ m], b[lane ^ m]
+                keep_max = low == desc
+                a = np.where(keep_max, np.maximum(a, pa), np.minimum(a, pa))
+                b = np.where(keep_max, np.maximum(b, pb), np.minimum(b, pb))
+                st >>= 1
+            swap = (a < b) == desc
+            a, b = np.where(swap, b, a), np.where(swap, a, b)
+            v[e0], v[e0 + 1] = a, b
+        size <<= 1
+    return v
+
+
+@pytest.mark.parametrize("n", [64, 128, 256, 2048, 8192])
+def test_block_sort_model_sorts(n):
+    rng = np.random.default_rng(n)
+    for kind in ("random", "ties", "zeros"):
+        if kind == "random":
+            v = rng.integers(0, 2 ** 63, n, dtype=np.uint64)
+        elif kind == "ties":
+            v = rng.integers(0, 5, n).astype(np.uint64) << np.uint64(40)
+        else:
+            v = np.zeros(n, dtype=np.uint64)
+            v[: n // 3] = rng.integers(1, 2 ** 40, n // 3, dtype=np.uint64)
+        assert np.array_equal(block_sort_desc_model(v), np.sort(v)[::-1]), (n, kind)
