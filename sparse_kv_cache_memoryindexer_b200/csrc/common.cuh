@@ -63,6 +63,31 @@ __device__ __forceinline__ float ordered_to_float(uint32_t u)
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
+// Buckets of a Top-k select.  The order-preserving score keys of one query lie in [umin, umax];
+// bucket(u) = (u - umin) >> shift with the smallest shift that leaves at most SEL_NB buckets, so
+// the buckets follow the spread of the query's own scores (a split on the top bits of the key
+// would put the scores of one binade into eight buckets).  Keys outside the range (there are
+// none) are clamped to the end buckets.
+constexpr int SEL_NB = 4096;
+struct SelRange {
+    uint32_t umin, shift;
+};
+__device__ __forceinline__ SelRange sel_range(uint32_t umin, uint32_t umax)
+{
+    SelRange r;
+    r.umin = umin;
+    const uint32_t d = umax > umin ? umax - umin : 0u;
+    const int bits = 32 - __clz((int)d);
+    r.shift = bits > 12 ? (uint32_t)(bits - 12) : 0u;
+    return r;
+}
+__device__ __forceinline__ uint32_t sel_bucket(const SelRange &r, uint32_t u)
+{
+    const uint32_t d = u > r.umin ? u - r.umin : 0u;
+    const uint32_t bk = d >> r.shift;
+    return bk < (uint32_t)(SEL_NB - 1) ? bk : (uint32_t)(SEL_NB - 1);
+}
+
 // Sequence owning global tile t: largest b with tile_start[b] <= t (tile_start has B+1 entries).
 __device__ __forceinline__ int seq_of_tile(const int *tile_start, int B, int t)
 {

@@ -5,18 +5,30 @@
 // reaches p of the total); an entry is golden for token i if at least theta layers keep it; the
 // window's label set is the union over its tokens.
 //
-// k_golden_nucleus   one CTA per (sequence, token, layer) row, the row staged in shared memory when
-//                    it fits (one read from DRAM).  The kept set is {key > K*} plus the
+// k_golden_nucleus   one CTA per (sequence, token, layer) row.  The kept set is {key > K*} plus the
 //                    first n of {key == K*} in entry order, where key is the order-preserving
-//                    integer image of the logit.  One pass gives the total mass Z = sum e
-//                    (e = exp(z - max z), double) and, for a few depths D, the mass and count of
-//                    the entries within D of the maximum.  The nucleus lies inside the smallest such
-//                    set whose mass reaches p Z; when that set has at most CAND entries they are
-//                    sorted in shared memory (logit descending, entry ascending) and scanned in
-//                    double for the crossing.  Otherwise (flat rows) K* and n come from a
-//                    most-significant-digit-first radix search on the key driven by the masses.
-//                    The row's kept bits go to a [tau][Lc][ceil(T/32)] bit plane, one atomicOr per
-//                    32-entry word (words can straddle two sequences).
+//                    integer image of the logit: the first n_p entries of the row sorted by
+//                    (logit desc, entry asc), n_p the first count whose mass sum e reaches p Z
+//                    (e = exp(z - max z), Z = sum of all e).
+//                    Fast path (two reads of the row): the maximum; then Z in fp32 exp with an
+//                    error bound of its own, while the entries within 8 of the maximum are
+//                    gathered in shared memory.  Their masses (in double) tell whether they hold
+//                    the nucleus (the kept set is a prefix of the sorted row, so any such prefix
+//                    of candidates gives the same crossing); they are sorted (only those within
+//                    4 when those suffice) and scanned in double for the crossing against both
+//                    ends of the target's interval p [Z - err, Z + err].  When both ends give the
+//                    same position it is the one an fp64 Z gives; otherwise Z is recomputed in
+//                    double and the scan repeated.  The kept entries' bits are set from the
+//                    sorted candidates.
+//                    General path (more than CAND entries within 8, or less than the target's
+//                    mass there): Z in double and, for a few depths D, the mass and count of the
+//                    entries within D of the maximum; the smallest such set whose mass reaches
+//                    p Z and that has at most CAND entries is sorted and scanned in double;
+//                    otherwise (flat rows) K* and n come from a most-significant-digit-first
+//                    radix search on the key driven by the masses, and a pass over the row sets
+//                    the bits.
+//                    Bits go to a [tau][Lc][ceil(T/32)] bit plane by atomicOr (words can
+//                    straddle two sequences).
 // k_golden_vote      one warp per 32-entry word: votes over the Lc layers per token, theta test,
 //                    OR over the tokens, one label byte per entry.
 #pragma once
@@ -26,7 +38,7 @@ namespace lsa {
 
 namespace golden {
 
-constexpr int THREADS = 1024;
+constexpr int THREADS = 256;
 constexpr int CAND = 4096;       // candidates sorted in shared memory
 constexpr int ND = 6;            // depths below the maximum tried for the candidate set
 __device__ __forceinline__ float depth(int k) { return k == 0 ? 4.f : (k == 1 ? 8.f : (k == 2 ? 12.f : (k == 3 ? 16.f : (k == 4 ? 24.f : 40.f)))); }
@@ -55,21 +67,65 @@ __device__ __forceinline__ double block_sum(double v, double *red)
     return r;
 }
 
-// Dynamic shared memory: room for `stage_cap` logits; a row of at most stage_cap entries is copied
-// there first (read from DRAM once, eight independent loads in flight per thread) and every pass
-// reads it from shared memory; a longer row is read from global memory at every pass.
+// Block-wide inclusive scan of one double per thread: returns this thread's inclusive prefix and
+// the block total in *total.  red: THREADS / 32 doubles.  Starts and ends with a barrier.
+__device__ __forceinline__ double block_incl_scan_d(double v, double *red, double *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) red[warp] = v;
+    __syncthreads();
+    double before = 0.0, t = 0.0;
+    for (int w = 0; w < THREADS / 32; w++) {
+        before += w < warp ? red[w] : 0.0;
+        t += red[w];
+    }
+    *total = t;
+    __syncthreads();
+    return before + v;
+}
+
+// Crossing of the sorted candidates cand[0..nc): the first position r whose cumulative mass
+// sum_{r' <= r} exp(z_r' - m) reaches target_lo (*cross_lo) and target_hi (*cross_hi); INT_MAX
+// when not reached.  Masses in double, summed in blocks of THREADS in candidate order.
+__device__ __forceinline__ void scan_crossing(const unsigned long long *cand, int nc, float m, double target_lo,
+                                              double target_hi, double *red, int *s_lo, int *s_hi)
+{
+    if (threadIdx.x == 0) {
+        *s_lo = INT_MAX;
+        *s_hi = INT_MAX;
+    }
+    double carry = 0.0;
+    for (int base = 0; base < nc; base += THREADS) {
+        const int r0 = base + threadIdx.x;
+        const double e = r0 < nc ? exp((double)ordered_to_float((uint32_t)(cand[r0] >> 32)) - (double)m) : 0.0;
+        double total;
+        const double inc = carry + block_incl_scan_d(e, red, &total);
+        if (r0 < nc && inc >= target_lo) atomicMin(s_lo, r0);
+        if (r0 < nc && inc >= target_hi) atomicMin(s_hi, r0);
+        carry += total;
+        __syncthreads();
+        if (*s_hi < INT_MAX) break;
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restrict__ z, const int64_t *__restrict__ offs,
                                                             int64_t T, int B, int tau, int Lc, double p,
                                                             uint32_t *__restrict__ bits, int64_t W32,
-                                                            int32_t *__restrict__ nsize, int stage_cap)
+                                                            int32_t *__restrict__ nsize)
 {
-    extern __shared__ float srow[];
     __shared__ double hmass[256];
     __shared__ int hcnt[256];
     __shared__ unsigned long long cand[CAND];  // (key << 32) | ~entry
     __shared__ double dmass[ND][THREADS / 32];
     __shared__ int dcnt[ND][THREADS / 32];
-    __shared__ int s_nc, s_depth, s_cross;
+    __shared__ int s_nc, s_depth, s_cross, s_cross_hi, s_n4;
     __shared__ float fred[THREADS / 32];
     __shared__ double dred[THREADS / 32];
     __shared__ uint32_t s_prefix;
@@ -84,26 +140,108 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
         return;
     }
     const float *row = z + ((int64_t)i * Lc + l) * T + off;
-    if (S <= stage_cap) {
-        for (int64_t base = 0; base < S; base += 8 * THREADS) {
-            float v[8];
+    uint32_t *plane = bits + ((int64_t)i * Lc + l) * W32;
+    float m = -INFINITY;
+    {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int64_t base = 0; base < S; base += 4 * THREADS) {
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
+            for (int q = 0; q < 4; q++) {
                 const int64_t s = base + q * THREADS + threadIdx.x;
-                v[q] = s < S ? __ldg(row + s) : 0.f;
+                if (s < S) m4[q] = fmaxf(m4[q], __ldg(row + s));
             }
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int64_t s = base + q * THREADS + threadIdx.x;
-                if (s < S) srow[s] = v[q];
+        }
+        m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+    }
+    m = block_max(m, fred);
+
+    // ---------------------------------------------------------------- fast path
+    if (m > -INFINITY && m < INFINITY) {
+        if (threadIdx.x == 0) s_nc = 0;
+        __syncthreads();
+        // Z in fp32 exp (summed in double) and the bound of its error: expf is within 2 ulp
+        // (2^-22 relative) and z - m is rounded once (an error of 2^-24 |x| in the exponent); a
+        // result below the smallest normal is off by at most 2^-126 absolute
+        double z32 = 0.0, zx = 0.0;
+        for (int64_t s = threadIdx.x; s < S; s += THREADS) {
+            const float zs = __ldg(row + s);
+            const float x = zs - m;
+            const float e = expf(x);
+            z32 += (double)e;
+            zx += (double)e * (double)(-x);
+            if (m - zs < 8.f) {
+                const int at = atomicAdd(&s_nc, 1);
+                if (at < CAND) cand[at] = ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s);
+            }
+        }
+        double Z32 = block_sum(z32, dred);
+        const double ZX = block_sum(zx, dred);
+        // (plus the rounding of sums in double, here and in an fp64 Z: terms per thread + 64 ulps)
+        const double err = 1.01 * (Z32 * 0x1p-22 + ZX * 0x1p-24) + (double)S * 0x1p-126 +
+                           2.0 * Z32 * ((double)S / THREADS + 64.0) * 0x1p-53;
+        const int nc8 = s_nc;
+        if (nc8 <= CAND) {
+            // exact masses of the entries within 8 and within 4 of the maximum
+            double m8 = 0.0, m4 = 0.0;
+            int c4 = 0;
+            for (int t = threadIdx.x; t < nc8; t += THREADS) {
+                const float zc = ordered_to_float((uint32_t)(cand[t] >> 32));
+                const double e = exp((double)zc - (double)m);
+                m8 += e;
+                if (m - zc < 4.f) {
+                    m4 += e;
+                    c4++;
+                }
+            }
+            m8 = block_sum(m8, dred);
+            m4 = block_sum(m4, dred);
+            const double t_hi = p * (Z32 + err) * (1.0 + 0x1p-50);
+            const double t_lo = p * (Z32 - err) * (1.0 - 0x1p-50);
+            if (m8 >= t_hi) {
+                int nc = nc8;
+                if (m4 >= t_hi) {  // the entries within 4 hold the nucleus: keep only them
+                    if (threadIdx.x == 0) s_n4 = 0;
+                    for (int base = 0; base < nc8; base += THREADS) {
+                        const int t = base + threadIdx.x;
+                        unsigned long long v = 0ull;
+                        bool keep = false;
+                        if (t < nc8) {
+                            v = cand[t];
+                            keep = m - ordered_to_float((uint32_t)(v >> 32)) < 4.f;
+                        }
+                        __syncthreads();  // every entry of this block read before any is overwritten
+                        if (keep) cand[atomicAdd(&s_n4, 1)] = v;
+                        __syncthreads();
+                    }
+                    nc = s_n4;
+                }
+                int np2 = 64;
+                while (np2 < nc) np2 <<= 1;
+                for (int t = nc + threadIdx.x; t < np2; t += THREADS) cand[t] = 0ull;
+                block_sort_desc_u64(cand, np2);
+                scan_crossing(cand, nc, m, t_lo, t_hi, dred, &s_cross, &s_cross_hi);
+                int cross = s_cross;
+                if (cross != s_cross_hi) {
+                    // the target's interval holds a crossing: Z in double decides
+                    double zd = 0.0;
+                    for (int64_t s = threadIdx.x; s < S; s += THREADS) zd += exp((double)__ldg(row + s) - (double)m);
+                    const double Zd = block_sum(zd, dred);
+                    scan_crossing(cand, nc, m, p * Zd, p * Zd, dred, &s_cross, &s_cross_hi);
+                    cross = s_cross;
+                }
+                if (cross >= nc) cross = nc - 1;  // rounding left the target above the candidates' mass
+                for (int t = threadIdx.x; t <= cross; t += THREADS) {
+                    const int64_t g = off + (int64_t)(int)(~(uint32_t)(cand[t] & 0xffffffffull));
+                    atomicOr(plane + (g >> 5), 1u << (g & 31));
+                }
+                if (threadIdx.x == 0 && nsize) nsize[r] = cross + 1;
+                return;
             }
         }
         __syncthreads();
-        row = srow;
     }
-    float m = -INFINITY;
-    for (int64_t s = threadIdx.x; s < S; s += THREADS) m = fmaxf(m, row[s]);
-    m = block_max(m, fred);
+
+    // ---------------------------------------------------------------- general path
     double tot = 0.0, dm[ND];
     int dc[ND];
 #pragma unroll
@@ -112,7 +250,7 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
         dc[k] = 0;
     }
     for (int64_t s = threadIdx.x; s < S; s += THREADS) {
-        const float zs = row[s];
+        const float zs = __ldg(row + s);
         const double e = exp((double)zs - (double)m);
         tot += e;
 #pragma unroll
@@ -300,7 +438,6 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     const uint32_t K = s_prefix;
     const int64_t last_eq = s_last_eq;
     // kept bits, one atomicOr per 32-entry word of the global entry numbering
-    uint32_t *plane = bits + ((int64_t)i * Lc + l) * W32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int64_t g0 = ((off >> 5) + warp) << 5; g0 < off + S; g0 += (int64_t)THREADS) {
         const int64_t g = g0 + lane, s = g - off;

@@ -43,6 +43,10 @@ struct Params {
     const int *item_start;   // [B+1]
     int *item_counter;       // next unclaimed item, zeroed by k_li_items
     float *Y;                // [tau*T]
+    uint32_t *range;         // one decode step (nq = 1): per sequence b, words range[b*range_stride]
+                             // and [+1] take the smallest and largest score key (atomicMin / Max);
+                             // null: not reported
+    int range_stride;
     int64_t T;
     int B, tau, groups, stages;
     int ch;                  // key tiles per work item
@@ -318,16 +322,15 @@ __global__ void __launch_bounds__(320, 1)
             __syncwarp();
             const int64_t off = __ldg(p.offs + w.b);
             float *Yb = p.Y + (int64_t)p.tau * off;
+            uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // score keys of this warp's entries of the item
             for (int kt = t0; kt < t1; kt++) {
-                if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
-                tc_fence_after();
                 const int64_t j = (int64_t)kt * TILE + quarter * 32 + lane;
                 const bool valid = j < F;
                 float sc = 1.f;
-                if (p.hsc && valid) {
-                    sc = __ldg(p.hsc + off + j);
-                    if (!(sc >= 0.f)) flag(ERRF_SCALE);
-                }
+                if (p.hsc && valid) sc = __ldg(p.hsc + off + j);  // issued before the wait: its latency hides there
+                if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                if (p.hsc && valid && !(sc >= 0.f)) flag(ERRF_SCALE);
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * NCOL + 128 * half;
                 float y[2] = {0.f, 0.f};
                 if (nqw == 0) {  // nothing of this warp in the slot: release it at once
@@ -368,6 +371,19 @@ __global__ void __launch_bounds__(320, 1)
                 if (valid) {
                     if (nqw > 0) Yb[(int64_t)i0 * S + j] = y[0];
                     if (nqw > 1) Yb[(int64_t)(i0 + 1) * S + j] = y[1];
+                    if (NQV == 1) {
+                        const uint32_t u = float_to_ordered(y[0]);
+                        kmin = min(kmin, u);
+                        kmax = max(kmax, u);
+                    }
+                }
+            }
+            if (NQV == 1 && p.range && nqw > 0) {
+                kmin = __reduce_min_sync(0xffffffffu, kmin);
+                kmax = __reduce_max_sync(0xffffffffu, kmax);
+                if (lane == 0 && kmin <= kmax) {
+                    atomicMin(p.range + (int64_t)w.b * p.range_stride, kmin);
+                    atomicMax(p.range + (int64_t)w.b * p.range_stride + 1, kmax);
                 }
             }
         }
@@ -396,16 +412,24 @@ inline bool li_tc_supported(int n_h, int d_I, int tau, int kdt, int nq = li::NQ)
 // item_counter: one device int (zeroed by the planner).
 // nq: queries per MMA group (li_tc_supported).  Launches the item planner and the scoring kernel;
 // *launches counts them.
+// planned: item_start and item_counter were already written for this call (ch = li_item_tiles(nq)),
+// so the planner is not launched.  range (nq = 1 only; nullable): per sequence b, the smallest and
+// largest order-preserving score key are folded into range[b * range_stride] and [+ 1].
+inline int li_item_tiles(int nq) { return nq == li::NQ ? li::CH : li::CH_STEP; }
+
 inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK, const float *hsc,
                                const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, int nq, float *Y,
-                               int *item_start, int *item_counter, int sms, cudaStream_t st, int *launches)
+                               int *item_start, int *item_counter, int sms, cudaStream_t st, int *launches,
+                               bool planned = false, uint32_t *range = nullptr, int range_stride = 0)
 {
     using namespace li;
     *launches = 0;
     if (nq != NQ && nq != 1) return LSA_ERR_UNSUPPORTED;
-    const int ch = nq == NQ ? CH : CH_STEP;
-    k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / nq, ch, item_start, item_counter);
-    (*launches)++;
+    const int ch = li_item_tiles(nq);
+    if (!planned) {
+        k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / nq, ch, item_start, item_counter);
+        (*launches)++;
+    }
     if (T == 0) return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
     CUtensorMap kmap, qmap;
     bool ok = make_map_2d(&kmap, hotK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)T, tc::DI, 64, 128);
@@ -419,6 +443,8 @@ inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK
     p.item_start = item_start;
     p.item_counter = item_counter;
     p.Y = Y;
+    p.range = range;
+    p.range_stride = range_stride;
     p.T = T;
     p.B = B;
     p.tau = tau;

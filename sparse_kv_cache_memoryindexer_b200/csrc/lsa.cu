@@ -241,9 +241,12 @@ lsa_status lsa_selftest_wait_timeout(int32_t *status_out, lsa_stream_t stream)
 // tensor-core path adds the partial sums of its K ranges there before rounding c once).
 size_t lsa_project_workspace_size(int L, int B, int d, int r, int n_h, int d_I, lsa_dtype dt)
 {
-    (void)d; (void)n_h; (void)d_I;
-    if (L <= 0 || B <= 0 || r <= 0) return 0;
-    return align_up((size_t)L * B * r * elem_bytes(dt), 256) + align_up((size_t)L * B * r * 4, 256);
+    (void)d; (void)d_I;
+    if (L <= 0 || B <= 0 || r <= 0 || n_h <= 0) return 0;
+    // c in its storage type, then the fp32 partial slices of c and w (K split in at most KSPLIT_MAX)
+    return align_up((size_t)L * B * r * elem_bytes(dt), 256) +
+           align_up((size_t)proj::KSPLIT_MAX * L * B * r * 4, 256) +
+           align_up((size_t)proj::KSPLIT_MAX * L * B * n_h * 4, 256);
 }
 
 lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const void *W_w, lsa_dtype dt,
@@ -265,21 +268,21 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
     void *c = workspace;
     if (proj_tc_supported(dt, B, d) && proj_tc_supported(dt, B, r)) {
         // c and w in one launch, split along d so that every SM streams weights (fp32 partial sums
-        // added into zeroed buffers); c rounded to bf16 once; then q, all of r per tile
+        // in slices of their own); the slices summed in order, c rounded to bf16 once; then q, all
+        // of r per tile
         const int sms = num_sms();
-        const int64_t nc = (int64_t)L * B * r;
-        float *c32 = (float *)((char *)workspace + align_up((size_t)nc * elem_bytes(dt), 256));
-        cudaError_t e = cudaMemsetAsync(c32, 0, sizeof(float) * (size_t)nc, st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(w_out, 0, sizeof(float) * (size_t)L * B * n_h, st);
-        if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_project: %s", cudaGetErrorString(e));
-        const ProjProblem cw[2] = {{W_dq, c32, r, true}, {W_w, w_out, n_h, true}};
+        const int64_t nc = (int64_t)L * B * r, nw = (int64_t)L * B * n_h;
+        float *pc = (float *)((char *)workspace + align_up((size_t)nc * elem_bytes(dt), 256));
+        float *pw = (float *)((char *)pc + align_up((size_t)proj::KSPLIT_MAX * nc * 4, 256));
+        const ProjProblem cw[2] = {{W_dq, pc, r, true}, {W_w, pw, n_h, true}};
         const bool split[2] = {true, true};
-        lsa_status s = launch_proj_tc(h, cw, split, 2, L, B, d, sms, 2, st);
+        int ks[2] = {1, 1};
+        lsa_status s = launch_proj_tc(h, cw, split, 2, L, B, d, sms, 2, st, ks);
         if (s == LSA_OK) s = launched("project c and w (tensor cores)");
         if (s == LSA_OK) {
-            k_proj_round<<<(unsigned)std::min<int64_t>((nc + 255) / 256, (int64_t)sms * 8), 256, 0, st>>>(
-                c32, (__nv_bfloat16 *)c, nc);
-            s = launched("project: round c");
+            k_proj_reduce<<<(unsigned)std::min<int64_t>((nc + nw + 255) / 256, (int64_t)sms * 8), 256, 0, st>>>(
+                pc, ks[0], nc, (__nv_bfloat16 *)c, pw, ks[1], nw, w_out);
+            s = launched("project: reduce c and w");
         }
         const ProjProblem qp = {W_iuq, q_out, nq, false};
         const bool nosplit = false;
@@ -601,15 +604,17 @@ static int64_t step_max_chunks(int B, int64_t total_S, int W)
 }
 
 // Select workspace of one decode step: chunk starts, state, bucket histograms with finish counters,
-// the stage (capacity S_b + W keys per query) and the selection (LSA_MAX_TOPK keys per query).
-static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[5])
+// the stage (capacity S_b + W keys per query), the selection (LSA_MAX_TOPK keys per query) and the
+// query of each chunk.
+static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[6])
 {
     sp[0] = align_up(sizeof(int) * (size_t)(B + 1), 256);
     sp[1] = align_up(sizeof(uint32_t) * stepsel::NS * (size_t)B, 256);
     sp[2] = align_up(sizeof(int) * (stepsel::NB + 1) * (size_t)B, 256);
     sp[3] = align_up(sizeof(unsigned long long) * (size_t)(total_S + (int64_t)B * W + 1), 256);
     sp[4] = align_up(sizeof(unsigned long long) * (size_t)B * LSA_MAX_TOPK, 256);
-    return sp[0] + sp[1] + sp[2] + sp[3] + sp[4];
+    sp[5] = align_up(sizeof(int) * (size_t)step_max_chunks(B, total_S, W), 256);
+    return sp[0] + sp[1] + sp[2] + sp[3] + sp[4] + sp[5];
 }
 
 static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[6])
@@ -619,7 +624,7 @@ static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, siz
     part[2] = align_up(sizeof(float) * (size_t)B * (W > 0 ? W : 1), 256);
     part[3] = align_up((size_t)4 * B * n_h * d_I, 256);
     part[4] = align_up(sizeof(float) * (size_t)B * n_h, 256);
-    size_t sp[5];
+    size_t sp[6];
     part[5] = step_sel_parts(B, total_S, W, sp);
     return part[0] + part[1] + part[2] + part[3] + part[4] + part[5];
 }
@@ -670,15 +675,65 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     // one query per sequence: the tensor-core scorer runs with one-query groups (MMA N = n_h)
     const bool tc = li_tc_supported(n_h, d_I, 1, kdt, 1);
     const int TQ = 1;
-    const int64_t rows = (int64_t)B * TQ * n_h;
-    k_step_prep<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(q_step, q_batch_stride, w_step, w_batch_stride, hdt, B, TQ,
-                                                            n_h, d_I, qw, ww);
-    LSA_TRY(launched("decode step: queries"));
+    size_t sp[6];
+    step_sel_parts(B, total_S, W, sp);
+    char *sb = p + part[0] + part[1] + part[2] + part[3] + part[4];
+    int *chunk_start = (int *)sb;
+    uint32_t *state = (uint32_t *)(sb + sp[0]);
+    int *ghist = (int *)(sb + sp[0] + sp[1]);
+    unsigned long long *stage = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2]);
+    unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
+    int *chunk_query = (int *)(sb + sp[0] + sp[1] + sp[2] + sp[3] + sp[4]);
+    const int32_t *tcnt = W > 0 ? win_count : nullptr;
+    // first launch: scorer items, select chunks and state, cleared histograms, the dense query copy
+    // and the window entries' scores
+    {
+        stepsel::FrontParams fp;
+        fp.count = count;
+        fp.offs = seq_offsets;
+        fp.win_count = tcnt;
+        fp.W = W;
+        fp.B = B;
+        fp.k = k;
+        fp.n_h = n_h;
+        fp.d_I = d_I;
+        fp.dt = hdt;
+        fp.ch = li_item_tiles(1);
+        fp.item_start = item_start;
+        fp.item_counter = item_counter;
+        fp.chunk_start = chunk_start;
+        fp.chunk_query = chunk_query;
+        fp.state = state;
+        fp.ghist = ghist;
+        fp.qs = q_step;
+        fp.q_bstride = q_batch_stride;
+        fp.ws = w_step;
+        fp.w_bstride = w_batch_stride;
+        fp.q_out = qw;
+        fp.w_out = ww;
+        fp.winK = win_K;
+        fp.winsc = win_scale;
+        fp.tail = tail;
+        fp.nclear = stepsel::front_clear_ctas(B);
+        const unsigned grid = (unsigned)(1 + fp.nclear + B);
+        const bool f32 = hdt == (int)DT_F32;
+        const size_t fsm = stepsel::front_smem(n_h, d_I, hdt);
+#define LSA_STEP_FRONT(E, F)                                                                   \
+    do {                                                                                       \
+        LSA_TRY(set_smem(stepsel::k_step_front<E, F>, fsm));                                   \
+        stepsel::k_step_front<E, F><<<grid, stepsel::FRONT_TH, fsm, st>>>(fp);                 \
+    } while (0)
+        if (d_I == 32) { if (f32) LSA_STEP_FRONT(1, true); else LSA_STEP_FRONT(1, false); }
+        else if (d_I == 64) { if (f32) LSA_STEP_FRONT(2, true); else LSA_STEP_FRONT(2, false); }
+        else { if (f32) LSA_STEP_FRONT(4, true); else LSA_STEP_FRONT(4, false); }
+#undef LSA_STEP_FRONT
+        LSA_TRY(launched("decode step: front"));
+    }
     if (tc) {
         LSA_REQUIRE(aligned(hot_K, 16), "lsa_lightning_topk_step: hot_K must be 16-byte aligned");
         int n = 0;
         const lsa_status s = launch_li_tc(qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, TQ, 1, Y, item_start,
-                                          item_counter, num_sms(), st, &n);
+                                          item_counter, num_sms(), st, &n, /*planned=*/true, state + 8, stepsel::NS);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK)
             return fail(s, "lsa_lightning_topk_step: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
@@ -689,43 +744,25 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         default: LSA_TRY(li_simt_d<128>(hdt, qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, 1, n_h, Y, st)); break;
         }
     }
-    if (W > 0) {
-        const int64_t warps = (int64_t)B * W;
-        const unsigned gw = (unsigned)((warps + 7) / 8);
-#define LSA_LI_WINDOW(E, F)                                                                                       \
-    k_li_window<E, F><<<gw, 256, 0, st>>>(qw, ww, TQ, win_K, win_scale, win_count, B, W, n_h, tail)
-        const bool f32 = hdt == (int)DT_F32;
-        if (d_I == 32) { if (f32) LSA_LI_WINDOW(1, true); else LSA_LI_WINDOW(1, false); }
-        else if (d_I == 64) { if (f32) LSA_LI_WINDOW(2, true); else LSA_LI_WINDOW(2, false); }
-        else { if (f32) LSA_LI_WINDOW(4, true); else LSA_LI_WINDOW(4, false); }
-#undef LSA_LI_WINDOW
-        LSA_TRY(launched("decode step: window entries"));
-    }
     // the select, spread over chunks of candidates (see step_select.cuh)
-    size_t sp[5];
-    step_sel_parts(B, total_S, W, sp);
-    char *sb = p + part[0] + part[1] + part[2] + part[3] + part[4];
-    int *chunk_start = (int *)sb;
-    uint32_t *state = (uint32_t *)(sb + sp[0]);
-    int *ghist = (int *)(sb + sp[0] + sp[1]);
-    unsigned long long *stage = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2]);
-    unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
     const int64_t mc = step_max_chunks(B, total_S, W);
-    const int32_t *tcnt = W > 0 ? win_count : nullptr;
-    const unsigned nclear = (unsigned)(((int64_t)B * (stepsel::NB + 1) + 4095) / 4096);
-    stepsel::k_ss_setup<<<1 + nclear, 1024, 0, st>>>(count, seq_offsets, tcnt, W, B, k, chunk_start, state, ghist);
+    if (!tc) {  // the SIMT scorer does not report the range of the score keys
+        stepsel::k_ss_range<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, B, chunk_start,
+                                                                     chunk_query, state);
+        LSA_TRY(launched("decode step: key range"));
+    }
     stepsel::k_ss_hist12<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
-                                                               state, ghist);
-    stepsel::k_ss_write<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
-                                                              state, LSA_MAX_TOPK, sel, stage);
+                                                               chunk_query, state, ghist);
     int kpow2 = 64;  // the block sort works on at least 64 keys
     while (kpow2 < k) kpow2 <<= 1;
     const size_t smem = sizeof(unsigned long long) * ((size_t)kpow2 + stepsel::SCAP);
-    LSA_TRY(set_smem(stepsel::k_ss_final, smem));
-    stepsel::k_ss_final<<<(unsigned)B, stepsel::SORT_TH, smem, st>>>(sel, LSA_MAX_TOPK, stage, state, W, idx, count,
-                                                                    seq_offsets, k, kpow2, topk_idx, topk_score);
+    LSA_TRY(set_smem(stepsel::k_ss_write, smem));
+    stepsel::k_ss_write<<<(unsigned)mc, stepsel::SORT_TH, smem, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B,
+                                                                      chunk_start, chunk_query, state, LSA_MAX_TOPK, sel,
+                                                                      stage, idx,
+                                                                      k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
-    g_launches.fetch_add(3, std::memory_order_relaxed);  // setup, histogram, write (+ final)
+    g_launches.fetch_add(3, std::memory_order_relaxed);  // front, histogram, write + final
     return ok();
 }
 
@@ -756,18 +793,8 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t) * (size_t)tau * Lc * W32, st);
     if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "lsa_golden_labels: %s", cudaGetErrorString(e));
     uint32_t *bits = (uint32_t *)workspace;
-    int stage_cap = 0;
-    {
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, golden::k_golden_nucleus) != cudaSuccess)
-            return fail(LSA_ERR_CUDA, "lsa_golden_labels: %s", cudaGetErrorString(cudaGetLastError()));
-        const int64_t room = ((int64_t)227 * 1024 - (int64_t)fa.sharedSizeBytes - 1024) / 4;
-        stage_cap = (int)std::min<int64_t>(room > 0 ? room : 0, total_S);
-    }
-    const size_t gsmem = sizeof(float) * (size_t)stage_cap;
-    LSA_TRY(set_smem(golden::k_golden_nucleus, gsmem));
-    golden::k_golden_nucleus<<<(unsigned)((int64_t)B * tau * Lc), golden::THREADS, gsmem, st>>>(
-        z, seq_offsets, total_S, B, tau, Lc, p, bits, W32, nsize_out, stage_cap);
+    golden::k_golden_nucleus<<<(unsigned)((int64_t)B * tau * Lc), golden::THREADS, 0, st>>>(
+        z, seq_offsets, total_S, B, tau, Lc, p, bits, W32, nsize_out);
     LSA_TRY(launched("golden labels: nucleus"));
     golden::k_golden_vote<<<(unsigned)((W32 + golden::THREADS / 32 - 1) / (golden::THREADS / 32)), golden::THREADS, 0,
                             st>>>(bits, W32, total_S, tau, Lc, theta, label_out);

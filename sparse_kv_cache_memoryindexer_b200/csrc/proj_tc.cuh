@@ -9,10 +9,11 @@
 //
 // A launch serves one or two problems with the same X (c and w both read h).  Its work units are
 // (problem, 128-row tile, range of K): a problem whose tiles alone would leave SMs idle is split
-// along K, its units adding fp32 partial sums into a zeroed fp32 output with atomics (c is rounded
-// to bf16 by k_proj_round afterwards; w is fp32 anyway); a problem with enough tiles takes all of K
-// per unit and its epilogue rounds to the output type (bf16 nearest-even, or fp32) and stores.
-// Either way every output is one fp32 sum of its K products, rounded once.
+// along K into at most KSPLIT_MAX ranges, each unit storing its fp32 partial sums into a slice of
+// its own (no atomics, nothing to zero); k_proj_reduce then adds the slices in a fixed order and
+// rounds (c to bf16; w stays fp32).  A problem with enough tiles takes all of K per unit and its
+// epilogue rounds to the output type (bf16 nearest-even, or fp32) and stores.  Either way every
+// output is an fp32 sum of its K products, rounded once, and the same on every run.
 //
 // Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue (one TMEM lane
 // quarter each).  Two accumulators, so a unit's epilogue overlaps the next unit's MMAs.  Every
@@ -26,14 +27,16 @@ namespace lsa {
 namespace proj {
 
 constexpr int KB = 64;              // K elements per stage (one 128-byte swizzle atom of bf16)
+constexpr int KSPLIT_MAX = 8;       // K ranges of a split problem (partial slices)
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 6 * 32;
 constexpr uint32_t A_BYTES = 128 * KB * 2;
 
 struct Prob {
-    void *out;          // [L][B][R]: bf16 or fp32 (stored), or fp32 (ksplit > 1: added atomically)
+    void *out;          // [L][B][R] bf16 or fp32; split: fp32 partial slices [ksplit][L][B][R]
     int R;              // output rows
     int out_f32;
+    int partial;        // split along K: store fp32 partial sums into slice ks
     int mtiles;         // 128-row tiles per layer
     int ksplit;         // K ranges per tile
     int nkb_per;        // K blocks per range
@@ -49,9 +52,9 @@ struct Params {
 };
 
 struct Unit {
-    int prob, l, m0, kb0, kb1;
+    int prob, l, m0, kb0, kb1, ks;
     void *out;
-    int R, out_f32, ksplit;
+    int R, out_f32, partial;
 };
 
 // The problem fields are picked with selects (no dynamic index into the kernel parameters).
@@ -69,10 +72,11 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int u, int nkb)
     x.m0 = (t % mtiles) * 128;
     x.kb0 = ks * nkb_per;
     x.kb1 = min(nkb, x.kb0 + nkb_per);
+    x.ks = ks;
     x.out = one ? p.pr[1].out : p.pr[0].out;
     x.R = one ? p.pr[1].R : p.pr[0].R;
     x.out_f32 = one ? p.pr[1].out_f32 : p.pr[0].out_f32;
-    x.ksplit = ksplit;
+    x.partial = one ? p.pr[1].partial : p.pr[0].partial;
     return x;
 }
 
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(THREADS)
                     const int b = b0 + i;
                     if (valid && b < p.B) {
                         const int64_t at = ((int64_t)x.l * p.B + b) * x.R + o;
-                        if (x.ksplit > 1) atomicAdd((float *)x.out + at, v[i]);
+                        if (x.partial) ((float *)x.out)[(int64_t)x.ks * p.L * p.B * x.R + at] = v[i];
                         else if (x.out_f32) ((float *)x.out)[at] = v[i];
                         else ((__nv_bfloat16 *)x.out)[at] = __float2bfloat16_rn(v[i]);
                     }
@@ -250,7 +254,7 @@ inline bool proj_tc_supported(int dt, int B, int K) { return dt == DT_BF16 && B 
 // One problem of a launch: out[l][b][o] = sum_k X[l][b][k] W[l][o][k], W bf16 [L][R][K].
 struct ProjProblem {
     const void *W;
-    void *out;          // fp32 (added atomically) when split along K, else stored as bf16 or fp32
+    void *out;          // split along K: fp32 partial slices [KSPLIT_MAX][L][B][R]; else bf16 or fp32
     int R;
     bool out_f32;
 };
@@ -265,17 +269,19 @@ inline void proj_split(int L, int R, int K, int want_units, bool split, int &ksp
     int ks = 1;
     if (split) {
         ks = (want_units + tiles - 1) / tiles;
-        const int cap = nkb / 2 > 1 ? nkb / 2 : 1;
+        int cap = nkb / 2 > 1 ? nkb / 2 : 1;
+        if (cap > KSPLIT_MAX) cap = KSPLIT_MAX;
         ks = ks < 1 ? 1 : (ks > cap ? cap : ks);
     }
     nkb_per = (nkb + ks - 1) / ks;
     ksplit = (nkb + nkb_per - 1) / nkb_per;
 }
 
-// One launch over one or two problems sharing X bf16 [L][B][K]; split problems need a zeroed fp32
-// output.  stages_max bounds the pipeline (fewer stages leave room for two CTAs per SM).
+// One launch over one or two problems sharing X bf16 [L][B][K]; a split problem's units store
+// partial slices, and ksplit_out[i] (nullable) reports how many.  ctas_per_sm bounds the pipeline
+// (fewer stages leave room for two CTAs per SM).
 inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const bool *split, int nprob, int L, int B,
-                                 int K, int sms, int ctas_per_sm, cudaStream_t st)
+                                 int K, int sms, int ctas_per_sm, cudaStream_t st, int *ksplit_out = nullptr)
 {
     using namespace proj;
     CUtensorMap wmap[2], xmap;
@@ -295,7 +301,9 @@ inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const boo
         r.R = q.R;
         r.out_f32 = q.out_f32 ? 1 : 0;
         r.mtiles = (q.R + 127) / 128;
+        r.partial = i < nprob && split[i] ? 1 : 0;
         proj_split(L, q.R, K, want, i < nprob && split[i], r.ksplit, r.nkb_per);
+        if (ksplit_out && i < nprob) ksplit_out[i] = r.ksplit;
         r.units = i < nprob ? L * r.mtiles * r.ksplit : 0;
         total += r.units;
         ok = ok && make_map_2d(&wmap[i], q.W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * q.R, (uint64_t)K, KB, 128);
@@ -314,12 +322,24 @@ inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const boo
     return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }
 
-// c (fp32 sums) -> bf16, n elements.
-__global__ void __launch_bounds__(256) k_proj_round(const float *__restrict__ in, __nv_bfloat16 *__restrict__ out,
-                                                    int64_t n)
+// The partial slices of the split problems summed in slice order: c = sum of pc's k0 slices of n0
+// elements, rounded to bf16; w = sum of pw's k1 slices of n1 elements (fp32).
+__global__ void __launch_bounds__(256) k_proj_reduce(const float *__restrict__ pc, int k0, int64_t n0,
+                                                     __nv_bfloat16 *__restrict__ c, const float *__restrict__ pw,
+                                                     int k1, int64_t n1, float *__restrict__ w)
 {
-    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256)
-        out[i] = __float2bfloat16_rn(in[i]);
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n0 + n1; i += (int64_t)gridDim.x * 256) {
+        if (i < n0) {
+            float s = 0.f;
+            for (int k = 0; k < k0; k++) s += __ldg(pc + (int64_t)k * n0 + i);
+            c[i] = __float2bfloat16_rn(s);
+        } else {
+            const int64_t j = i - n0;
+            float s = 0.f;
+            for (int k = 0; k < k1; k++) s += __ldg(pw + (int64_t)k * n1 + j);
+            w[j] = s;
+        }
+    }
 }
 
 }  // namespace lsa

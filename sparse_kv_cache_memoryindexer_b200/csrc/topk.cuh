@@ -3,8 +3,9 @@
 //
 // Scores of sequence b, query i, fetched slot j live at Y[tau*off_b + i*S_b + j] (fp32).
 // Selection: per query, the k-th largest score is found on order-preserving keys held in shared
-// memory (a 12-bit bucket histogram, then the bucket's keys); the survivors are sorted by (score
-// desc, entry asc) with a bitonic sort in shared memory (k_topk_select).
+// memory (a histogram of 4096 buckets spread over the query's own key range, then the bucket's
+// keys); the survivors are sorted by (score desc, entry asc) with a bitonic sort in shared memory
+// (k_topk_select).
 #pragma once
 #include "common.cuh"
 
@@ -80,10 +81,11 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total)
     return r;
 }
 
-// The k-th largest key of a query is found from a 12-bit histogram of the order-preserving score
-// keys (its bucket beta) and then inside the bucket; a candidate's 64-bit key (score key << 32) |
-// ~slot orders by score and then by smaller slot, and no two are equal.
-constexpr int SEL_BINS = 4096;
+// The k-th largest key of a query is found from a histogram of the order-preserving score keys
+// over SEL_NB buckets of the query's key range (its bucket beta) and then inside the bucket; a
+// candidate's 64-bit key (score key << 32) | ~slot orders by score and then by smaller slot, and
+// no two are equal.
+constexpr int SEL_BINS = SEL_NB;
 constexpr int SEL_CAP = 4096;      // bucket keys sorted in shared memory
 
 // The bin holding the `want`-th largest key of a histogram of NB bins (thread t owns NB / SEL_THREADS
@@ -123,12 +125,13 @@ __host__ __device__ inline size_t topk_select_smem(int kpow2, int fcap)
 // One block per (sequence, query).  kpow2 = next power of two >= max(k, 64).  Dynamic shared memory:
 // kpow2 selection keys, SEL_CAP staged keys, then the query's score keys when it has at most fcap
 // candidates (read from the scores once, eight independent loads in flight per thread; a larger
-// query reads its scores from global memory at every pass).  With more than k candidates: a 12-bit
-// histogram gives the bucket beta of the k-th largest key; the keys of higher buckets are appended
+// query reads its scores from global memory at every pass).  With more than k candidates: the range
+// of the query's keys, then a histogram over 4096 buckets of that range gives the bucket beta of
+// the k-th largest key; the keys of higher buckets are appended
 // to the selection and the bucket's keys to the stage (any order: the keys carry their slots); the
 // stage sorted by key gives the bucket's largest keys.  A bucket of more than SEL_CAP keys is
-// resolved by three more radix passes (8/8/4 bits) and an ordered pass (the first keys equal to
-// the k-th in slot order).  The k keys are sorted by (score desc, slot asc).
+// resolved by radix passes over the bits below the bucket's and an ordered pass (the first keys
+// equal to the k-th in slot order).  The k keys are sorted by (score desc, slot asc).
 __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__restrict__ Y,
                                                              const int32_t *__restrict__ idx,
                                                              const int32_t *__restrict__ count,
@@ -142,6 +145,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
     __shared__ unsigned int hist[SEL_BINS];
     __shared__ int warp_tot[32];
     __shared__ int tot_a, tot_b, s_bin, s_above, s_ngt, s_nst;
+    __shared__ uint32_t s_umin, s_umax;
 
     const int b = blockIdx.x / tau, i = blockIdx.x % tau;
     const int64_t off = offs[b], S = offs[b + 1] - offs[b];
@@ -154,6 +158,12 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
     auto key64 = [](uint32_t u, int j) { return ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j); };
     auto key_at = [&](int j) -> uint32_t { return resident ? keys[j] : float_to_ordered(__ldg(row + j)); };
 
+    if (threadIdx.x == 0) {
+        s_umin = 0xFFFFFFFFu;
+        s_umax = 0u;
+    }
+    __syncthreads();
+    uint32_t tmin = 0xFFFFFFFFu, tmax = 0u;  // the range of the query's score keys
     if (resident) {
         for (int base = 0; base < F; base += 8 * SEL_THREADS) {
             float v[8];
@@ -165,9 +175,26 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
 #pragma unroll
             for (int q = 0; q < 8; q++) {
                 const int j = base + q * SEL_THREADS + threadIdx.x;
-                if (j < F) keys[j] = float_to_ordered(v[q]);
+                if (j < F) {
+                    const uint32_t u = float_to_ordered(v[q]);
+                    keys[j] = u;
+                    tmin = min(tmin, u);
+                    tmax = max(tmax, u);
+                }
             }
         }
+    } else if (F > k) {
+        for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
+            const uint32_t u = float_to_ordered(__ldg(row + j));
+            tmin = min(tmin, u);
+            tmax = max(tmax, u);
+        }
+    }
+    tmin = __reduce_min_sync(0xffffffffu, tmin);
+    tmax = __reduce_max_sync(0xffffffffu, tmax);
+    if (lane == 0) {
+        atomicMin(&s_umin, tmin);
+        atomicMax(&s_umax, tmax);
     }
     for (int t = threadIdx.x; t < kpow2; t += SEL_THREADS) sel[t] = 0ull;
     __syncthreads();
@@ -178,7 +205,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
         for (int t = threadIdx.x; t < SEL_BINS; t += SEL_THREADS) hist[t] = 0;
         if (threadIdx.x == 0) s_ngt = s_nst = 0;
         __syncthreads();
-        for (int j = threadIdx.x; j < F; j += SEL_THREADS) atomicAdd(&hist[key_at(j) >> 20], 1u);
+        const SelRange rg = sel_range(s_umin, s_umax);
+        for (int j = threadIdx.x; j < F; j += SEL_THREADS) atomicAdd(&hist[sel_bucket(rg, key_at(j))], 1u);
         __syncthreads();
         sel_find_bin<SEL_BINS>(hist, k, warp_tot, &tot_a, &s_bin, &s_above);
         const uint32_t beta = (uint32_t)s_bin;
@@ -193,8 +221,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
             bool gt = false, eq = false;
             if (j < F) {
                 u = key_at(j);
-                gt = (u >> 20) > beta;
-                eq = staged && (u >> 20) == beta;
+                const uint32_t bk = sel_bucket(rg, u);
+                gt = bk > beta;
+                eq = staged && bk == beta;
             }
             const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
             int pg = 0, pe = 0;
@@ -215,27 +244,30 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
             block_sort_desc_u64(stage, np);
             for (int t = threadIdx.x; t < want; t += SEL_THREADS) sel[above + t] = stage[t];
         } else {
-            // a crowded bucket: three radix passes (8/8/4 bits) for the k-th key K, then the
-            // bucket's keys above K and the first keys equal to K in slot order
-            uint32_t prefix = beta << 20, pmask = 0xFFF00000u;
+            // a crowded bucket: radix passes of up to 8 bits over the offsets d = u - umin below
+            // the bucket's bits give the k-th key K; then the bucket's keys above K and the first
+            // keys equal to K in slot order
+            uint32_t dprefix = beta << rg.shift, dmask = 0xFFFFFFFFu << rg.shift;
             int remaining = want;
 #pragma unroll 1
-            for (int pass = 0; pass < 3; pass++) {
-                const int shift = pass < 2 ? 12 - 8 * pass : 0;
-                const uint32_t bins = pass < 2 ? 255u : 15u;
+            for (int pos = (int)rg.shift; pos > 0;) {
+                const int wbits = pos >= 8 ? 8 : pos, sh = pos - wbits;
+                const uint32_t bins = (1u << wbits) - 1u;
                 for (int t = threadIdx.x; t < 1024; t += SEL_THREADS) hist[t] = 0;
                 __syncthreads();
                 for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
-                    const uint32_t u = key_at(j);
-                    if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & bins], 1u);
+                    const uint32_t u = key_at(j), d = u > rg.umin ? u - rg.umin : 0u;
+                    if ((d & dmask) == dprefix) atomicAdd(&hist[(d >> sh) & bins], 1u);
                 }
                 __syncthreads();
                 sel_find_bin<1024>(hist, remaining, warp_tot, &tot_a, &s_bin, &s_above);
-                prefix |= (uint32_t)s_bin << shift;
+                dprefix |= (uint32_t)s_bin << sh;
                 remaining -= s_above;
-                pmask |= bins << shift;
+                dmask |= bins << sh;
+                pos = sh;
                 __syncthreads();
             }
+            const uint32_t prefix = rg.umin + dprefix;  // the k-th largest score key
             int cg = 0, ce = 0;
             for (int base = 0; base < F; base += SEL_THREADS) {
                 const int j = base + threadIdx.x;
@@ -243,7 +275,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
                 int gt = 0, eq = 0;
                 if (j < F) {
                     u = key_at(j);
-                    gt = (u >> 20) == beta && u > prefix;
+                    gt = sel_bucket(rg, u) == beta && u > prefix;
                     eq = u == prefix;
                 }
                 const int pg = block_excl_scan(gt, warp_tot, &tot_a) + cg;
@@ -273,65 +305,32 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
 }
 
 // ------------------------------------------------------------------ one decode step
-// Stage 5 for one decode step: each sequence's query of the step is copied into TQ query slots
-// (slot 0; the others are zero, as are their weights) so that the scorers built for groups of
-// queries serve the step unchanged.  qs / ws are the step's queries and weights with a batch
-// stride (elements) between sequences.
-__global__ void __launch_bounds__(256) k_step_prep(const void *__restrict__ qs, int64_t q_bstride,
-                                                   const float *__restrict__ ws, int64_t w_bstride, int dt, int B,
-                                                   int TQ, int n_h, int d_I, void *__restrict__ q_out,
-                                                   float *__restrict__ w_out)
-{
-    const int64_t rows = (int64_t)B * TQ * n_h;
-    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (r >= rows) return;
-    const int h = (int)(r % n_h);
-    const int qi = (int)((r / n_h) % TQ);
-    const int b = (int)(r / ((int64_t)n_h * TQ));
-    const size_t es = dt == DT_F32 ? 4 : 2;
-    uint8_t *dst = (uint8_t *)q_out + (size_t)r * d_I * es;
-    const uint8_t *src = (const uint8_t *)qs + ((size_t)b * q_bstride + (size_t)h * d_I) * es;
-    for (int e = lane; e < d_I; e += 32) {
-        if (es == 4) ((float *)dst)[e] = qi == 0 ? ((const float *)src)[e] : 0.f;
-        else ((uint16_t *)dst)[e] = qi == 0 ? ((const uint16_t *)src)[e] : (uint16_t)0;
-    }
-    if (lane == 0) w_out[r] = qi == 0 ? ws[(size_t)b * w_bstride + h] : 0.f;
-}
+// Device part of one decode step's Top-k (the first launch of the step, k_step_front, runs it).
 
-// Scores of the entries compressed during the window: one warp per (sequence, entry j < W);
-// y = sum_h w_h ReLU(scale_j q_h . k_j).  Keys [B][W][d_I] in the hot-key type, scales nullable.
-// Lane l holds key elements l E .. l E + E - 1 (E = d_I / 32).  Heads go in groups of 16: the
-// lanes' query parts of the 16 heads are loaded first (one coalesced row per head), then the 16
-// partial dot products are summed over the warp by a reduce-scatter (16 shuffles: after it, lanes
-// l and l ^ 1 hold the whole dot product of one head of the group).
+// Score of window entry j of sequence b (one warp): y = sum_h w_h ReLU(scale_j q_h . k_j) for the
+// entries compressed during the window.  Keys [B][W][d_I] in the hot-key type, scales nullable;
+// q [n_h][d_I] and w [n_h] are the sequence's query and weights (any memory space).  Lane l holds
+// key elements l E .. l E + E - 1 (E = d_I / 32).  Heads go in groups of 16: the lanes' query
+// parts of the 16 heads are loaded first (one coalesced row per head), then the 16 partial dot
+// products are summed over the warp by a reduce-scatter (16 shuffles: after it, lanes l and l ^ 1
+// hold the whole dot product of one head of the group).  Every lane returns y.
 template <int E, bool F32>
-__global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, const float *__restrict__ w, int TQ,
-                                                   const void *__restrict__ winK, const float *__restrict__ winsc,
-                                                   const int32_t *__restrict__ win_count, int B, int W, int n_h,
-                                                   float *__restrict__ tail)
+__device__ __forceinline__ float li_window_entry(int b, int j, int lane, const void *q, const float *w,
+                                                 const void *__restrict__ winK, const float *__restrict__ winsc,
+                                                 int W, int n_h)
 {
     constexpr int D = 32 * E;
-    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (gw >= (int64_t)B * W) return;
-    const int b = (int)(gw / W), j = (int)(gw % W);
-    int n = win_count[b];
-    if (n < 0 || n > W) {
-        if (lane == 0 && j == 0) flag(ERRF_COUNT);
-        n = n < 0 ? 0 : W;
-    }
-    if (j >= n) return;
     const float sc = winsc ? winsc[(int64_t)b * W + j] : 1.f;
     if (winsc && lane == 0 && !(sc >= 0.f)) flag(ERRF_SCALE);
-    auto ld = [&](const void *base, int64_t at) {
-        return F32 ? __ldg((const float *)base + at) : bf16_bits_to_float(__ldg((const unsigned short *)base + at));
-    };
     float kv[E];
 #pragma unroll
-    for (int e = 0; e < E; e++) kv[e] = ld(winK, ((int64_t)b * W + j) * D + lane * E + e);
-    const int64_t qb = (int64_t)b * TQ * n_h * D + (int64_t)lane * E;  // query slot 0
-    const float *wr = w + (int64_t)b * TQ * n_h;
+    for (int e = 0; e < E; e++) {
+        const int64_t at = ((int64_t)b * W + j) * D + lane * E + e;
+        kv[e] = F32 ? __ldg((const float *)winK + at) : bf16_bits_to_float(__ldg((const unsigned short *)winK + at));
+    }
+    auto ldq = [&](int at) {
+        return F32 ? ((const float *)q)[at] : bf16_bits_to_float(((const unsigned short *)q)[at]);
+    };
     // the head of the group whose dot product this lane holds after the reduce-scatter
     const int hl = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
     float y = 0.f;
@@ -340,7 +339,7 @@ __global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, c
 #pragma unroll
         for (int g = 0; g < 16; g++)
 #pragma unroll
-            for (int e = 0; e < E; e++) qv[g][e] = h0 + g < n_h ? ld(q, qb + (int64_t)(h0 + g) * D + e) : 0.f;
+            for (int e = 0; e < E; e++) qv[g][e] = h0 + g < n_h ? ldq((h0 + g) * D + lane * E + e) : 0.f;
         float v[16];
 #pragma unroll
         for (int g = 0; g < 16; g++) {
@@ -362,12 +361,12 @@ __global__ void __launch_bounds__(256) k_li_window(const void *__restrict__ q, c
         }
         const float dot = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
         const int h = h0 + hl;
-        float c = ((lane & 1) == 0 && h < n_h) ? __ldg(wr + h) * fmaxf(sc * dot, 0.f) : 0.f;
+        float c = ((lane & 1) == 0 && h < n_h) ? w[h] * fmaxf(sc * dot, 0.f) : 0.f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
         y += c;
     }
-    if (lane == 0) tail[(int64_t)b * W + j] = y;
+    return y;
 }
 
 }  // namespace lsa

@@ -1,8 +1,11 @@
 """Golden labels (lsa_golden_labels) against the oracle: label bytes and nucleus sizes exact.
 
-The logits are float32 and both sides take softmax masses and their sums in double, so only a row
-whose cumulative mass lands within rounding of p at the boundary could disagree; none does in these
-inputs.  Rows of exactly equal logits (ties at the boundary) exercise the entry-order tie rule.
+The logits are float32.  The oracle takes softmax masses and their sums in double.  The kernel takes
+the total mass Z in fp32 exp with an error bound, and the candidates' cumulative masses in double;
+when the target's interval p [Z - err, Z + err] holds a crossing it recomputes Z in double.  So only
+a row whose cumulative mass lands within double rounding of p Z could disagree; none does in these
+inputs.  Rows of exactly equal logits (ties at the boundary) exercise the entry-order tie rule, and
+the crossing exactly at p Z the recomputation in double.
 """
 import numpy as np
 import pytest
@@ -113,3 +116,30 @@ def test_golden_long_flat_rows_take_the_radix_search(m, p):
             for b in range(2):
                 assert not candidate_set_fits(zn[i, l, offs[b]:offs[b + 1]], p)
     check(m, z, offs, p=p, theta=2)
+
+
+def test_golden_each_path(m):
+    # sequence 0: the entries within 8 of the maximum hold the nucleus (sorted candidates);
+    # sequence 1: more than 4096 entries within 8, but those within 4 hold the nucleus (the general
+    # path's candidate sort); sequence 2: the entries within 8 hold too little mass and the rest is
+    # flat (the general path's radix search); sequence 3: all equal, the crossing exactly at p Z
+    # (the total mass recomputed in double)
+    S = (5000, 9000, 30001, 1000)
+    offs = torch.from_numpy(np.concatenate([[0], np.cumsum(S)]).astype(np.int64))
+    g = torch.Generator().manual_seed(5)
+    z = torch.zeros((2, 2, sum(S)), dtype=torch.float32)
+    o = offs.numpy()
+    z[:, :, o[0]:o[1]] = torch.randn((2, 2, S[0]), generator=g)
+    z[:, :, o[0] + 100:o[0] + 400] += 6.0
+    z[:, :, o[1]:o[1] + 3000] = 5.0 + 0.01 * torch.randn((2, 2, 3000), generator=g)
+    z[:, :, o[1] + 3000:o[2]] = 0.5
+    z[:, :, o[2]] = 10.0
+    z[:, :, o[2] + 1:o[3]] = torch.rand((2, 2, S[2] - 1), generator=g) * 0.01
+    z[:, :, o[3]:o[4]] = -2.0
+    zn = z.numpy()
+    row1 = zn[0, 0, o[1]:o[2]]
+    assert ((row1.max() - row1) < 8).sum() > 4096 and candidate_set_fits(row1, 0.6)
+    row2 = zn[0, 0, o[2]:o[3]]
+    assert not candidate_set_fits(row2, 0.6)
+    label, ref = check(m, z, offs, p=0.6, theta=1)
+    assert ref["nsize"][3, 0, 0] == 600

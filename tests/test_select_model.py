@@ -1,21 +1,27 @@
 """Numpy models of the two Top-k selects' steps against a plain sort (key descending, ties to the
 smaller slot), on the CPU.
 
-Decode-step select (csrc/step_select.cuh): over chunks of 2,048 candidates, a 12-bit histogram of
-the score keys gives the bucket of the k-th largest key; keys of higher buckets go to the selection
-and the bucket's keys to a stage, both in an arbitrary order (the model shuffles them), because every
-key carries its slot: key64 = (score key << 32) | ~slot orders by score, then smaller slot, and no
-two keys are equal.  The bucket's largest keys come from a sort (at most SCAP staged keys) or, for
-a crowded bucket, a 64-bit radix select over the stage; one sort orders the k keys.  With at most k
-candidates the select takes every candidate whatever its key, including a key that orders as 0.
+Both selects bucket a query's order-preserving score keys u over the query's own key range:
+bucket(u) = (u - umin) >> shift, with the smallest shift that leaves at most 4,096 buckets.
 
-Batched select (csrc/topk.cuh, k_topk_select): a 12-bit histogram of all keys gives the bucket of
+Decode-step select (csrc/step_select.cuh): over chunks of 2,048 candidates, a histogram of the
+buckets gives the bucket of the k-th largest key; keys of higher buckets go to the selection and the
+bucket's keys to a stage, both in an arbitrary order (the model shuffles them), because every key
+carries its slot: key64 = (score key << 32) | ~slot orders by score, then smaller slot, and no two
+keys are equal.  The bucket's largest keys come from a sort (at most SCAP staged keys) or, for a
+crowded bucket, a radix select over the stage on key64 - (umin << 32), 8 bits at a time below the
+bucket's bits, stopping once a digit holds exactly the keys still wanted; one sort orders the k
+keys.  With at most k candidates the select takes every candidate whatever its key, including a key
+that orders as 0.
+
+Batched select (csrc/topk.cuh, k_topk_select): the same histogram over all keys gives the bucket of
 the k-th key; keys of higher buckets and the bucket's keys (at most SEL_CAP of them) are appended in
-any order, and the stage sorted by 64-bit key gives the bucket's largest keys; a crowded bucket takes
-three 8/8/4-bit passes over all keys and an ordered pass instead.
+any order, and the stage sorted by 64-bit key gives the bucket's largest keys; a crowded bucket
+takes radix passes of up to 8 bits over u - umin below the bucket's bits and an ordered pass
+instead.
 
-The cases cover heavy ties in every digit, all-equal keys, keys of 0, k at and above the candidate
-count, and empty queries.
+The cases cover heavy ties in every digit, all-equal keys, keys of 0, a narrow and a wide key range
+(one outlier far above the rest), k at and above the candidate count, and empty queries.
 """
 import zlib
 
@@ -41,37 +47,55 @@ def key64(u):
     return (u.astype(np.uint64) << np.uint64(32)) | (~slots & np.uint64(0xFFFFFFFF))
 
 
+def sel_range(u):
+    """(umin, shift) of a query's keys: the smallest shift leaving at most 4,096 buckets."""
+    umin, umax = int(u.min()), int(u.max())
+    return umin, max(0, (umax - umin).bit_length() - 12)
+
+
+def sel_bucket(u, umin, shift):
+    return np.minimum((u.astype(np.int64) - umin) >> shift, 4095)
+
+
 def select_model(u, k, scap=8192, seed=0):
-    """The decode-step select (k_ss_hist12, k_ss_write, k_ss_final): 12-bit bucket histogram, keys
-    of higher buckets and of the k-th key's bucket appended in an arbitrary order (shuffled here),
-    the bucket's want largest keys by a sort (at most scap keys) or a 64-bit radix select over the
-    stage, then one sort of the k keys; returns the selected slots in output order."""
+    """The decode-step select (k_ss_hist12, k_ss_write and its final step): bucket histogram over the
+    query's key range, keys of higher buckets and of the k-th key's bucket appended in an arbitrary
+    order (shuffled here), the bucket's want largest keys by a sort (at most scap keys) or a radix
+    select over the stage, then one sort of the k keys; returns the selected slots in output order."""
     rng = np.random.default_rng(seed)
     nc = u.size
     kk = key64(u)
     if nc <= k:
         slots = rng.permutation(nc)
     else:
-        hist = np.bincount(u >> 20, minlength=4096)
+        umin, shift = sel_range(u)
+        bk = sel_bucket(u, umin, shift)
+        hist = np.bincount(bk, minlength=4096)
         beta, above = _find_bin(hist, k)
-        gt = rng.permutation(np.nonzero((u >> 20) > beta)[0])
-        staged = rng.permutation(np.nonzero((u >> 20) == beta)[0])
+        gt = rng.permutation(np.nonzero(bk > beta)[0])
+        staged = rng.permutation(np.nonzero(bk == beta)[0])
         assert gt.size == above
         want = k - above
         if staged.size <= scap:
             top = staged[np.lexsort((staged, -u[staged].astype(np.int64)))][:want]
         else:
-            prefix, pmask, rem = np.uint64(beta) << np.uint64(52), np.uint64(0xFFF) << np.uint64(52), want
-            v = kk[staged]
-            for ps in range(7):
-                shift = np.uint64(44 - 8 * ps if ps < 6 else 0)
-                dmask = np.uint64(255 if ps < 6 else 15)
+            v = kk[staged] - (np.uint64(umin) << np.uint64(32))
+            prefix = np.uint64(beta << shift) << np.uint64(32)
+            pmask = np.uint64((0xFFFFFFFFFFFFFFFF << (32 + shift)) & 0xFFFFFFFFFFFFFFFF)
+            rem, pos = want, 32 + shift
+            while pos > 0:
+                wb = min(8, pos)
+                sh = pos - wb
+                dm = np.uint64((1 << wb) - 1)
                 m = (v & pmask) == prefix
-                h = np.bincount(((v[m] >> shift) & dmask).astype(np.int64), minlength=256)
+                h = np.bincount(((v[m] >> np.uint64(sh)) & dm).astype(np.int64), minlength=256)
                 d, ab = _find_bin(h, rem)
-                prefix |= np.uint64(d) << shift
-                pmask |= dmask << shift
+                prefix |= np.uint64(d) << np.uint64(sh)
+                pmask |= dm << np.uint64(sh)
                 rem -= ab
+                pos = sh
+                if h[d] == rem:
+                    break
             top = staged[v >= prefix]
             assert top.size == want
         slots = np.concatenate([gt, top]).astype(np.int64)
@@ -95,11 +119,16 @@ def keys(rng, kind, nc):
         return np.full(nc, 0x3F800000, dtype=np.uint32)
     if kind == "zeros_and_ones":
         return rng.integers(0, 2, nc).astype(np.uint32)
+    if kind == "narrow_with_outlier":  # scores of one binade and one entry far above them
+        v = (100.0 + rng.standard_normal(nc)).astype(np.float32)
+        if nc:
+            v[rng.integers(0, nc)] = 1e6
+        return v.view(np.uint32) ^ np.uint32(0x80000000)
     return rng.standard_normal(nc).astype(np.float32).view(np.uint32) ^ np.uint32(0x80000000)
 
 
 @pytest.mark.parametrize("kind", ["random", "ties_every_digit", "ties_low_digits", "all_equal", "zeros_and_ones",
-                                  "float"])
+                                  "narrow_with_outlier", "float"])
 @pytest.mark.parametrize("scap", [8192, 16])
 def test_select_model_equals_plain_sort(kind, scap):
     rng = np.random.default_rng(zlib.crc32(kind.encode()))
@@ -120,35 +149,43 @@ def test_few_candidates_keep_a_zero_key():
 # ------------------------------------------------------------------ batched select (csrc/topk.cuh)
 
 def batched_select_model(u, k, cap=4096, seed=0):
-    """The batched call's select (k_topk_select): a 12-bit histogram gives the bucket beta of the
-    k-th key; keys of higher buckets and (at most `cap`) keys of bucket beta are appended in any
-    order (shuffled here), the stage sorted by 64-bit key gives the bucket's largest keys; a
-    crowded bucket takes three 8/8/4-bit passes over all keys and an ordered pass; returns the
-    selected slots in output order."""
+    """The batched call's select (k_topk_select): a histogram over the query's key range gives the
+    bucket beta of the k-th key; keys of higher buckets and (at most `cap`) keys of bucket beta are
+    appended in any order (shuffled here), the stage sorted by 64-bit key gives the bucket's largest
+    keys; a crowded bucket takes radix passes over u - umin below the bucket's bits and an ordered
+    pass; returns the selected slots in output order."""
     rng = np.random.default_rng(seed)
     F = u.size
     kk = key64(u)
     if F <= k:
         slots = rng.permutation(F)
     else:
-        hist = np.bincount(u >> 20, minlength=4096)
+        umin, shift = sel_range(u)
+        bk = sel_bucket(u, umin, shift)
+        hist = np.bincount(bk, minlength=4096)
         beta, above = _find_bin(hist, k)
-        sel = rng.permutation(np.nonzero((u >> 20) > beta)[0])
+        sel = rng.permutation(np.nonzero(bk > beta)[0])
         assert sel.size == above
         want = k - above
         if hist[beta] <= cap:
-            staged = rng.permutation(np.nonzero((u >> 20) == beta)[0])
+            staged = rng.permutation(np.nonzero(bk == beta)[0])
             top = staged[np.argsort(kk[staged])[::-1]][:want]
         else:
-            prefix, pmask, remaining = beta << 20, 0xFFF00000, want
-            for shift, bins in ((12, 255), (4, 255), (0, 15)):
-                m = (u & pmask) == prefix
-                h = np.bincount((u[m] >> shift) & bins, minlength=1024)
+            d_all = u.astype(np.int64) - umin
+            dprefix, dmask, remaining, pos = beta << shift, (0xFFFFFFFF << shift) & 0xFFFFFFFF, want, shift
+            while pos > 0:
+                wb = min(8, pos)
+                sh = pos - wb
+                bins = (1 << wb) - 1
+                m = (d_all & dmask) == dprefix
+                h = np.bincount((d_all[m] >> sh) & bins, minlength=1024)
                 d, ab = _find_bin(h, remaining)
-                prefix |= d << shift
+                dprefix |= d << sh
                 remaining -= ab
-                pmask |= bins << shift
-            inb = np.arange(F)[(u >> 20) == beta]
+                dmask |= bins << sh
+                pos = sh
+            prefix = umin + dprefix
+            inb = np.arange(F)[bk == beta]
             gt = [j for j in inb if u[j] > prefix]
             eq = [j for j in inb if u[j] == prefix][:remaining]
             assert len(gt) == want - remaining
@@ -159,7 +196,7 @@ def batched_select_model(u, k, cap=4096, seed=0):
 
 
 @pytest.mark.parametrize("kind", ["random", "ties_every_digit", "ties_low_digits", "all_equal", "zeros_and_ones",
-                                  "float"])
+                                  "narrow_with_outlier", "float"])
 @pytest.mark.parametrize("cap", [4096, 16])
 def test_batched_select_model_equals_plain_sort(kind, cap):
     rng = np.random.default_rng(zlib.crc32((kind + "batched").encode()))
