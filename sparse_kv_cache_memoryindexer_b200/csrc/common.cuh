@@ -63,29 +63,31 @@ __device__ __forceinline__ float ordered_to_float(uint32_t u)
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
-// Buckets of a Top-k select.  The order-preserving score keys of one query lie in [umin, umax];
-// bucket(u) = (u - umin) >> shift with the smallest shift that leaves at most SEL_NB buckets, so
-// the buckets follow the spread of the query's own scores (a split on the top bits of the key
-// would put the scores of one binade into eight buckets).  Keys outside the range (there are
-// none) are clamped to the end buckets.
+// Buckets of a Top-k select.  The order-preserving score keys of one query lie in [umin, umax],
+// scores [ymin, ymax]; bucket(u) = floor((y - ymin) * SEL_NB / (ymax - ymin)) clamped to
+// [0, SEL_NB), linear in the score so that the buckets follow the spread of the query's own scores
+// (a split on the bits of the key would put the scores of one binade into eight buckets).  It is
+// non-decreasing in the key (fp32 subtraction and multiplication are monotone), and degenerate
+// ranges (a single value, an infinite span) put every finite score into bucket 0.  A NaN goes to
+// the end its key sorts to.
 constexpr int SEL_NB = 4096;
 struct SelRange {
-    uint32_t umin, shift;
+    float ymin, scale;
 };
 __device__ __forceinline__ SelRange sel_range(uint32_t umin, uint32_t umax)
 {
     SelRange r;
-    r.umin = umin;
-    const uint32_t d = umax > umin ? umax - umin : 0u;
-    const int bits = 32 - __clz((int)d);
-    r.shift = bits > 12 ? (uint32_t)(bits - 12) : 0u;
+    r.ymin = ordered_to_float(umin);
+    const float span = ordered_to_float(umax) - r.ymin;
+    r.scale = span > 0.f ? (float)SEL_NB / span : 0.f;
     return r;
 }
 __device__ __forceinline__ uint32_t sel_bucket(const SelRange &r, uint32_t u)
 {
-    const uint32_t d = u > r.umin ? u - r.umin : 0u;
-    const uint32_t bk = d >> r.shift;
-    return bk < (uint32_t)(SEL_NB - 1) ? bk : (uint32_t)(SEL_NB - 1);
+    const float y = ordered_to_float(u);
+    if (y != y) return (u & 0x80000000u) ? (uint32_t)(SEL_NB - 1) : 0u;
+    const float t = (y - r.ymin) * r.scale;
+    return t >= (float)(SEL_NB - 1) ? (uint32_t)(SEL_NB - 1) : (t > 0.f ? (uint32_t)t : 0u);
 }
 
 // Sequence owning global tile t: largest b with tile_start[b] <= t (tile_start has B+1 entries).

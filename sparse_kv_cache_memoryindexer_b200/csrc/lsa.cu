@@ -758,8 +758,8 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     const size_t smem = sizeof(unsigned long long) * ((size_t)kpow2 + stepsel::SCAP);
     LSA_TRY(set_smem(stepsel::k_ss_write, smem));
     stepsel::k_ss_write<<<(unsigned)mc, stepsel::SORT_TH, smem, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B,
-                                                                      chunk_start, chunk_query, state, LSA_MAX_TOPK, sel,
-                                                                      stage, idx,
+                                                                      chunk_start, chunk_query, state, LSA_MAX_TOPK, ghist,
+                                                                      sel, stage, idx,
                                                                       k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
     g_launches.fetch_add(3, std::memory_order_relaxed);  // front, histogram, write + final

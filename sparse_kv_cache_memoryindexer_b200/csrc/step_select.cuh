@@ -33,6 +33,7 @@ constexpr int SORT_TH = 1024;
 constexpr int NB = SEL_NB; // buckets of the histogram (over the query's key range)
 constexpr int SCAP = 8192; // staged keys a final CTA sorts in shared memory
 constexpr int NS = 12;     // state words per query
+constexpr int RANK_SEG = 64; // largest bucket above beta whose keys the final step ranks by counting
 
 struct Query {
     const float *row;   // fetched scores (query slot 0 of the Y layout)
@@ -63,7 +64,8 @@ __device__ __forceinline__ uint32_t key_of(const Query &q, int j)
 
 // state per query (NS words): [0] bucket beta, [1] keys wanted from bucket beta (0: the query takes
 // every candidate), [2] keys of higher buckets, [3] candidates, [4] keys appended to the selection,
-// [5] keys appended to the stage, [6] finish counter of the write step, [8] smallest and [9]
+// [5] keys appended to the stage, [6] finish counter of the write step, [7] keys of the largest
+// bucket above beta, [8] smallest and [9]
 // largest score key of the query (the window entries' from the first launch, the fetched entries'
 // added by the scorer).  ghist: [B][NB] bucket histograms, then the finish counters [B].
 __device__ __forceinline__ SelRange query_range(const uint32_t *st) { return sel_range(st[8], st[9]); }
@@ -363,28 +365,48 @@ __global__ void __launch_bounds__(TH) k_ss_hist12(const float *__restrict__ Y, i
     if (!last_chunk_of_query(done, b, chunk_start[b + 1] - chunk_start[b])) return;
     // the bucket of the want-th largest key: thread t owns buckets NB - 16 (t + 1) .. NB - 16 t - 1
     constexpr int PER = NB / TH;
+    __shared__ int s_maxseg;
+    if (threadIdx.x == 0) s_maxseg = 0;
     const int hi = NB - PER * (int)threadIdx.x;
-    int cnt = 0;
+    int h[PER], cnt = 0;
 #pragma unroll
-    for (int i = 1; i <= PER; i++) cnt += __ldcg(gh + hi - i);
-    int above, unused_p, total, unused_t;
-    block_excl_scan2(cnt, 0, above, unused_p, total, unused_t);
+    for (int i = 1; i <= PER; i++) {
+        h[i - 1] = __ldcg(gh + hi - i);
+        cnt += h[i - 1];
+    }
+    int above0, unused_p, total, unused_t;
+    block_excl_scan2(cnt, 0, above0, unused_p, total, unused_t);
+    int above = above0;
     if (above < want && above + cnt >= want) {
         for (int i = 1; i <= PER; i++) {
-            const int h = __ldcg(gh + hi - i);
-            if (above + h >= want) {
+            if (above + h[i - 1] >= want) {
                 s_beta = hi - i;
                 s_above = above;
                 break;
             }
-            above += h;
+            above += h[i - 1];
         }
     }
+    __syncthreads();
+    // every bucket above beta becomes the start of its segment of the selection (higher buckets
+    // first); the largest such bucket decides how the final step orders the selection
+    int run = above0, mx = 0;
+#pragma unroll
+    for (int i = 1; i <= PER; i++) {
+        if (hi - i > s_beta) {
+            gh[hi - i] = run;
+            run += h[i - 1];
+            mx = max(mx, h[i - 1]);
+        }
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if ((threadIdx.x & 31) == 0) atomicMax(&s_maxseg, mx);
     __syncthreads();
     if (threadIdx.x == 0) {
         st[0] = (uint32_t)s_beta;
         st[2] = (uint32_t)s_above;
         st[1] = (uint32_t)(want - s_above);
+        st[7] = (uint32_t)s_maxseg;
     }
 }
 
@@ -393,7 +415,8 @@ __global__ void __launch_bounds__(TH) k_ss_hist12(const float *__restrict__ Y, i
 // sk: kpow2 + SCAP keys of shared memory.  The selection and the stage were written by other CTAs
 // of the same launch: they are read through L2.
 __device__ __forceinline__ void final_of_query(int b, unsigned long long *sk, const unsigned long long *sel, int kcap,
-                                               const unsigned long long *stage, const uint32_t *state, int W,
+                                               const unsigned long long *stage, const uint32_t *state,
+                                               const int *gh, int W,
                                                const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
                                                const int64_t *__restrict__ offs, int k, int kpow2,
                                                int32_t *__restrict__ topk_idx, float *__restrict__ topk_score)
@@ -413,6 +436,12 @@ __device__ __forceinline__ void final_of_query(int b, unsigned long long *sk, co
     const unsigned long long *mine = sel + (int64_t)b * kcap;
     const int nfirst = want == 0 ? nsel : above;  // keys already in the selection
     for (int t = threadIdx.x; t < kpow2; t += nth) sk[t] = t < nfirst ? __ldcg(mine + t) : 0ull;
+    auto emit = [&](int r, unsigned long long v) {
+        const int64_t o = (int64_t)b * k + r;
+        const int j = (int)~(uint32_t)(v & 0xffffffffull);  // candidate slot
+        topk_idx[o] = (j >= 0 && j < F0) ? __ldg(idx + off + j) : ((j >= F0 && j < nc) ? (int32_t)(S + (j - F0)) : -1);
+        if (topk_score) topk_score[o] = ordered_to_float((uint32_t)(v >> 32));
+    };
     if (want > 0) {
         const unsigned long long *stg = stage + off + (int64_t)b * W;
         const int ns = (int)__ldcg(st + 5);  // the keys of bucket beta (at least want)
@@ -421,25 +450,35 @@ __device__ __forceinline__ void final_of_query(int b, unsigned long long *sk, co
             while (np < ns) np <<= 1;
             for (int t = threadIdx.x; t < np; t += nth) ss[t] = t < ns ? __ldcg(stg + t) : 0ull;
             block_sort_desc_u64(ss, np);
+            if (__ldcg(st + 7) <= (uint32_t)RANK_SEG) {
+                // the selection lies in segments by bucket (higher buckets first): a key's output
+                // position is its segment's start plus the keys of its segment above it; the
+                // stage's largest keys follow in order
+                const SelRange rg = sel_range(__ldcg(st + 8), __ldcg(st + 9));
+                for (int t = threadIdx.x; t < above; t += nth) {
+                    const unsigned long long v = sk[t];
+                    const uint32_t bk = sel_bucket(rg, (uint32_t)(v >> 32));
+                    const int lo = bk + 1 < (uint32_t)NB ? __ldcg(gh + bk + 1) : 0, hi = __ldcg(gh + bk);
+                    int r = lo;
+                    for (int q = lo; q < hi; q++) r += sk[q] > v;
+                    emit(r, v);
+                }
+                for (int t = threadIdx.x; t < want; t += nth) emit(above + t, ss[t]);
+                return;
+            }
             for (int t = threadIdx.x; t < want; t += nth) sk[above + t] = ss[t];
         } else {
-            // a crowded bucket: radix select of the want-th largest key over the stage.  Keys are
-            // taken relative to the query's smallest score key (key' = key - (umin << 32), same
-            // order); in every staged key the bits of key' from 32 + shift up are beta's, so the
-            // passes go over the bits below, 8 at a time, until the digit's keys are exactly the
-            // ones still wanted
-            const SelRange rg = sel_range(__ldcg(st + 8), __ldcg(st + 9));
-            const unsigned long long base = (unsigned long long)rg.umin << 32;
-            unsigned long long prefix = (unsigned long long)(__ldcg(st) << rg.shift) << 32;
-            unsigned long long pmask = ~0ull << (32 + rg.shift);
+            // a crowded bucket: radix select of the want-th largest key over the stage, 8 bits at a
+            // time from the top, until the digit's keys are exactly the ones still wanted
+            unsigned long long prefix = 0ull, pmask = 0ull;
             int remaining = want;
-            for (int pos = 32 + (int)rg.shift; pos > 0;) {
+            for (int pos = 64; pos > 0;) {
                 const int wb = pos >= 8 ? 8 : pos, sh = pos - wb;
                 const unsigned long long dm = (1ull << wb) - 1ull;
                 for (int t = threadIdx.x; t < 256; t += nth) hist[t] = 0;
                 __syncthreads();
                 for (int i = threadIdx.x; i < ns; i += nth) {
-                    const unsigned long long v = __ldcg(stg + i) - base;
+                    const unsigned long long v = __ldcg(stg + i);
                     if ((v & pmask) == prefix) atomicAdd(&hist[(int)((v >> sh) & dm)], 1);
                 }
                 __syncthreads();
@@ -474,13 +513,12 @@ __device__ __forceinline__ void final_of_query(int b, unsigned long long *sk, co
                 __syncthreads();
                 if (whole) break;
             }
-            // the wanted keys are exactly those with key' >= prefix (its bits below the last pass
-            // are zero)
+            // the wanted keys are exactly those >= prefix (its bits below the last pass are zero)
             if (threadIdx.x == 0) s_n = 0;
             __syncthreads();
             for (int i = threadIdx.x; i < ns; i += nth) {
                 const unsigned long long v = __ldcg(stg + i);
-                if (v - base >= prefix) {
+                if (v >= prefix) {
                     const int pos = atomicAdd(&s_n, 1);
                     if (pos < want) sk[above + pos] = v;
                 }
@@ -489,14 +527,10 @@ __device__ __forceinline__ void final_of_query(int b, unsigned long long *sk, co
     }
     block_sort_desc_u64(sk, kpow2);
     for (int r = threadIdx.x; r < k; r += nth) {
-        const int64_t o = (int64_t)b * k + r;
         if (r < nsel) {
-            const unsigned long long v = sk[r];
-            const int j = (int)~(uint32_t)(v & 0xffffffffull);  // candidate slot
-            topk_idx[o] = (j >= 0 && j < F0) ? __ldg(idx + off + j)
-                                             : ((j >= F0 && j < nc) ? (int32_t)(S + (j - F0)) : -1);
-            if (topk_score) topk_score[o] = ordered_to_float((uint32_t)(v >> 32));
+            emit(r, sk[r]);
         } else {
+            const int64_t o = (int64_t)b * k + r;
             topk_idx[o] = -1;
             if (topk_score) topk_score[o] = -INFINITY;
         }
@@ -506,12 +540,12 @@ __device__ __forceinline__ void final_of_query(int b, unsigned long long *sk, co
 // Per chunk (SORT_TH threads): keys of higher buckets appended to the query's selection, keys of
 // bucket beta to its stage; the query's last chunk to finish completes the query (final_of_query).
 // Dynamic shared memory: kpow2 + SCAP keys.
-__global__ void __launch_bounds__(SORT_TH) k_ss_write(const float *__restrict__ Y, int tau_y,
+__global__ void __launch_bounds__(SORT_TH, 1) k_ss_write(const float *__restrict__ Y, int tau_y,
                                                       const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
                                                       const float *__restrict__ tail,
                                                       const int32_t *__restrict__ tail_count, int W, int B,
                                                       const int *__restrict__ chunk_start, const int *__restrict__ chunk_query, uint32_t *state, int kcap,
-                                                      unsigned long long *sel, unsigned long long *stage,
+                                                      int *ghist, unsigned long long *sel, unsigned long long *stage,
                                                       const int32_t *__restrict__ idx, int k, int kpow2,
                                                       int32_t *__restrict__ topk_idx, float *__restrict__ topk_score)
 {
@@ -528,6 +562,7 @@ __global__ void __launch_bounds__(SORT_TH) k_ss_write(const float *__restrict__ 
     const SelRange rg = query_range(st);
     unsigned long long *out = sel + (int64_t)b * kcap;
     unsigned long long *stg = stage + q.off + (int64_t)b * W;  // capacity S_b + W
+    int *gh = ghist + (int64_t)b * NB;                          // segment starts of the buckets above beta
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     for (int base = j0; base < j1; base += SORT_TH) {
@@ -540,7 +575,11 @@ __global__ void __launch_bounds__(SORT_TH) k_ss_write(const float *__restrict__ 
             gt = every || bk > beta;
             eq = !every && bk == beta;
         }
-        const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+        const unsigned long long key64 = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);
+        // with more than k candidates a key of a higher bucket goes to its bucket's segment;
+        // otherwise every candidate is appended
+        if (gt && !every) out[atomicAdd(gh + sel_bucket(rg, u), 1)] = key64;
+        const unsigned bg = __ballot_sync(0xffffffffu, gt && every), be = __ballot_sync(0xffffffffu, eq);
         int pg = 0, pe = 0;
         if (lane == 0) {
             if (bg) pg = (int)atomicAdd(st + 4, (uint32_t)__popc(bg));
@@ -548,13 +587,13 @@ __global__ void __launch_bounds__(SORT_TH) k_ss_write(const float *__restrict__ 
         }
         pg = __shfl_sync(0xffffffffu, pg, 0);
         pe = __shfl_sync(0xffffffffu, pe, 0);
-        const unsigned long long key64 = ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j);
-        if (gt) out[pg + __popc(bg & lt)] = key64;
+        if (gt && every) out[pg + __popc(bg & lt)] = key64;
         if (eq) stg[pe + __popc(be & lt)] = key64;
     }
     // the finish counter of the query: state word 6 (zeroed by the front launch)
     if (!last_chunk_of_query((int *)(st + 6), 0, chunk_start[b + 1] - chunk_start[b])) return;
-    final_of_query(b, sk, sel, kcap, stage, state, W, idx, count, offs, k, kpow2, topk_idx, topk_score);
+    final_of_query(b, sk, sel, kcap, stage, state, ghist + (int64_t)b * NB, W, idx, count, offs, k, kpow2, topk_idx,
+                   topk_score);
 }
 
 }  // namespace stepsel

@@ -87,20 +87,22 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total)
 // no two are equal.
 constexpr int SEL_BINS = SEL_NB;
 constexpr int SEL_CAP = 4096;      // bucket keys sorted in shared memory
+constexpr int SEL_RANK_SEG = 64;   // largest bucket above beta whose keys are ranked by counting
 
 // The bin holding the `want`-th largest key of a histogram of NB bins (thread t owns NB / SEL_THREADS
 // consecutive bins, highest first): *bin_out, and *above_out = keys in higher bins.  want >= 1 and
-// at most the histogram's total.  Ends with a barrier.
+// at most the histogram's total.  Returns the keys in bins above this thread's.  Ends with a barrier.
 template <int NB>
-__device__ __forceinline__ void sel_find_bin(const unsigned int *hist, int want, int *warp_tot, int *tot, int *bin_out,
-                                             int *above_out)
+__device__ __forceinline__ int sel_find_bin(const unsigned int *hist, int want, int *warp_tot, int *tot, int *bin_out,
+                                            int *above_out)
 {
     constexpr int PER = NB / SEL_THREADS;
     const int hi = NB - PER * (int)threadIdx.x;  // bins [hi - PER, hi)
     int cnt = 0;
 #pragma unroll
     for (int q = 1; q <= PER; q++) cnt += (int)hist[hi - q];
-    int above = block_excl_scan(cnt, warp_tot, tot);
+    const int above0 = block_excl_scan(cnt, warp_tot, tot);
+    int above = above0;
     if (above < want && above + cnt >= want) {
 #pragma unroll
         for (int q = 1; q <= PER; q++) {
@@ -114,6 +116,7 @@ __device__ __forceinline__ void sel_find_bin(const unsigned int *hist, int want,
         }
     }
     __syncthreads();
+    return above0;
 }
 
 // Shared memory of k_topk_select for kpow2 and a key capacity fcap (dynamic part).
@@ -127,11 +130,14 @@ __host__ __device__ inline size_t topk_select_smem(int kpow2, int fcap)
 // candidates (read from the scores once, eight independent loads in flight per thread; a larger
 // query reads its scores from global memory at every pass).  With more than k candidates: the range
 // of the query's keys, then a histogram over 4096 buckets of that range gives the bucket beta of
-// the k-th largest key; the keys of higher buckets are appended
-// to the selection and the bucket's keys to the stage (any order: the keys carry their slots); the
-// stage sorted by key gives the bucket's largest keys.  A bucket of more than SEL_CAP keys is
-// resolved by radix passes over the bits below the bucket's and an ordered pass (the first keys
-// equal to the k-th in slot order).  The k keys are sorted by (score desc, slot asc).
+// the k-th largest key.  Each bucket above beta gets a segment of the selection (higher buckets
+// first) and its keys are scattered into it; the bucket's keys go to the stage (any order: the keys
+// carry their slots), and the stage sorted by key gives the bucket's largest keys.  When no bucket
+// above beta holds more than SEL_RANK_SEG keys, a key's output position is its segment's start plus
+// the keys of its segment above it (no sort of the selection); otherwise the k keys are sorted.  A
+// bucket beta of more than SEL_CAP keys is resolved by four radix passes over its keys and
+// an ordered pass (the first keys equal to the k-th in slot order).  The output is
+// ordered by (score desc, slot asc).
 __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__restrict__ Y,
                                                              const int32_t *__restrict__ idx,
                                                              const int32_t *__restrict__ count,
@@ -144,8 +150,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
     uint32_t *keys = (uint32_t *)(stage + SEL_CAP);
     __shared__ unsigned int hist[SEL_BINS];
     __shared__ int warp_tot[32];
-    __shared__ int tot_a, tot_b, s_bin, s_above, s_ngt, s_nst;
+    __shared__ int tot_a, tot_b, s_bin, s_above, s_ngt, s_nst, s_maxseg;
     __shared__ uint32_t s_umin, s_umax;
+    bool ranked = false;
 
     const int b = blockIdx.x / tau, i = blockIdx.x % tau;
     const int64_t off = offs[b], S = offs[b + 1] - offs[b];
@@ -161,6 +168,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
     if (threadIdx.x == 0) {
         s_umin = 0xFFFFFFFFu;
         s_umax = 0u;
+        s_maxseg = 0;
     }
     __syncthreads();
     uint32_t tmin = 0xFFFFFFFFu, tmax = 0u;  // the range of the query's score keys
@@ -208,66 +216,100 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
         const SelRange rg = sel_range(s_umin, s_umax);
         for (int j = threadIdx.x; j < F; j += SEL_THREADS) atomicAdd(&hist[sel_bucket(rg, key_at(j))], 1u);
         __syncthreads();
-        sel_find_bin<SEL_BINS>(hist, k, warp_tot, &tot_a, &s_bin, &s_above);
+        const int my_above = sel_find_bin<SEL_BINS>(hist, k, warp_tot, &tot_a, &s_bin, &s_above);
         const uint32_t beta = (uint32_t)s_bin;
         const int above = s_above;              // keys of higher buckets: all selected
         const int nbeta = (int)hist[beta];
         const bool staged = nbeta <= SEL_CAP;
         const int want = k - above;             // keys still to take from bucket beta (>= 1)
-        // higher buckets to the selection, bucket beta to the stage (appends in any order)
+        {
+            // every bucket above beta becomes the start of its segment of the selection (higher
+            // buckets first); the largest such bucket decides how the selection is ordered
+            constexpr int PER = SEL_BINS / SEL_THREADS;
+            const int hi = SEL_BINS - PER * (int)threadIdx.x;
+            int run = my_above, mx = 0;
+#pragma unroll
+            for (int q = 1; q <= PER; q++) {
+                const int bin = hi - q;
+                if (bin > (int)beta) {
+                    const int c = (int)hist[bin];
+                    hist[bin] = (unsigned int)run;
+                    run += c;
+                    mx = max(mx, c);
+                }
+            }
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            if (lane == 0) atomicMax(&s_maxseg, mx);
+        }
+        __syncthreads();
+        // higher buckets scattered to their segments, bucket beta to the stage (any order)
         for (int base = 0; base < F; base += SEL_THREADS) {
             const int j = base + threadIdx.x;
-            uint32_t u = 0;
-            bool gt = false, eq = false;
+            uint32_t u = 0, bk = 0;
+            bool eq = false;
             if (j < F) {
                 u = key_at(j);
-                const uint32_t bk = sel_bucket(rg, u);
-                gt = bk > beta;
+                bk = sel_bucket(rg, u);
+                if (bk > beta) sel[atomicAdd(&hist[bk], 1u)] = key64(u, j);
                 eq = staged && bk == beta;
             }
-            const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
-            int pg = 0, pe = 0;
-            if (lane == 0) {
-                if (bg) pg = atomicAdd(&s_ngt, __popc(bg));
-                if (be) pe = atomicAdd(&s_nst, __popc(be));
-            }
-            pg = __shfl_sync(0xffffffffu, pg, 0);
+            const unsigned be = __ballot_sync(0xffffffffu, eq);
+            int pe = 0;
+            if (lane == 0 && be) pe = atomicAdd(&s_nst, __popc(be));
             pe = __shfl_sync(0xffffffffu, pe, 0);
-            if (gt) sel[pg + __popc(bg & lt)] = key64(u, j);
             if (eq) stage[pe + __popc(be & lt)] = key64(u, j);
         }
         __syncthreads();
+        ranked = staged && s_maxseg <= SEL_RANK_SEG;
         if (staged) {
             int np = 64;
             while (np < nbeta) np <<= 1;
             for (int t = nbeta + threadIdx.x; t < np; t += SEL_THREADS) stage[t] = 0ull;
             block_sort_desc_u64(stage, np);
+            if (ranked) {
+                // output position of a selected key = its segment's start + the keys of the segment
+                // above it; the stage's largest keys follow in order
+                const int64_t o0 = ((int64_t)b * tau + i) * k;
+                for (int t = threadIdx.x; t < above; t += SEL_THREADS) {
+                    const unsigned long long v = sel[t];
+                    const uint32_t bk = sel_bucket(rg, (uint32_t)(v >> 32));
+                    const int lo = bk + 1 < (uint32_t)SEL_BINS ? (int)hist[bk + 1] : 0, hi = (int)hist[bk];
+                    int r = lo;
+                    for (int q = lo; q < hi; q++) r += sel[q] > v;
+                    const int jj = (int)~(uint32_t)(v & 0xffffffffull);
+                    topk_idx[o0 + r] = __ldg(idx + off + jj);
+                    if (topk_score) topk_score[o0 + r] = ordered_to_float((uint32_t)(v >> 32));
+                }
+                for (int t = threadIdx.x; t < want; t += SEL_THREADS) {
+                    const unsigned long long v = stage[t];
+                    const int jj = (int)~(uint32_t)(v & 0xffffffffull);
+                    topk_idx[o0 + above + t] = __ldg(idx + off + jj);
+                    if (topk_score) topk_score[o0 + above + t] = ordered_to_float((uint32_t)(v >> 32));
+                }
+                return;
+            }
             for (int t = threadIdx.x; t < want; t += SEL_THREADS) sel[above + t] = stage[t];
         } else {
-            // a crowded bucket: radix passes of up to 8 bits over the offsets d = u - umin below
-            // the bucket's bits give the k-th key K; then the bucket's keys above K and the first
-            // keys equal to K in slot order
-            uint32_t dprefix = beta << rg.shift, dmask = 0xFFFFFFFFu << rg.shift;
+            // a crowded bucket: four radix passes of 8 bits over the keys of bucket beta give the
+            // k-th key K; then the bucket's keys above K and the first keys equal to K in slot order
+            uint32_t prefix = 0u, pmask = 0u;
             int remaining = want;
 #pragma unroll 1
-            for (int pos = (int)rg.shift; pos > 0;) {
-                const int wbits = pos >= 8 ? 8 : pos, sh = pos - wbits;
-                const uint32_t bins = (1u << wbits) - 1u;
+            for (int pass = 0; pass < 4; pass++) {
+                const int sh = 24 - 8 * pass;
                 for (int t = threadIdx.x; t < 1024; t += SEL_THREADS) hist[t] = 0;
                 __syncthreads();
                 for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
-                    const uint32_t u = key_at(j), d = u > rg.umin ? u - rg.umin : 0u;
-                    if ((d & dmask) == dprefix) atomicAdd(&hist[(d >> sh) & bins], 1u);
+                    const uint32_t u = key_at(j);
+                    if ((u & pmask) == prefix && sel_bucket(rg, u) == beta) atomicAdd(&hist[(u >> sh) & 255u], 1u);
                 }
                 __syncthreads();
                 sel_find_bin<1024>(hist, remaining, warp_tot, &tot_a, &s_bin, &s_above);
-                dprefix |= (uint32_t)s_bin << sh;
+                prefix |= (uint32_t)s_bin << sh;
                 remaining -= s_above;
-                dmask |= bins << sh;
-                pos = sh;
+                pmask |= 255u << sh;
                 __syncthreads();
             }
-            const uint32_t prefix = rg.umin + dprefix;  // the k-th largest score key
             int cg = 0, ce = 0;
             for (int base = 0; base < F; base += SEL_THREADS) {
                 const int j = base + threadIdx.x;

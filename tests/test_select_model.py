@@ -1,24 +1,24 @@
 """Numpy models of the two Top-k selects' steps against a plain sort (key descending, ties to the
 smaller slot), on the CPU.
 
-Both selects bucket a query's order-preserving score keys u over the query's own key range:
-bucket(u) = (u - umin) >> shift, with the smallest shift that leaves at most 4,096 buckets.
+Both selects bucket a query's scores linearly over the query's own score range:
+bucket = floor((y - ymin) * 4096 / (ymax - ymin)) in fp32, clamped to [0, 4096), NaN to the end its
+key sorts to; the bucket never decreases along the key order.
 
 Decode-step select (csrc/step_select.cuh): over chunks of 2,048 candidates, a histogram of the
 buckets gives the bucket of the k-th largest key; keys of higher buckets go to the selection and the
 bucket's keys to a stage, both in an arbitrary order (the model shuffles them), because every key
 carries its slot: key64 = (score key << 32) | ~slot orders by score, then smaller slot, and no two
 keys are equal.  The bucket's largest keys come from a sort (at most SCAP staged keys) or, for a
-crowded bucket, a radix select over the stage on key64 - (umin << 32), 8 bits at a time below the
-bucket's bits, stopping once a digit holds exactly the keys still wanted; one sort orders the k
+crowded bucket, a radix select over the stage's 64-bit keys, 8 bits at a time from the top, stopping
+once a digit holds exactly the keys still wanted; one sort orders the k
 keys.  With at most k candidates the select takes every candidate whatever its key, including a key
 that orders as 0.
 
 Batched select (csrc/topk.cuh, k_topk_select): the same histogram over all keys gives the bucket of
 the k-th key; keys of higher buckets and the bucket's keys (at most SEL_CAP of them) are appended in
 any order, and the stage sorted by 64-bit key gives the bucket's largest keys; a crowded bucket
-takes radix passes of up to 8 bits over u - umin below the bucket's bits and an ordered pass
-instead.
+takes four radix passes of 8 bits over the bucket's keys and an ordered pass instead.
 
 The cases cover heavy ties in every digit, all-equal keys, keys of 0, a narrow and a wide key range
 (one outlier far above the rest), k at and above the candidate count, and empty queries.
@@ -47,14 +47,28 @@ def key64(u):
     return (u.astype(np.uint64) << np.uint64(32)) | (~slots & np.uint64(0xFFFFFFFF))
 
 
+def _ordered_to_float(u):
+    u = np.asarray(u, dtype=np.uint32)
+    b = np.where(u & np.uint32(0x80000000), u & np.uint32(0x7FFFFFFF), ~u).astype(np.uint32)
+    return b.view(np.float32)
+
+
 def sel_range(u):
-    """(umin, shift) of a query's keys: the smallest shift leaving at most 4,096 buckets."""
-    umin, umax = int(u.min()), int(u.max())
-    return umin, max(0, (umax - umin).bit_length() - 12)
+    """(ymin, scale) of a query's keys: 4,096 buckets linear in the score over [ymin, ymax]."""
+    ymin = _ordered_to_float(np.array([u.min()]))[0]
+    with np.errstate(invalid="ignore", over="ignore"):  # NaN / infinite ends, spans below 2^-114
+        span = np.float32(_ordered_to_float(np.array([u.max()]))[0] - ymin)
+        scale = np.float32(np.float32(4096.0) / span) if span > 0 else np.float32(0.0)
+    return ymin, scale
 
 
-def sel_bucket(u, umin, shift):
-    return np.minimum((u.astype(np.int64) - umin) >> shift, 4095)
+def sel_bucket(u, ymin, scale):
+    y = _ordered_to_float(u)
+    with np.errstate(invalid="ignore", over="ignore"):
+        t = (y - ymin).astype(np.float32) * scale
+        bk = np.where(t >= np.float32(4095), 4095, np.where(t > 0, t, 0).astype(np.int64))
+    nan = np.isnan(y)
+    return np.where(nan, np.where(np.asarray(u) & np.uint32(0x80000000), 4095, 0), bk).astype(np.int64)
 
 
 def select_model(u, k, scap=8192, seed=0):
@@ -68,8 +82,8 @@ def select_model(u, k, scap=8192, seed=0):
     if nc <= k:
         slots = rng.permutation(nc)
     else:
-        umin, shift = sel_range(u)
-        bk = sel_bucket(u, umin, shift)
+        ymin, scale = sel_range(u)
+        bk = sel_bucket(u, ymin, scale)
         hist = np.bincount(bk, minlength=4096)
         beta, above = _find_bin(hist, k)
         gt = rng.permutation(np.nonzero(bk > beta)[0])
@@ -79,10 +93,9 @@ def select_model(u, k, scap=8192, seed=0):
         if staged.size <= scap:
             top = staged[np.lexsort((staged, -u[staged].astype(np.int64)))][:want]
         else:
-            v = kk[staged] - (np.uint64(umin) << np.uint64(32))
-            prefix = np.uint64(beta << shift) << np.uint64(32)
-            pmask = np.uint64((0xFFFFFFFFFFFFFFFF << (32 + shift)) & 0xFFFFFFFFFFFFFFFF)
-            rem, pos = want, 32 + shift
+            v = kk[staged]
+            prefix, pmask = np.uint64(0), np.uint64(0)
+            rem, pos = want, 64
             while pos > 0:
                 wb = min(8, pos)
                 sh = pos - wb
@@ -152,16 +165,16 @@ def batched_select_model(u, k, cap=4096, seed=0):
     """The batched call's select (k_topk_select): a histogram over the query's key range gives the
     bucket beta of the k-th key; keys of higher buckets and (at most `cap`) keys of bucket beta are
     appended in any order (shuffled here), the stage sorted by 64-bit key gives the bucket's largest
-    keys; a crowded bucket takes radix passes over u - umin below the bucket's bits and an ordered
-    pass; returns the selected slots in output order."""
+    keys; a crowded bucket takes four radix passes over the bucket's keys and an ordered pass;
+    returns the selected slots in output order."""
     rng = np.random.default_rng(seed)
     F = u.size
     kk = key64(u)
     if F <= k:
         slots = rng.permutation(F)
     else:
-        umin, shift = sel_range(u)
-        bk = sel_bucket(u, umin, shift)
+        ymin, scale = sel_range(u)
+        bk = sel_bucket(u, ymin, scale)
         hist = np.bincount(bk, minlength=4096)
         beta, above = _find_bin(hist, k)
         sel = rng.permutation(np.nonzero(bk > beta)[0])
@@ -171,20 +184,15 @@ def batched_select_model(u, k, cap=4096, seed=0):
             staged = rng.permutation(np.nonzero(bk == beta)[0])
             top = staged[np.argsort(kk[staged])[::-1]][:want]
         else:
-            d_all = u.astype(np.int64) - umin
-            dprefix, dmask, remaining, pos = beta << shift, (0xFFFFFFFF << shift) & 0xFFFFFFFF, want, shift
-            while pos > 0:
-                wb = min(8, pos)
-                sh = pos - wb
-                bins = (1 << wb) - 1
-                m = (d_all & dmask) == dprefix
-                h = np.bincount((d_all[m] >> sh) & bins, minlength=1024)
+            prefix, pmask, remaining = 0, 0, want
+            inb_mask = bk == beta
+            for sh in (24, 16, 8, 0):
+                m = inb_mask & ((u & np.uint32(pmask)) == prefix)
+                h = np.bincount((u[m] >> np.uint32(sh)) & np.uint32(255), minlength=1024)
                 d, ab = _find_bin(h, remaining)
-                dprefix |= d << sh
+                prefix |= d << sh
                 remaining -= ab
-                dmask |= bins << sh
-                pos = sh
-            prefix = umin + dprefix
+                pmask |= 255 << sh
             inb = np.arange(F)[bk == beta]
             gt = [j for j in inb if u[j] > prefix]
             eq = [j for j in inb if u[j] == prefix][:remaining]
@@ -260,3 +268,48 @@ def test_block_sort_model_sorts(n):
             v = np.zeros(n, dtype=np.uint64)
             v[: n // 3] = rng.integers(1, 2 ** 40, n // 3, dtype=np.uint64)
         assert np.array_equal(block_sort_desc_model(v), np.sort(v)[::-1]), (n, kind)
+
+
+# ------------------------------------------------------------------ selection order without a sort
+
+def ranked_order_model(u, k, seed=0):
+    """Both selects' ordering of the selection when no bucket above beta is large: every bucket
+    above beta gets a segment of the selection (higher buckets first, each segment's start the keys
+    of the buckets above it), its keys are scattered into it in any order (shuffled here), and a
+    key's output position is its segment's start plus the keys of its segment above it; the k-th
+    key's bucket's largest keys follow in key order.  Returns (slots in output order, largest
+    segment)."""
+    rng = np.random.default_rng(seed)
+    kk = key64(u)
+    ymin, scale = sel_range(u)
+    bk = sel_bucket(u, ymin, scale)
+    hist = np.bincount(bk, minlength=4096)
+    beta, above = _find_bin(hist, k)
+    start = np.zeros(4097, dtype=np.int64)       # start[b] = keys in buckets above b (b > beta)
+    start[:4096] = np.cumsum(hist[::-1])[::-1] - hist
+    sel = np.zeros(above, dtype=np.uint64)
+    fill = start.copy()
+    for j in rng.permutation(np.nonzero(bk > beta)[0]):
+        sel[fill[bk[j]]] = kk[j]
+        fill[bk[j]] += 1
+    out = np.zeros(k, dtype=np.uint64)
+    for t in range(above):
+        v = sel[t]
+        b = sel_bucket(np.array([v >> np.uint64(32)], dtype=np.uint32), ymin, scale)[0]
+        lo = fill[b + 1] if b + 1 < 4096 else 0  # the end of the next bucket up is this one's start
+        hi = fill[b]
+        out[lo + int((sel[lo:hi] > v).sum())] = v
+    staged = np.nonzero(bk == beta)[0]
+    out[above:] = np.sort(kk[staged])[::-1][:k - above]
+    slots = (~out & np.uint64(0xFFFFFFFF)).astype(np.int64)
+    return slots, int(hist[beta + 1:].max()) if beta + 1 < 4096 else 0
+
+
+@pytest.mark.parametrize("kind", ["random", "ties_every_digit", "ties_low_digits", "narrow_with_outlier", "float"])
+def test_ranked_order_equals_plain_sort(kind):
+    rng = np.random.default_rng(zlib.crc32((kind + "ranked").encode()))
+    for nc in (2049, 5000, 31000):
+        for k in (1, 7, 512, 2048):
+            u = keys(rng, kind, nc)
+            slots, _ = ranked_order_model(u, k, seed=nc + k)
+            assert np.array_equal(slots, plain_sort(u, k)), (kind, nc, k)
