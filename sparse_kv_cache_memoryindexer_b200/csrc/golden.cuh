@@ -67,6 +67,20 @@ __device__ __forceinline__ double block_sum(double v, double *red)
     return r;
 }
 
+// Appends v to cand when `take` (at most CAND entries; *counter counts every append, so a count
+// above CAND tells that some did not fit): one shared atomic per warp.  Every lane of the warp calls.
+__device__ __forceinline__ void warp_append(bool take, unsigned long long v, int *counter, unsigned long long *cand)
+{
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (!m) return;
+    const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(counter, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    const int at = base + __popc(m & ((1u << lane) - 1u));
+    if (take && at < CAND) cand[at] = v;
+}
+
 // Block-wide inclusive scan of one double per thread: returns this thread's inclusive prefix and
 // the block total in *total.  red: THREADS / 32 doubles.  Starts and ends with a barrier.
 __device__ __forceinline__ double block_incl_scan_d(double v, double *red, double *total)
@@ -163,16 +177,15 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
         // (2^-22 relative) and z - m is rounded once (an error of 2^-24 |x| in the exponent); a
         // result below the smallest normal is off by at most 2^-126 absolute
         double z32 = 0.0, zx = 0.0;
-        for (int64_t s = threadIdx.x; s < S; s += THREADS) {
-            const float zs = __ldg(row + s);
+        for (int64_t base = 0; base < S; base += THREADS) {  // whole warps per step (warp-wide appends)
+            const int64_t s = base + threadIdx.x;
+            const float zs = s < S ? __ldg(row + s) : -INFINITY;
             const float x = zs - m;
-            const float e = expf(x);
+            const float e = s < S ? expf(x) : 0.f;
             z32 += (double)e;
-            zx += (double)e * (double)(-x);
-            if (m - zs < 8.f) {
-                const int at = atomicAdd(&s_nc, 1);
-                if (at < CAND) cand[at] = ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s);
-            }
+            zx += s < S ? (double)e * (double)(-x) : 0.0;
+            warp_append(s < S && m - zs < 8.f,
+                        ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s), &s_nc, cand);
         }
         double Z32 = block_sum(z32, dred);
         const double ZX = block_sum(zx, dred);
@@ -210,7 +223,7 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
                             keep = m - ordered_to_float((uint32_t)(v >> 32)) < 4.f;
                         }
                         __syncthreads();  // every entry of this block read before any is overwritten
-                        if (keep) cand[atomicAdd(&s_n4, 1)] = v;
+                        warp_append(keep, v, &s_n4, cand);
                         __syncthreads();
                     }
                     nc = s_n4;
@@ -300,13 +313,11 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     if (s_depth >= 0) {
         // ---- candidate path: the entries within depth(k) of the maximum, sorted
         const float D = depth(s_depth);
-        for (int64_t s = threadIdx.x; s < S; s += THREADS) {
-            const float zs = row[s];
-            if (m - zs < D) {
-                const int at = atomicAdd(&s_nc, 1);
-                if (at < CAND)
-                    cand[at] = ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s);
-            }
+        for (int64_t base = 0; base < S; base += THREADS) {
+            const int64_t s = base + threadIdx.x;
+            const float zs = s < S ? row[s] : -INFINITY;
+            warp_append(s < S && m - zs < D,
+                        ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s), &s_nc, cand);
         }
         __syncthreads();
         const int nc = s_nc < CAND ? s_nc : CAND;

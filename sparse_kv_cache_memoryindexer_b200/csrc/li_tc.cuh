@@ -25,6 +25,13 @@
 
 namespace lsa {
 
+// A work item as the planner writes it, so that a claim costs one table read (two 16-byte loads).
+struct __align__(16) ItemInfo {
+    int b, g, t0, t1;  // sequence, query group, key tiles [t0, t1)
+    int F, S;          // fetched entries and length of the sequence
+    long long off;     // its first entry
+};
+
 namespace li {
 
 constexpr int NQ = 4;              // decode queries per MMA (batched call; one decode step: 1)
@@ -41,6 +48,7 @@ struct Params {
     const int32_t *count;    // [B]
     const int64_t *offs;     // [B+1]
     const int *item_start;   // [B+1]
+    const ItemInfo *items;   // [items] the planner's table
     int *item_counter;       // next unclaimed item, zeroed by k_li_items
     float *Y;                // [tau*T]
     uint32_t *range;         // one decode step (nq = 1): per sequence b, words range[b*range_stride]
@@ -67,33 +75,45 @@ struct Smem {
     }
 };
 
-struct Item {
-    int b, c, g;
-};
 
-__device__ __forceinline__ Item decode_item(const int *item_start, int B, int groups, int it)
+// Table entries of sequence b's items (items it0 ..): chunk c of ch key tiles and query group g at
+// it0 + c groups + g.  The lanes of one warp write them.
+__device__ __forceinline__ void write_items(ItemInfo *items, int it0, int b, int F, int S, int64_t off, int groups,
+                                           int ch, int lane)
 {
-    int lo = 0, hi = B;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(item_start + mid) <= it) lo = mid;
-        else hi = mid;
+    const int tiles = (F + TILE - 1) / TILE, nch = (tiles + ch - 1) / ch;
+    for (int r = lane; r < nch * groups; r += 32) {
+        const int c = r / groups;
+        ItemInfo x;
+        x.b = b;
+        x.g = r % groups;
+        x.t0 = c * ch;
+        x.t1 = min(tiles, (c + 1) * ch);
+        x.F = F;
+        x.S = S;
+        x.off = off;
+        items[it0 + r] = x;
     }
-    const int r = it - __ldg(item_start + lo);
-    return Item{lo, r / groups, r % groups};
 }
 
-__device__ __forceinline__ int fetched_count(const Params &p, int b, int64_t &S)
+__device__ __forceinline__ ItemInfo load_item(const ItemInfo *items, int it)
 {
-    S = __ldg(p.offs + b + 1) - __ldg(p.offs + b);
-    int F = __ldg(p.count + b);
-    return F < 0 ? 0 : (F > S ? (int)S : F);
+    const int4 a = __ldg((const int4 *)(items + it)), c = __ldg((const int4 *)(items + it) + 1);
+    ItemInfo x;
+    x.b = a.x;
+    x.g = a.y;
+    x.t0 = a.z;
+    x.t1 = a.w;
+    x.F = c.x;
+    x.S = c.y;
+    x.off = (long long)(((unsigned long long)(uint32_t)c.w << 32) | (uint32_t)c.z);
+    return x;
 }
 
-// work items per sequence: ceil(ceil(F/128)/ch) chunks x groups.  One block.
+// work items per sequence: ceil(ceil(F/128)/ch) chunks x groups, and their table.  One block.
 __global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
                                                    int B, int groups, int ch, int *__restrict__ item_start,
-                                                   int *__restrict__ item_counter)
+                                                   int *__restrict__ item_counter, ItemInfo *__restrict__ items)
 {
     __shared__ int warp_tot[32];
     __shared__ int carry;
@@ -128,6 +148,13 @@ __global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ c
         __syncthreads();
         if (threadIdx.x == blockDim.x - 1) carry = pos;
         __syncthreads();
+    }
+    // the table, a warp per sequence (item_start was written by this block: visible after the barrier)
+    for (int b = warp; b < B; b += (int)(blockDim.x >> 5)) {
+        const int64_t off = offs[b], S = offs[b + 1] - off;
+        int F = count[b];
+        F = F < 0 ? 0 : (F > S ? (int)S : F);
+        write_items(items, item_start[b], b, F, (int)S, off, groups, ch, lane);
     }
 }
 
@@ -205,19 +232,17 @@ __global__ void __launch_bounds__(320, 1)
             bool ok = true;
             int islot = 0;
             uint32_t iphase = 0;
+            int claim = atomicAdd(p.item_counter, 1);
             while (ok) {
-                const int claim = atomicAdd(p.item_counter, 1);
                 const int it = claim < NI ? claim : -1;  // -1: no work left, the consumers stop
                 if (!mbar_wait(iempty(islot), iphase ^ 1, abort_flag)) { ok = false; break; }
                 ring[islot] = it;
                 mbar_arrive(ifull(islot));  // release: the ring entry is visible to the waiters
                 if (++islot == NRING) { islot = 0; iphase ^= 1; }
                 if (it < 0) break;
-                const Item w = decode_item(p.item_start, B, p.groups, it);
-                int64_t S;
-                const int F = fetched_count(p, w.b, S);
-                const int ntiles = (F + TILE - 1) / TILE;
-                const int t0 = w.c * p.ch, t1 = min(ntiles, t0 + p.ch);
+                const ItemInfo w = load_item(p.items, it);
+                claim = atomicAdd(p.item_counter, 1);  // the next claim, in flight while this item's loads go out
+                const int t0 = w.t0, t1 = w.t1;
                 qslot ^= 1;
                 if (!mbar_wait(qempty(qslot), (quse[qslot] & 1) ^ 1, abort_flag)) { ok = false; break; }
                 quse[qslot]++;
@@ -226,7 +251,7 @@ __global__ void __launch_bounds__(320, 1)
                 const int qrow = (w.b * p.tau + NQV * w.g) * NH;
                 tma_load_2d(qd, &qmap, 0, qrow, qfull(qslot));
                 tma_load_2d(qd + (uint32_t)ncol * 128, &qmap, 64, qrow, qfull(qslot));
-                const int64_t off = __ldg(p.offs + w.b);
+                const int64_t off = w.off;
                 for (int kt = t0; kt < t1; kt++) {
                     if (!mbar_wait(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
                     mbar_expect_tx(full(stage), kbytes);
@@ -261,11 +286,8 @@ __global__ void __launch_bounds__(320, 1)
                 mbar_arrive(iempty(islot));
                 if (++islot == NRING) { islot = 0; iphase ^= 1; }
                 if (it < 0) break;
-                const Item w = decode_item(p.item_start, B, p.groups, it);
-                int64_t S;
-                const int F = fetched_count(p, w.b, S);
-                const int ntiles = (F + TILE - 1) / TILE;
-                const int t0 = w.c * p.ch, t1 = min(ntiles, t0 + p.ch);
+                const ItemInfo w = load_item(p.items, it);
+                const int t0 = w.t0, t1 = w.t1;
                 qslot ^= 1;
                 if (!mbar_wait(qfull(qslot), quse[qslot] & 1, abort_flag)) { ok = false; break; }
                 quse[qslot]++;
@@ -310,17 +332,16 @@ __global__ void __launch_bounds__(320, 1)
             if (lane == 0) mbar_arrive(iempty(islot));
             if (++islot == NRING) { islot = 0; iphase ^= 1; }
             if (it < 0) break;
-            const Item w = decode_item(p.item_start, B, p.groups, it);
-            int64_t S;
-            const int F = fetched_count(p, w.b, S);
-            const int ntiles = (F + TILE - 1) / TILE;
-            const int t0 = w.c * p.ch, t1 = min(ntiles, t0 + p.ch);
+            const ItemInfo w = load_item(p.items, it);
+            const int64_t S = w.S;
+            const int F = w.F;
+            const int t0 = w.t0, t1 = w.t1;
             const int i0 = NQV * w.g + 2 * half;  // first of this warp's queries
             __syncwarp();
             for (int t = lane; t < nqw * NH; t += 32)
                 myw[t] = __ldg(p.wd + ((int64_t)w.b * p.tau + i0 + t / NH) * NH + (t % NH));
             __syncwarp();
-            const int64_t off = __ldg(p.offs + w.b);
+            const int64_t off = w.off;
             float *Yb = p.Y + (int64_t)p.tau * off;
             uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // score keys of this warp's entries of the item
             for (int kt = t0; kt < t1; kt++) {
@@ -417,17 +438,24 @@ inline bool li_tc_supported(int n_h, int d_I, int tau, int kdt, int nq = li::NQ)
 // largest order-preserving score key are folded into range[b * range_stride] and [+ 1].
 inline int li_item_tiles(int nq) { return nq == li::NQ ? li::CH : li::CH_STEP; }
 
+// Upper bound on the work items of a call (sum over sequences of ceil(ceil(F_b/128)/ch) x groups).
+inline int64_t li_max_items(int B, int64_t T, int tau, int nq)
+{
+    const int ch = li_item_tiles(nq);
+    return (T / ((int64_t)TILE * ch) + B + 1) * (int64_t)(tau / nq);
+}
+
 inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK, const float *hsc,
                                const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, int nq, float *Y,
-                               int *item_start, int *item_counter, int sms, cudaStream_t st, int *launches,
-                               bool planned = false, uint32_t *range = nullptr, int range_stride = 0)
+                               int *item_start, int *item_counter, ItemInfo *items, int sms, cudaStream_t st,
+                               int *launches, bool planned = false, uint32_t *range = nullptr, int range_stride = 0)
 {
     using namespace li;
     *launches = 0;
     if (nq != NQ && nq != 1) return LSA_ERR_UNSUPPORTED;
     const int ch = li_item_tiles(nq);
     if (!planned) {
-        k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / nq, ch, item_start, item_counter);
+        k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / nq, ch, item_start, item_counter, items);
         (*launches)++;
     }
     if (T == 0) return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
@@ -441,6 +469,7 @@ inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK
     p.count = count;
     p.offs = offs;
     p.item_start = item_start;
+    p.items = items;
     p.item_counter = item_counter;
     p.Y = Y;
     p.range = range;

@@ -277,7 +277,7 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
         const ProjProblem cw[2] = {{W_dq, pc, r, true}, {W_w, pw, n_h, true}};
         const bool split[2] = {true, true};
         int ks[2] = {1, 1};
-        lsa_status s = launch_proj_tc(h, cw, split, 2, L, B, d, sms, 2, st, ks);
+        lsa_status s = launch_proj_tc(h, cw, split, 2, L, B, d, sms, st, ks);
         if (s == LSA_OK) s = launched("project c and w (tensor cores)");
         if (s == LSA_OK) {
             k_proj_reduce<<<(unsigned)std::min<int64_t>((nc + nw + 255) / 256, (int64_t)sms * 8), 256, 0, st>>>(
@@ -286,7 +286,7 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
         }
         const ProjProblem qp = {W_iuq, q_out, nq, false};
         const bool nosplit = false;
-        if (s == LSA_OK) s = launch_proj_tc(c, &qp, &nosplit, 1, L, B, r, sms, 2, st);
+        if (s == LSA_OK) s = launch_proj_tc(c, &qp, &nosplit, 1, L, B, r, sms, st);
         if (s == LSA_OK) s = launched("project q (tensor cores)");
         if (s != LSA_OK) return fail(s, "lsa_project: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
     } else if (dt == LSA_BF16) {
@@ -528,12 +528,19 @@ return ok();
 
 // ------------------------------------------------------------------------------ stage 5
 
-// Workspace of lsa_lightning_topk: [item_start: B+1 ints, item counter: 1 int][Y: tau * total_S floats].
+// Workspace of lsa_lightning_topk: [item_start: B+1 ints, item counter: 1 int][item table]
+// [Y: tau * total_S floats].
+static size_t topk_items_bytes(int B, int tau, int64_t total_S)
+{
+    return align_up(sizeof(ItemInfo) * (size_t)li_max_items(B, total_S, tau < li::NQ ? li::NQ : tau, li::NQ), 256);
+}
+
 size_t lsa_lightning_topk_workspace_size(int B, int tau, int64_t total_S, int k)
 {
     (void)k;
     if (B <= 0 || tau <= 0 || total_S < 0) return 0;
-    return align_up(sizeof(int) * (size_t)(B + 2), 256) + align_up(sizeof(float) * (size_t)tau * (size_t)total_S, 256);
+    return align_up(sizeof(int) * (size_t)(B + 2), 256) + topk_items_bytes(B, tau, total_S) +
+           align_up(sizeof(float) * (size_t)tau * (size_t)total_S, 256);
 }
 
 lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void *hot_K, const float *hot_scale,
@@ -556,14 +563,15 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     if (n_h > 128) return fail(LSA_ERR_UNSUPPORTED, "lsa_lightning_topk: n_h must be <= 128");
     int *item_start = (int *)workspace;
     int *item_counter = item_start + B + 1;
-    float *Y = (float *)((char *)workspace + align_up(sizeof(int) * (size_t)(B + 2), 256));
+    ItemInfo *items = (ItemInfo *)((char *)workspace + align_up(sizeof(int) * (size_t)(B + 2), 256));
+    float *Y = (float *)((char *)items + topk_items_bytes(B, tau, total_S));
     // E4M3 keys arrive here decoded to bf16 by lsa_fetch_gather (scales in hot_scale)
     const int hdt = (kdt == LSA_FP8_E4M3) ? (int)DT_BF16 : (int)kdt;
     if (li_tc_supported(n_h, d_I, tau, kdt)) {
         LSA_REQUIRE(aligned(q_dec, 16) && aligned(hot_K, 16), "lsa_lightning_topk: q_dec and hot_K must be 16-byte aligned");
         int n = 0;
         const lsa_status s = launch_li_tc(q_dec, w_dec, hot_K, hot_scale, count, seq_offsets, B, total_S, tau, li::NQ,
-                                          Y, item_start, item_counter, num_sms(), st, &n);
+                                          Y, item_start, item_counter, items, num_sms(), st, &n);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK) return fail(s, "lsa_lightning_topk: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
     } else {
@@ -619,7 +627,8 @@ static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[6])
 
 static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[6])
 {
-    part[0] = align_up(sizeof(int) * (size_t)(B + 2), 256);
+    part[0] = align_up(sizeof(int) * (size_t)(B + 2), 256) +
+              align_up(sizeof(ItemInfo) * (size_t)li_max_items(B, total_S, 1, 1), 256);
     part[1] = align_up(sizeof(float) * (size_t)(total_S > 0 ? total_S : 1), 256);
     part[2] = align_up(sizeof(float) * (size_t)B * (W > 0 ? W : 1), 256);
     part[3] = align_up((size_t)4 * B * n_h * d_I, 256);
@@ -667,6 +676,7 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     char *p = (char *)workspace;
     int *item_start = (int *)p;
     int *item_counter = item_start + B + 1;
+    ItemInfo *items = (ItemInfo *)(p + align_up(sizeof(int) * (size_t)(B + 2), 256));
     float *Y = (float *)(p + part[0]);
     float *tail = (float *)(p + part[0] + part[1]);
     void *qw = (void *)(p + part[0] + part[1] + part[2]);
@@ -701,6 +711,7 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         fp.ch = li_item_tiles(1);
         fp.item_start = item_start;
         fp.item_counter = item_counter;
+        fp.items = items;
         fp.chunk_start = chunk_start;
         fp.chunk_query = chunk_query;
         fp.state = state;
@@ -733,7 +744,8 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         LSA_REQUIRE(aligned(hot_K, 16), "lsa_lightning_topk_step: hot_K must be 16-byte aligned");
         int n = 0;
         const lsa_status s = launch_li_tc(qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, TQ, 1, Y, item_start,
-                                          item_counter, num_sms(), st, &n, /*planned=*/true, state + 8, stepsel::NS);
+                                          item_counter, items, num_sms(), st, &n, /*planned=*/true, state + 8,
+                                          stepsel::NS);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK)
             return fail(s, "lsa_lightning_topk_step: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));

@@ -26,7 +26,8 @@ namespace lsa {
 
 namespace proj {
 
-constexpr int KB = 64;              // K elements per stage (one 128-byte swizzle atom of bf16)
+constexpr int KB = 64;              // K elements per box (one 128-byte swizzle atom of bf16)
+constexpr int MAX_BOX = 4;          // boxes per stage: 512 contiguous bytes of every weight row
 constexpr int KSPLIT_MAX = 8;       // K ranges of a split problem (partial slices)
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 6 * 32;
@@ -49,6 +50,7 @@ struct Params {
     int L, B, K;        // layers, batch, reduction length
     int NB;             // MMA N = B rounded up to 16
     int stages;
+    int nbox;           // K boxes per stage
 };
 
 struct Unit {
@@ -81,8 +83,12 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int u, int nkb)
 }
 
 __host__ __device__ inline uint32_t b_bytes(int NB) { return (uint32_t)NB * KB * 2; }
-__host__ __device__ inline uint32_t stage_bytes(int NB) { return A_BYTES + b_bytes(NB); }
-__host__ __device__ inline uint32_t smem_total(int NB, int stages) { return stage_bytes(NB) * stages + 8 * (2 * MAX_STAGES + 4) + 64 + 1024; }
+// a stage: nbox weight boxes (128 rows x 64 K each), then nbox X boxes (NB rows x 64 K each)
+__host__ __device__ inline uint32_t stage_bytes(int NB, int nbox) { return (uint32_t)nbox * (A_BYTES + b_bytes(NB)); }
+__host__ __device__ inline uint32_t smem_total(int NB, int stages, int nbox)
+{
+    return stage_bytes(NB, nbox) * stages + 8 * (2 * MAX_STAGES + 4) + 64 + 1024;
+}
 // TMEM columns per accumulator: N rounded up to 32, so that 32-column loads stay inside it.
 __host__ __device__ inline uint32_t acc_cols(int NB) { return (uint32_t)(NB + 31) / 32 * 32; }
 __host__ __device__ inline uint32_t tmem_cols(int NB)  // two accumulators, a power of two >= 32
@@ -100,7 +106,7 @@ __global__ void __launch_bounds__(THREADS)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(base);
-    const uint32_t sbytes = stage_bytes(p.NB);
+    const uint32_t sbytes = stage_bytes(p.NB, p.nbox), bbox = b_bytes(p.NB);
     const uint32_t bars = sbase + sbytes * p.stages;
     auto full = [&](int i) { return bars + 8u * i; };
     auto empty = [&](int i) { return bars + 8u * (MAX_STAGES + i); };
@@ -154,13 +160,17 @@ __global__ void __launch_bounds__(THREADS)
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const Unit x = unit_of(p, u, nkb);
             const CUtensorMap *wm = x.prob == 0 ? &wmap0 : &wmap1;
-            for (int kb = x.kb0; kb < x.kb1; kb++) {
+            for (int kb = x.kb0; kb < x.kb1; kb += p.nbox) {
+                const int nb = min(p.nbox, x.kb1 - kb);
                 if (!mbar_wait_warp(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
                 if (leader) {
-                    mbar_expect_tx(full(stage), sbytes);
+                    mbar_expect_tx(full(stage), (uint32_t)nb * (A_BYTES + bbox));
                     const uint32_t dst = sbase + (uint32_t)stage * sbytes;
-                    tma_load_2d(dst, wm, kb * KB, x.l * x.R + x.m0, full(stage));
-                    tma_load_2d(dst + A_BYTES, &xmap, kb * KB, x.l * p.B, full(stage));
+                    for (int i = 0; i < nb; i++) {  // the boxes of a stage back to back: row segments of 512 bytes
+                        tma_load_2d(dst + (uint32_t)i * A_BYTES, wm, (kb + i) * KB, x.l * x.R + x.m0, full(stage));
+                        tma_load_2d(dst + (uint32_t)p.nbox * A_BYTES + (uint32_t)i * bbox, &xmap, (kb + i) * KB,
+                                    x.l * p.B, full(stage));
+                    }
                 }
                 __syncwarp();
                 issued[stage] = true;
@@ -185,17 +195,21 @@ __global__ void __launch_bounds__(THREADS)
             if (!mbar_wait_warp(tempty(acc), accphase ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d = tmem + (uint32_t)acc * acol;
-            for (int kb = x.kb0; kb < x.kb1; kb++) {
+            for (int kb = x.kb0; kb < x.kb1; kb += p.nbox) {
+                const int nb = min(p.nbox, x.kb1 - kb);
                 if (!mbar_wait_warp(full(stage), phase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a_base = sbase + (uint32_t)stage * sbytes;
-                const uint32_t b_base = a_base + A_BYTES;
+                const uint32_t b_base = a_base + (uint32_t)p.nbox * A_BYTES;
                 if (elect_one()) {
+                    for (int i = 0; i < nb; i++) {
 #pragma unroll
-                    for (int kk = 0; kk < KB / 16; kk++)
-                        mma_bf16(d, sdesc(a_base + 32 * kk), sdesc(b_base + 32 * kk), idesc, (kb > x.kb0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < KB / 16; kk++)
+                            mma_bf16(d, sdesc(a_base + (uint32_t)i * A_BYTES + 32 * kk), sdesc(b_base + (uint32_t)i * bbox + 32 * kk),
+                                     idesc, (kb > x.kb0 || i > 0 || kk > 0) ? 1u : 0u);
+                    }
                     mma_commit(empty(stage));
-                    if (kb == x.kb1 - 1) mma_commit(tfull(acc));
+                    if (kb + nb >= x.kb1) mma_commit(tfull(acc));
                 }
                 __syncwarp();
                 if (++stage == p.stages) { stage = 0; phase ^= 1; }
@@ -259,29 +273,13 @@ struct ProjProblem {
     bool out_f32;
 };
 
-// K ranges of a problem so that all problems of a launch reach about `want_units` units (at least
-// two K blocks each); split == false keeps all of K per unit.
-inline void proj_split(int L, int R, int K, int want_units, bool split, int &ksplit, int &nkb_per)
-{
-    using namespace proj;
-    const int nkb = (K + KB - 1) / KB;
-    const int tiles = L * ((R + 127) / 128);
-    int ks = 1;
-    if (split) {
-        ks = (want_units + tiles - 1) / tiles;
-        int cap = nkb / 2 > 1 ? nkb / 2 : 1;
-        if (cap > KSPLIT_MAX) cap = KSPLIT_MAX;
-        ks = ks < 1 ? 1 : (ks > cap ? cap : ks);
-    }
-    nkb_per = (nkb + ks - 1) / ks;
-    ksplit = (nkb + nkb_per - 1) / nkb_per;
-}
-
 // One launch over one or two problems sharing X bf16 [L][B][K]; a split problem's units store
-// partial slices, and ksplit_out[i] (nullable) reports how many.  ctas_per_sm bounds the pipeline
-// (fewer stages leave room for two CTAs per SM).
+// partial slices, and ksplit_out[i] (nullable) reports how many.  One CTA per SM; a stage holds up
+// to MAX_BOX boxes of K so that every weight row is read in segments of 512 bytes.  Split problems
+// take the number of K ranges (at most KSPLIT_MAX, in whole stages) that balances the units best
+// over the CTAs.
 inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const bool *split, int nprob, int L, int B,
-                                 int K, int sms, int ctas_per_sm, cudaStream_t st, int *ksplit_out = nullptr)
+                                 int K, int sms, cudaStream_t st, int *ksplit_out = nullptr)
 {
     using namespace proj;
     CUtensorMap wmap[2], xmap;
@@ -291,7 +289,36 @@ inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const boo
     p.B = B;
     p.K = K;
     p.NB = (B + 15) / 16 * 16;
-    const int want = sms * ctas_per_sm;
+    const uint32_t max_smem = 227 * 1024 - 1024;
+    p.nbox = MAX_BOX;
+    while (p.nbox > 1 && smem_total(p.NB, 2, p.nbox) > max_smem) p.nbox >>= 1;
+    p.stages = MAX_STAGES;
+    while (p.stages > 2 && smem_total(p.NB, p.stages, p.nbox) > max_smem) p.stages--;
+    const uint32_t smem = smem_total(p.NB, p.stages, p.nbox);
+    if (smem > max_smem) return LSA_ERR_UNSUPPORTED;
+    const int nkb = (K + KB - 1) / KB;
+    const int nst = (nkb + p.nbox - 1) / p.nbox;  // stages of all of K
+    int tiles = 0;
+    for (int i = 0; i < nprob; i++) tiles += L * ((pb[i].R + 127) / 128);
+    // K ranges of the split problems: the count (whole stages each) whose units fill the CTAs best
+    int ks = 1;
+    bool any_split = false;
+    for (int i = 0; i < nprob; i++) any_split = any_split || split[i];
+    if (any_split) {
+        double best = -1.0;
+        for (int c = 1; c <= KSPLIT_MAX && c <= nst; c++) {
+            const int spc = (nst + c - 1) / c;          // stages per range
+            const int ranges = (nst + spc - 1) / spc;
+            if (ranges != c) continue;
+            const int64_t units = (int64_t)tiles * c;
+            const int64_t waves = (units + sms - 1) / sms;
+            const double eff = (double)units / (double)(waves * sms);
+            if (eff > best + 1e-9) {
+                best = eff;
+                ks = c;
+            }
+        }
+    }
     bool ok = make_map_2d(&xmap, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * B, (uint64_t)K, KB, (uint32_t)p.NB);
     int total = 0;
     for (int i = 0; i < 2; i++) {
@@ -301,22 +328,20 @@ inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const boo
         r.R = q.R;
         r.out_f32 = q.out_f32 ? 1 : 0;
         r.mtiles = (q.R + 127) / 128;
-        r.partial = i < nprob && split[i] ? 1 : 0;
-        proj_split(L, q.R, K, want, i < nprob && split[i], r.ksplit, r.nkb_per);
+        const bool sp = i < nprob && split[i];
+        r.partial = sp ? 1 : 0;
+        const int spc = (nst + (sp ? ks : 1) - 1) / (sp ? ks : 1);
+        r.nkb_per = spc * p.nbox;
+        r.ksplit = (nkb + r.nkb_per - 1) / r.nkb_per;
         if (ksplit_out && i < nprob) ksplit_out[i] = r.ksplit;
         r.units = i < nprob ? L * r.mtiles * r.ksplit : 0;
         total += r.units;
         ok = ok && make_map_2d(&wmap[i], q.W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * q.R, (uint64_t)K, KB, 128);
     }
     if (!ok) return LSA_ERR_CUDA;
-    const uint32_t max_smem = (uint32_t)((227 * 1024) / ctas_per_sm) - 1024;
-    p.stages = MAX_STAGES;
-    while (p.stages > 2 && smem_total(p.NB, p.stages) > max_smem) p.stages--;
-    const uint32_t smem = smem_total(p.NB, p.stages);
-    if (smem > max_smem) return LSA_ERR_UNSUPPORTED;
     cudaError_t e = cudaFuncSetAttribute(k_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return LSA_ERR_CUDA;
-    const int grid = total < want ? total : want;
+    const int grid = total < sms ? total : sms;
     k_proj_tc<<<grid, THREADS, smem, st>>>(wmap[0], wmap[1], xmap, p);
     e = cudaGetLastError();
     return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;

@@ -21,6 +21,7 @@
 // last (a counter per query, reset by that CTA), and kernel boundaries order the rest.
 #pragma once
 #include "common.cuh"
+#include "li_tc.cuh"
 #include "topk.cuh"
 
 namespace lsa {
@@ -85,6 +86,7 @@ struct FrontParams {
     int ch;                    // key tiles per scorer work item
     int *item_start;           // [B+1]
     int *item_counter;
+    ItemInfo *items;           // the scorer's item table
     int *chunk_start;          // [B+1]
     int *chunk_query;          // [chunks] the query of each chunk
     uint32_t *state;           // [B][NS]
@@ -260,9 +262,15 @@ __global__ void __launch_bounds__(FRONT_TH) k_step_front(FrontParams p)
         }
         __syncthreads();
     }
-    // the query of every chunk (chunk_start was written by this block: visible after the barrier)
-    for (int b = threadIdx.x; b < p.B; b += FRONT_TH)
-        for (int c = p.chunk_start[b]; c < p.chunk_start[b + 1]; c++) p.chunk_query[c] = b;
+    // the query of every chunk and the scorer's item table, a warp per sequence (chunk_start and
+    // item_start were written by this block: visible after the barrier)
+    for (int b = warp; b < p.B; b += NW) {
+        for (int c = p.chunk_start[b] + lane; c < p.chunk_start[b + 1]; c += 32) p.chunk_query[c] = b;
+        const int64_t off = p.offs[b], S = p.offs[b + 1] - off;
+        int F = p.count[b];
+        F = F < 0 ? 0 : (F > S ? (int)S : F);
+        li::write_items(p.items, p.item_start[b], b, F, (int)S, off, 1, p.ch, lane);
+    }
 }
 
 // Range of the fetched entries' score keys, added to the query's state words 8 and 9, for a scorer
