@@ -32,7 +32,7 @@
 // k_golden_vote      one warp per 32-entry word: votes over the Lc layers per token, theta test,
 //                    OR over the tokens, one label byte per entry.
 #pragma once
-#include "common.cuh"
+#include "select_common.cuh"
 
 namespace lsa {
 

@@ -20,7 +20,7 @@
 // another: the per-query step after the histogram runs in whichever chunk CTA of the query finishes
 // last (a counter per query, reset by that CTA), and kernel boundaries order the rest.
 #pragma once
-#include "common.cuh"
+#include "select_common.cuh"
 #include "li_tc.cuh"
 #include "topk.cuh"
 

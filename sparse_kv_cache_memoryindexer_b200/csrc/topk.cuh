@@ -7,7 +7,7 @@
 // keys); the survivors are sorted by (score desc, entry asc) with a bitonic sort in shared memory
 // (k_topk_select).
 #pragma once
-#include "common.cuh"
+#include "select_common.cuh"
 
 namespace lsa {
 

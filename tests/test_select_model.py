@@ -214,7 +214,7 @@ def test_batched_select_model_equals_plain_sort(kind, cap):
             assert np.array_equal(batched_select_model(u, k, cap, seed=nc + k), plain_sort(u, k)), (kind, nc, k, cap)
 
 
-# ------------------------------------------------------------------ block sort (csrc/common.cuh)
+# ------------------------------------------------------------------ block sort (csrc/select_common.cuh)
 
 def block_sort_desc_model(v, nw=32):
     """block_sort_desc_u64: bitonic sort, strides >= 64 through shared memory, strides below 64 in
