@@ -41,6 +41,8 @@ constexpr int CH = 16;             // key tiles per work item (batched call; one
 constexpr int CH_STEP = 4;
 constexpr int MAX_STAGES = 8;
 constexpr int NRING = 4;           // claimed items in flight inside a CTA
+constexpr int HIST_SHIFT = 18;     // one decode step's score histogram: the top 14 bits of the
+constexpr int HIST_BINS = 1 << (32 - HIST_SHIFT);  // order-preserving score key (sign, exponent, 5 bits)
 
 struct Params {
     const float *wd;         // [B][tau][64]
@@ -51,10 +53,9 @@ struct Params {
     const ItemInfo *items;   // [items] the planner's table
     int *item_counter;       // next unclaimed item, zeroed by k_li_items
     float *Y;                // [tau*T]
-    uint32_t *range;         // one decode step (nq = 1): per sequence b, words range[b*range_stride]
-                             // and [+1] take the smallest and largest score key (atomicMin / Max);
-                             // null: not reported
-    int range_stride;
+    int *hist;               // one decode step (nq = 1): per sequence b, HIST_BINS counters of the
+                             // score keys' top bits (hist[b*HIST_BINS + (key >> HIST_SHIFT)]);
+                             // null: not counted
     int64_t T;
     int B, tau, groups, stages;
     int ch;                  // key tiles per work item
@@ -343,7 +344,6 @@ __global__ void __launch_bounds__(320, 1)
             __syncwarp();
             const int64_t off = w.off;
             float *Yb = p.Y + (int64_t)p.tau * off;
-            uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // score keys of this warp's entries of the item
             for (int kt = t0; kt < t1; kt++) {
                 const int64_t j = (int64_t)kt * TILE + quarter * 32 + lane;
                 const bool valid = j < F;
@@ -392,19 +392,12 @@ __global__ void __launch_bounds__(320, 1)
                 if (valid) {
                     if (nqw > 0) Yb[(int64_t)i0 * S + j] = y[0];
                     if (nqw > 1) Yb[(int64_t)(i0 + 1) * S + j] = y[1];
-                    if (NQV == 1) {
-                        const uint32_t u = float_to_ordered(y[0]);
-                        kmin = min(kmin, u);
-                        kmax = max(kmax, u);
-                    }
                 }
-            }
-            if (NQV == 1 && p.range && nqw > 0) {
-                kmin = __reduce_min_sync(0xffffffffu, kmin);
-                kmax = __reduce_max_sync(0xffffffffu, kmax);
-                if (lane == 0 && kmin <= kmax) {
-                    atomicMin(p.range + (int64_t)w.b * p.range_stride, kmin);
-                    atomicMax(p.range + (int64_t)w.b * p.range_stride + 1, kmax);
+                if (NQV == 1 && p.hist && nqw > 0) {  // the step's histogram, one atomic per bin per warp
+                    const uint32_t bin = valid ? float_to_ordered(y[0]) >> HIST_SHIFT : 0xFFFFFFFFu;
+                    const unsigned grp = __match_any_sync(0xffffffffu, bin);
+                    if (valid && lane == __ffs(grp) - 1)
+                        atomicAdd(p.hist + (int64_t)w.b * HIST_BINS + bin, __popc(grp));
                 }
             }
         }
@@ -434,8 +427,8 @@ inline bool li_tc_supported(int n_h, int d_I, int tau, int kdt, int nq = li::NQ)
 // nq: queries per MMA group (li_tc_supported).  Launches the item planner and the scoring kernel;
 // *launches counts them.
 // planned: item_start and item_counter were already written for this call (ch = li_item_tiles(nq)),
-// so the planner is not launched.  range (nq = 1 only; nullable): per sequence b, the smallest and
-// largest order-preserving score key are folded into range[b * range_stride] and [+ 1].
+// so the planner is not launched.  hist (nq = 1 only; nullable, zeroed): per sequence b, HIST_BINS
+// counters of the scores' top key bits.
 inline int li_item_tiles(int nq) { return nq == li::NQ ? li::CH : li::CH_STEP; }
 
 // Upper bound on the work items of a call (sum over sequences of ceil(ceil(F_b/128)/ch) x groups).
@@ -448,7 +441,7 @@ inline int64_t li_max_items(int B, int64_t T, int tau, int nq)
 inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK, const float *hsc,
                                const int32_t *count, const int64_t *offs, int B, int64_t T, int tau, int nq, float *Y,
                                int *item_start, int *item_counter, ItemInfo *items, int sms, cudaStream_t st,
-                               int *launches, bool planned = false, uint32_t *range = nullptr, int range_stride = 0)
+                               int *launches, bool planned = false, int *hist = nullptr)
 {
     using namespace li;
     *launches = 0;
@@ -472,8 +465,7 @@ inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK
     p.items = items;
     p.item_counter = item_counter;
     p.Y = Y;
-    p.range = range;
-    p.range_stride = range_stride;
+    p.hist = hist;
     p.T = T;
     p.B = B;
     p.tau = tau;

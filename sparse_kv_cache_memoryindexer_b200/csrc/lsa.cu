@@ -603,28 +603,8 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
 
 // ------------------------------------------------------------------------------ stage 5, one decode step
 
-// Workspace of lsa_lightning_topk_step: [item_start B+1, counter][Y: total_S][tail: B * W]
-// [queries: B * n_h * d_I (4-byte elements)][weights: B * n_h][select: chunk starts, state,
-// histograms and pass counters, chunk counts, the selection (LSA_MAX_TOPK per sequence)].
-static int64_t step_max_chunks(int B, int64_t total_S, int W)
-{
-    return (total_S + (int64_t)B * W) / stepsel::CH + B + 1;
-}
-
-// Select workspace of one decode step: chunk starts, state, bucket histograms with finish counters,
-// the stage (capacity S_b + W keys per query), the selection (LSA_MAX_TOPK keys per query) and the
-// query of each chunk.
-static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[6])
-{
-    sp[0] = align_up(sizeof(int) * (size_t)(B + 1), 256);
-    sp[1] = align_up(sizeof(uint32_t) * stepsel::NS * (size_t)B, 256);
-    sp[2] = align_up(sizeof(int) * (stepsel::NB + 1) * (size_t)B, 256);
-    sp[3] = align_up(sizeof(unsigned long long) * (size_t)(total_S + (int64_t)B * W + 1), 256);
-    sp[4] = align_up(sizeof(unsigned long long) * (size_t)B * LSA_MAX_TOPK, 256);
-    sp[5] = align_up(sizeof(int) * (size_t)step_max_chunks(B, total_S, W), 256);
-    return sp[0] + sp[1] + sp[2] + sp[3] + sp[4] + sp[5];
-}
-
+// Workspace of lsa_lightning_topk_step: [item_start B+1, counter][item table][Y: total_S]
+// [tail: B * W][queries: B * n_h * d_I (4-byte elements)][weights: B * n_h][histograms: B * HB].
 static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[6])
 {
     part[0] = align_up(sizeof(int) * (size_t)(B + 2), 256) +
@@ -633,8 +613,7 @@ static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, siz
     part[2] = align_up(sizeof(float) * (size_t)B * (W > 0 ? W : 1), 256);
     part[3] = align_up((size_t)4 * B * n_h * d_I, 256);
     part[4] = align_up(sizeof(float) * (size_t)B * n_h, 256);
-    size_t sp[6];
-    part[5] = step_sel_parts(B, total_S, W, sp);
+    part[5] = align_up(sizeof(int) * (size_t)B * stepsel::HB, 256);
     return part[0] + part[1] + part[2] + part[3] + part[4] + part[5];
 }
 
@@ -685,18 +664,10 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     // one query per sequence: the tensor-core scorer runs with one-query groups (MMA N = n_h)
     const bool tc = li_tc_supported(n_h, d_I, 1, kdt, 1);
     const int TQ = 1;
-    size_t sp[6];
-    step_sel_parts(B, total_S, W, sp);
-    char *sb = p + part[0] + part[1] + part[2] + part[3] + part[4];
-    int *chunk_start = (int *)sb;
-    uint32_t *state = (uint32_t *)(sb + sp[0]);
-    int *ghist = (int *)(sb + sp[0] + sp[1]);
-    unsigned long long *stage = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2]);
-    unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
-    int *chunk_query = (int *)(sb + sp[0] + sp[1] + sp[2] + sp[3] + sp[4]);
+    int *ghist = (int *)(p + part[0] + part[1] + part[2] + part[3] + part[4]);
     const int32_t *tcnt = W > 0 ? win_count : nullptr;
-    // first launch: scorer items, select chunks and state, cleared histograms, the dense query copy
-    // and the window entries' scores
+    // first launch: the scorer's items and their table, cleared histograms, the dense query copy and
+    // the window entries' scores
     {
         stepsel::FrontParams fp;
         fp.count = count;
@@ -704,7 +675,6 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         fp.win_count = tcnt;
         fp.W = W;
         fp.B = B;
-        fp.k = k;
         fp.n_h = n_h;
         fp.d_I = d_I;
         fp.dt = hdt;
@@ -712,9 +682,6 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         fp.item_start = item_start;
         fp.item_counter = item_counter;
         fp.items = items;
-        fp.chunk_start = chunk_start;
-        fp.chunk_query = chunk_query;
-        fp.state = state;
         fp.ghist = ghist;
         fp.qs = q_step;
         fp.q_bstride = q_batch_stride;
@@ -744,8 +711,7 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         LSA_REQUIRE(aligned(hot_K, 16), "lsa_lightning_topk_step: hot_K must be 16-byte aligned");
         int n = 0;
         const lsa_status s = launch_li_tc(qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, TQ, 1, Y, item_start,
-                                          item_counter, items, num_sms(), st, &n, /*planned=*/true, state + 8,
-                                          stepsel::NS);
+                                          item_counter, items, num_sms(), st, &n, /*planned=*/true, ghist);
         g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
         if (s != LSA_OK)
             return fail(s, "lsa_lightning_topk_step: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
@@ -755,26 +721,19 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         case 64: LSA_TRY(li_simt_d<64>(hdt, qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, 1, n_h, Y, st)); break;
         default: LSA_TRY(li_simt_d<128>(hdt, qw, ww, hot_K, hot_scale, count, seq_offsets, B, total_S, 1, n_h, Y, st)); break;
         }
+        // the SIMT scorer does not count the histogram
+        stepsel::k_step_hist<<<dim3(16, (unsigned)B), 256, 0, st>>>(Y, count, seq_offsets, ghist);
+        LSA_TRY(launched("decode step: histogram"));
     }
-    // the select, spread over chunks of candidates (see step_select.cuh)
-    const int64_t mc = step_max_chunks(B, total_S, W);
-    if (!tc) {  // the SIMT scorer does not report the range of the score keys
-        stepsel::k_ss_range<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, B, chunk_start,
-                                                                     chunk_query, state);
-        LSA_TRY(launched("decode step: key range"));
-    }
-    stepsel::k_ss_hist12<<<(unsigned)mc, stepsel::TH, 0, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B, chunk_start,
-                                                               chunk_query, state, ghist);
+    // the select: one CTA per query
     int kpow2 = 64;  // the block sort works on at least 64 keys
     while (kpow2 < k) kpow2 <<= 1;
-    const size_t smem = sizeof(unsigned long long) * ((size_t)kpow2 + stepsel::SCAP);
-    LSA_TRY(set_smem(stepsel::k_ss_write, smem));
-    stepsel::k_ss_write<<<(unsigned)mc, stepsel::SORT_TH, smem, st>>>(Y, TQ, count, seq_offsets, tail, tcnt, W, B,
-                                                                      chunk_start, chunk_query, state, LSA_MAX_TOPK, ghist,
-                                                                      sel, stage, idx,
+    const size_t smem = stepsel::select_smem(kpow2);
+    LSA_TRY(set_smem(stepsel::k_ss_select, smem));
+    stepsel::k_ss_select<<<(unsigned)B, stepsel::SEL_TH, smem, st>>>(Y, count, seq_offsets, tail, tcnt, W, ghist, idx,
                                                                       k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
-    g_launches.fetch_add(3, std::memory_order_relaxed);  // front, histogram, write + final
+    g_launches.fetch_add(2, std::memory_order_relaxed);  // front, select
     return ok();
 }
 
