@@ -11,16 +11,16 @@
 //                    (logit desc, entry asc), n_p the first count whose mass sum e reaches p Z
 //                    (e = exp(z - max z), Z = sum of all e).
 //                    Fast path (two reads of the row): the maximum; then Z in fp32 exp with an
-//                    error bound of its own, while the entries within 8 of the maximum are
-//                    gathered in shared memory.  Their masses (in double) tell whether they hold
+//                    error bound of its own, while the entries within 4 of the maximum are
+//                    gathered in shared memory.  Their mass (in double) tells whether they hold
 //                    the nucleus (the kept set is a prefix of the sorted row, so any such prefix
-//                    of candidates gives the same crossing); they are sorted (only those within
-//                    4 when those suffice) and scanned in double for the crossing against both
-//                    ends of the target's interval p [Z - err, Z + err].  When both ends give the
+//                    of candidates gives the same crossing); they are sorted and scanned in double
+//                    for the crossing against both ends of the target's interval
+//                    p [Z - err, Z + err].  When both ends give the
 //                    same position it is the one an fp64 Z gives; otherwise Z is recomputed in
 //                    double and the scan repeated.  The kept entries' bits are set from the
 //                    sorted candidates.
-//                    General path (more than CAND entries within 8, or less than the target's
+//                    General path (more than CAND entries within 4, or less than the target's
 //                    mass there): Z in double and, for a few depths D, the mass and count of the
 //                    entries within D of the maximum; the smallest such set whose mass reaches
 //                    p Z and that has at most CAND entries is sorted and scanned in double;
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     __shared__ unsigned long long cand[CAND];  // (key << 32) | ~entry
     __shared__ double dmass[ND][THREADS / 32];
     __shared__ int dcnt[ND][THREADS / 32];
-    __shared__ int s_nc, s_depth, s_cross, s_cross_hi, s_n4;
+    __shared__ int s_nc, s_depth, s_cross, s_cross_hi;
     __shared__ float fred[THREADS / 32];
     __shared__ double dred[THREADS / 32];
     __shared__ uint32_t s_prefix;
@@ -173,61 +173,32 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     if (m > -INFINITY && m < INFINITY) {
         if (threadIdx.x == 0) s_nc = 0;
         __syncthreads();
-        // Z in fp32 exp (summed in double) and the bound of its error: expf is within 2 ulp
-        // (2^-22 relative) and z - m is rounded once (an error of 2^-24 |x| in the exponent); a
-        // result below the smallest normal is off by at most 2^-126 absolute
-        double z32 = 0.0, zx = 0.0;
+        // Z in fp32 exp and the bound of its error: expf is within 2 ulp (2^-22 relative); z - m is
+        // rounded once (an error of 2^-24 |x| in the exponent, |x| < 104 wherever the result is
+        // normal); each thread's fp32 sum of its S / THREADS terms rounds by at most that many
+        // ulps; a result below the smallest normal is off by at most 2^-126 absolute
+        float zf = 0.f;
         for (int64_t base = 0; base < S; base += THREADS) {  // whole warps per step (warp-wide appends)
             const int64_t s = base + threadIdx.x;
             const float zs = s < S ? __ldg(row + s) : -INFINITY;
-            const float x = zs - m;
-            const float e = s < S ? expf(x) : 0.f;
-            z32 += (double)e;
-            zx += s < S ? (double)e * (double)(-x) : 0.0;
-            warp_append(s < S && m - zs < 8.f,
+            zf += s < S ? expf(zs - m) : 0.f;
+            warp_append(s < S && m - zs < 4.f,
                         ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s), &s_nc, cand);
         }
-        double Z32 = block_sum(z32, dred);
-        const double ZX = block_sum(zx, dred);
+        const double Z32 = block_sum((double)zf, dred);
         // (plus the rounding of sums in double, here and in an fp64 Z: terms per thread + 64 ulps)
-        const double err = 1.01 * (Z32 * 0x1p-22 + ZX * 0x1p-24) + (double)S * 0x1p-126 +
-                           2.0 * Z32 * ((double)S / THREADS + 64.0) * 0x1p-53;
-        const int nc8 = s_nc;
-        if (nc8 <= CAND) {
-            // exact masses of the entries within 8 and within 4 of the maximum
-            double m8 = 0.0, m4 = 0.0;
-            int c4 = 0;
-            for (int t = threadIdx.x; t < nc8; t += THREADS) {
-                const float zc = ordered_to_float((uint32_t)(cand[t] >> 32));
-                const double e = exp((double)zc - (double)m);
-                m8 += e;
-                if (m - zc < 4.f) {
-                    m4 += e;
-                    c4++;
-                }
-            }
-            m8 = block_sum(m8, dred);
+        const double err = 1.01 * Z32 * (0x1p-22 + 104.0 * 0x1p-24 + ((double)S / THREADS + 1.0) * 0x1p-24) +
+                           (double)S * 0x1p-126 + 2.0 * Z32 * ((double)S / THREADS + 64.0) * 0x1p-53;
+        const int nc = s_nc;
+        if (nc <= CAND) {
+            // the exact mass of the entries within 4 of the maximum
+            double m4 = 0.0;
+            for (int t = threadIdx.x; t < nc; t += THREADS)
+                m4 += exp((double)ordered_to_float((uint32_t)(cand[t] >> 32)) - (double)m);
             m4 = block_sum(m4, dred);
             const double t_hi = p * (Z32 + err) * (1.0 + 0x1p-50);
             const double t_lo = p * (Z32 - err) * (1.0 - 0x1p-50);
-            if (m8 >= t_hi) {
-                int nc = nc8;
-                if (m4 >= t_hi) {  // the entries within 4 hold the nucleus: keep only them
-                    if (threadIdx.x == 0) s_n4 = 0;
-                    for (int base = 0; base < nc8; base += THREADS) {
-                        const int t = base + threadIdx.x;
-                        unsigned long long v = 0ull;
-                        bool keep = false;
-                        if (t < nc8) {
-                            v = cand[t];
-                            keep = m - ordered_to_float((uint32_t)(v >> 32)) < 4.f;
-                        }
-                        __syncthreads();  // every entry of this block read before any is overwritten
-                        warp_append(keep, v, &s_n4, cand);
-                        __syncthreads();
-                    }
-                    nc = s_n4;
-                }
+            if (m4 >= t_hi) {  // the entries within 4 hold the nucleus
                 int np2 = 64;
                 while (np2 < nc) np2 <<= 1;
                 for (int t = nc + threadIdx.x; t < np2; t += THREADS) cand[t] = 0ull;

@@ -119,11 +119,11 @@ def test_golden_long_flat_rows_take_the_radix_search(m, p):
 
 
 def test_golden_each_path(m):
-    # sequence 0: the entries within 8 of the maximum hold the nucleus (sorted candidates);
-    # sequence 1: more than 4096 entries within 8, but those within 4 hold the nucleus (the general
-    # path's candidate sort); sequence 2: the entries within 8 hold too little mass and the rest is
-    # flat (the general path's radix search); sequence 3: all equal, the crossing exactly at p Z
-    # (the total mass recomputed in double)
+    # sequence 0: the entries within 4 of the maximum hold the nucleus (the fast path's candidates);
+    # sequence 1: those within 4 hold too little mass, those within 8 (at most 4096) hold it (the
+    # general path's candidate sort); sequence 2: the entries within 4 hold too little mass and the
+    # rest is flat (the general path's radix search); sequence 3: all equal, the crossing exactly at
+    # p Z (the total mass recomputed in double)
     S = (5000, 9000, 30001, 1000)
     offs = torch.from_numpy(np.concatenate([[0], np.cumsum(S)]).astype(np.int64))
     g = torch.Generator().manual_seed(5)
@@ -131,14 +131,17 @@ def test_golden_each_path(m):
     o = offs.numpy()
     z[:, :, o[0]:o[1]] = torch.randn((2, 2, S[0]), generator=g)
     z[:, :, o[0] + 100:o[0] + 400] += 6.0
-    z[:, :, o[1]:o[1] + 3000] = 5.0 + 0.01 * torch.randn((2, 2, 3000), generator=g)
-    z[:, :, o[1] + 3000:o[2]] = 0.5
+    z[:, :, o[1]] = 10.0
+    z[:, :, o[1] + 1:o[1] + 3001] = 5.0 + 0.01 * torch.randn((2, 2, 3000), generator=g)
+    z[:, :, o[1] + 3001:o[2]] = 0.5
     z[:, :, o[2]] = 10.0
     z[:, :, o[2] + 1:o[3]] = torch.rand((2, 2, S[2] - 1), generator=g) * 0.01
     z[:, :, o[3]:o[4]] = -2.0
     zn = z.numpy()
     row1 = zn[0, 0, o[1]:o[2]]
-    assert ((row1.max() - row1) < 8).sum() > 4096 and candidate_set_fits(row1, 0.6)
+    e1 = np.exp(row1.astype(np.float64) - row1.max())
+    near4 = (row1.max() - row1) < 4
+    assert e1[near4].sum() < 0.6 * e1.sum() and candidate_set_fits(row1, 0.6)
     row2 = zn[0, 0, o[2]:o[3]]
     assert not candidate_set_fits(row2, 0.6)
     label, ref = check(m, z, offs, p=0.6, theta=1)
