@@ -604,7 +604,25 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
 // ------------------------------------------------------------------------------ stage 5, one decode step
 
 // Workspace of lsa_lightning_topk_step: [item_start B+1, counter][item table][Y: total_S]
-// [tail: B * W][queries: B * n_h * d_I (4-byte elements)][weights: B * n_h][histograms: B * HB].
+// [tail: B * W][queries: B * n_h * d_I (4-byte elements)][weights: B * n_h][select: histograms
+// B * HB, chunk starts B+1, the query of each chunk, state B * NS, the selections B * LSA_MAX_TOPK,
+// the stages total_S + B * W].
+static int64_t step_max_chunks(int B, int64_t total_S, int W)
+{
+    return (total_S + (int64_t)B * W) / stepsel::CH + B + 1;
+}
+
+static size_t step_sel_parts(int B, int64_t total_S, int W, size_t sp[6])
+{
+    sp[0] = align_up(sizeof(int) * (size_t)B * stepsel::HB, 256);
+    sp[1] = align_up(sizeof(int) * (size_t)(B + 1), 256);
+    sp[2] = align_up(sizeof(int) * (size_t)step_max_chunks(B, total_S, W), 256);
+    sp[3] = align_up(sizeof(uint32_t) * stepsel::NS * (size_t)B, 256);
+    sp[4] = align_up(sizeof(unsigned long long) * (size_t)B * LSA_MAX_TOPK, 256);
+    sp[5] = align_up(sizeof(unsigned long long) * (size_t)(total_S + (int64_t)B * W + 1), 256);
+    return sp[0] + sp[1] + sp[2] + sp[3] + sp[4] + sp[5];
+}
+
 static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, size_t part[6])
 {
     part[0] = align_up(sizeof(int) * (size_t)(B + 2), 256) +
@@ -613,7 +631,8 @@ static size_t step_ws_parts(int B, int64_t total_S, int n_h, int d_I, int W, siz
     part[2] = align_up(sizeof(float) * (size_t)B * (W > 0 ? W : 1), 256);
     part[3] = align_up((size_t)4 * B * n_h * d_I, 256);
     part[4] = align_up(sizeof(float) * (size_t)B * n_h, 256);
-    part[5] = align_up(sizeof(int) * (size_t)B * stepsel::HB, 256);
+    size_t sp[6];
+    part[5] = step_sel_parts(B, total_S, W, sp);
     return part[0] + part[1] + part[2] + part[3] + part[4] + part[5];
 }
 
@@ -664,7 +683,15 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     // one query per sequence: the tensor-core scorer runs with one-query groups (MMA N = n_h)
     const bool tc = li_tc_supported(n_h, d_I, 1, kdt, 1);
     const int TQ = 1;
-    int *ghist = (int *)(p + part[0] + part[1] + part[2] + part[3] + part[4]);
+    size_t sp[6];
+    step_sel_parts(B, total_S, W, sp);
+    char *sb = p + part[0] + part[1] + part[2] + part[3] + part[4];
+    int *ghist = (int *)sb;
+    int *chunk_start = (int *)(sb + sp[0]);
+    int *chunk_query = (int *)(sb + sp[0] + sp[1]);
+    uint32_t *state = (uint32_t *)(sb + sp[0] + sp[1] + sp[2]);
+    unsigned long long *sel = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3]);
+    unsigned long long *stage = (unsigned long long *)(sb + sp[0] + sp[1] + sp[2] + sp[3] + sp[4]);
     const int32_t *tcnt = W > 0 ? win_count : nullptr;
     // first launch: the scorer's items and their table, cleared histograms, the dense query copy and
     // the window entries' scores
@@ -675,6 +702,10 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         fp.win_count = tcnt;
         fp.W = W;
         fp.B = B;
+        fp.k = k;
+        fp.chunk_start = chunk_start;
+        fp.chunk_query = chunk_query;
+        fp.state = state;
         fp.n_h = n_h;
         fp.d_I = d_I;
         fp.dt = hdt;
@@ -725,13 +756,15 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         stepsel::k_step_hist<<<dim3(16, (unsigned)B), 256, 0, st>>>(Y, count, seq_offsets, ghist);
         LSA_TRY(launched("decode step: histogram"));
     }
-    // the select: one CTA per query
+    // the select: one CTA per chunk of candidates, the query's last chunk completing it
     int kpow2 = 64;  // the block sort works on at least 64 keys
     while (kpow2 < k) kpow2 <<= 1;
-    const size_t smem = stepsel::select_smem(kpow2);
-    LSA_TRY(set_smem(stepsel::k_ss_select, smem));
-    stepsel::k_ss_select<<<(unsigned)B, stepsel::SEL_TH, smem, st>>>(Y, count, seq_offsets, tail, tcnt, W, ghist, idx,
-                                                                      k, kpow2, topk_idx, topk_score);
+    const size_t smem = stepsel::write_smem(kpow2);
+    LSA_TRY(set_smem(stepsel::k_ss_write, smem));
+    const int64_t mc = step_max_chunks(B, total_S, W);
+    stepsel::k_ss_write<<<(unsigned)mc, stepsel::SEL_TH, smem, st>>>(Y, count, seq_offsets, tail, tcnt, W, B, chunk_start,
+                                                                     chunk_query, state, ghist, LSA_MAX_TOPK, sel, stage,
+                                                                     idx, k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
     g_launches.fetch_add(2, std::memory_order_relaxed);  // front, select
     return ok();

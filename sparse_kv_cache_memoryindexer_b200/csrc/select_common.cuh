@@ -85,4 +85,103 @@ __device__ __forceinline__ void block_sort_desc_u64(unsigned long long *v, int n
     }
 }
 
+
+// Block-wide minimum and maximum of one key per thread (threads without a key pass 0xFFFFFFFF and
+// 0); *lo / *hi: shared words, written by this call.  Starts and ends with a barrier.
+__device__ __forceinline__ void block_min_max(uint32_t vmin, uint32_t vmax, uint32_t *lo, uint32_t *hi)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        *lo = 0xFFFFFFFFu;
+        *hi = 0u;
+    }
+    __syncthreads();
+    vmin = __reduce_min_sync(0xffffffffu, vmin);
+    vmax = __reduce_max_sync(0xffffffffu, vmax);
+    if ((threadIdx.x & 31) == 0) {
+        atomicMin(lo, vmin);
+        atomicMax(hi, vmax);
+    }
+    __syncthreads();
+}
+
+// The n distinct 64-bit keys of v (any order; blockDim.x = 1024) put in descending order without a
+// sort of all of them: SEL_NB buckets linear in the score (key >> 32) over the keys' own range, the
+// keys scattered into their buckets' segments (higher buckets first), and a key's position = its
+// segment's start + the keys of its segment above it.  When a bucket holds more than max_seg keys,
+// the keys are sorted instead (bitonic, v padded to npow2 >= n with zeros; npow2 a power of two
+// >= 64).  emit(position, key) is called once per key.  tmp: n keys of shared memory; cnt: SEL_NB
+// ints of shared memory.  Ends with a barrier.
+template <typename Emit>
+__device__ __forceinline__ void order_desc(unsigned long long *v, int n, int npow2, unsigned long long *tmp, int *cnt,
+                                           int max_seg, Emit emit)
+{
+    __shared__ uint32_t s_lo, s_hi;
+    __shared__ int s_mx;
+    __shared__ int s_wt[32];
+    constexpr int PER = SEL_NB / 1024;
+    uint32_t tmin = 0xFFFFFFFFu, tmax = 0u;
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+        const uint32_t u = (uint32_t)(v[t] >> 32);
+        tmin = min(tmin, u);
+        tmax = max(tmax, u);
+    }
+    for (int t = threadIdx.x; t < SEL_NB; t += blockDim.x) cnt[t] = 0;
+    if (threadIdx.x == 0) s_mx = 0;
+    block_min_max(tmin, tmax, &s_lo, &s_hi);
+    const SelRange rg = sel_range(s_lo, s_hi);
+    for (int t = threadIdx.x; t < n; t += blockDim.x) atomicAdd(&cnt[sel_bucket(rg, (uint32_t)(v[t] >> 32))], 1);
+    __syncthreads();
+    {
+        // exclusive counts from the top: thread t owns buckets SEL_NB - PER (t + 1) .. SEL_NB - PER t - 1
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        const int hi = SEL_NB - PER * (int)threadIdx.x;
+        int c[PER], sum = 0, mx = 0;
+#pragma unroll
+        for (int i = 0; i < PER; i++) {
+            c[i] = cnt[hi - 1 - i];
+            sum += c[i];
+            mx = max(mx, c[i]);
+        }
+        const int inc = warp_incl_scan(sum);
+        if (lane == 31) s_wt[warp] = inc;
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) atomicMax(&s_mx, mx);
+        __syncthreads();
+        if (warp == 0) {
+            const int x = lane < (int)(blockDim.x >> 5) ? s_wt[lane] : 0;
+            s_wt[lane] = warp_incl_scan(x) - x;
+        }
+        __syncthreads();
+        int run = s_wt[warp] + inc - sum;
+#pragma unroll
+        for (int i = 0; i < PER; i++) {
+            cnt[hi - 1 - i] = run;
+            run += c[i];
+        }
+    }
+    __syncthreads();
+    if (s_mx <= max_seg) {
+        for (int t = threadIdx.x; t < n; t += blockDim.x) {
+            const unsigned long long x = v[t];
+            tmp[atomicAdd(&cnt[sel_bucket(rg, (uint32_t)(x >> 32))], 1)] = x;
+        }
+        __syncthreads();
+        // cnt[b] is now the end of bucket b's segment, and the end of bucket b + 1's is b's start
+        for (int t = threadIdx.x; t < n; t += blockDim.x) {
+            const unsigned long long x = tmp[t];
+            const uint32_t b = sel_bucket(rg, (uint32_t)(x >> 32));
+            const int lo = b + 1 < (uint32_t)SEL_NB ? cnt[b + 1] : 0, hi = cnt[b];
+            int r = lo;
+            for (int i = lo; i < hi; i++) r += tmp[i] > x;
+            emit(r, x);
+        }
+    } else {
+        for (int t = n + threadIdx.x; t < npow2; t += blockDim.x) v[t] = 0ull;
+        block_sort_desc_u64(v, npow2);
+        for (int t = threadIdx.x; t < n; t += blockDim.x) emit(t, v[t]);
+    }
+    __syncthreads();
+}
+
 }  // namespace lsa

@@ -3,19 +3,19 @@
 // entries S_b + j).  A candidate's 64-bit key is (order-preserving score key << 32) | ~slot: larger
 // score first, then smaller slot, and no two keys are equal.
 //   k_step_front   one grid, CTA roles that do not wait for one another: the scorer's work items
-//                  and their table; the cleared score histograms; per sequence the step's query
-//                  and weights copied to the scorer's dense layout and the window entries' scores
+//                  and their table, the select's chunks (CH candidates each) and state; the cleared
+//                  score histograms; per sequence the step's query and weights copied to the
+//                  scorer's dense layout and the window entries' scores
 //   k_li_tc<1>     (li_tc.cuh) the fetched entries' scores, and their histogram: the top 14 bits
 //                  of the score key (HIST_BINS bins, li_tc.cuh) counted per sequence
-//   k_ss_select    one CTA per query: the histogram (plus the window entries) gives the bin beta of
-//                  the k-th largest key; one pass over the candidates scatters the keys of higher
-//                  bins into their bins' segments of the selection and stages bin beta's keys; the
-//                  stage sorted gives its largest keys, and when no bin above beta is large a key's
-//                  output position is its segment's start plus the keys of its segment above it
-//                  (otherwise the k keys are sorted).  A bin beta of more than SCAP keys is
-//                  resolved by four radix passes over its keys and an ordered pass (the first keys
-//                  equal to the k-th in slot order).  A query with at most k candidates takes them
-//                  all.  The output is as the batched select writes it.
+//   k_ss_write     one CTA per chunk: the query's histogram (plus its window entries) gives the bin
+//                  beta of the k-th largest key (each chunk finds the same); the chunk's keys of
+//                  higher bins are appended to the query's selection and bin beta's to its stage
+//                  (any order: the keys carry their slots).  The query's last chunk to finish then
+//                  takes the want largest staged keys (a sort in shared memory, or a radix select
+//                  over a crowded stage) and orders the k keys (order_desc: buckets over their own
+//                  score range, counting within a bucket).  A query with at most k candidates takes
+//                  them all.  The output is as the batched select writes it.
 #pragma once
 #include "select_common.cuh"
 #include "li_tc.cuh"
@@ -27,8 +27,10 @@ namespace stepsel {
 
 constexpr int HB = li::HIST_BINS;  // histogram bins per query
 constexpr int SEL_TH = SEL_THREADS;
+constexpr int CH = 4096;           // candidates per chunk
 constexpr int SCAP = 4096;         // staged keys sorted in shared memory
-constexpr int RANK_SEG = 64;       // largest bin above beta whose keys are ranked by counting
+constexpr int RANK_SEG = 32;       // largest bucket of the final order whose keys are ranked by counting
+constexpr int NS = 8;              // state words per query
 
 __device__ __forceinline__ uint32_t bin_of(uint32_t u) { return u >> li::HIST_SHIFT; }
 
@@ -60,8 +62,9 @@ __device__ __forceinline__ uint32_t key_of(const Query &q, int j)
 }
 
 // The step's first launch: three CTA roles in one grid, none waiting on another.
-//   CTA 0           the prefix over the sequences of the scorer's work items (ceil(ceil(F_b/128)/ch)
-//                   per sequence, claim counter zeroed) and the item table, a warp per sequence
+//   CTA 0           two prefixes over the sequences: the scorer's work items (ceil(ceil(F_b/128)/ch)
+//                   per sequence, claim counter zeroed) and the select's chunks; the select state;
+//                   then, a warp per sequence, the item table and the query of every chunk
 //   nclear CTAs     zero the histograms, 4096 words each
 //   B CTAs          one per sequence: its query and weights copied to the scorer's dense layout
 //                   (and to shared memory) and the window entries' scores (a warp an entry)
@@ -69,8 +72,13 @@ struct FrontParams {
     const int32_t *count;      // [B] fetched entries
     const int64_t *offs;       // [B+1]
     const int32_t *win_count;  // [B] window entries, or null (no window entries)
-    int W, B, n_h, d_I, dt;
+    int W, B, k, n_h, d_I, dt;
     int ch;                    // key tiles per scorer work item
+    int *chunk_start;          // [B+1]
+    int *chunk_query;          // [chunks] the query of each chunk
+    uint32_t *state;           // [B][NS]: [1] k if the query has more than k candidates, else 0;
+                               // [3] candidates; [4] keys in the selection; [5] keys staged;
+                               // [6] the write step's finish counter
     int *item_start;           // [B+1]
     int *item_counter;
     ItemInfo *items;           // the scorer's item table
@@ -167,44 +175,72 @@ __global__ void __launch_bounds__(FRONT_TH) k_step_front(FrontParams p)
         }
         return;
     }
-    // ---- CTA 0: the scorer's items
-    __shared__ int wt_items[NW];
-    __shared__ int carry_items;
+    // ---- CTA 0: the scorer's items and the select's chunks
+    __shared__ int wt_items[NW], wt_chunks[NW];
+    __shared__ int carry_items, carry_chunks;
     if (threadIdx.x == 0) {
         carry_items = 0;
+        carry_chunks = 0;
         p.item_start[0] = 0;
         *p.item_counter = 0;
+        p.chunk_start[0] = 0;
     }
     __syncthreads();
     for (int base = 0; base < p.B; base += FRONT_TH) {
         const int b = base + threadIdx.x;
-        int ni = 0;
+        int ni = 0, nchunk = 0;
         if (b < p.B) {
             const int64_t S = p.offs[b + 1] - p.offs[b];
             int F = p.count[b];
             if (F < 0 || F > S) flag(ERRF_COUNT);
             F = F < 0 ? 0 : (F > S ? (int)S : F);
+            int nt = p.win_count ? p.win_count[b] : 0;
+            nt = nt < 0 ? 0 : (nt > p.W ? p.W : nt);
             const int tiles = (F + TILE - 1) / TILE;
             ni = (tiles + p.ch - 1) / p.ch;
+            const int nc = F + nt;
+            nchunk = nc > 0 ? (nc + CH - 1) / CH : 1;  // a query without candidates still writes its row
+            uint32_t *st = p.state + NS * b;
+            st[0] = 0u;
+            st[1] = nc > p.k ? (uint32_t)p.k : 0u;
+            st[2] = 0u;
+            st[3] = (uint32_t)nc;
+            st[4] = 0u;
+            st[5] = 0u;
+            st[6] = 0u;
+            st[7] = 0u;
         }
-        const int ii = warp_incl_scan(ni);
-        if (lane == 31) wt_items[warp] = ii;
+        const int ii = warp_incl_scan(ni), ic = warp_incl_scan(nchunk);
+        if (lane == 31) {
+            wt_items[warp] = ii;
+            wt_chunks[warp] = ic;
+        }
         __syncthreads();
         if (warp == 0) {
-            const int vi = lane < NW ? wt_items[lane] : 0;
-            const int si = warp_incl_scan(vi) - vi;
-            if (lane < NW) wt_items[lane] = si;
+            const int vi = lane < NW ? wt_items[lane] : 0, vc = lane < NW ? wt_chunks[lane] : 0;
+            const int si = warp_incl_scan(vi) - vi, sc = warp_incl_scan(vc) - vc;
+            if (lane < NW) {
+                wt_items[lane] = si;
+                wt_chunks[lane] = sc;
+            }
         }
         __syncthreads();
-        const int pi = carry_items + wt_items[warp] + ii;
-        if (b < p.B) p.item_start[b + 1] = pi;
+        const int pi = carry_items + wt_items[warp] + ii, pc = carry_chunks + wt_chunks[warp] + ic;
+        if (b < p.B) {
+            p.item_start[b + 1] = pi;
+            p.chunk_start[b + 1] = pc;
+        }
         __syncthreads();
-        if (threadIdx.x == FRONT_TH - 1) carry_items = pi;
+        if (threadIdx.x == FRONT_TH - 1) {
+            carry_items = pi;
+            carry_chunks = pc;
+        }
         __syncthreads();
     }
-    // the item table, a warp per sequence (item_start was written by this block: visible after the
-    // barrier)
+    // the item table and the query of every chunk, a warp per sequence (item_start and chunk_start
+    // were written by this block: visible after the barrier)
     for (int b = warp; b < p.B; b += NW) {
+        for (int c = p.chunk_start[b] + lane; c < p.chunk_start[b + 1]; c += 32) p.chunk_query[c] = b;
         const int64_t off = p.offs[b], S = p.offs[b + 1] - off;
         int F = p.count[b];
         F = F < 0 ? 0 : (F > S ? (int)S : F);
@@ -226,168 +262,183 @@ __global__ void __launch_bounds__(256) k_step_hist(const float *__restrict__ Y, 
         atomicAdd(h + bin_of(float_to_ordered(Y[off + j])), 1);
 }
 
-// Dynamic shared memory of k_ss_select: kpow2 selection keys, SCAP staged keys, HB bin counters.
-__host__ __device__ inline size_t select_smem(int kpow2)
+// Called by every thread of the chunk CTA after its appends are in global memory: true in the CTA
+// that finishes the query's chunks last.
+__device__ __forceinline__ bool last_chunk_of_query(int *done, int nch)
 {
-    return sizeof(unsigned long long) * ((size_t)kpow2 + SCAP) + sizeof(int) * (size_t)HB;
+    __shared__ int is_last;
+    __threadfence();  // this CTA's global writes before its count
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(done, 1) == nch - 1;
+    __syncthreads();
+    if (!is_last) return false;
+    __threadfence();  // the other chunks' writes, counted before ours, are read after this
+    return true;
 }
 
-__global__ void __launch_bounds__(SEL_TH, 1) k_ss_select(const float *__restrict__ Y, const int32_t *__restrict__ count,
-                                                         const int64_t *__restrict__ offs, const float *__restrict__ tail,
-                                                         const int32_t *__restrict__ tail_count, int W,
-                                                         const int *__restrict__ ghist, const int32_t *__restrict__ idx,
-                                                         int k, int kpow2, int32_t *__restrict__ topk_idx,
-                                                         float *__restrict__ topk_score)
+// Dynamic shared memory of k_ss_write: the histogram (HB ints) while the chunk appends; then, in
+// the query's last chunk, kpow2 selection keys, SCAP staged keys, kpow2 keys of scratch and SEL_NB
+// bucket counters.
+__host__ __device__ inline size_t write_smem(int kpow2)
 {
-    extern __shared__ unsigned long long sk[];  // [kpow2] selection, [SCAP] stage, then HB ints
-    unsigned long long *stage = sk + kpow2;
-    int *hs = (int *)(stage + SCAP);
+    const size_t fin = sizeof(unsigned long long) * (2 * (size_t)kpow2 + SCAP) + sizeof(int) * (size_t)SEL_NB;
+    const size_t hist = sizeof(int) * (size_t)HB;
+    return fin > hist ? fin : hist;
+}
+
+__global__ void __launch_bounds__(SEL_TH, 1) k_ss_write(const float *__restrict__ Y, const int32_t *__restrict__ count,
+                                                        const int64_t *__restrict__ offs,
+                                                        const float *__restrict__ tail,
+                                                        const int32_t *__restrict__ tail_count, int W, int B,
+                                                        const int *__restrict__ chunk_start,
+                                                        const int *__restrict__ chunk_query, uint32_t *state,
+                                                        const int *__restrict__ ghist, int kcap,
+                                                        unsigned long long *sel, unsigned long long *stage,
+                                                        const int32_t *__restrict__ idx, int k, int kpow2,
+                                                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_score)
+{
+    extern __shared__ unsigned long long dsm[];
     __shared__ int warp_tot[32];
-    __shared__ int tot_a, tot_b, s_bin, s_above, s_nst, s_maxseg;
-    const int b = blockIdx.x;
+    __shared__ int tot_a, s_bin, s_above, s_dig, s_dabove, s_dn, s_n;
+    const int c = blockIdx.x;
+    if (c >= chunk_start[B]) return;
+    const int b = chunk_query[c];
+    uint32_t *st = state + NS * b;
     const Query q = query(b, Y, count, offs, tail, tail_count, W);
     const int nc = q.F0 + q.nt;
+    const int j0 = (c - chunk_start[b]) * CH, j1 = min(nc, j0 + CH);
+    const bool every = st[1] == 0u;  // at most k candidates: every one, whatever its key
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     auto key64 = [](uint32_t u, int j) { return ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j); };
-    auto emit = [&](int r, unsigned long long v) {
+    uint32_t beta = 0;
+    int above = 0;
+    if (!every) {
+        // the bin of the k-th largest key, from the scorer's histogram and the window entries
+        int *hs = (int *)dsm;
+        const int4 *g4 = (const int4 *)(ghist + (int64_t)b * HB);
+        for (int t = threadIdx.x; t < HB / 4; t += SEL_TH) ((int4 *)hs)[t] = __ldg(g4 + t);
+        __syncthreads();
+        for (int j = q.F0 + threadIdx.x; j < nc; j += SEL_TH) atomicAdd(&hs[bin_of(key_of(q, j))], 1);
+        __syncthreads();
+        sel_find_bin<HB>((const unsigned int *)hs, k, warp_tot, &tot_a, &s_bin, &s_above);
+        beta = (uint32_t)s_bin;
+        above = s_above;
+    }
+    // this chunk's appends: keys of higher bins to the selection, bin beta's to the stage
+    unsigned long long *out = sel + (int64_t)b * kcap;
+    unsigned long long *stg = stage + q.off + (int64_t)b * W;  // capacity S_b + W
+    for (int base = j0; base < j1; base += SEL_TH) {
+        const int j = base + threadIdx.x;
+        uint32_t u = 0;
+        bool gt = false, eq = false;
+        if (j < j1) {
+            u = key_of(q, j);
+            const uint32_t bn = bin_of(u);
+            gt = every || bn > beta;
+            eq = !every && bn == beta;
+        }
+        const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+        int pg = 0, pe = 0;
+        if (lane == 0) {
+            if (bg) pg = (int)atomicAdd(st + 4, (uint32_t)__popc(bg));
+            if (be) pe = (int)atomicAdd(st + 5, (uint32_t)__popc(be));
+        }
+        pg = __shfl_sync(0xffffffffu, pg, 0);
+        pe = __shfl_sync(0xffffffffu, pe, 0);
+        if (gt) out[pg + __popc(bg & lt)] = key64(u, j);
+        if (eq) stg[pe + __popc(be & lt)] = key64(u, j);
+    }
+    if (!last_chunk_of_query((int *)(st + 6), chunk_start[b + 1] - chunk_start[b])) return;
+
+    // ---- the query's final step: the want largest staged keys complete the selection; its order
+    unsigned long long *sk = dsm;                   // kpow2
+    unsigned long long *ss = sk + kpow2;            // SCAP
+    unsigned long long *tmp = ss + SCAP;            // kpow2
+    int *cnt = (int *)(tmp + kpow2);                // SEL_NB
+    int *h256 = cnt;                                // (the radix select's digits, before the order)
+    const int nsel = nc < k ? nc : k;
+    const int nfirst = every ? nsel : above;  // keys already in the selection
+    __syncthreads();                          // the histogram in shared memory is done with
+    for (int t = threadIdx.x; t < nfirst; t += SEL_TH) sk[t] = __ldcg(out + t);
+    if (!every) {
+        const int want = k - above;
+        const int ns = (int)__ldcg(st + 5);  // the keys of bin beta
+        if (ns <= SCAP) {
+            int np = 64;
+            while (np < ns) np <<= 1;
+            for (int t = threadIdx.x; t < np; t += SEL_TH) ss[t] = t < ns ? __ldcg(stg + t) : 0ull;
+            block_sort_desc_u64(ss, np);
+            for (int t = threadIdx.x; t < want; t += SEL_TH) sk[above + t] = ss[t];
+        } else {
+            // a crowded bin: radix select of the want-th largest key over the stage, 8 bits at a
+            // time from the top, until the digit's keys are exactly the ones still wanted
+            unsigned long long prefix = 0ull, pmask = 0ull;
+            int remaining = want;
+            for (int pos = 64; pos > 0;) {
+                const int wb = pos >= 8 ? 8 : pos, sh = pos - wb;
+                const unsigned long long dm = (1ull << wb) - 1ull;
+                for (int t = threadIdx.x; t < 256; t += SEL_TH) h256[t] = 0;
+                __syncthreads();
+                for (int i = threadIdx.x; i < ns; i += SEL_TH) {
+                    const unsigned long long v = __ldcg(stg + i);
+                    if ((v & pmask) == prefix) atomicAdd(&h256[(int)((v >> sh) & dm)], 1);
+                }
+                __syncthreads();
+                if (threadIdx.x < 32) {  // the digit holding the remaining-th largest key, from the top
+                    int cc[8], sum = 0;
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        cc[i] = h256[255 - 8 * lane - i];
+                        sum += cc[i];
+                    }
+                    int ab = warp_incl_scan(sum) - sum;
+                    if (ab < remaining && ab + sum >= remaining) {
+#pragma unroll
+                        for (int i = 0; i < 8; i++) {
+                            if (ab + cc[i] >= remaining) {
+                                s_dig = 255 - 8 * lane - i;
+                                s_dabove = ab;
+                                s_dn = cc[i];
+                                break;
+                            }
+                            ab += cc[i];
+                        }
+                    }
+                }
+                __syncthreads();
+                prefix |= (unsigned long long)s_dig << sh;
+                pmask |= dm << sh;
+                remaining -= s_dabove;
+                pos = sh;
+                const bool whole = s_dn == remaining;  // every key of the digit is wanted
+                __syncthreads();
+                if (whole) break;
+            }
+            // the wanted keys are exactly those >= prefix (its bits below the last pass are zero)
+            if (threadIdx.x == 0) s_n = 0;
+            __syncthreads();
+            for (int i = threadIdx.x; i < ns; i += SEL_TH) {
+                const unsigned long long v = __ldcg(stg + i);
+                if (v >= prefix) {
+                    const int pos = atomicAdd(&s_n, 1);
+                    if (pos < want) sk[above + pos] = v;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    order_desc(sk, nsel, kpow2, tmp, cnt, RANK_SEG, [&](int r, unsigned long long v) {
         const int64_t o = (int64_t)b * k + r;
         const int j = (int)~(uint32_t)(v & 0xffffffffull);  // candidate slot
         topk_idx[o] = (j >= 0 && j < q.F0) ? __ldg(idx + q.off + j)
                                            : ((j >= q.F0 && j < nc) ? (int32_t)(q.S + (j - q.F0)) : -1);
         if (topk_score) topk_score[o] = ordered_to_float((uint32_t)(v >> 32));
-    };
-    for (int t = threadIdx.x; t < kpow2; t += SEL_TH) sk[t] = 0ull;
-    if (nc <= k) {
-        __syncthreads();
-        for (int j = threadIdx.x; j < nc; j += SEL_TH) sk[j] = key64(key_of(q, j), j);
-    } else {
-        // the histogram: the fetched entries' (from the scorer) and the window entries'
-        const int4 *g4 = (const int4 *)(ghist + (int64_t)b * HB);
-        for (int t = threadIdx.x; t < HB / 4; t += SEL_TH) ((int4 *)hs)[t] = __ldg(g4 + t);
-        if (threadIdx.x == 0) {
-            s_nst = 0;
-            s_maxseg = 0;
-        }
-        __syncthreads();
-        for (int j = q.F0 + threadIdx.x; j < nc; j += SEL_TH) atomicAdd(&hs[bin_of(key_of(q, j))], 1);
-        __syncthreads();
-        const int my_above = sel_find_bin<HB>((const unsigned int *)hs, k, warp_tot, &tot_a, &s_bin, &s_above);
-        const uint32_t beta = (uint32_t)s_bin;
-        const int above = s_above;              // keys of higher bins: all selected
-        const int nbeta = hs[beta];
-        const bool staged = nbeta <= SCAP;
-        const int want = k - above;             // keys still to take from bin beta (>= 1)
-        __syncthreads();                        // every thread has read hs[beta] before the bins change
-        {
-            // every bin above beta becomes the start of its segment of the selection
-            constexpr int PER = HB / SEL_TH;
-            const int hi = HB - PER * (int)threadIdx.x;
-            int run = my_above, mx = 0;
-#pragma unroll
-            for (int i = 1; i <= PER; i++) {
-                const int bin = hi - i;
-                if (bin > (int)beta) {
-                    const int c = hs[bin];
-                    hs[bin] = run;
-                    run += c;
-                    mx = max(mx, c);
-                }
-            }
-            mx = __reduce_max_sync(0xffffffffu, mx);
-            if (lane == 0) atomicMax(&s_maxseg, mx);
-        }
-        __syncthreads();
-        // higher bins scattered to their segments, bin beta to the stage (any order)
-        for (int base = 0; base < nc; base += SEL_TH) {
-            const int j = base + threadIdx.x;
-            uint32_t u = 0;
-            bool eq = false;
-            if (j < nc) {
-                u = key_of(q, j);
-                const uint32_t bn = bin_of(u);
-                if (bn > beta) sk[atomicAdd(&hs[bn], 1)] = key64(u, j);
-                eq = staged && bn == beta;
-            }
-            const unsigned be = __ballot_sync(0xffffffffu, eq);
-            int pe = 0;
-            if (lane == 0 && be) pe = atomicAdd(&s_nst, __popc(be));
-            pe = __shfl_sync(0xffffffffu, pe, 0);
-            if (eq) stage[pe + __popc(be & lt)] = key64(u, j);
-        }
-        __syncthreads();
-        if (staged) {
-            int np = 64;
-            while (np < nbeta) np <<= 1;
-            for (int t = nbeta + threadIdx.x; t < np; t += SEL_TH) stage[t] = 0ull;
-            block_sort_desc_u64(stage, np);
-            if (s_maxseg <= RANK_SEG) {
-                // output position of a selected key = its segment's start + the keys of its segment
-                // above it; the stage's largest keys follow in order
-                for (int t = threadIdx.x; t < above; t += SEL_TH) {
-                    const unsigned long long v = sk[t];
-                    const uint32_t bn = bin_of((uint32_t)(v >> 32));
-                    const int lo = bn + 1 < (uint32_t)HB ? hs[bn + 1] : 0, hi = hs[bn];
-                    int r = lo;
-                    for (int i = lo; i < hi; i++) r += sk[i] > v;
-                    emit(r, v);
-                }
-                for (int t = threadIdx.x; t < want; t += SEL_TH) emit(above + t, stage[t]);
-                return;
-            }
-            for (int t = threadIdx.x; t < want; t += SEL_TH) sk[above + t] = stage[t];
-        } else {
-            // a crowded bin: four radix passes of 8 bits over its keys give the k-th key K; then the
-            // bin's keys above K and the first keys equal to K in slot order
-            unsigned int *h256 = (unsigned int *)stage;  // the stage is free here
-            uint32_t prefix = 0u, pmask = 0u;
-            int remaining = want;
-#pragma unroll 1
-            for (int pass = 0; pass < 4; pass++) {
-                const int sh = 24 - 8 * pass;
-                for (int t = threadIdx.x; t < 1024; t += SEL_TH) h256[t] = 0;
-                __syncthreads();
-                for (int j = threadIdx.x; j < nc; j += SEL_TH) {
-                    const uint32_t u = key_of(q, j);
-                    if ((u & pmask) == prefix && bin_of(u) == beta) atomicAdd(&h256[(u >> sh) & 255u], 1u);
-                }
-                __syncthreads();
-                sel_find_bin<1024>(h256, remaining, warp_tot, &tot_a, &s_bin, &s_above);
-                prefix |= (uint32_t)s_bin << sh;
-                remaining -= s_above;
-                pmask |= 255u << sh;
-                __syncthreads();
-            }
-            int cg = 0, ce = 0;
-            for (int base = 0; base < nc; base += SEL_TH) {
-                const int j = base + threadIdx.x;
-                uint32_t u = 0;
-                int gt = 0, eq = 0;
-                if (j < nc) {
-                    u = key_of(q, j);
-                    gt = bin_of(u) == beta && u > prefix;
-                    eq = u == prefix;
-                }
-                const int pg = block_excl_scan(gt, warp_tot, &tot_a) + cg;
-                const int pe = block_excl_scan(eq, warp_tot, &tot_b) + ce;
-                if (gt) sk[above + pg] = key64(u, j);
-                if (eq && pe < remaining) sk[k - remaining + pe] = key64(u, j);
-                cg += tot_a;
-                ce += tot_b;
-                __syncthreads();
-            }
-        }
-    }
-    block_sort_desc_u64(sk, kpow2);
-    const int nsel = nc < k ? nc : k;
-    for (int r = threadIdx.x; r < k; r += SEL_TH) {
-        if (r < nsel) {
-            emit(r, sk[r]);
-        } else {
-            const int64_t o = (int64_t)b * k + r;
-            topk_idx[o] = -1;
-            if (topk_score) topk_score[o] = -INFINITY;
-        }
+    });
+    for (int r = nsel + threadIdx.x; r < k; r += SEL_TH) {
+        const int64_t o = (int64_t)b * k + r;
+        topk_idx[o] = -1;
+        if (topk_score) topk_score[o] = -INFINITY;
     }
 }
 

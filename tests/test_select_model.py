@@ -71,51 +71,76 @@ def sel_bucket(u, ymin, scale):
     return np.where(nan, np.where(np.asarray(u) & np.uint32(0x80000000), 4095, 0), bk).astype(np.int64)
 
 
+def order_desc_model(v, max_seg=32, seed=0):
+    """order_desc: distinct 64-bit keys put in descending order by 4,096 buckets linear in the score
+    over the keys' own range, scattered into their buckets' segments in any order (shuffled here),
+    a key's position = its segment's start + the keys of its segment above it; a sort when a bucket
+    holds more than max_seg keys.  Returns the ordered keys."""
+    rng = np.random.default_rng(seed)
+    if v.size == 0:
+        return v
+    u = (v >> np.uint64(32)).astype(np.uint32)
+    ymin, scale = sel_range(u)
+    bk = sel_bucket(u, ymin, scale)
+    cnt = np.bincount(bk, minlength=4096)
+    if cnt.max() > max_seg:
+        return np.sort(v)[::-1]
+    start = np.cumsum(cnt[::-1])[::-1] - cnt
+    fill = start.copy()
+    tmp = np.zeros(v.size, dtype=np.uint64)
+    for t in rng.permutation(v.size):
+        tmp[fill[bk[t]]] = v[t]
+        fill[bk[t]] += 1
+    out = np.zeros(v.size, dtype=np.uint64)
+    tb = sel_bucket((tmp >> np.uint64(32)).astype(np.uint32), ymin, scale)
+    for t in range(v.size):
+        b = tb[t]
+        lo = fill[b + 1] if b + 1 < 4096 else 0  # the end of the next bucket up is this one's start
+        out[lo + int((tmp[lo:fill[b]] > tmp[t]).sum())] = tmp[t]
+    return out
+
+
 def select_model(u, k, scap=4096, seed=0):
-    """The decode-step select (k_ss_select, with the histogram the scorer counts): bins = the top 14
-    bits of the score key; keys of higher bins scattered into their bins' segments of the selection
-    in an arbitrary order (shuffled here) and ranked by counting within a segment, the k-th key's
-    bin's largest keys by a sort (at most scap keys) or, for a crowded bin, four radix passes over
-    the bin's keys and an ordered pass; returns the selected slots in output order."""
+    """The decode-step select (k_ss_write): the scorer's histogram of the top 14 bits of the score
+    keys gives the bin beta of the k-th largest key; keys of higher bins and of bin beta are
+    appended in an arbitrary order (shuffled here); bin beta's want largest keys by a sort (at most
+    scap keys) or a 64-bit radix select over the stage; the k keys ordered by order_desc; returns
+    the selected slots in output order."""
     rng = np.random.default_rng(seed)
     nc = u.size
     kk = key64(u)
     if nc <= k:
-        slots = rng.permutation(nc)
-        return slots[np.argsort(kk[slots])[::-1]]
-    bn = (u >> np.uint32(18)).astype(np.int64)
-    hist = np.bincount(bn, minlength=1 << 14)
-    beta, above = _find_bin(hist, k)
-    want = k - above
-    start = np.cumsum(hist[::-1])[::-1] - hist        # keys in higher bins
-    fill = start.copy()
-    sel = np.zeros(above, dtype=np.uint64)
-    for j in rng.permutation(np.nonzero(bn > beta)[0]):
-        sel[fill[bn[j]]] = kk[j]
-        fill[bn[j]] += 1
-    out = np.zeros(k, dtype=np.uint64)
-    for t in range(above):                            # rank within the segment [end of bin + 1, end of bin)
-        v = sel[t]
-        b = int(v >> np.uint64(50))
-        lo = fill[b + 1] if b + 1 < (1 << 14) else 0
-        out[lo + int((sel[lo:fill[b]] > v).sum())] = v
-    if hist[beta] <= scap:
-        staged = rng.permutation(np.nonzero(bn == beta)[0])
-        out[above:] = np.sort(kk[staged])[::-1][:want]
+        sel = kk[rng.permutation(nc)]
     else:
-        prefix, pmask, remaining = 0, 0, want
-        inb = bn == beta
-        for sh in (24, 16, 8, 0):
-            m = inb & ((u & np.uint32(pmask)) == prefix)
-            h = np.bincount((u[m] >> np.uint32(sh)) & np.uint32(255), minlength=1024)
-            d, ab = _find_bin(h, remaining)
-            prefix |= d << sh
-            remaining -= ab
-            pmask |= 255 << sh
-        gt = [j for j in np.nonzero(inb)[0] if u[j] > prefix]
-        eq = [j for j in range(nc) if u[j] == prefix][:remaining]
-        assert len(gt) == want - remaining
-        out[above:] = np.sort(kk[np.array(gt + eq, dtype=np.int64)])[::-1]
+        bn = (u >> np.uint32(18)).astype(np.int64)
+        hist = np.bincount(bn, minlength=1 << 14)
+        beta, above = _find_bin(hist, k)
+        want = k - above
+        gt = kk[rng.permutation(np.nonzero(bn > beta)[0])]
+        assert gt.size == above
+        staged = kk[rng.permutation(np.nonzero(bn == beta)[0])]
+        if staged.size <= scap:
+            top = np.sort(staged)[::-1][:want]
+        else:
+            prefix, pmask = np.uint64(0), np.uint64(0)
+            rem, pos = want, 64
+            while pos > 0:
+                wb = min(8, pos)
+                sh = pos - wb
+                dm = np.uint64((1 << wb) - 1)
+                m = (staged & pmask) == prefix
+                h = np.bincount(((staged[m] >> np.uint64(sh)) & dm).astype(np.int64), minlength=256)
+                d, ab = _find_bin(h, rem)
+                prefix |= np.uint64(d) << np.uint64(sh)
+                pmask |= dm << np.uint64(sh)
+                rem -= ab
+                pos = sh
+                if h[d] == rem:
+                    break
+            top = staged[staged >= prefix]
+            assert top.size == want
+        sel = np.concatenate([gt, top])
+    out = order_desc_model(sel, seed=seed)
     return (~out & np.uint64(0xFFFFFFFF)).astype(np.int64)
 
 
