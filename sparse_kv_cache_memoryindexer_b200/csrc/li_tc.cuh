@@ -38,7 +38,7 @@ constexpr int NQ = 4;              // decode queries per MMA (batched call; one 
 constexpr int NH = 64;             // heads
 constexpr int NCOL = NQ * NH;      // MMA N = 256 (TMEM columns per accumulator slot)
 constexpr int CH = 16;             // key tiles per work item (batched call; one decode step: CH_STEP)
-constexpr int CH_STEP = 4;
+constexpr int CH_STEP = 8;
 constexpr int MAX_STAGES = 8;
 constexpr int NRING = 4;           // claimed items in flight inside a CTA
 constexpr int HIST_SHIFT = 18;     // one decode step's score histogram: the top 14 bits of the

@@ -918,11 +918,13 @@ lsa_status lsa_indexer_train_step(const void *h, const void *W_dq, const void *W
         train::k_outer<VD, BM><<<gout(n_h, d), 256, 0, st>>>(dw, h, L, B, n_h, d, g_Ww);                     \
     } while (0)
     if (dt == LSA_F32) {
-        train::k_train_dc<DT_F32><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        if (B <= 8) train::k_train_dc<DT_F32, 8><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        else train::k_train_dc<DT_F32, train::DC_BMAX><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
         if (B <= 8) LSA_OUTER3(DT_F32, 8);
         else LSA_OUTER3(DT_F32, train::DC_BMAX);
     } else {
-        train::k_train_dc<DT_BF16><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        if (B <= 8) train::k_train_dc<DT_BF16, 8><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
+        else train::k_train_dc<DT_BF16, train::DC_BMAX><<<gdc, 256, 0, st>>>(dq, W_iuq, L, B, nq, r, dc);
         if (B <= 8) LSA_OUTER3(DT_BF16, 8);
         else LSA_OUTER3(DT_BF16, train::DC_BMAX);
     }

@@ -258,60 +258,70 @@ __global__ void __launch_bounds__(THREADS, 1) k_train_entries(const void *__rest
 }
 
 // dc[l][b][j] = sum_o dq[l][b][o] W_iuq[l][o][j] (W^IUQ read once, memory-bound): one CTA per
-// (layer, 512 columns, DC_OCH rows o); thread t takes columns 2t, 2t + 1 of the block (one 4- or
-// 8-byte load of W per row, coalesced, 16 rows in flight), the CTA's dq rows of all sequences sit in
-// shared memory, and the partial sums over the CTA's rows are added to dc (zeroed before) with
-// atomics.
+// (layer, DC_COLS columns, DC_OCH rows o); thread t takes 4 consecutive columns (one 8- or 16-byte
+// load of W per row, coalesced, 16 rows in flight) and keeps BM sequences' sums (BM = B rounded up
+// to 8 or 16, so no FMA is predicated off); the CTA's dq rows sit in shared memory as [o][BM]
+// (read as float4 broadcasts), and the partial sums over the CTA's rows are added to dc (zeroed
+// before) with atomics.
 constexpr int DC_BMAX = 16;
 constexpr int DC_OCH = 128;
-constexpr int DC_COLS = 512;
+constexpr int DC_COLS = 1024;
 
-template <int DT>
+template <int DT, int BM>
 __global__ void __launch_bounds__(256) k_train_dc(const float *__restrict__ dq, const void *__restrict__ W_iuq, int L,
                                                   int B, int nq, int r, float *__restrict__ dc)
 {
-    __shared__ float sdq[DC_BMAX][DC_OCH];
+    __shared__ float4 sdq4[DC_OCH][BM / 4];
+    float *sdq = (float *)sdq4;
     const int l = blockIdx.z;
     const int o0 = blockIdx.y * DC_OCH;
-    const int j = blockIdx.x * DC_COLS + 2 * threadIdx.x;
+    const int j = blockIdx.x * DC_COLS + 4 * threadIdx.x;
     const int on = min(DC_OCH, nq - o0);
-    for (int i = threadIdx.x; i < B * DC_OCH; i += 256) {
+    for (int i = threadIdx.x; i < BM * DC_OCH; i += 256) {  // coalesced over o
         const int bb = i / DC_OCH, o = i % DC_OCH;
-        sdq[bb][o] = o < on ? __ldg(dq + ((int64_t)l * B + bb) * nq + o0 + o) : 0.f;
+        sdq[o * BM + bb] = (o < on && bb < B) ? __ldg(dq + ((int64_t)l * B + bb) * nq + o0 + o) : 0.f;
     }
     __syncthreads();
-    if (j >= r) return;
-    float acc[DC_BMAX][2];
+    if (j >= r) return;  // r is a multiple of 4
+    float acc[BM][4];
 #pragma unroll
-    for (int bb = 0; bb < DC_BMAX; bb++) acc[bb][0] = acc[bb][1] = 0.f;
+    for (int bb = 0; bb < BM; bb++) acc[bb][0] = acc[bb][1] = acc[bb][2] = acc[bb][3] = 0.f;
     const int64_t wrow = (int64_t)l * nq + o0;
 #pragma unroll 16
     for (int o = 0; o < on; o++) {
-        float w0, w1;
+        float w[4];
         if (DT == DT_F32) {
-            const float2 v = __ldg((const float2 *)((const float *)W_iuq + (wrow + o) * r + j));
-            w0 = v.x;
-            w1 = v.y;
+            const float4 v = __ldg((const float4 *)((const float *)W_iuq + (wrow + o) * r + j));
+            w[0] = v.x;
+            w[1] = v.y;
+            w[2] = v.z;
+            w[3] = v.w;
         } else {
-            const uint32_t v = __ldg((const unsigned int *)((const unsigned short *)W_iuq + (wrow + o) * r + j));
-            w0 = bf16_bits_to_float((unsigned short)(v & 0xffffu));
-            w1 = bf16_bits_to_float((unsigned short)(v >> 16));
+            const uint2 v = __ldg((const uint2 *)((const unsigned short *)W_iuq + (wrow + o) * r + j));
+            w[0] = __uint_as_float(v.x << 16);
+            w[1] = __uint_as_float(v.x & 0xffff0000u);
+            w[2] = __uint_as_float(v.y << 16);
+            w[3] = __uint_as_float(v.y & 0xffff0000u);
         }
 #pragma unroll
-        for (int bb = 0; bb < DC_BMAX; bb++) {
-            if (bb < B) {
-                const float d = sdq[bb][o];
-                acc[bb][0] = fmaf(d, w0, acc[bb][0]);
-                acc[bb][1] = fmaf(d, w1, acc[bb][1]);
+        for (int bq = 0; bq < BM / 4; bq++) {
+            const float4 d = sdq4[o][bq];
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                acc[4 * bq + 0][c] = fmaf(d.x, w[c], acc[4 * bq + 0][c]);
+                acc[4 * bq + 1][c] = fmaf(d.y, w[c], acc[4 * bq + 1][c]);
+                acc[4 * bq + 2][c] = fmaf(d.z, w[c], acc[4 * bq + 2][c]);
+                acc[4 * bq + 3][c] = fmaf(d.w, w[c], acc[4 * bq + 3][c]);
             }
         }
     }
 #pragma unroll
-    for (int bb = 0; bb < DC_BMAX; bb++) {
+    for (int bb = 0; bb < BM; bb++) {
         if (bb < B) {
             float *dst = dc + ((int64_t)l * B + bb) * r + j;
-            if (acc[bb][0] != 0.f) atomicAdd(dst, acc[bb][0]);
-            if (acc[bb][1] != 0.f) atomicAdd(dst + 1, acc[bb][1]);
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                if (acc[bb][c] != 0.f) atomicAdd(dst + c, acc[bb][c]);
         }
     }
 }
