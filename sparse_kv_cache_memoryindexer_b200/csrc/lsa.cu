@@ -761,7 +761,8 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
     while (kpow2 < k) kpow2 <<= 1;
     const size_t smem = stepsel::write_smem(kpow2);
     LSA_TRY(set_smem(stepsel::k_ss_write, smem));
-    const int64_t mc = step_max_chunks(B, total_S, W);
+    // (the chunks are counted on the device: one CTA per SM walks them)
+    const int64_t mc = std::min<int64_t>(step_max_chunks(B, total_S, W), (int64_t)num_sms());
     stepsel::k_ss_write<<<(unsigned)mc, stepsel::SEL_TH, smem, st>>>(Y, count, seq_offsets, tail, tcnt, W, B, chunk_start,
                                                                      chunk_query, state, ghist, LSA_MAX_TOPK, sel, stage,
                                                                      idx, k, kpow2, topk_idx, topk_score);

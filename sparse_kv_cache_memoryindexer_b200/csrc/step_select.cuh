@@ -8,7 +8,8 @@
 //                  scorer's dense layout and the window entries' scores
 //   k_li_tc<1>     (li_tc.cuh) the fetched entries' scores, and their histogram: the top 14 bits
 //                  of the score key (HIST_BINS bins, li_tc.cuh) counted per sequence
-//   k_ss_write     one CTA per chunk: the query's histogram (plus its window entries) gives the bin
+//   k_ss_write     per chunk (one CTA per SM walks the chunks): the query's histogram (plus its
+//                  window entries) gives the bin
 //                  beta of the k-th largest key (each chunk finds the same); the chunk's keys of
 //                  higher bins are appended to the query's selection and bin beta's to its stage
 //                  (any order: the keys carry their slots).  The query's last chunk to finish then
@@ -286,22 +287,18 @@ __host__ __device__ inline size_t write_smem(int kpow2)
     return fin > hist ? fin : hist;
 }
 
-__global__ void __launch_bounds__(SEL_TH, 1) k_ss_write(const float *__restrict__ Y, const int32_t *__restrict__ count,
-                                                        const int64_t *__restrict__ offs,
-                                                        const float *__restrict__ tail,
-                                                        const int32_t *__restrict__ tail_count, int W, int B,
-                                                        const int *__restrict__ chunk_start,
-                                                        const int *__restrict__ chunk_query, uint32_t *state,
-                                                        const int *__restrict__ ghist, int kcap,
-                                                        unsigned long long *sel, unsigned long long *stage,
-                                                        const int32_t *__restrict__ idx, int k, int kpow2,
-                                                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_score)
+// One chunk of k_ss_write (and, in the query's last chunk to finish, the query's final step).
+__device__ __forceinline__ void write_chunk(int c, unsigned long long *dsm, int *warp_tot, int &tot_a, int &s_bin,
+                                            int &s_above, int &s_dig, int &s_dabove, int &s_dn, int &s_n,
+                                            const float *__restrict__ Y, const int32_t *__restrict__ count,
+                                            const int64_t *__restrict__ offs, const float *__restrict__ tail,
+                                            const int32_t *__restrict__ tail_count, int W, int B,
+                                            const int *__restrict__ chunk_start, const int *__restrict__ chunk_query,
+                                            uint32_t *state, const int *__restrict__ ghist, int kcap,
+                                            unsigned long long *sel, unsigned long long *stage,
+                                            const int32_t *__restrict__ idx, int k, int kpow2,
+                                            int32_t *__restrict__ topk_idx, float *__restrict__ topk_score)
 {
-    extern __shared__ unsigned long long dsm[];
-    __shared__ int warp_tot[32];
-    __shared__ int tot_a, s_bin, s_above, s_dig, s_dabove, s_dn, s_n;
-    const int c = blockIdx.x;
-    if (c >= chunk_start[B]) return;
     const int b = chunk_query[c];
     uint32_t *st = state + NS * b;
     const Query q = query(b, Y, count, offs, tail, tail_count, W);
@@ -439,6 +436,29 @@ __global__ void __launch_bounds__(SEL_TH, 1) k_ss_write(const float *__restrict_
         const int64_t o = (int64_t)b * k + r;
         topk_idx[o] = -1;
         if (topk_score) topk_score[o] = -INFINITY;
+    }
+}
+
+__global__ void __launch_bounds__(SEL_TH, 1) k_ss_write(const float *__restrict__ Y, const int32_t *__restrict__ count,
+                                                        const int64_t *__restrict__ offs,
+                                                        const float *__restrict__ tail,
+                                                        const int32_t *__restrict__ tail_count, int W, int B,
+                                                        const int *__restrict__ chunk_start,
+                                                        const int *__restrict__ chunk_query, uint32_t *state,
+                                                        const int *__restrict__ ghist, int kcap,
+                                                        unsigned long long *sel, unsigned long long *stage,
+                                                        const int32_t *__restrict__ idx, int k, int kpow2,
+                                                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_score)
+{
+    extern __shared__ unsigned long long dsm[];
+    __shared__ int warp_tot[32];
+    __shared__ int tot_a, s_bin, s_above, s_dig, s_dabove, s_dn, s_n;
+    const int nchunks = chunk_start[B];
+    for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
+        __syncthreads();  // shared memory of the previous chunk done with
+        write_chunk(c, dsm, warp_tot, tot_a, s_bin, s_above, s_dig, s_dabove, s_dn, s_n, Y, count, offs, tail,
+                    tail_count, W, B, chunk_start, chunk_query, state, ghist, kcap, sel, stage, idx, k, kpow2,
+                    topk_idx, topk_score);
     }
 }
 
