@@ -13,9 +13,9 @@
 //                  beta of the k-th largest key (each chunk finds the same); the chunk's keys of
 //                  higher bins are appended to the query's selection and bin beta's to its stage
 //                  (any order: the keys carry their slots).  The query's last chunk to finish then
-//                  takes the want largest staged keys (a sort in shared memory, or a radix select
-//                  over a crowded stage) and orders the k keys (order_desc: buckets over their own
-//                  score range, counting within a bucket).  A query with at most k candidates takes
+//                  orders the selection and the stage together (order_desc: buckets over their own
+//                  score range, counting within a bucket) and writes the first k (a crowded stage
+//                  is cut to its want largest keys by a radix select first).  A query with at most k candidates takes
 //                  them all.  The output is as the batched select writes it.
 #pragma once
 #include "select_common.cuh"
@@ -278,11 +278,19 @@ __device__ __forceinline__ bool last_chunk_of_query(int *done, int nch)
 }
 
 // Dynamic shared memory of k_ss_write: the histogram (HB ints) while the chunk appends; then, in
-// the query's last chunk, kpow2 selection keys, SCAP staged keys, kpow2 keys of scratch and SEL_NB
-// bucket counters.
+// the query's last chunk, order_cap keys to order, as many of scratch, and SEL_NB bucket counters.
+// Keys the final step may order: kpow2 + SCAP rounded up to a power of two (room for the bitonic
+// fallback's padding).
+__host__ __device__ inline int order_cap(int kpow2)
+{
+    int c = 64;
+    while (c < kpow2 + SCAP) c <<= 1;
+    return c;
+}
+
 __host__ __device__ inline size_t write_smem(int kpow2)
 {
-    const size_t fin = sizeof(unsigned long long) * (2 * (size_t)kpow2 + SCAP) + sizeof(int) * (size_t)SEL_NB;
+    const size_t fin = sizeof(unsigned long long) * 2 * (size_t)order_cap(kpow2) + sizeof(int) * (size_t)SEL_NB;
     const size_t hist = sizeof(int) * (size_t)HB;
     return fin > hist ? fin : hist;
 }
@@ -348,26 +356,27 @@ __device__ __forceinline__ void write_chunk(int c, unsigned long long *dsm, int 
     }
     if (!last_chunk_of_query((int *)(st + 6), chunk_start[b + 1] - chunk_start[b])) return;
 
-    // ---- the query's final step: the want largest staged keys complete the selection; its order
-    unsigned long long *sk = dsm;                   // kpow2
-    unsigned long long *ss = sk + kpow2;            // SCAP
-    unsigned long long *tmp = ss + SCAP;            // kpow2
-    int *cnt = (int *)(tmp + kpow2);                // SEL_NB
+    // ---- the query's final step.  With at most SCAP staged keys, the selection and the whole stage
+    // are ordered together (order_desc) and the first k positions written; otherwise a radix select
+    // over the stage picks its want largest keys first.
+    const int ocap = order_cap(kpow2);
+    unsigned long long *sk = dsm;                   // ocap
+    unsigned long long *tmp = sk + ocap;            // ocap
+    int *cnt = (int *)(tmp + ocap);                 // SEL_NB
     int *h256 = cnt;                                // (the radix select's digits, before the order)
     const int nsel = nc < k ? nc : k;
     const int nfirst = every ? nsel : above;  // keys already in the selection
+    int nord = nfirst;                        // keys to order
     __syncthreads();                          // the histogram in shared memory is done with
     for (int t = threadIdx.x; t < nfirst; t += SEL_TH) sk[t] = __ldcg(out + t);
     if (!every) {
         const int want = k - above;
         const int ns = (int)__ldcg(st + 5);  // the keys of bin beta
         if (ns <= SCAP) {
-            int np = 64;
-            while (np < ns) np <<= 1;
-            for (int t = threadIdx.x; t < np; t += SEL_TH) ss[t] = t < ns ? __ldcg(stg + t) : 0ull;
-            block_sort_desc_u64(ss, np);
-            for (int t = threadIdx.x; t < want; t += SEL_TH) sk[above + t] = ss[t];
+            for (int t = threadIdx.x; t < ns; t += SEL_TH) sk[above + t] = __ldcg(stg + t);
+            nord = above + ns;
         } else {
+            nord = k;
             // a crowded bin: radix select of the want-th largest key over the stage, 8 bits at a
             // time from the top, until the digit's keys are exactly the ones still wanted
             unsigned long long prefix = 0ull, pmask = 0ull;
@@ -425,7 +434,10 @@ __device__ __forceinline__ void write_chunk(int c, unsigned long long *dsm, int 
         }
     }
     __syncthreads();
-    order_desc(sk, nsel, kpow2, tmp, cnt, RANK_SEG, [&](int r, unsigned long long v) {
+    int npow2 = 64;
+    while (npow2 < nord) npow2 <<= 1;
+    order_desc(sk, nord, npow2, tmp, cnt, RANK_SEG, [&](int r, unsigned long long v) {
+        if (r >= k) return;  // a staged key below the k-th
         const int64_t o = (int64_t)b * k + r;
         const int j = (int)~(uint32_t)(v & 0xffffffffull);  // candidate slot
         topk_idx[o] = (j >= 0 && j < q.F0) ? __ldg(idx + q.off + j)

@@ -103,9 +103,9 @@ def order_desc_model(v, max_seg=32, seed=0):
 def select_model(u, k, scap=4096, seed=0):
     """The decode-step select (k_ss_write): the scorer's histogram of the top 14 bits of the score
     keys gives the bin beta of the k-th largest key; keys of higher bins and of bin beta are
-    appended in an arbitrary order (shuffled here); bin beta's want largest keys by a sort (at most
-    scap keys) or a 64-bit radix select over the stage; the k keys ordered by order_desc; returns
-    the selected slots in output order."""
+    appended in an arbitrary order (shuffled here); with at most scap staged keys the selection and
+    the stage are ordered together by order_desc and the first k kept, otherwise a 64-bit radix
+    select picks the stage's want largest keys first; returns the selected slots in output order."""
     rng = np.random.default_rng(seed)
     nc = u.size
     kk = key64(u)
@@ -120,25 +120,26 @@ def select_model(u, k, scap=4096, seed=0):
         assert gt.size == above
         staged = kk[rng.permutation(np.nonzero(bn == beta)[0])]
         if staged.size <= scap:
-            top = np.sort(staged)[::-1][:want]
-        else:
-            prefix, pmask = np.uint64(0), np.uint64(0)
-            rem, pos = want, 64
-            while pos > 0:
-                wb = min(8, pos)
-                sh = pos - wb
-                dm = np.uint64((1 << wb) - 1)
-                m = (staged & pmask) == prefix
-                h = np.bincount(((staged[m] >> np.uint64(sh)) & dm).astype(np.int64), minlength=256)
-                d, ab = _find_bin(h, rem)
-                prefix |= np.uint64(d) << np.uint64(sh)
-                pmask |= dm << np.uint64(sh)
-                rem -= ab
-                pos = sh
-                if h[d] == rem:
-                    break
-            top = staged[staged >= prefix]
-            assert top.size == want
+            # the selection and the whole stage ordered together; the first k kept
+            out = order_desc_model(np.concatenate([gt, staged]), seed=seed)[:k]
+            return (~out & np.uint64(0xFFFFFFFF)).astype(np.int64)
+        prefix, pmask = np.uint64(0), np.uint64(0)
+        rem, pos = want, 64
+        while pos > 0:
+            wb = min(8, pos)
+            sh = pos - wb
+            dm = np.uint64((1 << wb) - 1)
+            m = (staged & pmask) == prefix
+            h = np.bincount(((staged[m] >> np.uint64(sh)) & dm).astype(np.int64), minlength=256)
+            d, ab = _find_bin(h, rem)
+            prefix |= np.uint64(d) << np.uint64(sh)
+            pmask |= dm << np.uint64(sh)
+            rem -= ab
+            pos = sh
+            if h[d] == rem:
+                break
+        top = staged[staged >= prefix]
+        assert top.size == want
         sel = np.concatenate([gt, top])
     out = order_desc_model(sel, seed=seed)
     return (~out & np.uint64(0xFFFFFFFF)).astype(np.int64)
