@@ -37,6 +37,12 @@ namespace li {
 constexpr int NQ = 4;              // decode queries per MMA (batched call; one decode step: 1)
 constexpr int NH = 64;             // heads
 constexpr int NCOL = NQ * NH;      // MMA N = 256 (TMEM columns per accumulator slot)
+// accumulator slots in the 512 TMEM columns: 2 of 256 columns (4-query groups) or 8 of 64 (one
+// query: more tiles between the MMA and the epilogue, whose two warp halves take alternate tiles)
+template <int NQV> struct Acc {
+    static constexpr int N = NQV == 1 ? 8 : 2;
+    static constexpr uint32_t COLS = NQV == 1 ? NH : NCOL;
+};
 constexpr int CH = 16;             // key tiles per work item (batched call; one decode step: CH_STEP)
 constexpr int CH_STEP = 8;
 constexpr int MAX_STAGES = 8;
@@ -178,8 +184,8 @@ __global__ void __launch_bounds__(320, 1)
     auto empty = [&](int i) { return bars + 8u * (MAX_STAGES + i); };
     auto qfull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + i); };
     auto qempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 2 + i); };
-    auto tfull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 4 + i); };
-    auto tempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 6 + i); };
+    auto tfull = [&](int i) { return bars + 8u * (2 * MAX_STAGES + i); };    // i < MAX_STAGES (8)
+    auto tempty = [&](int i) { return bars + 8u * (3 * MAX_STAGES + i); };
     auto ifull = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 8 + i); };
     auto iempty = [&](int i) { return bars + 8u * (4 * MAX_STAGES + 8 + NRING + i); };
     uint32_t *tmem_holder = (uint32_t *)(base + sp.misc);
@@ -197,8 +203,10 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < 2; i++) {
             mbar_init(qfull(i), 1);
             mbar_init(qempty(i), 1);
+        }
+        for (int i = 0; i < Acc<NQV>::N; i++) {
             mbar_init(tfull(i), 1);
-            mbar_init(tempty(i), 8);
+            mbar_init(tempty(i), NQV == 1 ? 4 : 8);  // one query: the 4 warps of the tile's half
         }
         for (int i = 0; i < NRING; i++) {
             mbar_init(ifull(i), 1);
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(320, 1)
                     const uint32_t a_base = kraw + (uint32_t)stage * 128 * 256;
                     if (!mbar_wait(tempty(acc), accphase ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t d = tmem + (uint32_t)acc * NCOL;
+                    const uint32_t d = tmem + (uint32_t)acc * Acc<NQV>::COLS;
 #pragma unroll
                     for (int kk = 0; kk < DI / 16; kk++) {
                         const uint32_t ka = a_base + (uint32_t)(kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32;
@@ -309,7 +317,7 @@ __global__ void __launch_bounds__(320, 1)
                     if (++stage == p.stages) { stage = 0; phase ^= 1; }
                     mma_commit(tfull(acc));
                     if (kt == t1 - 1) mma_commit(qempty(qslot));
-                    if (++acc == 2) { acc = 0; accphase ^= 1; }
+                    if (++acc == Acc<NQV>::N) { acc = 0; accphase ^= 1; }
                 }
                 if (ok && t1 <= t0) mma_commit(qempty(qslot));  // an item without tiles still frees its slot
             }
@@ -318,10 +326,11 @@ __global__ void __launch_bounds__(320, 1)
     } else if (warp < 10) {
         // ------------------------------------------------------------- epilogue
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
-        const int half = (warp - 2) >> 2;        // queries 2*half, 2*half+1 of the group
-        const int nqw = NQV >= 4 ? 2 : (half == 0 ? NQV : 0);  // of them in the group
+        const int half = (warp - 2) >> 2;        // queries 2*half, 2*half+1 of the group (one query:
+                                                 // the half that takes alternate tiles)
+        const int nqw = NQV >= 4 ? 2 : NQV;      // this warp's queries of the group
         float *myw = sw + (size_t)(warp - 2) * 2 * NH;
-        int acc = 0;
+        int acc = 0, tseq = 0;
         uint32_t accphase = 0;
         bool ok = true;
         int islot = 0;
@@ -337,7 +346,7 @@ __global__ void __launch_bounds__(320, 1)
             const int64_t S = w.S;
             const int F = w.F;
             const int t0 = w.t0, t1 = w.t1;
-            const int i0 = NQV * w.g + 2 * half;  // first of this warp's queries
+            const int i0 = NQV * w.g + (NQV >= 4 ? 2 * half : 0);  // first of this warp's queries
             __syncwarp();
             for (int t = lane; t < nqw * NH; t += 32)
                 myw[t] = __ldg(p.wd + ((int64_t)w.b * p.tau + i0 + t / NH) * NH + (t % NH));
@@ -345,6 +354,10 @@ __global__ void __launch_bounds__(320, 1)
             const int64_t off = w.off;
             float *Yb = p.Y + (int64_t)p.tau * off;
             for (int kt = t0; kt < t1; kt++) {
+                if (NQV == 1 && ((tseq++ & 1) != half)) {  // the other half's tile
+                    if (++acc == Acc<NQV>::N) { acc = 0; accphase ^= 1; }
+                    continue;
+                }
                 const int64_t j = (int64_t)kt * TILE + quarter * 32 + lane;
                 const bool valid = j < F;
                 float sc = 1.f;
@@ -352,7 +365,8 @@ __global__ void __launch_bounds__(320, 1)
                 if (!mbar_wait_warp(tfull(acc), accphase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 if (p.hsc && valid && !(sc >= 0.f)) flag(ERRF_SCALE);
-                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * NCOL + 128 * half;
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * Acc<NQV>::COLS +
+                                       (NQV >= 4 ? 128 * half : 0);
                 float y[2] = {0.f, 0.f};
                 if (nqw == 0) {  // nothing of this warp in the slot: release it at once
                     tc_fence_before();
@@ -388,7 +402,7 @@ __global__ void __launch_bounds__(320, 1)
                     }
                     y[qq] = ((x0 + x1) + (x2 + x3)) * sc;  // ReLU(sc d) = sc ReLU(d) for sc >= 0
                 }
-                if (++acc == 2) { acc = 0; accphase ^= 1; }
+                if (++acc == Acc<NQV>::N) { acc = 0; accphase ^= 1; }
                 if (valid) {
                     if (nqw > 0) Yb[(int64_t)i0 * S + j] = y[0];
                     if (nqw > 1) Yb[(int64_t)(i0 + 1) * S + j] = y[1];

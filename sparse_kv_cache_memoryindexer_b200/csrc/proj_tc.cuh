@@ -27,7 +27,7 @@ namespace lsa {
 namespace proj {
 
 constexpr int KB = 64;              // K elements per box (one 128-byte swizzle atom of bf16)
-constexpr int MAX_BOX = 4;          // boxes per stage: 512 contiguous bytes of every weight row
+constexpr int MAX_BOX = 2;          // boxes per stage: 256 contiguous bytes of every weight row
 constexpr int KSPLIT_MAX = 8;       // K ranges of a split problem (partial slices)
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 6 * 32;
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(THREADS)
                 if (leader) {
                     mbar_expect_tx(full(stage), (uint32_t)nb * (A_BYTES + bbox));
                     const uint32_t dst = sbase + (uint32_t)stage * sbytes;
-                    for (int i = 0; i < nb; i++) {  // the boxes of a stage back to back: row segments of 512 bytes
+                    for (int i = 0; i < nb; i++) {  // the boxes of a stage back to back: row segments of 256 bytes
                         tma_load_2d(dst + (uint32_t)i * A_BYTES, wm, (kb + i) * KB, x.l * x.R + x.m0, full(stage));
                         tma_load_2d(dst + (uint32_t)p.nbox * A_BYTES + (uint32_t)i * bbox, &xmap, (kb + i) * KB,
                                     x.l * p.B, full(stage));
@@ -275,7 +275,7 @@ struct ProjProblem {
 
 // One launch over one or two problems sharing X bf16 [L][B][K]; a split problem's units store
 // partial slices, and ksplit_out[i] (nullable) reports how many.  One CTA per SM; a stage holds up
-// to MAX_BOX boxes of K so that every weight row is read in segments of 512 bytes.  Split problems
+// to MAX_BOX boxes of K so that every weight row is read in segments of 256 bytes.  Split problems
 // take the number of K ranges (at most KSPLIT_MAX, in whole stages) that balances the units best
 // over the CTAs.
 inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const bool *split, int nprob, int L, int B,
