@@ -157,15 +157,17 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     uint32_t *plane = bits + ((int64_t)i * Lc + l) * W32;
     float m = -INFINITY;
     {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        for (int64_t base = 0; base < S; base += 4 * THREADS) {
+        float m8[8];
 #pragma unroll
-            for (int q = 0; q < 4; q++) {
+        for (int q = 0; q < 8; q++) m8[q] = -INFINITY;
+        for (int64_t base = 0; base < S; base += 8 * THREADS) {  // eight loads in flight
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
                 const int64_t s = base + q * THREADS + threadIdx.x;
-                if (s < S) m4[q] = fmaxf(m4[q], __ldg(row + s));
+                if (s < S) m8[q] = fmaxf(m8[q], __ldg(row + s));
             }
         }
-        m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
     }
     m = block_max(m, fred);
 
@@ -178,12 +180,21 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
         // normal); each thread's fp32 sum of its S / THREADS terms rounds by at most that many
         // ulps; a result below the smallest normal is off by at most 2^-126 absolute
         float zf = 0.f;
-        for (int64_t base = 0; base < S; base += THREADS) {  // whole warps per step (warp-wide appends)
-            const int64_t s = base + threadIdx.x;
-            const float zs = s < S ? __ldg(row + s) : -INFINITY;
-            zf += s < S ? expf(zs - m) : 0.f;
-            warp_append(s < S && m - zs < 4.f,
-                        ((unsigned long long)float_to_ordered(zs) << 32) | (uint32_t)(~(uint32_t)s), &s_nc, cand);
+        for (int64_t base = 0; base < S; base += 4 * THREADS) {  // whole warps per step (warp-wide appends)
+            float zq[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {  // four loads in flight
+                const int64_t s = base + u * THREADS + threadIdx.x;
+                zq[u] = s < S ? __ldg(row + s) : -INFINITY;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int64_t s = base + u * THREADS + threadIdx.x;
+                zf += s < S ? expf(zq[u] - m) : 0.f;
+                warp_append(s < S && m - zq[u] < 4.f,
+                            ((unsigned long long)float_to_ordered(zq[u]) << 32) | (uint32_t)(~(uint32_t)s), &s_nc,
+                            cand);
+            }
         }
         const double Z32 = block_sum((double)zf, dred);
         // (plus the rounding of sums in double, here and in an fp64 Z: terms per thread + 64 ulps)

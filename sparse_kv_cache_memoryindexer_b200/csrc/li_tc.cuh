@@ -84,12 +84,12 @@ struct Smem {
 
 
 // Table entries of sequence b's items (items it0 ..): chunk c of ch key tiles and query group g at
-// it0 + c groups + g.  The lanes of one warp write them.
+// it0 + c groups + g.  nt threads write them, thread t every nt-th.
 __device__ __forceinline__ void write_items(ItemInfo *items, int it0, int b, int F, int S, int64_t off, int groups,
-                                           int ch, int lane)
+                                           int ch, int t, int nt)
 {
     const int tiles = (F + TILE - 1) / TILE, nch = (tiles + ch - 1) / ch;
-    for (int r = lane; r < nch * groups; r += 32) {
+    for (int r = t; r < nch * groups; r += nt) {
         const int c = r / groups;
         ItemInfo x;
         x.b = b;
@@ -117,52 +117,46 @@ __device__ __forceinline__ ItemInfo load_item(const ItemInfo *items, int it)
     return x;
 }
 
-// work items per sequence: ceil(ceil(F/128)/ch) chunks x groups, and their table.  One block.
-__global__ void __launch_bounds__(1024) k_li_items(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
-                                                   int B, int groups, int ch, int *__restrict__ item_start,
-                                                   int *__restrict__ item_counter, ItemInfo *__restrict__ items)
+// Work items per sequence: ceil(ceil(F/128)/ch) chunks x groups, and their table.  One block per
+// sequence: it sums the items of the sequences before it (its first item), writes item_start[b + 1]
+// and its table entries; block 0 also writes item_start[0] and zeroes the claim counter.
+__device__ __forceinline__ int items_of(const int32_t *count, const int64_t *offs, int s, int groups, int ch, int &F,
+                                        int64_t &S)
 {
-    __shared__ int warp_tot[32];
-    __shared__ int carry;
-    if (threadIdx.x == 0) {
-        carry = 0;
-        item_start[0] = 0;
-        *item_counter = 0;
-    }
+    S = offs[s + 1] - offs[s];
+    F = count[s];
+    F = F < 0 ? 0 : (F > S ? (int)S : F);
+    const int tiles = (F + TILE - 1) / TILE;
+    return ((tiles + ch - 1) / ch) * groups;
+}
+
+__global__ void __launch_bounds__(256) k_li_items(const int32_t *__restrict__ count, const int64_t *__restrict__ offs,
+                                                  int B, int groups, int ch, int *__restrict__ item_start,
+                                                  int *__restrict__ item_counter, ItemInfo *__restrict__ items)
+{
+    __shared__ int red[8];
+    const int b = blockIdx.x;
+    int part = 0, F;
+    int64_t S;
+    for (int s = threadIdx.x; s < b; s += 256) part += items_of(count, offs, s, groups, ch, F, S);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
     __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int base = 0; base < B; base += blockDim.x) {
-        const int b = base + threadIdx.x;
-        int n = 0;
-        if (b < B) {
-            const int64_t S = offs[b + 1] - offs[b];
-            int F = count[b];
-            if (F < 0 || F > S) flag(ERRF_COUNT);
-            F = F < 0 ? 0 : (F > S ? (int)S : F);
-            const int tiles = (F + TILE - 1) / TILE;
-            n = ((tiles + ch - 1) / ch) * groups;
+    int start = 0;
+#pragma unroll
+    for (int w = 0; w < 8; w++) start += red[w];
+    const int n = items_of(count, offs, b, groups, ch, F, S);
+    if (threadIdx.x == 0) {
+        const int F0 = count[b];
+        if (F0 < 0 || F0 > S) flag(ERRF_COUNT);
+        item_start[b + 1] = start + n;
+        if (b == 0) {
+            item_start[0] = 0;
+            *item_counter = 0;
         }
-        const int inc = warp_incl_scan(n);
-        if (lane == 31) warp_tot[warp] = inc;
-        __syncthreads();
-        if (warp == 0) {
-            const int v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
-            warp_tot[lane] = warp_incl_scan(v) - v;
-        }
-        __syncthreads();
-        const int pos = carry + warp_tot[warp] + inc;
-        if (b < B) item_start[b + 1] = pos;
-        __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) carry = pos;
-        __syncthreads();
     }
-    // the table, a warp per sequence (item_start was written by this block: visible after the barrier)
-    for (int b = warp; b < B; b += (int)(blockDim.x >> 5)) {
-        const int64_t off = offs[b], S = offs[b + 1] - off;
-        int F = count[b];
-        F = F < 0 ? 0 : (F > S ? (int)S : F);
-        write_items(items, item_start[b], b, F, (int)S, off, groups, ch, lane);
-    }
+    write_items(items, start, b, F, (int)S, offs[b], groups, ch, threadIdx.x, 256);
 }
 
 template <int NQV>  // queries per group: NQ (batched call) or 1 (one decode step)
@@ -462,7 +456,7 @@ inline lsa_status launch_li_tc(const void *qd, const float *wd, const void *hotK
     if (nq != NQ && nq != 1) return LSA_ERR_UNSUPPORTED;
     const int ch = li_item_tiles(nq);
     if (!planned) {
-        k_li_items<<<1, 1024, 0, st>>>(count, offs, B, tau / nq, ch, item_start, item_counter, items);
+        k_li_items<<<(unsigned)B, 256, 0, st>>>(count, offs, B, tau / nq, ch, item_start, item_counter, items);
         (*launches)++;
     }
     if (T == 0) return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;

@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(FRONT_TH) k_step_front(FrontParams p)
         const int64_t off = p.offs[b], S = p.offs[b + 1] - off;
         int F = p.count[b];
         F = F < 0 ? 0 : (F > S ? (int)S : F);
-        li::write_items(p.items, p.item_start[b], b, F, (int)S, off, 1, p.ch, lane);
+        li::write_items(p.items, p.item_start[b], b, F, (int)S, off, 1, p.ch, lane, 32);
     }
 }
 
