@@ -756,7 +756,15 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
         stepsel::k_step_hist<<<dim3(16, (unsigned)B), 256, 0, st>>>(Y, count, seq_offsets, ghist);
         LSA_TRY(launched("decode step: histogram"));
     }
-    // the select: one CTA per chunk of candidates, the query's last chunk completing it
+    // the select: the k-th key's bin per query, then the chunks of candidates, the query's last chunk
+    // completing it
+    {
+        const size_t hsm = sizeof(int) * (size_t)stepsel::HB;
+        LSA_TRY(set_smem(stepsel::k_ss_beta, hsm));
+        stepsel::k_ss_beta<<<(unsigned)B, stepsel::SEL_TH, hsm, st>>>(Y, count, seq_offsets, tail, tcnt, W, state, ghist,
+                                                                      k);
+        LSA_TRY(launched("decode step: bin of the k-th key"));
+    }
     int kpow2 = 64;  // the block sort works on at least 64 keys
     while (kpow2 < k) kpow2 <<= 1;
     const size_t smem = stepsel::write_smem(kpow2);
@@ -767,7 +775,6 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride, c
                                                                      chunk_query, state, ghist, LSA_MAX_TOPK, sel, stage,
                                                                      idx, k, kpow2, topk_idx, topk_score);
     LSA_TRY(launched("decode step: select"));
-    g_launches.fetch_add(2, std::memory_order_relaxed);  // front, select
     return ok();
 }
 

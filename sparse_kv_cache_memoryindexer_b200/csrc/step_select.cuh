@@ -1,4 +1,4 @@
-// Top-k of one decode step (three launches).  A step has one query per sequence; its candidates
+// Top-k of one decode step (four launches).  A step has one query per sequence; its candidates
 // are the F fetched slots, then the window entries as candidates F .. F + n - 1 (reported as
 // entries S_b + j).  A candidate's 64-bit key is (order-preserving score key << 32) | ~slot: larger
 // score first, then smaller slot, and no two keys are equal.
@@ -8,10 +8,10 @@
 //                  scorer's dense layout and the window entries' scores
 //   k_li_tc<1>     (li_tc.cuh) the fetched entries' scores, and their histogram: the top 14 bits
 //                  of the score key (HIST_BINS bins, li_tc.cuh) counted per sequence
-//   k_ss_write     per chunk (one CTA per SM walks the chunks): the query's histogram (plus its
-//                  window entries) gives the bin
-//                  beta of the k-th largest key (each chunk finds the same); the chunk's keys of
-//                  higher bins are appended to the query's selection and bin beta's to its stage
+//   k_ss_beta      one CTA per query: the histogram plus the window entries give the bin beta of
+//                  the k-th largest key
+//   k_ss_write     per chunk (one CTA per SM walks the chunks): the chunk's keys of higher bins are
+//                  appended to the query's selection and bin beta's to its stage
 //                  (any order: the keys carry their slots).  The query's last chunk to finish then
 //                  orders the selection and the stage together (order_desc: buckets over their own
 //                  score range, counting within a bucket) and writes the first k (a crowded stage
@@ -263,6 +263,34 @@ __global__ void __launch_bounds__(256) k_step_hist(const float *__restrict__ Y, 
         atomicAdd(h + bin_of(float_to_ordered(Y[off + j])), 1);
 }
 
+// Per query with more than k candidates (one CTA of SEL_TH threads each): the bin beta of the k-th
+// largest key from the scorer's histogram plus the window entries, into state words 0 (beta) and 2
+// (keys of higher bins).  Dynamic shared memory: HB ints.
+__global__ void __launch_bounds__(SEL_TH, 1) k_ss_beta(const float *__restrict__ Y, const int32_t *__restrict__ count,
+                                                       const int64_t *__restrict__ offs, const float *__restrict__ tail,
+                                                       const int32_t *__restrict__ tail_count, int W,
+                                                       uint32_t *state, const int *__restrict__ ghist, int k)
+{
+    extern __shared__ int hs[];
+    __shared__ int warp_tot[32];
+    __shared__ int tot_a, s_bin, s_above;
+    const int b = blockIdx.x;
+    uint32_t *st = state + NS * b;
+    if (st[1] == 0u) return;  // at most k candidates: no bin needed
+    const Query q = query(b, Y, count, offs, tail, tail_count, W);
+    const int nc = q.F0 + q.nt;
+    const int4 *g4 = (const int4 *)(ghist + (int64_t)b * HB);
+    for (int t = threadIdx.x; t < HB / 4; t += SEL_TH) ((int4 *)hs)[t] = __ldg(g4 + t);
+    __syncthreads();
+    for (int j = q.F0 + threadIdx.x; j < nc; j += SEL_TH) atomicAdd(&hs[bin_of(key_of(q, j))], 1);
+    __syncthreads();
+    sel_find_bin<HB>((const unsigned int *)hs, k, warp_tot, &tot_a, &s_bin, &s_above);
+    if (threadIdx.x == 0) {
+        st[0] = (uint32_t)s_bin;
+        st[2] = (uint32_t)s_above;
+    }
+}
+
 // Called by every thread of the chunk CTA after its appends are in global memory: true in the CTA
 // that finishes the query's chunks last.
 __device__ __forceinline__ bool last_chunk_of_query(int *done, int nch)
@@ -277,8 +305,8 @@ __device__ __forceinline__ bool last_chunk_of_query(int *done, int nch)
     return true;
 }
 
-// Dynamic shared memory of k_ss_write: the histogram (HB ints) while the chunk appends; then, in
-// the query's last chunk, order_cap keys to order, as many of scratch, and SEL_NB bucket counters.
+// Dynamic shared memory of k_ss_write (the query's last chunk): order_cap keys to order, as many of
+// scratch, and SEL_NB bucket counters.
 // Keys the final step may order: kpow2 + SCAP rounded up to a power of two (room for the bitonic
 // fallback's padding).
 __host__ __device__ inline int order_cap(int kpow2)
@@ -290,9 +318,7 @@ __host__ __device__ inline int order_cap(int kpow2)
 
 __host__ __device__ inline size_t write_smem(int kpow2)
 {
-    const size_t fin = sizeof(unsigned long long) * 2 * (size_t)order_cap(kpow2) + sizeof(int) * (size_t)SEL_NB;
-    const size_t hist = sizeof(int) * (size_t)HB;
-    return fin > hist ? fin : hist;
+    return sizeof(unsigned long long) * 2 * (size_t)order_cap(kpow2) + sizeof(int) * (size_t)SEL_NB;
 }
 
 // One chunk of k_ss_write (and, in the query's last chunk to finish, the query's final step).
@@ -316,20 +342,8 @@ __device__ __forceinline__ void write_chunk(int c, unsigned long long *dsm, int 
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     auto key64 = [](uint32_t u, int j) { return ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j); };
-    uint32_t beta = 0;
-    int above = 0;
-    if (!every) {
-        // the bin of the k-th largest key, from the scorer's histogram and the window entries
-        int *hs = (int *)dsm;
-        const int4 *g4 = (const int4 *)(ghist + (int64_t)b * HB);
-        for (int t = threadIdx.x; t < HB / 4; t += SEL_TH) ((int4 *)hs)[t] = __ldg(g4 + t);
-        __syncthreads();
-        for (int j = q.F0 + threadIdx.x; j < nc; j += SEL_TH) atomicAdd(&hs[bin_of(key_of(q, j))], 1);
-        __syncthreads();
-        sel_find_bin<HB>((const unsigned int *)hs, k, warp_tot, &tot_a, &s_bin, &s_above);
-        beta = (uint32_t)s_bin;
-        above = s_above;
-    }
+    const uint32_t beta = st[0];      // the bin of the k-th largest key (k_ss_beta)
+    const int above = (int)st[2];     // keys of higher bins
     // this chunk's appends: keys of higher bins to the selection, bin beta's to the stage
     unsigned long long *out = sel + (int64_t)b * kcap;
     unsigned long long *stg = stage + q.off + (int64_t)b * W;  // capacity S_b + W
@@ -367,7 +381,6 @@ __device__ __forceinline__ void write_chunk(int c, unsigned long long *dsm, int 
     const int nsel = nc < k ? nc : k;
     const int nfirst = every ? nsel : above;  // keys already in the selection
     int nord = nfirst;                        // keys to order
-    __syncthreads();                          // the histogram in shared memory is done with
     for (int t = threadIdx.x; t < nfirst; t += SEL_TH) sk[t] = __ldcg(out + t);
     if (!every) {
         const int want = k - above;
