@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -13,6 +14,7 @@
 #include "project.cuh"
 #include "score_select.cuh"
 #include "score_tc.cuh"
+#include "score_pair.cuh"
 #include "li_tc.cuh"
 #include "proj_tc.cuh"
 #include "golden.cuh"
@@ -197,6 +199,17 @@ lsa_status li_simt_d(int kdt, const void *qd, const float *wd, const void *hotK,
     }
 }
 
+// The E4M3 score runs on CTA pairs unless LSA_SCORE_PAIR=0 (the one-CTA kernel, k_score_tc, the
+// same result).
+bool score_pair_enabled()
+{
+    static const bool on = [] {
+        const char *v = getenv("LSA_SCORE_PAIR");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
+
 bool valid_dtype(int dt) { return dt == DT_F32 || dt == DT_BF16 || dt == DT_FP8; }
 
 }  // namespace
@@ -344,7 +357,19 @@ lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *
         k_tile_setup<<<1, 1024, 0, st>>>(seq_offsets, B, total_S, ws.tile_start, ws.chunk_start, count_out);
         LSA_TRY(launched("tile setup"));
     }
-    if (tc) {
+    if (tc && kdt == LSA_FP8_E4M3 && score_pair_enabled() && score_pair_supported(DT_FP8, B, num_sms())) {
+        // E4M3 keys on CTA pairs (score_pair.cuh): the query split (with the tile setup), then the score
+        const int R = L * B * tc::NH;
+        tc::k_q_split_e4m3<<<(R + 7) / 8 + 1, 256, 0, st>>>((const __nv_bfloat16 *)q, w, (uint8_t *)ws.qh, ws.wh, R,
+                                                            seq_offsets, B, total_S, ws.tile_start, ws.chunk_start,
+                                                            count_out);
+        LSA_TRY(launched("E4M3 query split"));
+        const lsa_status s = launch_score_pair(ws.qh, ws.wh, K, k_scale, seq_offsets, ws.tile_start, B, total_S, L,
+                                               thr_logit, scores_out, ws.tile_mask, num_sms(), st);
+        if (s != LSA_OK) return fail(s, "lsa_memindex_score_select: CTA-pair launch failed (%s)",
+                                     cudaGetErrorString(cudaGetLastError()));
+        LSA_TRY(launched("index score (CTA pairs)"));
+    } else if (tc) {
         int n = 0;
         const lsa_status s = launch_score_tc(q, w, K, k_scale, kdt, seq_offsets, ws.tile_start, ws.chunk_start,
                                              count_out, B, total_S, L, thr_logit, scores_out, ws.tile_mask, ws.qh,
