@@ -96,21 +96,24 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one k_score_tc launch, from one ncu
-# capture of a smaller batch of the same workload, per entry and layer: the kernel streams every key
-# row once, so the traffic grows in proportion to the entries.  Reported only while the kernel sources
-# hash to the value the capture was taken on (null otherwise).
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the score kernel,
+# from one ncu capture of a smaller batch of the same workload, per entry and layer: the kernel
+# streams every key row once, so the traffic grows in proportion to the entries.  Reported only
+# while the kernel's sources hash to the value the capture was taken on (null otherwise).
 SCORE_TRAFFIC = {
-    "fp8": {"bytes_per_entry_layer": 133.10, "capture": "ctx1m_fp8_b32 with B=4 (1,048,576 entries x 3 layers)"},
-    "bf16": {"bytes_per_entry_layer": 260.23, "capture": "ctx500k_bf16_b8 with B=2 (262,144 entries x 3 layers)"},
+    "fp8": {"bytes_per_entry_layer": 134.11, "capture": "ctx1m_fp8_b32 with B=4 (1,048,576 entries x 3 layers)",
+            "kernel": "k_score_pair", "sources": ("score_pair.cuh", "score_tc.cuh", "tc_common.cuh", "common.cuh"),
+            "hash": "3a38e0b395165e2e"},
+    "bf16": {"bytes_per_entry_layer": 260.23, "capture": "ctx500k_bf16_b8 with B=2 (262,144 entries x 3 layers)",
+             "kernel": "k_score_tc<0>", "sources": ("score_tc.cuh", "tc_common.cuh", "common.cuh"),
+             "hash": "75fc9bee86641ea6"},
 }
-SCORE_TRAFFIC_SRC = "75fc9bee86641ea6"
 
 
-def score_kernel_src_hash():
+def score_kernel_src_hash(sources=("score_tc.cuh", "tc_common.cuh", "common.cuh")):
     import hashlib
     h = hashlib.sha256()
-    for f in ("score_tc.cuh", "tc_common.cuh", "common.cuh"):
+    for f in sources:
         with open(os.path.join(ROOT, "sparse_kv_cache_memoryindexer_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -118,9 +121,9 @@ def score_kernel_src_hash():
 
 def score_traffic(wl):
     tr = SCORE_TRAFFIC.get(wl.kdtype)
-    if tr is None or score_kernel_src_hash() != SCORE_TRAFFIC_SRC:
+    if tr is None or score_kernel_src_hash(tr["sources"]) != tr["hash"]:
         return None, None
-    return tr["bytes_per_entry_layer"] * wl.L * wl.total_S, tr["capture"]
+    return tr["bytes_per_entry_layer"] * wl.L * wl.total_S, tr["kernel"] + ": " + tr["capture"]
 
 
 # ------------------------------------------------------------------------------------ clocks
@@ -766,7 +769,7 @@ def run_lsa(args, rank, world, device):
                              frac=score_gbs / peaks["hbm_gbs"], frac_of_nominal_8tbs=score_gbs / 8000.0,
                              traffic=traffic,
                              traffic_note=None if traffic is None else
-                             "ncu DRAM bytes of k_score_tc on %s, scaled by entries" % traffic_src,
+                             "ncu DRAM bytes of %s, scaled by entries" % traffic_src,
                              bytes_per_launch=alg["score_bytes"], peak_source=peaks["source"]),
             "rooflines": rooflines,
             "gpu_launches": launches,
