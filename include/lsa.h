@@ -290,7 +290,8 @@ lsa_status lsa_lightning_topk_step(const void *q_step, int64_t q_batch_stride,
  *   descending (ties: smaller entry first) until their mass reaches p; golden_i = entries kept by
  *   at least theta layers; label = union of golden_i over the window.  The pages use p = 0.6,
  *   theta = 3 and the 21 CSA layers.
- *   z            [tau][Lc][T] fp32 device, entry s of sequence b at column seq_offsets[b] + s
+ *   z            [tau][Lc][T] fp32 device, entry s of sequence b at column seq_offsets[b] + s;
+ *                1 <= Lc <= 255 and total_S < 2^31 (else LSA_ERR_INVALID_ARG)
  *   label_out    [T] uint8 device: 1 for a golden entry of the window, else 0
  *   nsize_out    [B][tau][Lc] int32 device (nullable): nucleus sizes
  * Softmax masses and their sums are taken in double.  Workspace:

@@ -29,8 +29,8 @@
 //                    the bits.
 //                    Bits go to a [tau][Lc][ceil(T/32)] bit plane by atomicOr (words can
 //                    straddle two sequences).
-// k_golden_vote      one warp per 32-entry word: votes over the Lc layers per token, theta test,
-//                    OR over the tokens, one label byte per entry.
+// k_golden_vote      32 words per CTA: bit-sliced vote counts over the Lc layers per token, theta
+//                    test, OR over the tokens, one label byte per entry.
 #pragma once
 #include "select_common.cuh"
 
@@ -155,19 +155,32 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     }
     const float *row = z + ((int64_t)i * Lc + l) * T + off;
     uint32_t *plane = bits + ((int64_t)i * Lc + l) * W32;
+    // the row in 16-byte vectors from its first 16-byte boundary; the at most three entries before
+    // it and the at most three after the last whole vector go to threads 0..5 one by one
+    const int head = (int)min((int64_t)((4 - (((uintptr_t)row >> 2) & 3)) & 3), S);
+    const int64_t nvec = (S - head) >> 2;
+    const int64_t tail0 = head + 4 * nvec;
+    const float4 *vrow = (const float4 *)(row + head);
+    const int64_t lone = threadIdx.x < head ? (int64_t)threadIdx.x
+                         : (threadIdx.x < head + (S - tail0) ? tail0 + (threadIdx.x - head) : (int64_t)-1);
     float m = -INFINITY;
     {
-        float m8[8];
+        float4 mv[4];
 #pragma unroll
-        for (int q = 0; q < 8; q++) m8[q] = -INFINITY;
-        for (int64_t base = 0; base < S; base += 8 * THREADS) {  // eight loads in flight
+        for (int q = 0; q < 4; q++) mv[q] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        for (int64_t base = 0; base < nvec; base += 4 * THREADS) {  // four vector loads in flight
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int64_t s = base + q * THREADS + threadIdx.x;
-                if (s < S) m8[q] = fmaxf(m8[q], __ldg(row + s));
+            for (int q = 0; q < 4; q++) {
+                const int64_t v = base + q * THREADS + threadIdx.x;
+                if (v < nvec) {
+                    const float4 x = __ldg(vrow + v);
+                    mv[q] = make_float4(fmaxf(mv[q].x, x.x), fmaxf(mv[q].y, x.y), fmaxf(mv[q].z, x.z), fmaxf(mv[q].w, x.w));
+                }
             }
         }
-        m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+#pragma unroll
+        for (int q = 0; q < 4; q++) m = fmaxf(m, fmaxf(fmaxf(mv[q].x, mv[q].y), fmaxf(mv[q].z, mv[q].w)));
+        if (lone >= 0) m = fmaxf(m, __ldg(row + lone));
     }
     m = block_max(m, fred);
 
@@ -175,30 +188,43 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     if (m > -INFINITY && m < INFINITY) {
         if (threadIdx.x == 0) s_nc = 0;
         __syncthreads();
-        // Z in fp32 exp and the bound of its error: expf is within 2 ulp (2^-22 relative); z - m is
-        // rounded once (an error of 2^-24 |x| in the exponent, |x| < 104 wherever the result is
-        // normal); each thread's fp32 sum of its S / THREADS terms rounds by at most that many
-        // ulps; a result below the smallest normal is off by at most 2^-126 absolute
+        // Z in fp32 and the bound of its error: e^x = 2^(x log2 e) with x = z - m rounded once, the
+        // product and log2 e rounded once each (an error of 3 * 2^-24 |x| in the exponent, |x| < 104
+        // wherever the result is normal); exp2f is within 2 ulp (2^-22 relative); each thread's
+        // fp32 sum of its at most S / THREADS + 5 terms rounds by at most that many ulps; a result
+        // below the smallest normal is off by at most 2^-126 absolute.  An entry within 4 of the
+        // maximum is appended to the candidates by its own thread (they are few).
+        constexpr float LOG2E = 1.4426950408889634f;
         float zf = 0.f;
-        for (int64_t base = 0; base < S; base += 4 * THREADS) {  // whole warps per step (warp-wide appends)
-            float zq[4];
+        auto take = [&](float x, int s) {  // (s: the entry, only formed for an appended one)
+            zf += exp2f((x - m) * LOG2E);
+            if (m - x < 4.f) {
+                const int at = atomicAdd(&s_nc, 1);
+                if (at < CAND) cand[at] = ((unsigned long long)float_to_ordered(x) << 32) | (uint32_t)(~(uint32_t)s);
+            }
+        };
+        const int nv = (int)nvec;  // (S < 2^31 entries)
+        for (int base = 0; base < nv; base += 4 * THREADS) {
+            float4 x[4];
 #pragma unroll
-            for (int u = 0; u < 4; u++) {  // four loads in flight
-                const int64_t s = base + u * THREADS + threadIdx.x;
-                zq[u] = s < S ? __ldg(row + s) : -INFINITY;
+            for (int q = 0; q < 4; q++) {  // four vector loads in flight
+                const int v = base + q * THREADS + (int)threadIdx.x;
+                x[q] = v < nv ? __ldg(vrow + v) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
             }
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int64_t s = base + u * THREADS + threadIdx.x;
-                zf += s < S ? expf(zq[u] - m) : 0.f;
-                warp_append(s < S && m - zq[u] < 4.f,
-                            ((unsigned long long)float_to_ordered(zq[u]) << 32) | (uint32_t)(~(uint32_t)s), &s_nc,
-                            cand);
+            for (int q = 0; q < 4; q++) {
+                const int s = head + 4 * (base + q * THREADS + (int)threadIdx.x);
+                take(x[q].x, s);
+                take(x[q].y, s + 1);
+                take(x[q].z, s + 2);
+                take(x[q].w, s + 3);
             }
         }
+        if (lone >= 0) take(__ldg(row + lone), (int)lone);
+        __syncthreads();
         const double Z32 = block_sum((double)zf, dred);
         // (plus the rounding of sums in double, here and in an fp64 Z: terms per thread + 64 ulps)
-        const double err = 1.01 * Z32 * (0x1p-22 + 104.0 * 0x1p-24 + ((double)S / THREADS + 1.0) * 0x1p-24) +
+        const double err = 1.01 * Z32 * (0x1p-22 + 3.0 * 104.0 * 0x1p-24 + ((double)S / THREADS + 5.0) * 0x1p-24) +
                            (double)S * 0x1p-126 + 2.0 * Z32 * ((double)S / THREADS + 64.0) * 0x1p-53;
         const int nc = s_nc;
         if (nc <= CAND) {
@@ -444,20 +470,66 @@ __global__ void __launch_bounds__(THREADS) k_golden_nucleus(const float *__restr
     }
 }
 
-__global__ void __launch_bounds__(THREADS) k_golden_vote(const uint32_t *__restrict__ bits, int64_t W32, int64_t T,
-                                                         int tau, int Lc, int theta, uint8_t *__restrict__ label)
+// One CTA per 32 consecutive 32-entry words: lane = word, warp = a group of tokens.  A thread adds
+// the Lc layer words of each of its tokens into a bit-sliced counter (slice k holds bit k of every
+// entry's vote count), compares the counts with theta slice by slice, and ORs the result over its
+// tokens; the warps' results are ORed in shared memory and written as one byte per entry.
+constexpr int VOTE_THREADS = 1024;
+constexpr int VOTE_SLICES = 8;  // vote counts up to 255 layers
+
+__global__ void __launch_bounds__(VOTE_THREADS, 2) k_golden_vote(const uint32_t *__restrict__ bits, int64_t W32, int64_t T,
+                                                              int tau, int Lc, int theta, uint8_t *__restrict__ label)
 {
-    const int64_t w = (int64_t)blockIdx.x * (THREADS / 32) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (w >= W32) return;
-    bool any = false;
-    for (int i = 0; i < tau; i++) {
-        int votes = 0;
-        for (int l = 0; l < Lc; l++) votes += (__ldg(bits + ((int64_t)i * Lc + l) * W32 + w) >> lane) & 1u;
-        any |= votes >= theta;
+    __shared__ uint32_t s_any[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t w = (int64_t)blockIdx.x * 32 + lane;
+    if (threadIdx.x < 32) s_any[threadIdx.x] = 0u;
+    __syncthreads();
+    int ns = 0;
+    while (ns < VOTE_SLICES && (Lc >> ns) != 0) ns++;  // slices holding counts up to Lc
+    uint32_t any = 0u;
+    if (w < W32 && theta <= Lc) {
+        for (int i = warp; i < tau; i += VOTE_THREADS / 32) {
+            const uint32_t *col = bits + (int64_t)i * Lc * W32 + w;
+            uint32_t c[VOTE_SLICES];
+#pragma unroll
+            for (int k = 0; k < VOTE_SLICES; k++) c[k] = 0u;
+            for (int l0 = 0; l0 < Lc; l0 += 4) {
+                uint32_t x[4];
+#pragma unroll
+                for (int u = 0; u < 4; u++) x[u] = l0 + u < Lc ? __ldg(col + (int64_t)(l0 + u) * W32) : 0u;
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    uint32_t carry = x[u];
+#pragma unroll
+                    for (int k = 0; k < VOTE_SLICES; k++) {
+                        const uint32_t t = c[k] & carry;
+                        c[k] ^= carry;
+                        carry = t;
+                    }
+                }
+            }
+            // count >= theta, from the most significant slice down
+            uint32_t gt = 0u, eq = 0xffffffffu;
+#pragma unroll
+            for (int k = VOTE_SLICES - 1; k >= 0; k--) {
+                if (k >= ns) continue;
+                if ((theta >> k) & 1) {
+                    eq &= c[k];
+                } else {
+                    gt |= eq & c[k];
+                    eq &= ~c[k];
+                }
+            }
+            any |= gt | eq;
+        }
     }
-    const int64_t g = w * 32 + lane;
-    if (g < T) label[g] = any ? 1 : 0;
+    if (any) atomicOr(&s_any[lane], any);
+    __syncthreads();
+    for (int t = threadIdx.x; t < 32 * 32; t += VOTE_THREADS) {
+        const int64_t g = (int64_t)blockIdx.x * 1024 + t;
+        if (g < T) label[g] = (uint8_t)((s_any[t >> 5] >> (t & 31)) & 1u);
+    }
 }
 
 }  // namespace golden

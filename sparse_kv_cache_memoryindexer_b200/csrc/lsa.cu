@@ -200,14 +200,11 @@ lsa_status li_simt_d(int kdt, const void *qd, const float *wd, const void *hotK,
 }
 
 // The E4M3 score runs on CTA pairs unless LSA_SCORE_PAIR=0 (the one-CTA kernel, k_score_tc, the
-// same result).
+// same result; read at every call, so the two kernels can be cross-checked in one process).
 bool score_pair_enabled()
 {
-    static const bool on = [] {
-        const char *v = getenv("LSA_SCORE_PAIR");
-        return !(v && v[0] == '0');
-    }();
-    return on;
+    const char *v = getenv("LSA_SCORE_PAIR");
+    return !(v && v[0] == '0');
 }
 
 bool valid_dtype(int dt) { return dt == DT_F32 || dt == DT_BF16 || dt == DT_FP8; }
@@ -254,12 +251,14 @@ lsa_status lsa_selftest_wait_timeout(int32_t *status_out, lsa_stream_t stream)
 // tensor-core path adds the partial sums of its K ranges there before rounding c once).
 size_t lsa_project_workspace_size(int L, int B, int d, int r, int n_h, int d_I, lsa_dtype dt)
 {
-    (void)d; (void)d_I;
-    if (L <= 0 || B <= 0 || r <= 0 || n_h <= 0) return 0;
-    // c in its storage type, then the fp32 partial slices of c and w (K split in at most KSPLIT_MAX)
-    return align_up((size_t)L * B * r * elem_bytes(dt), 256) +
-           align_up((size_t)proj::KSPLIT_MAX * L * B * r * 4, 256) +
-           align_up((size_t)proj::KSPLIT_MAX * L * B * n_h * 4, 256);
+    (void)d;
+    if (L <= 0 || B <= 0 || r <= 0 || n_h <= 0 || d_I <= 0) return 0;
+    // c in its storage type, then the fp32 partial slices of c and w (K split in at most KSPLIT_MAX),
+    // which the partial slices of q reuse once c and w are summed
+    const size_t cw = align_up((size_t)proj::KSPLIT_MAX * L * B * r * 4, 256) +
+                      align_up((size_t)proj::KSPLIT_MAX * L * B * n_h * 4, 256);
+    const size_t qs = align_up((size_t)proj::KSPLIT_MAX * L * B * n_h * d_I * 4, 256);
+    return align_up((size_t)L * B * r * elem_bytes(dt), 256) + (cw > qs ? cw : qs);
 }
 
 lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const void *W_w, lsa_dtype dt,
@@ -281,10 +280,12 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
     void *c = workspace;
     if (proj_tc_supported(dt, B, d) && proj_tc_supported(dt, B, r)) {
         // c and w in one launch, split along d so that every SM streams weights (fp32 partial sums
-        // in slices of their own); the slices summed in order, c rounded to bf16 once; then q, all
-        // of r per tile
+        // in slices of their own); the slices summed in order, c rounded to bf16 once; then q,
+        // split along r the same way when that balances the SMs better.  Every launch after the
+        // first is a programmatic dependent of the one before (the q launch streams its first
+        // weight stages while c is summed).
         const int sms = num_sms();
-        const int64_t nc = (int64_t)L * B * r, nw = (int64_t)L * B * n_h;
+        const int64_t nc = (int64_t)L * B * r, nw = (int64_t)L * B * n_h, nqt = (int64_t)L * B * nq;
         float *pc = (float *)((char *)workspace + align_up((size_t)nc * elem_bytes(dt), 256));
         float *pw = (float *)((char *)pc + align_up((size_t)proj::KSPLIT_MAX * nc * 4, 256));
         const ProjProblem cw[2] = {{W_dq, pc, r, true}, {W_w, pw, n_h, true}};
@@ -292,15 +293,19 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
         int ks[2] = {1, 1};
         lsa_status s = launch_proj_tc(h, cw, split, 2, L, B, d, sms, st, ks);
         if (s == LSA_OK) s = launched("project c and w (tensor cores)");
-        if (s == LSA_OK) {
-            k_proj_reduce<<<(unsigned)std::min<int64_t>((nc + nw + 255) / 256, (int64_t)sms * 8), 256, 0, st>>>(
-                pc, ks[0], nc, (__nv_bfloat16 *)c, pw, ks[1], nw, w_out);
-            s = launched("project: reduce c and w");
-        }
-        const ProjProblem qp = {W_iuq, q_out, nq, false};
-        const bool nosplit = false;
-        if (s == LSA_OK) s = launch_proj_tc(c, &qp, &nosplit, 1, L, B, r, sms, st);
+        if (s == LSA_OK && launch_proj_reduce(pc, ks[0], nc, (__nv_bfloat16 *)c, pw, ks[1], nw, w_out, sms, st) !=
+                               cudaSuccess)
+            s = LSA_ERR_CUDA;
+        if (s == LSA_OK) s = launched("project: reduce c and w");
+        const bool qsplit = proj_ksplit((int64_t)L * ((nq + 127) / 128), proj_stages_of_k(B, r), sms) > 1;
+        const ProjProblem qp = {W_iuq, qsplit ? (void *)pc : q_out, nq, false};  // (pc: summed already)
+        int kq = 1;
+        if (s == LSA_OK) s = launch_proj_tc(c, &qp, &qsplit, 1, L, B, r, sms, st, &kq, true);
         if (s == LSA_OK) s = launched("project q (tensor cores)");
+        if (s == LSA_OK && qsplit &&
+            launch_proj_reduce(pc, kq, nqt, (__nv_bfloat16 *)q_out, nullptr, 0, 0, nullptr, sms, st) != cudaSuccess)
+            s = LSA_ERR_CUDA;
+        if (s == LSA_OK && qsplit) s = launched("project: reduce q");
         if (s != LSA_OK) return fail(s, "lsa_project: tensor-core launch failed (%s)", cudaGetErrorString(cudaGetLastError()));
     } else if (dt == LSA_BF16) {
         k_rowdot<DT_BF16, DT_BF16><<<dim3((r + 7) / 8, L), 256, 0, st>>>(h, W_dq, c, B, d, r);
@@ -820,6 +825,8 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
     LSA_REQUIRE(B > 0 && tau > 0 && Lc > 0 && total_S >= 0, "lsa_golden_labels: sizes must be positive");
     LSA_REQUIRE(p > 0.0 && p <= 1.0, "lsa_golden_labels: p must be in (0, 1]");
     LSA_REQUIRE(theta >= 1, "lsa_golden_labels: theta must be at least 1");
+    LSA_REQUIRE(Lc <= 255, "lsa_golden_labels: at most 255 layers");
+    LSA_REQUIRE(total_S < ((int64_t)1 << 31), "lsa_golden_labels: total_S must be below 2^31");
     LSA_REQUIRE((int64_t)B * tau * Lc < ((int64_t)1 << 31), "lsa_golden_labels: too many rows");
     const size_t need = lsa_golden_labels_workspace_size(tau, Lc, total_S);
     if (!workspace || workspace_bytes < need)
@@ -833,8 +840,8 @@ lsa_status lsa_golden_labels(const float *z, const int64_t *seq_offsets, int64_t
     golden::k_golden_nucleus<<<(unsigned)((int64_t)B * tau * Lc), golden::THREADS, 0, st>>>(
         z, seq_offsets, total_S, B, tau, Lc, p, bits, W32, nsize_out);
     LSA_TRY(launched("golden labels: nucleus"));
-    golden::k_golden_vote<<<(unsigned)((W32 + golden::THREADS / 32 - 1) / (golden::THREADS / 32)), golden::THREADS, 0,
-                            st>>>(bits, W32, total_S, tau, Lc, theta, label_out);
+    golden::k_golden_vote<<<(unsigned)((W32 + 31) / 32), golden::VOTE_THREADS, 0, st>>>(bits, W32, total_S, tau, Lc,
+                                                                                      theta, label_out);
     LSA_TRY(launched("golden labels: vote"));
     return ok();
 }

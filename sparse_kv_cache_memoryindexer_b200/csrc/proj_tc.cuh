@@ -15,6 +15,13 @@
 // epilogue rounds to the output type (bf16 nearest-even, or fp32) and stores.  Either way every
 // output is an fp32 sum of its K products, rounded once, and the same on every run.
 //
+// Launches of one projection follow each other as programmatic dependents: every kernel here lets
+// its dependents start at once, and a dependent waits for its predecessor (griddepcontrol.wait)
+// before it touches what the predecessor writes.  The tensor-core kernel issues the weight boxes
+// of its first stages before that wait (the weights are inputs of the call, not results of the
+// previous launch), so its weight stream starts while the previous launch drains; the X boxes
+// follow the wait.
+//
 // Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue (one TMEM lane
 // quarter each).  Two accumulators, so a unit's epilogue overlaps the next unit's MMAs.  Every
 // ring is consumed in order by one consumer (group); waits are bounded as in the other
@@ -82,6 +89,11 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int u, int nkb)
     return x;
 }
 
+// programmatic dependent launch: let the next launch start / wait for the previous one (both are
+// no-ops for a launch without the programmatic-serialization attribute)
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __host__ __device__ inline uint32_t b_bytes(int NB) { return (uint32_t)NB * KB * 2; }
 // a stage: nbox weight boxes (128 rows x 64 K each), then nbox X boxes (NB rows x 64 K each)
 __host__ __device__ inline uint32_t stage_bytes(int NB, int nbox) { return (uint32_t)nbox * (A_BYTES + b_bytes(NB)); }
@@ -120,6 +132,7 @@ __global__ void __launch_bounds__(THREADS)
     const int nunits = p.pr[0].units + (p.nprob > 1 ? p.pr[1].units : 0);
     const int nkb = (p.K + KB - 1) / KB;
     const uint32_t ncols = tmem_cols(p.NB), acol = acc_cols(p.NB);
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; i++) {
@@ -156,21 +169,42 @@ __global__ void __launch_bounds__(THREADS)
         uint32_t last_phase[MAX_STAGES];
         bool issued[MAX_STAGES];
         for (int i = 0; i < MAX_STAGES; i++) issued[i] = false;
+        // stages whose weight boxes went out before the wait for the previous launch: their X boxes
+        // (K block, count, X row) follow the wait
+        int pend_kb[MAX_STAGES], pend_nb[MAX_STAGES], pend_row[MAX_STAGES];
+        int pending = 0;
+        bool waited = false;
+        auto x_boxes = [&](int st_i, int kb, int nb, int xrow) {
+            const uint32_t dst = sbase + (uint32_t)st_i * sbytes + (uint32_t)p.nbox * A_BYTES;
+            for (int i = 0; i < nb; i++) tma_load_2d(dst + (uint32_t)i * bbox, &xmap, (kb + i) * KB, xrow, full(st_i));
+        };
+        auto release = [&]() {  // wait for the previous launch, then the X boxes of the pending stages
+            pdl_wait();
+            if (leader)
+                for (int j = 0; j < pending; j++) x_boxes(j, pend_kb[j], pend_nb[j], pend_row[j]);
+            __syncwarp();
+            waited = true;
+        };
         bool ok = true;
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const Unit x = unit_of(p, u, nkb);
             const CUtensorMap *wm = x.prob == 0 ? &wmap0 : &wmap1;
             for (int kb = x.kb0; kb < x.kb1; kb += p.nbox) {
                 const int nb = min(p.nbox, x.kb1 - kb);
+                if (!waited && pending == p.stages) release();  // every stage holds weights: nothing more before X
                 if (!mbar_wait_warp(empty(stage), phase ^ 1, abort_flag)) { ok = false; break; }
                 if (leader) {
                     mbar_expect_tx(full(stage), (uint32_t)nb * (A_BYTES + bbox));
                     const uint32_t dst = sbase + (uint32_t)stage * sbytes;
-                    for (int i = 0; i < nb; i++) {  // the boxes of a stage back to back: row segments of 256 bytes
+                    for (int i = 0; i < nb; i++)  // the boxes of a stage back to back: row segments of 256 bytes
                         tma_load_2d(dst + (uint32_t)i * A_BYTES, wm, (kb + i) * KB, x.l * x.R + x.m0, full(stage));
-                        tma_load_2d(dst + (uint32_t)p.nbox * A_BYTES + (uint32_t)i * bbox, &xmap, (kb + i) * KB,
-                                    x.l * p.B, full(stage));
-                    }
+                    if (waited) x_boxes(stage, kb, nb, x.l * p.B);
+                }
+                if (!waited) {  // (the first stages, in order: stage == pending)
+                    pend_kb[pending] = kb;
+                    pend_nb[pending] = nb;
+                    pend_row[pending] = x.l * p.B;
+                    pending++;
                 }
                 __syncwarp();
                 issued[stage] = true;
@@ -178,6 +212,7 @@ __global__ void __launch_bounds__(THREADS)
                 if (++stage == p.stages) { stage = 0; phase ^= 1; }
             }
         }
+        if (!waited) release();  // (also on an abort: every issued stage gets its X bytes)
         if (*abort_flag && leader) {
             volatile int never = 0;
             for (int i = 0; i < p.stages; i++)
@@ -273,13 +308,62 @@ struct ProjProblem {
     bool out_f32;
 };
 
+// Boxes per stage and stages of a launch with batch B (the shared memory decides).
+struct ProjShape {
+    int NB, nbox, stages;
+    uint32_t smem;
+};
+inline ProjShape proj_shape(int B)
+{
+    using namespace proj;
+    ProjShape s;
+    s.NB = (B + 15) / 16 * 16;
+    const uint32_t max_smem = 227 * 1024 - 1024;
+    s.nbox = MAX_BOX;
+    while (s.nbox > 1 && smem_total(s.NB, 2, s.nbox) > max_smem) s.nbox >>= 1;
+    s.stages = MAX_STAGES;
+    while (s.stages > 2 && smem_total(s.NB, s.stages, s.nbox) > max_smem) s.stages--;
+    s.smem = smem_total(s.NB, s.stages, s.nbox);
+    if (s.smem > max_smem) s.smem = 0;  // unsupported
+    return s;
+}
+
+// K ranges for `tiles` 128-row tiles over K of `nst` stages: the count (at most KSPLIT_MAX, whole
+// stages each) whose units fill `sms` CTAs best (1: no split).
+inline int proj_ksplit(int64_t tiles, int nst, int sms)
+{
+    int ks = 1;
+    double best = -1.0;
+    for (int c = 1; c <= proj::KSPLIT_MAX && c <= nst; c++) {
+        const int spc = (nst + c - 1) / c;  // stages per range
+        const int ranges = (nst + spc - 1) / spc;
+        if (ranges != c) continue;
+        const int64_t units = tiles * c;
+        const int64_t waves = (units + sms - 1) / sms;
+        const double eff = (double)units / (double)(waves * sms);
+        if (eff > best + 1e-9) {
+            best = eff;
+            ks = c;
+        }
+    }
+    return ks;
+}
+
+// Stages of all of K for a launch of batch B.
+inline int proj_stages_of_k(int B, int K)
+{
+    const ProjShape sh = proj_shape(B);
+    const int nkb = (K + proj::KB - 1) / proj::KB;
+    return (nkb + sh.nbox - 1) / sh.nbox;
+}
+
 // One launch over one or two problems sharing X bf16 [L][B][K]; a split problem's units store
 // partial slices, and ksplit_out[i] (nullable) reports how many.  One CTA per SM; a stage holds up
 // to MAX_BOX boxes of K so that every weight row is read in segments of 256 bytes.  Split problems
-// take the number of K ranges (at most KSPLIT_MAX, in whole stages) that balances the units best
-// over the CTAs.
+// take the number of K ranges (proj_ksplit) that balances the units best over the CTAs.  pdl: the
+// launch is a programmatic dependent of the previous one on the stream.
 inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const bool *split, int nprob, int L, int B,
-                                 int K, int sms, cudaStream_t st, int *ksplit_out = nullptr)
+                                 int K, int sms, cudaStream_t st, int *ksplit_out = nullptr, bool pdl = false)
 {
     using namespace proj;
     CUtensorMap wmap[2], xmap;
@@ -288,37 +372,19 @@ inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const boo
     p.L = L;
     p.B = B;
     p.K = K;
-    p.NB = (B + 15) / 16 * 16;
-    const uint32_t max_smem = 227 * 1024 - 1024;
-    p.nbox = MAX_BOX;
-    while (p.nbox > 1 && smem_total(p.NB, 2, p.nbox) > max_smem) p.nbox >>= 1;
-    p.stages = MAX_STAGES;
-    while (p.stages > 2 && smem_total(p.NB, p.stages, p.nbox) > max_smem) p.stages--;
-    const uint32_t smem = smem_total(p.NB, p.stages, p.nbox);
-    if (smem > max_smem) return LSA_ERR_UNSUPPORTED;
+    const ProjShape sh = proj_shape(B);
+    if (sh.smem == 0) return LSA_ERR_UNSUPPORTED;
+    p.NB = sh.NB;
+    p.nbox = sh.nbox;
+    p.stages = sh.stages;
+    const uint32_t smem = sh.smem;
     const int nkb = (K + KB - 1) / KB;
     const int nst = (nkb + p.nbox - 1) / p.nbox;  // stages of all of K
     int tiles = 0;
     for (int i = 0; i < nprob; i++) tiles += L * ((pb[i].R + 127) / 128);
-    // K ranges of the split problems: the count (whole stages each) whose units fill the CTAs best
-    int ks = 1;
     bool any_split = false;
     for (int i = 0; i < nprob; i++) any_split = any_split || split[i];
-    if (any_split) {
-        double best = -1.0;
-        for (int c = 1; c <= KSPLIT_MAX && c <= nst; c++) {
-            const int spc = (nst + c - 1) / c;          // stages per range
-            const int ranges = (nst + spc - 1) / spc;
-            if (ranges != c) continue;
-            const int64_t units = (int64_t)tiles * c;
-            const int64_t waves = (units + sms - 1) / sms;
-            const double eff = (double)units / (double)(waves * sms);
-            if (eff > best + 1e-9) {
-                best = eff;
-                ks = c;
-            }
-        }
-    }
+    const int ks = any_split ? proj_ksplit(tiles, nst, sms) : 1;
     bool ok = make_map_2d(&xmap, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L * B, (uint64_t)K, KB, (uint32_t)p.NB);
     int total = 0;
     for (int i = 0; i < 2; i++) {
@@ -342,8 +408,20 @@ inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const boo
     cudaError_t e = cudaFuncSetAttribute(k_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return LSA_ERR_CUDA;
     const int grid = total < sms ? total : sms;
-    k_proj_tc<<<grid, THREADS, smem, st>>>(wmap[0], wmap[1], xmap, p);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    e = cudaLaunchKernelEx(&cfg, k_proj_tc, wmap[0], wmap[1], xmap, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }
 
@@ -353,6 +431,8 @@ __global__ void __launch_bounds__(256) k_proj_reduce(const float *__restrict__ p
                                                      __nv_bfloat16 *__restrict__ c, const float *__restrict__ pw,
                                                      int k1, int64_t n1, float *__restrict__ w)
 {
+    proj::pdl_trigger();
+    proj::pdl_wait();  // the partial slices of the previous launch
     for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n0 + n1; i += (int64_t)gridDim.x * 256) {
         if (i < n0) {
             float s = 0.f;
@@ -365,6 +445,25 @@ __global__ void __launch_bounds__(256) k_proj_reduce(const float *__restrict__ p
             w[j] = s;
         }
     }
+}
+
+// k_proj_reduce as a programmatic dependent of the previous launch on the stream.
+inline cudaError_t launch_proj_reduce(const float *pc, int k0, int64_t n0, __nv_bfloat16 *c, const float *pw, int k1,
+                                      int64_t n1, float *w, int sms, cudaStream_t st)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    // few enough CTAs to sit beside the previous launch's CTAs while they wait for it
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>((n0 + n1 + 255) / 256, (int64_t)sms * 4));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_proj_reduce, pc, k0, n0, c, pw, k1, n1, w);
+    return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 }  // namespace lsa

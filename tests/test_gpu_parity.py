@@ -82,6 +82,14 @@ def kernel_path(request, monkeypatch):
     return request.param
 
 
+@pytest.fixture(params=["pair", "one_cta"])
+def e4m3_path(request, monkeypatch):
+    """E4M3 keys: 'pair' takes the CTA-pair score kernel (the default), 'one_cta' the one-CTA one."""
+    if request.param == "one_cta":
+        monkeypatch.setenv("LSA_SCORE_PAIR", "0")
+    return request.param
+
+
 @pytest.mark.parametrize("name", list(CASES))
 def test_select_parity(m, name, kernel_path):
     wl, inp = inputs(name)
@@ -91,6 +99,22 @@ def test_select_parity(m, name, kernel_path):
     n_ex, n_flip = check_select(mask, idx, cnt, I, ref, offs, what=name)
     assert n_flip <= max(3, n_ex // 10)
     assert cnt.sum() == ref["count"].sum() or n_flip > 0
+
+
+def test_select_parity_e4m3_one_cta(m, monkeypatch):
+    """The one-CTA E4M3 score kernel (taken for more than 1,024 sequences) against the oracle, and
+    bit for bit against the CTA-pair kernel."""
+    wl, inp = inputs("ctx1m_fp8_seq0")
+    monkeypatch.setenv("LSA_SCORE_PAIR", "0")
+    offs = inp.seq_offsets.numpy()
+    ref = oracle.score(inp.q, inp.w, inp.K, inp.k_scale, offs)
+    mask, idx, cnt, I = run_select(m, inp)
+    n_ex, n_flip = check_select(mask, idx, cnt, I, ref, offs, what="ctx1m_fp8_seq0 one-CTA")
+    assert n_flip <= max(3, n_ex // 10)
+    monkeypatch.delenv("LSA_SCORE_PAIR")
+    mask2, idx2, cnt2, I2 = run_select(m, inp)
+    assert np.array_equal(mask, mask2) and np.array_equal(cnt, cnt2) and np.array_equal(idx, idx2)
+    assert np.array_equal(I, I2)
 
 
 @pytest.mark.parametrize("thr", [0.3, 0.9])
@@ -375,7 +399,7 @@ def _fp8_case(codes_fn, seed):
     return wl, inp
 
 
-def test_select_e4m3_subnormal_codes(m):
+def test_select_e4m3_subnormal_codes(m, e4m3_path):
     """Only subnormal E4M3 codes (exponent field 0) with scale 2^9, so every key value is a small
     integer: a flush of subnormals anywhere on the device path would zero every logit."""
     def codes(rng, shape):
@@ -391,7 +415,7 @@ def test_select_e4m3_subnormal_codes(m):
     check_select(mask, idx, cnt, I, ref, offs, what="subnormal codes")
 
 
-def test_select_e4m3_all_codes(m):
+def test_select_e4m3_all_codes(m, e4m3_path):
     """Every finite E4M3 code (0x7F and 0xFF are NaN and excluded), uniformly, with random scales."""
     def codes(rng, shape):
         c = rng.integers(0, 254, size=shape).astype(np.uint8)          # 0..253
