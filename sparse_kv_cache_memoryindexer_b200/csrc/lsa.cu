@@ -614,19 +614,10 @@ lsa_status lsa_lightning_topk(const void *q_dec, const float *w_dec, const void 
     }
     int kpow2 = 64;  // the block sort works on at least 64 keys
     while (kpow2 < k) kpow2 <<= 1;
-    // the queries' score keys stay in shared memory up to the capacity left beside the static part
-    int fcap = 0;
-    {
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, k_topk_select) != cudaSuccess)
-            return fail(LSA_ERR_CUDA, "lsa_lightning_topk: %s", cudaGetErrorString(cudaGetLastError()));
-        const int64_t room = (int64_t)227 * 1024 - (int64_t)fa.sharedSizeBytes - (int64_t)topk_select_smem(kpow2, 0) - 1024;
-        fcap = room > 0 ? (int)(room / 4) : 0;
-    }
-    const size_t smem = topk_select_smem(kpow2, fcap);
+    const size_t smem = topk_select_smem(kpow2);
     LSA_TRY(set_smem(k_topk_select, smem));
     k_topk_select<<<(unsigned)((int64_t)B * tau), SEL_THREADS, smem, st>>>(Y, idx, count, seq_offsets, tau, k, kpow2,
-                                                                  fcap, topk_idx, topk_score);
+                                                                  topk_idx, topk_score);
     LSA_TRY(launched("top-k select"));
     return ok();
 }

@@ -27,6 +27,7 @@
 // ring is consumed in order by one consumer (group); waits are bounded as in the other
 // tensor-core kernels.
 #pragma once
+#include "pdl.cuh"
 #include "tc_common.cuh"
 
 namespace lsa {
@@ -88,11 +89,6 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int u, int nkb)
     x.partial = one ? p.pr[1].partial : p.pr[0].partial;
     return x;
 }
-
-// programmatic dependent launch: let the next launch start / wait for the previous one (both are
-// no-ops for a launch without the programmatic-serialization attribute)
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __host__ __device__ inline uint32_t b_bytes(int NB) { return (uint32_t)NB * KB * 2; }
 // a stage: nbox weight boxes (128 rows x 64 K each), then nbox X boxes (NB rows x 64 K each)
@@ -408,18 +404,9 @@ inline lsa_status launch_proj_tc(const void *X, const ProjProblem *pb, const boo
     cudaError_t e = cudaFuncSetAttribute(k_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return LSA_ERR_CUDA;
     const int grid = total < sms ? total : sms;
-    cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    if (pdl) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
+    cudaLaunchConfig_t cfg = pdl_config(dim3((unsigned)grid), dim3(THREADS), smem, st, attr);
+    if (!pdl) cfg.numAttrs = 0;
     e = cudaLaunchKernelEx(&cfg, k_proj_tc, wmap[0], wmap[1], xmap, p);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
@@ -431,19 +418,22 @@ __global__ void __launch_bounds__(256) k_proj_reduce(const float *__restrict__ p
                                                      __nv_bfloat16 *__restrict__ c, const float *__restrict__ pw,
                                                      int k1, int64_t n1, float *__restrict__ w)
 {
-    proj::pdl_trigger();
-    proj::pdl_wait();  // the partial slices of the previous launch
+    pdl_trigger();
+    pdl_wait();  // the partial slices of the previous launch
+    // every slice's value loaded before the sum (the loads in flight together), summed in slice order
+    auto sum = [](const float *src, int ks, int64_t n, int64_t at) {
+        float v[proj::KSPLIT_MAX];
+#pragma unroll
+        for (int k = 0; k < proj::KSPLIT_MAX; k++) v[k] = k < ks ? __ldg(src + (int64_t)k * n + at) : 0.f;
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < proj::KSPLIT_MAX; k++)
+            if (k < ks) s += v[k];
+        return s;
+    };
     for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n0 + n1; i += (int64_t)gridDim.x * 256) {
-        if (i < n0) {
-            float s = 0.f;
-            for (int k = 0; k < k0; k++) s += __ldg(pc + (int64_t)k * n0 + i);
-            c[i] = __float2bfloat16_rn(s);
-        } else {
-            const int64_t j = i - n0;
-            float s = 0.f;
-            for (int k = 0; k < k1; k++) s += __ldg(pw + (int64_t)k * n1 + j);
-            w[j] = s;
-        }
+        if (i < n0) c[i] = __float2bfloat16_rn(sum(pc, k0, n0, i));
+        else w[i - n0] = sum(pw, k1, n1, i - n0);
     }
 }
 
@@ -451,17 +441,10 @@ __global__ void __launch_bounds__(256) k_proj_reduce(const float *__restrict__ p
 inline cudaError_t launch_proj_reduce(const float *pc, int k0, int64_t n0, __nv_bfloat16 *c, const float *pw, int k1,
                                       int64_t n1, float *w, int sms, cudaStream_t st)
 {
-    cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     // few enough CTAs to sit beside the previous launch's CTAs while they wait for it
-    cfg.gridDim = dim3((unsigned)std::min<int64_t>((n0 + n1 + 255) / 256, (int64_t)sms * 4));
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cudaLaunchConfig_t cfg =
+        pdl_config(dim3((unsigned)std::min<int64_t>((n0 + n1 + 255) / 256, (int64_t)sms * 4)), dim3(256), 0, st, attr);
     cudaError_t e = cudaLaunchKernelEx(&cfg, k_proj_reduce, pc, k0, n0, c, pw, k1, n1, w);
     return e == cudaSuccess ? cudaGetLastError() : e;
 }

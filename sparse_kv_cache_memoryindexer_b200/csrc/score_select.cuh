@@ -201,7 +201,9 @@ __global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__res
     }
     const int pos = base + before + inc - cnt;  // list position of this tile's first entry
     if (ct1 == t1 && threadIdx.x == 0) count_out[b] = base + total;
-    // coalesced writes: the warp walks its 32 tiles
+    // coalesced writes: the warp walks its 32 tiles; the mask goes out as 4 bytes per lane when the
+    // sequence's bytes start on a 4-byte boundary
+    const bool mask_words = mask_out && (((uintptr_t)(mask_out + off)) & 3u) == 0;
     for (int j = 0; j < 32; j++) {
         const int tj = ct0 + warp * 32 + j;
         if (tj >= ct1) break;
@@ -216,7 +218,22 @@ __global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__res
             const uint32_t wk = words[k];
             if ((wk >> lane) & 1u) idx_out[off + p + __popc(wk & below)] = (int32_t)(s0 + 32 * k + lane);
             p += __popc(wk);
-            if (mask_out && s0 + 32 * k + lane < S) mask_out[off + s0 + 32 * k + lane] = (uint8_t)((wk >> lane) & 1u);
+            if (mask_out && !mask_words && s0 + 32 * k + lane < S)
+                mask_out[off + s0 + 32 * k + lane] = (uint8_t)((wk >> lane) & 1u);
+        }
+        if (mask_words) {
+            // lane: entries 4 lane .. 4 lane + 3 of the tile (bits 4 (lane % 8) .. of word lane / 8)
+            const uint32_t wl = lane < 8 ? w0 : (lane < 16 ? w1 : (lane < 24 ? w2 : w3));
+            const uint32_t nib = (wl >> (4 * (lane & 7))) & 0xFu;
+            const uint32_t bytes = (nib & 1u) | ((nib & 2u) << 7) | ((nib & 4u) << 14) | ((nib & 8u) << 21);
+            const int64_t e = s0 + 4 * lane;
+            if (e + 3 < S) {
+                *(uint32_t *)(mask_out + off + e) = bytes;
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; q++)
+                    if (e + q < S) mask_out[off + e + q] = (uint8_t)((bytes >> (8 * q)) & 1u);
+            }
         }
     }
 }

@@ -31,6 +31,24 @@ __device__ __forceinline__ uint32_t sel_bucket(const SelRange &r, uint32_t u)
     const float t = (y - r.ymin) * r.scale;
     return t >= (float)(SEL_NB - 1) ? (uint32_t)(SEL_NB - 1) : (t > 0.f ? (uint32_t)t : 0u);
 }
+// The same bucket from the score itself: sel_bucket(r, float_to_ordered(y)) (a NaN's key sorts to
+// the top when its sign bit is clear, to the bottom otherwise).
+__device__ __forceinline__ uint32_t sel_bucket_f(const SelRange &r, float y)
+{
+    if (y != y) return signbit(y) ? 0u : (uint32_t)(SEL_NB - 1);
+    const float t = (y - r.ymin) * r.scale;
+    return t >= (float)(SEL_NB - 1) ? (uint32_t)(SEL_NB - 1) : (t > 0.f ? (uint32_t)t : 0u);
+}
+// The range from the smallest and largest scores that are not NaN (none: every score in bucket 0
+// or at its NaN end).
+__device__ __forceinline__ SelRange sel_range_f(float ymin, float ymax)
+{
+    SelRange r;
+    r.ymin = ymin;
+    const float span = ymax - ymin;
+    r.scale = span > 0.f ? (float)SEL_NB / span : 0.f;
+    return r;
+}
 
 // Descending bitonic sort of n 64-bit keys in shared memory by the whole block (n a power of two,
 // at least 64; blockDim.x a multiple of 32).  Strides of 64 and more exchange through shared memory

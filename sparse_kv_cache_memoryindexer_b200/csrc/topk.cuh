@@ -119,102 +119,128 @@ __device__ __forceinline__ int sel_find_bin(const unsigned int *hist, int want, 
     return above0;
 }
 
-// Shared memory of k_topk_select for kpow2 and a key capacity fcap (dynamic part).
-__host__ __device__ inline size_t topk_select_smem(int kpow2, int fcap)
+// Shared memory of k_topk_select for kpow2 (dynamic part): the selection and the stage.
+__host__ __device__ inline size_t topk_select_smem(int kpow2)
 {
-    return sizeof(unsigned long long) * ((size_t)kpow2 + SEL_CAP) + sizeof(uint32_t) * (size_t)fcap;
+    return sizeof(unsigned long long) * ((size_t)kpow2 + SEL_CAP);
 }
 
+// A query's scores in 16-byte vectors from their first 16-byte boundary; the at most three scores
+// before it and the at most three after the last whole vector belong to threads 0..5 (lone()).
+struct ScoreRow {
+    const float *row;
+    const float4 *vec;
+    int F, head, nvec, tail0;
+    __device__ ScoreRow(const float *r, int f) : row(r), F(f)
+    {
+        head = min((int)((4 - (((uintptr_t)r >> 2) & 3)) & 3), f);
+        nvec = (f - head) >> 2;
+        tail0 = head + 4 * nvec;
+        vec = (const float4 *)(r + head);
+    }
+    __device__ int lone() const
+    {
+        const int t = (int)threadIdx.x;
+        return t < head ? t : (t < head + (F - tail0) ? tail0 + (t - head) : -1);
+    }
+};
+
 // One block per (sequence, query).  kpow2 = next power of two >= max(k, 64).  Dynamic shared memory:
-// kpow2 selection keys, SEL_CAP staged keys, then the query's score keys when it has at most fcap
-// candidates (read from the scores once, eight independent loads in flight per thread; a larger
-// query reads its scores from global memory at every pass).  With more than k candidates: the range
-// of the query's keys, then a histogram over 4096 buckets of that range gives the bucket beta of
-// the k-th largest key.  Each bucket above beta gets a segment of the selection (higher buckets
-// first) and its keys are scattered into it; the bucket's keys go to the stage (any order: the keys
-// carry their slots), and the stage sorted by key gives the bucket's largest keys.  When no bucket
-// above beta holds more than SEL_RANK_SEG keys, a key's output position is its segment's start plus
-// the keys of its segment above it (no sort of the selection); otherwise the k keys are sorted.  A
-// bucket beta of more than SEL_CAP keys is resolved by four radix passes over its keys and
-// an ordered pass (the first keys equal to the k-th in slot order).  The output is
-// ordered by (score desc, slot asc).
-__global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__restrict__ Y,
-                                                             const int32_t *__restrict__ idx,
-                                                             const int32_t *__restrict__ count,
-                                                             const int64_t *__restrict__ offs, int tau, int k,
-                                                             int kpow2, int fcap, int32_t *__restrict__ topk_idx,
-                                                             float *__restrict__ topk_score)
+// kpow2 selection keys and SEL_CAP staged keys; the query's scores are read from global memory at
+// every pass (as 16-byte vectors, four in flight per thread; after the first pass they come from
+// L2), so two blocks fit on an SM.  With more than k candidates: the range of the query's scores,
+// then a histogram over 4096 buckets of that range gives the bucket beta of the k-th largest key.
+// Each bucket above beta gets a segment of the selection (higher buckets first) and its keys are
+// scattered into it; the bucket's keys go to the stage (any order: the keys carry their slots), and
+// the stage sorted by key gives the bucket's largest keys.  When no bucket above beta holds more
+// than SEL_RANK_SEG keys, a key's output position is its segment's start plus the keys of its
+// segment above it (no sort of the selection); otherwise the k keys are sorted.  A bucket beta of
+// more than SEL_CAP keys is resolved by four radix passes over its keys and an ordered pass (the
+// first keys equal to the k-th in slot order).  The output is ordered by (score desc, slot asc).
+__global__ void __launch_bounds__(SEL_THREADS, 2) k_topk_select(const float *__restrict__ Y,
+                                                                const int32_t *__restrict__ idx,
+                                                                const int32_t *__restrict__ count,
+                                                                const int64_t *__restrict__ offs, int tau, int k,
+                                                                int kpow2, int32_t *__restrict__ topk_idx,
+                                                                float *__restrict__ topk_score)
 {
-    extern __shared__ unsigned long long sel[];  // [kpow2] selection, [SEL_CAP] stage, then keys
+    extern __shared__ unsigned long long sel[];  // [kpow2] selection, [SEL_CAP] stage
     unsigned long long *stage = sel + kpow2;
-    uint32_t *keys = (uint32_t *)(stage + SEL_CAP);
     __shared__ unsigned int hist[SEL_BINS];
     __shared__ int warp_tot[32];
     __shared__ int tot_a, tot_b, s_bin, s_above, s_ngt, s_nst, s_maxseg;
-    __shared__ uint32_t s_umin, s_umax;
-    bool ranked = false;
+    __shared__ float s_fmin[32], s_fmax[32];
 
     const int b = blockIdx.x / tau, i = blockIdx.x % tau;
     const int64_t off = offs[b], S = offs[b + 1] - offs[b];
     int F = count[b];
     F = F < 0 ? 0 : (F > S ? (int)S : F);
     const float *row = Y + (int64_t)tau * off + (int64_t)i * S;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned lt = (1u << lane) - 1u;
-    const bool resident = F <= fcap;
     auto key64 = [](uint32_t u, int j) { return ((unsigned long long)u << 32) | (uint32_t)(~(uint32_t)j); };
-    auto key_at = [&](int j) -> uint32_t { return resident ? keys[j] : float_to_ordered(__ldg(row + j)); };
-
-    if (threadIdx.x == 0) {
-        s_umin = 0xFFFFFFFFu;
-        s_umax = 0u;
-        s_maxseg = 0;
-    }
-    __syncthreads();
-    uint32_t tmin = 0xFFFFFFFFu, tmax = 0u;  // the range of the query's score keys
-    if (resident) {
-        for (int base = 0; base < F; base += 8 * SEL_THREADS) {
-            float v[8];
+    auto key_at = [&](int j) -> uint32_t { return float_to_ordered(__ldg(row + j)); };
+    const ScoreRow sr(row, F);
+    const int lone = sr.lone();
+    const float4 NONE = make_float4(NAN, NAN, NAN, NAN);
+    // fn(y, j) for every score of the query, four vector loads in flight per thread
+    auto each = [&](auto fn) {
+        for (int v0 = 0; v0 < sr.nvec; v0 += 4 * SEL_THREADS) {
+            float4 x[4];
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int j = base + q * SEL_THREADS + threadIdx.x;
-                v[q] = j < F ? __ldg(row + j) : 0.f;
+            for (int q = 0; q < 4; q++) {
+                const int v = v0 + q * SEL_THREADS + (int)threadIdx.x;
+                x[q] = v < sr.nvec ? __ldg(sr.vec + v) : NONE;
             }
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int j = base + q * SEL_THREADS + threadIdx.x;
-                if (j < F) {
-                    const uint32_t u = float_to_ordered(v[q]);
-                    keys[j] = u;
-                    tmin = min(tmin, u);
-                    tmax = max(tmax, u);
+            for (int q = 0; q < 4; q++) {
+                const int v = v0 + q * SEL_THREADS + (int)threadIdx.x;
+                if (v < sr.nvec) {
+                    const int j = sr.head + 4 * v;
+                    fn(x[q].x, j);
+                    fn(x[q].y, j + 1);
+                    fn(x[q].z, j + 2);
+                    fn(x[q].w, j + 3);
                 }
             }
         }
-    } else if (F > k) {
-        for (int j = threadIdx.x; j < F; j += SEL_THREADS) {
-            const uint32_t u = float_to_ordered(__ldg(row + j));
-            tmin = min(tmin, u);
-            tmax = max(tmax, u);
-        }
-    }
-    tmin = __reduce_min_sync(0xffffffffu, tmin);
-    tmax = __reduce_max_sync(0xffffffffu, tmax);
-    if (lane == 0) {
-        atomicMin(&s_umin, tmin);
-        atomicMax(&s_umax, tmax);
-    }
-    for (int t = threadIdx.x; t < kpow2; t += SEL_THREADS) sel[t] = 0ull;
-    __syncthreads();
+        if (lone >= 0) fn(__ldg(row + lone), lone);
+    };
 
+    for (int t = threadIdx.x; t < kpow2; t += SEL_THREADS) sel[t] = 0ull;
     if (F <= k) {
+        __syncthreads();
         for (int j = threadIdx.x; j < F; j += SEL_THREADS) sel[j] = key64(key_at(j), j);
     } else {
+        // the range of the query's scores (NaN aside), then the histogram
+        float fmn = INFINITY, fmx = -INFINITY;
+        each([&](float y, int) {
+            fmn = fminf(fmn, y);
+            fmx = fmaxf(fmx, y);
+        });
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            fmn = fminf(fmn, __shfl_xor_sync(0xffffffffu, fmn, o));
+            fmx = fmaxf(fmx, __shfl_xor_sync(0xffffffffu, fmx, o));
+        }
+        if (lane == 0) {
+            s_fmin[warp] = fmn;
+            s_fmax[warp] = fmx;
+        }
         for (int t = threadIdx.x; t < SEL_BINS; t += SEL_THREADS) hist[t] = 0;
-        if (threadIdx.x == 0) s_ngt = s_nst = 0;
+        if (threadIdx.x == 0) {
+            s_ngt = s_nst = 0;
+            s_maxseg = 0;
+        }
         __syncthreads();
-        const SelRange rg = sel_range(s_umin, s_umax);
-        for (int j = threadIdx.x; j < F; j += SEL_THREADS) atomicAdd(&hist[sel_bucket(rg, key_at(j))], 1u);
+        fmn = INFINITY;
+        fmx = -INFINITY;
+        for (int w = 0; w < SEL_THREADS / 32; w++) {
+            fmn = fminf(fmn, s_fmin[w]);
+            fmx = fmaxf(fmx, s_fmax[w]);
+        }
+        const SelRange rg = sel_range_f(fmn, fmx);
+        each([&](float y, int) { atomicAdd(&hist[sel_bucket_f(rg, y)], 1u); });
         __syncthreads();
         const int my_above = sel_find_bin<SEL_BINS>(hist, k, warp_tot, &tot_a, &s_bin, &s_above);
         const uint32_t beta = (uint32_t)s_bin;
@@ -242,25 +268,41 @@ __global__ void __launch_bounds__(SEL_THREADS) k_topk_select(const float *__rest
             if (lane == 0) atomicMax(&s_maxseg, mx);
         }
         __syncthreads();
-        // higher buckets scattered to their segments, bucket beta to the stage (any order)
-        for (int base = 0; base < F; base += SEL_THREADS) {
-            const int j = base + threadIdx.x;
-            uint32_t u = 0, bk = 0;
-            bool eq = false;
-            if (j < F) {
-                u = key_at(j);
-                bk = sel_bucket(rg, u);
-                if (bk > beta) sel[atomicAdd(&hist[bk], 1u)] = key64(u, j);
-                eq = staged && bk == beta;
-            }
+        // higher buckets scattered to their segments, bucket beta to the stage (any order); the
+        // loop runs the same trips in every lane (the stage appends are warp-aggregated)
+        auto scatter = [&](bool in, float y, int j) {
+            const uint32_t bk = in ? sel_bucket_f(rg, y) : 0u;
+            if (in && bk > beta) sel[atomicAdd(&hist[bk], 1u)] = key64(float_to_ordered(y), j);
+            const bool eq = in && staged && bk == beta;
             const unsigned be = __ballot_sync(0xffffffffu, eq);
-            int pe = 0;
-            if (lane == 0 && be) pe = atomicAdd(&s_nst, __popc(be));
-            pe = __shfl_sync(0xffffffffu, pe, 0);
-            if (eq) stage[pe + __popc(be & lt)] = key64(u, j);
+            if (be) {
+                int pe = 0;
+                if (lane == 0) pe = atomicAdd(&s_nst, __popc(be));
+                pe = __shfl_sync(0xffffffffu, pe, 0);
+                if (eq) stage[pe + __popc(be & lt)] = key64(float_to_ordered(y), j);
+            }
+        };
+        for (int v0 = 0; v0 < sr.nvec; v0 += 2 * SEL_THREADS) {
+            float4 x[2];
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                const int v = v0 + q * SEL_THREADS + (int)threadIdx.x;
+                x[q] = v < sr.nvec ? __ldg(sr.vec + v) : NONE;
+            }
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                const int v = v0 + q * SEL_THREADS + (int)threadIdx.x;
+                const bool in = v < sr.nvec;
+                const int j = sr.head + 4 * v;
+                scatter(in, x[q].x, j);
+                scatter(in, x[q].y, j + 1);
+                scatter(in, x[q].z, j + 2);
+                scatter(in, x[q].w, j + 3);
+            }
         }
+        scatter(lone >= 0, lone >= 0 ? __ldg(row + lone) : 0.f, lone);
         __syncthreads();
-        ranked = staged && s_maxseg <= SEL_RANK_SEG;
+        const bool ranked = staged && s_maxseg <= SEL_RANK_SEG;
         if (staged) {
             int np = 64;
             while (np < nbeta) np <<= 1;

@@ -15,8 +15,8 @@ once a digit holds exactly the keys still wanted; one sort orders the k
 keys.  With at most k candidates the select takes every candidate whatever its key, including a key
 that orders as 0.
 
-Batched select (csrc/topk.cuh, k_topk_select): the same histogram over all keys gives the bucket of
-the k-th key; keys of higher buckets and the bucket's keys (at most SEL_CAP of them) are appended in
+Batched select (csrc/topk.cuh, k_topk_select): the range is that of the scores that are not NaN;
+the same histogram over all keys gives the bucket of the k-th key; keys of higher buckets and the bucket's keys (at most SEL_CAP of them) are appended in
 any order, and the stage sorted by 64-bit key gives the bucket's largest keys; a crowded bucket
 takes four radix passes of 8 bits over the bucket's keys and an ordered pass instead.
 
@@ -58,6 +58,19 @@ def sel_range(u):
     ymin = _ordered_to_float(np.array([u.min()]))[0]
     with np.errstate(invalid="ignore", over="ignore"):  # NaN / infinite ends, spans below 2^-114
         span = np.float32(_ordered_to_float(np.array([u.max()]))[0] - ymin)
+        scale = np.float32(np.float32(4096.0) / span) if span > 0 else np.float32(0.0)
+    return ymin, scale
+
+
+def sel_range_f(u):
+    """The batched select's (ymin, scale): the smallest and largest scores that are not NaN (fminf /
+    fmaxf over the scores; none: +inf and -inf, so every score falls into bucket 0 or its NaN end)."""
+    y = _ordered_to_float(u)
+    y = y[~np.isnan(y)]
+    ymin = np.float32(y.min()) if y.size else np.float32(np.inf)
+    ymax = np.float32(y.max()) if y.size else np.float32(-np.inf)
+    with np.errstate(invalid="ignore", over="ignore"):
+        span = np.float32(ymax - ymin)
         scale = np.float32(np.float32(4096.0) / span) if span > 0 else np.float32(0.0)
     return ymin, scale
 
@@ -202,7 +215,7 @@ def batched_select_model(u, k, cap=4096, seed=0):
     if F <= k:
         slots = rng.permutation(F)
     else:
-        ymin, scale = sel_range(u)
+        ymin, scale = sel_range_f(u)
         bk = sel_bucket(u, ymin, scale)
         hist = np.bincount(bk, minlength=4096)
         beta, above = _find_bin(hist, k)
@@ -301,7 +314,7 @@ def test_block_sort_model_sorts(n):
 
 # ------------------------------------------------------------------ selection order without a sort
 
-def ranked_order_model(u, k, seed=0):
+def ranked_order_model(u, k, seed=0, rangef=None):
     """Both selects' ordering of the selection when no bucket above beta is large: every bucket
     above beta gets a segment of the selection (higher buckets first, each segment's start the keys
     of the buckets above it), its keys are scattered into it in any order (shuffled here), and a
@@ -310,7 +323,7 @@ def ranked_order_model(u, k, seed=0):
     segment)."""
     rng = np.random.default_rng(seed)
     kk = key64(u)
-    ymin, scale = sel_range(u)
+    ymin, scale = (rangef or sel_range)(u)
     bk = sel_bucket(u, ymin, scale)
     hist = np.bincount(bk, minlength=4096)
     beta, above = _find_bin(hist, k)
@@ -334,11 +347,14 @@ def ranked_order_model(u, k, seed=0):
     return slots, int(hist[beta + 1:].max()) if beta + 1 < 4096 else 0
 
 
+@pytest.mark.parametrize("rangef", ["keys", "scores"])
 @pytest.mark.parametrize("kind", ["random", "ties_every_digit", "ties_low_digits", "narrow_with_outlier", "float"])
-def test_ranked_order_equals_plain_sort(kind):
+def test_ranked_order_equals_plain_sort(kind, rangef):
+    """rangef: the range of the keys (the decode step's order) or of the non-NaN scores (the
+    batched select)."""
     rng = np.random.default_rng(zlib.crc32((kind + "ranked").encode()))
     for nc in (2049, 5000, 31000):
         for k in (1, 7, 512, 2048):
             u = keys(rng, kind, nc)
-            slots, _ = ranked_order_model(u, k, seed=nc + k)
+            slots, _ = ranked_order_model(u, k, seed=nc + k, rangef=sel_range if rangef == "keys" else sel_range_f)
             assert np.array_equal(slots, plain_sort(u, k)), (kind, nc, k)
