@@ -281,7 +281,7 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
     if (proj_tc_supported(dt, B, d) && proj_tc_supported(dt, B, r)) {
         // c and w in one launch, split along d so that every SM streams weights (fp32 partial sums
         // in slices of their own); the slices summed in order, c rounded to bf16 once; then q,
-        // split along r the same way when that balances the SMs better.  Every launch after the
+        // split along r the same way when it has fewer tiles than SMs.  Every launch after the
         // first is a programmatic dependent of the one before (the q launch streams its first
         // weight stages while c is summed).
         const int sms = num_sms();
@@ -297,7 +297,10 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
                                cudaSuccess)
             s = LSA_ERR_CUDA;
         if (s == LSA_OK) s = launched("project: reduce c and w");
-        const bool qsplit = proj_ksplit((int64_t)L * ((nq + 127) / 128), proj_stages_of_k(B, r), sms) > 1;
+        // (q is split only when its tiles leave SMs idle: measured at 192 tiles on 148 SMs, the split's
+        // better balance did not pay for the slice sums)
+        const int64_t qtiles = (int64_t)L * ((nq + 127) / 128);
+        const bool qsplit = qtiles < sms && proj_ksplit(qtiles, proj_stages_of_k(B, r), sms) > 1;
         const ProjProblem qp = {W_iuq, qsplit ? (void *)pc : q_out, nq, false};  // (pc: summed already)
         int kq = 1;
         if (s == LSA_OK) s = launch_proj_tc(c, &qp, &qsplit, 1, L, B, r, sms, st, &kq, true);

@@ -274,6 +274,8 @@ PROJ_CASES = {
     "b37": lambda: synth.workload("ctx128k_bf16", B=37, S=(64,) * 37, fetch=(0.1,) * 37, name="proj_b37"),
     "b100_small": lambda: synth.workload("ctx128k_bf16", B=100, S=(64,) * 100, fetch=(0.1,) * 100, d=512, r=256,
                                          name="proj_b100"),
+    # one layer: 64 tiles of q on 148 SMs, so q is split along r too (slices summed by k_proj_reduce)
+    "l1_q_split": lambda: synth.workload("ctx128k_bf16", L=1, name="proj_l1"),
 }
 
 
