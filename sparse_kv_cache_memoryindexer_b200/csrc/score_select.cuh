@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(TILE) k_score_simt(const void *__restrict__ q,
 // fetched entries in the sequence's earlier tiles (summed from their fetch words, a few KB read
 // from L2), its tiles' starts come from a block scan, and each warp writes the entries of its 32
 // tiles with consecutive lanes on consecutive list positions.
+constexpr int COMPACT_SMEM_B = 1024;  // sequences whose chunk starts k_compact keeps in shared memory
 __device__ __forceinline__ int popc4(uint4 m) { return __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w); }
 
 __global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__restrict__ tile_mask,
@@ -164,12 +165,21 @@ __global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__res
 {
     __shared__ int red[COMPACT_TILES / 32];
     __shared__ int scan[COMPACT_TILES / 32];
+    __shared__ int s_cs[COMPACT_SMEM_B + 1];
     const int c = blockIdx.x;
-    if (c >= chunk_start[B]) return;
-    int lo = 0, hi = B - 1;  // the sequence of chunk c: largest b with chunk_start[b] <= c
+    // the sequence of chunk c: largest b with chunk_start[b] <= c (the chunk starts read in one
+    // coalesced pass into shared memory when there are few sequences, not one load per search step)
+    const bool in_smem = B <= COMPACT_SMEM_B;
+    if (in_smem) {
+        for (int t = threadIdx.x; t <= B; t += COMPACT_TILES) s_cs[t] = chunk_start[t];
+        __syncthreads();
+    }
+    const int *cs = in_smem ? s_cs : chunk_start;
+    if (c >= cs[B]) return;
+    int lo = 0, hi = B - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (chunk_start[mid] <= c) lo = mid;
+        if (cs[mid] <= c) lo = mid;
         else hi = mid - 1;
     }
     const int b = lo;
@@ -204,9 +214,10 @@ __global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__res
     // coalesced writes: the warp walks its 32 tiles; the mask goes out as 4 bytes per lane when the
     // sequence's bytes start on a 4-byte boundary
     const bool mask_words = mask_out && (((uintptr_t)(mask_out + off)) & 3u) == 0;
-    for (int j = 0; j < 32; j++) {
+    const int nj = max(0, min(32, ct1 - (ct0 + warp * 32)));  // this warp's tiles
+#pragma unroll 4
+    for (int j = 0; j < nj; j++) {  // (unrolled: four tiles' shuffles and stores in flight)
         const int tj = ct0 + warp * 32 + j;
-        if (tj >= ct1) break;
         const uint32_t w0 = __shfl_sync(0xffffffffu, m.x, j), w1 = __shfl_sync(0xffffffffu, m.y, j);
         const uint32_t w2 = __shfl_sync(0xffffffffu, m.z, j), w3 = __shfl_sync(0xffffffffu, m.w, j);
         int p = __shfl_sync(0xffffffffu, pos, j);
