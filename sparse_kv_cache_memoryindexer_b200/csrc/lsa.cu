@@ -398,8 +398,8 @@ lsa_status lsa_memindex_score_select(const void *q, const float *w, const void *
         }
     }
     const int64_t chunks = (max_tiles(B, total_S) + COMPACT_TILES - 1) / COMPACT_TILES + B;
-    k_compact<<<(unsigned)chunks, COMPACT_TILES, 0, st>>>(ws.tile_mask, ws.tile_start, ws.chunk_start, seq_offsets, B,
-                                                        idx_out, count_out, mask_out);
+    k_compact<<<(unsigned)chunks, COMPACT_THREADS, 0, st>>>(ws.tile_mask, ws.tile_start, ws.chunk_start, seq_offsets,
+                                                          B, idx_out, count_out, mask_out);
     LSA_TRY(launched("compact"));
     return ok();
 }

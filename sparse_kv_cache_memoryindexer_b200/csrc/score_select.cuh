@@ -146,32 +146,37 @@ __global__ void __launch_bounds__(TILE) k_score_simt(const void *__restrict__ q,
     if ((threadIdx.x & 31) == 0) tile_mask[(int64_t)tile * 4 + (threadIdx.x >> 5)] = m;
 }
 
-// Compaction (stage 4a): one block per sequence scans its tiles' fetch words in order and writes
-// the ascending list of fetched entries, the count, and optionally a byte mask.
-// Stage 4a: the ascending list of fetched entries of each sequence from the fetch words.  One CTA
-// per chunk of COMPACT_TILES tiles of one sequence: its sequence-local start is the number of
-// fetched entries in the sequence's earlier tiles (summed from their fetch words, a few KB read
-// from L2), its tiles' starts come from a block scan, and each warp writes the entries of its 32
-// tiles with consecutive lanes on consecutive list positions.
+// Compaction (stage 4a): the ascending list of fetched entries of each sequence from the fetch
+// words, the count, and optionally a byte mask.  One CTA per chunk of COMPACT_TILES tiles of one
+// sequence: its sequence-local start is the number of fetched entries in the sequence's earlier
+// tiles (summed from their fetch words, a few KB read from L2), its tiles' starts come from a block
+// scan, and each of its 32 warps writes the entries of 8 tiles with consecutive lanes on
+// consecutive list positions.
 constexpr int COMPACT_SMEM_B = 1024;  // sequences whose chunk starts k_compact keeps in shared memory
 __device__ __forceinline__ int popc4(uint4 m) { return __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w); }
 
-__global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__restrict__ tile_mask,
-                                                          const int *__restrict__ tile_start,
-                                                          const int *__restrict__ chunk_start,
-                                                          const int64_t *__restrict__ offs, int B,
-                                                          int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out,
-                                                          uint8_t *__restrict__ mask_out)
+constexpr int COMPACT_THREADS = 4 * COMPACT_TILES;  // the chunk's tiles counted by the first COMPACT_TILES
+                                                    // threads, written by all warps (8 tiles each)
+
+__global__ void __launch_bounds__(COMPACT_THREADS, 2) k_compact(const uint32_t *__restrict__ tile_mask,
+                                                            const int *__restrict__ tile_start,
+                                                            const int *__restrict__ chunk_start,
+                                                            const int64_t *__restrict__ offs, int B,
+                                                            int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out,
+                                                            uint8_t *__restrict__ mask_out)
 {
-    __shared__ int red[COMPACT_TILES / 32];
+    constexpr int NW = COMPACT_THREADS / 32, TPW = COMPACT_TILES / NW;  // warps, tiles written per warp
+    __shared__ int red[NW];
     __shared__ int scan[COMPACT_TILES / 32];
     __shared__ int s_cs[COMPACT_SMEM_B + 1];
+    __shared__ uint4 s_mask[COMPACT_TILES];
+    __shared__ int s_pos[COMPACT_TILES];
     const int c = blockIdx.x;
     // the sequence of chunk c: largest b with chunk_start[b] <= c (the chunk starts read in one
     // coalesced pass into shared memory when there are few sequences, not one load per search step)
     const bool in_smem = B <= COMPACT_SMEM_B;
     if (in_smem) {
-        for (int t = threadIdx.x; t <= B; t += COMPACT_TILES) s_cs[t] = chunk_start[t];
+        for (int t = threadIdx.x; t <= B; t += COMPACT_THREADS) s_cs[t] = chunk_start[t];
         __syncthreads();
     }
     const int *cs = in_smem ? s_cs : chunk_start;
@@ -190,40 +195,45 @@ __global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__res
     const int64_t off = offs[b], S = offs[b + 1] - off;
     // fetched entries before this chunk
     int part = 0;
-    for (int t = t0 + threadIdx.x; t < ct0; t += COMPACT_TILES) part += popc4(*(const uint4 *)(tile_mask + (int64_t)t * 4));
+    for (int t = t0 + threadIdx.x; t < ct0; t += COMPACT_THREADS) part += popc4(*(const uint4 *)(tile_mask + (int64_t)t * 4));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if (lane == 0) red[warp] = part;
-    // this chunk: one tile per thread
+    // this chunk: one tile per thread of the first COMPACT_TILES
     const int t = ct0 + threadIdx.x;
     uint4 m = make_uint4(0, 0, 0, 0);
-    if (t < ct1) m = *(const uint4 *)(tile_mask + (int64_t)t * 4);
+    if (threadIdx.x < COMPACT_TILES && t < ct1) m = *(const uint4 *)(tile_mask + (int64_t)t * 4);
     const int cnt = popc4(m);
     const int inc = warp_incl_scan(cnt);
-    if (lane == 31) scan[warp] = inc;
+    if (lane == 31 && warp < COMPACT_TILES / 32) scan[warp] = inc;
     __syncthreads();
-    int base = 0, before = 0, total = 0;
+    int base = 0, total = 0;
 #pragma unroll
-    for (int w = 0; w < COMPACT_TILES / 32; w++) {
-        base += red[w];
-        before += w < warp ? scan[w] : 0;
-        total += scan[w];
+    for (int w = 0; w < NW; w++) base += red[w];
+    if (threadIdx.x < COMPACT_TILES) {
+        int before = 0;
+#pragma unroll
+        for (int w = 0; w < COMPACT_TILES / 32; w++) {
+            before += w < warp ? scan[w] : 0;
+            total += scan[w];
+        }
+        s_mask[threadIdx.x] = m;
+        s_pos[threadIdx.x] = base + before + inc - cnt;  // list position of this tile's first entry
+        if (ct1 == t1 && threadIdx.x == 0) count_out[b] = base + total;
     }
-    const int pos = base + before + inc - cnt;  // list position of this tile's first entry
-    if (ct1 == t1 && threadIdx.x == 0) count_out[b] = base + total;
-    // coalesced writes: the warp walks its 32 tiles; the mask goes out as 4 bytes per lane when the
-    // sequence's bytes start on a 4-byte boundary
+    __syncthreads();
+    // coalesced writes: warp w walks tiles w TPW .. w TPW + TPW - 1 of the chunk; the mask goes out as
+    // 4 bytes per lane when the sequence's bytes start on a 4-byte boundary
     const bool mask_words = mask_out && (((uintptr_t)(mask_out + off)) & 3u) == 0;
-    const int nj = max(0, min(32, ct1 - (ct0 + warp * 32)));  // this warp's tiles
-#pragma unroll 4
-    for (int j = 0; j < nj; j++) {  // (unrolled: four tiles' shuffles and stores in flight)
-        const int tj = ct0 + warp * 32 + j;
-        const uint32_t w0 = __shfl_sync(0xffffffffu, m.x, j), w1 = __shfl_sync(0xffffffffu, m.y, j);
-        const uint32_t w2 = __shfl_sync(0xffffffffu, m.z, j), w3 = __shfl_sync(0xffffffffu, m.w, j);
-        int p = __shfl_sync(0xffffffffu, pos, j);
-        const int64_t s0 = (int64_t)(tj - t0) * TILE;
+    const int nj = max(0, min(TPW, ct1 - (ct0 + warp * TPW)));  // this warp's tiles
+#pragma unroll 2
+    for (int j = 0; j < nj; j++) {
+        const int jt = warp * TPW + j;  // tile within the chunk
+        const uint4 mw = s_mask[jt];
+        int p = s_pos[jt];
+        const int64_t s0 = (int64_t)(ct0 + jt - t0) * TILE;
         const uint32_t below = (1u << lane) - 1u;
-        const uint32_t words[4] = {w0, w1, w2, w3};
+        const uint32_t words[4] = {mw.x, mw.y, mw.z, mw.w};
 #pragma unroll
         for (int k = 0; k < 4; k++) {
             const uint32_t wk = words[k];
@@ -234,7 +244,7 @@ __global__ void __launch_bounds__(COMPACT_TILES) k_compact(const uint32_t *__res
         }
         if (mask_words) {
             // lane: entries 4 lane .. 4 lane + 3 of the tile (bits 4 (lane % 8) .. of word lane / 8)
-            const uint32_t wl = lane < 8 ? w0 : (lane < 16 ? w1 : (lane < 24 ? w2 : w3));
+            const uint32_t wl = lane < 8 ? mw.x : (lane < 16 ? mw.y : (lane < 24 ? mw.z : mw.w));
             const uint32_t nib = (wl >> (4 * (lane & 7))) & 0xFu;
             const uint32_t bytes = (nib & 1u) | ((nib & 2u) << 7) | ((nib & 4u) << 14) | ((nib & 8u) << 21);
             const int64_t e = s0 + 4 * lane;
