@@ -183,52 +183,29 @@ __global__ void __launch_bounds__(128) k_gather_keys(const int32_t *__restrict__
     const int total = block_count_prefix(count, offs, B, pre, warp_sum);
     const int64_t kb = (int64_t)krow16 * 16, kbo = kconv ? 2 * kb : kb;
     const int64_t units = (int64_t)total * krow16;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    constexpr int U = 4;  // units per thread in flight: the index loads, then the key loads, then the stores
-    for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < units; u0 += U * stride) {
-        int64_t src[U], dst[U];
-        int ch[U];
-        bool ok[U];
-#pragma unroll
-        for (int q = 0; q < U; q++) {
-            const int64_t u = u0 + q * stride;
-            ok[q] = u < units;
-            src[q] = dst[q] = 0;
-            ch[q] = 0;
-            if (ok[q]) {
-                const int64_t g = u / krow16;
-                ch[q] = (int)(u - g * krow16);
-                const int b = sequence_of_row(pre, B, g);
-                const int64_t off = offs[b], S = offs[b + 1] - off;
-                const int64_t j = g - pre[b];
-                const int s = __ldg(idx + off + j);
-                if (s < 0 || s >= S) {
-                    if (ch[q] == 0) flag(ERRF_INDEX);
-                    ok[q] = false;
-                } else {
-                    src[q] = off + s;
-                    dst[q] = off + j;
-                }
-            }
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t g = u / krow16;
+        const int ch = (int)(u - g * krow16);
+        const int b = sequence_of_row(pre, B, g);
+        const int64_t off = offs[b], S = offs[b + 1] - off;
+        const int64_t j = g - pre[b];
+        const int s = __ldg(idx + off + j);
+        if (s < 0 || s >= S) {
+            if (ch == 0) flag(ERRF_INDEX);
+            continue;
         }
-        uint4 v[U];
-#pragma unroll
-        for (int q = 0; q < U; q++)
-            v[q] = ok[q] ? __ldg((const uint4 *)(Ksel + src[q] * kb + (int64_t)ch[q] * 16)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int q = 0; q < U; q++) {
-            if (!ok[q]) continue;
-            if (kconv) {
-                uint4 lo, hi;
-                e4m3x16_to_bf16(v[q], lo, hi);
-                uint4 *d = (uint4 *)(hotK + dst[q] * kbo + (int64_t)ch[q] * 32);
-                d[0] = lo;
-                d[1] = hi;
-            } else {
-                *(uint4 *)(hotK + dst[q] * kbo + (int64_t)ch[q] * 16) = v[q];
-            }
-            if (ksc && ch[q] == 0) hotsc[dst[q]] = __ldg(ksc + src[q]);
+        const int64_t src = off + s, dst = off + j;
+        const uint4 v = __ldg((const uint4 *)(Ksel + src * kb + (int64_t)ch * 16));
+        if (kconv) {
+            uint4 lo, hi;
+            e4m3x16_to_bf16(v, lo, hi);
+            uint4 *d = (uint4 *)(hotK + dst * kbo + (int64_t)ch * 32);
+            d[0] = lo;
+            d[1] = hi;
+        } else {
+            *(uint4 *)(hotK + dst * kbo + (int64_t)ch * 16) = v;
         }
+        if (ksc && ch == 0) hotsc[dst] = __ldg(ksc + src);
     }
 }
 
