@@ -111,15 +111,33 @@ def check_project(h, W_dq, W_iuq, W_w, n_h, d_I, q_gpu, w_gpu, c_gpu, what=""):
     cb = (2.0 ** -22) * d * torch.einsum("lbi,lji->lbj", h64.abs(), W_dq.double().abs())
     dc = (c_gpu.double() - c_ref.double()).abs()
     assert (dc <= ulp(c_gpu.double(), c_ref.double()) * 1.0001 + cb).all(), f"{what}: c"
-    if bf:  # neighbours only where the exact c lies near a rounding boundary
-        assert (dc > 0).double().mean() < 0.15, f"{what}: too many c differ"
+    if bf:
+        # a stored c may differ from the oracle's only as the other side of a rounding boundary
+        # that the exact sum lies within the fp32 bound of: the GPU's fp32 sum s is within cb of
+        # the exact sum x and rounds to the other neighbour, so the midpoint between the two
+        # neighbours lies between x and s
+        c_exact = torch.einsum("lbi,lji->lbj", h64, W_dq.double())
+        _near_boundary(c_exact, c_ref.double(), c_gpu.double(), cb, f"{what}: c")
     eye = torch.eye(r, dtype=h.dtype).expand(L, r, r).contiguous()
     q2, _ = oracle.project(c_gpu.contiguous(), eye, W_iuq, torch.zeros((L, n_h, r), dtype=h.dtype), n_h, d_I)
     qb = (2.0 ** -22) * r * torch.einsum("lbj,loj->lbo", c_gpu.double().abs(), W_iuq.double().abs())
     dq = (q_gpu.double() - q2.double()).reshape(qb.shape).abs()
     assert (dq <= ulp(q_gpu.double(), q2.double()).reshape(qb.shape) * 1.0001 + qb).all(), f"{what}: q"
     if bf:
-        assert (dq > 0).double().mean() < 0.05, f"{what}: too many q differ"
+        q_exact = torch.einsum("lbj,loj->lbo", c_gpu.double(), W_iuq.double())
+        _near_boundary(q_exact, q2.double().reshape(qb.shape), q_gpu.double().reshape(qb.shape), qb, f"{what}: q")
+
+
+def _near_boundary(exact, ref, got, bound, what):
+    """Where got != ref (both rounded values), the rounding boundary between them (their midpoint)
+    is within bound of the exact value (1e-12 relative slack for the double sums)."""
+    diff = got != ref
+    if not bool(diff.any()):
+        return
+    mid = (ref[diff] + got[diff]) / 2
+    gap = (exact[diff] - mid).abs()
+    lim = bound[diff] * 1.0001 + exact[diff].abs() * 1e-12
+    assert (gap <= lim).all(), f"{what}: a value differs away from a rounding boundary"
 
 
 # ------------------------------------------------------------------------------ training step
