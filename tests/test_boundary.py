@@ -58,6 +58,11 @@ def test_host_side_validation_without_gpu():
                                          None) == 1
     assert lib.lsa_lightning_topk(p, p, p, None, 1, p, p, p, 10, 1, 1, 1, 32, 5000, p, None, p, 1 << 20, None) == 1
     assert lib.lsa_project(p, p, p, p, 2, 1, 1, 8, 8, 1, 1, p, p, p, 1 << 20, None) == 2
+    # golden labels: vote counts are held in 8 bit slices (at most 255 layers), entries in 32 bits
+    assert lib.lsa_golden_labels(p, p, 1000, 1, 4, 256, 0.6, 3, p, None, p, 1 << 20, None) == 1
+    assert b"255 layers" in lib.lsa_last_error()
+    assert lib.lsa_golden_labels(p, p, 1 << 31, 1, 4, 21, 0.6, 3, p, None, p, 1 << 40, None) == 1
+    assert b"2^31" in lib.lsa_last_error()
     # a workspace that is too small
     assert lib.lsa_memindex_score_select(p, p, p, None, 1, p, 1 << 20, 3, 4, 64, 128, 0.5, None, None, p, p, p, 16,
                                          None) == 5
