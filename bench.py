@@ -123,6 +123,8 @@ def score_traffic(wl):
     tr = SCORE_TRAFFIC.get(wl.kdtype)
     if tr is None or score_kernel_src_hash(tr["sources"]) != tr["hash"]:
         return None, None
+    if os.environ.get("LSA_DISABLE_TC"):
+        return None, None  # the SIMT kernels run then
     if wl.kdtype == "fp8" and (os.environ.get("LSA_SCORE_PAIR", "1").startswith("0") or wl.B > 1024):
         return None, None  # the one-CTA E4M3 kernel runs then: no capture of its traffic at this version
     return tr["bytes_per_entry_layer"] * wl.L * wl.total_S, tr["kernel"] + ": " + tr["capture"]
