@@ -113,8 +113,9 @@ lsa_status lsa_project(const void *h, const void *W_dq, const void *W_iuq, const
  *   idx_out     [T] int32        segment b: the fetched s in ascending order in the first
  *                                count_out[b] slots; the other slots are left unchanged
  *   count_out   [B] int32        number of fetched entries of each sequence
- * Kernels: tcgen05 tensor-core path for n_h = 64, d_I = 128 with bf16 or E4M3 keys; a SIMT
- * path for other shapes (d_I in {32, 64, 128}, n_h <= 128) and for fp32.
+ * Kernels: tcgen05 tensor-core path for n_h = 64, d_I = 128 with bf16 or E4M3 keys (E4M3 on
+ * pairs of CTAs for B <= 1024 unless the environment sets LSA_SCORE_PAIR=0; the same result
+ * either way); a SIMT path for other shapes (d_I in {32, 64, 128}, n_h <= 128) and for fp32.
  * Workspace: lsa_score_select_workspace_size.
  * ---------------------------------------------------------------------------------------- */
 size_t lsa_score_select_workspace_size(int L, int B, int64_t total_S);
@@ -234,7 +235,8 @@ lsa_status lsa_fetch_gather_incremental(const int32_t *idx, const int32_t *count
  *   topk_idx   [B][tau][k] int32
  *   topk_score [B][tau][k] fp32     (nullable)
  * Kernels: tcgen05 tensor-core scoring for n_h = 64, d_I = 128, tau a multiple of 4 (bf16 or
- * E4M3 keys); a SIMT path otherwise.  Then a radix select per query.
+ * E4M3 keys); a SIMT path otherwise.  Then a bucket select per query (4,096 buckets over the
+ * query's score range; a radix search inside a crowded bucket).
  * Workspace: lsa_lightning_topk_workspace_size (work plan and the fp32 scores y).
  * ---------------------------------------------------------------------------------------- */
 size_t lsa_lightning_topk_workspace_size(int B, int tau, int64_t total_S, int k);
